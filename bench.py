@@ -1,0 +1,386 @@
+"""Benchmark: decode of one CSA layer at 128K context (B=32 sequences, 1 new token each, 32768 FP4
+compressed entries per sequence, top-512, window 128, 64 heads x 512) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = the whole hot path for one decode token of every sequence: compress the completed group
+(pooling), FP4-pack the new entry and its indexer key, lightning-indexer scores over all entries,
+top-k, attention over the selected entries plus the window.  Eight independent layer states (3.7 GB)
+are rotated so every step reads its caches from HBM, not from the 126 MB L2.  Steps are replayed from
+CUDA graphs; timing uses CUDA events on the launching stream, max over ranks.  Under torchrun every
+rank runs its own batch of 32 sequences (weak scaling, no collective on the data path).
+`--impl reference` times the CPU oracle (the reference arm) on a bounded sample.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode CSA tokens/sec (all heads) at 128K ctx on 1 B200; HBM GB/s as % of peak"
+UNIT = "tokens/s"
+LAYERS = 8
+SCORE_PROFILE = os.path.join(ROOT, "profiles", "index_score_kernel_cfg2_decode.txt")
+INDEX_SRC = os.path.join(ROOT, "compressed_sparse_attention_18_b200", "csrc", "index.cu")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20000)
+    p.add_argument("--warmup", type=int, default=64)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=400)
+    p.add_argument("--cpu-sample", type=int, default=2, help="sequences the CPU oracle times (cpu_baseline)")
+    return p.parse_args()
+
+
+def dist_init(n):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def config_dict(s):
+    return {"workload": s.name, "B": s.B, "context_tokens": s.T, "entries": s.n_c, "ratio": s.r, "heads": s.H,
+            "head_dim": s.d, "fp4_dims": s.d_n, "rope_dims": s.d_r, "indexer": f"{s.H_I}x{s.d_I} fp4", "top_k": s.k,
+            "window": s.W, "layers_rotated": LAYERS, "l2": "inputs larger than L2 (8 rotated layer states)",
+            "cuda_graph": True}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def score_kernel_bytes(s, B):
+    """Algorithmic bytes of one index-score launch: every visible key (64 B codes + 4 B scales), the
+    score written per key, the queries (bf16) and head weights."""
+    return B * (s.n_c * (s.d_I // 2 + s.d_I // 32 + 4) + s.H_I * s.d_I * 2 + s.H_I * 4)
+
+
+def profiled_traffic():
+    """dram bytes per launch from the committed ncu summary, if it was taken on the current kernel."""
+    if not os.path.exists(SCORE_PROFILE):
+        return None
+    text = open(SCORE_PROFILE).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"index_cu_sha256:\s*([0-9a-f]+)", text)
+    if not m or not h:
+        return None
+    cur = hashlib.sha256(open(INDEX_SRC, "rb").read()).hexdigest()
+    return float(m.group(1)) if h.group(1) == cur else None
+
+
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index):
+        self.dev = dev_index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for i, n in enumerate(names):
+                if "Active" in r[5 + i] and "Not" not in r[5 + i]:
+                    reasons.add(n)
+        # the samples while the GPU is busy (the top half of the clock readings)
+        busy = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from csa_workloads import CFG2
+    from oracle import csa_oracle as O
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+    s = CFG2
+    # each step: one sequence's decode through the oracle (index over 32768 entries, top-k, attention)
+    n = s.n_c
+    g = torch.Generator().manual_seed(1)
+    kv = torch.randn((n, s.d), generator=g).to(torch.bfloat16).double().numpy()
+    ki = torch.randn((n, s.d_I), generator=g).to(torch.bfloat16).double().numpy()
+    win = torch.randn((s.W, s.d), generator=g).to(torch.bfloat16).double().numpy()
+    with threadpool_limits(1):
+        kc, ks, _ = O.pack_fp4(ki, 0, 1.0)
+        c, sc, rp = O.pack_fp4(kv, s.d_r, 1.0)
+        rows = O.entry_kv(c, sc, rp, s.d_n, 1.0)
+
+        def step(i):
+            gg = torch.Generator().manual_seed(100 + i)
+            q = torch.randn((1, s.H, s.d), generator=gg).to(torch.bfloat16).double().numpy()
+            qI = torch.randn((1, s.H_I, s.d_I), generator=gg).to(torch.bfloat16).double().numpy()
+            w = (torch.randn((1, s.H_I), generator=gg) * s.H_I ** -0.5).double().numpy()
+            scr, ids = O.index_scores(qI, w, 1.0, kc, ks, 1.0, [s.T - 1], n, s.r)
+            idx, _ = O.topk(scr, ids, s.k)
+            O.attention(q, [s.T - 1], rows, idx, n, win, s.T - s.W, s.W, s.d ** -0.5)
+
+        for i in range(min(args.warmup, 1)):
+            step(i)
+        budget = 90.0
+        t0 = time.perf_counter()
+        done = 0
+        while done < args.steps and (done == 0 or time.perf_counter() - t0 < budget):
+            step(done)
+            done += 1
+        el = time.perf_counter() - t0
+    val = done / el
+    line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": done, "warmup": min(args.warmup, 1),
+            "ms_per_step": el * 1e3 / done, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference", "config": config_dict(s),
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{done} decode tokens (one sequence each: index over {n} entries, top-{s.k}, "
+                                       f"attention over {s.k}+{s.W} keys), numpy fp64, 1 thread"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------------------- our arm
+
+def cpu_baseline(nseq):
+    """The oracle as it stands on a bounded sample: nseq decode tokens on 1 host thread."""
+    from csa_workloads import CFG2
+    from oracle import csa_oracle as O
+    from threadpoolctl import threadpool_limits
+    s = CFG2
+    g = torch.Generator().manual_seed(2)
+    kv = torch.randn((s.n_c, s.d), generator=g).to(torch.bfloat16).double().numpy()
+    ki = torch.randn((s.n_c, s.d_I), generator=g).to(torch.bfloat16).double().numpy()
+    win = torch.randn((s.W, s.d), generator=g).to(torch.bfloat16).double().numpy()
+    with threadpool_limits(1):
+        kc, ks, _ = O.pack_fp4(ki, 0, 1.0)
+        c, sc, rp = O.pack_fp4(kv, s.d_r, 1.0)
+        rows = O.entry_kv(c, sc, rp, s.d_n, 1.0)
+        t0 = time.perf_counter()
+        for i in range(nseq):
+            q = torch.randn((1, s.H, s.d), generator=g).to(torch.bfloat16).double().numpy()
+            qI = torch.randn((1, s.H_I, s.d_I), generator=g).to(torch.bfloat16).double().numpy()
+            w = (torch.randn((1, s.H_I), generator=g) * s.H_I ** -0.5).double().numpy()
+            scr, ids = O.index_scores(qI, w, 1.0, kc, ks, 1.0, [s.T - 1], s.n_c, s.r)
+            idx, _ = O.topk(scr, ids, s.k)
+            O.attention(q, [s.T - 1], rows, idx, s.n_c, win, s.T - s.W, s.W, s.d ** -0.5)
+        el = time.perf_counter() - t0
+    return {"value": nseq / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{nseq} decode tokens of the same workload (one sequence each: index over {s.n_c} entries, "
+                      f"top-{s.k}, attention over {s.k}+{s.W} keys; pack of the caches untimed), numpy fp64, 1 thread"}
+
+
+def run_ours(args, rank, world):
+    import compressed_sparse_attention_18_b200 as csa
+    from compressed_sparse_attention_18_b200.layer import CSADecodeLayer, LayerShape
+    from csa_workloads import CFG2, decode_inputs
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    s = CFG2
+    ls = LayerShape(B=s.B, n_max=s.n_c, r=s.r, H=s.H, d=s.d, d_r=s.d_r, H_I=s.H_I, d_I=s.d_I, k=s.k, W=s.W)
+    layers, inputs = [], []
+    for li in range(LAYERS):
+        L = CSADecodeLayer(ls, dev)
+        inp = decode_inputs(s, seed=1000 * rank + li, device=dev)
+        L.load_history(inp["kv_src"], inp["kI_src"], s.n_c)
+        L.win.copy_(inp["win_kv"])
+        del inp["kv_src"], inp["kI_src"]
+        layers.append(L)
+        inputs.append(inp)
+        torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    stream = torch.cuda.Stream(dev)
+    marks = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)] for _ in range(LAYERS)]
+
+    def run_layers(n, with_marks):
+        for li in range(n):
+            inp = inputs[li]
+            layers[li].step(inp["C"], inp["Z"], inp["b_pos"], inp["W_IK"], inp["q"], inp["q_I"], inp["w"],
+                            stream=stream, marks=marks[li] if with_marks else None)
+
+    # eager warm-up (also sets kernel attributes before capture)
+    with torch.cuda.stream(stream):
+        run_layers(LAYERS, False)
+    stream.synchronize()
+    graphs = {}
+
+    def graph_for(n):
+        if n not in graphs:
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph, stream=stream, capture_error_mode="relaxed"):
+                run_layers(n, True)
+            graphs[n] = gph
+        return graphs[n]
+
+    full = graph_for(LAYERS)
+
+    def run_steps(k):
+        with torch.cuda.stream(stream):
+            for _ in range(k // LAYERS):
+                full.replay()
+            if k % LAYERS:
+                graph_for(k % LAYERS).replay()
+
+    run_steps(max(args.warmup, 3))
+    stream.synchronize()
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    run_steps(args.steps)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = clk.stop()
+    ms = t0.elapsed_time(t1)
+    # per-stage times of the last rotation of the timed region (events inside the graph)
+    last = min(args.steps, LAYERS)
+    stage = [[marks[li][j].elapsed_time(marks[li][j + 1]) for j in range(4)] for li in range(last)]
+    score_ms = statistics.mean(st[1] for st in stage)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms = float(tt.item())
+    tokens = s.B * args.steps * world
+    value = tokens / (ms / 1e3)
+
+    # ---- end to end through the public API: pinned host inputs in, result out, every step
+    e2e = run_e2e(args, layers, inputs, stream, dev, world)
+
+    if rank != 0:
+        return
+    hbm, kind = peaks()
+    bpl = score_kernel_bytes(s, s.B)
+    achieved = bpl / (score_ms / 1e3) / 1e9
+    traffic = profiled_traffic()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp4-e2m1/bf16", "data": "synthetic", "config": config_dict(s),
+        "gpu_launches": CSADecodeLayer.KERNELS_PER_STEP * args.steps,
+        "clocks": clocks,
+        "stages_ms": {"compress_pack": statistics.mean(st[0] for st in stage), "index_score": score_ms,
+                      "topk": statistics.mean(st[2] for st in stage),
+                      "attention": statistics.mean(st[3] for st in stage)},
+        "roofline": {"bound": "hbm", "kernel": "index_score_kernel<128>", "achieved": achieved, "peak": hbm,
+                     "peak_kind": kind, "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": bpl},
+        "step_hbm_gbs": 2682432 * s.B / (ms / args.steps / 1e3) / 1e9,
+        "e2e": e2e,
+    }
+    if world == 1 or rank == 0:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_sample) if world == 1 else None
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, layers, inputs, stream, dev, world):
+    """The same metric through the public API with host buffers: every step copies its inputs (C, Z,
+    q, q_I, w and the new token's window row) from pinned host memory to the device and reads the
+    attention output back."""
+    s_layers = len(layers)
+    host_in, host_out = [], []
+    for li in range(s_layers):
+        inp = inputs[li]
+        h = {k: inp[k].cpu().pin_memory() for k in ("C", "Z", "q", "q_I", "w")}
+        h["win_row"] = layers[li].win[:, -1:].cpu().pin_memory()
+        host_in.append(h)
+        host_out.append(torch.empty_like(layers[li].out, device="cpu").pin_memory())
+    nbytes_in = sum(v.numel() * v.element_size() for v in host_in[0].values())
+    nbytes_out = host_out[0].numel() * host_out[0].element_size()
+    steps = max(args.e2e_steps, 8)
+
+    def one(i):
+        li = i % s_layers
+        L, inp, h = layers[li], inputs[li], host_in[li]
+        for k in ("C", "Z", "q", "q_I", "w"):
+            inp[k].copy_(h[k], non_blocking=True)
+        L.win[:, -1:].copy_(h["win_row"], non_blocking=True)
+        L.step(inp["C"], inp["Z"], inp["b_pos"], inp["W_IK"], inp["q"], inp["q_I"], inp["w"], stream=stream)
+        host_out[li].copy_(L.out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(8):
+            one(i)
+    stream.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for i in range(steps):
+            one(i)
+        t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms = float(tt.item())
+    B = layers[0].s.B
+    return {"value": B * steps * world / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": nbytes_in,
+            "d2h_bytes_per_step": nbytes_out, "steps": steps}
+
+
+def main():
+    args = parse()
+    rank, world = dist_init(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,286 @@
+"""Python binding of the B200 CSA library (libcsa_b200.so, C ABI in include/csa.h).
+
+Argument marshalling only: every step runs in the CUDA kernels behind the C ABI.  torch supplies
+device memory, streams and output/workspace allocation.  There is no CPU fallback: importing this
+package fails loudly when the library has not been built, and every call requires CUDA tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcsa_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m compressed_sparse_attention_18_b200.build` "
+        "(nvcc, sm_100a).  There is no CPU fallback.")
+_lib = ctypes.CDLL(LIB_PATH)
+
+ENTRY_POINTS = ("csa_status_string", "csa_version", "csa_last_cuda_error", "csa_compress", "csa_pack_fp4",
+                "csa_index_topk_workspace_size", "csa_index_topk", "csa_index_scores", "csa_topk_workspace_size",
+                "csa_topk", "csa_attn_workspace_size", "csa_sparse_attn", "hca_dense_attn")
+
+_u32, _i32, _f32, _vp = ctypes.c_uint32, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p
+
+
+class CompressArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("B", _i32), ("T", _i32), ("d_model", _i32), ("d", _i32),
+                ("d_rope", _i32), ("d_index", _i32), ("ratio", _i32), ("rope_theta", _f32), ("pos0", _vp),
+                ("x", _vp), ("W_kv", _vp), ("W_g", _vp), ("C", _vp), ("Z", _vp), ("b_pos", _vp),
+                ("W_IK", _vp), ("c_out", _vp), ("kI_out", _vp)]
+
+
+class PackArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("B", _i32), ("n", _i32), ("d", _i32), ("d_rope", _i32),
+                ("n_max", _i32), ("global_scale", _f32), ("src", _vp), ("row0", _vp), ("codes", _vp),
+                ("scales", _vp), ("rope", _vp)]
+
+
+class IndexArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("B", _i32), ("Nq", _i32), ("H_I", _i32), ("d_I", _i32),
+                ("ratio", _i32), ("k", _i32), ("n_max", _i32), ("g_q", _f32), ("g_k", _f32), ("q_I", _vp),
+                ("w", _vp), ("k_codes", _vp), ("k_scales", _vp), ("n_c", _vp), ("q_pos", _vp),
+                ("cand", _vp), ("n_cand", _i32), ("pool_blocks", _i32), ("pool_block_size", _i32),
+                ("pool_out", _vp), ("idx_out", _vp), ("scores_out", _vp)]
+
+
+class AttnArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("B", _i32), ("Nq", _i32), ("H", _i32), ("d", _i32), ("d_rope", _i32),
+                ("ratio", _i32), ("n_max", _i32), ("k", _i32), ("Wn", _i32), ("window", _i32),
+                ("g_kv", _f32), ("softmax_scale", _f32), ("q", _vp), ("q_pos", _vp), ("kv_codes", _vp),
+                ("kv_scales", _vp), ("kv_rope", _vp), ("n_c", _vp), ("idx", _vp), ("win_kv", _vp),
+                ("win_pos0", _vp), ("out", _vp), ("lse", _vp)]
+
+
+_lib.csa_status_string.restype = ctypes.c_char_p
+_lib.csa_status_string.argtypes = [ctypes.c_int]
+_lib.csa_version.restype = ctypes.c_int
+_lib.csa_last_cuda_error.restype = ctypes.c_int
+for _name, _st in (("csa_compress", CompressArgs), ("csa_pack_fp4", PackArgs)):
+    getattr(_lib, _name).restype = ctypes.c_int
+    getattr(_lib, _name).argtypes = [ctypes.POINTER(_st), _vp]
+_lib.csa_index_topk_workspace_size.restype = ctypes.c_size_t
+_lib.csa_index_topk_workspace_size.argtypes = [ctypes.POINTER(IndexArgs)]
+_lib.csa_index_topk.restype = ctypes.c_int
+_lib.csa_index_topk.argtypes = [ctypes.POINTER(IndexArgs), _vp, ctypes.c_size_t, _vp]
+_lib.csa_index_scores.restype = ctypes.c_int
+_lib.csa_index_scores.argtypes = [ctypes.POINTER(IndexArgs), _vp, ctypes.c_int64, _vp]
+_lib.csa_topk_workspace_size.restype = ctypes.c_size_t
+_lib.csa_topk_workspace_size.argtypes = [ctypes.POINTER(IndexArgs)]
+_lib.csa_topk.restype = ctypes.c_int
+_lib.csa_topk.argtypes = [ctypes.POINTER(IndexArgs), _vp, ctypes.c_int64, _vp, ctypes.c_size_t, _vp]
+_lib.csa_attn_workspace_size.restype = ctypes.c_size_t
+_lib.csa_attn_workspace_size.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_int]
+for _name in ("csa_sparse_attn", "hca_dense_attn"):
+    getattr(_lib, _name).restype = ctypes.c_int
+    getattr(_lib, _name).argtypes = [ctypes.POINTER(AttnArgs), _vp, ctypes.c_size_t, _vp]
+
+
+class CSAError(RuntimeError):
+    pass
+
+
+def version() -> int:
+    return _lib.csa_version()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        msg = _lib.csa_status_string(status).decode()
+        if status == 4:
+            msg += f" (cudaError {_lib.csa_last_cuda_error()})"
+        raise CSAError(f"{what}: {msg}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise CSAError("tensor is not on a CUDA device (no CPU path)")
+    if not t.is_contiguous():
+        raise CSAError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ws(nbytes: int, device, ws=None):
+    if nbytes == 0:
+        return None
+    if ws is not None and ws.numel() * ws.element_size() >= nbytes:
+        return ws
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------------------------------- API
+
+def compress(*, b_pos, ratio, d_rope=0, rope_theta=0.0, pos0=None, x=None, W_kv=None, W_g=None, C=None, Z=None,
+             W_IK=None, c_out=None, kI_out=None, stream=None):
+    """Compressor.  Projection mode (x [B,T,d_m], W_kv/W_g [d_m,d]) fills C, Z [B,T,d]; pooling mode
+    reads C, Z.  Returns (c [B,T//r,d], k_I [B,T//r,d_I] or None, C, Z)."""
+    if x is not None:
+        B, T, dm = x.shape
+        d = W_kv.shape[1]
+        if C is None:
+            C = torch.empty((B, T, d), dtype=torch.bfloat16, device=x.device)
+        if Z is None:
+            Z = torch.empty((B, T, d), dtype=torch.bfloat16, device=x.device)
+    else:
+        B, T, d = C.shape
+        dm = 0
+    n = T // ratio
+    dI = W_IK.shape[1] if W_IK is not None else 0
+    if c_out is None:
+        c_out = torch.empty((B, n, d), dtype=torch.bfloat16, device=C.device)
+    if W_IK is not None and kI_out is None:
+        kI_out = torch.empty((B, n, dI), dtype=torch.bfloat16, device=C.device)
+    a = CompressArgs(ctypes.sizeof(CompressArgs), B, T, dm, d, d_rope, dI, ratio, rope_theta, _ptr(pos0),
+                     _ptr(x), _ptr(W_kv), _ptr(W_g), _ptr(C), _ptr(Z), _ptr(b_pos), _ptr(W_IK), _ptr(c_out),
+                     _ptr(kI_out) if W_IK is not None else None)
+    _check(_lib.csa_compress(ctypes.byref(a), _stream(stream)), "csa_compress")
+    return c_out, (kI_out if W_IK is not None else None), C, Z
+
+
+class PackedCache:
+    """FP4 cache storage [B, n_max, ...]: codes u8, scales u8 (E4M3), rope bf16."""
+
+    def __init__(self, B, n_max, d, d_rope, device, global_scale=1.0):
+        d_n = d - d_rope
+        s_pad = (d_n // 32 + 3) // 4 * 4
+        self.B, self.n_max, self.d, self.d_rope, self.g = B, n_max, d, d_rope, float(global_scale)
+        self.codes = torch.zeros((B, n_max, d_n // 2), dtype=torch.uint8, device=device)
+        self.scales = torch.zeros((B, n_max, s_pad), dtype=torch.uint8, device=device)
+        self.rope = torch.zeros((B, n_max, max(d_rope, 1) if d_rope else 0), dtype=torch.bfloat16, device=device)
+
+
+def pack_fp4(src, cache: PackedCache, row0=None, stream=None):
+    """Pack src [B, n, d] bf16 into cache rows row0[b] + j (row0 int32 [B] or None = 0)."""
+    B, n, d = src.shape
+    a = PackArgs(ctypes.sizeof(PackArgs), B, n, d, cache.d_rope, cache.n_max, cache.g, _ptr(src), _ptr(row0),
+                 _ptr(cache.codes), _ptr(cache.scales), _ptr(cache.rope) if cache.d_rope else None)
+    _check(_lib.csa_pack_fp4(ctypes.byref(a), _stream(stream)), "csa_pack_fp4")
+    return cache
+
+
+def _index_args(q_I, w, kcache: PackedCache, n_c, q_pos, ratio, k, g_q, cand, pool_blocks, pool_block_size,
+                pool_out, idx_out, scores_out):
+    B, Nq, H_I, d_I = q_I.shape
+    return IndexArgs(ctypes.sizeof(IndexArgs), B, Nq, H_I, d_I, ratio, k, kcache.n_max, g_q, kcache.g, _ptr(q_I),
+                     _ptr(w), _ptr(kcache.codes), _ptr(kcache.scales), _ptr(n_c), _ptr(q_pos), _ptr(cand),
+                     cand.shape[-1] if cand is not None else 0, pool_blocks, pool_block_size, _ptr(pool_out),
+                     _ptr(idx_out), _ptr(scores_out))
+
+
+def index_topk(q_I, w, kcache: PackedCache, n_c, q_pos, *, ratio, k, g_q=1.0, cand=None, pool_blocks=0,
+               pool_block_size=8, want_scores=False, idx_out=None, scores_out=None, pool_out=None, ws=None,
+               stream=None):
+    """Lightning indexer + top-k.  Returns (idx [B,Nq,k] int32, scores [B,Nq,k] or None, pool or None)."""
+    B, Nq = q_I.shape[:2]
+    dev = q_I.device
+    if idx_out is None:
+        idx_out = torch.empty((B, Nq, k), dtype=torch.int32, device=dev)
+    if want_scores and scores_out is None:
+        scores_out = torch.empty((B, Nq, k), dtype=torch.float32, device=dev)
+    if pool_blocks and pool_out is None:
+        pool_out = torch.empty((B, Nq, pool_blocks * pool_block_size), dtype=torch.int32, device=dev)
+    a = _index_args(q_I, w, kcache, n_c, q_pos, ratio, k, g_q, cand, pool_blocks, pool_block_size, pool_out,
+                    idx_out, scores_out)
+    nbytes = _lib.csa_index_topk_workspace_size(ctypes.byref(a))
+    wbuf = _ws(nbytes, dev, ws)
+    _check(_lib.csa_index_topk(ctypes.byref(a), _ptr(wbuf) if wbuf is not None else None, nbytes,
+                               _stream(stream)), "csa_index_topk")
+    return idx_out, scores_out, pool_out
+
+
+def index_scores(q_I, w, kcache: PackedCache, n_c, q_pos, scores, *, ratio, g_q=1.0, cand=None, stream=None):
+    """Lightning-indexer scores only, into scores [B*Nq, ld] fp32 (see csa_index_scores)."""
+    a = _index_args(q_I, w, kcache, n_c, q_pos, ratio, 1, g_q, cand, 0, 8, None, None, None)
+    _check(_lib.csa_index_scores(ctypes.byref(a), _ptr(scores), scores.shape[-1], _stream(stream)),
+           "csa_index_scores")
+    return scores
+
+
+def topk(scores, kcache: PackedCache, n_c, q_pos, *, B, Nq, ratio, k, cand=None, pool_blocks=0, pool_block_size=8,
+         want_scores=False, idx_out=None, scores_out=None, pool_out=None, ws=None, stream=None):
+    """Top-k (+ hierarchical pool) over a score matrix written by index_scores (see csa_topk)."""
+    dev = scores.device
+    if idx_out is None:
+        idx_out = torch.empty((B, Nq, k), dtype=torch.int32, device=dev)
+    if want_scores and scores_out is None:
+        scores_out = torch.empty((B, Nq, k), dtype=torch.float32, device=dev)
+    if pool_blocks and pool_out is None:
+        pool_out = torch.empty((B, Nq, pool_blocks * pool_block_size), dtype=torch.int32, device=dev)
+    d_I = 2 * kcache.codes.shape[-1]
+    a = IndexArgs(ctypes.sizeof(IndexArgs), B, Nq, 1, d_I, ratio, k, kcache.n_max, 1.0, kcache.g, None, None,
+                  None, None, _ptr(n_c), _ptr(q_pos), _ptr(cand), cand.shape[-1] if cand is not None else 0,
+                  pool_blocks, pool_block_size, _ptr(pool_out), _ptr(idx_out), _ptr(scores_out))
+    nbytes = _lib.csa_topk_workspace_size(ctypes.byref(a))
+    wbuf = _ws(nbytes, dev, ws)
+    _check(_lib.csa_topk(ctypes.byref(a), _ptr(scores), scores.shape[-1], _ptr(wbuf) if wbuf is not None else None,
+                         nbytes, _stream(stream)), "csa_topk")
+    return idx_out, scores_out, pool_out
+
+
+def topk_workspace_size(kcache, n_c, q_pos, *, B, Nq, ratio, k, cand=None, pool_blocks=0, pool_block_size=8):
+    d_I = 2 * kcache.codes.shape[-1]
+    a = IndexArgs(ctypes.sizeof(IndexArgs), B, Nq, 1, d_I, ratio, k, kcache.n_max, 1.0, kcache.g, None, None,
+                  None, None, _ptr(n_c), _ptr(q_pos), _ptr(cand), cand.shape[-1] if cand is not None else 0,
+                  pool_blocks, pool_block_size, 256 if pool_blocks else None, 256, None)
+    return _lib.csa_topk_workspace_size(ctypes.byref(a))
+
+
+def index_topk_workspace_size(q_I, w, kcache, n_c, q_pos, *, ratio, k, g_q=1.0, cand=None, pool_blocks=0,
+                              pool_block_size=8):
+    a = _index_args(q_I, w, kcache, n_c, q_pos, ratio, k, g_q, cand, pool_blocks, pool_block_size, None, None,
+                    None)
+    return _lib.csa_index_topk_workspace_size(ctypes.byref(a))
+
+
+def _attn_args(q, q_pos, cache: PackedCache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse):
+    B, Nq, H, d = q.shape
+    k = idx.shape[-1] if idx is not None else 0
+    Wn = win_kv.shape[1] if win_kv is not None else 0
+    return AttnArgs(ctypes.sizeof(AttnArgs), B, Nq, H, d, cache.d_rope, ratio, cache.n_max, k, Wn, window, cache.g,
+                    softmax_scale, _ptr(q), _ptr(q_pos), _ptr(cache.codes), _ptr(cache.scales), _ptr(cache.rope),
+                    _ptr(n_c), _ptr(idx), _ptr(win_kv), _ptr(win_pos0), _ptr(out), _ptr(lse))
+
+
+def _attn(fn, hca, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse, ws,
+          stream):
+    B, Nq, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Nq, H), dtype=torch.float32, device=q.device)
+    a = _attn_args(q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse)
+    nbytes = _lib.csa_attn_workspace_size(ctypes.byref(a), hca)
+    wbuf = _ws(nbytes, q.device, ws)
+    _check(fn(ctypes.byref(a), _ptr(wbuf) if wbuf is not None else None, nbytes, _stream(stream)),
+           "hca_dense_attn" if hca else "csa_sparse_attn")
+    return out, lse
+
+
+def sparse_attn(q, q_pos, cache: PackedCache, n_c, idx, win_kv=None, win_pos0=None, *, ratio=4, window=128,
+                softmax_scale=0.0, out=None, lse=None, ws=None, stream=None):
+    """CSA attention over the selected entries idx [B,Nq,k] plus the window.  Returns (out, lse)."""
+    return _attn(_lib.csa_sparse_attn, 0, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window,
+                 softmax_scale, out, lse, ws, stream)
+
+
+def hca_attn(q, q_pos, cache: PackedCache, n_c, win_kv=None, win_pos0=None, *, ratio=128, window=128,
+             softmax_scale=0.0, out=None, lse=None, ws=None, stream=None):
+    """HCA attention over every visible entry plus the window.  Returns (out, lse)."""
+    return _attn(_lib.hca_dense_attn, 1, q, q_pos, cache, n_c, None, win_kv, win_pos0, ratio, window,
+                 softmax_scale, out, lse, ws, stream)
+
+
+def attn_workspace_size(q, q_pos, cache, n_c, idx, win_kv, win_pos0, *, ratio, window, hca=False):
+    a = _attn_args(q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, 0.0, None, None)
+    return _lib.csa_attn_workspace_size(ctypes.byref(a), 1 if hca else 0)

@@ -1,0 +1,444 @@
+// Attention over compressed entries plus the sliding window: CSA (the selected entries) and HCA
+// (every visible entry).  One joint softmax per (query, head); one KV head shared by all query heads.
+// Sources: "DeepSeek-V4: エージェントが実際に使える100万トークンのコンテキスト", §ハイブリッド注意, Fig. 3 (attention
+// over the top-k compressed entries, with a sliding-window branch for the recent uncompressed tokens)
+// and Fig. 4 (HCA: dense attention over the compressed stream, same window branch).
+//
+// Kernel: a CTA takes one query (all H heads, padded to 16-row groups) and a range of 64-key chunks
+// of that query's key list [selected or visible entries ‖ window rows].  Per chunk: gather + dequantise
+// the keys into shared memory as bf16 (E2M1 x E4M3 scale x g is exact in bf16), S = Q·K^T on the
+// tensor pipe (mma.sync bf16, fp32 accumulate; the head dim is split over DS warps and the partial S
+// tiles are summed through shared memory), online softmax in fp32 (exp2 with log2(e) folded into the
+// scale), O += P·V with P in bf16.  Split-K partials (O, lse) are merged by a second kernel.
+#include "csa_common.cuh"
+
+namespace csa {
+
+constexpr int AT_KC = 64;        // keys per chunk
+constexpr int AT_WARPS = 8;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Byte offset of 16-byte chunk `c` of row `r` in a [rows][D] bf16 tile, chunks XOR-swizzled by row.
+template <int D>
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+  return (uint32_t)(r * (D * 2) + ((c ^ (r & 7)) << 4));
+}
+
+struct AttnParams {
+  int B, Nq, H, d_r, ratio, n_max, k, Wn, window, splits, chunks_per_split, hca;
+  float g, scale_log2;
+  const uint16_t* q;
+  const int64_t* q_pos;
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const uint16_t* rope;
+  const int32_t* n_c;
+  const int32_t* idx;
+  const uint16_t* win;
+  const int64_t* win_pos0;
+  uint16_t* out;
+  float* lse;
+  float* part_o;    // [B*Nq][splits][H][D]
+  float* part_lse;  // [B*Nq][splits][H]
+};
+
+template <int D, int DS>
+__global__ void __launch_bounds__(AT_WARPS * 32, 1) attn_kernel(AttnParams P) {
+  constexpr int HG = AT_WARPS / DS;         // 16-row head groups
+  constexpr int HP = HG * 16;               // padded heads
+  constexpr int DSL = D / DS;               // head-dim slice of one warp
+  constexpr int NT_O = DSL / 8;             // O n-tiles per warp
+  constexpr int NT_S = AT_KC / 8;           // S n-tiles
+  constexpr int CH = D / 8;                 // 16-byte chunks per row
+  const int d_n = D - P.d_r;
+  const int S_blocks = d_n / 32;
+  const int S_pad = (S_blocks + 3) & ~3;
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* sQ = smem;                                   // [HP][D] bf16
+  uint8_t* sK = sQ + HP * D * 2;                        // [AT_KC][D] bf16
+  float* sS = reinterpret_cast<float*>(sK + AT_KC * D * 2);  // [HG][DS][16][AT_KC]
+  __shared__ int s_valid[AT_KC];
+
+  const int unit = blockIdx.x;
+  const int bq = unit / P.splits, split = unit % P.splits;
+  const int b = bq / P.Nq;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int hg = warp / DS, ds = warp % DS;
+  const int g = lane >> 2, t = lane & 3;
+
+  const long long tq = P.q_pos[bq];
+  const int ncb = min(P.n_c[b], P.n_max);   // entries beyond the cache capacity do not exist
+  int n_sel;
+  if (P.hca) {
+    long long nv = (tq + 1) / P.ratio;
+    n_sel = (int)max(0LL, min((long long)ncb, nv));
+  } else {
+    n_sel = P.k;
+  }
+  long long wlo = 0, whi = -1;
+  if (P.win && P.Wn > 0) {
+    const long long p0 = P.win_pos0[b];
+    wlo = max(max(0LL, tq - P.window + 1), p0);
+    whi = min(tq, p0 + P.Wn - 1);
+  }
+  const int n_win = whi >= wlo ? (int)(whi - wlo + 1) : 0;
+  const int n_list = n_sel + n_win;
+  const int n_chunks = (n_list + AT_KC - 1) / AT_KC;
+  const int c_begin = split * P.chunks_per_split;
+  const int c_end = min(n_chunks, c_begin + P.chunks_per_split);
+
+  // Q -> shared (rows >= H zero)
+  const uint16_t* qsrc = P.q + (size_t)bq * P.H * D;
+  for (int i = tid; i < HP * CH; i += blockDim.x) {
+    const int r = i / CH, c = i % CH;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < P.H) v = *reinterpret_cast<const uint4*>(qsrc + (size_t)r * D + c * 8);
+    *reinterpret_cast<uint4*>(sQ + swz<D>(r, c)) = v;
+  }
+
+  float o[NT_O][4];
+#pragma unroll
+  for (int j = 0; j < NT_O; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
+
+  const uint32_t sQa = (uint32_t)__cvta_generic_to_shared(sQ);
+  const uint32_t sKa = (uint32_t)__cvta_generic_to_shared(sK);
+  const uint8_t* codes_b = P.codes + (size_t)b * P.n_max * (d_n / 2);
+  const uint8_t* scales_b = P.scales + (size_t)b * P.n_max * S_pad;
+  const uint16_t* rope_b = P.rope + (size_t)b * P.n_max * P.d_r;
+  const int32_t* idx_row = P.idx ? P.idx + (size_t)bq * P.k : nullptr;
+
+  for (int c = c_begin; c < c_end; ++c) {
+    __syncthreads();  // previous chunk's K tile fully consumed
+    // ---- gather: each warp fills AT_KC / AT_WARPS rows
+    for (int rr = 0; rr < AT_KC / AT_WARPS; ++rr) {
+      const int row = warp * (AT_KC / AT_WARPS) + rr;
+      const int li = c * AT_KC + row;
+      int kind = 0;  // 0 invalid, 1 entry, 2 window
+      long long src = 0;
+      if (li < n_sel) {
+        const int id = P.hca ? li : idx_row[li];
+        if (id >= 0 && id < ncb) { kind = 1; src = id; }
+      } else if (li < n_list) {
+        kind = 2;
+        src = (wlo + (li - n_sel)) - P.win_pos0[b];
+      }
+      if (kind == 1) {
+        if (lane < S_blocks) {
+          const uint4 cv = *reinterpret_cast<const uint4*>(codes_b + src * (d_n / 2) + lane * 16);
+          const float s = e4m3_to_f32(scales_b[src * S_pad + lane]) * P.g;
+          const uint32_t w4[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t outw[4];
+#pragma unroll
+            for (int bb = 0; bb < 4; bb += 2) {
+              const uint32_t h0 = e2m1x2_to_h2(w4[q4] >> (bb * 8));
+              const uint32_t h1 = e2m1x2_to_h2(w4[q4] >> (bb * 8 + 8));
+              const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+              const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+              outw[bb] = pack_bf16x2(f0.x * s, f0.y * s);
+              outw[bb + 1] = pack_bf16x2(f1.x * s, f1.y * s);
+            }
+            *reinterpret_cast<uint4*>(sK + swz<D>(row, lane * 4 + q4)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+          }
+        } else if (lane >= 16 && lane < 16 + P.d_r / 8) {
+          const int rc = lane - 16;
+          const uint4 v = *reinterpret_cast<const uint4*>(rope_b + src * P.d_r + rc * 8);
+          *reinterpret_cast<uint4*>(sK + swz<D>(row, d_n / 8 + rc)) = v;
+        }
+      } else if (kind == 2) {
+        const uint16_t* wrow = P.win + ((size_t)b * P.Wn + src) * D;
+        for (int cc = lane; cc < CH; cc += 32)
+          *reinterpret_cast<uint4*>(sK + swz<D>(row, cc)) = *reinterpret_cast<const uint4*>(wrow + cc * 8);
+      } else {
+        for (int cc = lane; cc < CH; cc += 32) *reinterpret_cast<uint4*>(sK + swz<D>(row, cc)) = make_uint4(0, 0, 0, 0);
+      }
+      if (lane == 0) s_valid[row] = kind != 0;
+    }
+    __syncthreads();
+
+    // ---- S partial over this warp's head-dim slice
+    float sacc[NT_S][4];
+#pragma unroll
+    for (int j = 0; j < NT_S; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
+#pragma unroll 4
+    for (int ks = 0; ks < DSL / 16; ++ks) {
+      const int k0 = ds * DSL + ks * 16;
+      uint32_t af[4];
+      {
+        const int r = hg * 16 + (lane & 15);
+        const int cchunk = k0 / 8 + (lane >> 4);
+        ldsm4(sQa + swz<D>(r, cchunk), af);
+      }
+#pragma unroll
+      for (int j = 0; j < NT_S; j += 2) {
+        uint32_t bf[4];
+        const int mi = lane >> 3;
+        const int key = j * 8 + (mi >> 1) * 8 + (lane & 7);
+        const int cchunk = k0 / 8 + (mi & 1);
+        ldsm4(sKa + swz<D>(key, cchunk), bf);
+        mma16816(sacc[j], af, bf[0], bf[1]);
+        mma16816(sacc[j + 1], af, bf[2], bf[3]);
+      }
+    }
+    if (DS > 1) {
+      float* mine = sS + ((size_t)(hg * DS + ds) * 16) * AT_KC;
+#pragma unroll
+      for (int j = 0; j < NT_S; ++j) {
+        mine[g * AT_KC + j * 8 + 2 * t] = sacc[j][0];
+        mine[g * AT_KC + j * 8 + 2 * t + 1] = sacc[j][1];
+        mine[(g + 8) * AT_KC + j * 8 + 2 * t] = sacc[j][2];
+        mine[(g + 8) * AT_KC + j * 8 + 2 * t + 1] = sacc[j][3];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int od = 0; od < DS; ++od) {
+        if (od == ds) continue;
+        const float* other = sS + ((size_t)(hg * DS + od) * 16) * AT_KC;
+#pragma unroll
+        for (int j = 0; j < NT_S; ++j) {
+          sacc[j][0] += other[g * AT_KC + j * 8 + 2 * t];
+          sacc[j][1] += other[g * AT_KC + j * 8 + 2 * t + 1];
+          sacc[j][2] += other[(g + 8) * AT_KC + j * 8 + 2 * t];
+          sacc[j][3] += other[(g + 8) * AT_KC + j * 8 + 2 * t + 1];
+        }
+      }
+    }
+    // ---- online softmax (rows g and g + 8 of this head group)
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int j = 0; j < NT_S; ++j) {
+      const bool v0 = s_valid[j * 8 + 2 * t], v1 = s_valid[j * 8 + 2 * t + 1];
+      sacc[j][0] = v0 ? sacc[j][0] * P.scale_log2 : -INFINITY;
+      sacc[j][1] = v1 ? sacc[j][1] * P.scale_log2 : -INFINITY;
+      sacc[j][2] = v0 ? sacc[j][2] * P.scale_log2 : -INFINITY;
+      sacc[j][3] = v1 ? sacc[j][3] * P.scale_log2 : -INFINITY;
+      mx[0] = fmaxf(mx[0], fmaxf(sacc[j][0], sacc[j][1]));
+      mx[1] = fmaxf(mx[1], fmaxf(sacc[j][2], sacc[j][3]));
+    }
+    float corr[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+      const float mnew = fmaxf(m_r[h], mx[h]);
+      corr[h] = (mnew == -INFINITY) ? 1.f : exp2f(m_r[h] - mnew);
+      m_r[h] = mnew;
+    }
+    float rs[2] = {0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < NT_S; ++j) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int h = e >> 1;
+        const float p = (m_r[h] == -INFINITY) ? 0.f : exp2f(sacc[j][e] - m_r[h]);
+        sacc[j][e] = p;
+        rs[h] += p;
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      rs[h] += __shfl_xor_sync(0xffffffffu, rs[h], 1);
+      rs[h] += __shfl_xor_sync(0xffffffffu, rs[h], 2);
+      l_r[h] = l_r[h] * corr[h] + rs[h];
+    }
+#pragma unroll
+    for (int j = 0; j < NT_O; ++j) {
+      o[j][0] *= corr[0]; o[j][1] *= corr[0];
+      o[j][2] *= corr[1]; o[j][3] *= corr[1];
+    }
+    // ---- O += P · V over this warp's head-dim slice
+#pragma unroll
+    for (int kk = 0; kk < AT_KC / 16; ++kk) {
+      uint32_t pa[4];
+      pa[0] = pack_bf16x2(sacc[2 * kk][0], sacc[2 * kk][1]);
+      pa[1] = pack_bf16x2(sacc[2 * kk][2], sacc[2 * kk][3]);
+      pa[2] = pack_bf16x2(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]);
+      pa[3] = pack_bf16x2(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3]);
+#pragma unroll
+      for (int j = 0; j < NT_O; j += 2) {
+        uint32_t bf[4];
+        const int mi = lane >> 3;
+        const int key = kk * 16 + (mi & 1) * 8 + (lane & 7);
+        const int cchunk = (ds * DSL + j * 8) / 8 + (mi >> 1);
+        ldsm4t(sKa + swz<D>(key, cchunk), bf);
+        mma16816(o[j], pa, bf[0], bf[1]);
+        mma16816(o[j + 1], pa, bf[2], bf[3]);
+      }
+    }
+  }
+
+  // ---- epilogue
+  float inv_l[2], lse_r[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    inv_l[h] = l_r[h] > 0.f ? 1.f / l_r[h] : 0.f;
+    lse_r[h] = l_r[h] > 0.f ? (m_r[h] + log2f(l_r[h])) * LN2 : -INFINITY;
+  }
+  const int rows[2] = {hg * 16 + g, hg * 16 + g + 8};
+  if (P.splits == 1) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (rows[h] >= P.H) continue;
+      uint16_t* orow = P.out + ((size_t)bq * P.H + rows[h]) * D + ds * DSL;
+#pragma unroll
+      for (int j = 0; j < NT_O; ++j)
+        *reinterpret_cast<uint32_t*>(orow + j * 8 + 2 * t) =
+            pack_bf16x2(o[j][2 * h] * inv_l[h], o[j][2 * h + 1] * inv_l[h]);
+      if (P.lse && ds == 0 && t == 0) P.lse[(size_t)bq * P.H + rows[h]] = lse_r[h];
+    }
+  } else {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (rows[h] >= P.H) continue;
+      float* orow = P.part_o + (((size_t)bq * P.splits + split) * P.H + rows[h]) * D + ds * DSL;
+#pragma unroll
+      for (int j = 0; j < NT_O; ++j)
+        *reinterpret_cast<float2*>(orow + j * 8 + 2 * t) = make_float2(o[j][2 * h] * inv_l[h], o[j][2 * h + 1] * inv_l[h]);
+      if (ds == 0 && t == 0) P.part_lse[((size_t)bq * P.splits + split) * P.H + rows[h]] = lse_r[h];
+    }
+  }
+}
+
+// Merge split partials: lse = log sum_s exp(lse_s); out = sum_s exp(lse_s - lse) O_s.
+__global__ void attn_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int splits,
+                                  int H, int D, uint16_t* __restrict__ out, float* __restrict__ lse) {
+  const int bq = blockIdx.x;
+  for (int hd = threadIdx.x; hd < H * D; hd += blockDim.x) {
+    const int h = hd / D;
+    float mx = -INFINITY;
+    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_lse[((size_t)bq * splits + s) * H + h]);
+    float acc = 0.f, wsum = 0.f;
+    if (mx > -INFINITY) {
+      for (int s = 0; s < splits; ++s) {
+        const float ls = part_lse[((size_t)bq * splits + s) * H + h];
+        if (ls == -INFINITY) continue;
+        const float w = exp2f((ls - mx) * LOG2E);
+        wsum += w;
+        acc = fmaf(w, part_o[(((size_t)bq * splits + s) * H + h) * D + (hd % D)], acc);
+      }
+    }
+    out[(size_t)bq * H * D + hd] = (uint16_t)f_to_bf16_bits(wsum > 0.f ? acc / wsum : 0.f);
+    if (lse && hd % D == 0) lse[(size_t)bq * H + h] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
+  }
+}
+
+struct AttnPlan {
+  int splits, cps;
+  size_t off_o, off_lse, total;
+};
+
+static AttnPlan plan_attn(const csa_attn_args* a, int hca) {
+  AttnPlan p{};
+  const long long n_sel = hca ? a->n_max : a->k;
+  const long long n_win = (a->win_kv && a->Wn > 0) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
+  const long long chunks = (n_sel + n_win + AT_KC - 1) / AT_KC;
+  const long long rows = (long long)a->B * a->Nq;
+  long long splits = rows >= 148 ? 1 : (296 + rows - 1) / rows;
+  if (splits > chunks) splits = chunks;
+  if (splits < 1) splits = 1;
+  p.cps = (int)((chunks + splits - 1) / splits);
+  if (p.cps < 1) p.cps = 1;
+  p.splits = (int)((chunks + p.cps - 1) / p.cps);
+  if (p.splits < 1) p.splits = 1;
+  size_t o = 0;
+  if (p.splits > 1) {
+    p.off_o = o;   o = align_up(o + (size_t)rows * p.splits * a->H * a->d * 4, 256);
+    p.off_lse = o; o = align_up(o + (size_t)rows * p.splits * a->H * 4, 256);
+  }
+  p.total = o;
+  return p;
+}
+
+static csa_status validate_attn(const csa_attn_args* a, int hca) {
+  CSA_REQUIRE(a != nullptr && a->struct_size == sizeof(csa_attn_args));
+  CSA_REQUIRE(a->B >= 0 && a->Nq >= 0 && a->H >= 1 && a->ratio >= 1 && a->n_max >= 0 && a->Wn >= 0 && a->window >= 1);
+  CSA_SUPPORTED((a->d == 512 && a->d_rope == 64) || (a->d == 128 && a->d_rope == 32));
+  CSA_SUPPORTED(a->H <= (a->d == 512 ? 64 : 16));
+  CSA_REQUIRE(a->g_kv > 0.0f);
+  if (!hca) CSA_REQUIRE(a->k >= 1);
+  if ((long long)a->B * a->Nq == 0) return CSA_OK;
+  CSA_REQUIRE(a->q && a->q_pos && a->n_c && a->out);
+  CSA_REQUIRE(a->n_max == 0 || (a->kv_codes && a->kv_scales && a->kv_rope));
+  if (!hca) CSA_REQUIRE(a->idx != nullptr);
+  if (a->Wn > 0) CSA_REQUIRE(a->win_kv && a->win_pos0);
+  return CSA_OK;
+}
+
+template <int D, int DS>
+static csa_status launch_attn(const AttnParams& P, int units, cudaStream_t st) {
+  constexpr int HG = AT_WARPS / DS;
+  const size_t smem = (size_t)HG * 16 * D * 2 + (size_t)AT_KC * D * 2 + (DS > 1 ? (size_t)HG * DS * 16 * AT_KC * 4 : 0);
+  static std::atomic<unsigned> attr_done{0};
+  set_smem_once((const void*)attn_kernel<D, DS>, (int)smem, attr_done);
+  attn_kernel<D, DS><<<units, AT_WARPS * 32, smem, st>>>(P);
+  return launch_status();
+}
+
+static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, void* stream, int hca) {
+  csa_status v = validate_attn(a, hca);
+  if (v != CSA_OK) return v;
+  const long long rows = (long long)a->B * a->Nq;
+  if (rows == 0) return CSA_OK;
+  const AttnPlan p = plan_attn(a, hca);
+  if (ws_bytes < p.total) return CSA_ERR_WORKSPACE;
+  CSA_REQUIRE(p.total == 0 || ws != nullptr);
+  cudaStream_t st = (cudaStream_t)stream;
+  AttnParams P{};
+  P.B = a->B; P.Nq = a->Nq; P.H = a->H; P.d_r = a->d_rope; P.ratio = a->ratio; P.n_max = a->n_max;
+  P.k = a->k; P.Wn = a->win_kv ? a->Wn : 0; P.window = a->window; P.splits = p.splits;
+  P.chunks_per_split = p.cps; P.hca = hca;
+  P.g = a->g_kv;
+  const float scale = a->softmax_scale != 0.0f ? a->softmax_scale : 1.0f / sqrtf((float)a->d);
+  P.scale_log2 = scale * LOG2E;
+  P.q = (const uint16_t*)a->q; P.q_pos = a->q_pos; P.codes = a->kv_codes; P.scales = a->kv_scales;
+  P.rope = (const uint16_t*)a->kv_rope; P.n_c = a->n_c; P.idx = hca ? nullptr : a->idx;
+  P.win = (const uint16_t*)a->win_kv; P.win_pos0 = a->win_pos0; P.out = (uint16_t*)a->out; P.lse = a->lse;
+  P.part_o = p.splits > 1 ? (float*)((uint8_t*)ws + p.off_o) : nullptr;
+  P.part_lse = p.splits > 1 ? (float*)((uint8_t*)ws + p.off_lse) : nullptr;
+  const int units = (int)(rows * p.splits);
+  csa_status s;
+  if (a->d == 512)
+    s = launch_attn<512, 2>(P, units, st);
+  else
+    s = launch_attn<128, 8>(P, units, st);
+  if (s != CSA_OK || p.splits == 1) return s;
+  attn_merge_kernel<<<(unsigned)rows, 256, 0, st>>>(P.part_o, P.part_lse, p.splits, a->H, a->d, (uint16_t*)a->out, a->lse);
+  return launch_status();
+}
+
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" size_t csa_attn_workspace_size(const csa_attn_args* a, int hca) {
+  if (validate_attn(a, hca) != CSA_OK) return 0;
+  return plan_attn(a, hca).total;
+}
+
+extern "C" csa_status csa_sparse_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, void* stream) {
+  return run_attn(a, ws, ws_bytes, stream, 0);
+}
+
+extern "C" csa_status hca_dense_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, void* stream) {
+  return run_attn(a, ws, ws_bytes, stream, 1);
+}

@@ -1,0 +1,257 @@
+// Compressor: C = x·W_kv and Z = x·W_g (bf16 out), then per-channel softmax-gated pooling of
+// non-overlapping groups of r tokens with a learned per-slot bias, RoPE on the pooled RoPE slice,
+// and the indexer-key projection k_I = c·W_IK.
+// Sources: "DeepSeek-V4: エージェントが実際に使える100万トークンのコンテキスト", §ハイブリッド注意, Fig. 3 (every 4
+// tokens folded into one entry by softmax-gated pooling with a learned positional bias) and Fig. 4
+// (128x for HCA); "DeepSeek-V4.1-Flash - Pushing the Limits of KV Cache Compression", CED bullet eq.(1)
+// (entries C and gate logits Z are separate projections) and CSA2 bullet (no overlapping entries;
+// indexer K projected from the main KV).
+#include "csa_common.cuh"
+
+namespace csa {
+
+// ------------------------------------------------------------------------------------------ GEMM
+// C[M][N] = A[M][K] · W[K][N], bf16 in, fp32 accumulate, bf16 out.  128x128x32 tiles, 8 warps
+// (2 x 4, 64x32 each), 3-stage cp.async pipeline, ldmatrix from XOR-swizzled shared memory.
+// blockIdx.z selects (W0, C0) or (W1, C1) so both projections run in one launch.
+
+constexpr int GBM = 128, GBN = 128, GBK = 32, GSTAGES = 3;
+constexpr int G_A_BYTES = GBM * GBK * 2;   // 8 KB
+constexpr int G_B_BYTES = GBK * GBN * 2;   // 8 KB
+constexpr int G_SMEM = GSTAGES * (G_A_BYTES + G_B_BYTES);
+
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g, bool pred) {
+  const int sz = pred ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(g), "r"(sz));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__global__ void __launch_bounds__(256) gemm_bf16_kernel(const uint16_t* __restrict__ A,
+                                                        const uint16_t* __restrict__ W0,
+                                                        const uint16_t* __restrict__ W1, uint16_t* C0,
+                                                        uint16_t* C1, int M, int N, int K) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint16_t* W = blockIdx.z ? W1 : W0;
+  uint16_t* C = blockIdx.z ? C1 : C0;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wm = warp >> 2, wn = warp & 3;
+  const int m0 = blockIdx.y * GBM, n0 = blockIdx.x * GBN;
+  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+  auto sA = [&](int st) { return sbase + st * (G_A_BYTES + G_B_BYTES); };
+  auto sB = [&](int st) { return sbase + st * (G_A_BYTES + G_B_BYTES) + G_A_BYTES; };
+
+  auto load_stage = [&](int st, int k0) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int c = tid + i * 256;          // A: 128 rows x 4 chunks
+      const int row = c >> 2, col = c & 3;
+      const int gm = m0 + row;
+      const bool ok = gm < M;
+      const uint16_t* g = A + (size_t)(ok ? gm : 0) * K + k0 + col * 8;
+      cp_async16(sA(st) + row * 64 + ((col ^ ((row >> 1) & 3)) << 4), g, ok);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int c = tid + i * 256;          // B: 32 rows (k) x 16 chunks (n)
+      const int row = c >> 4, col = c & 15;
+      const uint16_t* g = W + (size_t)(k0 + row) * N + n0 + col * 8;
+      cp_async16(sB(st) + row * 256 + ((col ^ (row & 7)) << 4), g, true);
+    }
+  };
+
+  float acc[4][4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.0f;
+
+  const int KT = K / GBK;
+#pragma unroll
+  for (int s = 0; s < GSTAGES - 1; ++s) {
+    if (s < KT) load_stage(s, s * GBK);
+    cp_async_commit();
+  }
+  for (int kt = 0; kt < KT; ++kt) {
+    cp_async_wait<GSTAGES - 2>();
+    __syncthreads();
+    const int nxt = kt + GSTAGES - 1;
+    if (nxt < KT) load_stage(nxt % GSTAGES, nxt * GBK);
+    cp_async_commit();
+    const int st = kt % GSTAGES;
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      uint32_t af[4][4], bfr[4][2];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int row = wm * 64 + i * 16 + (lane & 15);
+        const int chunk = kk * 2 + (lane >> 4);
+        ldsm_x4(sA(st) + row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4), af[i][0], af[i][1], af[i][2], af[i][3]);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; j += 2) {
+        const int krow = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int nchunk = (wn * 32 + j * 8) / 8 + (lane >> 4);
+        ldsm_x4_t(sB(st) + krow * 256 + ((nchunk ^ (krow & 7)) << 4), bfr[j][0], bfr[j][1], bfr[j + 1][0],
+                  bfr[j + 1][1]);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mma_bf16(acc[i][j], af[i], bfr[j]);
+    }
+  }
+  cp_async_wait<0>();
+  // epilogue: bf16 round, 32-bit stores
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int col = n0 + wn * 32 + j * 8 + 2 * t;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = m0 + wm * 64 + i * 16 + g + h * 8;
+        if (row < M)
+          *reinterpret_cast<uint32_t*>(C + (size_t)row * N + col) = pack_bf16x2(acc[i][j][2 * h], acc[i][j][2 * h + 1]);
+      }
+    }
+}
+
+// --------------------------------------------------------------------------------------- pooling
+// One CTA per (sequence, group of ENT entries).  Threads walk the d channels: per-channel online
+// softmax over the r slots of (Z + b_pos), weighted sum of C; RoPE on the last d_r channels at the
+// group-start position (angles in double); bf16 round; then k_I = bf16(c · W_IK).
+constexpr int POOL_ENT = 4;
+
+__global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ C, const uint16_t* __restrict__ Z,
+                                                   const float* __restrict__ b_pos, int T, int d, int d_r,
+                                                   int r, float theta, const int64_t* __restrict__ pos0,
+                                                   const uint16_t* __restrict__ W_IK, int d_I,
+                                                   uint16_t* __restrict__ c_out, uint16_t* __restrict__ kI_out) {
+  extern __shared__ float pooled[];  // [POOL_ENT][d]
+  const int b = blockIdx.y;
+  const int n_out = T / r;
+  const int e0 = blockIdx.x * POOL_ENT;
+  const int ne = min(POOL_ENT, n_out - e0);
+  const int d_n = d - d_r;
+  for (int q = 0; q < ne; ++q) {
+    const int e = e0 + q;
+    const size_t tok0 = (size_t)b * T + (size_t)e * r;
+    for (int ch = threadIdx.x; ch < d; ch += blockDim.x) {
+      float m = -INFINITY, l = 0.0f, acc = 0.0f;
+      for (int j = 0; j < r; ++j) {
+        const float a = bf16_bits_to_f(Z[(tok0 + j) * d + ch]) + b_pos[(size_t)j * d + ch];
+        const float c = bf16_bits_to_f(C[(tok0 + j) * d + ch]);
+        if (a > m) {
+          const float sc = __expf(m - a);
+          l *= sc;
+          acc *= sc;
+          m = a;
+        }
+        const float p = __expf(a - m);
+        l += p;
+        acc = fmaf(p, c, acc);
+      }
+      pooled[q * d + ch] = acc / l;
+    }
+  }
+  __syncthreads();
+  const int half = d_r >> 1;
+  const long long p0 = pos0 ? pos0[b] : 0;
+  for (int q = 0; q < ne; ++q) {
+    const int e = e0 + q;
+    float* row = pooled + q * d;
+    if (theta != 0.0f) {
+      for (int mm = threadIdx.x; mm < half; mm += blockDim.x) {
+        const double p = (double)(p0 + (long long)e * r);
+        const double inv_freq = pow((double)theta, -2.0 * mm / (double)d_r);
+        double sn, cs;
+        sincos(p * inv_freq, &sn, &cs);
+        const double x1 = row[d_n + mm], x2 = row[d_n + half + mm];
+        row[d_n + mm] = (float)(x1 * cs - x2 * sn);
+        row[d_n + half + mm] = (float)(x1 * sn + x2 * cs);
+      }
+    }
+  }
+  __syncthreads();
+  for (int q = 0; q < ne; ++q) {
+    const int e = e0 + q;
+    float* row = pooled + q * d;
+    for (int ch = threadIdx.x; ch < d; ch += blockDim.x) {
+      const uint32_t bits = f_to_bf16_bits(row[ch]);
+      c_out[((size_t)b * n_out + e) * d + ch] = (uint16_t)bits;
+      row[ch] = bf16_bits_to_f(bits);
+    }
+  }
+  if (W_IK == nullptr) return;
+  __syncthreads();
+  for (int j = threadIdx.x; j < d_I; j += blockDim.x) {
+    float acc[POOL_ENT];
+#pragma unroll
+    for (int q = 0; q < POOL_ENT; ++q) acc[q] = 0.0f;
+    for (int ch = 0; ch < d; ++ch) {
+      const float wv = bf16_bits_to_f(W_IK[(size_t)ch * d_I + j]);
+#pragma unroll
+      for (int q = 0; q < POOL_ENT; ++q) acc[q] = fmaf(pooled[q * d + ch], wv, acc[q]);
+    }
+    for (int q = 0; q < ne; ++q) kI_out[((size_t)b * n_out + e0 + q) * d_I + j] = (uint16_t)f_to_bf16_bits(acc[q]);
+  }
+}
+
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" csa_status csa_compress(const csa_compress_args* a, void* stream) {
+  CSA_REQUIRE(a != nullptr && a->struct_size == sizeof(csa_compress_args));
+  CSA_REQUIRE(a->B >= 0 && a->T >= 0 && a->d > 0 && a->ratio >= 1 && a->d_rope >= 0 && a->d_rope <= a->d);
+  CSA_REQUIRE(a->d_rope % 2 == 0 && a->d_index >= 0);
+  CSA_SUPPORTED(a->d % 8 == 0);
+  CSA_REQUIRE(a->C && a->Z && a->b_pos && a->c_out);
+  CSA_REQUIRE(a->W_IK == nullptr || (a->kI_out && a->d_index > 0));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (a->x) {
+    CSA_REQUIRE(a->W_kv && a->W_g && a->d_model > 0);
+    CSA_SUPPORTED(a->d % GBN == 0 && a->d_model % GBK == 0);
+    const long long M = (long long)a->B * a->T;
+    if (M > 0) {
+      static std::atomic<unsigned> attr_done{0};
+      set_smem_once((const void*)gemm_bf16_kernel, G_SMEM, attr_done);
+      dim3 grid(a->d / GBN, (unsigned)((M + GBM - 1) / GBM), 2);
+      gemm_bf16_kernel<<<grid, 256, G_SMEM, st>>>((const uint16_t*)a->x, (const uint16_t*)a->W_kv,
+                                                   (const uint16_t*)a->W_g, (uint16_t*)a->C, (uint16_t*)a->Z,
+                                                   (int)M, a->d, a->d_model);
+      csa_status s = launch_status();
+      if (s != CSA_OK) return s;
+    }
+  }
+  const int n_out = a->T / a->ratio;
+  if (a->B == 0 || n_out == 0) return CSA_OK;
+  const size_t smem = (size_t)POOL_ENT * a->d * sizeof(float);
+  CSA_SUPPORTED(smem <= 48 * 1024);
+  dim3 grid((n_out + POOL_ENT - 1) / POOL_ENT, a->B);
+  pool_kernel<<<grid, 256, smem, st>>>((const uint16_t*)a->C, (const uint16_t*)a->Z, a->b_pos, a->T, a->d,
+                                       a->d_rope, a->ratio, a->rope_theta, a->pos0, (const uint16_t*)a->W_IK,
+                                       a->d_index, (uint16_t*)a->c_out, (uint16_t*)a->kI_out);
+  return launch_status();
+}

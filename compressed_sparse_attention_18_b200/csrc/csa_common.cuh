@@ -1,0 +1,144 @@
+// Shared device helpers of the CSA kernels (sm_100a): bf16 / FP8 / FP4 conversions through the
+// hardware cvt instructions, warp reductions, launch-error plumbing.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "csa.h"
+
+namespace csa {
+
+// ----------------------------------------------------------------------------- host-side status
+
+void set_last_cuda_error(cudaError_t e);
+
+inline csa_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return CSA_ERR_CUDA;
+  }
+  return CSA_OK;
+}
+
+#define CSA_REQUIRE(cond) \
+  do {                    \
+    if (!(cond)) return CSA_ERR_INVALID; \
+  } while (0)
+
+#define CSA_SUPPORTED(cond) \
+  do {                      \
+    if (!(cond)) return CSA_ERR_UNSUPPORTED; \
+  } while (0)
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute is per device); later
+// calls, including those made while a stream is being captured into a CUDA graph, skip the runtime call.
+inline void set_smem_once(const void* func, int bytes, std::atomic<unsigned>& done) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const unsigned bit = 1u << (dev & 31);
+  if (done.load(std::memory_order_acquire) & bit) return;
+  cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  done.fetch_or(bit, std::memory_order_acq_rel);
+}
+
+// ----------------------------------------------------------------------------- number formats
+
+__device__ __forceinline__ float bf16_bits_to_f(uint32_t b) { return __uint_as_float(b << 16); }
+
+__device__ __forceinline__ uint32_t f_to_bf16_bits(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return (uint32_t)(*reinterpret_cast<uint16_t*>(&h));
+}
+
+// Two floats -> packed bf16x2 (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// fp32 -> E4M3 byte: round to nearest even, saturate to +-448, subnormals kept (PTX cvt ... satfinite).
+__device__ __forceinline__ uint32_t f32_to_e4m3(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return r & 0xFFu;
+}
+
+// E4M3 byte -> float (exact).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+  uint32_t h2;
+  uint16_t in = (uint16_t)(code & 0xFFu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// E4M3 byte -> f16x2 with the value in both halves (exact).
+__device__ __forceinline__ uint32_t e4m3_to_h2_splat(uint32_t code) {
+  uint32_t h2;
+  uint16_t in = (uint16_t)((code & 0xFFu) * 0x0101u);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return h2;
+}
+
+// fp32 -> E2M1 nibble: round to nearest even, saturate to +-6; -0 is returned as +0.
+__device__ __forceinline__ uint32_t f32_to_e2m1(float x) {
+  uint32_t r;
+  asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u32.u8 %0, t; }"
+      : "=r"(r) : "f"(0.0f), "f"(x));
+  r &= 0xFu;
+  return (r & 0x7u) ? r : 0u;
+}
+
+// One byte of two E2M1 codes -> f16x2 (low nibble -> low half), exact.
+__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
+  uint32_t h2;
+  asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h2) : "r"(byte & 0xFFu));
+  return h2;
+}
+
+__device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// E2M1 value of a code: bits s|e1 e0|m, exponent bias 1; e = 0 is the subnormal 0.5*m.
+__device__ __forceinline__ float e2m1_value(uint32_t code) {
+  const uint32_t e = (code >> 1) & 3u, m = code & 1u;
+  const float v = e ? ldexpf(1.0f + 0.5f * (float)m, (int)e - 1) : 0.5f * (float)m;
+  return (code & 8u) ? -v : v;
+}
+
+// ----------------------------------------------------------------------------- warp helpers
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Order-preserving map float -> uint32 (larger float -> larger key); -0 and +0 map to the same key.
+__device__ __forceinline__ uint32_t float_order_key(float f) {
+  f += 0.0f;  // -0 -> +0
+  uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float order_key_float(uint32_t k) {
+  uint32_t b = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  return __uint_as_float(b);
+}
+
+}  // namespace csa

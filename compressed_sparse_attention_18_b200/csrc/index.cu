@@ -1,0 +1,673 @@
+// Lightning indexer (FP4 multi-head ReLU dot product), per-query top-k, Reindex over a candidate list,
+// and the hierarchical candidate pool.
+// Sources: "DeepSeek-V4: エージェントが実際に使える100万トークンのコンテキスト", §ハイブリッド注意, Fig. 3 (an FP4
+// indexer with ReLU scores and several heads picks the top-k compressed blocks per query);
+// "DeepSeek-V4.1-Flash - Pushing the Limits of KV Cache Compression", CSA2 bullet + Fig. 4 (Reindex
+// re-scores the previous layer's keys with this layer's query) and the Hierarchical Sparse Indexer
+// bullet + Fig. 5 (blocks of positions ranked by their best score form a candidate pool).
+//
+// Score of key i for query (b, t):
+//   s = g_q g_k sum_h w_h max(0, sum_blk sq[h][blk] sk[i][blk] sum_{e in blk} q_e k_e)
+// Computed on the tensor pipe with mma.sync m16n8k16 (f16 in, fp32 accumulate): A = 16 keys, each
+// element the exact f16 product e2m1(k_e)*sk, B = the 8 indexer heads of one query, each element
+// e2m1(q_e)*sq.  The products are exact; the fp32 sums over the 128 elements are the kernel's only
+// rounding.  Each thread of a quad owns one 32-element scale block of its two key rows, so the key
+// side needs one 128-bit load per row and one scale byte.
+#include "csa_common.cuh"
+
+namespace csa {
+
+constexpr int IDX_HEADS = 8;           // MMA N: indexer heads, padded with zero heads
+constexpr int IDX_WARPS = 4;
+constexpr int IDX_TILES_PER_WARP = 8;  // 16-key tiles per warp per CTA
+constexpr int IDX_KEYS_PER_CTA = IDX_WARPS * IDX_TILES_PER_WARP * 16;
+constexpr int IDX_QT = 32;             // max queries per CTA (query fragments staged in shared memory)
+constexpr int TOPK_THREADS = 1024;
+constexpr int TOPK_CHUNK = 32768;      // max row length held in shared memory (implicit ids)
+constexpr int TOPK_CHUNK_IDS = 16384;  // max row length with explicit ids
+
+// ---------------------------------------------------------------------------- query quantisation
+// One warp per (query, head) row of q_I: FP4 pack rule (global scale g_q), then the f16 products
+// e2m1(q_e)*sq (exact in f16) written to the CTA's query tile; heads >= H_I are zero.
+// w' = w * g_q * g_k (the global scales factor out of the ReLU: both are positive).
+__device__ void quantize_query_tile(const uint16_t* __restrict__ qI, const float* __restrict__ w, int row0, int nq,
+                                    int H_I, int d_I, float g_q, float gg, __half* s_q, float* s_w) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const float six_g = 6.0f * g_q;
+  for (int rh = warp; rh < nq * IDX_HEADS; rh += nw) {
+    const int qq = rh / IDX_HEADS, h = rh % IDX_HEADS;
+    __half* dst = s_q + (size_t)rh * d_I;
+    if (h >= H_I) {
+      for (int e = lane; e < d_I; e += 32) dst[e] = __float2half(0.0f);
+      if (lane == 0) s_w[rh] = 0.0f;
+      continue;
+    }
+    const uint16_t* src = qI + ((size_t)(row0 + qq) * H_I + h) * d_I;
+    for (int blk = 0; blk < d_I / 32; ++blk) {
+      const float x = bf16_bits_to_f(src[blk * 32 + lane]);
+      const float amax = warp_max(fabsf(x));
+      const uint32_t s_code = f32_to_e4m3(__fdiv_rn(amax, six_g));
+      const float sv = e4m3_to_f32(s_code);
+      uint32_t code = 0;
+      if (sv != 0.0f) code = f32_to_e2m1(__fdiv_rn(x, __fmul_rn(sv, g_q)));
+      dst[blk * 32 + lane] = __float2half(e2m1_value(code) * sv);
+    }
+    if (lane == 0) s_w[rh] = w[(size_t)(row0 + qq) * H_I + h] * gg;
+  }
+}
+
+// ------------------------------------------------------------------------------------- scoring
+__device__ __forceinline__ void mma_f16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int DI>
+struct KeyRow {
+  // DI = 128: a thread holds one 32-element block (16 bytes); DI = 64: half a block (8 bytes).
+  static constexpr int BYTES = DI == 128 ? 16 : 8;
+  static constexpr int REGS = BYTES;  // one f16x2 per code byte
+  uint32_t w[BYTES / 4];
+};
+
+template <int DI>
+__device__ __forceinline__ void load_key(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                         int key, bool valid, int t, KeyRow<DI>& raw, uint32_t& sc) {
+  constexpr int S_PAD = ((DI / 32) + 3) & ~3;
+  if (!valid) {
+#pragma unroll
+    for (int i = 0; i < KeyRow<DI>::BYTES / 4; ++i) raw.w[i] = 0;
+    sc = 0;
+    return;
+  }
+  const uint8_t* p = codes + (size_t)key * (DI / 2) + t * KeyRow<DI>::BYTES;
+  if constexpr (DI == 128) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    raw.w[0] = v.x; raw.w[1] = v.y; raw.w[2] = v.z; raw.w[3] = v.w;
+    sc = __ldg(scales + (size_t)key * S_PAD + t);
+  } else {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    raw.w[0] = v.x; raw.w[1] = v.y;
+    sc = __ldg(scales + (size_t)key * S_PAD + (t >> 1));
+  }
+}
+
+template <int DI>
+__device__ __forceinline__ void convert_key(const KeyRow<DI>& raw, uint32_t sc, uint32_t* a) {
+  const uint32_t s2 = e4m3_to_h2_splat(sc);
+#pragma unroll
+  for (int i = 0; i < KeyRow<DI>::BYTES; ++i) a[i] = hmul2_bits(e2m1x2_to_h2(raw.w[i >> 2] >> ((i & 3) * 8)), s2);
+}
+
+// Grid: x = key chunk (IDX_KEYS_PER_CTA keys or candidates), y = query tile, z = sequence.
+// cand != nullptr: Reindex mode, one query per CTA, keys gathered by id.  Dynamic shared memory holds
+// the tile's query fragments [qt][IDX_HEADS][DI] f16.
+template <int DI>
+__global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
+    const uint16_t* __restrict__ q_I, const float* __restrict__ w, int H_I, float g_q, float gg, int Nq, int qt,
+    const uint8_t* __restrict__ k_codes, const uint8_t* __restrict__ k_scales, int n_max,
+    const int32_t* __restrict__ n_c, const int64_t* __restrict__ q_pos, int ratio,
+    const int32_t* __restrict__ cand, int n_cand, float* __restrict__ scores, long long ld) {
+  constexpr int STEPS = DI / 16;
+  constexpr int BREGS = DI / 8;           // f16x2 registers of one head slice per thread
+  constexpr int S_PAD = ((DI / 32) + 3) & ~3;
+  extern __shared__ __align__(16) uint8_t s_dyn[];
+  __half* s_q = reinterpret_cast<__half*>(s_dyn);          // [qt][IDX_HEADS][DI]
+  __shared__ float s_w[IDX_QT][IDX_HEADS];
+  __shared__ int s_nvis[IDX_QT];
+  __shared__ long long s_t[IDX_QT];
+
+  const int b = blockIdx.z;
+  const int q0 = cand ? blockIdx.y : blockIdx.y * qt;
+  const int nq = cand ? 1 : min(qt, Nq - q0);
+  const int ncb = min(n_c[b], n_max);   // entries beyond the cache capacity do not exist
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int chunk0 = blockIdx.x * IDX_KEYS_PER_CTA;
+  const int n_cols = cand ? n_cand : n_max;
+  if (chunk0 >= n_cols) return;
+
+  quantize_query_tile(q_I, w, b * Nq + q0, nq, H_I, DI, g_q, gg, s_q, &s_w[0][0]);
+  int max_vis = 0;
+  for (int qq = 0; qq < nq; ++qq) {
+    const long long tq = q_pos[(size_t)b * Nq + q0 + qq];
+    long long nv = (tq + 1) / ratio;
+    if (nv > ncb) nv = ncb;
+    if (nv < 0) nv = 0;
+    if (tid == 0) { s_nvis[qq] = (int)nv; s_t[qq] = tq; }
+    max_vis = max(max_vis, (int)nv);
+  }
+  __syncthreads();
+  if (!cand && chunk0 >= max_vis) return;
+
+  const int chunk_end = min(n_cols, chunk0 + IDX_KEYS_PER_CTA);
+  const int col_end = cand ? chunk_end : min(chunk_end, max_vis);
+  const uint8_t* codes_b = k_codes + (size_t)b * n_max * (DI / 2);
+  const uint8_t* scales_b = k_scales + (size_t)b * n_max * S_PAD;
+  const int32_t* cand_row = cand ? cand + ((size_t)b * Nq + q0) * n_cand : nullptr;
+  const long long t0 = s_t[0];
+
+  auto key_of = [&](int col, int& key, bool& ok) {
+    if (cand_row) {
+      const int id = col < col_end ? cand_row[col] : -1;
+      key = id;
+      ok = id >= 0 && id < ncb && (long long)ratio * id + ratio - 1 <= t0;
+    } else {
+      key = col;
+      ok = col < col_end && col < ncb;
+    }
+  };
+
+  const int first_col = chunk0 + warp * IDX_TILES_PER_WARP * 16;
+  int key[2][2];
+  bool kval[2][2];
+  KeyRow<DI> raw[2][2];
+  uint32_t sc[2][2];
+  // software pipeline: raw[cur] holds the tile being converted, raw[cur ^ 1] the next tile in flight
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    key_of(first_col + g + 8 * h, key[0][h], kval[0][h]);
+    load_key<DI>(codes_b, scales_b, key[0][h], kval[0][h], t, raw[0][h], sc[0][h]);
+  }
+#pragma unroll 2
+  for (int tile = 0; tile < IDX_TILES_PER_WARP; ++tile) {
+    const int cur = tile & 1;
+    const int col0 = first_col + tile * 16;
+    if (col0 >= col_end) break;
+    if (tile + 1 < IDX_TILES_PER_WARP) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        key_of(col0 + 16 + g + 8 * h, key[cur ^ 1][h], kval[cur ^ 1][h]);
+        load_key<DI>(codes_b, scales_b, key[cur ^ 1][h], kval[cur ^ 1][h], t, raw[cur ^ 1][h], sc[cur ^ 1][h]);
+      }
+    }
+    uint32_t a[2][KeyRow<DI>::REGS];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) convert_key<DI>(raw[cur][h], sc[cur][h], a[h]);
+
+    for (int qq = 0; qq < nq; ++qq) {
+      // B fragment: head g, elements [t*DI/4 + 4s, +4) for k16 step s -> one contiguous slice
+      const uint4* bq = reinterpret_cast<const uint4*>(s_q + ((size_t)qq * IDX_HEADS + g) * DI + t * (DI / 4));
+      uint32_t bfr[BREGS];
+#pragma unroll
+      for (int i = 0; i < BREGS / 4; ++i) {
+        const uint4 v = bq[i];
+        bfr[4 * i] = v.x; bfr[4 * i + 1] = v.y; bfr[4 * i + 2] = v.z; bfr[4 * i + 3] = v.w;
+      }
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < STEPS; ++s) {
+        const uint32_t af[4] = {a[0][2 * s], a[1][2 * s], a[0][2 * s + 1], a[1][2 * s + 1]};
+        mma_f16(acc, af, bfr[2 * s], bfr[2 * s + 1]);
+      }
+      const float w0 = s_w[qq][2 * t], w1 = s_w[qq][2 * t + 1];
+      float r0 = w0 * fmaxf(acc[0], 0.f) + w1 * fmaxf(acc[1], 0.f);
+      float r1 = w0 * fmaxf(acc[2], 0.f) + w1 * fmaxf(acc[3], 0.f);
+      r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
+      r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
+      r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+      r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
+      if (t < 2) {
+        const int col = col0 + g + 8 * t;
+        const float v = (t ? r1 : r0) + 0.0f;
+        float* row = scores + (size_t)(b * Nq + q0 + qq) * ld;
+        if (cand_row) {
+          if (col < col_end) row[col] = (t ? kval[cur][1] : kval[cur][0]) ? v : -INFINITY;
+        } else if (col < s_nvis[qq]) {
+          row[col] = v;
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------- top-k
+// Block-wide selection over one row held in shared memory as order-preserving 32-bit keys.
+// Total order: score desc, then key id asc, then position asc (ids repeat only in malformed
+// candidate lists).  MSB-first radix passes with 8-bit digits find the threshold, then every element
+// above it is emitted and the ties are taken in (id, position) order.
+
+struct TopkSmem {
+  uint32_t hist[256];
+  uint32_t scan[TOPK_THREADS / 32];
+  uint32_t bcast[4];
+  uint32_t counter;
+};
+
+// Find the R-th largest value of key(j) over positions j < n with filt(j).  Returns the threshold
+// key; *n_above = number of filtered elements with key > threshold.
+template <class KeyF, class FiltF>
+__device__ uint32_t radix_threshold(TopkSmem& sm, int n, uint32_t R, KeyF key, FiltF filt, uint32_t* n_above) {
+  uint32_t prefix = 0, mask = 0, rem = R;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) sm.hist[i] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+      if (!filt(j)) continue;
+      const uint32_t k = key(j);
+      if ((k & mask) == prefix) atomicAdd(&sm.hist[(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // suffix sums over 256 bins: lane l owns bins [8l, 8l+8)
+      const int l = threadIdx.x;
+      uint32_t loc[8], tot = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { loc[i] = sm.hist[8 * l + i]; tot += loc[i]; }
+      // exclusive suffix over lanes: sum of totals of lanes > l
+      uint32_t suf = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
+        if (l + o < 32) suf += v;
+      }
+      uint32_t above = suf - tot;  // elements in bins of higher lanes
+      int found = -1;
+      uint32_t found_above = 0;
+      for (int i = 7; i >= 0; --i) {
+        if (found < 0 && above + loc[i] >= rem && above < rem) { found = 8 * l + i; found_above = above; }
+        above += loc[i];
+      }
+      if (found >= 0) { sm.bcast[0] = (uint32_t)found; sm.bcast[1] = found_above; }
+    }
+    __syncthreads();
+    const uint32_t digit = sm.bcast[0];
+    rem -= sm.bcast[1];
+    prefix |= digit << shift;
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+  *n_above = R - rem;
+  return prefix;
+}
+
+// Exclusive block scan of one value per thread; returns the prefix, *total = sum.
+__device__ uint32_t block_exclusive_scan(TopkSmem& sm, uint32_t v, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sm.scan[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    uint32_t s = lane < nw ? sm.scan[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < nw) sm.scan[lane] = s;
+  }
+  __syncthreads();
+  const uint32_t base = warp ? sm.scan[warp - 1] : 0;
+  *total = sm.scan[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return base + x - v;
+}
+
+// One CTA per row.  Row r: scores at in_scores + r*in_ld, length len (from lens[r] or the visibility
+// rule), ids from in_ids (explicit) or id = id_base + position.  Writes k slots of out_idx /
+// out_scores at row r (stride k_out).
+struct TopkRowArgs {
+  const float* in_scores;
+  const int32_t* in_ids;
+  long long in_ld;
+  int n_cols;              // columns available in this call's rows
+  int col_base;            // first column of the row segment (tournament chunks)
+  const int64_t* q_pos;    // when lens come from visibility (may be null)
+  const int32_t* n_c;
+  int ratio, Nq, rows_per_seg;
+  int k;
+  int32_t* out_idx;
+  float* out_scores;
+  long long out_ld;
+};
+
+__global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(TopkRowArgs A) {
+  extern __shared__ __align__(16) uint32_t s_keys[];
+  __shared__ TopkSmem sm;
+  const int seg = blockIdx.x;                  // segment (chunk) of the row
+  const int row = blockIdx.y;
+  const int col0 = A.col_base + seg * A.rows_per_seg;
+  int len = min(A.rows_per_seg, A.n_cols - col0);
+  if (A.q_pos) {
+    const int b = row / A.Nq;
+    long long nv = (A.q_pos[row] + 1) / A.ratio;
+    if (nv > A.n_c[b]) nv = A.n_c[b];
+    len = (int)max(0LL, min((long long)len, nv - col0));
+  }
+  if (len < 0) len = 0;
+  uint32_t* keys = s_keys;
+  int32_t* ids = reinterpret_cast<int32_t*>(s_keys + (A.in_ids ? TOPK_CHUNK_IDS : 0));
+  const float* src = A.in_scores + row * A.in_ld + col0;
+  const int32_t* isrc = A.in_ids ? A.in_ids + row * A.in_ld + col0 : nullptr;
+  uint32_t nvalid_loc = 0;
+  for (int j = threadIdx.x; j < len; j += blockDim.x) {
+    const float s = src[j];
+    const bool ok = s > -INFINITY && (!isrc || isrc[j] >= 0);
+    keys[j] = ok ? float_order_key(s) : 0u;   // 0 marks "not a candidate"
+    if (isrc) ids[j] = isrc[j];
+    nvalid_loc += ok;
+  }
+  uint32_t nvalid;
+  block_exclusive_scan(sm, nvalid_loc, &nvalid);
+  const int out_seg = blockIdx.x;
+  int32_t* oi = A.out_idx + row * A.out_ld + (long long)out_seg * A.k;
+  float* os = A.out_scores ? A.out_scores + row * A.out_ld + (long long)out_seg * A.k : nullptr;
+  const uint32_t K = min((uint32_t)A.k, nvalid);
+  auto idof = [&](int j) -> uint32_t { return isrc ? (uint32_t)ids[j] : (uint32_t)(A.col_base + seg * A.rows_per_seg + j); };
+  auto valid = [&](int j) { return keys[j] != 0u; };
+
+  uint32_t T1 = 0, above1 = 0, T2 = 0xFFFFFFFFu, need_pos = 0;
+  bool all_ties = true;
+  if (K > 0 && K < nvalid) {
+    T1 = radix_threshold(sm, len, K, [&](int j) { return keys[j]; }, valid, &above1);
+    const uint32_t need = K - above1;
+    // count ties
+    uint32_t tl = 0;
+    for (int j = threadIdx.x; j < len; j += blockDim.x) tl += (keys[j] == T1);
+    uint32_t nties;
+    block_exclusive_scan(sm, tl, &nties);
+    if (nties > need) {
+      all_ties = false;
+      uint32_t above2;
+      T2 = radix_threshold(sm, len, need, [&](int j) { return ~idof(j); },
+                           [&](int j) { return keys[j] == T1; }, &above2);
+      need_pos = need - above2;  // ties on (score, id) taken in position order
+    }
+  }
+  if (threadIdx.x == 0) sm.counter = 0;
+  __syncthreads();
+  // emission; contiguous ranges per thread so that position-order ties are deterministic
+  const int per = (len + blockDim.x - 1) / blockDim.x;
+  const int j0 = threadIdx.x * per, j1 = min(len, j0 + per);
+  uint32_t mine = 0;
+  if (!all_ties)
+    for (int j = j0; j < j1; ++j) mine += (keys[j] == T1 && ~idof(j) == T2);
+  uint32_t total3;
+  uint32_t rank = block_exclusive_scan(sm, mine, &total3);
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t kj = keys[j];
+    if (kj == 0u) continue;
+    bool take;
+    if (K >= nvalid) take = true;
+    else if (kj > T1) take = true;
+    else if (kj < T1) take = false;
+    else if (all_ties) take = true;
+    else {
+      const uint32_t k2 = ~idof(j);
+      if (k2 > T2) take = true;
+      else if (k2 < T2) take = false;
+      else take = (rank++ < need_pos);
+    }
+    if (take) {
+      const uint32_t slot = atomicAdd(&sm.counter, 1u);
+      oi[slot] = (int32_t)idof(j);
+      if (os) os[slot] = order_key_float(kj);
+    }
+  }
+  __syncthreads();
+  for (int s = (int)K + threadIdx.x; s < A.k; s += blockDim.x) {
+    oi[s] = -1;
+    if (os) os[s] = -INFINITY;
+  }
+}
+
+// ------------------------------------------------------------------------- hierarchical pool
+__global__ void block_max_kernel(const float* __restrict__ scores, long long ld, int n_cols,
+                                 const int64_t* __restrict__ q_pos, const int32_t* __restrict__ n_c, int ratio,
+                                 int Nq, int G, int nblk, float* __restrict__ bs) {
+  const int row = blockIdx.y;
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= nblk) return;
+  long long nv = (q_pos[row] + 1) / ratio;
+  if (nv > n_c[row / Nq]) nv = n_c[row / Nq];
+  if (nv > n_cols) nv = n_cols;
+  float m = -INFINITY;
+  for (int e = 0; e < G; ++e) {
+    const long long i = (long long)j * G + e;
+    if (i < nv) m = fmaxf(m, scores[row * ld + i]);
+  }
+  bs[(long long)row * nblk + j] = m;
+}
+
+__global__ void pool_expand_kernel(const int32_t* __restrict__ blk, int P, int G, const float* __restrict__ scores,
+                                   long long ld, int n_cols, const int64_t* __restrict__ q_pos,
+                                   const int32_t* __restrict__ n_c, int ratio, int Nq, int32_t* __restrict__ pool) {
+  const int row = blockIdx.y;
+  const int s = blockIdx.x * blockDim.x + threadIdx.x;
+  if (s >= P * G) return;
+  long long nv = (q_pos[row] + 1) / ratio;
+  if (nv > n_c[row / Nq]) nv = n_c[row / Nq];
+  if (nv > n_cols) nv = n_cols;
+  const int b = blk[(long long)row * P + s / G];
+  int out = -1;
+  if (b >= 0) {
+    const long long i = (long long)b * G + s % G;
+    if (i < nv && scores[row * ld + i] > -INFINITY) out = (int)i;
+  }
+  pool[(long long)row * P * G + s] = out;
+}
+
+// ------------------------------------------------------------------------------ orchestration
+struct IndexPlan {
+  int rows, n_cols, segs, seg_len;
+  size_t off_scores, off_tidx, off_tsc, off_bs, off_bidx, sel_total, total;
+};
+
+// Workspace of the selection step (tournament buffers, pool block scores); the fused entry point
+// places the score matrix in front of it.
+static IndexPlan plan_index(const csa_index_args* a) {
+  IndexPlan p{};
+  p.rows = a->B * a->Nq;
+  p.n_cols = a->cand ? a->n_cand : a->n_max;
+  const int cap = TOPK_CHUNK;
+  p.segs = (p.n_cols + cap - 1) / cap;
+  if (p.segs < 1) p.segs = 1;
+  p.seg_len = p.segs == 1 ? p.n_cols : cap;
+  size_t o = 0;
+  if (p.segs > 1) {
+    p.off_tidx = o; o = align_up(o + (size_t)p.rows * p.segs * a->k * 4, 256);
+    p.off_tsc = o;  o = align_up(o + (size_t)p.rows * p.segs * a->k * 4, 256);
+  }
+  if (a->pool_blocks > 0) {
+    const int G = a->pool_block_size;
+    const int nblk = (p.n_cols + G - 1) / G;
+    p.off_bs = o;   o = align_up(o + (size_t)p.rows * nblk * 4, 256);
+    p.off_bidx = o; o = align_up(o + (size_t)p.rows * a->pool_blocks * 4, 256);
+  }
+  p.sel_total = o;
+  p.off_scores = o;
+  p.total = align_up(o + (size_t)p.rows * p.n_cols * 4, 256);
+  return p;
+}
+
+static csa_status validate_index(const csa_index_args* a, bool need_select) {
+  CSA_REQUIRE(a != nullptr && a->struct_size == sizeof(csa_index_args));
+  CSA_REQUIRE(a->B >= 0 && a->Nq >= 0 && a->H_I >= 1 && a->ratio >= 1 && a->k >= 1 && a->n_max >= 0);
+  CSA_SUPPORTED(a->d_I == 64 || a->d_I == 128);
+  CSA_SUPPORTED(a->H_I <= IDX_HEADS && a->k <= 4096);
+  CSA_REQUIRE(a->g_q > 0.0f && a->g_k > 0.0f);
+  if (a->cand) {
+    CSA_REQUIRE(a->n_cand >= 1);
+    CSA_SUPPORTED(a->n_cand <= TOPK_CHUNK_IDS && a->pool_blocks == 0);
+  }
+  {
+    const int n_cols = a->cand ? a->n_cand : a->n_max;
+    const int segs = (n_cols + TOPK_CHUNK - 1) / TOPK_CHUNK;
+    if (segs > 1) CSA_SUPPORTED((long long)segs * a->k <= TOPK_CHUNK_IDS);
+  }
+  if (a->pool_blocks > 0) {
+    CSA_REQUIRE(a->pool_block_size >= 1 && a->pool_out != nullptr);
+    const int nblk = (a->n_max + a->pool_block_size - 1) / a->pool_block_size;
+    CSA_SUPPORTED(nblk <= TOPK_CHUNK && a->pool_blocks <= 4096);
+  }
+  if ((long long)a->B * a->Nq == 0) return CSA_OK;
+  CSA_REQUIRE(a->n_c && a->q_pos);
+  if (need_select) CSA_REQUIRE(a->idx_out != nullptr);
+  else CSA_REQUIRE(a->q_I && a->w && a->k_codes && a->k_scales);
+  return CSA_OK;
+}
+
+static csa_status run_scores(const csa_index_args* a, float* scores, long long ld, cudaStream_t st) {
+  const int n_cols = a->cand ? a->n_cand : a->n_max;
+  const int qt = a->cand ? 1 : (a->Nq < IDX_QT ? a->Nq : IDX_QT);
+  dim3 grid((n_cols + IDX_KEYS_PER_CTA - 1) / IDX_KEYS_PER_CTA, a->cand ? a->Nq : (a->Nq + qt - 1) / qt, a->B);
+  if (grid.x == 0) return CSA_OK;
+  const int smem = qt * IDX_HEADS * a->d_I * 2;
+  const float gg = a->g_q * a->g_k;
+  static std::atomic<unsigned> attr128{0}, attr64{0};
+  if (a->d_I == 128) {
+    set_smem_once((const void*)index_score_kernel<128>, IDX_QT * IDX_HEADS * 128 * 2, attr128);
+    index_score_kernel<128><<<grid, IDX_WARPS * 32, smem, st>>>(
+        (const uint16_t*)a->q_I, a->w, a->H_I, a->g_q, gg, a->Nq, qt, a->k_codes, a->k_scales, a->n_max, a->n_c,
+        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld);
+  } else {
+    set_smem_once((const void*)index_score_kernel<64>, IDX_QT * IDX_HEADS * 64 * 2, attr64);
+    index_score_kernel<64><<<grid, IDX_WARPS * 32, smem, st>>>(
+        (const uint16_t*)a->q_I, a->w, a->H_I, a->g_q, gg, a->Nq, qt, a->k_codes, a->k_scales, a->n_max, a->n_c,
+        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld);
+  }
+  return launch_status();
+}
+
+static csa_status launch_topk(TopkRowArgs ta, int rows, int segs, bool ids, cudaStream_t st) {
+  static_assert(TOPK_CHUNK_IDS * 8 == TOPK_CHUNK * 4, "one shared-memory size for both row kinds");
+  const size_t smem = (size_t)TOPK_CHUNK * 4;
+  static std::atomic<unsigned> attr_done{0};
+  set_smem_once((const void*)topk_kernel, (int)smem, attr_done);
+  dim3 grid(segs, rows);
+  topk_kernel<<<grid, TOPK_THREADS, smem, st>>>(ta);
+  return launch_status();
+}
+
+static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const float* scores, long long ld,
+                             uint8_t* w8, cudaStream_t st) {
+  TopkRowArgs ta{};
+  ta.in_scores = scores;
+  ta.in_ids = a->cand;
+  ta.in_ld = ld;
+  ta.n_cols = p.n_cols;
+  ta.col_base = 0;
+  ta.q_pos = a->cand ? nullptr : a->q_pos;
+  ta.n_c = a->n_c;
+  ta.ratio = a->ratio;
+  ta.Nq = a->Nq;
+  ta.rows_per_seg = p.seg_len;
+  ta.k = a->k;
+  if (a->cand) CSA_SUPPORTED(ld == a->n_cand);   // explicit ids are read with the score row stride
+  if (p.segs == 1) {
+    ta.out_idx = a->idx_out;
+    ta.out_scores = a->scores_out;
+    ta.out_ld = a->k;
+    csa_status s = launch_topk(ta, p.rows, 1, a->cand != nullptr, st);
+    if (s != CSA_OK) return s;
+  } else {
+    int32_t* tidx = (int32_t*)(w8 + p.off_tidx);
+    float* tsc = (float*)(w8 + p.off_tsc);
+    ta.out_idx = tidx;
+    ta.out_scores = tsc;
+    ta.out_ld = (long long)p.segs * a->k;
+    csa_status s = launch_topk(ta, p.rows, p.segs, false, st);
+    if (s != CSA_OK) return s;
+    TopkRowArgs tb{};
+    tb.in_scores = tsc;
+    tb.in_ids = tidx;
+    tb.in_ld = (long long)p.segs * a->k;
+    tb.n_cols = p.segs * a->k;
+    tb.rows_per_seg = p.segs * a->k;
+    tb.k = a->k;
+    tb.out_idx = a->idx_out;
+    tb.out_scores = a->scores_out;
+    tb.out_ld = a->k;
+    CSA_SUPPORTED(tb.n_cols <= TOPK_CHUNK_IDS);
+    s = launch_topk(tb, p.rows, 1, true, st);
+    if (s != CSA_OK) return s;
+  }
+  if (a->pool_blocks > 0) {
+    const int G = a->pool_block_size;
+    const int nblk = (p.n_cols + G - 1) / G;
+    float* bs = (float*)(w8 + p.off_bs);
+    int32_t* bidx = (int32_t*)(w8 + p.off_bidx);
+    block_max_kernel<<<dim3((nblk + 255) / 256, p.rows), 256, 0, st>>>(scores, ld, p.n_cols, a->q_pos, a->n_c,
+                                                                        a->ratio, a->Nq, G, nblk, bs);
+    csa_status s = launch_status();
+    if (s != CSA_OK) return s;
+    TopkRowArgs tc{};
+    tc.in_scores = bs;
+    tc.in_ld = nblk;
+    tc.n_cols = nblk;
+    tc.rows_per_seg = nblk;
+    tc.k = a->pool_blocks;
+    tc.out_idx = bidx;
+    tc.out_ld = a->pool_blocks;
+    s = launch_topk(tc, p.rows, 1, false, st);
+    if (s != CSA_OK) return s;
+    const int PG = a->pool_blocks * G;
+    pool_expand_kernel<<<dim3((PG + 255) / 256, p.rows), 256, 0, st>>>(bidx, a->pool_blocks, G, scores, ld,
+                                                                        p.n_cols, a->q_pos, a->n_c, a->ratio, a->Nq,
+                                                                        a->pool_out);
+    s = launch_status();
+    if (s != CSA_OK) return s;
+  }
+  return CSA_OK;
+}
+
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" csa_status csa_index_scores(const csa_index_args* a, float* scores, int64_t ld, void* stream) {
+  csa_status v = validate_index(a, false);
+  if (v != CSA_OK) return v;
+  if ((long long)a->B * a->Nq == 0) return CSA_OK;
+  const int n_cols = a->cand ? a->n_cand : a->n_max;
+  CSA_REQUIRE(scores != nullptr && ld >= n_cols);
+  return run_scores(a, scores, ld, (cudaStream_t)stream);
+}
+
+extern "C" size_t csa_topk_workspace_size(const csa_index_args* a) {
+  if (validate_index(a, true) != CSA_OK) return 0;
+  return plan_index(a).sel_total;
+}
+
+extern "C" csa_status csa_topk(const csa_index_args* a, const float* scores, int64_t ld, void* ws, size_t ws_bytes,
+                               void* stream) {
+  csa_status v = validate_index(a, true);
+  if (v != CSA_OK) return v;
+  const IndexPlan p = plan_index(a);
+  if (p.rows == 0) return CSA_OK;
+  CSA_REQUIRE(scores != nullptr && ld >= p.n_cols);
+  if (ws_bytes < p.sel_total) return CSA_ERR_WORKSPACE;
+  CSA_REQUIRE(ws != nullptr || p.sel_total == 0);
+  return run_select(a, p, scores, ld, (uint8_t*)ws, (cudaStream_t)stream);
+}
+
+extern "C" size_t csa_index_topk_workspace_size(const csa_index_args* a) {
+  if (validate_index(a, true) != CSA_OK || validate_index(a, false) != CSA_OK) return 0;
+  return plan_index(a).total;
+}
+
+extern "C" csa_status csa_index_topk(const csa_index_args* a, void* ws, size_t ws_bytes, void* stream) {
+  csa_status v = validate_index(a, true);
+  if (v != CSA_OK) return v;
+  v = validate_index(a, false);
+  if (v != CSA_OK) return v;
+  const IndexPlan p = plan_index(a);
+  if (p.rows == 0) return CSA_OK;
+  CSA_REQUIRE(ws != nullptr);
+  if (ws_bytes < p.total) return CSA_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  uint8_t* w8 = (uint8_t*)ws;
+  float* scores = (float*)(w8 + p.off_scores);
+  csa_status s = run_scores(a, scores, p.n_cols, st);
+  if (s != CSA_OK) return s;
+  return run_select(a, p, scores, p.n_cols, w8, st);
+}

@@ -1,0 +1,215 @@
+/*
+ * csa.h — C ABI of the B200 (sm_100a) Compressed Sparse Attention layer over an FP4 KV cache.
+ *
+ * The layer (sources, by page title):
+ *   [V4 blog]    "DeepSeek-V4: エージェントが実際に使える100万トークンのコンテキスト", §ハイブリッド注意：CSAとHCA,
+ *                Fig. 3 (CSA: 4x softmax-gated compressor, FP4 ReLU "lightning" indexer, top-k, sliding window),
+ *                Fig. 4 (HCA: 128x compressor, dense attention), storage paragraph (BF16 RoPE dims, FP4 indexer).
+ *   [V4.1 notes] "DeepSeek-V4.1-Flash - Pushing the Limits of KV Cache Compression", §提案手法/アーキテクチャ:
+ *                CED bullet eq.(1) (C, Z projections), CSA2 bullet + Fig. 4 (Full / Reindex / Reuse),
+ *                Hierarchical Sparse Indexer bullet + Fig. 5, FP4 主 KV キャッシュ bullet.
+ *
+ * Conventions for every entry point:
+ *   - Every pointer is caller-owned DEVICE memory (unless stated otherwise); the library allocates
+ *     nothing.  Scratch comes from a caller workspace whose size the matching *_workspace_size() call
+ *     returns for the same arguments (0 means none is needed; ws may then be NULL).
+ *   - bf16 = IEEE bfloat16 stored as uint16; tensors are dense row-major with the shapes given.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy default
+ *     stream).  Argument errors are detected on the host before any launch and returned as
+ *     CSA_ERR_INVALID / CSA_ERR_UNSUPPORTED / CSA_ERR_WORKSPACE; nothing is launched then.
+ *     A launch failure returns CSA_ERR_CUDA.  No exception crosses the ABI; no global mutable state.
+ *   - Arguments are passed as structs whose first field `struct_size` must equal sizeof(struct).
+ *   - FP4 formats (E2M1 codes, one E4M3 scale per 32 elements, per-tensor fp32 global scale g):
+ *       codes[n][d_n/2] u8 (element 2j in the low nibble of byte j), scales[n][S_pad] u8
+ *       (S = d_n/32, S_pad = round_up(S, 4), pad bytes 0), rope[n][d_r] bf16.
+ *       Dequantised element = e2m1(code) * e4m3(scale) * g.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum csa_status {
+  CSA_OK = 0,
+  CSA_ERR_INVALID = 1,      /* a NULL pointer, a bad size or a struct_size mismatch                    */
+  CSA_ERR_UNSUPPORTED = 2,  /* a valid shape this build has no kernel for (e.g. d_I not 64/128)         */
+  CSA_ERR_WORKSPACE = 3,    /* ws_bytes smaller than *_workspace_size() for the same arguments          */
+  CSA_ERR_CUDA = 4,         /* a kernel launch or CUDA runtime call failed (see csa_last_cuda_error)   */
+  CSA_ERR_DEVICE = 5        /* reserved: device-side check failed                                       */
+} csa_status;
+
+/* Human-readable name of a status code (static string). */
+const char* csa_status_string(int status);
+/* Library version as 10000*major + 100*minor + patch. */
+int csa_version(void);
+/* The cudaError_t of the last CSA_ERR_CUDA returned on the calling host thread (0 if none). */
+int csa_last_cuda_error(void);
+
+/* ------------------------------------------------------------------------------------------------
+ * csa_compress — the compressor ([V4 blog] Fig. 3 / Fig. 4; [V4.1 notes] eq.(1) and CSA2 bullet).
+ *
+ * Projection mode (x != NULL): C = bf16(x·W_kv), Z = bf16(x·W_g) are computed (tensor cores, fp32
+ * accumulate) and written to the caller's C and Z buffers (C also serves as the token's window KV).
+ * Pooling mode (x == NULL): C and Z are read.  Then, for every sequence b and entry i < T/ratio:
+ *   c[b][i][ch] = sum_j softmax_j(Z[b][r i + j][ch] + b_pos[j][ch]) * C[b][r i + j][ch]
+ * (one gate per channel, non-overlapping groups), RoPE on the last d_rope channels at position
+ * pos0[b] + r i (half-split pairs, angle p * theta^(-2m/d_rope); rope_theta == 0 disables it),
+ * rounded to bf16 into c_out; then k_I = bf16(c · W_IK) into kI_out when W_IK != NULL.
+ * Trailing T % ratio tokens are ignored (the caller keeps them pending).
+ * Shapes: x[B][T][d_model], W_kv/W_g[d_model][d], C/Z[B][T][d], b_pos[ratio][d] fp32,
+ *         W_IK[d][d_index], c_out[B][T/ratio][d], kI_out[B][T/ratio][d_index], pos0[B] int64 (NULL = 0).
+ * Limits: d % 8 == 0, d_rope even and <= d, ratio >= 1; projection mode needs d % 128 == 0 and
+ *         d_model % 32 == 0 (else CSA_ERR_UNSUPPORTED).  No workspace.
+ * ------------------------------------------------------------------------------------------------ */
+typedef struct csa_compress_args {
+  uint32_t struct_size;
+  int32_t B, T, d_model, d, d_rope, d_index, ratio;
+  float rope_theta;
+  const int64_t* pos0;
+  const void* x;
+  const void* W_kv;
+  const void* W_g;
+  void* C;
+  void* Z;
+  const float* b_pos;
+  const void* W_IK;
+  void* c_out;
+  void* kI_out;
+} csa_compress_args;
+
+csa_status csa_compress(const csa_compress_args* args, void* stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * csa_pack_fp4 — FP4 pack of compressed entries into a cache ([V4.1 notes] FP4 主 KV キャッシュ bullet;
+ * [V4 blog] storage paragraph: the RoPE slice stays BF16).
+ *
+ * For rows src[b][j] (j < n), written to cache row row0[b] + j of sequence b:
+ *   per 32-block of the first d - d_rope channels: s = E4M3_rne_satfinite(fp32(amax / fp32(6 g)));
+ *   s == 0 zeroes the block; else code_e = E2M1_rne_satfinite(fp32(x_e / fp32(s g))), -0 -> +0;
+ *   the last d_rope channels are copied to rope.
+ * Shapes: src[B][n][d] bf16; codes[B][n_max][(d-d_rope)/2]; scales[B][n_max][S_pad];
+ *         rope[B][n_max][d_rope] bf16 (may be NULL iff d_rope == 0); row0[B] int32 (NULL = 0).
+ * Limits: (d - d_rope) % 32 == 0, d_rope % 8 == 0, row0[b] + n <= n_max (not checked on the device:
+ *         the caller owns the cache bookkeeping).  No workspace.
+ * ------------------------------------------------------------------------------------------------ */
+typedef struct csa_pack_args {
+  uint32_t struct_size;
+  int32_t B, n, d, d_rope, n_max;
+  float global_scale;
+  const void* src;
+  const int32_t* row0;
+  uint8_t* codes;
+  uint8_t* scales;
+  void* rope;
+} csa_pack_args;
+
+csa_status csa_pack_fp4(const csa_pack_args* args, void* stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * csa_index_topk — lightning indexer scores + per-query top-k ([V4 blog] §ハイブリッド注意, Fig. 3;
+ * Reindex mode and the hierarchical candidate pool: [V4.1 notes] CSA2 bullet Fig. 4, Fig. 5).
+ *
+ * q_I is quantised with the FP4 pack rule (global scale g_q).  For query (b, q) at t = q_pos[b][q]
+ * and a visible key i (i < n_c[b], ratio*i + ratio - 1 <= t):
+ *   s = g_q g_k sum_h w[b][q][h] * max(0, sum_blk sq[h][blk] sk[i][blk] P[h][i][blk]),
+ *   P = E2M1 block dot product.  -0 is taken as +0.
+ * Candidates: all visible keys (cand == NULL; Full mode) or cand[b][q][0..n_cand) (Reindex mode;
+ * -1 entries and invisible ids are dropped).  Selected: the k_eff = min(k, #candidates) keys by
+ * (score desc, key id asc), written to idx_out[b][q][0..k) in unspecified order, remaining slots -1;
+ * scores_out (optional) gets the matching scores (-inf in padded slots).
+ * Hierarchical pool (pool_blocks > 0, cand == NULL only): block score = max over the visible keys
+ * of [G j, G j + G) (G = pool_block_size); the top pool_blocks blocks by (block score desc, block id
+ * asc) are written to pool_out[b][q][0 .. pool_blocks*G) as G consecutive key ids per block (block
+ * order unspecified; -1 for invisible keys and missing blocks).
+ * Shapes: q_I[B][Nq][H_I][d_I] bf16, w[B][Nq][H_I] fp32, k_codes[B][n_max][d_I/2],
+ *         k_scales[B][n_max][S_pad(d_I/32)], n_c[B] int32, q_pos[B][Nq] int64.
+ * Limits: d_I in {64, 128}; H_I <= 8; 1 <= k <= 4096; with cand: n_cand <= 16384.
+ * Workspace: csa_index_topk_workspace_size().
+ * ------------------------------------------------------------------------------------------------ */
+typedef struct csa_index_args {
+  uint32_t struct_size;
+  int32_t B, Nq, H_I, d_I, ratio, k, n_max;
+  float g_q, g_k;
+  const void* q_I;
+  const float* w;
+  const uint8_t* k_codes;
+  const uint8_t* k_scales;
+  const int32_t* n_c;
+  const int64_t* q_pos;
+  const int32_t* cand;
+  int32_t n_cand;
+  int32_t pool_blocks;
+  int32_t pool_block_size;
+  int32_t* pool_out;
+  int32_t* idx_out;
+  float* scores_out;
+} csa_index_args;
+
+size_t csa_index_topk_workspace_size(const csa_index_args* args);
+csa_status csa_index_topk(const csa_index_args* args, void* ws, size_t ws_bytes, void* stream);
+
+/* csa_index_scores — the scoring half of csa_index_topk on its own ([V4 blog] §ハイブリッド注意: the
+ * lightning indexer).  Writes scores[(b*Nq + q)*ld + j] fp32 for j < n_vis(t) = min(n_c[b],
+ * floor((t+1)/ratio)) in Full mode, or for every j < n_cand in Reindex mode (-inf for dropped
+ * candidates); other columns are left untouched.  ld >= n_max (Full) or >= n_cand (Reindex).
+ * idx_out / scores_out / pool_out are ignored.  No workspace. */
+csa_status csa_index_scores(const csa_index_args* args, float* scores, int64_t ld, void* stream);
+
+/* csa_topk — the selection half of csa_index_topk ([V4 blog] Fig. 3: top-k per query; [V4.1 notes]
+ * Fig. 5: hierarchical pool) over a score matrix laid out as csa_index_scores writes it, with the
+ * same args (q_I, w, k_codes, k_scales may be NULL).  In Reindex mode ld must equal n_cand.
+ * Workspace: csa_topk_workspace_size() (tournament buffers for rows longer than 32768, pool scores). */
+size_t csa_topk_workspace_size(const csa_index_args* args);
+csa_status csa_topk(const csa_index_args* args, const float* scores, int64_t ld, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * csa_sparse_attn / hca_dense_attn — softmax attention over compressed entries plus the sliding
+ * window ([V4 blog] Fig. 3 for CSA: the selected entries; Fig. 4 for HCA: every visible entry).
+ *
+ * For query (b, q) at t = q_pos[b][q] with heads q[b][q][h][0..d):
+ *   keys = values = the dequantised cache entries [e2m1*scale*g_kv over d - d_rope channels ‖ rope]
+ *          for idx[b][q][j] in [0, n_c[b]) (csa_sparse_attn; other ids are skipped) or for every
+ *          i < n_c[b] with ratio*i + ratio - 1 <= t (hca_dense_attn; idx ignored),
+ *        ∪ window rows for tokens p in [max(0, t - window + 1), t] held by win_kv[b] at positions
+ *          win_pos0[b] .. win_pos0[b] + Wn - 1 (absent positions are skipped).
+ *   One joint softmax with logits softmax_scale * (q_h · K_j) (softmax_scale == 0 -> 1/sqrt(d)).
+ *   out = bf16(sum_j p_j V_j); lse = ln sum_j exp(logit_j) (fp32; -inf and out = 0 for no keys).
+ * Shapes: q/out[B][Nq][H][d] bf16, q_pos[B][Nq] int64, kv_codes[B][n_max][(d-d_rope)/2],
+ *         kv_scales[B][n_max][S_pad], kv_rope[B][n_max][d_rope] bf16, n_c[B] int32,
+ *         idx[B][Nq][k] int32, win_kv[B][Wn][d] bf16 (may be NULL with Wn = 0), win_pos0[B] int64,
+ *         lse[B][Nq][H] fp32 (may be NULL).
+ * Limits: d in {128, 512} with d_rope == 64 (d = 512) or 32 (d = 128); H <= 64.
+ * Workspace: csa_attn_workspace_size() (split-K partials); `hca` selects the HCA key set.
+ * ------------------------------------------------------------------------------------------------ */
+typedef struct csa_attn_args {
+  uint32_t struct_size;
+  int32_t B, Nq, H, d, d_rope, ratio, n_max, k, Wn, window;
+  float g_kv, softmax_scale;
+  const void* q;
+  const int64_t* q_pos;
+  const uint8_t* kv_codes;
+  const uint8_t* kv_scales;
+  const void* kv_rope;
+  const int32_t* n_c;
+  const int32_t* idx;
+  const void* win_kv;
+  const int64_t* win_pos0;
+  void* out;
+  float* lse;
+} csa_attn_args;
+
+size_t csa_attn_workspace_size(const csa_attn_args* args, int hca);
+csa_status csa_sparse_attn(const csa_attn_args* args, void* ws, size_t ws_bytes, void* stream);
+csa_status hca_dense_attn(const csa_attn_args* args, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H_ */

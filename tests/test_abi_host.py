@@ -1,0 +1,96 @@
+"""The C-ABI library loads and exports every entry point include/csa.h declares; host-side argument
+validation returns the documented status codes without launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa.h")
+
+
+@pytest.fixture(scope="module")
+def csa():
+    from compressed_sparse_attention_18_b200 import build
+    build.build()
+    import compressed_sparse_attention_18_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\*?\s+\**([a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(csa):
+    names = declared_functions()
+    assert len(names) >= 10, names
+    lib = ctypes.CDLL(csa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in csa.h but not exported"
+    assert set(csa.ENTRY_POINTS) <= set(names)
+
+
+def test_status_strings_and_version(csa):
+    lib = csa._lib
+    assert lib.csa_status_string(0) == b"CSA_OK"
+    assert lib.csa_status_string(3) == b"CSA_ERR_WORKSPACE"
+    assert lib.csa_status_string(99) == b"CSA_ERR_UNKNOWN"
+    assert csa.version() >= 100
+
+
+def test_struct_sizes_match_the_header(csa):
+    # the ctypes mirrors are the binding's only knowledge of the layout; a wrong struct_size is rejected
+    a = csa.PackArgs(ctypes.sizeof(csa.PackArgs) + 4, 1, 1, 64, 0, 1, 1.0)
+    assert csa._lib.csa_pack_fp4(ctypes.byref(a), None) == 1
+
+
+def test_invalid_arguments_are_rejected_on_the_host(csa):
+    lib = csa._lib
+    # pack: d_n not a multiple of 32 -> unsupported; null pointers -> invalid
+    a = csa.PackArgs(ctypes.sizeof(csa.PackArgs), 1, 4, 40, 0, 4, 1.0)
+    assert lib.csa_pack_fp4(ctypes.byref(a), None) == 2
+    a = csa.PackArgs(ctypes.sizeof(csa.PackArgs), 1, 4, 64, 0, 4, 1.0)
+    assert lib.csa_pack_fp4(ctypes.byref(a), None) == 1
+    a = csa.PackArgs(ctypes.sizeof(csa.PackArgs), 0, 4, 64, 0, 4, 1.0)
+    assert lib.csa_pack_fp4(ctypes.byref(a), None) == 0          # empty batch: nothing to do
+    assert lib.csa_pack_fp4(None, None) == 1
+    # index: unsupported d_I, too many heads, bad k
+    ia = csa.IndexArgs(ctypes.sizeof(csa.IndexArgs), 1, 1, 8, 96, 4, 8, 16, 1.0, 1.0)
+    assert lib.csa_index_topk(ctypes.byref(ia), None, 0, None) == 2
+    ia = csa.IndexArgs(ctypes.sizeof(csa.IndexArgs), 1, 1, 9, 128, 4, 8, 16, 1.0, 1.0)
+    assert lib.csa_index_topk(ctypes.byref(ia), None, 0, None) == 2
+    ia = csa.IndexArgs(ctypes.sizeof(csa.IndexArgs), 1, 1, 8, 128, 4, 0, 16, 1.0, 1.0)
+    assert lib.csa_index_topk(ctypes.byref(ia), None, 0, None) == 1
+    # index: valid shape, missing pointers -> invalid; workspace query works on the host
+    ia = csa.IndexArgs(ctypes.sizeof(csa.IndexArgs), 2, 1, 8, 128, 4, 16, 4096, 1.0, 1.0)
+    assert lib.csa_index_topk(ctypes.byref(ia), None, 0, None) == 1
+    dummy = 256
+    for f in ("q_I", "w", "k_codes", "k_scales", "n_c", "q_pos", "idx_out"):
+        setattr(ia, f, dummy)
+    ws = lib.csa_index_topk_workspace_size(ctypes.byref(ia))
+    assert ws >= 2 * 4096 * 4                                      # materialised scores
+    assert lib.csa_index_topk(ctypes.byref(ia), ctypes.c_void_p(dummy), ws - 1, None) == 3
+    # attention: unsupported head dim / too many heads
+    aa = csa.AttnArgs(ctypes.sizeof(csa.AttnArgs), 1, 1, 8, 256, 32, 4, 16, 8, 0, 128, 1.0, 0.0)
+    assert lib.csa_sparse_attn(ctypes.byref(aa), None, 0, None) == 2
+    aa = csa.AttnArgs(ctypes.sizeof(csa.AttnArgs), 1, 1, 65, 512, 64, 4, 16, 8, 0, 128, 1.0, 0.0)
+    assert lib.hca_dense_attn(ctypes.byref(aa), None, 0, None) == 2
+    aa = csa.AttnArgs(ctypes.sizeof(csa.AttnArgs), 1, 1, 64, 512, 64, 4, 16, 8, 0, 128, 1.0, 0.0)
+    assert lib.csa_sparse_attn(ctypes.byref(aa), None, 0, None) == 1   # null q / idx
+    # compress: bad ratio, projection mode with unsupported width
+    ca = csa.CompressArgs(ctypes.sizeof(csa.CompressArgs), 1, 8, 64, 64, 0, 0, 0, 0.0)
+    assert lib.csa_compress(ctypes.byref(ca), None) == 1
+
+
+def test_workspace_sizes_scale_with_the_problem(csa):
+    lib = csa._lib
+    def attn_ws(B, k):
+        a = csa.AttnArgs(ctypes.sizeof(csa.AttnArgs), B, 1, 64, 512, 64, 4, 32768, k, 128, 128, 1.0, 0.0)
+        for f in ("q", "q_pos", "kv_codes", "kv_scales", "kv_rope", "n_c", "idx", "win_kv", "win_pos0", "out"):
+            setattr(a, f, 256)
+        return lib.csa_attn_workspace_size(ctypes.byref(a), 0)
+    assert attn_ws(32, 512) > 0                                     # decode: split-K partials
+    assert attn_ws(1024, 512) == 0                                  # enough queries: no split

@@ -1,0 +1,155 @@
+"""GPU parity at full workload sizes, in the launch configuration the benchmark times, checked on
+sampled sequences the oracle computes one by one (every value of those sequences), plus properties
+that hold at any size (all planted needles selected)."""
+import numpy as np
+import pytest
+import torch
+
+from csa_workloads import CFG2, CFG4_HCA, CFG4_REUSE, CFG5, decode_inputs, gen, normal
+from oracle import csa_oracle as O
+from tests.cmp_utils import (LSE_ATOL, LSE_RTOL, OUT_ATOL, OUT_RTOL, assert_close, check_topk_row, f64, np_u8)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _seq_oracle_index(layer, inp, b, s):
+    codes = np_u8(layer.ki.codes[b])
+    scales = np_u8(layer.ki.scales[b])
+    n_c = int(layer.n_c[b])
+    t = int(layer.q_pos[b, 0])
+    sc, ids = O.index_scores(f64(inp["q_I"][b, 0])[None], f64(inp["w"][b, 0])[None], s.g, codes, scales, s.g,
+                             [t], n_c, s.r)
+    return sc, ids, codes, scales
+
+
+def test_decode_cfg2_full_size(cuda_lib):
+    from compressed_sparse_attention_18_b200.layer import CSADecodeLayer, LayerShape
+    s = CFG2
+    ls = LayerShape(B=s.B, n_max=s.n_c, r=s.r, H=s.H, d=s.d, d_r=s.d_r, H_I=s.H_I, d_I=s.d_I, k=s.k, W=s.W)
+    layer = CSADecodeLayer(ls)
+    inp = decode_inputs(s, seed=1, device=DEV)
+    layer.load_history(inp["kv_src"], inp["kI_src"], s.n_c)
+    layer.win.copy_(inp["win_kv"])
+    out, lse, idx = layer.step(inp["C"], inp["Z"], inp["b_pos"], inp["W_IK"], inp["q"], inp["q_I"], inp["w"])
+    torch.cuda.synchronize()
+    # property at full size: every planted needle is selected, in every sequence
+    for b in range(s.B):
+        sel = set(idx[b, 0].tolist())
+        assert set(inp["needle_pos"][b].tolist()) <= sel, f"needle missed in b={b}"
+        assert len(sel) == s.k
+    for b in (0, 17, 31):
+        # compressor + pack of the new entry
+        c_ref = O.compress_pool(f64(inp["C"][b]), f64(inp["Z"][b]), f64(inp["b_pos"]), s.r, s.d_r, 10000.0,
+                                s.r * (s.n_c - 1))
+        assert_close(f64(layer.c_new[b]), c_ref, 1e-3, 2.0 ** -7 * 1.01, "c")
+        codes, scales, rope = O.pack_fp4(f64(layer.c_new[b]), s.d_r, 1.0)
+        assert np.array_equal(np_u8(layer.kv.codes[b, s.n_c - 1:]), codes)
+        assert np.array_equal(np_u8(layer.kv.scales[b, s.n_c - 1:]), scales)
+        kI_ref = O.index_key(f64(layer.c_new[b]), f64(inp["W_IK"]))
+        assert_close(f64(layer.kI_new[b]), kI_ref, 1e-3, 2.0 ** -7 * 1.01, "k_I")
+        # history pack bit-exact for this sequence
+        hc, hs, hr = O.pack_fp4(f64(inp["kv_src"][b, : s.n_c - 1]), s.d_r, 1.0)
+        assert np.array_equal(np_u8(layer.kv.codes[b, : s.n_c - 1]), hc)
+        assert np.array_equal(np_u8(layer.kv.scales[b, : s.n_c - 1]), hs)
+        # index + top-k on the same cache bytes
+        sc, ids, _, _ = _seq_oracle_index(layer, inp, b, s)
+        check_topk_row(idx[b, 0].cpu().numpy(), sc[0], ids[0], s.k, f"cfg2 b={b}")
+        # attention on the GPU's selection (same upstream bytes)
+        rows = O.entry_kv(np_u8(layer.kv.codes[b]), np_u8(layer.kv.scales[b]), f64(layer.kv.rope[b]), s.d_n, 1.0)
+        o_ref, l_ref = O.attention(f64(inp["q"][b]), [s.T - 1], rows, idx[b].cpu().numpy(), s.n_c,
+                                   f64(layer.win[b]), s.T - s.W, s.W, s.d ** -0.5)
+        assert_close(f64(out[b]), o_ref, OUT_ATOL, OUT_RTOL, f"out b={b}")
+        assert_close(lse[b].cpu().numpy(), l_ref, LSE_ATOL, LSE_RTOL, f"lse b={b}")
+
+
+def test_decode_cfg5_hierarchical_full_size(cuda_lib):
+    """1M-token contexts: level-1 full index (tournament top-k over 262144 entries) with a pool of 1024
+    blocks x 8, level 2 re-scores the pool with the next layer's query."""
+    csa = cuda_lib
+    s = CFG5
+    inp = decode_inputs(s, seed=4, device=DEV, needles=0, qnorm_student_t=True)
+    ki = csa.PackedCache(s.B, s.n_c, s.d_I, 0, DEV)
+    csa.pack_fp4(inp["kI_src"], ki)
+    n_c = inp["n_c"]
+    q_pos = inp["q_pos"]
+    idx1, sc1, pool = csa.index_topk(inp["q_I"], inp["w"], ki, n_c, q_pos, ratio=s.r, k=s.k,
+                                     pool_blocks=s.pool_blocks, want_scores=True)
+    G = gen(99, DEV)
+    qI2 = normal(inp["q_I"].shape, 1.0, G, DEV)
+    w2 = normal(inp["w"].shape, 0.35, G, DEV, torch.float32)
+    idx2, _, _ = csa.index_topk(qI2, w2, ki, n_c, q_pos, ratio=s.r, k=s.k, cand=pool)
+    torch.cuda.synchronize()
+    b = 2
+    codes, scales = np_u8(ki.codes[b]), np_u8(ki.scales[b])
+    t = int(q_pos[b, 0])
+    sc, ids = O.index_scores(f64(inp["q_I"][b, 0])[None], f64(inp["w"][b, 0])[None], 1.0, codes, scales, 1.0, [t],
+                             s.n_c, s.r)
+    check_topk_row(idx1[b, 0].cpu().numpy(), sc[0], ids[0], s.k, "level 1")
+    pool_ref, blk_ref = O.hierarchical_pool(sc, s.pool_blocks, 8)
+    gp = pool[b, 0].cpu().numpy().reshape(s.pool_blocks, 8)
+    got_blocks = np.array(sorted(int(r[r >= 0][0]) // 8 for r in gp if np.any(r >= 0)))
+    bs = sc[0].reshape(-1, 8).max(axis=1)
+    check_topk_row(got_blocks, bs, np.arange(len(bs)), s.pool_blocks, "pool blocks")
+    # level 2 over the GPU's pool (same upstream ids)
+    cand = pool[b].cpu().numpy()
+    sc2, ids2 = O.index_scores(f64(qI2[b, 0])[None], f64(w2[b, 0])[None], 1.0, codes, scales, 1.0, [t], s.n_c, s.r,
+                               keys=cand)
+    check_topk_row(idx2[b, 0].cpu().numpy(), sc2[0], ids2[0], s.k, "level 2")
+
+
+def test_hca_cfg4_full_size(cuda_lib):
+    """HCA: 128x pooling of 1,048,576 tokens (8192 entries) for one sequence, decode attention of 16
+    sequences over all 8192 entries plus the window."""
+    csa = cuda_lib
+    s = CFG4_HCA
+    G = gen(3, DEV)
+    C = normal((1, s.T, s.d), 1.0, G, DEV)
+    Z = normal((1, s.T, s.d), 1.0, G, DEV)
+    b_pos = normal((s.r, s.d), 0.1, G, DEV, torch.float32)
+    c, _, _, _ = csa.compress(C=C, Z=Z, b_pos=b_pos, ratio=s.r, d_rope=s.d_r, rope_theta=10000.0)
+    torch.cuda.synchronize()
+    for e in (0, 4095, 8191):                              # sampled entries: 128 tokens each
+        sl = slice(e * s.r, (e + 1) * s.r)
+        ref = O.compress_pool(f64(C[0, sl]), f64(Z[0, sl]), f64(b_pos), s.r, s.d_r, 10000.0, e * s.r)
+        assert_close(f64(c[0, e:e + 1]), ref, 1e-3, 2.0 ** -7 * 1.01, f"hca entry {e}")
+    del C, Z
+    inp = decode_inputs(s, seed=3, device=DEV, needles=0)
+    kv_src = inp["kv_src"]
+    kv_src[0] = c[0]                                       # sequence 0 holds the pooled entries
+    cache = csa.PackedCache(s.B, s.n_c, s.d, s.d_r, DEV)
+    csa.pack_fp4(kv_src, cache)
+    out, lse = csa.hca_attn(inp["q"], inp["q_pos"], cache, inp["n_c"], inp["win_kv"], inp["win_pos0"], ratio=s.r)
+    torch.cuda.synchronize()
+    for b in (0, 9):
+        rows = O.entry_kv(np_u8(cache.codes[b]), np_u8(cache.scales[b]), f64(cache.rope[b]), s.d_n, 1.0)
+        o_ref, l_ref = O.hca_attention(f64(inp["q"][b]), [s.T - 1], rows, s.n_c, s.r, f64(inp["win_kv"][b]),
+                                       s.T - s.W, s.W, s.d ** -0.5)
+        assert_close(f64(out[b]), o_ref, OUT_ATOL, OUT_RTOL, f"hca out b={b}")
+        assert_close(lse[b].cpu().numpy(), l_ref, LSE_ATOL, LSE_RTOL, f"hca lse b={b}")
+
+
+def test_reuse_cfg4_full_size(cuda_lib):
+    """Cross-layer reuse: layer 1 Full over 262144 entries -> top-2048; layer 2 Reindex of those 2048
+    with its own query -> top-512; Reuse passes layer 2's indices to attention unchanged."""
+    csa = cuda_lib
+    s = CFG4_REUSE
+    B = 4
+    inp = decode_inputs(s, seed=5, device=DEV, B=B, needles=0)
+    ki = csa.PackedCache(B, s.n_c, s.d_I, 0, DEV)
+    csa.pack_fp4(inp["kI_src"], ki)
+    idx1, _, _ = csa.index_topk(inp["q_I"], inp["w"], ki, inp["n_c"], inp["q_pos"], ratio=s.r, k=s.k)
+    G = gen(77, DEV)
+    qI2 = normal(inp["q_I"].shape, 1.0, G, DEV)
+    w2 = normal(inp["w"].shape, 0.35, G, DEV, torch.float32)
+    idx2, _, _ = csa.index_topk(qI2, w2, ki, inp["n_c"], inp["q_pos"], ratio=s.r, k=s.extra["k2"], cand=idx1)
+    torch.cuda.synchronize()
+    b = 1
+    codes, scales = np_u8(ki.codes[b]), np_u8(ki.scales[b])
+    t = int(inp["q_pos"][b, 0])
+    sc, ids = O.index_scores(f64(inp["q_I"][b, 0])[None], f64(inp["w"][b, 0])[None], 1.0, codes, scales, 1.0, [t],
+                             s.n_c, s.r)
+    check_topk_row(idx1[b, 0].cpu().numpy(), sc[0], ids[0], s.k, "layer 1 full")
+    sc2, ids2 = O.index_scores(f64(qI2[b, 0])[None], f64(w2[b, 0])[None], 1.0, codes, scales, 1.0, [t], s.n_c, s.r,
+                               keys=idx1[b].cpu().numpy())
+    check_topk_row(idx2[b, 0].cpu().numpy(), sc2[0], ids2[0], s.extra["k2"], "layer 2 reindex")

@@ -1,0 +1,295 @@
+"""GPU parity: every stage of the CUDA path (through the C ABI) against the CPU oracle on the same
+seeded inputs and the same upstream bytes, at sizes the oracle finishes in seconds that still span
+several tiles and a ragged tail, plus the edge cases (empty / ragged / fully masked / ties / k >= n)."""
+import numpy as np
+import pytest
+import torch
+
+from csa_workloads import CFG1, gen, normal, small_layer_inputs
+from oracle import csa_oracle as O
+from tests.cmp_utils import (LSE_ATOL, LSE_RTOL, OUT_ATOL, OUT_RTOL, SCORE_RTOL, assert_close,
+                             check_topk_row, f64, np_u8)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def bf16_bits(t):
+    return t.detach().to("cpu").view(torch.int16).numpy()
+
+
+# ------------------------------------------------------------------------------------------ pack
+
+@pytest.mark.parametrize("d,d_r,g", [(512, 64, 1.0), (128, 32, 2.0 ** -4), (128, 0, 1.0), (64, 0, 0.5)])
+def test_pack_bit_exact(cuda_lib, d, d_r, g):
+    csa = cuda_lib
+    B, n, n_max = 3, 37, 60
+    G = gen(11)
+    x = torch.randn((B, n, d), generator=G)
+    x[0, 0] = 0.0                                        # all-zero row -> zero scales
+    x[0, 1] *= 1e-7                                      # scales underflow toward E4M3 subnormals / zero
+    x[0, 2] *= 1e4                                       # scales saturate at 448
+    x[1, 3, :32] = torch.tensor(O.e2m1_decode(np.arange(32) % 16) * 0.75)   # exactly representable block
+    x[2, 4, 1::2] = -1e-3                                # rounds to -0 -> +0
+    src = x.to(torch.bfloat16)
+    cache = csa.PackedCache(B, n_max, d, d_r, DEV, g)
+    row0 = torch.tensor([0, 5, n_max - n], dtype=torch.int32, device=DEV)
+    csa.pack_fp4(src.to(DEV), cache, row0)
+    torch.cuda.synchronize()
+    for b in range(B):
+        codes, scales, rope = O.pack_fp4(f64(src[b]), d_r, g)
+        r0 = int(row0[b])
+        assert np.array_equal(np_u8(cache.codes[b, r0:r0 + n]), codes), f"codes b={b}"
+        assert np.array_equal(np_u8(cache.scales[b, r0:r0 + n]), scales), f"scales b={b}"
+        if d_r:
+            assert np.array_equal(bf16_bits(cache.rope[b, r0:r0 + n]), bf16_bits(src[b, :, d - d_r:]))
+    # rows outside [row0, row0 + n) untouched
+    assert int(cache.codes[0, n:].abs().sum()) == 0
+
+
+# ------------------------------------------------------------------------------------ compressor
+
+def _ulp_close(got, ref, what):
+    rms = float(np.sqrt(np.mean(ref ** 2))) or 1.0
+    assert_close(got, ref, 1e-3 * rms, 2.0 ** -7 * 1.01, what)
+
+
+def test_compress_projection_mode_cfg1(cuda_lib):
+    csa = cuda_lib
+    inp = small_layer_inputs(CFG1, seed=0)
+    t = {k: v.to(DEV) for k, v in inp.items()}
+    c, kI, C, Z = csa.compress(x=t["x"], W_kv=t["W_kv"], W_g=t["W_g"], b_pos=t["b_pos"], ratio=4,
+                               d_rope=CFG1.d_r, rope_theta=10000.0, W_IK=t["W_IK"])
+    torch.cuda.synchronize()
+    x = f64(inp["x"][0])
+    _ulp_close(f64(C[0]), O.project(x, f64(inp["W_kv"])), "C")
+    _ulp_close(f64(Z[0]), O.project(x, f64(inp["W_g"])), "Z")
+    # pooling and the index-key projection on the same upstream bytes
+    c_ref = O.compress_pool(f64(C[0]), f64(Z[0]), f64(inp["b_pos"]), 4, CFG1.d_r, 10000.0, 0)
+    _ulp_close(f64(c[0]), c_ref, "c")
+    _ulp_close(f64(kI[0]), O.index_key(f64(c[0]), f64(inp["W_IK"])), "k_I")
+
+
+@pytest.mark.parametrize("r,T,d,d_r,pos0", [(4, 4 * 97 + 3, 512, 64, 4 * 1000), (128, 128 * 9 + 17, 512, 64, 0),
+                                            (1, 33, 128, 32, 7)])
+def test_compress_pooling_mode(cuda_lib, r, T, d, d_r, pos0):
+    csa = cuda_lib
+    G = gen(3)
+    B = 2
+    C = normal((B, T, d), 1.0, G)
+    Z = normal((B, T, d), 1.0, G)
+    b_pos = normal((r, d), 0.1, G, dtype=torch.float32)
+    W_IK = normal((d, 128), d ** -0.5, G)
+    p0 = torch.tensor([pos0, pos0 + 8 * r], dtype=torch.int64)
+    c, kI, _, _ = csa.compress(C=C.to(DEV), Z=Z.to(DEV), b_pos=b_pos.to(DEV), ratio=r, d_rope=d_r,
+                               rope_theta=10000.0, pos0=p0.to(DEV), W_IK=W_IK.to(DEV))
+    torch.cuda.synchronize()
+    for b in range(B):
+        ref = O.compress_pool(f64(C[b]), f64(Z[b]), f64(b_pos), r, d_r, 10000.0, int(p0[b]))
+        assert c.shape[1] == T // r
+        _ulp_close(f64(c[b]), ref, f"c b={b}")
+        _ulp_close(f64(kI[b]), O.index_key(f64(c[b]), f64(W_IK)), f"k_I b={b}")
+
+
+# ---------------------------------------------------------------------------------------- indexer
+
+def _index_case(csa, *, B, n_max, n_c, d_I, H_I, Nq, q_pos, k, g_q=1.0, g_k=1.0, key_std=1.0, seed=0,
+                cand=None, pool_blocks=0, identical_keys=False):
+    G = gen(seed)
+    kI = normal((B, n_max, d_I), key_std, G)
+    if identical_keys:
+        kI[:] = kI[:, :1]
+    qI = normal((B, Nq, H_I, d_I), 1.0, G)
+    w = normal((B, Nq, H_I), H_I ** -0.5, G, dtype=torch.float32)
+    kc = csa.PackedCache(B, n_max, d_I, 0, DEV, g_k)
+    csa.pack_fp4(kI.to(DEV), kc)
+    n_c_t = torch.tensor(n_c, dtype=torch.int32)
+    q_pos_t = torch.tensor(q_pos, dtype=torch.int64).view(B, Nq)
+    idx, sc, pool = csa.index_topk(qI.to(DEV), w.to(DEV), kc, n_c_t.to(DEV), q_pos_t.to(DEV), ratio=4, k=k, g_q=g_q,
+                                   cand=cand.to(DEV) if cand is not None else None, pool_blocks=pool_blocks,
+                                   want_scores=True)
+    torch.cuda.synchronize()
+    swaps = 0
+    for b in range(B):
+        codes, scales, _ = O.pack_fp4(f64(kI[b]), 0, g_k)
+        assert np.array_equal(np_u8(kc.codes[b]), codes)
+        keys = None if cand is None else cand[b].numpy()
+        s_ref, ids = O.index_scores(f64(qI[b]), f64(w[b]), g_q, codes, scales, g_k, q_pos_t[b].numpy(), n_c[b], 4,
+                                    keys=keys)
+        gi = idx[b].cpu().numpy()
+        gs = sc[b].cpu().numpy()
+        for q in range(Nq):
+            swaps += check_topk_row(gi[q], s_ref[q], ids[q], k, f"b={b} q={q}")
+            # scores the kernel returns for its selection match the oracle's for the same ids
+            score_of = dict(zip(ids[q].tolist(), s_ref[q].tolist()))
+            sel = gi[q] >= 0
+            ref = np.array([score_of[i] for i in gi[q][sel]])
+            rowmax = np.max(np.abs(s_ref[q][np.isfinite(s_ref[q])])) if np.any(np.isfinite(s_ref[q])) else 0
+            assert_close(gs[q][sel], ref, SCORE_RTOL * rowmax, SCORE_RTOL, f"scores b={b} q={q}")
+            assert np.all(np.isneginf(gs[q][~sel]))
+        if pool_blocks:
+            pr, blk = O.hierarchical_pool(s_ref, pool_blocks, 8)
+            gp = pool[b].cpu().numpy().reshape(Nq, pool_blocks, 8)
+            for q in range(Nq):
+                # each GPU block: 8 consecutive ids (or -1 where not visible); block set vs oracle's
+                got_blocks = set()
+                for j in range(pool_blocks):
+                    row = gp[q, j]
+                    ok = row[row >= 0]
+                    if len(ok) == 0:
+                        continue
+                    bid = int(ok[0]) // 8
+                    got_blocks.add(bid)
+                    for e in range(8):
+                        i = bid * 8 + e
+                        want = i if (i < s_ref.shape[1] and np.isfinite(s_ref[q, i])) else -1
+                        assert row[e] == want
+                bscore = {int(bb): np.max(s_ref[q, bb * 8: bb * 8 + 8]) for bb in range(s_ref.shape[1] // 8 + 1)
+                          if bb * 8 < s_ref.shape[1]}
+                ids_b = np.array(sorted(bscore)); sc_b = np.array([bscore[i] for i in ids_b])
+                gsel = np.array(sorted(got_blocks) + [-1] * (pool_blocks - len(got_blocks)))
+                swaps += check_topk_row(gsel, sc_b, ids_b, pool_blocks, f"pool b={b} q={q}")
+    return idx, swaps
+
+
+def test_index_cfg1_small_layer(cuda_lib):
+    q_pos = list(range(4080, 4096))
+    _index_case(cuda_lib, B=1, n_max=1024, n_c=[1024], d_I=64, H_I=4, Nq=16, q_pos=q_pos, k=64,
+                g_q=1.0, g_k=2.0 ** -4, key_std=0.03)
+
+
+def test_index_decode_ragged(cuda_lib):
+    n_c = [4096, 1000, 37, 2048]
+    q_pos = [4 * 4096 - 1, 4 * 1000 - 1, 4 * 37 - 1, 4 * 500 + 2]   # last: only 500 visible
+    _index_case(cuda_lib, B=4, n_max=4096, n_c=n_c, d_I=128, H_I=8, Nq=1, q_pos=q_pos, k=512, seed=1)
+
+
+def test_index_prefill_causal_multi_query(cuda_lib):
+    q_pos = list(range(1000, 1048))                       # 48 queries: one full 32-query tile + a tail
+    _index_case(cuda_lib, B=1, n_max=512, n_c=[300], d_I=128, H_I=8, Nq=48, q_pos=q_pos, k=64, seed=2)
+
+
+def test_index_tournament_long_row(cuda_lib):
+    n = 40000                                             # > one 32768-column top-k chunk
+    _index_case(cuda_lib, B=2, n_max=n, n_c=[n, n - 123], d_I=128, H_I=8, Nq=1, q_pos=[4 * n - 1, 4 * n - 1],
+                k=256, seed=3)
+
+
+def test_index_reindex_candidates(cuda_lib):
+    G = gen(5)
+    B, Nq, n_max, n_cand = 2, 2, 3000, 2048
+    cand = torch.randint(-1, n_max + 50, (B, Nq, n_cand), generator=G, dtype=torch.int32)
+    for b in range(B):
+        for q in range(Nq):                               # distinct ids (a previous layer's selection)
+            cand[b, q] = torch.randperm(n_max + 50, generator=G)[:n_cand].to(torch.int32) - 1
+    _index_case(cuda_lib, B=B, n_max=n_max, n_c=[n_max, 2500], d_I=128, H_I=8, Nq=Nq,
+                q_pos=[4 * n_max - 1, 4 * 2000, 4 * 2500 - 1, 4 * 100], k=512, seed=5, cand=cand)
+
+
+def test_index_hierarchical_pool(cuda_lib):
+    _index_case(cuda_lib, B=2, n_max=8192, n_c=[8192, 5000], d_I=128, H_I=8, Nq=1,
+                q_pos=[4 * 8192 - 1, 4 * 4000 + 1], k=128, seed=6, pool_blocks=64)
+
+
+def test_index_exact_ties_take_smallest_ids(cuda_lib):
+    idx, swaps = _index_case(cuda_lib, B=1, n_max=64, n_c=[64], d_I=128, H_I=8, Nq=1, q_pos=[255], k=10, seed=7,
+                             identical_keys=True)
+    assert swaps == 0
+    assert sorted(idx[0, 0].tolist()) == list(range(10))
+
+
+def test_index_k_larger_than_visible(cuda_lib):
+    idx, _ = _index_case(cuda_lib, B=2, n_max=256, n_c=[256, 256], d_I=64, H_I=4, Nq=1, q_pos=[4 * 20 - 1, 2],
+                         k=100, seed=8)
+    assert sorted(idx[0, 0].tolist())[-20:] == list(range(20)) and (idx[0, 0] == -1).sum() == 80
+    assert (idx[1, 0] == -1).all()                        # t = 2: nothing visible yet
+
+
+# -------------------------------------------------------------------------------------- attention
+
+def _attn_case(csa, *, B, Nq, H, d, d_r, n_max, n_c, q_pos, k=0, Wn=128, win_pos0=None, hca=False, ratio=4,
+               seed=0, g=1.0, q_scale=1.0):
+    G = gen(seed)
+    kv = normal((B, n_max, d), 1.0, G)
+    q = normal((B, Nq, H, d), q_scale, G)
+    win = normal((B, Wn, d), 1.0, G) if Wn else None
+    cache = csa.PackedCache(B, n_max, d, d_r, DEV, g)
+    csa.pack_fp4(kv.to(DEV), cache)
+    q_pos_t = torch.tensor(q_pos, dtype=torch.int64).view(B, Nq)
+    if win_pos0 is None:
+        win_pos0 = [int(q_pos_t[b].max()) - Wn + 1 for b in range(B)]
+    wp0 = torch.tensor(win_pos0, dtype=torch.int64)
+    n_c_t = torch.tensor(n_c, dtype=torch.int32)
+    idx = None
+    if not hca:
+        idx = torch.empty((B, Nq, k), dtype=torch.int32)
+        for b in range(B):
+            for qq in range(Nq):
+                perm = torch.randperm(n_max + 40, generator=G)[:k].to(torch.int32) - 20   # some < 0, some >= n_c
+                idx[b, qq] = perm
+    if hca:
+        out, lse = csa.hca_attn(q.to(DEV), q_pos_t.to(DEV), cache, n_c_t.to(DEV),
+                                win.to(DEV) if win is not None else None, wp0.to(DEV) if win is not None else None,
+                                ratio=ratio)
+    else:
+        out, lse = csa.sparse_attn(q.to(DEV), q_pos_t.to(DEV), cache, n_c_t.to(DEV), idx.to(DEV),
+                                   win.to(DEV) if win is not None else None, wp0.to(DEV) if win is not None else None,
+                                   ratio=ratio)
+    torch.cuda.synchronize()
+    scale = d ** -0.5
+    for b in range(B):
+        codes, scales, rope = O.pack_fp4(f64(kv[b]), d_r, g)
+        rows = O.entry_kv(codes, scales, rope, d - d_r, g)
+        wb = f64(win[b]) if win is not None else np.zeros((0, d))
+        if hca:
+            o_ref, l_ref = O.hca_attention(f64(q[b]), q_pos_t[b].numpy(), rows, n_c[b], ratio, wb, win_pos0[b], 128,
+                                           scale)
+        else:
+            o_ref, l_ref = O.attention(f64(q[b]), q_pos_t[b].numpy(), rows, idx[b].numpy(), n_c[b], wb, win_pos0[b],
+                                       128, scale)
+        assert_close(f64(out[b]), o_ref, OUT_ATOL, OUT_RTOL, f"out b={b}")
+        assert_close(lse[b].cpu().numpy(), l_ref, LSE_ATOL, LSE_RTOL, f"lse b={b}")
+    return out, lse
+
+
+def test_attn_cfg1_shapes(cuda_lib):
+    q_pos = list(range(4080, 4096))
+    _attn_case(cuda_lib, B=1, Nq=16, H=8, d=128, d_r=32, n_max=1024, n_c=[1024], q_pos=q_pos, k=64, Wn=143,
+               g=2.0 ** -4, seed=1)
+
+
+def test_attn_cfg1_peaked_queries(cuda_lib):
+    q_pos = list(range(4080, 4096))
+    _attn_case(cuda_lib, B=1, Nq=16, H=8, d=128, d_r=32, n_max=1024, n_c=[1024], q_pos=q_pos, k=64, Wn=143,
+               seed=2, q_scale=128 ** 0.5 / 4)
+
+
+def test_attn_decode_d512(cuda_lib):
+    n_c = [2048, 700, 2048]
+    q_pos = [4 * 2048 - 1, 4 * 700 - 1, 4 * 1500 + 3]
+    _attn_case(cuda_lib, B=3, Nq=1, H=64, d=512, d_r=64, n_max=2048, n_c=n_c, q_pos=q_pos, k=512, seed=3)
+
+
+def test_attn_no_window_and_partial_window(cuda_lib):
+    _attn_case(cuda_lib, B=2, Nq=1, H=64, d=512, d_r=64, n_max=600, n_c=[600, 600], q_pos=[2399, 2399], k=100,
+               Wn=0, seed=4)
+    # window buffer that starts after t - W + 1 (only part of the window held) and a query near the start
+    _attn_case(cuda_lib, B=2, Nq=1, H=64, d=512, d_r=64, n_max=64, n_c=[64, 2], q_pos=[255, 9], k=64, Wn=50,
+               win_pos0=[206, 0], seed=5)
+
+
+def test_attn_many_queries_single_split(cuda_lib):
+    q_pos = list(range(3000, 3000 + 150))                # >= 148 rows: the direct-write path
+    _attn_case(cuda_lib, B=1, Nq=150, H=64, d=512, d_r=64, n_max=800, n_c=[800], q_pos=q_pos, k=64, Wn=300,
+               seed=6)
+
+
+def test_attn_hca(cuda_lib):
+    _attn_case(cuda_lib, B=2, Nq=1, H=64, d=512, d_r=64, n_max=300, n_c=[300, 300],
+               q_pos=[128 * 300 - 1, 128 * 150 + 5], hca=True, ratio=128, seed=7)
+
+
+def test_attn_hca_empty_set(cuda_lib):
+    out, lse = _attn_case(cuda_lib, B=1, Nq=1, H=64, d=512, d_r=64, n_max=16, n_c=[0], q_pos=[100], hca=True,
+                          ratio=128, Wn=0, seed=8)
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
