@@ -35,6 +35,16 @@ __device__ __forceinline__ void mma16816(float* c, const uint32_t* a, uint32_t b
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void cpa16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src));
+}
+__device__ __forceinline__ void cpa4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src));
+}
+__device__ __forceinline__ void cpa_commit_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // Byte offset of 16-byte chunk `c` of row `r` in a [rows][D] bf16 tile, chunks XOR-swizzled by row.
 template <int D>
 __device__ __forceinline__ uint32_t swz(int r, int c) {
@@ -71,10 +81,14 @@ __global__ void __launch_bounds__(AT_WARPS * 32, 1) attn_kernel(AttnParams P) {
   const int S_blocks = d_n / 32;
   const int S_pad = (S_blocks + 3) & ~3;
 
+  constexpr int RAW_SC = (D - (D == 512 ? 64 : 32)) / 2;   // staging row: codes | scales (16) | rope
+  constexpr int RAW_ROPE = RAW_SC + 16;
+  constexpr int RAW = RAW_ROPE + (D == 512 ? 64 : 32) * 2;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* sQ = smem;                                   // [HP][D] bf16
   uint8_t* sK = sQ + HP * D * 2;                        // [AT_KC][D] bf16
   float* sS = reinterpret_cast<float*>(sK + AT_KC * D * 2);  // [HG][DS][16][AT_KC]
+  uint8_t* sRaw = reinterpret_cast<uint8_t*>(sS) + (DS > 1 ? HG * DS * 16 * AT_KC * 4 : 0);  // [AT_KC][RAW]
   __shared__ int s_valid[AT_KC];
 
   const int unit = blockIdx.x;
@@ -107,11 +121,11 @@ __global__ void __launch_bounds__(AT_WARPS * 32, 1) attn_kernel(AttnParams P) {
 
   // Q -> shared (rows >= H zero)
   const uint16_t* qsrc = P.q + (size_t)bq * P.H * D;
+  const uint32_t sQa0 = (uint32_t)__cvta_generic_to_shared(sQ);
   for (int i = tid; i < HP * CH; i += blockDim.x) {
     const int r = i / CH, c = i % CH;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < P.H) v = *reinterpret_cast<const uint4*>(qsrc + (size_t)r * D + c * 8);
-    *reinterpret_cast<uint4*>(sQ + swz<D>(r, c)) = v;
+    if (r < P.H) cpa16(sQa0 + swz<D>(r, c), qsrc + (size_t)r * D + c * 8);
+    else *reinterpret_cast<uint4*>(sQ + swz<D>(r, c)) = make_uint4(0, 0, 0, 0);
   }
 
   float o[NT_O][4];
@@ -128,7 +142,8 @@ __global__ void __launch_bounds__(AT_WARPS * 32, 1) attn_kernel(AttnParams P) {
 
   for (int c = c_begin; c < c_end; ++c) {
     __syncthreads();  // previous chunk's K tile fully consumed
-    // ---- gather: each warp fills AT_KC / AT_WARPS rows
+    // ---- gather, phase 1: asynchronous copies (raw FP4 rows -> staging, window rows -> K tile)
+    const uint32_t sRawa = (uint32_t)__cvta_generic_to_shared(sRaw);
     for (int rr = 0; rr < AT_KC / AT_WARPS; ++rr) {
       const int row = warp * (AT_KC / AT_WARPS) + rr;
       const int li = c * AT_KC + row;
@@ -142,37 +157,46 @@ __global__ void __launch_bounds__(AT_WARPS * 32, 1) attn_kernel(AttnParams P) {
         src = (wlo + (li - n_sel)) - P.win_pos0[b];
       }
       if (kind == 1) {
-        if (lane < S_blocks) {
-          const uint4 cv = *reinterpret_cast<const uint4*>(codes_b + src * (d_n / 2) + lane * 16);
-          const float s = e4m3_to_f32(scales_b[src * S_pad + lane]) * P.g;
-          const uint32_t w4[4] = {cv.x, cv.y, cv.z, cv.w};
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t outw[4];
-#pragma unroll
-            for (int bb = 0; bb < 4; bb += 2) {
-              const uint32_t h0 = e2m1x2_to_h2(w4[q4] >> (bb * 8));
-              const uint32_t h1 = e2m1x2_to_h2(w4[q4] >> (bb * 8 + 8));
-              const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
-              const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-              outw[bb] = pack_bf16x2(f0.x * s, f0.y * s);
-              outw[bb + 1] = pack_bf16x2(f1.x * s, f1.y * s);
-            }
-            *reinterpret_cast<uint4*>(sK + swz<D>(row, lane * 4 + q4)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-          }
-        } else if (lane >= 16 && lane < 16 + P.d_r / 8) {
-          const int rc = lane - 16;
-          const uint4 v = *reinterpret_cast<const uint4*>(rope_b + src * P.d_r + rc * 8);
-          *reinterpret_cast<uint4*>(sK + swz<D>(row, d_n / 8 + rc)) = v;
-        }
+        const uint32_t dst = sRawa + row * RAW;
+        if (lane < d_n / 32) cpa16(dst + lane * 16, codes_b + src * (d_n / 2) + lane * 16);
+        else if (lane >= 16 && lane < 16 + P.d_r / 8)
+          cpa16(dst + RAW_ROPE + (lane - 16) * 16, rope_b + src * P.d_r + (lane - 16) * 8);
+        else if (lane == 31)
+          for (int q4 = 0; q4 < S_pad; q4 += 4) cpa4(dst + RAW_SC + q4, scales_b + src * S_pad + q4);
       } else if (kind == 2) {
         const uint16_t* wrow = P.win + ((size_t)b * P.Wn + src) * D;
-        for (int cc = lane; cc < CH; cc += 32)
-          *reinterpret_cast<uint4*>(sK + swz<D>(row, cc)) = *reinterpret_cast<const uint4*>(wrow + cc * 8);
+        for (int cc = lane; cc < CH; cc += 32) cpa16(sKa + swz<D>(row, cc), wrow + cc * 8);
       } else {
         for (int cc = lane; cc < CH; cc += 32) *reinterpret_cast<uint4*>(sK + swz<D>(row, cc)) = make_uint4(0, 0, 0, 0);
       }
-      if (lane == 0) s_valid[row] = kind != 0;
+      if (lane == 0) s_valid[row] = kind;
+    }
+    cpa_commit_wait_all();
+    __syncthreads();
+    // ---- gather, phase 2: dequantise staged FP4 rows into the K tile (bf16, exact)
+    for (int rr = 0; rr < AT_KC / AT_WARPS; ++rr) {
+      const int row = warp * (AT_KC / AT_WARPS) + rr;
+      if (s_valid[row] != 1) continue;
+      const uint8_t* raw = sRaw + row * RAW;
+      if (lane < d_n / 32) {
+        const uint4 cv = *reinterpret_cast<const uint4*>(raw + lane * 16);
+        const float sc = e4m3_to_f32(raw[RAW_SC + lane]) * P.g;
+        const uint32_t w4[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t outw[4];
+#pragma unroll
+          for (int bb = 0; bb < 4; ++bb) {
+            const uint32_t h = e2m1x2_to_h2(w4[q4] >> (bb * 8));
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+            outw[bb] = pack_bf16x2(f.x * sc, f.y * sc);
+          }
+          *reinterpret_cast<uint4*>(sK + swz<D>(row, lane * 4 + q4)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+        }
+      } else if (lane >= 16 && lane < 16 + P.d_r / 8) {
+        const int rc = lane - 16;
+        *reinterpret_cast<uint4*>(sK + swz<D>(row, d_n / 8 + rc)) = *reinterpret_cast<const uint4*>(raw + RAW_ROPE + rc * 16);
+      }
     }
     __syncthreads();
 
@@ -227,7 +251,7 @@ __global__ void __launch_bounds__(AT_WARPS * 32, 1) attn_kernel(AttnParams P) {
     float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int j = 0; j < NT_S; ++j) {
-      const bool v0 = s_valid[j * 8 + 2 * t], v1 = s_valid[j * 8 + 2 * t + 1];
+      const bool v0 = s_valid[j * 8 + 2 * t] != 0, v1 = s_valid[j * 8 + 2 * t + 1] != 0;
       sacc[j][0] = v0 ? sacc[j][0] * P.scale_log2 : -INFINITY;
       sacc[j][1] = v1 ? sacc[j][1] * P.scale_log2 : -INFINITY;
       sacc[j][2] = v0 ? sacc[j][2] * P.scale_log2 : -INFINITY;
@@ -320,26 +344,48 @@ __global__ void __launch_bounds__(AT_WARPS * 32, 1) attn_kernel(AttnParams P) {
 }
 
 // Merge split partials: lse = log sum_s exp(lse_s); out = sum_s exp(lse_s - lse) O_s.
-__global__ void attn_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int splits,
-                                  int H, int D, uint16_t* __restrict__ out, float* __restrict__ lse) {
-  const int bq = blockIdx.x;
-  for (int hd = threadIdx.x; hd < H * D; hd += blockDim.x) {
-    const int h = hd / D;
+// One CTA per (query, head); each thread owns 4 consecutive output dims, the split weights are
+// computed once per CTA in shared memory.
+constexpr int MERGE_MAX_SPLITS = 64;
+__global__ void __launch_bounds__(128) attn_merge_kernel(const float* __restrict__ part_o,
+                                                         const float* __restrict__ part_lse, int splits, int H, int D,
+                                                         uint16_t* __restrict__ out, float* __restrict__ lse) {
+  __shared__ float s_w[MERGE_MAX_SPLITS];
+  __shared__ float s_tot[2];
+  const int bq = blockIdx.x / H, h = blockIdx.x % H;
+  if (threadIdx.x < 32) {
     float mx = -INFINITY;
-    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_lse[((size_t)bq * splits + s) * H + h]);
-    float acc = 0.f, wsum = 0.f;
-    if (mx > -INFINITY) {
-      for (int s = 0; s < splits; ++s) {
-        const float ls = part_lse[((size_t)bq * splits + s) * H + h];
-        if (ls == -INFINITY) continue;
-        const float w = exp2f((ls - mx) * LOG2E);
-        wsum += w;
-        acc = fmaf(w, part_o[(((size_t)bq * splits + s) * H + h) * D + (hd % D)], acc);
-      }
+    for (int s = threadIdx.x; s < splits; s += 32) mx = fmaxf(mx, part_lse[((size_t)bq * splits + s) * H + h]);
+    mx = warp_max(mx);
+    float sum = 0.f;
+    for (int s = threadIdx.x; s < splits; s += 32) {
+      const float ls = part_lse[((size_t)bq * splits + s) * H + h];
+      const float wgt = (mx == -INFINITY || ls == -INFINITY) ? 0.f : exp2f((ls - mx) * LOG2E);
+      s_w[s] = wgt;
+      sum += wgt;
     }
-    out[(size_t)bq * H * D + hd] = (uint16_t)f_to_bf16_bits(wsum > 0.f ? acc / wsum : 0.f);
-    if (lse && hd % D == 0) lse[(size_t)bq * H + h] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
+    sum = warp_sum(sum);
+    if (threadIdx.x == 0) { s_tot[0] = sum; s_tot[1] = mx; }
   }
+  __syncthreads();
+  const float sum = s_tot[0];
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  for (int d4 = threadIdx.x * 4; d4 < D; d4 += blockDim.x * 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int s = 0; s < splits; ++s) {
+      const float wgt = s_w[s];
+      if (wgt == 0.f) continue;
+      const float4 v = *reinterpret_cast<const float4*>(part_o + (((size_t)bq * splits + s) * H + h) * D + d4);
+      acc.x = fmaf(wgt, v.x, acc.x); acc.y = fmaf(wgt, v.y, acc.y);
+      acc.z = fmaf(wgt, v.z, acc.z); acc.w = fmaf(wgt, v.w, acc.w);
+    }
+    uint2 o2;
+    o2.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    o2.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(out + ((size_t)bq * H + h) * D + d4) = o2;
+  }
+  if (lse && threadIdx.x == 0) lse[(size_t)bq * H + h] = sum > 0.f ? s_tot[1] + logf(sum) : -INFINITY;
 }
 
 struct AttnPlan {
@@ -353,8 +399,9 @@ static AttnPlan plan_attn(const csa_attn_args* a, int hca) {
   const long long n_win = (a->win_kv && a->Wn > 0) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
   const long long chunks = (n_sel + n_win + AT_KC - 1) / AT_KC;
   const long long rows = (long long)a->B * a->Nq;
-  long long splits = rows >= 148 ? 1 : (296 + rows - 1) / rows;
+  long long splits = rows >= 148 ? 1 : 148 / rows;
   if (splits > chunks) splits = chunks;
+  if (splits > MERGE_MAX_SPLITS) splits = MERGE_MAX_SPLITS;
   if (splits < 1) splits = 1;
   p.cps = (int)((chunks + splits - 1) / splits);
   if (p.cps < 1) p.cps = 1;
@@ -387,7 +434,9 @@ static csa_status validate_attn(const csa_attn_args* a, int hca) {
 template <int D, int DS>
 static csa_status launch_attn(const AttnParams& P, int units, cudaStream_t st) {
   constexpr int HG = AT_WARPS / DS;
-  const size_t smem = (size_t)HG * 16 * D * 2 + (size_t)AT_KC * D * 2 + (DS > 1 ? (size_t)HG * DS * 16 * AT_KC * 4 : 0);
+  constexpr int RAW = (D - (D == 512 ? 64 : 32)) / 2 + 16 + (D == 512 ? 64 : 32) * 2;
+  const size_t smem = (size_t)HG * 16 * D * 2 + (size_t)AT_KC * D * 2 + (DS > 1 ? (size_t)HG * DS * 16 * AT_KC * 4 : 0) +
+                      (size_t)AT_KC * RAW;
   static std::atomic<unsigned> attr_done{0};
   set_smem_once((const void*)attn_kernel<D, DS>, (int)smem, attr_done);
   attn_kernel<D, DS><<<units, AT_WARPS * 32, smem, st>>>(P);
@@ -422,7 +471,8 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
   else
     s = launch_attn<128, 8>(P, units, st);
   if (s != CSA_OK || p.splits == 1) return s;
-  attn_merge_kernel<<<(unsigned)rows, 256, 0, st>>>(P.part_o, P.part_lse, p.splits, a->H, a->d, (uint16_t*)a->out, a->lse);
+  attn_merge_kernel<<<(unsigned)(rows * a->H), 128, 0, st>>>(P.part_o, P.part_lse, p.splits, a->H, a->d,
+                                                               (uint16_t*)a->out, a->lse);
   return launch_status();
 }
 

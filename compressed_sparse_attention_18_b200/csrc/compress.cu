@@ -138,27 +138,49 @@ __global__ void __launch_bounds__(256) gemm_bf16_kernel(const uint16_t* __restri
 }
 
 // --------------------------------------------------------------------------------------- pooling
-// One CTA per (sequence, group of ENT entries).  Threads walk the d channels: per-channel online
-// softmax over the r slots of (Z + b_pos), weighted sum of C; RoPE on the last d_r channels at the
-// group-start position (angles in double); bf16 round; then k_I = bf16(c · W_IK).
+// One CTA per (sequence, group of POOL_ENT entries).  Threads walk the d channels: per-channel softmax
+// over the r slots of (Z + b_pos), weighted sum of C (all r loads issued together when r <= 8; an
+// online softmax streams longer groups); RoPE on the last d_r channels at the group-start position
+// (angles and rotation in double); bf16 round; then k_I = bf16(c · W_IK) with W_IK staged through
+// shared memory in 128-row tiles.
 constexpr int POOL_ENT = 4;
+constexpr int POOL_KT = 128;   // W_IK rows per shared-memory tile
 
 __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ C, const uint16_t* __restrict__ Z,
                                                    const float* __restrict__ b_pos, int T, int d, int d_r,
                                                    int r, float theta, const int64_t* __restrict__ pos0,
                                                    const uint16_t* __restrict__ W_IK, int d_I,
                                                    uint16_t* __restrict__ c_out, uint16_t* __restrict__ kI_out) {
-  extern __shared__ float pooled[];  // [POOL_ENT][d]
+  extern __shared__ __align__(16) float pooled[];   // [POOL_ENT][d], then the W_IK tile / partial sums
   const int b = blockIdx.y;
   const int n_out = T / r;
   const int e0 = blockIdx.x * POOL_ENT;
   const int ne = min(POOL_ENT, n_out - e0);
   const int d_n = d - d_r;
-  for (int q = 0; q < ne; ++q) {
-    const int e = e0 + q;
-    const size_t tok0 = (size_t)b * T + (size_t)e * r;
-    for (int ch = threadIdx.x; ch < d; ch += blockDim.x) {
-      float m = -INFINITY, l = 0.0f, acc = 0.0f;
+  for (int i = threadIdx.x; i < ne * d; i += blockDim.x) {
+    const int q = i / d, ch = i % d;
+    const size_t tok0 = (size_t)b * T + (size_t)(e0 + q) * r;
+    float res;
+    if (r <= 8) {
+      float a[8], c[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        a[j] = j < r ? bf16_bits_to_f(Z[(tok0 + j) * d + ch]) + b_pos[(size_t)j * d + ch] : -INFINITY;
+        c[j] = j < r ? bf16_bits_to_f(C[(tok0 + j) * d + ch]) : 0.f;
+      }
+      float m = a[0];
+#pragma unroll
+      for (int j = 1; j < 8; ++j) m = fmaxf(m, a[j]);
+      float l = 0.f, acc = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float p = j < r ? __expf(a[j] - m) : 0.f;
+        l += p;
+        acc = fmaf(p, c[j], acc);
+      }
+      res = acc / l;
+    } else {
+      float m = -INFINITY, l = 0.f, acc = 0.f;
       for (int j = 0; j < r; ++j) {
         const float a = bf16_bits_to_f(Z[(tok0 + j) * d + ch]) + b_pos[(size_t)j * d + ch];
         const float c = bf16_bits_to_f(C[(tok0 + j) * d + ch]);
@@ -172,49 +194,64 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
         l += p;
         acc = fmaf(p, c, acc);
       }
-      pooled[q * d + ch] = acc / l;
+      res = acc / l;
     }
+    pooled[q * d + ch] = res;
   }
   __syncthreads();
   const int half = d_r >> 1;
   const long long p0 = pos0 ? pos0[b] : 0;
-  for (int q = 0; q < ne; ++q) {
-    const int e = e0 + q;
-    float* row = pooled + q * d;
-    if (theta != 0.0f) {
-      for (int mm = threadIdx.x; mm < half; mm += blockDim.x) {
-        const double p = (double)(p0 + (long long)e * r);
-        const double inv_freq = pow((double)theta, -2.0 * mm / (double)d_r);
-        double sn, cs;
-        sincos(p * inv_freq, &sn, &cs);
-        const double x1 = row[d_n + mm], x2 = row[d_n + half + mm];
-        row[d_n + mm] = (float)(x1 * cs - x2 * sn);
-        row[d_n + half + mm] = (float)(x1 * sn + x2 * cs);
-      }
+  if (theta != 0.0f) {
+    for (int i = threadIdx.x; i < ne * half; i += blockDim.x) {
+      const int q = i / half, mm = i % half;
+      float* row = pooled + q * d;
+      const double p = (double)(p0 + (long long)(e0 + q) * r);
+      const double inv_freq = pow((double)theta, -2.0 * mm / (double)d_r);
+      double sn, cs;
+      sincos(p * inv_freq, &sn, &cs);
+      const double x1 = row[d_n + mm], x2 = row[d_n + half + mm];
+      row[d_n + mm] = (float)(x1 * cs - x2 * sn);
+      row[d_n + half + mm] = (float)(x1 * sn + x2 * cs);
     }
+    __syncthreads();
   }
-  __syncthreads();
-  for (int q = 0; q < ne; ++q) {
-    const int e = e0 + q;
-    float* row = pooled + q * d;
-    for (int ch = threadIdx.x; ch < d; ch += blockDim.x) {
-      const uint32_t bits = f_to_bf16_bits(row[ch]);
-      c_out[((size_t)b * n_out + e) * d + ch] = (uint16_t)bits;
-      row[ch] = bf16_bits_to_f(bits);
-    }
+  for (int i = threadIdx.x; i < ne * d; i += blockDim.x) {
+    const int q = i / d, ch = i % d;
+    const uint32_t bits = f_to_bf16_bits(pooled[i]);
+    c_out[((size_t)b * n_out + e0 + q) * d + ch] = (uint16_t)bits;
+    pooled[i] = bf16_bits_to_f(bits);
   }
   if (W_IK == nullptr) return;
   __syncthreads();
-  for (int j = threadIdx.x; j < d_I; j += blockDim.x) {
-    float acc[POOL_ENT];
+  // k_I: thread (j, part) accumulates output j over the channels part, part + S, ... of each tile
+  uint16_t* wt = reinterpret_cast<uint16_t*>(pooled + POOL_ENT * d);   // [POOL_KT][d_I]
+  const int S = blockDim.x / d_I;               // d_I divides 256 (64 or 128)
+  const int j = threadIdx.x % d_I, part = threadIdx.x / d_I;
+  float acc[POOL_ENT];
 #pragma unroll
-    for (int q = 0; q < POOL_ENT; ++q) acc[q] = 0.0f;
-    for (int ch = 0; ch < d; ++ch) {
-      const float wv = bf16_bits_to_f(W_IK[(size_t)ch * d_I + j]);
+  for (int q = 0; q < POOL_ENT; ++q) acc[q] = 0.f;
+  for (int ch0 = 0; ch0 < d; ch0 += POOL_KT) {
+    const int rows = min(POOL_KT, d - ch0);
+    const int n16 = rows * d_I / 8;
+    for (int i = threadIdx.x; i < n16; i += blockDim.x)
+      reinterpret_cast<uint4*>(wt)[i] = reinterpret_cast<const uint4*>(W_IK + (size_t)ch0 * d_I)[i];
+    __syncthreads();
+    for (int ch = part; ch < rows; ch += S) {
+      const float wv = bf16_bits_to_f(wt[ch * d_I + j]);
 #pragma unroll
-      for (int q = 0; q < POOL_ENT; ++q) acc[q] = fmaf(pooled[q * d + ch], wv, acc[q]);
+      for (int q = 0; q < POOL_ENT; ++q) acc[q] = fmaf(pooled[q * d + ch0 + ch], wv, acc[q]);
     }
-    for (int q = 0; q < ne; ++q) kI_out[((size_t)b * n_out + e0 + q) * d_I + j] = (uint16_t)f_to_bf16_bits(acc[q]);
+    __syncthreads();
+  }
+  float* red = reinterpret_cast<float*>(wt);    // [S][POOL_ENT][d_I] partial sums
+#pragma unroll
+  for (int q = 0; q < POOL_ENT; ++q) red[(part * POOL_ENT + q) * d_I + j] = acc[q];
+  __syncthreads();
+  for (int i = threadIdx.x; i < ne * d_I; i += blockDim.x) {
+    const int q = i / d_I, jj = i % d_I;
+    float v = 0.f;
+    for (int pp = 0; pp < S; ++pp) v += red[(pp * POOL_ENT + q) * d_I + jj];
+    kI_out[((size_t)b * n_out + e0 + q) * d_I + jj] = (uint16_t)f_to_bf16_bits(v);
   }
 }
 
@@ -247,7 +284,8 @@ extern "C" csa_status csa_compress(const csa_compress_args* a, void* stream) {
   }
   const int n_out = a->T / a->ratio;
   if (a->B == 0 || n_out == 0) return CSA_OK;
-  const size_t smem = (size_t)POOL_ENT * a->d * sizeof(float);
+  if (a->W_IK) CSA_SUPPORTED(a->d_index == 64 || a->d_index == 128);
+  const size_t smem = (size_t)POOL_ENT * a->d * sizeof(float) + (a->W_IK ? (size_t)POOL_KT * a->d_index * 2 : 0);
   CSA_SUPPORTED(smem <= 48 * 1024);
   dim3 grid((n_out + POOL_ENT - 1) / POOL_ENT, a->B);
   pool_kernel<<<grid, 256, smem, st>>>((const uint16_t*)a->C, (const uint16_t*)a->Z, a->b_pos, a->T, a->d,

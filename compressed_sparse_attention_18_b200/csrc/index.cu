@@ -19,8 +19,7 @@ namespace csa {
 
 constexpr int IDX_HEADS = 8;           // MMA N: indexer heads, padded with zero heads
 constexpr int IDX_WARPS = 4;
-constexpr int IDX_TILES_PER_WARP = 8;  // 16-key tiles per warp per CTA
-constexpr int IDX_KEYS_PER_CTA = IDX_WARPS * IDX_TILES_PER_WARP * 16;
+constexpr int IDX_TARGET_CTAS = 148 * 4;  // about one wave of resident CTAs
 constexpr int IDX_QT = 32;             // max queries per CTA (query fragments staged in shared memory)
 constexpr int TOPK_THREADS = 1024;
 constexpr int TOPK_CHUNK = 32768;      // max row length held in shared memory (implicit ids)
@@ -102,7 +101,7 @@ __device__ __forceinline__ void convert_key(const KeyRow<DI>& raw, uint32_t sc, 
   for (int i = 0; i < KeyRow<DI>::BYTES; ++i) a[i] = hmul2_bits(e2m1x2_to_h2(raw.w[i >> 2] >> ((i & 3) * 8)), s2);
 }
 
-// Grid: x = key chunk (IDX_KEYS_PER_CTA keys or candidates), y = query tile, z = sequence.
+// Grid: x = key range (4 warps x tpw tiles of 16 keys or candidates), y = query tile, z = sequence.
 // cand != nullptr: Reindex mode, one query per CTA, keys gathered by id.  Dynamic shared memory holds
 // the tile's query fragments [qt][IDX_HEADS][DI] f16.
 template <int DI>
@@ -110,7 +109,7 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
     const uint16_t* __restrict__ q_I, const float* __restrict__ w, int H_I, float g_q, float gg, int Nq, int qt,
     const uint8_t* __restrict__ k_codes, const uint8_t* __restrict__ k_scales, int n_max,
     const int32_t* __restrict__ n_c, const int64_t* __restrict__ q_pos, int ratio,
-    const int32_t* __restrict__ cand, int n_cand, float* __restrict__ scores, long long ld) {
+    const int32_t* __restrict__ cand, int n_cand, float* __restrict__ scores, long long ld, int tpw) {
   constexpr int STEPS = DI / 16;
   constexpr int BREGS = DI / 8;           // f16x2 registers of one head slice per thread
   constexpr int S_PAD = ((DI / 32) + 3) & ~3;
@@ -126,7 +125,8 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
   const int ncb = min(n_c[b], n_max);   // entries beyond the cache capacity do not exist
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int chunk0 = blockIdx.x * IDX_KEYS_PER_CTA;
+  const int keys_per_cta = IDX_WARPS * tpw * 16;
+  const int chunk0 = blockIdx.x * keys_per_cta;
   const int n_cols = cand ? n_cand : n_max;
   if (chunk0 >= n_cols) return;
 
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
   __syncthreads();
   if (!cand && chunk0 >= max_vis) return;
 
-  const int chunk_end = min(n_cols, chunk0 + IDX_KEYS_PER_CTA);
+  const int chunk_end = min(n_cols, chunk0 + keys_per_cta);
   const int col_end = cand ? chunk_end : min(chunk_end, max_vis);
   const uint8_t* codes_b = k_codes + (size_t)b * n_max * (DI / 2);
   const uint8_t* scales_b = k_scales + (size_t)b * n_max * S_PAD;
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
     }
   };
 
-  const int first_col = chunk0 + warp * IDX_TILES_PER_WARP * 16;
+  const int first_col = chunk0 + warp * tpw * 16;
   int key[2][2];
   bool kval[2][2];
   KeyRow<DI> raw[2][2];
@@ -173,11 +173,11 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
     load_key<DI>(codes_b, scales_b, key[0][h], kval[0][h], t, raw[0][h], sc[0][h]);
   }
 #pragma unroll 2
-  for (int tile = 0; tile < IDX_TILES_PER_WARP; ++tile) {
+  for (int tile = 0; tile < tpw; ++tile) {
     const int cur = tile & 1;
     const int col0 = first_col + tile * 16;
     if (col0 >= col_end) break;
-    if (tile + 1 < IDX_TILES_PER_WARP) {
+    if (tile + 1 < tpw) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         key_of(col0 + 16 + g + 8 * h, key[cur ^ 1][h], kval[cur ^ 1][h]);
@@ -245,10 +245,15 @@ __device__ uint32_t radix_threshold(TopkSmem& sm, int n, uint32_t R, KeyF key, F
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x) sm.hist[i] = 0;
     __syncthreads();
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
-      if (!filt(j)) continue;
-      const uint32_t k = key(j);
-      if ((k & mask) == prefix) atomicAdd(&sm.hist[(k >> shift) & 255u], 1u);
+    // warp-aggregated increments: lanes hitting the same bin add once (scores cluster in few bins)
+    for (int j0 = 0; j0 < n; j0 += blockDim.x) {
+      const int j = j0 + threadIdx.x;
+      bool ok = j < n && filt(j);
+      const uint32_t k = ok ? key(j) : 0u;
+      ok = ok && (k & mask) == prefix;
+      const uint32_t dig = ok ? ((k >> shift) & 255u) : 256u + (threadIdx.x & 31);
+      const unsigned peers = __match_any_sync(0xffffffffu, dig);
+      if (ok && (int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&sm.hist[dig], (uint32_t)__popc(peers));
     }
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -349,12 +354,25 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(TopkRowArgs A) {
   const float* src = A.in_scores + row * A.in_ld + col0;
   const int32_t* isrc = A.in_ids ? A.in_ids + row * A.in_ld + col0 : nullptr;
   uint32_t nvalid_loc = 0;
-  for (int j = threadIdx.x; j < len; j += blockDim.x) {
-    const float s = src[j];
-    const bool ok = s > -INFINITY && (!isrc || isrc[j] >= 0);
-    keys[j] = ok ? float_order_key(s) : 0u;   // 0 marks "not a candidate"
-    if (isrc) ids[j] = isrc[j];
-    nvalid_loc += ok;
+  constexpr int U = 8;   // independent loads in flight per thread
+  for (int j0 = threadIdx.x; j0 < len; j0 += U * blockDim.x) {
+    float v[U];
+    int32_t id[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * blockDim.x;
+      v[u] = j < len ? src[j] : -INFINITY;
+      id[u] = (isrc && j < len) ? isrc[j] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * blockDim.x;
+      if (j >= len) continue;
+      const bool ok = v[u] > -INFINITY && id[u] >= 0;
+      keys[j] = ok ? float_order_key(v[u]) : 0u;   // 0 marks "not a candidate"
+      if (isrc) ids[j] = id[u];
+      nvalid_loc += ok;
+    }
   }
   uint32_t nvalid;
   block_exclusive_scan(sm, nvalid_loc, &nvalid);
@@ -519,8 +537,15 @@ static csa_status validate_index(const csa_index_args* a, bool need_select) {
 static csa_status run_scores(const csa_index_args* a, float* scores, long long ld, cudaStream_t st) {
   const int n_cols = a->cand ? a->n_cand : a->n_max;
   const int qt = a->cand ? 1 : (a->Nq < IDX_QT ? a->Nq : IDX_QT);
-  dim3 grid((n_cols + IDX_KEYS_PER_CTA - 1) / IDX_KEYS_PER_CTA, a->cand ? a->Nq : (a->Nq + qt - 1) / qt, a->B);
-  if (grid.x == 0) return CSA_OK;
+  const long long qtiles = (long long)a->B * (a->cand ? a->Nq : (a->Nq + qt - 1) / qt);
+  // key range per CTA: enough CTAs for about one wave, at least one 16-key tile per warp
+  long long per_seq = IDX_TARGET_CTAS / (qtiles > 0 ? qtiles : 1);
+  if (per_seq < 1) per_seq = 1;
+  long long tpw = (n_cols + IDX_WARPS * 16 * per_seq - 1) / (IDX_WARPS * 16 * per_seq);
+  if (tpw < 1) tpw = 1;
+  const long long kpc = IDX_WARPS * 16 * tpw;
+  dim3 grid((unsigned)((n_cols + kpc - 1) / kpc), a->cand ? a->Nq : (a->Nq + qt - 1) / qt, a->B);
+  if (n_cols == 0) return CSA_OK;
   const int smem = qt * IDX_HEADS * a->d_I * 2;
   const float gg = a->g_q * a->g_k;
   static std::atomic<unsigned> attr128{0}, attr64{0};
@@ -528,12 +553,12 @@ static csa_status run_scores(const csa_index_args* a, float* scores, long long l
     set_smem_once((const void*)index_score_kernel<128>, IDX_QT * IDX_HEADS * 128 * 2, attr128);
     index_score_kernel<128><<<grid, IDX_WARPS * 32, smem, st>>>(
         (const uint16_t*)a->q_I, a->w, a->H_I, a->g_q, gg, a->Nq, qt, a->k_codes, a->k_scales, a->n_max, a->n_c,
-        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld);
+        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld, (int)tpw);
   } else {
     set_smem_once((const void*)index_score_kernel<64>, IDX_QT * IDX_HEADS * 64 * 2, attr64);
     index_score_kernel<64><<<grid, IDX_WARPS * 32, smem, st>>>(
         (const uint16_t*)a->q_I, a->w, a->H_I, a->g_q, gg, a->Nq, qt, a->k_codes, a->k_scales, a->n_max, a->n_c,
-        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld);
+        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld, (int)tpw);
   }
   return launch_status();
 }

@@ -33,11 +33,24 @@ def test_decode_cfg2_full_size(cuda_lib):
     layer.win.copy_(inp["win_kv"])
     out, lse, idx = layer.step(inp["C"], inp["Z"], inp["b_pos"], inp["W_IK"], inp["q"], inp["q_I"], inp["w"])
     torch.cuda.synchronize()
-    # property at full size: every planted needle is selected, in every sequence
+    # property at full size, every sequence: a planted needle whose oracle score clears the kernel's
+    # k-th score (with the boundary tolerance) is selected.  (A sequence whose head weights are all
+    # <= 0 gives every key a score <= 0, so needles are not high-scoring there by construction.)
+    gpu_scores = layer.scores.cpu().numpy()
+    planted_selected = 0
     for b in range(s.B):
         sel = set(idx[b, 0].tolist())
-        assert set(inp["needle_pos"][b].tolist()) <= sel, f"needle missed in b={b}"
-        assert len(sel) == s.k
+        assert len(sel) == s.k and -1 not in sel
+        kth = np.partition(gpu_scores[b], -s.k)[-s.k]
+        pos = inp["needle_pos"][b].cpu().numpy()
+        codes, scales, _ = O.pack_fp4(f64(inp["kI_src"][b, pos]), 0, 1.0)
+        ns, _ = O.index_scores(f64(inp["q_I"][b, 0])[None], f64(inp["w"][b, 0])[None], 1.0, codes, scales, 1.0,
+                               [10 ** 9], len(pos), s.r)
+        for i, sc in zip(pos, ns[0]):
+            if sc > kth + 1e-3 * abs(kth):
+                assert int(i) in sel, f"needle {i} (score {sc} > k-th {kth}) missed in b={b}"
+                planted_selected += 1
+    assert planted_selected >= 8 * s.B // 2
     for b in (0, 17, 31):
         # compressor + pack of the new entry
         c_ref = O.compress_pool(f64(inp["C"][b]), f64(inp["Z"][b]), f64(inp["b_pos"]), s.r, s.d_r, 10000.0,
