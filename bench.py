@@ -316,7 +316,7 @@ def run_ours(args, rank, world):
         "e2e": e2e,
     }
     if world == 1 or rank == 0:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_sample) if world == 1 else None
+        line["cpu_baseline"] = cpu_baseline(args.cpu_sample) if (world == 1 and args.cpu_sample > 0) else None
     print(json.dumps(line), flush=True)
 
 

@@ -162,6 +162,15 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
   };
 
   const int first_col = chunk0 + warp * tpw * 16;
+  uint32_t bq0[BREGS];
+  {
+    const uint4* bq = reinterpret_cast<const uint4*>(s_q + (size_t)g * DI + t * (DI / 4));
+#pragma unroll
+    for (int i = 0; i < BREGS / 4; ++i) {
+      const uint4 v = bq[i];
+      bq0[4 * i] = v.x; bq0[4 * i + 1] = v.y; bq0[4 * i + 2] = v.z; bq0[4 * i + 3] = v.w;
+    }
+  }
   int key[2][2];
   bool kval[2][2];
   KeyRow<DI> raw[2][2];
@@ -190,12 +199,18 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
 
     for (int qq = 0; qq < nq; ++qq) {
       // B fragment: head g, elements [t*DI/4 + 4s, +4) for k16 step s -> one contiguous slice
-      const uint4* bq = reinterpret_cast<const uint4*>(s_q + ((size_t)qq * IDX_HEADS + g) * DI + t * (DI / 4));
+      // (decode: one query, fragments loaded once before the tile loop)
       uint32_t bfr[BREGS];
+      if (nq == 1) {
 #pragma unroll
-      for (int i = 0; i < BREGS / 4; ++i) {
-        const uint4 v = bq[i];
-        bfr[4 * i] = v.x; bfr[4 * i + 1] = v.y; bfr[4 * i + 2] = v.z; bfr[4 * i + 3] = v.w;
+        for (int i = 0; i < BREGS; ++i) bfr[i] = bq0[i];
+      } else {
+        const uint4* bq = reinterpret_cast<const uint4*>(s_q + ((size_t)qq * IDX_HEADS + g) * DI + t * (DI / 4));
+#pragma unroll
+        for (int i = 0; i < BREGS / 4; ++i) {
+          const uint4 v = bq[i];
+          bfr[4 * i] = v.x; bfr[4 * i + 1] = v.y; bfr[4 * i + 2] = v.z; bfr[4 * i + 3] = v.w;
+        }
       }
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -232,6 +247,7 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
 
 struct TopkSmem {
   uint32_t hist[256];
+  uint32_t whist[TOPK_THREADS / 32][256];   // per-warp histograms: contention only inside a warp
   uint32_t scan[TOPK_THREADS / 32];
   uint32_t bcast[4];
   uint32_t counter;
@@ -243,17 +259,21 @@ template <class KeyF, class FiltF>
 __device__ uint32_t radix_threshold(TopkSmem& sm, int n, uint32_t R, KeyF key, FiltF filt, uint32_t* n_above) {
   uint32_t prefix = 0, mask = 0, rem = R;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) sm.hist[i] = 0;
+    const int nw = blockDim.x >> 5, wid = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < nw * 256; i += blockDim.x) (&sm.whist[0][0])[i] = 0;
     __syncthreads();
-    // warp-aggregated increments: lanes hitting the same bin add once (scores cluster in few bins)
-    for (int j0 = 0; j0 < n; j0 += blockDim.x) {
-      const int j = j0 + threadIdx.x;
-      bool ok = j < n && filt(j);
-      const uint32_t k = ok ? key(j) : 0u;
-      ok = ok && (k & mask) == prefix;
-      const uint32_t dig = ok ? ((k >> shift) & 255u) : 256u + (threadIdx.x & 31);
-      const unsigned peers = __match_any_sync(0xffffffffu, dig);
-      if (ok && (int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&sm.hist[dig], (uint32_t)__popc(peers));
+    // per-warp histograms: scores cluster in a few bins, so a block-wide histogram serialises
+    uint32_t* wh = sm.whist[wid];
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+      if (!filt(j)) continue;
+      const uint32_t k = key(j);
+      if ((k & mask) == prefix) atomicAdd(&wh[(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+      uint32_t c = 0;
+      for (int w = 0; w < nw; ++w) c += sm.whist[w][i];
+      sm.hist[i] = c;
     }
     __syncthreads();
     if (threadIdx.x < 32) {
