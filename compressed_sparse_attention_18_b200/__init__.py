@@ -16,13 +16,14 @@ LIB_PATH = os.path.join(_PKG, "libcsa_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m compressed_sparse_attention_18_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python compressed_sparse_attention_18_b200/build.py` "
         "(nvcc, sm_100a).  There is no CPU fallback.")
 _lib = ctypes.CDLL(LIB_PATH)
 
 ENTRY_POINTS = ("csa_status_string", "csa_version", "csa_last_cuda_error", "csa_compress", "csa_pack_fp4",
                 "csa_index_topk_workspace_size", "csa_index_topk", "csa_index_scores", "csa_topk_workspace_size",
-                "csa_topk", "csa_attn_workspace_size", "csa_sparse_attn", "hca_dense_attn")
+                "csa_topk", "csa_attn_workspace_size", "csa_sparse_attn", "hca_dense_attn",
+                "csa_index_topk_noalloc")
 
 _u32, _i32, _f32, _vp = ctypes.c_uint32, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p
 
@@ -67,6 +68,8 @@ _lib.csa_index_topk_workspace_size.restype = ctypes.c_size_t
 _lib.csa_index_topk_workspace_size.argtypes = [ctypes.POINTER(IndexArgs)]
 _lib.csa_index_topk.restype = ctypes.c_int
 _lib.csa_index_topk.argtypes = [ctypes.POINTER(IndexArgs), _vp, ctypes.c_size_t, _vp]
+_lib.csa_index_topk_noalloc.restype = ctypes.c_int
+_lib.csa_index_topk_noalloc.argtypes = [ctypes.POINTER(IndexArgs), _vp]
 _lib.csa_index_scores.restype = ctypes.c_int
 _lib.csa_index_scores.argtypes = [ctypes.POINTER(IndexArgs), _vp, ctypes.c_int64, _vp]
 _lib.csa_topk_workspace_size.restype = ctypes.c_size_t

@@ -665,9 +665,58 @@ static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const 
   return CSA_OK;
 }
 
+// ------------------------------------------------------------------ allocation-free variant
+// Scratch for csa_index_topk_noalloc: a file-scope device array, present in every GPU that loads
+// this library for the life of the process.  Host code cannot use the symbol as a pointer (it is a
+// host-side stand-in); its device address is looked up once per device with that device current.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[CSA_NOALLOC_SCRATCH_BYTES];
+constexpr int NOALLOC_MAX_DEVICES = 64;
+static std::atomic<uintptr_t> g_noalloc_ptr[NOALLOC_MAX_DEVICES];
+
+static csa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) { set_last_cuda_error(e); return CSA_ERR_CUDA; }
+  if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return CSA_ERR_UNSUPPORTED;
+  uintptr_t p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p == 0) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || ptr == nullptr) {
+      set_last_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+      return CSA_ERR_CUDA;
+    }
+    p = (uintptr_t)ptr;
+    g_noalloc_ptr[dev].store(p, std::memory_order_release);
+  }
+  *out = (void*)p;
+  return CSA_OK;
+}
+
 }  // namespace csa
 
 using namespace csa;
+
+extern "C" csa_status csa_index_topk_noalloc(const csa_index_args* a, void* stream) {
+  csa_status v = validate_index(a, true);
+  if (v != CSA_OK) return v;
+  v = validate_index(a, false);
+  if (v != CSA_OK) return v;
+  const IndexPlan p = plan_index(a);
+  if (p.rows == 0) return CSA_OK;
+  if (p.total > CSA_NOALLOC_SCRATCH_BYTES) return CSA_ERR_WORKSPACE;   // before any CUDA call
+  void* ws = nullptr;
+  v = noalloc_scratch(&ws);
+  if (v != CSA_OK) return v;
+  // Nothing in the scratch needs to start at zero: every byte a call reads was written earlier in
+  // the same call (scores of the visible columns, the tournament's k slots per segment, pool buffers).
+  cudaStream_t st = (cudaStream_t)stream;
+  uint8_t* w8 = (uint8_t*)ws;
+  float* scores = (float*)(w8 + p.off_scores);
+  csa_status s = run_scores(a, scores, p.n_cols, st);
+  if (s != CSA_OK) return s;
+  return run_select(a, p, scores, p.n_cols, w8, st);
+}
 
 extern "C" csa_status csa_index_scores(const csa_index_args* a, float* scores, int64_t ld, void* stream) {
   csa_status v = validate_index(a, false);

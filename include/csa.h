@@ -168,6 +168,21 @@ size_t csa_topk_workspace_size(const csa_index_args* args);
 csa_status csa_topk(const csa_index_args* args, const float* scores, int64_t ld, void* ws, size_t ws_bytes,
                     void* stream);
 
+/* csa_index_topk_noalloc — csa_index_topk for callers that cannot allocate device memory: code that
+ * runs where cudaMalloc is unavailable or forbidden (inside an allocator-free runtime or plugin
+ * host, an embedded service with a fixed memory budget, or a caller that must not synchronise the
+ * device the way cudaMalloc/cudaFree can).  The paper has no counterpart; this is a deployment
+ * convenience of this library.  Same arguments, same results as csa_index_topk, no ws argument.
+ * Its scratch is a static device array of CSA_NOALLOC_SCRATCH_BYTES that every GPU loading the
+ * library holds until the process exits.  Problems needing more scratch than that (see
+ * csa_index_topk_workspace_size) return CSA_ERR_WORKSPACE before any CUDA call.
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.  All calls share the one
+ * array: calls that overlap on the GPU (other streams, other host threads) race and must be
+ * serialised by the caller.  It calls no cudaMalloc / cudaFree. */
+#define CSA_NOALLOC_SCRATCH_BYTES (8u << 20)
+csa_status csa_index_topk_noalloc(const csa_index_args* args, void* stream);
+
 /* ------------------------------------------------------------------------------------------------
  * csa_sparse_attn / hca_dense_attn — softmax attention over compressed entries plus the sliding
  * window ([V4 blog] Fig. 3 for CSA: the selected entries; Fig. 4 for HCA: every visible entry).
