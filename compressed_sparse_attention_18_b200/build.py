@@ -1,6 +1,8 @@
 """Build the CUDA library (libcsa_b200.so) in-tree for sm_100a with nvcc.
 
-    python -m compressed_sparse_attention_18_b200.build
+    python compressed_sparse_attention_18_b200/build.py [-v]
+
+(Run it as a script: importing the package itself loads the library.)
 """
 from __future__ import annotations
 

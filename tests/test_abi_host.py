@@ -12,8 +12,8 @@ HEADER = os.path.join(ROOT, "include", "csa.h")
 
 @pytest.fixture(scope="module")
 def csa():
-    from compressed_sparse_attention_18_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._build_module().build()
     import compressed_sparse_attention_18_b200 as m
     return m
 
