@@ -23,16 +23,21 @@ _lib = ctypes.CDLL(LIB_PATH)
 ENTRY_POINTS = ("csa_status_string", "csa_version", "csa_last_cuda_error", "csa_compress", "csa_pack_fp4",
                 "csa_index_topk_workspace_size", "csa_index_topk", "csa_index_scores", "csa_topk_workspace_size",
                 "csa_topk", "csa_attn_workspace_size", "csa_sparse_attn", "hca_dense_attn",
-                "csa_index_topk_noalloc")
+                "csa_index_topk_noalloc", "csa_device_status")
 
 _u32, _i32, _f32, _vp = ctypes.c_uint32, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p
+
+
+class Fp4Cache(ctypes.Structure):
+    _fields_ = [("codes", _vp), ("scales", _vp), ("rope", _vp), ("row0", _vp), ("n_max", _i32),
+                ("global_scale", _f32)]
 
 
 class CompressArgs(ctypes.Structure):
     _fields_ = [("struct_size", _u32), ("B", _i32), ("T", _i32), ("d_model", _i32), ("d", _i32),
                 ("d_rope", _i32), ("d_index", _i32), ("ratio", _i32), ("rope_theta", _f32), ("pos0", _vp),
                 ("x", _vp), ("W_kv", _vp), ("W_g", _vp), ("C", _vp), ("Z", _vp), ("b_pos", _vp),
-                ("W_IK", _vp), ("c_out", _vp), ("kI_out", _vp)]
+                ("W_IK", _vp), ("c_out", _vp), ("kI_out", _vp), ("kv_pack", Fp4Cache), ("ki_pack", Fp4Cache)]
 
 
 class PackArgs(ctypes.Structure):
@@ -46,7 +51,7 @@ class IndexArgs(ctypes.Structure):
                 ("ratio", _i32), ("k", _i32), ("n_max", _i32), ("g_q", _f32), ("g_k", _f32), ("q_I", _vp),
                 ("w", _vp), ("k_codes", _vp), ("k_scales", _vp), ("n_c", _vp), ("q_pos", _vp),
                 ("cand", _vp), ("n_cand", _i32), ("pool_blocks", _i32), ("pool_block_size", _i32),
-                ("pool_out", _vp), ("idx_out", _vp), ("scores_out", _vp)]
+                ("pool_out", _vp), ("idx_out", _vp), ("scores_out", _vp), ("hist", _vp)]
 
 
 class AttnArgs(ctypes.Structure):
@@ -61,6 +66,8 @@ _lib.csa_status_string.restype = ctypes.c_char_p
 _lib.csa_status_string.argtypes = [ctypes.c_int]
 _lib.csa_version.restype = ctypes.c_int
 _lib.csa_last_cuda_error.restype = ctypes.c_int
+_lib.csa_device_status.restype = ctypes.c_int
+_lib.csa_device_status.argtypes = [_vp]
 for _name, _st in (("csa_compress", CompressArgs), ("csa_pack_fp4", PackArgs)):
     getattr(_lib, _name).restype = ctypes.c_int
     getattr(_lib, _name).argtypes = [ctypes.POINTER(_st), _vp]
@@ -89,6 +96,11 @@ class CSAError(RuntimeError):
 
 def version() -> int:
     return _lib.csa_version()
+
+
+def device_status(stream=None):
+    """Synchronise and raise if a kernel recorded a device-side error (a bounded wait gave up)."""
+    _check(_lib.csa_device_status(_stream(stream)), "device status")
 
 
 def _check(status: int, what: str):
@@ -124,10 +136,18 @@ def _ws(nbytes: int, device, ws=None):
 
 # ------------------------------------------------------------------------------------------- API
 
+def _fp4_target(cache, row0):
+    if cache is None:
+        return Fp4Cache()
+    return Fp4Cache(_ptr(cache.codes), _ptr(cache.scales), _ptr(cache.rope) if cache.d_rope else None, _ptr(row0),
+                    cache.n_max, cache.g)
+
+
 def compress(*, b_pos, ratio, d_rope=0, rope_theta=0.0, pos0=None, x=None, W_kv=None, W_g=None, C=None, Z=None,
-             W_IK=None, c_out=None, kI_out=None, stream=None):
+             W_IK=None, c_out=None, kI_out=None, kv_cache=None, ki_cache=None, row0=None, stream=None):
     """Compressor.  Projection mode (x [B,T,d_m], W_kv/W_g [d_m,d]) fills C, Z [B,T,d]; pooling mode
-    reads C, Z.  Returns (c [B,T//r,d], k_I [B,T//r,d_I] or None, C, Z)."""
+    reads C, Z.  kv_cache / ki_cache (PackedCache, rows row0[b] + i) also receive the FP4-packed entries
+    and indexer keys from the same launch.  Returns (c [B,T//r,d], k_I [B,T//r,d_I] or None, C, Z)."""
     if x is not None:
         B, T, dm = x.shape
         d = W_kv.shape[1]
@@ -146,7 +166,8 @@ def compress(*, b_pos, ratio, d_rope=0, rope_theta=0.0, pos0=None, x=None, W_kv=
         kI_out = torch.empty((B, n, dI), dtype=torch.bfloat16, device=C.device)
     a = CompressArgs(ctypes.sizeof(CompressArgs), B, T, dm, d, d_rope, dI, ratio, rope_theta, _ptr(pos0),
                      _ptr(x), _ptr(W_kv), _ptr(W_g), _ptr(C), _ptr(Z), _ptr(b_pos), _ptr(W_IK), _ptr(c_out),
-                     _ptr(kI_out) if W_IK is not None else None)
+                     _ptr(kI_out) if W_IK is not None else None, _fp4_target(kv_cache, row0),
+                     _fp4_target(ki_cache, row0))
     _check(_lib.csa_compress(ctypes.byref(a), _stream(stream)), "csa_compress")
     return c_out, (kI_out if W_IK is not None else None), C, Z
 
@@ -202,16 +223,19 @@ def index_topk(q_I, w, kcache: PackedCache, n_c, q_pos, *, ratio, k, g_q=1.0, ca
     return idx_out, scores_out, pool_out
 
 
-def index_scores(q_I, w, kcache: PackedCache, n_c, q_pos, scores, *, ratio, g_q=1.0, cand=None, stream=None):
-    """Lightning-indexer scores only, into scores [B*Nq, ld] fp32 (see csa_index_scores)."""
+def index_scores(q_I, w, kcache: PackedCache, n_c, q_pos, scores, *, ratio, g_q=1.0, cand=None, hist=None,
+                 stream=None):
+    """Lightning-indexer scores only, into scores [B*Nq, ld] fp32 (see csa_index_scores); hist
+    ([B*Nq, 4096] uint32 as int32, optional) receives the score histogram for topk()."""
     a = _index_args(q_I, w, kcache, n_c, q_pos, ratio, 1, g_q, cand, 0, 8, None, None, None)
+    a.hist = _ptr(hist)
     _check(_lib.csa_index_scores(ctypes.byref(a), _ptr(scores), scores.shape[-1], _stream(stream)),
            "csa_index_scores")
     return scores
 
 
 def topk(scores, kcache: PackedCache, n_c, q_pos, *, B, Nq, ratio, k, cand=None, pool_blocks=0, pool_block_size=8,
-         want_scores=False, idx_out=None, scores_out=None, pool_out=None, ws=None, stream=None):
+         want_scores=False, idx_out=None, scores_out=None, pool_out=None, hist=None, ws=None, stream=None):
     """Top-k (+ hierarchical pool) over a score matrix written by index_scores (see csa_topk)."""
     dev = scores.device
     if idx_out is None:
@@ -223,7 +247,7 @@ def topk(scores, kcache: PackedCache, n_c, q_pos, *, B, Nq, ratio, k, cand=None,
     d_I = 2 * kcache.codes.shape[-1]
     a = IndexArgs(ctypes.sizeof(IndexArgs), B, Nq, 1, d_I, ratio, k, kcache.n_max, 1.0, kcache.g, None, None,
                   None, None, _ptr(n_c), _ptr(q_pos), _ptr(cand), cand.shape[-1] if cand is not None else 0,
-                  pool_blocks, pool_block_size, _ptr(pool_out), _ptr(idx_out), _ptr(scores_out))
+                  pool_blocks, pool_block_size, _ptr(pool_out), _ptr(idx_out), _ptr(scores_out), _ptr(hist))
     nbytes = _lib.csa_topk_workspace_size(ctypes.byref(a))
     wbuf = _ws(nbytes, dev, ws)
     _check(_lib.csa_topk(ctypes.byref(a), _ptr(scores), scores.shape[-1], _ptr(wbuf) if wbuf is not None else None,

@@ -139,24 +139,52 @@ __global__ void __launch_bounds__(256) gemm_bf16_kernel(const uint16_t* __restri
 
 // --------------------------------------------------------------------------------------- pooling
 // One CTA per (sequence, group of POOL_ENT entries).  Threads walk the d channels: per-channel softmax
-// over the r slots of (Z + b_pos), weighted sum of C (all r loads issued together when r <= 8; an
-// online softmax streams longer groups); RoPE on the last d_r channels at the group-start position
-// (angles and rotation in double); bf16 round; then k_I = bf16(c · W_IK) with W_IK staged through
-// shared memory in 128-row tiles.
+// over the r slots of (Z + b_pos), weighted sum of C (all loads of a channel issued together when
+// r <= 8; an online softmax streams longer groups); RoPE on the last d_r channels at the group-start
+// position (angle and rotation in double); bf16 round; k_I = bf16(c · W_IK) with W_IK staged through
+// shared memory in 128-row tiles; optionally the FP4 pack of c and k_I straight into the caches.
 constexpr int POOL_ENT = 4;
 constexpr int POOL_KT = 128;   // W_IK rows per shared-memory tile
 
-__global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ C, const uint16_t* __restrict__ Z,
-                                                   const float* __restrict__ b_pos, int T, int d, int d_r,
-                                                   int r, float theta, const int64_t* __restrict__ pos0,
-                                                   const uint16_t* __restrict__ W_IK, int d_I,
-                                                   uint16_t* __restrict__ c_out, uint16_t* __restrict__ kI_out) {
+struct PoolParams {
+  const uint16_t* C;
+  const uint16_t* Z;
+  const float* b_pos;
+  int T, d, d_r, r;
+  float theta;
+  const int64_t* pos0;
+  const uint16_t* W_IK;
+  int d_I;
+  uint16_t* c_out;
+  uint16_t* kI_out;
+  csa_fp4_cache kv, ki;
+};
+
+__device__ __forceinline__ void pack_row_to_cache(const float* row, int d, int d_r, const csa_fp4_cache& cc, int b,
+                                                  int entry) {
+  const int d_n = d - d_r;
+  const int S = d_n / 32, S_pad = (S + 3) & ~3;
+  const long long dst = (long long)b * cc.n_max + (cc.row0 ? cc.row0[b] : 0) + entry;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int blk = warp; blk < S; blk += nw)
+    pack_block_warp(row[blk * 32 + lane], cc.global_scale, cc.codes + dst * (d_n / 2) + blk * 16,
+                    cc.scales + dst * S_pad + blk);
+  if (threadIdx.x < S_pad - S) cc.scales[dst * S_pad + S + threadIdx.x] = 0;
+  for (int e = threadIdx.x; e < d_r; e += blockDim.x)
+    reinterpret_cast<uint16_t*>(cc.rope)[dst * d_r + e] = (uint16_t)(__float_as_uint(row[d_n + e]) >> 16);
+}
+
+__global__ void __launch_bounds__(256) pool_kernel(PoolParams P) {
   extern __shared__ __align__(16) float pooled[];   // [POOL_ENT][d], then the W_IK tile / partial sums
   const int b = blockIdx.y;
+  const int d = P.d, d_r = P.d_r, r = P.r, T = P.T, d_I = P.d_I;
   const int n_out = T / r;
   const int e0 = blockIdx.x * POOL_ENT;
   const int ne = min(POOL_ENT, n_out - e0);
   const int d_n = d - d_r;
+  const uint16_t* __restrict__ C = P.C;
+  const uint16_t* __restrict__ Z = P.Z;
+  const float* __restrict__ b_pos = P.b_pos;
   for (int i = threadIdx.x; i < ne * d; i += blockDim.x) {
     const int q = i / d, ch = i % d;
     const size_t tok0 = (size_t)b * T + (size_t)(e0 + q) * r;
@@ -200,13 +228,14 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
   }
   __syncthreads();
   const int half = d_r >> 1;
-  const long long p0 = pos0 ? pos0[b] : 0;
-  if (theta != 0.0f) {
+  const long long p0 = P.pos0 ? P.pos0[b] : 0;
+  if (P.theta != 0.0f) {
+    const double l2t = log2((double)P.theta);
     for (int i = threadIdx.x; i < ne * half; i += blockDim.x) {
       const int q = i / half, mm = i % half;
       float* row = pooled + q * d;
       const double p = (double)(p0 + (long long)(e0 + q) * r);
-      const double inv_freq = pow((double)theta, -2.0 * mm / (double)d_r);
+      const double inv_freq = exp2(-2.0 * mm / (double)d_r * l2t);
       double sn, cs;
       sincos(p * inv_freq, &sn, &cs);
       const double x1 = row[d_n + mm], x2 = row[d_n + half + mm];
@@ -218,11 +247,13 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
   for (int i = threadIdx.x; i < ne * d; i += blockDim.x) {
     const int q = i / d, ch = i % d;
     const uint32_t bits = f_to_bf16_bits(pooled[i]);
-    c_out[((size_t)b * n_out + e0 + q) * d + ch] = (uint16_t)bits;
+    if (P.c_out) P.c_out[((size_t)b * n_out + e0 + q) * d + ch] = (uint16_t)bits;
     pooled[i] = bf16_bits_to_f(bits);
   }
-  if (W_IK == nullptr) return;
   __syncthreads();
+  if (P.kv.codes)
+    for (int q = 0; q < ne; ++q) pack_row_to_cache(pooled + q * d, d, d_r, P.kv, b, e0 + q);
+  if (P.W_IK == nullptr) return;
   // k_I: thread (j, part) accumulates output j over the channels part, part + S, ... of each tile
   uint16_t* wt = reinterpret_cast<uint16_t*>(pooled + POOL_ENT * d);   // [POOL_KT][d_I]
   const int S = blockDim.x / d_I;               // d_I divides 256 (64 or 128)
@@ -233,8 +264,20 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
   for (int ch0 = 0; ch0 < d; ch0 += POOL_KT) {
     const int rows = min(POOL_KT, d - ch0);
     const int n16 = rows * d_I / 8;
-    for (int i = threadIdx.x; i < n16; i += blockDim.x)
-      reinterpret_cast<uint4*>(wt)[i] = reinterpret_cast<const uint4*>(W_IK + (size_t)ch0 * d_I)[i];
+    const uint4* wsrc = reinterpret_cast<const uint4*>(P.W_IK + (size_t)ch0 * d_I);
+    for (int i0 = threadIdx.x; i0 < n16; i0 += 8 * blockDim.x) {   // 8 loads in flight per thread
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < n16) v[u] = wsrc[i];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < n16) reinterpret_cast<uint4*>(wt)[i] = v[u];
+      }
+    }
     __syncthreads();
     for (int ch = part; ch < rows; ch += S) {
       const float wv = bf16_bits_to_f(wt[ch * d_I + j]);
@@ -243,15 +286,22 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
     }
     __syncthreads();
   }
-  float* red = reinterpret_cast<float*>(wt);    // [S][POOL_ENT][d_I] partial sums
+  float* red = reinterpret_cast<float*>(wt);    // [S][POOL_ENT][d_I] partial sums, then the k_I rows
 #pragma unroll
   for (int q = 0; q < POOL_ENT; ++q) red[(part * POOL_ENT + q) * d_I + j] = acc[q];
   __syncthreads();
+  float* krow = red + S * POOL_ENT * d_I;        // [POOL_ENT][d_I]
   for (int i = threadIdx.x; i < ne * d_I; i += blockDim.x) {
     const int q = i / d_I, jj = i % d_I;
     float v = 0.f;
     for (int pp = 0; pp < S; ++pp) v += red[(pp * POOL_ENT + q) * d_I + jj];
-    kI_out[((size_t)b * n_out + e0 + q) * d_I + jj] = (uint16_t)f_to_bf16_bits(v);
+    const uint32_t bits = f_to_bf16_bits(v);
+    if (P.kI_out) P.kI_out[((size_t)b * n_out + e0 + q) * d_I + jj] = (uint16_t)bits;
+    krow[q * d_I + jj] = bf16_bits_to_f(bits);
+  }
+  if (P.ki.codes) {
+    __syncthreads();
+    for (int q = 0; q < ne; ++q) pack_row_to_cache(krow + q * d_I, d_I, 0, P.ki, b, e0 + q);
   }
 }
 
@@ -264,7 +314,7 @@ extern "C" csa_status csa_compress(const csa_compress_args* a, void* stream) {
   CSA_REQUIRE(a->B >= 0 && a->T >= 0 && a->d > 0 && a->ratio >= 1 && a->d_rope >= 0 && a->d_rope <= a->d);
   CSA_REQUIRE(a->d_rope % 2 == 0 && a->d_index >= 0);
   CSA_SUPPORTED(a->d % 8 == 0);
-  CSA_REQUIRE(a->C && a->Z && a->b_pos && a->c_out);
+  CSA_REQUIRE(a->C && a->Z && a->b_pos && (a->c_out || a->kv_pack.codes));
   CSA_REQUIRE(a->W_IK == nullptr || (a->kI_out && a->d_index > 0));
   cudaStream_t st = (cudaStream_t)stream;
   if (a->x) {
@@ -285,11 +335,19 @@ extern "C" csa_status csa_compress(const csa_compress_args* a, void* stream) {
   const int n_out = a->T / a->ratio;
   if (a->B == 0 || n_out == 0) return CSA_OK;
   if (a->W_IK) CSA_SUPPORTED(a->d_index == 64 || a->d_index == 128);
+  if (a->kv_pack.codes) {
+    CSA_REQUIRE(a->kv_pack.scales && (a->d_rope == 0 || a->kv_pack.rope) && a->kv_pack.global_scale > 0.0f);
+    CSA_SUPPORTED((a->d - a->d_rope) % 32 == 0);
+  }
+  if (a->ki_pack.codes) CSA_REQUIRE(a->W_IK && a->ki_pack.scales && a->ki_pack.global_scale > 0.0f);
   const size_t smem = (size_t)POOL_ENT * a->d * sizeof(float) + (a->W_IK ? (size_t)POOL_KT * a->d_index * 2 : 0);
   CSA_SUPPORTED(smem <= 48 * 1024);
+  PoolParams P{};
+  P.C = (const uint16_t*)a->C; P.Z = (const uint16_t*)a->Z; P.b_pos = a->b_pos; P.T = a->T; P.d = a->d;
+  P.d_r = a->d_rope; P.r = a->ratio; P.theta = a->rope_theta; P.pos0 = a->pos0; P.W_IK = (const uint16_t*)a->W_IK;
+  P.d_I = a->d_index; P.c_out = (uint16_t*)a->c_out; P.kI_out = (uint16_t*)a->kI_out; P.kv = a->kv_pack;
+  P.ki = a->ki_pack;
   dim3 grid((n_out + POOL_ENT - 1) / POOL_ENT, a->B);
-  pool_kernel<<<grid, 256, smem, st>>>((const uint16_t*)a->C, (const uint16_t*)a->Z, a->b_pos, a->T, a->d,
-                                       a->d_rope, a->ratio, a->rope_theta, a->pos0, (const uint16_t*)a->W_IK,
-                                       a->d_index, (uint16_t*)a->c_out, (uint16_t*)a->kI_out);
+  pool_kernel<<<grid, 256, smem, st>>>(P);
   return launch_status();
 }

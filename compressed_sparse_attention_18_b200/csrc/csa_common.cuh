@@ -117,6 +117,29 @@ __device__ __forceinline__ float e2m1_value(uint32_t code) {
 
 // ----------------------------------------------------------------------------- warp helpers
 
+__device__ __forceinline__ float warp_max(float v);
+
+// FP4 pack of one 32-element block by one warp (lane e holds element e, an fp32 copy of a bf16):
+//   s = E4M3_rne_satfinite(fp32(amax / fp32(6 g))); s == 0 -> all codes 0;
+//   code_e = E2M1_rne_satfinite(fp32(x_e / fp32(s g))), -0 -> +0; element 2j in the low nibble of byte j.
+// Writes the 16 code bytes at codes16 and the scale byte at *scale.
+__device__ __forceinline__ void pack_block_warp(float x, float g, uint8_t* codes16, uint8_t* scale) {
+  const int lane = threadIdx.x & 31;
+  const float amax = warp_max(fabsf(x));
+  const uint32_t s_code = f32_to_e4m3(__fdiv_rn(amax, 6.0f * g));
+  const float s = e4m3_to_f32(s_code);
+  uint32_t code = 0;
+  if (s != 0.0f) code = f32_to_e2m1(__fdiv_rn(x, __fmul_rn(s, g)));
+  const uint32_t pair = code | (__shfl_down_sync(0xffffffffu, code, 1) << 4);
+  // bytes 4m..4m+3 gathered on lane 8m, one 32-bit store per 8 lanes
+  const uint32_t b1 = __shfl_down_sync(0xffffffffu, pair, 2);
+  const uint32_t b2 = __shfl_down_sync(0xffffffffu, pair, 4);
+  const uint32_t b3 = __shfl_down_sync(0xffffffffu, pair, 6);
+  if ((lane & 7) == 0)
+    reinterpret_cast<uint32_t*>(codes16)[lane >> 3] = (pair & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
+  if (lane == 0) *scale = (uint8_t)s_code;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

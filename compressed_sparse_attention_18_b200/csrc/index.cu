@@ -24,6 +24,8 @@ constexpr int IDX_QT = 32;             // max queries per CTA (query fragments s
 constexpr int TOPK_THREADS = 1024;
 constexpr int TOPK_CHUNK = 32768;      // max row length held in shared memory (implicit ids)
 constexpr int TOPK_CHUNK_IDS = 16384;  // max row length with explicit ids
+constexpr int HIST_BINS = 4096;        // score histogram: top 12 bits of the order-preserving key
+constexpr int HIST_SHIFT = 20;
 
 // ---------------------------------------------------------------------------- query quantisation
 // One warp per (query, head) row of q_I: FP4 pack rule (global scale g_q), then the f16 products
@@ -109,12 +111,15 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
     const uint16_t* __restrict__ q_I, const float* __restrict__ w, int H_I, float g_q, float gg, int Nq, int qt,
     const uint8_t* __restrict__ k_codes, const uint8_t* __restrict__ k_scales, int n_max,
     const int32_t* __restrict__ n_c, const int64_t* __restrict__ q_pos, int ratio,
-    const int32_t* __restrict__ cand, int n_cand, float* __restrict__ scores, long long ld, int tpw) {
+    const int32_t* __restrict__ cand, int n_cand, float* __restrict__ scores, long long ld, int tpw,
+    uint32_t* __restrict__ hist) {
   constexpr int STEPS = DI / 16;
   constexpr int BREGS = DI / 8;           // f16x2 registers of one head slice per thread
   constexpr int S_PAD = ((DI / 32) + 3) & ~3;
   extern __shared__ __align__(16) uint8_t s_dyn[];
   __half* s_q = reinterpret_cast<__half*>(s_dyn);          // [qt][IDX_HEADS][DI]
+  // single-query CTAs may also count their scores in HIST_BINS bins (key >> HIST_SHIFT) for the top-k
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_dyn + (size_t)qt * IDX_HEADS * DI * 2);
   __shared__ float s_w[IDX_QT][IDX_HEADS];
   __shared__ int s_nvis[IDX_QT];
   __shared__ long long s_t[IDX_QT];
@@ -131,6 +136,8 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
   if (chunk0 >= n_cols) return;
 
   quantize_query_tile(q_I, w, b * Nq + q0, nq, H_I, DI, g_q, gg, s_q, &s_w[0][0]);
+  if (hist)
+    for (int i = tid; i < HIST_BINS; i += blockDim.x) s_hist[i] = 0;
   int max_vis = 0;
   for (int qq = 0; qq < nq; ++qq) {
     const long long tq = q_pos[(size_t)b * Nq + q0 + qq];
@@ -229,12 +236,27 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
         const int col = col0 + g + 8 * t;
         const float v = (t ? r1 : r0) + 0.0f;
         float* row = scores + (size_t)(b * Nq + q0 + qq) * ld;
+        bool counted = false;
         if (cand_row) {
-          if (col < col_end) row[col] = (t ? kval[cur][1] : kval[cur][0]) ? v : -INFINITY;
+          if (col < col_end) {
+            const bool ok = t ? kval[cur][1] : kval[cur][0];
+            row[col] = ok ? v : -INFINITY;
+            counted = ok;
+          }
         } else if (col < s_nvis[qq]) {
           row[col] = v;
+          counted = true;
         }
+        if (hist && counted) atomicAdd(&s_hist[float_order_key(v) >> HIST_SHIFT], 1u);
       }
+    }
+  }
+  if (hist) {
+    __syncthreads();
+    uint32_t* h = hist + (size_t)(b * Nq + q0) * HIST_BINS;
+    for (int i = tid; i < HIST_BINS; i += blockDim.x) {
+      const uint32_t c = s_hist[i];
+      if (c) atomicAdd(&h[i], c);
     }
   }
 }
@@ -251,6 +273,7 @@ struct TopkSmem {
   uint32_t scan[TOPK_THREADS / 32];
   uint32_t bcast[4];
   uint32_t counter;
+  uint32_t tie_taken;
 };
 
 // Find the R-th largest value of key(j) over positions j < n with filt(j).  Returns the threshold
@@ -355,6 +378,85 @@ struct TopkRowArgs {
   long long out_ld;
 };
 
+// Select the K largest of keys[0..len) (0 = not a candidate; nvalid candidates in all) by (key desc,
+// id asc), writing ids / scores to oi[base + slot], os[base + slot] in unspecified order.  Candidates
+// with equal key and equal id (a repeated id) are interchangeable: any of them gives the same output.
+template <class IdF>
+__device__ void select_in_smem(TopkSmem& sm, const uint32_t* keys, int len, uint32_t K, uint32_t nvalid, IdF idof,
+                               int32_t* oi, float* os, uint32_t base) {
+  auto valid = [&](int j) { return keys[j] != 0u; };
+  uint32_t T1 = 0, above1 = 0, T2 = 0xFFFFFFFFu, need_pos = 0;
+  bool all_ties = true;
+  if (K > 0 && K < nvalid) {
+    T1 = radix_threshold(sm, len, K, [&](int j) { return keys[j]; }, valid, &above1);
+    const uint32_t need = K - above1;
+    uint32_t tl = 0;
+    for (int j = threadIdx.x; j < len; j += blockDim.x) tl += (keys[j] == T1);
+    uint32_t nties;
+    block_exclusive_scan(sm, tl, &nties);
+    if (nties > need) {
+      all_ties = false;
+      uint32_t above2;
+      T2 = radix_threshold(sm, len, need, [&](int j) { return ~idof(j); },
+                           [&](int j) { return keys[j] == T1; }, &above2);
+      need_pos = need - above2;
+    }
+  }
+  if (threadIdx.x == 0) { sm.counter = 0; sm.tie_taken = 0; }
+  __syncthreads();
+  for (int j = threadIdx.x; j < len; j += blockDim.x) {
+    const uint32_t kj = keys[j];
+    if (kj == 0u) continue;
+    bool take;
+    if (K >= nvalid) take = true;
+    else if (kj > T1) take = true;
+    else if (kj < T1) take = false;
+    else if (all_ties) take = true;
+    else {
+      const uint32_t k2 = ~idof(j);
+      if (k2 > T2) take = true;
+      else if (k2 < T2) take = false;
+      else take = atomicAdd(&sm.tie_taken, 1u) < need_pos;
+    }
+    if (take) {
+      const uint32_t slot = base + atomicAdd(&sm.counter, 1u);
+      oi[slot] = (int32_t)idof(j);
+      if (os) os[slot] = order_key_float(kj);
+    }
+  }
+  __syncthreads();
+}
+
+// Load one row segment into shared memory as order-preserving keys (0 = not a candidate) and, with
+// explicit ids, the ids; returns the number of candidates.  8 independent loads in flight per thread.
+__device__ uint32_t load_row_keys(TopkSmem& sm, const float* __restrict__ src, const int32_t* __restrict__ isrc,
+                                  int len, uint32_t* keys, int32_t* ids) {
+  uint32_t nvalid_loc = 0;
+  constexpr int U = 8;
+  for (int j0 = threadIdx.x; j0 < len; j0 += U * blockDim.x) {
+    float v[U];
+    int32_t id[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * blockDim.x;
+      v[u] = j < len ? src[j] : -INFINITY;
+      id[u] = (isrc && j < len) ? isrc[j] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * blockDim.x;
+      if (j >= len) continue;
+      const bool ok = v[u] > -INFINITY && id[u] >= 0;
+      keys[j] = ok ? float_order_key(v[u]) : 0u;
+      if (isrc) ids[j] = id[u];
+      nvalid_loc += ok;
+    }
+  }
+  uint32_t nvalid;
+  block_exclusive_scan(sm, nvalid_loc, &nvalid);
+  return nvalid;
+}
+
 __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(TopkRowArgs A) {
   extern __shared__ __align__(16) uint32_t s_keys[];
   __shared__ TopkSmem sm;
@@ -373,88 +475,135 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(TopkRowArgs A) {
   int32_t* ids = reinterpret_cast<int32_t*>(s_keys + (A.in_ids ? TOPK_CHUNK_IDS : 0));
   const float* src = A.in_scores + row * A.in_ld + col0;
   const int32_t* isrc = A.in_ids ? A.in_ids + row * A.in_ld + col0 : nullptr;
-  uint32_t nvalid_loc = 0;
-  constexpr int U = 8;   // independent loads in flight per thread
-  for (int j0 = threadIdx.x; j0 < len; j0 += U * blockDim.x) {
-    float v[U];
-    int32_t id[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int j = j0 + u * blockDim.x;
-      v[u] = j < len ? src[j] : -INFINITY;
-      id[u] = (isrc && j < len) ? isrc[j] : 0;
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int j = j0 + u * blockDim.x;
-      if (j >= len) continue;
-      const bool ok = v[u] > -INFINITY && id[u] >= 0;
-      keys[j] = ok ? float_order_key(v[u]) : 0u;   // 0 marks "not a candidate"
-      if (isrc) ids[j] = id[u];
-      nvalid_loc += ok;
-    }
-  }
-  uint32_t nvalid;
-  block_exclusive_scan(sm, nvalid_loc, &nvalid);
+  const uint32_t nvalid = load_row_keys(sm, src, isrc, len, keys, ids);
   const int out_seg = blockIdx.x;
   int32_t* oi = A.out_idx + row * A.out_ld + (long long)out_seg * A.k;
   float* os = A.out_scores ? A.out_scores + row * A.out_ld + (long long)out_seg * A.k : nullptr;
   const uint32_t K = min((uint32_t)A.k, nvalid);
   auto idof = [&](int j) -> uint32_t { return isrc ? (uint32_t)ids[j] : (uint32_t)(A.col_base + seg * A.rows_per_seg + j); };
-  auto valid = [&](int j) { return keys[j] != 0u; };
 
-  uint32_t T1 = 0, above1 = 0, T2 = 0xFFFFFFFFu, need_pos = 0;
-  bool all_ties = true;
-  if (K > 0 && K < nvalid) {
-    T1 = radix_threshold(sm, len, K, [&](int j) { return keys[j]; }, valid, &above1);
-    const uint32_t need = K - above1;
-    // count ties
-    uint32_t tl = 0;
-    for (int j = threadIdx.x; j < len; j += blockDim.x) tl += (keys[j] == T1);
-    uint32_t nties;
-    block_exclusive_scan(sm, tl, &nties);
-    if (nties > need) {
-      all_ties = false;
-      uint32_t above2;
-      T2 = radix_threshold(sm, len, need, [&](int j) { return ~idof(j); },
-                           [&](int j) { return keys[j] == T1; }, &above2);
-      need_pos = need - above2;  // ties on (score, id) taken in position order
-    }
-  }
-  if (threadIdx.x == 0) sm.counter = 0;
-  __syncthreads();
-  // emission; contiguous ranges per thread so that position-order ties are deterministic
-  const int per = (len + blockDim.x - 1) / blockDim.x;
-  const int j0 = threadIdx.x * per, j1 = min(len, j0 + per);
-  uint32_t mine = 0;
-  if (!all_ties)
-    for (int j = j0; j < j1; ++j) mine += (keys[j] == T1 && ~idof(j) == T2);
-  uint32_t total3;
-  uint32_t rank = block_exclusive_scan(sm, mine, &total3);
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t kj = keys[j];
-    if (kj == 0u) continue;
-    bool take;
-    if (K >= nvalid) take = true;
-    else if (kj > T1) take = true;
-    else if (kj < T1) take = false;
-    else if (all_ties) take = true;
-    else {
-      const uint32_t k2 = ~idof(j);
-      if (k2 > T2) take = true;
-      else if (k2 < T2) take = false;
-      else take = (rank++ < need_pos);
-    }
-    if (take) {
-      const uint32_t slot = atomicAdd(&sm.counter, 1u);
-      oi[slot] = (int32_t)idof(j);
-      if (os) os[slot] = order_key_float(kj);
-    }
-  }
-  __syncthreads();
+  select_in_smem(sm, keys, len, K, nvalid, idof, oi, os, 0u);
   for (int s = (int)K + threadIdx.x; s < A.k; s += blockDim.x) {
     oi[s] = -1;
     if (os) os[s] = -INFINITY;
+  }
+}
+
+
+// Histogram-guided selection for one row (decode / Reindex rows): the score kernel has counted the
+// row's scores in 4096 bins of the top 12 bits of their order-preserving keys.  The bin holding the
+// K-th largest score is found from the histogram; one pass over the row emits every score in a higher
+// bin and collects the boundary bin's scores, and only those go through the exact radix selection.
+// If the boundary bin overflows the candidate buffer the row is selected by the full path instead.
+__global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, const uint32_t* __restrict__ hist) {
+  extern __shared__ __align__(16) uint32_t s_keys[];   // candidates: keys [TOPK_CHUNK_IDS] | ids [TOPK_CHUNK_IDS]
+  __shared__ TopkSmem sm;
+  __shared__ uint32_t s_cnt[2];                         // emitted above the boundary bin, boundary candidates
+  const int row = blockIdx.y;
+  int len = min(A.rows_per_seg, A.n_cols);
+  if (A.q_pos) {
+    const int b = row / A.Nq;
+    long long nv = (A.q_pos[row] + 1) / A.ratio;
+    if (nv > A.n_c[b]) nv = A.n_c[b];
+    len = (int)max(0LL, min((long long)len, nv));
+  }
+  if (len < 0) len = 0;
+  int32_t* oi = A.out_idx + row * A.out_ld;
+  float* os = A.out_scores ? A.out_scores + row * A.out_ld : nullptr;
+  const float* src = A.in_scores + row * A.in_ld;
+  const int32_t* isrc = A.in_ids ? A.in_ids + row * A.in_ld : nullptr;
+
+  // suffix counts over the bins: thread t owns the 4 bins [4(T-1-t), 4(T-1-t)+4), highest bins first
+  const int owner = (int)blockDim.x - 1 - (int)threadIdx.x;
+  const uint4 hv = reinterpret_cast<const uint4*>(hist + (size_t)row * HIST_BINS)[owner];
+  const uint32_t mine = hv.x + hv.y + hv.z + hv.w;
+  uint32_t nvalid;
+  const uint32_t above_me = block_exclusive_scan(sm, mine, &nvalid);
+  const uint32_t K = min((uint32_t)A.k, nvalid);
+  if (threadIdx.x == 0) { s_cnt[0] = 0; s_cnt[1] = 0; sm.bcast[0] = 0; sm.bcast[1] = 0; sm.bcast[2] = 0; }
+  __syncthreads();
+  if (K > 0 && above_me < K && K <= above_me + mine) {
+    const uint32_t c[4] = {hv.w, hv.z, hv.y, hv.x};
+    uint32_t acc = above_me;
+    for (int i = 0; i < 4; ++i) {
+      if (acc + c[i] >= K) {
+        sm.bcast[0] = (uint32_t)(owner * 4 + 3 - i);
+        sm.bcast[1] = acc;
+        sm.bcast[2] = c[i];
+        break;
+      }
+      acc += c[i];
+    }
+  }
+  __syncthreads();
+  const uint32_t Tbin = sm.bcast[0], above = sm.bcast[1], nT = sm.bcast[2];
+  const uint32_t need = K - above;
+  uint32_t* ckeys = s_keys;
+  int32_t* cids = reinterpret_cast<int32_t*>(s_keys + TOPK_CHUNK_IDS);
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  if (K > 0) {
+    constexpr int U = 8;
+    for (int jb = 0; jb < len; jb += U * blockDim.x) {
+      float v[U];
+      int32_t id[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = jb + u * blockDim.x + threadIdx.x;
+        v[u] = j < len ? src[j] : -INFINITY;
+        id[u] = j < len ? (isrc ? isrc[j] : j) : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const bool ok = v[u] > -INFINITY && id[u] >= 0;
+        const uint32_t key = float_order_key(v[u]);
+        const uint32_t bin = key >> HIST_SHIFT;
+        const bool up = ok && bin > Tbin, at = ok && bin == Tbin;
+        const unsigned mu = __ballot_sync(0xffffffffu, up), ma = __ballot_sync(0xffffffffu, at);
+        uint32_t bu = 0, ba = 0;
+        if (lane == 0) {
+          if (mu) bu = atomicAdd(&s_cnt[0], (uint32_t)__popc(mu));
+          if (ma) ba = atomicAdd(&s_cnt[1], (uint32_t)__popc(ma));
+        }
+        bu = __shfl_sync(0xffffffffu, bu, 0);
+        ba = __shfl_sync(0xffffffffu, ba, 0);
+        if (up) {
+          const uint32_t slot = bu + __popc(mu & lt);
+          oi[slot] = id[u];
+          if (os) os[slot] = v[u] + 0.0f;
+        }
+        if (at) {
+          const uint32_t slot = ba + __popc(ma & lt);
+          if (slot < TOPK_CHUNK_IDS) { ckeys[slot] = key; cids[slot] = id[u]; }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t ncand = s_cnt[1];
+  if (K > 0 && ncand <= TOPK_CHUNK_IDS && s_cnt[0] == above && ncand == nT) {
+    auto idof = [&](int j) -> uint32_t { return (uint32_t)cids[j]; };
+    if (ncand == need) {
+      for (int j = threadIdx.x; j < (int)ncand; j += blockDim.x) {
+        oi[above + j] = cids[j];
+        if (os) os[above + j] = order_key_float(ckeys[j]);
+      }
+      __syncthreads();
+    } else {
+      select_in_smem(sm, ckeys, (int)ncand, need, ncand, idof, oi, os, above);
+    }
+  } else if (K > 0) {
+    // boundary bin larger than the buffer (or inconsistent counts): select the whole row
+    __syncthreads();
+    const uint32_t nv2 = load_row_keys(sm, src, isrc, len, s_keys,
+                                       reinterpret_cast<int32_t*>(s_keys + (isrc ? TOPK_CHUNK_IDS : 0)));
+    int32_t* ids2 = reinterpret_cast<int32_t*>(s_keys + TOPK_CHUNK_IDS);
+    auto idof2 = [&](int j) -> uint32_t { return isrc ? (uint32_t)ids2[j] : (uint32_t)j; };
+    select_in_smem(sm, s_keys, len, min((uint32_t)A.k, nv2), nv2, idof2, oi, os, 0u);
+  }
+  for (int s2 = (int)K + threadIdx.x; s2 < A.k; s2 += blockDim.x) {
+    oi[s2] = -1;
+    if (os) os[s2] = -INFINITY;
   }
 }
 
@@ -494,11 +643,18 @@ __global__ void pool_expand_kernel(const int32_t* __restrict__ blk, int P, int G
   pool[(long long)row * P * G + s] = out;
 }
 
+// tensor-core scoring of single-query Full rows (index_tc.cu)
+bool index_tc_eligible(const csa_index_args* a);
+csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, uint32_t* hist, cudaStream_t st);
+
 // ------------------------------------------------------------------------------ orchestration
 struct IndexPlan {
   int rows, n_cols, segs, seg_len;
-  size_t off_scores, off_tidx, off_tsc, off_bs, off_bidx, sel_total, total;
+  bool hist;   // single-query rows that fit one top-k pass: histogram-guided selection
+  size_t off_scores, off_tidx, off_tsc, off_bs, off_bidx, off_hist, sel_total, total;
 };
+
+static bool one_query_per_cta(const csa_index_args* a) { return a->cand != nullptr || a->Nq == 1; }
 
 // Workspace of the selection step (tournament buffers, pool block scores); the fused entry point
 // places the score matrix in front of it.
@@ -523,7 +679,11 @@ static IndexPlan plan_index(const csa_index_args* a) {
   }
   p.sel_total = o;
   p.off_scores = o;
-  p.total = align_up(o + (size_t)p.rows * p.n_cols * 4, 256);
+  o = align_up(o + (size_t)p.rows * p.n_cols * 4, 256);
+  p.hist = one_query_per_cta(a) && p.segs == 1;
+  p.off_hist = o;
+  if (p.hist) o = align_up(o + (size_t)p.rows * HIST_BINS * 4, 256);
+  p.total = o;
   return p;
 }
 
@@ -554,8 +714,14 @@ static csa_status validate_index(const csa_index_args* a, bool need_select) {
   return CSA_OK;
 }
 
-static csa_status run_scores(const csa_index_args* a, float* scores, long long ld, cudaStream_t st) {
+static csa_status run_scores(const csa_index_args* a, float* scores, long long ld, uint32_t* hist, cudaStream_t st) {
   const int n_cols = a->cand ? a->n_cand : a->n_max;
+  if (!one_query_per_cta(a)) hist = nullptr;
+  if (hist) {
+    cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)a->B * a->Nq * HIST_BINS * 4, st);
+    if (e != cudaSuccess) { set_last_cuda_error(e); return CSA_ERR_CUDA; }
+  }
+  if (index_tc_eligible(a)) return run_scores_tc(a, scores, ld, hist, st);
   const int qt = a->cand ? 1 : (a->Nq < IDX_QT ? a->Nq : IDX_QT);
   const long long qtiles = (long long)a->B * (a->cand ? a->Nq : (a->Nq + qt - 1) / qt);
   // key range per CTA: enough CTAs for about one wave, at least one 16-key tile per warp
@@ -566,19 +732,19 @@ static csa_status run_scores(const csa_index_args* a, float* scores, long long l
   const long long kpc = IDX_WARPS * 16 * tpw;
   dim3 grid((unsigned)((n_cols + kpc - 1) / kpc), a->cand ? a->Nq : (a->Nq + qt - 1) / qt, a->B);
   if (n_cols == 0) return CSA_OK;
-  const int smem = qt * IDX_HEADS * a->d_I * 2;
+  const int smem = qt * IDX_HEADS * a->d_I * 2 + (hist ? HIST_BINS * 4 : 0);
   const float gg = a->g_q * a->g_k;
   static std::atomic<unsigned> attr128{0}, attr64{0};
   if (a->d_I == 128) {
-    set_smem_once((const void*)index_score_kernel<128>, IDX_QT * IDX_HEADS * 128 * 2, attr128);
+    set_smem_once((const void*)index_score_kernel<128>, IDX_QT * IDX_HEADS * 128 * 2 + HIST_BINS * 4, attr128);
     index_score_kernel<128><<<grid, IDX_WARPS * 32, smem, st>>>(
         (const uint16_t*)a->q_I, a->w, a->H_I, a->g_q, gg, a->Nq, qt, a->k_codes, a->k_scales, a->n_max, a->n_c,
-        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld, (int)tpw);
+        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld, (int)tpw, hist);
   } else {
-    set_smem_once((const void*)index_score_kernel<64>, IDX_QT * IDX_HEADS * 64 * 2, attr64);
+    set_smem_once((const void*)index_score_kernel<64>, IDX_QT * IDX_HEADS * 64 * 2 + HIST_BINS * 4, attr64);
     index_score_kernel<64><<<grid, IDX_WARPS * 32, smem, st>>>(
         (const uint16_t*)a->q_I, a->w, a->H_I, a->g_q, gg, a->Nq, qt, a->k_codes, a->k_scales, a->n_max, a->n_c,
-        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld, (int)tpw);
+        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld, (int)tpw, hist);
   }
   return launch_status();
 }
@@ -594,7 +760,7 @@ static csa_status launch_topk(TopkRowArgs ta, int rows, int segs, bool ids, cuda
 }
 
 static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const float* scores, long long ld,
-                             uint8_t* w8, cudaStream_t st) {
+                             const uint32_t* hist, uint8_t* w8, cudaStream_t st) {
   TopkRowArgs ta{};
   ta.in_scores = scores;
   ta.in_ids = a->cand;
@@ -608,7 +774,16 @@ static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const 
   ta.rows_per_seg = p.seg_len;
   ta.k = a->k;
   if (a->cand) CSA_SUPPORTED(ld == a->n_cand);   // explicit ids are read with the score row stride
-  if (p.segs == 1) {
+  if (p.segs == 1 && hist != nullptr && p.hist) {
+    ta.out_idx = a->idx_out;
+    ta.out_scores = a->scores_out;
+    ta.out_ld = a->k;
+    static std::atomic<unsigned> attr_h{0};
+    set_smem_once((const void*)topk_hist_kernel, TOPK_CHUNK * 4, attr_h);
+    topk_hist_kernel<<<dim3(1, p.rows), TOPK_THREADS, TOPK_CHUNK * 4, st>>>(ta, hist);
+    csa_status s = launch_status();
+    if (s != CSA_OK) return s;
+  } else if (p.segs == 1) {
     ta.out_idx = a->idx_out;
     ta.out_scores = a->scores_out;
     ta.out_ld = a->k;
@@ -713,9 +888,10 @@ extern "C" csa_status csa_index_topk_noalloc(const csa_index_args* a, void* stre
   cudaStream_t st = (cudaStream_t)stream;
   uint8_t* w8 = (uint8_t*)ws;
   float* scores = (float*)(w8 + p.off_scores);
-  csa_status s = run_scores(a, scores, p.n_cols, st);
+  uint32_t* hist = p.hist ? (uint32_t*)(w8 + p.off_hist) : nullptr;
+  csa_status s = run_scores(a, scores, p.n_cols, hist, st);
   if (s != CSA_OK) return s;
-  return run_select(a, p, scores, p.n_cols, w8, st);
+  return run_select(a, p, scores, p.n_cols, hist, w8, st);
 }
 
 extern "C" csa_status csa_index_scores(const csa_index_args* a, float* scores, int64_t ld, void* stream) {
@@ -724,7 +900,7 @@ extern "C" csa_status csa_index_scores(const csa_index_args* a, float* scores, i
   if ((long long)a->B * a->Nq == 0) return CSA_OK;
   const int n_cols = a->cand ? a->n_cand : a->n_max;
   CSA_REQUIRE(scores != nullptr && ld >= n_cols);
-  return run_scores(a, scores, ld, (cudaStream_t)stream);
+  return run_scores(a, scores, ld, a->hist, (cudaStream_t)stream);
 }
 
 extern "C" size_t csa_topk_workspace_size(const csa_index_args* a) {
@@ -741,7 +917,7 @@ extern "C" csa_status csa_topk(const csa_index_args* a, const float* scores, int
   CSA_REQUIRE(scores != nullptr && ld >= p.n_cols);
   if (ws_bytes < p.sel_total) return CSA_ERR_WORKSPACE;
   CSA_REQUIRE(ws != nullptr || p.sel_total == 0);
-  return run_select(a, p, scores, ld, (uint8_t*)ws, (cudaStream_t)stream);
+  return run_select(a, p, scores, ld, a->hist, (uint8_t*)ws, (cudaStream_t)stream);
 }
 
 extern "C" size_t csa_index_topk_workspace_size(const csa_index_args* a) {
@@ -761,7 +937,8 @@ extern "C" csa_status csa_index_topk(const csa_index_args* a, void* ws, size_t w
   cudaStream_t st = (cudaStream_t)stream;
   uint8_t* w8 = (uint8_t*)ws;
   float* scores = (float*)(w8 + p.off_scores);
-  csa_status s = run_scores(a, scores, p.n_cols, st);
+  uint32_t* hist = p.hist ? (uint32_t*)(w8 + p.off_hist) : nullptr;
+  csa_status s = run_scores(a, scores, p.n_cols, hist, st);
   if (s != CSA_OK) return s;
-  return run_select(a, p, scores, p.n_cols, w8, st);
+  return run_select(a, p, scores, p.n_cols, hist, w8, st);
 }

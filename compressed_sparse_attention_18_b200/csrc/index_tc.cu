@@ -1,0 +1,337 @@
+// Lightning-indexer scores on the 5th-generation tensor cores (tcgen05, block-scaled FP4), for rows
+// that score every visible key of one query (decode and the Full layer of cross-layer reuse).
+// Sources: "DeepSeek-V4: エージェントが実際に使える100万トークンのコンテキスト", §ハイブリッド注意, Fig. 3 (an FP4
+// multi-head ReLU indexer over the compressed entries); "DeepSeek-V4.1-Flash - Pushing the Limits of
+// KV Cache Compression", FP4 主 KV キャッシュ bullet (E2M1 values with E4M3 scale factors).
+//
+// One MMA tile = 128 keys (M) x the 8 indexer heads of the query (N) x 128 elements (K, two K64
+// instructions of kind::mxf4nvf4 with UE4M3 scales per 16 elements; the key's E4M3 scale of each
+// 32-block is written for both of its 16-element halves).  The tensor core forms exactly
+//   D[key][h] = sum_blk sq[h][blk] * sk[key][blk] * sum_{e in blk} e2m1(q_e) e2m1(k_e)
+// in fp32, i.e. the indexer's per-head dot product before the ReLU.  The epilogue applies
+// s = sum_h w'[h] * max(0, D[key][h]) with w' = w * g_q * g_k.
+//
+// Warp roles (192 threads, persistent over a contiguous range of key tiles of one query row):
+//   warp 0      TMA producer: 128 x 64 B FP4 code tile (2-D tensor map, 64-byte swizzle) and the
+//               tile's 512 B of key scales (bulk copy) into a STAGES-deep shared-memory ring;
+//   warp 1      allocates tensor memory and issues the MMAs (one thread);
+//   warps 2..5  write each tile's scale factors into tensor memory (tcgen05.st), then read the
+//               previous tile's accumulator (tcgen05.ld), compute the scores, store them and count
+//               them in the row histogram used by the top-k.
+// Every wait is bounded; on a timeout the kernel records CSA device error 1 and leaves.
+#include "csa_common.cuh"
+#include "sm100.cuh"
+
+namespace csa {
+
+using namespace sm100;
+
+constexpr int TC_STAGES = 6;
+constexpr int TC_TILE = 128;                     // keys per tile (MMA M)
+constexpr int TC_CODE_BYTES = TC_TILE * 64;      // 128 keys x 128 FP4
+constexpr int TC_SC_BYTES = TC_TILE * 4;         // 128 keys x 4 E4M3 scales
+constexpr int TC_THREADS = 192;
+constexpr uint32_t TC_TMEM_COLS = 64;
+constexpr uint32_t TC_COL_D = 0;                 // 2 accumulators x 8 columns
+constexpr uint32_t TC_COL_SFA = 16;              // 2 buffers x 2 atoms x 4 columns
+constexpr uint32_t TC_COL_SFB = 32;              // 2 atoms x 4 columns
+constexpr int TC_HIST_BINS = 4096, TC_HIST_SHIFT = 20;
+
+__device__ uint32_t g_csa_device_error = 0;
+
+struct TcSmem {
+  alignas(1024) uint8_t codes[TC_STAGES][TC_CODE_BYTES];
+  alignas(1024) uint8_t qtile[8 * 64];
+  alignas(16) uint8_t sc[TC_STAGES][TC_SC_BYTES];
+  uint32_t hist[TC_HIST_BINS];
+  float wq[8];
+  uint8_t qsc[8][4];
+  alignas(8) uint64_t full[TC_STAGES];
+  alignas(8) uint64_t empty[TC_STAGES];
+  alignas(8) uint64_t sfa_full[2];
+  alignas(8) uint64_t acc_full[2];
+  alignas(8) uint64_t acc_empty[2];
+  uint32_t tmem_base;
+  uint32_t err;
+};
+
+struct TcParams {
+  const uint16_t* q_I;      // [B][H_I][128] bf16 (Nq == 1)
+  const float* w;           // [B][H_I]
+  const uint8_t* k_scales;  // [B][n_max][4]
+  const int32_t* n_c;
+  const int64_t* q_pos;
+  float* scores;            // [B][ld]
+  uint32_t* hist;           // [B][4096] or null
+  long long ld;
+  int n_max, ratio, H_I, ctas_per_row;
+  float g_q, gg;
+};
+
+// FP4-quantise 32 elements held one per lane (pack rule, global scale g); returns this lane's code.
+__device__ __forceinline__ uint32_t quant_lane(float x, float g, uint32_t* s_code_out) {
+  const float amax = warp_max(fabsf(x));
+  const uint32_t s_code = f32_to_e4m3(__fdiv_rn(amax, 6.0f * g));
+  const float s = e4m3_to_f32(s_code);
+  *s_code_out = s_code;
+  return s != 0.0f ? f32_to_e2m1(__fdiv_rn(x, __fmul_rn(s, g))) : 0u;
+}
+
+__global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                                       const TcParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  TcSmem& S = *reinterpret_cast<TcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  // key tiles of this CTA
+  long long nv = (P.q_pos[b] + 1) / P.ratio;
+  const int ncb = min(P.n_c[b], P.n_max);
+  if (nv > ncb) nv = ncb;
+  if (nv < 0) nv = 0;
+  const int n_vis = (int)nv;
+  const int n_tiles = (n_vis + TC_TILE - 1) / TC_TILE;
+  const int per = (n_tiles + P.ctas_per_row - 1) / P.ctas_per_row;
+  const int t_begin = min(n_tiles, (int)blockIdx.x * per);
+  const int t_end = min(n_tiles, t_begin + per);
+  const int ntile = t_end - t_begin;
+
+  if (threadIdx.x == 0) {
+    S.err = 0;
+    for (int s = 0; s < TC_STAGES; ++s) { mbar_init(&S.full[s], 1); mbar_init(&S.empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&S.sfa_full[a], 4); mbar_init(&S.acc_full[a], 1); mbar_init(&S.acc_empty[a], 4); }
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tensormap(&kmap);
+  for (int i = threadIdx.x; i < TC_HIST_BINS; i += blockDim.x) S.hist[i] = 0;
+  if (warp == 1) { tmem_alloc(&S.tmem_base, TC_TMEM_COLS); tmem_relinquish(); }
+  // query: FP4 B tile (8 heads x 64 B, 64-byte swizzle), its scales, the head weights
+  if (warp >= 2) {
+    const int t = threadIdx.x - 64;          // 0..127
+    const int wg = t >> 5;                   // 0..3: heads 2wg, 2wg+1
+    for (int hh = 0; hh < 2; ++hh) {
+      const int h = 2 * wg + hh;
+      for (int blk = 0; blk < 4; ++blk) {
+        uint32_t code = 0, s_code = 0;
+        if (h < P.H_I) {
+          const float x = bf16_bits_to_f(P.q_I[((size_t)b * P.H_I + h) * 128 + blk * 32 + lane]);
+          code = quant_lane(x, P.g_q, &s_code);
+        }
+        const uint32_t pair = code | (__shfl_down_sync(0xffffffffu, code, 1) << 4);
+        if ((lane & 1) == 0) {
+          const int byte = blk * 16 + (lane >> 1);               // byte of the 64-byte row
+          const int c = byte >> 4;
+          S.qtile[h * 64 + ((c ^ ((h >> 1) & 3)) << 4) + (byte & 15)] = (uint8_t)pair;
+        }
+        if (lane == 0) S.qsc[h][blk] = (uint8_t)s_code;
+      }
+      if (lane == 0) S.wq[h] = h < P.H_I ? P.w[(size_t)b * P.H_I + h] * P.gg : 0.0f;
+    }
+    fence_proxy_async_smem();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = S.tmem_base;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      const long long rows_total = (long long)gridDim.y * P.n_max;
+      int issued = 0;
+      for (int i = 0; i < ntile && ok; ++i) {
+        const int s = i % TC_STAGES, f = i / TC_STAGES;
+        if (f > 0 && !mbar_wait(&S.empty[s], (f - 1) & 1)) { ok = false; break; }
+        const long long row = (long long)b * P.n_max + (long long)(t_begin + i) * TC_TILE;
+        long long nrow = rows_total - row;
+        if (nrow > TC_TILE) nrow = TC_TILE;
+        const uint32_t sc_bytes = (uint32_t)nrow * 4;          // multiple of 16: n_max % 4 == 0
+        mbar_arrive_expect_tx(&S.full[s], TC_CODE_BYTES + sc_bytes);
+        tma_load_2d(S.codes[s], &kmap, 0, (int)row, &S.full[s]);
+        bulk_load(S.sc[s], P.k_scales + row * 4, sc_bytes, &S.full[s]);
+        ++issued;
+      }
+      if (!ok) atomicOr(&S.err, 1u);
+      // drain: wait (bounded) for the copies this thread issued before leaving
+      for (int i = max(0, issued - TC_STAGES); i < issued; ++i)
+        mbar_wait(&S.full[i % TC_STAGES], (i / TC_STAGES) & 1, 1u << 16);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_mxf4_ue4m3(TC_TILE, 8);
+      const uint32_t qa = smem_addr(S.qtile);
+      for (int i = 0; i < ntile && ok; ++i) {
+        const int s = i % TC_STAGES, a = i & 1;
+        if (!mbar_wait(&S.full[s], (i / TC_STAGES) & 1)) { ok = false; break; }
+        if (!mbar_wait(&S.sfa_full[a], (i >> 1) & 1)) { ok = false; break; }
+        if (i >= 2 && !mbar_wait(&S.acc_empty[a], ((i >> 1) - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ca = smem_addr(S.codes[s]);
+        for (int k = 0; k < 2; ++k) {
+          const uint64_t ad = smem_desc(ca + 32 * k, 16, 512, LAYOUT_SW64);
+          const uint64_t bd = smem_desc(qa + 32 * k, 16, 512, LAYOUT_SW64);
+          mma_mxf4(tbase + TC_COL_D + 8 * a, ad, bd, idesc, tbase + TC_COL_SFA + 8 * a + 4 * k,
+                   tbase + TC_COL_SFB + 4 * k, k > 0);
+        }
+        mma_commit(&S.acc_full[a]);
+        mma_commit(&S.empty[s]);
+      }
+      if (!ok) atomicOr(&S.err, 1u);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------ scale factors + epilogue
+    const int q = warp & 3;                                      // tensor-memory lane quadrant
+    const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
+    float wq[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) wq[h] = S.wq[h];
+    {
+      // query scale factors, written once: row h (< 8) at lane h of every quadrant, column j = 0
+      uint32_t w0 = 0, w1 = 0;
+      if (lane < 8) {
+        const uint32_t* s4 = reinterpret_cast<const uint32_t*>(S.qsc[lane]);
+        const uint32_t v = *s4;
+        w0 = __byte_perm(v, 0, 0x1100);
+        w1 = __byte_perm(v, 0, 0x3322);
+      }
+      tmem_st_x4(lane_base + TC_COL_SFB + 0, w0, 0, 0, 0);
+      tmem_st_x4(lane_base + TC_COL_SFB + 4, w1, 0, 0, 0);
+    }
+    float* srow = P.scores + (size_t)b * P.ld;
+    auto epilogue = [&](int i) -> bool {
+      const int a = i & 1;
+      if (!mbar_wait(&S.acc_full[a], (i >> 1) & 1)) return false;
+      tc_fence_after();
+      float d[8];
+      tmem_ld_x8(lane_base + TC_COL_D + 8 * a, d);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.acc_empty[a]);
+      const int key = (t_begin + i) * TC_TILE + 32 * q + lane;
+      if (key < n_vis) {
+        float sc = 0.f;
+#pragma unroll
+        for (int h = 0; h < 8; ++h) sc = fmaf(wq[h], fmaxf(d[h], 0.f), sc);
+        sc += 0.0f;
+        srow[key] = sc;
+        if (P.hist) atomicAdd(&S.hist[float_order_key(sc) >> TC_HIST_SHIFT], 1u);
+      }
+      return true;
+    };
+    for (int i = 0; i < ntile && ok; ++i) {
+      const int s = i % TC_STAGES, a = i & 1;
+      if (!mbar_wait(&S.full[s], (i / TC_STAGES) & 1)) { ok = false; break; }
+      // key scale factors of tile i: lane L of every quadrant holds rows L%32 + 32j, j = column
+      const uint32_t* sc = reinterpret_cast<const uint32_t*>(S.sc[s]);
+      uint32_t v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = sc[lane + 32 * j];
+      tmem_st_x4(lane_base + TC_COL_SFA + 8 * a + 0, __byte_perm(v[0], 0, 0x1100), __byte_perm(v[1], 0, 0x1100),
+                 __byte_perm(v[2], 0, 0x1100), __byte_perm(v[3], 0, 0x1100));
+      tmem_st_x4(lane_base + TC_COL_SFA + 8 * a + 4, __byte_perm(v[0], 0, 0x3322), __byte_perm(v[1], 0, 0x3322),
+                 __byte_perm(v[2], 0, 0x3322), __byte_perm(v[3], 0, 0x3322));
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.sfa_full[a]);
+      if (i >= 1 && !epilogue(i - 1)) { ok = false; break; }
+    }
+    if (ok && ntile > 0 && !epilogue(ntile - 1)) ok = false;
+    if (!ok && lane == 0) atomicOr(&S.err, 1u);
+  }
+  __syncthreads();
+  if (S.err && threadIdx.x == 0) atomicOr(&g_csa_device_error, 1u);
+  if (P.hist && S.err == 0) {
+    uint32_t* h = P.hist + (size_t)b * TC_HIST_BINS;
+    for (int i = threadIdx.x; i < TC_HIST_BINS; i += blockDim.x) {
+      const uint32_t c = S.hist[i];
+      if (c) atomicAdd(&h[i], c);
+    }
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, TC_TMEM_COLS);
+  }
+}
+
+// --------------------------------------------------------------------------------------- host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load();
+  if (!f) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      f = (EncodeTiledFn)p;
+    fn.store(f);
+  }
+  return f;
+}
+
+bool index_tc_eligible(const csa_index_args* a) {
+  return a->cand == nullptr && a->Nq == 1 && a->d_I == 128 && a->H_I <= 8 && a->n_max % 4 == 0 && a->n_max > 0 &&
+         (reinterpret_cast<uintptr_t>(a->k_codes) & 15) == 0 && (reinterpret_cast<uintptr_t>(a->k_scales) & 15) == 0 &&
+         encode_fn() != nullptr;
+}
+
+csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, uint32_t* hist, cudaStream_t st) {
+  CUtensorMap map;
+  const cuuint64_t gdim[2] = {64, (cuuint64_t)a->B * (cuuint64_t)a->n_max};
+  const cuuint64_t gstride[1] = {64};
+  const cuuint32_t box[2] = {64, TC_TILE};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode_fn()(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void*)a->k_codes, gdim, gstride, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return CSA_ERR_CUDA;
+  TcParams P{};
+  P.q_I = (const uint16_t*)a->q_I;
+  P.w = a->w;
+  P.k_scales = a->k_scales;
+  P.n_c = a->n_c;
+  P.q_pos = a->q_pos;
+  P.scores = scores;
+  P.hist = hist;
+  P.ld = ld;
+  P.n_max = a->n_max;
+  P.ratio = a->ratio;
+  P.H_I = a->H_I;
+  P.g_q = a->g_q;
+  P.gg = a->g_q * a->g_k;
+  // about two CTAs per SM in total, at most one per tile
+  const int tiles_row = (a->n_max + TC_TILE - 1) / TC_TILE;
+  int per_row = (2 * 148 + a->B - 1) / a->B;
+  if (per_row > tiles_row) per_row = tiles_row;
+  if (per_row < 1) per_row = 1;
+  P.ctas_per_row = per_row;
+  const int smem = (int)sizeof(TcSmem) + 1024;
+  static std::atomic<unsigned> attr_done{0};
+  set_smem_once((const void*)index_score_tc_kernel, smem, attr_done);
+  index_score_tc_kernel<<<dim3(per_row, a->B), TC_THREADS, smem, st>>>(map, P);
+  return launch_status();
+}
+
+}  // namespace csa
+
+extern "C" csa_status csa_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    csa::set_last_cuda_error(e);
+    return CSA_ERR_CUDA;
+  }
+  uint32_t v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, csa::g_csa_device_error, sizeof(v));
+  if (e == cudaSuccess && v) e = cudaMemcpyToSymbol(csa::g_csa_device_error, &zero, sizeof(zero));
+  if (e != cudaSuccess) {
+    csa::set_last_cuda_error(e);
+    return CSA_ERR_CUDA;
+  }
+  return v ? CSA_ERR_DEVICE : CSA_OK;
+}

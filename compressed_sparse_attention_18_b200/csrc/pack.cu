@@ -7,8 +7,8 @@
 
 namespace csa {
 
-// One warp per cache row: lane e holds element e of the current 32-block.
-//   s = E4M3(fp32(amax / fp32(6 g))); s == 0 -> zero block; code = E2M1(fp32(x / fp32(s g))).
+// One warp per cache row: every element of the row is loaded first (one memory latency per row),
+// then each 32-block is packed by the whole warp (lane e = element e of the block).
 __global__ void __launch_bounds__(256) pack_fp4_kernel(const uint16_t* __restrict__ src, int B, int n, int d,
                                                        int d_r, float g, const int32_t* __restrict__ row0,
                                                        int n_max, uint8_t* __restrict__ codes,
@@ -19,7 +19,6 @@ __global__ void __launch_bounds__(256) pack_fp4_kernel(const uint16_t* __restric
   const int d_n = d - d_r;
   const int S = d_n >> 5;
   const int S_pad = (S + 3) & ~3;
-  const float six_g = 6.0f * g;
   for (long long row = (long long)blockIdx.x * warps + (threadIdx.x >> 5); row < total;
        row += (long long)gridDim.x * warps) {
     const int b = (int)(row / n);
@@ -27,16 +26,13 @@ __global__ void __launch_bounds__(256) pack_fp4_kernel(const uint16_t* __restric
     const long long dst = (long long)b * n_max + (row0 ? row0[b] : 0) + j;
     const uint16_t* s_row = src + row * d;
     uint8_t* c_row = codes + dst * (d_n >> 1);
-    for (int blk = 0; blk < S; ++blk) {
-      const float x = bf16_bits_to_f(s_row[blk * 32 + lane]);
-      const float amax = warp_max(fabsf(x));
-      const uint32_t s_code = f32_to_e4m3(__fdiv_rn(amax, six_g));
-      const float s = e4m3_to_f32(s_code);
-      uint32_t code = 0;
-      if (s != 0.0f) code = f32_to_e2m1(__fdiv_rn(x, __fmul_rn(s, g)));
-      const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
-      if ((lane & 1) == 0) c_row[blk * 16 + (lane >> 1)] = (uint8_t)(code | (hi << 4));
-      if (lane == 0) scales[dst * S_pad + blk] = (uint8_t)s_code;
+    for (int blk0 = 0; blk0 < S; blk0 += 16) {
+      float x[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) x[u] = blk0 + u < S ? bf16_bits_to_f(s_row[(blk0 + u) * 32 + lane]) : 0.0f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if (blk0 + u < S) pack_block_warp(x[u], g, c_row + (blk0 + u) * 16, scales + dst * S_pad + blk0 + u);
     }
     if (lane < S_pad - S) scales[dst * S_pad + S + lane] = 0;
     for (int e = lane; e < d_r; e += 32) rope[dst * d_r + e] = s_row[d_n + e];

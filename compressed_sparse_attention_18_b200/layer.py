@@ -4,9 +4,10 @@ Plumbing only: caches, window buffer, workspaces and outputs are torch allocatio
 construction, so a step allocates nothing and can be captured in a CUDA graph.  The step is the
 layer's hot path (sources: "DeepSeek-V4: エージェントが実際に使える100万トークンのコンテキスト", §ハイブリッド注意,
 Fig. 3): the token that completes a group of r folds the group into one compressed entry
-(csa_compress, pooling mode: C and Z are the token projections the model already computed), the entry
-and its indexer key are packed into the FP4 caches (csa_pack_fp4), the lightning indexer picks the
-top-k entries (csa_index_topk) and attention runs over them plus the window (csa_sparse_attn).
+(csa_compress, pooling mode: C and Z are the token projections the model already computed) and the
+same launch appends the entry and its indexer key to the FP4 caches; the lightning indexer scores every
+entry (csa_index_scores), the top-k entries are selected (csa_topk) and attention runs over them plus
+the window (csa_sparse_attn).
 """
 from __future__ import annotations
 
@@ -57,6 +58,7 @@ class CSADecodeLayer:
         w = torch.empty((s.B, 1, s.H_I), dtype=torch.float32, device=dev)
         q = torch.empty((s.B, 1, s.H, s.d), dtype=torch.bfloat16, device=dev)
         self.scores = torch.empty((s.B, s.n_max), dtype=torch.float32, device=dev)
+        self.hist = torch.zeros((s.B, 4096), dtype=torch.int32, device=dev)   # score histogram (uint32 bits)
         ws_i = topk_workspace_size(self.ki, self.n_c, self.q_pos, B=s.B, Nq=1, ratio=s.r, k=s.k)
         ws_a = attn_workspace_size(q, self.q_pos, self.kv, self.n_c, self.idx, self.win, self.win_pos0, ratio=s.r,
                                    window=s.W)
@@ -79,7 +81,7 @@ class CSADecodeLayer:
         self.q_pos.fill_(t)
         self.win_pos0.fill_(t - s.W + 1)
 
-    KERNELS_PER_STEP = 7   # pool, 2 x pack, index score, top-k, attention, split-K merge
+    KERNELS_PER_STEP = 5   # pool + FP4 append, index score, top-k, attention, split-K merge
 
     def step(self, C, Z, b_pos, W_IK, q, q_I, w, stream=None, marks=None):
         """One decode step.  C, Z [B, r, d] bf16 (projections of the group's r tokens), q [B,1,H,d],
@@ -95,14 +97,14 @@ class CSADecodeLayer:
 
         mark(0)
         compress(C=C, Z=Z, b_pos=b_pos, ratio=s.r, d_rope=s.d_r, rope_theta=s.rope_theta, pos0=self.pos0,
-                 W_IK=W_IK, c_out=self.c_new, kI_out=self.kI_new, stream=st)
-        pack_fp4(self.c_new, self.kv, self.row0, stream=st)
-        pack_fp4(self.kI_new, self.ki, self.row0, stream=st)
+                 W_IK=W_IK, c_out=self.c_new, kI_out=self.kI_new, kv_cache=self.kv, ki_cache=self.ki, row0=self.row0,
+                 stream=st)
         mark(1)
-        index_scores(q_I, w, self.ki, self.n_c, self.q_pos, self.scores, ratio=s.r, g_q=s.g_q, stream=st)
+        index_scores(q_I, w, self.ki, self.n_c, self.q_pos, self.scores, ratio=s.r, g_q=s.g_q, hist=self.hist,
+                     stream=st)
         mark(2)
         topk(self.scores, self.ki, self.n_c, self.q_pos, B=s.B, Nq=1, ratio=s.r, k=s.k, idx_out=self.idx,
-             ws=self.ws_index, stream=st)
+             hist=self.hist, ws=self.ws_index, stream=st)
         mark(3)
         sparse_attn(q, self.q_pos, self.kv, self.n_c, self.idx, self.win, self.win_pos0, ratio=s.r, window=s.W,
                     out=self.out, lse=self.lse, ws=self.ws_attn, stream=st)

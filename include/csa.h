@@ -49,6 +49,10 @@ const char* csa_status_string(int status);
 int csa_version(void);
 /* The cudaError_t of the last CSA_ERR_CUDA returned on the calling host thread (0 if none). */
 int csa_last_cuda_error(void);
+/* Synchronises `stream`, then reports and clears the device-side error word of the current device:
+ * CSA_ERR_DEVICE if a kernel gave up a bounded wait (a pipeline stalled; its outputs are incomplete),
+ * CSA_OK otherwise, CSA_ERR_CUDA if the synchronisation itself failed. */
+csa_status csa_device_status(void* stream);
 
 /* ------------------------------------------------------------------------------------------------
  * csa_compress — the compressor ([V4 blog] Fig. 3 / Fig. 4; [V4.1 notes] eq.(1) and CSA2 bullet).
@@ -61,11 +65,24 @@ int csa_last_cuda_error(void);
  * pos0[b] + r i (half-split pairs, angle p * theta^(-2m/d_rope); rope_theta == 0 disables it),
  * rounded to bf16 into c_out; then k_I = bf16(c · W_IK) into kI_out when W_IK != NULL.
  * Trailing T % ratio tokens are ignored (the caller keeps them pending).
+ * Fused append (decode): with kv_pack.codes / ki_pack.codes set, the same launch also packs c and k_I
+ * into the FP4 caches exactly as csa_pack_fp4 would (then c_out / kI_out may be NULL).
  * Shapes: x[B][T][d_model], W_kv/W_g[d_model][d], C/Z[B][T][d], b_pos[ratio][d] fp32,
  *         W_IK[d][d_index], c_out[B][T/ratio][d], kI_out[B][T/ratio][d_index], pos0[B] int64 (NULL = 0).
  * Limits: d % 8 == 0, d_rope even and <= d, ratio >= 1; projection mode needs d % 128 == 0 and
  *         d_model % 32 == 0 (else CSA_ERR_UNSUPPORTED).  No workspace.
  * ------------------------------------------------------------------------------------------------ */
+/* An FP4 cache to append packed rows to (the layout csa_pack_fp4 writes): row i of sequence b goes to
+ * cache row row0[b] + i.  codes == NULL means "no cache". */
+typedef struct csa_fp4_cache {
+  uint8_t* codes;          /* [B][n_max][d_n/2] */
+  uint8_t* scales;         /* [B][n_max][S_pad] */
+  void* rope;              /* [B][n_max][d_rope] bf16 (NULL when d_rope == 0) */
+  const int32_t* row0;     /* [B] (NULL = 0) */
+  int32_t n_max;
+  float global_scale;
+} csa_fp4_cache;
+
 typedef struct csa_compress_args {
   uint32_t struct_size;
   int32_t B, T, d_model, d, d_rope, d_index, ratio;
@@ -80,6 +97,8 @@ typedef struct csa_compress_args {
   const void* W_IK;
   void* c_out;
   void* kI_out;
+  csa_fp4_cache kv_pack;   /* optional: also FP4-pack each entry c into this cache (same bytes as csa_pack_fp4) */
+  csa_fp4_cache ki_pack;   /* optional: also FP4-pack each indexer key k_I (d_rope = 0) into this cache */
 } csa_compress_args;
 
 csa_status csa_compress(const csa_compress_args* args, void* stream);
@@ -148,6 +167,9 @@ typedef struct csa_index_args {
   int32_t* pool_out;
   int32_t* idx_out;
   float* scores_out;
+  uint32_t* hist;          /* optional, split calls only: [B*Nq][4096] score histogram that csa_index_scores
+                              fills (single-query rows: Nq == 1 or cand != NULL) and csa_topk uses to find
+                              the k-th score's neighbourhood in one pass; NULL = plain radix selection */
 } csa_index_args;
 
 size_t csa_index_topk_workspace_size(const csa_index_args* args);

@@ -47,6 +47,24 @@ def test_struct_sizes_match_the_header(csa):
     assert csa._lib.csa_pack_fp4(ctypes.byref(a), None) == 1
 
 
+def test_ctypes_mirrors_match_the_c_structs(csa, tmp_path):
+    """sizeof of every argument struct as a C compiler sees include/csa.h == the binding's mirror."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "sz.c"
+    src.write_text('#include <stdio.h>\n#include "csa.h"\nint main(void){printf("%zu %zu %zu %zu %zu\\n",'
+                   'sizeof(csa_compress_args),sizeof(csa_fp4_cache),sizeof(csa_pack_args),'
+                   'sizeof(csa_index_args),sizeof(csa_attn_args));return 0;}\n')
+    exe = tmp_path / "sz"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    want = [ctypes.sizeof(t) for t in (csa.CompressArgs, csa.Fp4Cache, csa.PackArgs, csa.IndexArgs, csa.AttnArgs)]
+    assert got == want
+
+
 def test_invalid_arguments_are_rejected_on_the_host(csa):
     lib = csa._lib
     # pack: d_n not a multiple of 32 -> unsupported; null pointers -> invalid

@@ -81,14 +81,26 @@ def test_compress_pooling_mode(cuda_lib, r, T, d, d_r, pos0):
     b_pos = normal((r, d), 0.1, G, dtype=torch.float32)
     W_IK = normal((d, 128), d ** -0.5, G)
     p0 = torch.tensor([pos0, pos0 + 8 * r], dtype=torch.int64)
+    n = T // r
+    # fused FP4 append into caches at per-sequence row offsets (same bytes as csa_pack_fp4)
+    kv = csa.PackedCache(B, n + 9, d, d_r, DEV, 0.5)
+    ki = csa.PackedCache(B, n + 9, 128, 0, DEV)
+    row0 = torch.tensor([0, 9], dtype=torch.int32, device=DEV)
     c, kI, _, _ = csa.compress(C=C.to(DEV), Z=Z.to(DEV), b_pos=b_pos.to(DEV), ratio=r, d_rope=d_r,
-                               rope_theta=10000.0, pos0=p0.to(DEV), W_IK=W_IK.to(DEV))
+                               rope_theta=10000.0, pos0=p0.to(DEV), W_IK=W_IK.to(DEV), kv_cache=kv, ki_cache=ki,
+                               row0=row0)
     torch.cuda.synchronize()
     for b in range(B):
         ref = O.compress_pool(f64(C[b]), f64(Z[b]), f64(b_pos), r, d_r, 10000.0, int(p0[b]))
-        assert c.shape[1] == T // r
+        assert c.shape[1] == n
         _ulp_close(f64(c[b]), ref, f"c b={b}")
         _ulp_close(f64(kI[b]), O.index_key(f64(c[b]), f64(W_IK)), f"k_I b={b}")
+        r0 = int(row0[b])
+        codes, scales, rope = O.pack_fp4(f64(c[b]), d_r, 0.5)
+        assert np.array_equal(np_u8(kv.codes[b, r0:r0 + n]), codes) and np.array_equal(np_u8(kv.scales[b, r0:r0 + n]), scales)
+        assert np.array_equal(bf16_bits(kv.rope[b, r0:r0 + n]), bf16_bits(c[b, :, d - d_r:]))
+        kc, ks, _ = O.pack_fp4(f64(kI[b]), 0, 1.0)
+        assert np.array_equal(np_u8(ki.codes[b, r0:r0 + n]), kc) and np.array_equal(np_u8(ki.scales[b, r0:r0 + n]), ks)
 
 
 # ---------------------------------------------------------------------------------------- indexer
@@ -196,6 +208,14 @@ def test_index_exact_ties_take_smallest_ids(cuda_lib):
                              identical_keys=True)
     assert swaps == 0
     assert sorted(idx[0, 0].tolist()) == list(range(10))
+
+
+def test_index_exact_ties_overflow_the_boundary_buffer(cuda_lib):
+    # 20000 equal scores: the histogram's boundary bin holds more candidates than the selection buffer,
+    # so the row takes the full selection path; the smallest ids must still win
+    idx, swaps = _index_case(cuda_lib, B=1, n_max=20000, n_c=[20000], d_I=128, H_I=8, Nq=1, q_pos=[80000], k=10,
+                             seed=9, identical_keys=True)
+    assert swaps == 0 and sorted(idx[0, 0].tolist()) == list(range(10))
 
 
 def test_index_k_larger_than_visible(cuda_lib):
