@@ -388,13 +388,33 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const float* __restrict
   if (lse && threadIdx.x == 0) lse[(size_t)bq * H + h] = sum > 0.f ? s_tot[1] + logf(sum) : -INFINITY;
 }
 
+// tensor-core decode path (attn_tc.cu)
+bool attn_tc_eligible(const csa_attn_args* a, int hca, long long rows);
+int attn_tc_splits(const csa_attn_args* a);
+csa_status launch_attn_tc(const csa_attn_args* a, int splits, float* part_o, float* part_lse, cudaStream_t st);
+
 struct AttnPlan {
   int splits, cps;
+  bool tc;
   size_t off_o, off_lse, total;
 };
 
 static AttnPlan plan_attn(const csa_attn_args* a, int hca) {
   AttnPlan p{};
+  const long long rows_tc = (long long)a->B * a->Nq;
+  if (attn_tc_eligible(a, hca, rows_tc)) {
+    p.tc = true;
+    p.cps = 1;
+    p.splits = attn_tc_splits(a);
+    if (p.splits < 1) p.splits = 1;
+    size_t o = 0;
+    if (p.splits > 1) {
+      p.off_o = o;   o = align_up(o + (size_t)rows_tc * p.splits * a->H * a->d * 4, 256);
+      p.off_lse = o; o = align_up(o + (size_t)rows_tc * p.splits * a->H * 4, 256);
+    }
+    p.total = o;
+    return p;
+  }
   const long long n_sel = hca ? a->n_max : a->k;
   const long long n_win = (a->win_kv && a->Wn > 0) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
   const long long chunks = (n_sel + n_win + AT_KC - 1) / AT_KC;
@@ -452,6 +472,14 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
   if (ws_bytes < p.total) return CSA_ERR_WORKSPACE;
   CSA_REQUIRE(p.total == 0 || ws != nullptr);
   cudaStream_t st = (cudaStream_t)stream;
+  if (p.tc) {
+    float* po = p.splits > 1 ? (float*)((uint8_t*)ws + p.off_o) : nullptr;
+    float* pl = p.splits > 1 ? (float*)((uint8_t*)ws + p.off_lse) : nullptr;
+    csa_status s = launch_attn_tc(a, p.splits, po, pl, st);
+    if (s != CSA_OK || p.splits == 1) return s;
+    attn_merge_kernel<<<(unsigned)(rows * a->H), 128, 0, st>>>(po, pl, p.splits, a->H, a->d, (uint16_t*)a->out, a->lse);
+    return launch_status();
+  }
   AttnParams P{};
   P.B = a->B; P.Nq = a->Nq; P.H = a->H; P.d_r = a->d_rope; P.ratio = a->ratio; P.n_max = a->n_max;
   P.k = a->k; P.Wn = a->win_kv ? a->Wn : 0; P.window = a->window; P.splits = p.splits;

@@ -7,6 +7,7 @@
 // (entries C and gate logits Z are separate projections) and CSA2 bullet (no overlapping entries;
 // indexer K projected from the main KV).
 #include "csa_common.cuh"
+#include "sm100.cuh"
 
 namespace csa {
 
@@ -141,10 +142,10 @@ __global__ void __launch_bounds__(256) gemm_bf16_kernel(const uint16_t* __restri
 // One CTA per (sequence, group of POOL_ENT entries).  Threads walk the d channels: per-channel softmax
 // over the r slots of (Z + b_pos), weighted sum of C (all loads of a channel issued together when
 // r <= 8; an online softmax streams longer groups); RoPE on the last d_r channels at the group-start
-// position (angle and rotation in double); bf16 round; k_I = bf16(c · W_IK) with W_IK staged through
-// shared memory in 128-row tiles; optionally the FP4 pack of c and k_I straight into the caches.
+// position (angle and rotation in double); bf16 round; k_I = bf16(c · W_IK) with W_IK brought into
+// shared memory by one bulk copy issued at kernel start (it lands while the pooling runs); optionally
+// the FP4 pack of c and k_I straight into the caches.
 constexpr int POOL_ENT = 4;
-constexpr int POOL_KT = 128;   // W_IK rows per shared-memory tile
 
 struct PoolParams {
   const uint16_t* C;
@@ -175,9 +176,22 @@ __device__ __forceinline__ void pack_row_to_cache(const float* row, int d, int d
 }
 
 __global__ void __launch_bounds__(256) pool_kernel(PoolParams P) {
-  extern __shared__ __align__(16) float pooled[];   // [POOL_ENT][d], then the W_IK tile / partial sums
+  // shared memory: pooled [POOL_ENT][d] fp32 | W_IK [d][d_I] bf16 | partial sums [2][POOL_ENT][d_I] | k_I rows
+  extern __shared__ __align__(128) float pooled[];
+  __shared__ __align__(8) uint64_t w_bar;
   const int b = blockIdx.y;
   const int d = P.d, d_r = P.d_r, r = P.r, T = P.T, d_I = P.d_I;
+  uint16_t* w_s = reinterpret_cast<uint16_t*>(pooled + POOL_ENT * d);
+  if (P.W_IK != nullptr && threadIdx.x == 0) {
+    // the whole projection matrix arrives while the pooling runs
+    sm100::mbar_init(&w_bar, 1);
+    sm100::fence_mbar_init();
+    const uint32_t bytes = (uint32_t)d * d_I * 2;
+    sm100::mbar_arrive_expect_tx(&w_bar, bytes);
+    for (uint32_t off = 0; off < bytes; off += 32768)
+      sm100::bulk_load(reinterpret_cast<uint8_t*>(w_s) + off, reinterpret_cast<const uint8_t*>(P.W_IK) + off,
+                       min(32768u, bytes - off), &w_bar);
+  }
   const int n_out = T / r;
   const int e0 = blockIdx.x * POOL_ENT;
   const int ne = min(POOL_ENT, n_out - e0);
@@ -254,47 +268,33 @@ __global__ void __launch_bounds__(256) pool_kernel(PoolParams P) {
   if (P.kv.codes)
     for (int q = 0; q < ne; ++q) pack_row_to_cache(pooled + q * d, d, d_r, P.kv, b, e0 + q);
   if (P.W_IK == nullptr) return;
-  // k_I: thread (j, part) accumulates output j over the channels part, part + S, ... of each tile
-  uint16_t* wt = reinterpret_cast<uint16_t*>(pooled + POOL_ENT * d);   // [POOL_KT][d_I]
-  const int S = blockDim.x / d_I;               // d_I divides 256 (64 or 128)
-  const int j = threadIdx.x % d_I, part = threadIdx.x / d_I;
-  float acc[POOL_ENT];
+  // k_I = c · W_IK from shared memory: thread (o, part) sums output o over the channels part, part + 2, ...
+  const bool w_ok = sm100::mbar_wait(&w_bar, 0);
+  if (!w_ok && threadIdx.x == 0) atomicOr(&g_csa_device_error, 1u);
+  float* red = reinterpret_cast<float*>(w_s + (size_t)d * d_I);     // [S][POOL_ENT][d_I], then the k_I rows
+  const int S = blockDim.x / d_I;                                    // d_I divides 256 (64 or 128)
+  {
+    const int o = threadIdx.x % d_I, part = threadIdx.x / d_I;
+    float acc[POOL_ENT];
 #pragma unroll
-  for (int q = 0; q < POOL_ENT; ++q) acc[q] = 0.f;
-  for (int ch0 = 0; ch0 < d; ch0 += POOL_KT) {
-    const int rows = min(POOL_KT, d - ch0);
-    const int n16 = rows * d_I / 8;
-    const uint4* wsrc = reinterpret_cast<const uint4*>(P.W_IK + (size_t)ch0 * d_I);
-    for (int i0 = threadIdx.x; i0 < n16; i0 += 8 * blockDim.x) {   // 8 loads in flight per thread
-      uint4 v[8];
+    for (int q = 0; q < POOL_ENT; ++q) acc[q] = 0.f;
+    if (w_ok) {
+#pragma unroll 8
+      for (int ch = part; ch < d; ch += S) {
+        const float wv = bf16_bits_to_f(w_s[(size_t)ch * d_I + o]);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * blockDim.x;
-        if (i < n16) v[u] = wsrc[i];
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * blockDim.x;
-        if (i < n16) reinterpret_cast<uint4*>(wt)[i] = v[u];
+        for (int q = 0; q < POOL_ENT; ++q) acc[q] = fmaf(pooled[q * d + ch], wv, acc[q]);
       }
     }
-    __syncthreads();
-    for (int ch = part; ch < rows; ch += S) {
-      const float wv = bf16_bits_to_f(wt[ch * d_I + j]);
 #pragma unroll
-      for (int q = 0; q < POOL_ENT; ++q) acc[q] = fmaf(pooled[q * d + ch0 + ch], wv, acc[q]);
-    }
-    __syncthreads();
+    for (int q = 0; q < POOL_ENT; ++q) red[((size_t)part * POOL_ENT + q) * d_I + o] = acc[q];
   }
-  float* red = reinterpret_cast<float*>(wt);    // [S][POOL_ENT][d_I] partial sums, then the k_I rows
-#pragma unroll
-  for (int q = 0; q < POOL_ENT; ++q) red[(part * POOL_ENT + q) * d_I + j] = acc[q];
   __syncthreads();
-  float* krow = red + S * POOL_ENT * d_I;        // [POOL_ENT][d_I]
+  float* krow = red + S * POOL_ENT * d_I;          // [POOL_ENT][d_I]
   for (int i = threadIdx.x; i < ne * d_I; i += blockDim.x) {
     const int q = i / d_I, jj = i % d_I;
     float v = 0.f;
-    for (int pp = 0; pp < S; ++pp) v += red[(pp * POOL_ENT + q) * d_I + jj];
+    for (int pp = 0; pp < S; ++pp) v += red[((size_t)pp * POOL_ENT + q) * d_I + jj];
     const uint32_t bits = f_to_bf16_bits(v);
     if (P.kI_out) P.kI_out[((size_t)b * n_out + e0 + q) * d_I + jj] = (uint16_t)bits;
     krow[q * d_I + jj] = bf16_bits_to_f(bits);
@@ -304,6 +304,8 @@ __global__ void __launch_bounds__(256) pool_kernel(PoolParams P) {
     for (int q = 0; q < ne; ++q) pack_row_to_cache(krow + q * d_I, d_I, 0, P.ki, b, e0 + q);
   }
 }
+
+cudaError_t compress_take_device_error(uint32_t* out) { return take_device_error_here(out); }
 
 }  // namespace csa
 
@@ -340,8 +342,12 @@ extern "C" csa_status csa_compress(const csa_compress_args* a, void* stream) {
     CSA_SUPPORTED((a->d - a->d_rope) % 32 == 0);
   }
   if (a->ki_pack.codes) CSA_REQUIRE(a->W_IK && a->ki_pack.scales && a->ki_pack.global_scale > 0.0f);
-  const size_t smem = (size_t)POOL_ENT * a->d * sizeof(float) + (a->W_IK ? (size_t)POOL_KT * a->d_index * 2 : 0);
-  CSA_SUPPORTED(smem <= 48 * 1024);
+  if (a->W_IK) CSA_SUPPORTED(((uintptr_t)a->W_IK & 15) == 0);
+  const size_t smem = (size_t)POOL_ENT * a->d * sizeof(float) +
+                      (a->W_IK ? (size_t)a->d * a->d_index * 2 + (size_t)(256 / a->d_index + 1) * POOL_ENT * a->d_index * 4 : 0);
+  CSA_SUPPORTED(smem <= 200 * 1024);
+  static std::atomic<unsigned> attr_done{0};
+  set_smem_once((const void*)pool_kernel, 200 * 1024, attr_done);
   PoolParams P{};
   P.C = (const uint16_t*)a->C; P.Z = (const uint16_t*)a->Z; P.b_pos = a->b_pos; P.T = a->T; P.d = a->d;
   P.d_r = a->d_rope; P.r = a->ratio; P.theta = a->rope_theta; P.pos0 = a->pos0; P.W_IK = (const uint16_t*)a->W_IK;

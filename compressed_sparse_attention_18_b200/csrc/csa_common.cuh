@@ -13,6 +13,19 @@
 
 namespace csa {
 
+// Device-side error word of this translation unit (bounded waits that gave up); every unit that
+// uses it exposes it to csa_device_status() through take_device_error_here().
+static __device__ uint32_t g_csa_device_error = 0;
+
+// Read and clear this unit's device error word (host side).
+static inline cudaError_t take_device_error_here(uint32_t* out) {
+  uint32_t v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_csa_device_error, sizeof(v));
+  if (e == cudaSuccess && v) e = cudaMemcpyToSymbol(g_csa_device_error, &zero, sizeof(zero));
+  *out |= v;
+  return e;
+}
+
 // ----------------------------------------------------------------------------- host-side status
 
 void set_last_cuda_error(cudaError_t e);

@@ -283,22 +283,34 @@ __device__ uint32_t radix_threshold(TopkSmem& sm, int n, uint32_t R, KeyF key, F
   uint32_t prefix = 0, mask = 0, rem = R;
   for (int shift = 24; shift >= 0; shift -= 8) {
     const int nw = blockDim.x >> 5, wid = threadIdx.x >> 5;
-    for (int i = threadIdx.x; i < nw * 256; i += blockDim.x) (&sm.whist[0][0])[i] = 0;
-    __syncthreads();
-    // per-warp histograms: scores cluster in a few bins, so a block-wide histogram serialises
-    uint32_t* wh = sm.whist[wid];
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
-      if (!filt(j)) continue;
-      const uint32_t k = key(j);
-      if ((k & mask) == prefix) atomicAdd(&wh[(k >> shift) & 255u], 1u);
+    if (n <= 8192) {
+      // few candidates: one block-wide histogram
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) sm.hist[i] = 0;
+      __syncthreads();
+      for (int j = threadIdx.x; j < n; j += blockDim.x) {
+        if (!filt(j)) continue;
+        const uint32_t k = key(j);
+        if ((k & mask) == prefix) atomicAdd(&sm.hist[(k >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+    } else {
+      for (int i = threadIdx.x; i < nw * 256; i += blockDim.x) (&sm.whist[0][0])[i] = 0;
+      __syncthreads();
+      // per-warp histograms: scores cluster in a few bins, so a block-wide histogram serialises
+      uint32_t* wh = sm.whist[wid];
+      for (int j = threadIdx.x; j < n; j += blockDim.x) {
+        if (!filt(j)) continue;
+        const uint32_t k = key(j);
+        if ((k & mask) == prefix) atomicAdd(&wh[(k >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+        uint32_t c = 0;
+        for (int w = 0; w < nw; ++w) c += sm.whist[w][i];
+        sm.hist[i] = c;
+      }
+      __syncthreads();
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) {
-      uint32_t c = 0;
-      for (int w = 0; w < nw; ++w) c += sm.whist[w][i];
-      sm.hist[i] = c;
-    }
-    __syncthreads();
     if (threadIdx.x < 32) {
       // suffix sums over 256 bins: lane l owns bins [8l, 8l+8)
       const int l = threadIdx.x;
@@ -543,7 +555,7 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
   if (K > 0) {
-    constexpr int U = 8;
+    constexpr int U = 16;   // loads in flight per thread: a 32768-score row takes two rounds
     for (int jb = 0; jb < len; jb += U * blockDim.x) {
       float v[U];
       int32_t id[U];

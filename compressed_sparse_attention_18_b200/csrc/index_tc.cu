@@ -4,21 +4,24 @@
 // multi-head ReLU indexer over the compressed entries); "DeepSeek-V4.1-Flash - Pushing the Limits of
 // KV Cache Compression", FP4 主 KV キャッシュ bullet (E2M1 values with E4M3 scale factors).
 //
-// One MMA tile = 128 keys (M) x the 8 indexer heads of the query (N) x 128 elements (K, two K64
-// instructions of kind::mxf4nvf4 with UE4M3 scales per 16 elements; the key's E4M3 scale of each
-// 32-block is written for both of its 16-element halves).  The tensor core forms exactly
+// One tile = 256 keys = two MMA sub-tiles of 128 keys (M) x the 8 indexer heads of the query (N) x
+// 128 elements (K, two K64 instructions of kind::mxf4nvf4 with UE4M3 scales per 16 elements; the
+// key's E4M3 scale of each 32-block is written for both of its 16-element halves).  The tensor core
+// forms exactly
 //   D[key][h] = sum_blk sq[h][blk] * sk[key][blk] * sum_{e in blk} e2m1(q_e) e2m1(k_e)
 // in fp32, i.e. the indexer's per-head dot product before the ReLU.  The epilogue applies
 // s = sum_h w'[h] * max(0, D[key][h]) with w' = w * g_q * g_k.
 //
 // Warp roles (192 threads, persistent over a contiguous range of key tiles of one query row):
-//   warp 0      TMA producer: 128 x 64 B FP4 code tile (2-D tensor map, 64-byte swizzle) and the
-//               tile's 512 B of key scales (bulk copy) into a STAGES-deep shared-memory ring;
+//   warp 0      TMA producer: 256 x 64 B FP4 code tile (2-D tensor map, 64-byte swizzle) and the
+//               tile's 1 KB of key scales (bulk copy) into a STAGES-deep shared-memory ring;
 //   warp 1      allocates tensor memory and issues the MMAs (one thread);
-//   warps 2..5  write each tile's scale factors into tensor memory (tcgen05.st), then read the
-//               previous tile's accumulator (tcgen05.ld), compute the scores, store them and count
-//               them in the row histogram used by the top-k.
-// Every wait is bounded; on a timeout the kernel records CSA device error 1 and leaves.
+//   warps 2..5  write tile i's scale factors into tensor memory (tcgen05.st) while the accumulator of
+//               tile i - LAG is being read (tcgen05.ld), then compute those scores, store them and
+//               count them in the row histogram used by the top-k.
+// Tensor memory holds a ring of NBUF tiles of scale factors and accumulators, so up to LAG MMAs are
+// in flight behind the epilogue.  Every wait is bounded; on a timeout the kernel records device
+// error 1 (csa_device_status) and leaves.
 #include "csa_common.cuh"
 #include "sm100.cuh"
 
@@ -26,18 +29,18 @@ namespace csa {
 
 using namespace sm100;
 
-constexpr int TC_STAGES = 6;
-constexpr int TC_TILE = 128;                     // keys per tile (MMA M)
-constexpr int TC_CODE_BYTES = TC_TILE * 64;      // 128 keys x 128 FP4
-constexpr int TC_SC_BYTES = TC_TILE * 4;         // 128 keys x 4 E4M3 scales
+constexpr int TC_STAGES = 4;
+constexpr int TC_SUB = 128;                      // keys per MMA (M)
+constexpr int TC_TILE = 2 * TC_SUB;              // keys per TMA box / pipeline step
+constexpr int TC_CODE_BYTES = TC_TILE * 64;      // 256 keys x 128 FP4
+constexpr int TC_SC_BYTES = TC_TILE * 4;         // 256 keys x 4 E4M3 scales
 constexpr int TC_THREADS = 192;
-constexpr uint32_t TC_TMEM_COLS = 64;
-constexpr uint32_t TC_COL_D = 0;                 // 2 accumulators x 8 columns
-constexpr uint32_t TC_COL_SFA = 16;              // 2 buffers x 2 atoms x 4 columns
-constexpr uint32_t TC_COL_SFB = 32;              // 2 atoms x 4 columns
+constexpr int TC_NBUF = 4, TC_LAG = 2;
+constexpr uint32_t TC_TMEM_COLS = 256;
+constexpr uint32_t TC_COL_D = 0;                 // NBUF x (2 sub-tiles x 8 heads)
+constexpr uint32_t TC_COL_SFA = 64;              // NBUF x (2 sub-tiles x 2 atoms x 4 columns)
+constexpr uint32_t TC_COL_SFB = 128;             // 2 atoms x 4 columns
 constexpr int TC_HIST_BINS = 4096, TC_HIST_SHIFT = 20;
-
-__device__ uint32_t g_csa_device_error = 0;
 
 struct TcSmem {
   alignas(1024) uint8_t codes[TC_STAGES][TC_CODE_BYTES];
@@ -48,9 +51,10 @@ struct TcSmem {
   uint8_t qsc[8][4];
   alignas(8) uint64_t full[TC_STAGES];
   alignas(8) uint64_t empty[TC_STAGES];
-  alignas(8) uint64_t sfa_full[2];
-  alignas(8) uint64_t acc_full[2];
-  alignas(8) uint64_t acc_empty[2];
+  alignas(8) uint64_t sfa_full[TC_NBUF];
+  alignas(8) uint64_t acc_full[TC_NBUF];
+  alignas(8) uint64_t acc_empty[TC_NBUF];
+  alignas(8) uint64_t q_ready;              // query tile, its scale factors and weights are in place
   uint32_t tmem_base;
   uint32_t err;
 };
@@ -98,36 +102,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
   if (threadIdx.x == 0) {
     S.err = 0;
     for (int s = 0; s < TC_STAGES; ++s) { mbar_init(&S.full[s], 1); mbar_init(&S.empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&S.sfa_full[a], 4); mbar_init(&S.acc_full[a], 1); mbar_init(&S.acc_empty[a], 4); }
+    for (int a = 0; a < TC_NBUF; ++a) {
+      mbar_init(&S.sfa_full[a], 4);
+      mbar_init(&S.acc_full[a], 1);
+      mbar_init(&S.acc_empty[a], 4);
+    }
+    mbar_init(&S.q_ready, 4);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) prefetch_tensormap(&kmap);
   for (int i = threadIdx.x; i < TC_HIST_BINS; i += blockDim.x) S.hist[i] = 0;
   if (warp == 1) { tmem_alloc(&S.tmem_base, TC_TMEM_COLS); tmem_relinquish(); }
-  // query: FP4 B tile (8 heads x 64 B, 64-byte swizzle), its scales, the head weights
-  if (warp >= 2) {
-    const int t = threadIdx.x - 64;          // 0..127
-    const int wg = t >> 5;                   // 0..3: heads 2wg, 2wg+1
-    for (int hh = 0; hh < 2; ++hh) {
-      const int h = 2 * wg + hh;
-      for (int blk = 0; blk < 4; ++blk) {
-        uint32_t code = 0, s_code = 0;
-        if (h < P.H_I) {
-          const float x = bf16_bits_to_f(P.q_I[((size_t)b * P.H_I + h) * 128 + blk * 32 + lane]);
-          code = quant_lane(x, P.g_q, &s_code);
-        }
-        const uint32_t pair = code | (__shfl_down_sync(0xffffffffu, code, 1) << 4);
-        if ((lane & 1) == 0) {
-          const int byte = blk * 16 + (lane >> 1);               // byte of the 64-byte row
-          const int c = byte >> 4;
-          S.qtile[h * 64 + ((c ^ ((h >> 1) & 3)) << 4) + (byte & 15)] = (uint8_t)pair;
-        }
-        if (lane == 0) S.qsc[h][blk] = (uint8_t)s_code;
-      }
-      if (lane == 0) S.wq[h] = h < P.H_I ? P.w[(size_t)b * P.H_I + h] * P.gg : 0.0f;
-    }
-    fence_proxy_async_smem();
-  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = S.tmem_base;
@@ -158,21 +143,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_mxf4_ue4m3(TC_TILE, 8);
+      const uint32_t idesc = idesc_mxf4_ue4m3(TC_SUB, 8);
       const uint32_t qa = smem_addr(S.qtile);
+      if (ntile > 0 && !mbar_wait(&S.q_ready, 0)) ok = false;
       for (int i = 0; i < ntile && ok; ++i) {
-        const int s = i % TC_STAGES, a = i & 1;
+        const int s = i % TC_STAGES, a = i % TC_NBUF, use = i / TC_NBUF;
         if (!mbar_wait(&S.full[s], (i / TC_STAGES) & 1)) { ok = false; break; }
-        if (!mbar_wait(&S.sfa_full[a], (i >> 1) & 1)) { ok = false; break; }
-        if (i >= 2 && !mbar_wait(&S.acc_empty[a], ((i >> 1) - 1) & 1)) { ok = false; break; }
+        if (!mbar_wait(&S.sfa_full[a], use & 1)) { ok = false; break; }
+        if (use > 0 && !mbar_wait(&S.acc_empty[a], (use - 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ca = smem_addr(S.codes[s]);
-        for (int k = 0; k < 2; ++k) {
-          const uint64_t ad = smem_desc(ca + 32 * k, 16, 512, LAYOUT_SW64);
-          const uint64_t bd = smem_desc(qa + 32 * k, 16, 512, LAYOUT_SW64);
-          mma_mxf4(tbase + TC_COL_D + 8 * a, ad, bd, idesc, tbase + TC_COL_SFA + 8 * a + 4 * k,
-                   tbase + TC_COL_SFB + 4 * k, k > 0);
-        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const uint64_t ad = smem_desc(ca + u * (TC_SUB * 64) + 32 * k, 16, 512, LAYOUT_SW64);
+            const uint64_t bd = smem_desc(qa + 32 * k, 16, 512, LAYOUT_SW64);
+            mma_mxf4(tbase + TC_COL_D + 16 * a + 8 * u, ad, bd, idesc, tbase + TC_COL_SFA + 16 * a + 8 * u + 4 * k,
+                     tbase + TC_COL_SFB + 4 * k, k > 0);
+          }
         mma_commit(&S.acc_full[a]);
         mma_commit(&S.empty[s]);
       }
@@ -183,62 +172,106 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
     // ------------------------------------------------------ scale factors + epilogue
     const int q = warp & 3;                                      // tensor-memory lane quadrant
     const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
-    float wq[8];
-#pragma unroll
-    for (int h = 0; h < 8; ++h) wq[h] = S.wq[h];
     {
-      // query scale factors, written once: row h (< 8) at lane h of every quadrant, column j = 0
+      // query: FP4 B tile (8 heads x 64 B, 64-byte swizzle), its scales and the head weights; warp
+      // wg = warp - 2 takes heads 2wg, 2wg+1 (all eight loads issued before any use)
+      const int wg = warp - 2;
+      float x[2][4];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+          const int h = 2 * wg + hh;
+          x[hh][blk] = h < P.H_I ? bf16_bits_to_f(P.q_I[((size_t)b * P.H_I + h) * 128 + blk * 32 + lane]) : 0.0f;
+        }
+      const float wv = (lane < 2 && 2 * wg + lane < P.H_I) ? P.w[(size_t)b * P.H_I + 2 * wg + lane] * P.gg : 0.0f;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int h = 2 * wg + hh;
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+          uint32_t s_code = 0;
+          const uint32_t code = quant_lane(x[hh][blk], P.g_q, &s_code);   // zero heads give code 0, scale 0
+          const uint32_t pair = code | (__shfl_down_sync(0xffffffffu, code, 1) << 4);
+          if ((lane & 1) == 0) {
+            const int byte = blk * 16 + (lane >> 1);             // byte of the 64-byte row
+            const int c = byte >> 4;
+            S.qtile[h * 64 + ((c ^ ((h >> 1) & 3)) << 4) + (byte & 15)] = (uint8_t)pair;
+          }
+          if (lane == 0) S.qsc[h][blk] = (uint8_t)s_code;
+        }
+      }
+      if (lane < 2) S.wq[2 * wg + lane] = wv;
+      fence_proxy_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");             // the four epilogue warps
+      // query scale factors: row h (< 8) at lane h of every quadrant, column j = 0
       uint32_t w0 = 0, w1 = 0;
       if (lane < 8) {
-        const uint32_t* s4 = reinterpret_cast<const uint32_t*>(S.qsc[lane]);
-        const uint32_t v = *s4;
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(S.qsc[lane]);
         w0 = __byte_perm(v, 0, 0x1100);
         w1 = __byte_perm(v, 0, 0x3322);
       }
       tmem_st_x4(lane_base + TC_COL_SFB + 0, w0, 0, 0, 0);
       tmem_st_x4(lane_base + TC_COL_SFB + 4, w1, 0, 0, 0);
-    }
-    float* srow = P.scores + (size_t)b * P.ld;
-    auto epilogue = [&](int i) -> bool {
-      const int a = i & 1;
-      if (!mbar_wait(&S.acc_full[a], (i >> 1) & 1)) return false;
-      tc_fence_after();
-      float d[8];
-      tmem_ld_x8(lane_base + TC_COL_D + 8 * a, d);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.acc_empty[a]);
-      const int key = (t_begin + i) * TC_TILE + 32 * q + lane;
-      if (key < n_vis) {
-        float sc = 0.f;
-#pragma unroll
-        for (int h = 0; h < 8; ++h) sc = fmaf(wq[h], fmaxf(d[h], 0.f), sc);
-        sc += 0.0f;
-        srow[key] = sc;
-        if (P.hist) atomicAdd(&S.hist[float_order_key(sc) >> TC_HIST_SHIFT], 1u);
-      }
-      return true;
-    };
-    for (int i = 0; i < ntile && ok; ++i) {
-      const int s = i % TC_STAGES, a = i & 1;
-      if (!mbar_wait(&S.full[s], (i / TC_STAGES) & 1)) { ok = false; break; }
-      // key scale factors of tile i: lane L of every quadrant holds rows L%32 + 32j, j = column
-      const uint32_t* sc = reinterpret_cast<const uint32_t*>(S.sc[s]);
-      uint32_t v[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = sc[lane + 32 * j];
-      tmem_st_x4(lane_base + TC_COL_SFA + 8 * a + 0, __byte_perm(v[0], 0, 0x1100), __byte_perm(v[1], 0, 0x1100),
-                 __byte_perm(v[2], 0, 0x1100), __byte_perm(v[3], 0, 0x1100));
-      tmem_st_x4(lane_base + TC_COL_SFA + 8 * a + 4, __byte_perm(v[0], 0, 0x3322), __byte_perm(v[1], 0, 0x3322),
-                 __byte_perm(v[2], 0, 0x3322), __byte_perm(v[3], 0, 0x3322));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.sfa_full[a]);
-      if (i >= 1 && !epilogue(i - 1)) { ok = false; break; }
+      if (lane == 0) mbar_arrive(&S.q_ready);
     }
-    if (ok && ntile > 0 && !epilogue(ntile - 1)) ok = false;
+    float wq[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) wq[h] = S.wq[h];
+    float* srow = P.scores + (size_t)b * P.ld;
+    uint32_t d[16];
+    auto finish = [&](int i) {
+      // d holds tile i's accumulators (issued by the caller): release them, then score
+      tmem_wait_ld_x16(d);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.acc_empty[i % TC_NBUF]);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int key = (t_begin + i) * TC_TILE + TC_SUB * u + 32 * q + lane;
+        if (key < n_vis) {
+          float sc = 0.f;
+#pragma unroll
+          for (int h = 0; h < 8; ++h) sc = fmaf(wq[h], fmaxf(__uint_as_float(d[8 * u + h]), 0.f), sc);
+          sc += 0.0f;
+          srow[key] = sc;
+          if (P.hist) atomicAdd(&S.hist[float_order_key(sc) >> TC_HIST_SHIFT], 1u);
+        }
+      }
+    };
+    for (int i = 0; i < ntile + TC_LAG && ok; ++i) {
+      const int e = i - TC_LAG;                                  // tile whose accumulators are read now
+      if (e >= 0) {
+        if (!mbar_wait(&S.acc_full[e % TC_NBUF], (e / TC_NBUF) & 1)) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld_x16(lane_base + TC_COL_D + 16 * (e % TC_NBUF), d);
+      }
+      if (i < ntile) {
+        const int s = i % TC_STAGES, a = i % TC_NBUF;
+        if (!mbar_wait(&S.full[s], (i / TC_STAGES) & 1)) { ok = false; break; }
+        // key scale factors of tile i: sub-tile u, lane L of every quadrant holds rows L%32 + 32j
+        const uint32_t* sc = reinterpret_cast<const uint32_t*>(S.sc[s]);
+        uint32_t v[8], wsf[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = sc[lane + 32 * j];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            wsf[8 * u + j] = __byte_perm(v[4 * u + j], 0, 0x1100);       // atom k = 0: blocks 0,0,1,1
+            wsf[8 * u + 4 + j] = __byte_perm(v[4 * u + j], 0, 0x3322);   // atom k = 1: blocks 2,2,3,3
+          }
+        tmem_st_x16(lane_base + TC_COL_SFA + 16 * a, wsf);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.sfa_full[a]);
+      }
+      if (e >= 0) finish(e);
+    }
     if (!ok && lane == 0) atomicOr(&S.err, 1u);
   }
   __syncthreads();
@@ -305,9 +338,9 @@ csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, u
   P.H_I = a->H_I;
   P.g_q = a->g_q;
   P.gg = a->g_q * a->g_k;
-  // about two CTAs per SM in total, at most one per tile
+  // at most two resident CTAs per SM (256 tensor-memory columns each): one wave, at most one per tile
   const int tiles_row = (a->n_max + TC_TILE - 1) / TC_TILE;
-  int per_row = (2 * 148 + a->B - 1) / a->B;
+  int per_row = (2 * 148) / a->B;
   if (per_row > tiles_row) per_row = tiles_row;
   if (per_row < 1) per_row = 1;
   P.ctas_per_row = per_row;
@@ -318,17 +351,17 @@ csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, u
   return launch_status();
 }
 
+cudaError_t compress_take_device_error(uint32_t* out);   // compress.cu
+cudaError_t attn_take_device_error(uint32_t* out);       // attn_tc.cu
+
 }  // namespace csa
 
 extern "C" csa_status csa_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
-  if (e != cudaSuccess) {
-    csa::set_last_cuda_error(e);
-    return CSA_ERR_CUDA;
-  }
-  uint32_t v = 0, zero = 0;
-  e = cudaMemcpyFromSymbol(&v, csa::g_csa_device_error, sizeof(v));
-  if (e == cudaSuccess && v) e = cudaMemcpyToSymbol(csa::g_csa_device_error, &zero, sizeof(zero));
+  uint32_t v = 0;
+  if (e == cudaSuccess) e = csa::take_device_error_here(&v);
+  if (e == cudaSuccess) e = csa::compress_take_device_error(&v);
+  if (e == cudaSuccess) e = csa::attn_take_device_error(&v);
   if (e != cudaSuccess) {
     csa::set_last_cuda_error(e);
     return CSA_ERR_CUDA;
