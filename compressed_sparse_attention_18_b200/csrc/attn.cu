@@ -346,8 +346,17 @@ __global__ void __launch_bounds__(AT_WARPS * 32, 1) attn_kernel(AttnParams P) {
 // Merge split partials: lse = log sum_s exp(lse_s); out = sum_s exp(lse_s - lse) O_s.
 // One CTA per (query, head); each thread owns 4 consecutive output dims, the split weights are
 // computed once per CTA in shared memory.
-constexpr int MERGE_MAX_SPLITS = 64;
-__global__ void __launch_bounds__(128) attn_merge_kernel(const float* __restrict__ part_o,
+constexpr int MERGE_MAX_SPLITS = 128;
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4(const uint16_t* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
+                     __uint_as_float(u.y & 0xFFFF0000u));
+}
+
+// Partials in fp32 (CUDA-core path) or bf16 (tensor-core path).
+template <typename PT>
+__global__ void __launch_bounds__(128) attn_merge_kernel(const PT* __restrict__ part_o,
                                                          const float* __restrict__ part_lse, int splits, int H, int D,
                                                          uint16_t* __restrict__ out, float* __restrict__ lse) {
   __shared__ float s_w[MERGE_MAX_SPLITS];
@@ -376,7 +385,7 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const float* __restrict
     for (int s = 0; s < splits; ++s) {
       const float wgt = s_w[s];
       if (wgt == 0.f) continue;
-      const float4 v = *reinterpret_cast<const float4*>(part_o + (((size_t)bq * splits + s) * H + h) * D + d4);
+      const float4 v = load4(part_o + (((size_t)bq * splits + s) * H + h) * D + d4);
       acc.x = fmaf(wgt, v.x, acc.x); acc.y = fmaf(wgt, v.y, acc.y);
       acc.z = fmaf(wgt, v.z, acc.z); acc.w = fmaf(wgt, v.w, acc.w);
     }
@@ -389,9 +398,10 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const float* __restrict
 }
 
 // tensor-core decode path (attn_tc.cu)
-bool attn_tc_eligible(const csa_attn_args* a, int hca, long long rows);
-int attn_tc_splits(const csa_attn_args* a);
-csa_status launch_attn_tc(const csa_attn_args* a, int splits, float* part_o, float* part_lse, cudaStream_t st);
+bool attn_tc_eligible(const csa_attn_args* a, int hca, int max_splits);
+int attn_tc_splits(const csa_attn_args* a, int hca);
+csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, uint16_t* part_o, float* part_lse,
+                          cudaStream_t st);
 
 struct AttnPlan {
   int splits, cps;
@@ -402,14 +412,14 @@ struct AttnPlan {
 static AttnPlan plan_attn(const csa_attn_args* a, int hca) {
   AttnPlan p{};
   const long long rows_tc = (long long)a->B * a->Nq;
-  if (attn_tc_eligible(a, hca, rows_tc)) {
+  if (attn_tc_eligible(a, hca, MERGE_MAX_SPLITS)) {
     p.tc = true;
     p.cps = 1;
-    p.splits = attn_tc_splits(a);
+    p.splits = attn_tc_splits(a, hca);
     if (p.splits < 1) p.splits = 1;
     size_t o = 0;
     if (p.splits > 1) {
-      p.off_o = o;   o = align_up(o + (size_t)rows_tc * p.splits * a->H * a->d * 4, 256);
+      p.off_o = o;   o = align_up(o + (size_t)rows_tc * p.splits * a->H * a->d * 2, 256);
       p.off_lse = o; o = align_up(o + (size_t)rows_tc * p.splits * a->H * 4, 256);
     }
     p.total = o;
@@ -473,11 +483,12 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
   CSA_REQUIRE(p.total == 0 || ws != nullptr);
   cudaStream_t st = (cudaStream_t)stream;
   if (p.tc) {
-    float* po = p.splits > 1 ? (float*)((uint8_t*)ws + p.off_o) : nullptr;
+    uint16_t* po = p.splits > 1 ? (uint16_t*)((uint8_t*)ws + p.off_o) : nullptr;
     float* pl = p.splits > 1 ? (float*)((uint8_t*)ws + p.off_lse) : nullptr;
-    csa_status s = launch_attn_tc(a, p.splits, po, pl, st);
+    csa_status s = launch_attn_tc(a, hca, p.splits, po, pl, st);
     if (s != CSA_OK || p.splits == 1) return s;
-    attn_merge_kernel<<<(unsigned)(rows * a->H), 128, 0, st>>>(po, pl, p.splits, a->H, a->d, (uint16_t*)a->out, a->lse);
+    attn_merge_kernel<uint16_t><<<(unsigned)(rows * a->H), 128, 0, st>>>(po, pl, p.splits, a->H, a->d,
+                                                                         (uint16_t*)a->out, a->lse);
     return launch_status();
   }
   AttnParams P{};
@@ -499,8 +510,8 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
   else
     s = launch_attn<128, 8>(P, units, st);
   if (s != CSA_OK || p.splits == 1) return s;
-  attn_merge_kernel<<<(unsigned)(rows * a->H), 128, 0, st>>>(P.part_o, P.part_lse, p.splits, a->H, a->d,
-                                                               (uint16_t*)a->out, a->lse);
+  attn_merge_kernel<float><<<(unsigned)(rows * a->H), 128, 0, st>>>(P.part_o, P.part_lse, p.splits, a->H, a->d,
+                                                                      (uint16_t*)a->out, a->lse);
   return launch_status();
 }
 

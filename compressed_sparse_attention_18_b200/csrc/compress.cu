@@ -139,13 +139,18 @@ __global__ void __launch_bounds__(256) gemm_bf16_kernel(const uint16_t* __restri
 }
 
 // --------------------------------------------------------------------------------------- pooling
-// One CTA per (sequence, group of POOL_ENT entries).  Threads walk the d channels: per-channel softmax
-// over the r slots of (Z + b_pos), weighted sum of C (all loads of a channel issued together when
-// r <= 8; an online softmax streams longer groups); RoPE on the last d_r channels at the group-start
-// position (angle and rotation in double); bf16 round; k_I = bf16(c · W_IK) with W_IK brought into
-// shared memory by one bulk copy issued at kernel start (it lands while the pooling runs); optionally
-// the FP4 pack of c and k_I straight into the caches.
+// One CTA per (sequence, group of POOL_ENT entries, slice of OW indexer-key outputs).  Threads walk the
+// d channels: per-channel softmax over the r slots of (Z + b_pos), weighted sum of C (all loads of a
+// channel issued together when r <= 8; an online softmax streams longer groups); RoPE on the last d_r
+// channels at the group-start position (the angle pos * theta^(-2m/d_r) and its reduction mod 2 pi in
+// double, computed while the pooling loads are in flight; sin / cos of the reduced angle and the
+// rotation in single precision); bf16 round; optionally the FP4 pack of c straight into the cache (slice
+// 0 only); k_I[slice] = bf16(c · W_IK[:, slice]) with W_IK read from global memory (for short channel
+// loops the slice is loaded into registers at kernel start), and its FP4 blocks packed into the cache.
 constexpr int POOL_ENT = 4;
+constexpr int POOL_THREADS = 256;
+constexpr int POOL_WARPS = POOL_THREADS / 32;
+constexpr int POOL_MAX_HALF = 32;   // RoPE pairs per row
 
 struct PoolParams {
   const uint16_t* C;
@@ -159,6 +164,7 @@ struct PoolParams {
   uint16_t* c_out;
   uint16_t* kI_out;
   csa_fp4_cache kv, ki;
+  double inv_freq[POOL_MAX_HALF];   // theta^(-2m/d_r), m < d_r/2
 };
 
 __device__ __forceinline__ void pack_row_to_cache(const float* row, int d, int d_r, const csa_fp4_cache& cc, int b,
@@ -175,53 +181,98 @@ __device__ __forceinline__ void pack_row_to_cache(const float* row, int d, int d
     reinterpret_cast<uint16_t*>(cc.rope)[dst * d_r + e] = (uint16_t)(__float_as_uint(row[d_n + e]) >> 16);
 }
 
-__global__ void __launch_bounds__(256) pool_kernel(PoolParams P) {
-  // shared memory: pooled [POOL_ENT][d] fp32 | W_IK [d][d_I] bf16 | partial sums [2][POOL_ENT][d_I] | k_I rows
-  extern __shared__ __align__(128) float pooled[];
-  __shared__ __align__(8) uint64_t w_bar;
-  const int b = blockIdx.y;
-  const int d = P.d, d_r = P.d_r, r = P.r, T = P.T, d_I = P.d_I;
-  uint16_t* w_s = reinterpret_cast<uint16_t*>(pooled + POOL_ENT * d);
-  if (P.W_IK != nullptr && threadIdx.x == 0) {
-    // the whole projection matrix arrives while the pooling runs
-    sm100::mbar_init(&w_bar, 1);
-    sm100::fence_mbar_init();
-    const uint32_t bytes = (uint32_t)d * d_I * 2;
-    sm100::mbar_arrive_expect_tx(&w_bar, bytes);
-    for (uint32_t off = 0; off < bytes; off += 32768)
-      sm100::bulk_load(reinterpret_cast<uint8_t*>(w_s) + off, reinterpret_cast<const uint8_t*>(P.W_IK) + off,
-                       min(32768u, bytes - off), &w_bar);
+__device__ __forceinline__ void fma8_bf16(float* acc, float p, const uint4& w) {
+  const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    acc[2 * k] = fmaf(p, __uint_as_float(ww[k] << 16), acc[2 * k]);
+    acc[2 * k + 1] = fmaf(p, __uint_as_float(ww[k] & 0xFFFF0000u), acc[2 * k + 1]);
   }
+}
+
+// OW: indexer-key outputs per CTA (32, 64 or 128); PRE: channels per thread when the W_IK slice is
+// preloaded into registers (0: streamed).
+template <int OW, int PRE>
+__global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
+  constexpr int NOC = OW / 8;                       // 8-output chunks of the slice
+  constexpr int NCHP = POOL_THREADS / NOC;          // channel phases
+  // shared memory: pooled [POOL_ENT][d] fp32 | red [POOL_WARPS][POOL_ENT][OW] | k_I rows [POOL_ENT][OW]
+  extern __shared__ __align__(128) float pooled[];
+  const int b = blockIdx.y, z = blockIdx.z;
+  const int d = P.d, d_r = P.d_r, r = P.r, T = P.T, d_I = P.d_I;
   const int n_out = T / r;
   const int e0 = blockIdx.x * POOL_ENT;
   const int ne = min(POOL_ENT, n_out - e0);
   const int d_n = d - d_r;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int oc = tid % NOC, chp = tid / NOC;
+  const int o_base = z * OW + oc * 8;
+  // W_IK slice into registers first (its latency overlaps the pooling)
+  uint4 wpre[PRE > 0 ? PRE : 1];
+  if (PRE > 0 && P.W_IK) {
+#pragma unroll
+    for (int i = 0; i < PRE; ++i) {
+      const int ch = chp + NCHP * i;
+      wpre[i] = ch < d ? __ldg(reinterpret_cast<const uint4*>(P.W_IK + (size_t)ch * d_I + o_base))
+                       : make_uint4(0, 0, 0, 0);
+    }
+  }
+  // RoPE angle of this thread's (entry, pair): pos * inv_freq and its reduction mod 2 pi in double, then
+  // sin / cos of the reduced angle (|a| <= pi) in single precision
+  const int half = d_r >> 1;
+  const long long p0 = P.pos0 ? P.pos0[b] : 0;
+  const bool rope_thread = P.theta != 0.0f && tid < ne * half;
+  float rs_sn = 0.f, rs_cs = 1.f;
+  auto rope_angle = [&]() {
+    const int q = tid / half, mm = tid % half;
+    const double ang = (double)(p0 + (long long)(e0 + q) * r) * P.inv_freq[mm];
+    const double kk = rint(ang * 0.15915494309189535);              // 1 / (2 pi)
+    double red = fma(-kk, 6.283185307179586, ang);                   // 2 pi, high part
+    red = fma(-kk, 2.4492935982947064e-16, red);                     // 2 pi, low part
+    sincosf((float)red, &rs_sn, &rs_cs);
+  };
   const uint16_t* __restrict__ C = P.C;
   const uint16_t* __restrict__ Z = P.Z;
   const float* __restrict__ b_pos = P.b_pos;
-  for (int i = threadIdx.x; i < ne * d; i += blockDim.x) {
-    const int q = i / d, ch = i % d;
-    const size_t tok0 = (size_t)b * T + (size_t)(e0 + q) * r;
-    float res;
-    if (r <= 8) {
-      float a[8], c[8];
+  if (r <= 8) {
+    // two channels per thread per round, all their loads issued before any arithmetic
+    for (int i0 = tid; i0 < ne * d; i0 += 2 * POOL_THREADS) {
+      float a[2][8], c[2][8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        a[j] = j < r ? bf16_bits_to_f(Z[(tok0 + j) * d + ch]) + b_pos[(size_t)j * d + ch] : -INFINITY;
-        c[j] = j < r ? bf16_bits_to_f(C[(tok0 + j) * d + ch]) : 0.f;
+      for (int u = 0; u < 2; ++u) {
+        const int i = min(i0 + u * POOL_THREADS, ne * d - 1);
+        const int q = i / d, ch = i % d;
+        const size_t tok0 = (size_t)b * T + (size_t)(e0 + q) * r;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          a[u][j] = j < r ? bf16_bits_to_f(Z[(tok0 + j) * d + ch]) + b_pos[(size_t)j * d + ch] : -INFINITY;
+          c[u][j] = j < r ? bf16_bits_to_f(C[(tok0 + j) * d + ch]) : 0.f;
+        }
       }
-      float m = a[0];
+      if (i0 == tid && rope_thread) rope_angle();    // overlaps the loads of the first round
 #pragma unroll
-      for (int j = 1; j < 8; ++j) m = fmaxf(m, a[j]);
-      float l = 0.f, acc = 0.f;
+      for (int u = 0; u < 2; ++u) {
+        const int i = i0 + u * POOL_THREADS;
+        if (i >= ne * d) continue;
+        float m = a[u][0];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float p = j < r ? __expf(a[j] - m) : 0.f;
-        l += p;
-        acc = fmaf(p, c[j], acc);
+        for (int j = 1; j < 8; ++j) m = fmaxf(m, a[u][j]);
+        float l = 0.f, acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float p = j < r ? __expf(a[u][j] - m) : 0.f;
+          l += p;
+          acc = fmaf(p, c[u][j], acc);
+        }
+        pooled[i] = acc / l;
       }
-      res = acc / l;
-    } else {
+    }
+    if (ne * d <= tid && rope_thread) rope_angle();
+  } else {
+    if (rope_thread) rope_angle();
+    for (int i = tid; i < ne * d; i += POOL_THREADS) {
+      const int q = i / d, ch = i % d;
+      const size_t tok0 = (size_t)b * T + (size_t)(e0 + q) * r;
       float m = -INFINITY, l = 0.f, acc = 0.f;
       for (int j = 0; j < r; ++j) {
         const float a = bf16_bits_to_f(Z[(tok0 + j) * d + ch]) + b_pos[(size_t)j * d + ch];
@@ -236,72 +287,87 @@ __global__ void __launch_bounds__(256) pool_kernel(PoolParams P) {
         l += p;
         acc = fmaf(p, c, acc);
       }
-      res = acc / l;
+      pooled[i] = acc / l;
     }
-    pooled[q * d + ch] = res;
   }
   __syncthreads();
-  const int half = d_r >> 1;
-  const long long p0 = P.pos0 ? P.pos0[b] : 0;
-  if (P.theta != 0.0f) {
-    const double l2t = log2((double)P.theta);
-    for (int i = threadIdx.x; i < ne * half; i += blockDim.x) {
-      const int q = i / half, mm = i % half;
-      float* row = pooled + q * d;
-      const double p = (double)(p0 + (long long)(e0 + q) * r);
-      const double inv_freq = exp2(-2.0 * mm / (double)d_r * l2t);
-      double sn, cs;
-      sincos(p * inv_freq, &sn, &cs);
-      const double x1 = row[d_n + mm], x2 = row[d_n + half + mm];
-      row[d_n + mm] = (float)(x1 * cs - x2 * sn);
-      row[d_n + half + mm] = (float)(x1 * sn + x2 * cs);
-    }
-    __syncthreads();
+  if (rope_thread) {
+    const int q = tid / half, mm = tid % half;
+    float* row = pooled + q * d;
+    const float x1 = row[d_n + mm], x2 = row[d_n + half + mm];
+    row[d_n + mm] = fmaf(x1, rs_cs, -x2 * rs_sn);
+    row[d_n + half + mm] = fmaf(x1, rs_sn, x2 * rs_cs);
   }
-  for (int i = threadIdx.x; i < ne * d; i += blockDim.x) {
+  __syncthreads();
+  for (int i = tid; i < ne * d; i += POOL_THREADS) {
     const int q = i / d, ch = i % d;
     const uint32_t bits = f_to_bf16_bits(pooled[i]);
-    if (P.c_out) P.c_out[((size_t)b * n_out + e0 + q) * d + ch] = (uint16_t)bits;
+    if (P.c_out && z == 0) P.c_out[((size_t)b * n_out + e0 + q) * d + ch] = (uint16_t)bits;
     pooled[i] = bf16_bits_to_f(bits);
   }
   __syncthreads();
-  if (P.kv.codes)
+  if (P.kv.codes && z == 0)
     for (int q = 0; q < ne; ++q) pack_row_to_cache(pooled + q * d, d, d_r, P.kv, b, e0 + q);
   if (P.W_IK == nullptr) return;
-  // k_I = c · W_IK from shared memory: thread (o, part) sums output o over the channels part, part + 2, ...
-  const bool w_ok = sm100::mbar_wait(&w_bar, 0);
-  if (!w_ok && threadIdx.x == 0) atomicOr(&g_csa_device_error, 1u);
-  float* red = reinterpret_cast<float*>(w_s + (size_t)d * d_I);     // [S][POOL_ENT][d_I], then the k_I rows
-  const int S = blockDim.x / d_I;                                    // d_I divides 256 (64 or 128)
-  {
-    const int o = threadIdx.x % d_I, part = threadIdx.x / d_I;
-    float acc[POOL_ENT];
+  // k_I slice: thread (oc, chp) sums outputs o_base..o_base+7 over channels chp, chp + NCHP, ...
+  float* red = pooled + POOL_ENT * d;               // [POOL_WARPS][POOL_ENT][OW]
+  float* krow = red + POOL_WARPS * POOL_ENT * OW;   // [POOL_ENT][OW]
+  float acc[POOL_ENT][8];
 #pragma unroll
-    for (int q = 0; q < POOL_ENT; ++q) acc[q] = 0.f;
-    if (w_ok) {
-#pragma unroll 8
-      for (int ch = part; ch < d; ch += S) {
-        const float wv = bf16_bits_to_f(w_s[(size_t)ch * d_I + o]);
+  for (int q = 0; q < POOL_ENT; ++q)
 #pragma unroll
-        for (int q = 0; q < POOL_ENT; ++q) acc[q] = fmaf(pooled[q * d + ch], wv, acc[q]);
-      }
+    for (int k = 0; k < 8; ++k) acc[q][k] = 0.f;
+  if (PRE > 0) {
+#pragma unroll
+    for (int i = 0; i < PRE; ++i) {
+      const int ch = chp + NCHP * i;
+      if (ch < d)
+#pragma unroll
+        for (int q = 0; q < POOL_ENT; ++q)
+          if (q < ne) fma8_bf16(acc[q], pooled[q * d + ch], wpre[i]);
     }
+  } else {
+#pragma unroll 4
+    for (int ch = chp; ch < d; ch += NCHP) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(P.W_IK + (size_t)ch * d_I + o_base));
 #pragma unroll
-    for (int q = 0; q < POOL_ENT; ++q) red[((size_t)part * POOL_ENT + q) * d_I + o] = acc[q];
+      for (int q = 0; q < POOL_ENT; ++q)
+        if (q < ne) fma8_bf16(acc[q], pooled[q * d + ch], w);
+    }
   }
+  // reduce over the channel phases: lanes NOC apart inside the warp, then the warps through smem
+#pragma unroll
+  for (int off = NOC; off < 32; off <<= 1)
+#pragma unroll
+    for (int q = 0; q < POOL_ENT; ++q)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[q][k] += __shfl_xor_sync(0xffffffffu, acc[q][k], off);
+  if (lane < NOC)
+#pragma unroll
+    for (int q = 0; q < POOL_ENT; ++q)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) red[(warp * POOL_ENT + q) * OW + oc * 8 + k] = acc[q][k];
   __syncthreads();
-  float* krow = red + S * POOL_ENT * d_I;          // [POOL_ENT][d_I]
-  for (int i = threadIdx.x; i < ne * d_I; i += blockDim.x) {
-    const int q = i / d_I, jj = i % d_I;
+  for (int i = tid; i < ne * OW; i += POOL_THREADS) {
+    const int q = i / OW, o = i % OW;
     float v = 0.f;
-    for (int pp = 0; pp < S; ++pp) v += red[((size_t)pp * POOL_ENT + q) * d_I + jj];
+#pragma unroll
+    for (int w = 0; w < POOL_WARPS; ++w) v += red[(w * POOL_ENT + q) * OW + o];
     const uint32_t bits = f_to_bf16_bits(v);
-    if (P.kI_out) P.kI_out[((size_t)b * n_out + e0 + q) * d_I + jj] = (uint16_t)bits;
-    krow[q * d_I + jj] = bf16_bits_to_f(bits);
+    if (P.kI_out) P.kI_out[((size_t)b * n_out + e0 + q) * d_I + z * OW + o] = (uint16_t)bits;
+    krow[q * OW + o] = bf16_bits_to_f(bits);
   }
   if (P.ki.codes) {
     __syncthreads();
-    for (int q = 0; q < ne; ++q) pack_row_to_cache(krow + q * d_I, d_I, 0, P.ki, b, e0 + q);
+    const csa_fp4_cache& cc = P.ki;
+    const int S = d_I / 32, S_pad = (S + 3) & ~3;
+    for (int t = warp; t < ne * (OW / 32); t += POOL_WARPS) {
+      const int q = t / (OW / 32), blk = z * (OW / 32) + t % (OW / 32);
+      const long long dst = (long long)b * cc.n_max + (cc.row0 ? cc.row0[b] : 0) + e0 + q;
+      pack_block_warp(krow[q * OW + (t % (OW / 32)) * 32 + lane], cc.global_scale, cc.codes + dst * (d_I / 2) + blk * 16,
+                      cc.scales + dst * S_pad + blk);
+      if (z == 0 && lane < S_pad - S) cc.scales[dst * S_pad + S + lane] = 0;
+    }
   }
 }
 
@@ -343,17 +409,32 @@ extern "C" csa_status csa_compress(const csa_compress_args* a, void* stream) {
   }
   if (a->ki_pack.codes) CSA_REQUIRE(a->W_IK && a->ki_pack.scales && a->ki_pack.global_scale > 0.0f);
   if (a->W_IK) CSA_SUPPORTED(((uintptr_t)a->W_IK & 15) == 0);
-  const size_t smem = (size_t)POOL_ENT * a->d * sizeof(float) +
-                      (a->W_IK ? (size_t)a->d * a->d_index * 2 + (size_t)(256 / a->d_index + 1) * POOL_ENT * a->d_index * 4 : 0);
+  if (a->W_IK) CSA_SUPPORTED((a->d_index * 2) % 16 == 0);
+  CSA_SUPPORTED(POOL_ENT * (a->d_rope / 2) <= POOL_THREADS && a->d_rope / 2 <= POOL_MAX_HALF);
+  // k_I output slices: enough CTAs for about one wave when there are few entry groups
+  const long long groups = (long long)a->B * ((n_out + POOL_ENT - 1) / POOL_ENT);
+  int OW = a->W_IK ? a->d_index : 32;
+  while (a->W_IK && OW > 32 && groups * (a->d_index / OW) * 2 <= 148) OW >>= 1;
+  const int nchp = POOL_THREADS / (OW / 8);
+  const bool pre = a->W_IK && a->d <= 8 * nchp;
+  const size_t smem = (size_t)POOL_ENT * a->d * sizeof(float) + (size_t)(POOL_WARPS + 1) * POOL_ENT * OW * 4;
   CSA_SUPPORTED(smem <= 200 * 1024);
-  static std::atomic<unsigned> attr_done{0};
-  set_smem_once((const void*)pool_kernel, 200 * 1024, attr_done);
   PoolParams P{};
   P.C = (const uint16_t*)a->C; P.Z = (const uint16_t*)a->Z; P.b_pos = a->b_pos; P.T = a->T; P.d = a->d;
   P.d_r = a->d_rope; P.r = a->ratio; P.theta = a->rope_theta; P.pos0 = a->pos0; P.W_IK = (const uint16_t*)a->W_IK;
   P.d_I = a->d_index; P.c_out = (uint16_t*)a->c_out; P.kI_out = (uint16_t*)a->kI_out; P.kv = a->kv_pack;
   P.ki = a->ki_pack;
-  dim3 grid((n_out + POOL_ENT - 1) / POOL_ENT, a->B);
-  pool_kernel<<<grid, 256, smem, st>>>(P);
+  for (int m = 0; m < a->d_rope / 2; ++m)
+    P.inv_freq[m] = a->rope_theta != 0.0f ? pow((double)a->rope_theta, -2.0 * m / (double)a->d_rope) : 0.0;
+  dim3 grid((n_out + POOL_ENT - 1) / POOL_ENT, a->B, a->W_IK ? a->d_index / OW : 1);
+  const void* fn;
+  if (OW == 32) fn = pre ? (const void*)pool_kernel<32, 8> : (const void*)pool_kernel<32, 0>;
+  else if (OW == 64) fn = pre ? (const void*)pool_kernel<64, 8> : (const void*)pool_kernel<64, 0>;
+  else fn = pre ? (const void*)pool_kernel<128, 8> : (const void*)pool_kernel<128, 0>;
+  static std::atomic<unsigned> attr_done[6];
+  set_smem_once(fn, 200 * 1024, attr_done[(OW == 32 ? 0 : OW == 64 ? 2 : 4) + (pre ? 1 : 0)]);
+  void* argv[] = {&P};
+  cudaError_t e = cudaLaunchKernel(fn, grid, dim3(POOL_THREADS), argv, smem, st);
+  if (e != cudaSuccess) { set_last_cuda_error(e); return CSA_ERR_CUDA; }
   return launch_status();
 }

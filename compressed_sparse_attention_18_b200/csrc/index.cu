@@ -14,6 +14,7 @@
 // rounding.  Each thread of a quad owns one 32-element scale block of its two key rows, so the key
 // side needs one 128-bit load per row and one scale byte.
 #include "csa_common.cuh"
+#include "sm100.cuh"
 
 namespace csa {
 
@@ -502,38 +503,48 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(TopkRowArgs A) {
 }
 
 
+// Exact selection of the `need` best of n <= 64 candidates (key desc, id asc, position asc) by one warp:
+// each candidate's rank is the number of candidates that beat it.  Writes the winners at oi/os[base + rank].
+__device__ void warp_rank_select(const uint32_t* keys, const int32_t* ids, int n, uint32_t need, int32_t* oi,
+                                 float* os, uint32_t base) {
+  const int lane = threadIdx.x & 31;
+  for (int i = lane; i < n; i += 32) {
+    const uint32_t ki = keys[i];
+    const int32_t ii = ids[i];
+    uint32_t rank = 0;
+    for (int j = 0; j < n; ++j) {
+      const uint32_t kj = keys[j];
+      const int32_t ij = ids[j];
+      rank += (kj > ki) || (kj == ki && (ij < ii || (ij == ii && j < i)));
+    }
+    if (rank < need) {
+      oi[base + rank] = ii;
+      if (os) os[base + rank] = order_key_float(ki);
+    }
+  }
+}
+
 // Histogram-guided selection for one row (decode / Reindex rows): the score kernel has counted the
 // row's scores in 4096 bins of the top 12 bits of their order-preserving keys.  The bin holding the
-// K-th largest score is found from the histogram; one pass over the row emits every score in a higher
-// bin and collects the boundary bin's scores, and only those go through the exact radix selection.
-// If the boundary bin overflows the candidate buffer the row is selected by the full path instead.
-__global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, const uint32_t* __restrict__ hist) {
-  extern __shared__ __align__(16) uint32_t s_keys[];   // candidates: keys [TOPK_CHUNK_IDS] | ids [TOPK_CHUNK_IDS]
-  __shared__ TopkSmem sm;
-  __shared__ uint32_t s_cnt[2];                         // emitted above the boundary bin, boundary candidates
-  const int row = blockIdx.y;
-  int len = min(A.rows_per_seg, A.n_cols);
-  if (A.q_pos) {
-    const int b = row / A.Nq;
-    long long nv = (A.q_pos[row] + 1) / A.ratio;
-    if (nv > A.n_c[b]) nv = A.n_c[b];
-    len = (int)max(0LL, min((long long)len, nv));
-  }
-  if (len < 0) len = 0;
-  int32_t* oi = A.out_idx + row * A.out_ld;
-  float* os = A.out_scores ? A.out_scores + row * A.out_ld : nullptr;
-  const float* src = A.in_scores + row * A.in_ld;
-  const int32_t* isrc = A.in_ids ? A.in_ids + row * A.in_ld : nullptr;
+// K-th largest score is found from the histogram; one pass over the row (bit masks in registers) emits
+// every score in a higher bin, at slots from one block scan, and collects the boundary bin's scores.
+// One warp resolves those on the remaining key bits.  If the boundary bin overflows the candidate
+// buffer the row is selected by the full path instead.
+constexpr int TOPK_HIST_PER_THREAD = TOPK_CHUNK / TOPK_THREADS;   // 32 scores per thread, 8 x float4
+constexpr int TOPK_RANK_MAX = 64;
+constexpr int TOPK_HIST_CAND = 4096;     // boundary-bin candidates held in shared memory
 
-  // suffix counts over the bins: thread t owns the 4 bins [4(T-1-t), 4(T-1-t)+4), highest bins first
+// Bin T (of HIST_BINS, thread t owning bins 4(T-1-t)..+3 counted from the top) holding the R-th largest
+// element given per-bin counts; returns {T, count above T, count in T} in sm.bcast[0..2] (zeros if R == 0
+// or R > total).  *total receives the number of counted elements.
+__device__ void hist_find_bin(TopkSmem& sm, const uint32_t* bins, uint32_t R, uint32_t* total) {
   const int owner = (int)blockDim.x - 1 - (int)threadIdx.x;
-  const uint4 hv = reinterpret_cast<const uint4*>(hist + (size_t)row * HIST_BINS)[owner];
+  const uint4 hv = reinterpret_cast<const uint4*>(bins)[owner];
   const uint32_t mine = hv.x + hv.y + hv.z + hv.w;
-  uint32_t nvalid;
-  const uint32_t above_me = block_exclusive_scan(sm, mine, &nvalid);
-  const uint32_t K = min((uint32_t)A.k, nvalid);
-  if (threadIdx.x == 0) { s_cnt[0] = 0; s_cnt[1] = 0; sm.bcast[0] = 0; sm.bcast[1] = 0; sm.bcast[2] = 0; }
+  const uint32_t above_me = block_exclusive_scan(sm, mine, total);
+  if (threadIdx.x == 0) { sm.bcast[0] = 0; sm.bcast[1] = 0; sm.bcast[2] = 0; }
   __syncthreads();
+  const uint32_t K = min(R, *total);
   if (K > 0 && above_me < K && K <= above_me + mine) {
     const uint32_t c[4] = {hv.w, hv.z, hv.y, hv.x};
     uint32_t acc = above_me;
@@ -548,70 +559,238 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
     }
   }
   __syncthreads();
+}
+
+__global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, const uint32_t* __restrict__ hist) {
+  // dynamic shared memory: the row [TOPK_CHUNK] (scores, or scores | ids for explicit-id rows), then the
+  // boundary-bin candidates: keys [TOPK_HIST_CAND] | ids [TOPK_HIST_CAND]
+  extern __shared__ __align__(16) uint32_t s_topk[];
+  __shared__ __align__(16) TopkSmem sm;
+  __shared__ __align__(8) uint64_t row_bar;
+  __shared__ uint32_t s_cnt[2];
+  static_assert(TOPK_HIST_PER_THREAD * TOPK_THREADS == TOPK_CHUNK && TOPK_HIST_PER_THREAD % 4 == 0 &&
+                TOPK_HIST_PER_THREAD <= 32, "row split");
+  static_assert(sizeof(TopkSmem::whist) >= HIST_BINS * 4, "second-level histogram in the per-warp histograms");
+  const int row = blockIdx.y;
+  int len = min(A.rows_per_seg, A.n_cols);
+  if (A.q_pos) {
+    const int b = row / A.Nq;
+    long long nv = (A.q_pos[row] + 1) / A.ratio;
+    if (nv > A.n_c[b]) nv = A.n_c[b];
+    len = (int)max(0LL, min((long long)len, nv));
+  }
+  if (len < 0) len = 0;
+  int32_t* oi = A.out_idx + row * A.out_ld;
+  float* os = A.out_scores ? A.out_scores + row * A.out_ld : nullptr;
+  const float* src = A.in_scores + row * A.in_ld;
+  const int32_t* isrc = A.in_ids ? A.in_ids + row * A.in_ld : nullptr;
+  float* s_row = reinterpret_cast<float*>(s_topk);
+  int32_t* s_rid = reinterpret_cast<int32_t*>(s_topk + TOPK_CHUNK_IDS);   // explicit ids (len <= TOPK_CHUNK_IDS)
+  uint32_t* ckeys = s_topk + TOPK_CHUNK;
+  int32_t* cids = reinterpret_cast<int32_t*>(s_topk + TOPK_CHUNK + TOPK_HIST_CAND);
+
+  // the row into shared memory: one bulk copy when aligned, else plain loads
+  const uint32_t bytes = (uint32_t)len * 4u;
+  const bool bulk = len > 0 && (len & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0 &&
+                    (!isrc || (reinterpret_cast<uintptr_t>(isrc) & 15) == 0);
+  if (bulk && threadIdx.x == 0) {
+    sm100::mbar_init(&row_bar, 1);
+    sm100::fence_mbar_init();
+    sm100::mbar_arrive_expect_tx(&row_bar, bytes * (isrc ? 2u : 1u));
+    for (uint32_t off = 0; off < bytes; off += 32768u) {
+      const uint32_t n = min(32768u, bytes - off);
+      sm100::bulk_load(reinterpret_cast<uint8_t*>(s_row) + off, reinterpret_cast<const uint8_t*>(src) + off, n, &row_bar);
+      if (isrc)
+        sm100::bulk_load(reinterpret_cast<uint8_t*>(s_rid) + off, reinterpret_cast<const uint8_t*>(isrc) + off, n,
+                         &row_bar);
+    }
+  } else if (!bulk) {
+    for (int j = threadIdx.x; j < len; j += blockDim.x) {
+      s_row[j] = src[j];
+      if (isrc) s_rid[j] = isrc[j];
+    }
+  }
+  uint32_t nvalid;
+  hist_find_bin(sm, hist + (size_t)row * HIST_BINS, (uint32_t)A.k, &nvalid);   // overlaps the copy
+  const uint32_t K = min((uint32_t)A.k, nvalid);
   const uint32_t Tbin = sm.bcast[0], above = sm.bcast[1], nT = sm.bcast[2];
   const uint32_t need = K - above;
-  uint32_t* ckeys = s_keys;
-  int32_t* cids = reinterpret_cast<int32_t*>(s_keys + TOPK_CHUNK_IDS);
-  const int lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
+  if (bulk && !sm100::mbar_wait(&row_bar, 0)) atomicOr(&g_csa_device_error, 1u);
+  // (plain loads: hist_find_bin's barriers have ordered them)
+  bool done = false;
   if (K > 0) {
-    constexpr int U = 16;   // loads in flight per thread: a 32768-score row takes two rounds
-    for (int jb = 0; jb < len; jb += U * blockDim.x) {
-      float v[U];
-      int32_t id[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = jb + u * blockDim.x + threadIdx.x;
-        v[u] = j < len ? src[j] : -INFINITY;
-        id[u] = j < len ? (isrc ? isrc[j] : j) : -1;
+    // one pass: bit masks "above the boundary bin" / "in it" over this thread's 32 scores, one block scan
+    // of the packed counts (above < 2^16, at <= 2^15) gives every thread its output slots
+    // the boundary bin as a float interval [lo, hi]: two compares per score (float order = key order)
+    const float lo = order_key_float(Tbin << HIST_SHIFT);
+    const float hi = order_key_float((Tbin << HIST_SHIFT) | ((1u << HIST_SHIFT) - 1u));
+    const bool fast = !isrc && Tbin > 0;                          // no ids; -inf lies below the bin
+    uint32_t m_up = 0, m_at = 0;
+    if (fast) {
+#pragma unroll 2
+      for (int i = 0; i < TOPK_HIST_PER_THREAD / 4; ++i) {
+        const int j0 = 4 * (threadIdx.x + TOPK_THREADS * i);
+        float4 f4 = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        if (j0 + 3 < len) {
+          f4 = *reinterpret_cast<const float4*>(s_row + j0);
+        } else if (j0 < len) {
+          f4.x = s_row[j0];
+          if (j0 + 1 < len) f4.y = s_row[j0 + 1];
+          if (j0 + 2 < len) f4.z = s_row[j0 + 2];
+        }
+        const uint32_t u = (uint32_t)(f4.x > hi) | ((uint32_t)(f4.y > hi) << 1) | ((uint32_t)(f4.z > hi) << 2) |
+                           ((uint32_t)(f4.w > hi) << 3);
+        const uint32_t g = (uint32_t)(f4.x >= lo) | ((uint32_t)(f4.y >= lo) << 1) | ((uint32_t)(f4.z >= lo) << 2) |
+                           ((uint32_t)(f4.w >= lo) << 3);
+        m_up |= u << (4 * i);
+        m_at |= (g & ~u) << (4 * i);
       }
+    } else {
+#pragma unroll 1
+      for (int i = 0; i < TOPK_HIST_PER_THREAD / 4; ++i) {
+        const int j0 = 4 * (threadIdx.x + TOPK_THREADS * i);
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const bool ok = v[u] > -INFINITY && id[u] >= 0;
-        const uint32_t key = float_order_key(v[u]);
-        const uint32_t bin = key >> HIST_SHIFT;
-        const bool up = ok && bin > Tbin, at = ok && bin == Tbin;
-        const unsigned mu = __ballot_sync(0xffffffffu, up), ma = __ballot_sync(0xffffffffu, at);
-        uint32_t bu = 0, ba = 0;
-        if (lane == 0) {
-          if (mu) bu = atomicAdd(&s_cnt[0], (uint32_t)__popc(mu));
-          if (ma) ba = atomicAdd(&s_cnt[1], (uint32_t)__popc(ma));
-        }
-        bu = __shfl_sync(0xffffffffu, bu, 0);
-        ba = __shfl_sync(0xffffffffu, ba, 0);
-        if (up) {
-          const uint32_t slot = bu + __popc(mu & lt);
-          oi[slot] = id[u];
-          if (os) os[slot] = v[u] + 0.0f;
-        }
-        if (at) {
-          const uint32_t slot = ba + __popc(ma & lt);
-          if (slot < TOPK_CHUNK_IDS) { ckeys[slot] = key; cids[slot] = id[u]; }
+        for (int c = 0; c < 4; ++c) {
+          const float v = j0 + c < len ? s_row[j0 + c] : -INFINITY;
+          const bool ok = v > -INFINITY && (!isrc || s_rid[j0 + c] >= 0);
+          const uint32_t bin = float_order_key(v) >> HIST_SHIFT;
+          if (ok && bin > Tbin) m_up |= 1u << (4 * i + c);
+          if (ok && bin == Tbin) m_at |= 1u << (4 * i + c);
         }
       }
     }
+    uint32_t tot;
+    const uint32_t pre = block_exclusive_scan(sm, (uint32_t)__popc(m_up) | ((uint32_t)__popc(m_at) << 16), &tot);
+    if ((tot & 0xFFFFu) == above && (tot >> 16) == nT && nT <= (uint32_t)TOPK_HIST_CAND) {
+      uint32_t su = pre & 0xFFFFu, sa = pre >> 16;
+      uint32_t mk = m_up | m_at;
+#pragma unroll 1
+      while (mk) {
+        const int e = __ffs(mk) - 1;
+        mk &= mk - 1u;
+        const int j = 4 * (threadIdx.x + TOPK_THREADS * (e >> 2)) + (e & 3);
+        const float v = s_row[j];
+        const int32_t id = isrc ? s_rid[j] : j;
+        if ((m_up >> e) & 1u) {
+          oi[su] = id;
+          if (os) os[su] = v + 0.0f;
+          ++su;
+        } else {
+          ckeys[sa] = float_order_key(v);
+          cids[sa] = id;
+          ++sa;
+        }
+      }
+      done = true;
+    }
   }
-  __syncthreads();
-  const uint32_t ncand = s_cnt[1];
-  if (K > 0 && ncand <= TOPK_CHUNK_IDS && s_cnt[0] == above && ncand == nT) {
-    auto idof = [&](int j) -> uint32_t { return (uint32_t)cids[j]; };
-    if (ncand == need) {
-      for (int j = threadIdx.x; j < (int)ncand; j += blockDim.x) {
+  // every thread takes the same branch: `done` depends only on block-uniform values
+  if (done) {
+    __syncthreads();
+    if (need == nT) {
+      for (int j = threadIdx.x; j < (int)nT; j += blockDim.x) {
         oi[above + j] = cids[j];
         if (os) os[above + j] = order_key_float(ckeys[j]);
       }
-      __syncthreads();
+    } else if (nT <= (uint32_t)TOPK_RANK_MAX) {
+      if (threadIdx.x < 32) warp_rank_select(ckeys, cids, (int)nT, need, oi, os, above);
     } else {
-      select_in_smem(sm, ckeys, (int)ncand, need, ncand, idof, oi, os, above);
+      // boundary bin: 8-bit digits of the remaining key bits (19..12, 11..4, 3..0), one 256-bin histogram
+      // per level scanned by one warp, until at most TOPK_RANK_MAX candidates share the threshold prefix;
+      // those go by rank (key, id, position), all of them by the block radix path if that never happens
+      uint32_t* h2 = &sm.whist[0][0];                                // 256 bins
+      uint32_t* k2 = &sm.whist[1][0];                                // TOPK_RANK_MAX keys, then ids
+      int32_t* i2 = reinterpret_cast<int32_t*>(&sm.whist[1][TOPK_RANK_MAX]);
+      uint32_t pref = 0, pmask = 0, rem = need, base_out = above, n_in = nT;
+      bool ranked = false;
+#pragma unroll 1
+      for (int level = 0; level < 3 && !ranked; ++level) {
+        const int sh = level == 0 ? 12 : level == 1 ? 4 : 0;
+        const uint32_t dm = level == 2 ? 15u : 255u;
+        if (threadIdx.x < 256) h2[threadIdx.x] = 0;
+        if (threadIdx.x == 0) { s_cnt[0] = 0; s_cnt[1] = 0; }
+        __syncthreads();
+        for (int j = threadIdx.x; j < (int)nT; j += blockDim.x) {
+          const uint32_t k = ckeys[j] & 0xFFFFFu;
+          if ((k & pmask) == pref) atomicAdd(&h2[(k >> sh) & dm], 1u);
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+          // lane l owns digits 8(31-l) .. 8(31-l)+7, highest first
+          const int lane = threadIdx.x;
+          uint32_t c[8], tot = 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) { c[i] = h2[8 * (31 - lane) + 7 - i]; tot += c[i]; }
+          uint32_t incl = tot;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          uint32_t acc = incl - tot;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (acc < rem && acc + c[i] >= rem) {
+              sm.bcast[0] = 8 * (31 - lane) + 7 - i;
+              sm.bcast[1] = acc;
+              sm.bcast[2] = c[i];
+            }
+            acc += c[i];
+          }
+        }
+        __syncthreads();
+        const uint32_t digit = sm.bcast[0], above2 = sm.bcast[1], n2 = sm.bcast[2];
+        const uint32_t npref = pref | (digit << sh), nmask = pmask | (dm << sh);
+        // write the candidates in a higher digit; keep the threshold digit's few for ranking
+        for (int j = threadIdx.x; j < (int)nT; j += blockDim.x) {
+          const uint32_t k = ckeys[j] & 0xFFFFFu;
+          if ((k & pmask) != pref) continue;
+          const uint32_t dj = (k >> sh) & dm;
+          if (dj > digit) {
+            const uint32_t slot = base_out + atomicAdd(&s_cnt[0], 1u);
+            oi[slot] = cids[j];
+            if (os) os[slot] = order_key_float(ckeys[j]);
+          } else if (dj == digit && n2 <= (uint32_t)TOPK_RANK_MAX) {
+            const uint32_t slot = atomicAdd(&s_cnt[1], 1u);
+            k2[slot] = ckeys[j];
+            i2[slot] = cids[j];
+          }
+        }
+        __syncthreads();
+        base_out += above2;
+        rem -= above2;
+        pref = npref;
+        pmask = nmask;
+        n_in = n2;
+        if (n2 <= (uint32_t)TOPK_RANK_MAX) {
+          if (threadIdx.x < 32) warp_rank_select(k2, i2, (int)n2, rem, oi, os, base_out);
+          ranked = true;
+        }
+      }
+      if (!ranked) {
+        // more than TOPK_RANK_MAX candidates with one full key: exact selection among them
+        for (int j = threadIdx.x; j < (int)nT; j += blockDim.x)
+          if ((ckeys[j] & 0xFFFFFu) != pref) ckeys[j] = 0u;
+        __syncthreads();
+        auto idof = [&](int j) -> uint32_t { return (uint32_t)cids[j]; };
+        select_in_smem(sm, ckeys, (int)nT, rem, n_in, idof, oi, os, base_out);
+      }
     }
   } else if (K > 0) {
-    // boundary bin larger than the buffer (or inconsistent counts): select the whole row
+    // inconsistent counts or a boundary bin larger than the candidate buffer: the whole row, in place
     __syncthreads();
-    const uint32_t nv2 = load_row_keys(sm, src, isrc, len, s_keys,
-                                       reinterpret_cast<int32_t*>(s_keys + (isrc ? TOPK_CHUNK_IDS : 0)));
-    int32_t* ids2 = reinterpret_cast<int32_t*>(s_keys + TOPK_CHUNK_IDS);
-    auto idof2 = [&](int j) -> uint32_t { return isrc ? (uint32_t)ids2[j] : (uint32_t)j; };
-    select_in_smem(sm, s_keys, len, min((uint32_t)A.k, nv2), nv2, idof2, oi, os, 0u);
+    uint32_t* keys = s_topk;
+    uint32_t nv_loc = 0;
+    for (int j = threadIdx.x; j < len; j += blockDim.x) {
+      const float v = s_row[j];
+      const bool ok = v > -INFINITY && (!isrc || s_rid[j] >= 0);
+      keys[j] = ok ? float_order_key(v) : 0u;
+      nv_loc += ok;
+    }
+    uint32_t nv2;
+    block_exclusive_scan(sm, nv_loc, &nv2);
+    auto idof2 = [&](int j) -> uint32_t { return isrc ? (uint32_t)s_rid[j] : (uint32_t)j; };
+    select_in_smem(sm, keys, len, min((uint32_t)A.k, nv2), nv2, idof2, oi, os, 0u);
   }
   for (int s2 = (int)K + threadIdx.x; s2 < A.k; s2 += blockDim.x) {
     oi[s2] = -1;
@@ -791,8 +970,9 @@ static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const 
     ta.out_scores = a->scores_out;
     ta.out_ld = a->k;
     static std::atomic<unsigned> attr_h{0};
-    set_smem_once((const void*)topk_hist_kernel, TOPK_CHUNK * 4, attr_h);
-    topk_hist_kernel<<<dim3(1, p.rows), TOPK_THREADS, TOPK_CHUNK * 4, st>>>(ta, hist);
+    const int smem_h = (TOPK_CHUNK + 2 * TOPK_HIST_CAND) * 4;
+    set_smem_once((const void*)topk_hist_kernel, smem_h, attr_h);
+    topk_hist_kernel<<<dim3(1, p.rows), TOPK_THREADS, smem_h, st>>>(ta, hist);
     csa_status s = launch_status();
     if (s != CSA_OK) return s;
   } else if (p.segs == 1) {

@@ -290,11 +290,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
 }
 
 // --------------------------------------------------------------------------------------- host
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
+namespace sm100 {
+EncodeTiledFn tensor_map_encoder() {
   static std::atomic<EncodeTiledFn> fn{nullptr};
   EncodeTiledFn f = fn.load();
   if (!f) {
@@ -307,11 +304,12 @@ static EncodeTiledFn encode_fn() {
   }
   return f;
 }
+}  // namespace sm100
 
 bool index_tc_eligible(const csa_index_args* a) {
   return a->cand == nullptr && a->Nq == 1 && a->d_I == 128 && a->H_I <= 8 && a->n_max % 4 == 0 && a->n_max > 0 &&
          (reinterpret_cast<uintptr_t>(a->k_codes) & 15) == 0 && (reinterpret_cast<uintptr_t>(a->k_scales) & 15) == 0 &&
-         encode_fn() != nullptr;
+         tensor_map_encoder() != nullptr;
 }
 
 csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, uint32_t* hist, cudaStream_t st) {
@@ -320,7 +318,7 @@ csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, u
   const cuuint64_t gstride[1] = {64};
   const cuuint32_t box[2] = {64, TC_TILE};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode_fn()(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void*)a->k_codes, gdim, gstride, box, estr,
+  CUresult r = tensor_map_encoder()(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void*)a->k_codes, gdim, gstride, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return CSA_ERR_CUDA;
