@@ -265,22 +265,20 @@ def run_ours(args, rank, world):
     stream.synchronize()
     graphs = {}
 
-    def graph_for(n):
-        if n not in graphs:
+    def graph_for(n, with_marks):
+        if (n, with_marks) not in graphs:
             gph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gph, stream=stream, capture_error_mode="relaxed"):
-                run_layers(n, True)
-            graphs[n] = gph
-        return graphs[n]
+                run_layers(n, with_marks)
+            graphs[(n, with_marks)] = gph
+        return graphs[(n, with_marks)]
 
-    full = graph_for(LAYERS)
-
-    def run_steps(k):
+    def run_steps(k, with_marks=False):
         with torch.cuda.stream(stream):
             for _ in range(k // LAYERS):
-                full.replay()
+                graph_for(LAYERS, with_marks).replay()
             if k % LAYERS:
-                graph_for(k % LAYERS).replay()
+                graph_for(k % LAYERS, with_marks).replay()
 
     run_steps(max(args.warmup, 3))
     stream.synchronize()
@@ -300,9 +298,13 @@ def run_ours(args, rank, world):
         torch.distributed.barrier()
     clocks = clk.stop()
     ms = t0.elapsed_time(t1)
-    # per-stage times of the last rotation of the timed region (events inside the graph)
-    last = min(args.steps, LAYERS)
-    stage = [[marks[li][j].elapsed_time(marks[li][j + 1]) for j in range(4)] for li in range(last)]
+    # per-stage times: a second timed region replaying the same steps from a graph with an event at every
+    # stage boundary (the events serialise the stages, so these times include each kernel's full launch)
+    run_steps(LAYERS, with_marks=True)
+    stream.synchronize()
+    run_steps(LAYERS, with_marks=True)
+    stream.synchronize()
+    stage = [[marks[li][j].elapsed_time(marks[li][j + 1]) for j in range(4)] for li in range(LAYERS)]
     score_ms = statistics.mean(st[1] for st in stage)
     if world > 1:
         tt = torch.tensor([ms], device=dev)

@@ -347,54 +347,132 @@ __global__ void __launch_bounds__(AT_WARPS * 32, 1) attn_kernel(AttnParams P) {
 // One CTA per (query, head); each thread owns 4 consecutive output dims, the split weights are
 // computed once per CTA in shared memory.
 constexpr int MERGE_MAX_SPLITS = 128;
-__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
-__device__ __forceinline__ float4 load4(const uint16_t* p) {
-  const uint2 u = *reinterpret_cast<const uint2*>(p);
-  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
-                     __uint_as_float(u.y & 0xFFFF0000u));
+// Split merge: one warp per (query, head).  Lane l owns dims 16l .. 16l+15 (D = 512) or 4l .. 4l+3
+// (D = 128); the split lse values and all partial loads of a chunk of splits (6 or 8) are issued
+// together, so a merge of up to that many splits costs about one memory round trip.  Partials are fp32 (CUDA-core path) or bf16 (tensor-core path).
+constexpr int MERGE_WARPS = 4;
+
+template <typename PT, int DPL>
+__device__ __forceinline__ void load_dims(const PT* p, float* v);
+template <>
+__device__ __forceinline__ void load_dims<uint16_t, 16>(const uint16_t* p, float* v) {
+  const uint4 a = *reinterpret_cast<const uint4*>(p), b = *reinterpret_cast<const uint4*>(p + 8);
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) { v[2 * i] = __uint_as_float(w[i] << 16); v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u); }
+}
+template <>
+__device__ __forceinline__ void load_dims<uint16_t, 4>(const uint16_t* p, float* v) {
+  const uint2 a = *reinterpret_cast<const uint2*>(p);
+  v[0] = __uint_as_float(a.x << 16); v[1] = __uint_as_float(a.x & 0xFFFF0000u);
+  v[2] = __uint_as_float(a.y << 16); v[3] = __uint_as_float(a.y & 0xFFFF0000u);
+}
+template <>
+__device__ __forceinline__ void load_dims<float, 16>(const float* p, float* v) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 f = reinterpret_cast<const float4*>(p)[i];
+    v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+  }
+}
+template <>
+__device__ __forceinline__ void load_dims<float, 4>(const float* p, float* v) {
+  const float4 f = *reinterpret_cast<const float4*>(p);
+  v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
 }
 
-// Partials in fp32 (CUDA-core path) or bf16 (tensor-core path).
-template <typename PT>
-__global__ void __launch_bounds__(128) attn_merge_kernel(const PT* __restrict__ part_o,
-                                                         const float* __restrict__ part_lse, int splits, int H, int D,
-                                                         uint16_t* __restrict__ out, float* __restrict__ lse) {
-  __shared__ float s_w[MERGE_MAX_SPLITS];
-  __shared__ float s_tot[2];
-  const int bq = blockIdx.x / H, h = blockIdx.x % H;
-  if (threadIdx.x < 32) {
-    float mx = -INFINITY;
-    for (int s = threadIdx.x; s < splits; s += 32) mx = fmaxf(mx, part_lse[((size_t)bq * splits + s) * H + h]);
+template <typename PT, int D>
+__global__ void __launch_bounds__(MERGE_WARPS * 32) attn_merge_kernel(const PT* __restrict__ part_o,
+                                                                     const float* __restrict__ part_lse, int splits,
+                                                                     int H, long long units, uint16_t* __restrict__ out,
+                                                                     float* __restrict__ lse) {
+  constexpr int DPL = D / 32;
+  constexpr int MERGE_CHUNK = D == 512 ? 6 : 8;   // splits whose partials are in flight at once
+  const int lane = threadIdx.x & 31;
+  const long long unit = (long long)blockIdx.x * MERGE_WARPS + (threadIdx.x >> 5);
+  pdl_trigger();
+  pdl_wait();
+  if (unit >= units) return;
+  const long long bq = unit / H;
+  const int h = (int)(unit % H);
+  float acc[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
+  const PT* base = part_o + (bq * splits * H + h) * (long long)D + lane * DPL;
+  const float* lrow = part_lse + bq * splits * H + h;
+  float mx = -INFINITY, sum = 0.f;
+  if (splits <= MERGE_CHUNK) {
+    // one round: every lane loads all split lse values (broadcast) and its dims of every partial; empty
+    // splits (lse = -inf, partial never written) are dropped by a select, never multiplied
+    float v[MERGE_CHUNK][DPL], ls[MERGE_CHUNK];
+#pragma unroll
+    for (int c = 0; c < MERGE_CHUNK; ++c) {
+      ls[c] = c < splits ? lrow[(long long)c * H] : -INFINITY;
+      if (c < splits) load_dims<PT, DPL>(base + (long long)c * H * D, v[c]);
+    }
+#pragma unroll
+    for (int c = 0; c < MERGE_CHUNK; ++c) mx = fmaxf(mx, ls[c]);
+#pragma unroll
+    for (int c = 0; c < MERGE_CHUNK; ++c) {
+      const float w = (mx == -INFINITY || ls[c] == -INFINITY) ? 0.f : exp2f((ls[c] - mx) * LOG2E);
+      sum += w;
+      if (w != 0.f)
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w, v[c][i], acc[i]);
+    }
+  } else {
+    // max and weights of the split lse values (lanes hold splits s = lane, lane + 32, ...)
+    for (int s = lane; s < splits; s += 32) mx = fmaxf(mx, lrow[(long long)s * H]);
     mx = warp_max(mx);
-    float sum = 0.f;
-    for (int s = threadIdx.x; s < splits; s += 32) {
-      const float ls = part_lse[((size_t)bq * splits + s) * H + h];
-      const float wgt = (mx == -INFINITY || ls == -INFINITY) ? 0.f : exp2f((ls - mx) * LOG2E);
-      s_w[s] = wgt;
-      sum += wgt;
+    for (int s = lane; s < splits; s += 32) {
+      const float l = lrow[(long long)s * H];
+      sum += (mx == -INFINITY || l == -INFINITY) ? 0.f : exp2f((l - mx) * LOG2E);
     }
     sum = warp_sum(sum);
-    if (threadIdx.x == 0) { s_tot[0] = sum; s_tot[1] = mx; }
-  }
-  __syncthreads();
-  const float sum = s_tot[0];
-  const float inv = sum > 0.f ? 1.f / sum : 0.f;
-  for (int d4 = threadIdx.x * 4; d4 < D; d4 += blockDim.x * 4) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int s = 0; s < splits; ++s) {
-      const float wgt = s_w[s];
-      if (wgt == 0.f) continue;
-      const float4 v = load4(part_o + (((size_t)bq * splits + s) * H + h) * D + d4);
-      acc.x = fmaf(wgt, v.x, acc.x); acc.y = fmaf(wgt, v.y, acc.y);
-      acc.z = fmaf(wgt, v.z, acc.z); acc.w = fmaf(wgt, v.w, acc.w);
+    for (int s0 = 0; s0 < splits; s0 += MERGE_CHUNK) {
+      float v[MERGE_CHUNK][DPL];
+      float wgt[MERGE_CHUNK];
+#pragma unroll
+      for (int c = 0; c < MERGE_CHUNK; ++c) {
+        const int s = s0 + c;
+        wgt[c] = 0.f;
+        if (s < splits) {
+          const float l = lrow[(long long)s * H];
+          wgt[c] = (mx == -INFINITY || l == -INFINITY) ? 0.f : exp2f((l - mx) * LOG2E);
+        }
+        if (wgt[c] != 0.f) load_dims<PT, DPL>(base + (long long)s * H * D, v[c]);
+      }
+#pragma unroll
+      for (int c = 0; c < MERGE_CHUNK; ++c)
+        if (wgt[c] != 0.f)
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) acc[i] = fmaf(wgt[c], v[c][i], acc[i]);
     }
-    uint2 o2;
-    o2.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    o2.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2*>(out + ((size_t)bq * H + h) * D + d4) = o2;
   }
-  if (lse && threadIdx.x == 0) lse[(size_t)bq * H + h] = sum > 0.f ? s_tot[1] + logf(sum) : -INFINITY;
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  uint16_t* o = out + (bq * H + h) * (long long)D + lane * DPL;
+  uint32_t pk[DPL / 2];
+#pragma unroll
+  for (int i = 0; i < DPL / 2; ++i) pk[i] = pack_bf16x2(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+  if (DPL == 16) {
+    reinterpret_cast<uint4*>(o)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  } else {
+    *reinterpret_cast<uint2*>(o) = make_uint2(pk[0], pk[1]);
+  }
+  if (lse && lane == 0) lse[bq * H + h] = sum > 0.f ? mx + logf(sum) : -INFINITY;
+}
+
+template <typename PT>
+static csa_status launch_merge(const PT* po, const float* pl, int splits, int H, int D, long long rows, uint16_t* out,
+                               float* lse, cudaStream_t st) {
+  const long long units = rows * H;
+  const unsigned grid = (unsigned)((units + MERGE_WARPS - 1) / MERGE_WARPS);
+  if (D == 512)
+    return launch_pdl(attn_merge_kernel<PT, 512>, dim3(grid), dim3(MERGE_WARPS * 32), 0, st, po, pl, splits, H, units,
+                      out, lse);
+  return launch_pdl(attn_merge_kernel<PT, 128>, dim3(grid), dim3(MERGE_WARPS * 32), 0, st, po, pl, splits, H, units,
+                    out, lse);
 }
 
 // tensor-core decode path (attn_tc.cu)
@@ -487,9 +565,7 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
     float* pl = p.splits > 1 ? (float*)((uint8_t*)ws + p.off_lse) : nullptr;
     csa_status s = launch_attn_tc(a, hca, p.splits, po, pl, st);
     if (s != CSA_OK || p.splits == 1) return s;
-    attn_merge_kernel<uint16_t><<<(unsigned)(rows * a->H), 128, 0, st>>>(po, pl, p.splits, a->H, a->d,
-                                                                         (uint16_t*)a->out, a->lse);
-    return launch_status();
+    return launch_merge<uint16_t>(po, pl, p.splits, a->H, a->d, rows, (uint16_t*)a->out, a->lse, st);
   }
   AttnParams P{};
   P.B = a->B; P.Nq = a->Nq; P.H = a->H; P.d_r = a->d_rope; P.ratio = a->ratio; P.n_max = a->n_max;
@@ -510,9 +586,7 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
   else
     s = launch_attn<128, 8>(P, units, st);
   if (s != CSA_OK || p.splits == 1) return s;
-  attn_merge_kernel<float><<<(unsigned)(rows * a->H), 128, 0, st>>>(P.part_o, P.part_lse, p.splits, a->H, a->d,
-                                                                      (uint16_t*)a->out, a->lse);
-  return launch_status();
+  return launch_merge<float>(P.part_o, P.part_lse, p.splits, a->H, a->d, rows, (uint16_t*)a->out, a->lse, st);
 }
 
 }  // namespace csa

@@ -29,7 +29,6 @@ constexpr int TA_WORKERS = 256;           // warps 0-7: gather, softmax (4 lane 
 constexpr int TA_THREADS = TA_WORKERS + 32; // warp 8: barriers, tensor memory, TMA and MMA issue
 constexpr int TA_KEYS = 128;
 constexpr int TA_WBOX = 32;                // window rows per TMA box
-constexpr int TA_CHUNKS = 14;              // 32-element FP4 blocks per entry (448 dims)
 constexpr uint32_t TA_TMEM_COLS = 512;
 constexpr uint32_t TA_COL_S = 0;           // S^T: 64 columns
 constexpr uint32_t TA_COL_O = 64;          // O^T: 4 x 64 columns
@@ -156,6 +155,28 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   const int key0 = split * TA_KEYS;
   // worker thread t owns tile row t/2 for the gather (its half of the row's FP4 blocks and RoPE slice)
   const int grow = (tid & (TA_WORKERS - 1)) >> 1, ghalf = tid & 1;
+  // setup that reads no global memory, then wait for the previous kernel (it writes the selected ids)
+  if (warp == 8) {
+    if (lane == 0) {
+      S.err = 0;
+      for (int j = 0; j < 8; ++j) {
+        mbar_init(&S.bar_q[j], 1);
+        mbar_init(&S.bar_w[j], 1);
+        mbar_init(&S.bar_k[j], TA_WORKERS / 32);
+      }
+      mbar_init(&S.bar_s, 1);
+      mbar_init(&S.bar_p, TA_WORKERS / 32);
+      for (int j = 0; j < 4; ++j) mbar_init(&S.bar_o[j], 1);
+      fence_mbar_init();
+      prefetch_tensormap(&qmap);
+      prefetch_tensormap(&wmap);
+    }
+    __syncwarp();
+    tmem_alloc(&S.tmem_base, TA_TMEM_COLS);
+    tmem_relinquish();
+  }
+  pdl_trigger();
+  pdl_wait();
   int id_raw = -1;
   if (!P.hca && tid < TA_WORKERS && key0 + grow < P.k) id_raw = P.idx[(size_t)bq * P.k + key0 + grow];
   const long long tq = P.q_pos[bq];
@@ -173,6 +194,26 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   }
   const int n_list = n_sel + (whi >= wlo ? (int)(whi - wlo + 1) : 0);
   const size_t unit_ho = ((size_t)bq * P.splits + split) * P.H;
+  // tile rows: [0, rs) entries, [rs, rw) window rows, [rw, 128) empty
+  const int rs = min(max(n_sel - key0, 0), TA_KEYS);
+  const int rw = max(min(n_list - key0, TA_KEYS), 0);
+  const int wa = (rs + TA_WBOX - 1) / TA_WBOX * TA_WBOX;            // window rows >= wa come by TMA boxes
+  const int we = rw > wa ? (rw + TA_WBOX - 1) / TA_WBOX * TA_WBOX : wa;
+  const int zs = rw > wa ? we : rw;                                 // rows >= zs are zero-filled
+  // window buffer row of tile row r (r >= rs)
+  const long long wrow_base = (wlo - p0) + (long long)(key0 - n_sel);
+  // entry ids of the tile rows for the softmax masks (the gather threads keep their own copies)
+  if (tid < TA_WORKERS && ghalf == 0) {
+    int id = -1;
+    if (grow < rs) {
+      const int v = P.hca ? key0 + grow : id_raw;
+      if (v >= 0 && v < ncb) id = v;
+    }
+    S.ids[grow] = id;
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = S.tmem_base;
 
   if (key0 >= n_list) {                          // nothing in this tile: an empty partial
     if (P.splits > 1) {
@@ -182,38 +223,9 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
         reinterpret_cast<uint32_t*>(P.out + (size_t)bq * P.H * 512)[i] = 0u;
       if (P.lse && tid < P.H) P.lse[(size_t)bq * P.H + tid] = -INFINITY;
     }
+    if (warp == 8) tmem_dealloc(tb, TA_TMEM_COLS);
     return;
   }
-  // tile rows: [0, rs) entries, [rs, rw) window rows, [rw, 128) empty
-  const int rs = min(max(n_sel - key0, 0), TA_KEYS);
-  const int rw = min(n_list - key0, TA_KEYS);
-  const int wa = (rs + TA_WBOX - 1) / TA_WBOX * TA_WBOX;            // window rows >= wa come by TMA boxes
-  const int we = rw > wa ? (rw + TA_WBOX - 1) / TA_WBOX * TA_WBOX : wa;
-  const int zs = rw > wa ? we : rw;                                 // rows >= zs are zero-filled
-  // window buffer row of tile row r (r >= rs)
-  const long long wrow_base = (wlo - p0) + (long long)(key0 - n_sel);
-
-  if (warp == 8) {
-    if (lane == 0) {
-      S.err = 0;
-      for (int j = 0; j < 8; ++j) {
-        mbar_init(&S.bar_q[j], 1);
-        mbar_init(&S.bar_w[j], 1);
-        mbar_init(&S.bar_k[j], TA_WORKERS / 32);
-      }
-      mbar_init(&S.bar_s, 1);
-      mbar_init(&S.bar_p, TA_WORKERS / 32);
-      for (int j = 0; j < 4; ++j) mbar_init(&S.bar_o[j], 1);
-      fence_mbar_init();
-      prefetch_tensormap(&qmap);
-    }
-    __syncwarp();
-    tmem_alloc(&S.tmem_base, TA_TMEM_COLS);
-    tmem_relinquish();
-  }
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tb = S.tmem_base;
 
   if (warp == 8) {
     // ------------------------------------------------------------------ control: TMA, then MMA issue
@@ -271,7 +283,6 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       const int v = P.hca ? key0 + grow : id_raw;
       if (v >= 0 && v < ncb) id = v;
     }
-    if (ghalf == 0) S.ids[grow] = id;
     // FP4 blocks 2j + ghalf (j = 0..6) of the row and its scale row; loads first
     uint4 cv[7];
     uint4 sc16 = make_uint4(0, 0, 0, 0);
@@ -477,8 +488,7 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, uint16_t*
   const int smem = (int)sizeof(TaSmem) + 1024;
   static std::atomic<unsigned> attr_done{0};
   set_smem_once((const void*)attn_tc_kernel, smem, attr_done);
-  attn_tc_kernel<<<(unsigned)(rows * splits), TA_THREADS, smem, st>>>(qmap, wmap, P);
-  return launch_status();
+  return launch_pdl(attn_tc_kernel, dim3((unsigned)(rows * splits)), dim3(TA_THREADS), (size_t)smem, st, qmap, wmap, P);
 }
 
 cudaError_t attn_take_device_error(uint32_t* out) { return take_device_error_here(out); }

@@ -192,21 +192,24 @@ __device__ __forceinline__ void fma8_bf16(float* acc, float p, const uint4& w) {
 
 // OW: indexer-key outputs per CTA (32, 64 or 128); PRE: channels per thread when the W_IK slice is
 // preloaded into registers (0: streamed).
-template <int OW, int PRE>
+template <int OW, int PRE, int ENT, int R>
 __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
   constexpr int NOC = OW / 8;                       // 8-output chunks of the slice
   constexpr int NCHP = POOL_THREADS / NOC;          // channel phases
-  // shared memory: pooled [POOL_ENT][d] fp32 | red [POOL_WARPS][POOL_ENT][OW] | k_I rows [POOL_ENT][OW]
+  // shared memory: pooled [ENT][d] fp32 | red [POOL_WARPS][ENT][OW] | k_I rows [ENT][OW]
   extern __shared__ __align__(128) float pooled[];
   const int b = blockIdx.y, z = blockIdx.z;
-  const int d = P.d, d_r = P.d_r, r = P.r, T = P.T, d_I = P.d_I;
+  const int d = P.d, d_r = P.d_r, r = R > 0 ? R : P.r, T = P.T, d_I = P.d_I;
+  constexpr int RJ = R > 0 ? R : 8;                 // slots loaded per channel in the short-group path
   const int n_out = T / r;
-  const int e0 = blockIdx.x * POOL_ENT;
-  const int ne = min(POOL_ENT, n_out - e0);
+  const int e0 = blockIdx.x * ENT;
+  const int ne = min(ENT, n_out - e0);
   const int d_n = d - d_r;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int oc = tid % NOC, chp = tid / NOC;
   const int o_base = z * OW + oc * 8;
+  pdl_trigger();
+  pdl_wait();                                       // C, Z, the caches may come from the previous kernel
   // W_IK slice into registers first (its latency overlaps the pooling)
   uint4 wpre[PRE > 0 ? PRE : 1];
   if (PRE > 0 && P.W_IK) {
@@ -234,17 +237,17 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
   const uint16_t* __restrict__ C = P.C;
   const uint16_t* __restrict__ Z = P.Z;
   const float* __restrict__ b_pos = P.b_pos;
-  if (r <= 8) {
+  if (R > 0 || r <= 8) {
     // two channels per thread per round, all their loads issued before any arithmetic
     for (int i0 = tid; i0 < ne * d; i0 += 2 * POOL_THREADS) {
-      float a[2][8], c[2][8];
+      float a[2][RJ], c[2][RJ];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int i = min(i0 + u * POOL_THREADS, ne * d - 1);
         const int q = i / d, ch = i % d;
         const size_t tok0 = (size_t)b * T + (size_t)(e0 + q) * r;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < RJ; ++j) {
           a[u][j] = j < r ? bf16_bits_to_f(Z[(tok0 + j) * d + ch]) + b_pos[(size_t)j * d + ch] : -INFINITY;
           c[u][j] = j < r ? bf16_bits_to_f(C[(tok0 + j) * d + ch]) : 0.f;
         }
@@ -256,10 +259,10 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
         if (i >= ne * d) continue;
         float m = a[u][0];
 #pragma unroll
-        for (int j = 1; j < 8; ++j) m = fmaxf(m, a[u][j]);
+        for (int j = 1; j < RJ; ++j) m = fmaxf(m, a[u][j]);
         float l = 0.f, acc = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < RJ; ++j) {
           const float p = j < r ? __expf(a[u][j] - m) : 0.f;
           l += p;
           acc = fmaf(p, c[u][j], acc);
@@ -268,7 +271,7 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
       }
     }
     if (ne * d <= tid && rope_thread) rope_angle();
-  } else {
+  } else if (R == 0) {
     if (rope_thread) rope_angle();
     for (int i = tid; i < ne * d; i += POOL_THREADS) {
       const int q = i / d, ch = i % d;
@@ -310,11 +313,11 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
     for (int q = 0; q < ne; ++q) pack_row_to_cache(pooled + q * d, d, d_r, P.kv, b, e0 + q);
   if (P.W_IK == nullptr) return;
   // k_I slice: thread (oc, chp) sums outputs o_base..o_base+7 over channels chp, chp + NCHP, ...
-  float* red = pooled + POOL_ENT * d;               // [POOL_WARPS][POOL_ENT][OW]
-  float* krow = red + POOL_WARPS * POOL_ENT * OW;   // [POOL_ENT][OW]
-  float acc[POOL_ENT][8];
+  float* red = pooled + ENT * d;               // [POOL_WARPS][ENT][OW]
+  float* krow = red + POOL_WARPS * ENT * OW;   // [ENT][OW]
+  float acc[ENT][8];
 #pragma unroll
-  for (int q = 0; q < POOL_ENT; ++q)
+  for (int q = 0; q < ENT; ++q)
 #pragma unroll
     for (int k = 0; k < 8; ++k) acc[q][k] = 0.f;
   if (PRE > 0) {
@@ -323,7 +326,7 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
       const int ch = chp + NCHP * i;
       if (ch < d)
 #pragma unroll
-        for (int q = 0; q < POOL_ENT; ++q)
+        for (int q = 0; q < ENT; ++q)
           if (q < ne) fma8_bf16(acc[q], pooled[q * d + ch], wpre[i]);
     }
   } else {
@@ -331,7 +334,7 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
     for (int ch = chp; ch < d; ch += NCHP) {
       const uint4 w = __ldg(reinterpret_cast<const uint4*>(P.W_IK + (size_t)ch * d_I + o_base));
 #pragma unroll
-      for (int q = 0; q < POOL_ENT; ++q)
+      for (int q = 0; q < ENT; ++q)
         if (q < ne) fma8_bf16(acc[q], pooled[q * d + ch], w);
     }
   }
@@ -339,20 +342,20 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
 #pragma unroll
   for (int off = NOC; off < 32; off <<= 1)
 #pragma unroll
-    for (int q = 0; q < POOL_ENT; ++q)
+    for (int q = 0; q < ENT; ++q)
 #pragma unroll
       for (int k = 0; k < 8; ++k) acc[q][k] += __shfl_xor_sync(0xffffffffu, acc[q][k], off);
   if (lane < NOC)
 #pragma unroll
-    for (int q = 0; q < POOL_ENT; ++q)
+    for (int q = 0; q < ENT; ++q)
 #pragma unroll
-      for (int k = 0; k < 8; ++k) red[(warp * POOL_ENT + q) * OW + oc * 8 + k] = acc[q][k];
+      for (int k = 0; k < 8; ++k) red[(warp * ENT + q) * OW + oc * 8 + k] = acc[q][k];
   __syncthreads();
   for (int i = tid; i < ne * OW; i += POOL_THREADS) {
     const int q = i / OW, o = i % OW;
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < POOL_WARPS; ++w) v += red[(w * POOL_ENT + q) * OW + o];
+    for (int w = 0; w < POOL_WARPS; ++w) v += red[(w * ENT + q) * OW + o];
     const uint32_t bits = f_to_bf16_bits(v);
     if (P.kI_out) P.kI_out[((size_t)b * n_out + e0 + q) * d_I + z * OW + o] = (uint16_t)bits;
     krow[q * OW + o] = bf16_bits_to_f(bits);
@@ -412,12 +415,15 @@ extern "C" csa_status csa_compress(const csa_compress_args* a, void* stream) {
   if (a->W_IK) CSA_SUPPORTED((a->d_index * 2) % 16 == 0);
   CSA_SUPPORTED(POOL_ENT * (a->d_rope / 2) <= POOL_THREADS && a->d_rope / 2 <= POOL_MAX_HALF);
   // k_I output slices: enough CTAs for about one wave when there are few entry groups
-  const long long groups = (long long)a->B * ((n_out + POOL_ENT - 1) / POOL_ENT);
+  // one entry per CTA when each sequence completes a single group (decode), else POOL_ENT
+  const int ent = n_out == 1 ? 1 : POOL_ENT;
+  const long long groups = (long long)a->B * ((n_out + ent - 1) / ent);
   int OW = a->W_IK ? a->d_index : 32;
   while (a->W_IK && OW > 32 && groups * (a->d_index / OW) * 2 <= 148) OW >>= 1;
   const int nchp = POOL_THREADS / (OW / 8);
   const bool pre = a->W_IK && a->d <= 8 * nchp;
-  const size_t smem = (size_t)POOL_ENT * a->d * sizeof(float) + (size_t)(POOL_WARPS + 1) * POOL_ENT * OW * 4;
+  const bool r4 = ent == 1 && a->ratio == 4;
+  const size_t smem = (size_t)ent * a->d * sizeof(float) + (size_t)(POOL_WARPS + 1) * ent * OW * 4;
   CSA_SUPPORTED(smem <= 200 * 1024);
   PoolParams P{};
   P.C = (const uint16_t*)a->C; P.Z = (const uint16_t*)a->Z; P.b_pos = a->b_pos; P.T = a->T; P.d = a->d;
@@ -426,15 +432,23 @@ extern "C" csa_status csa_compress(const csa_compress_args* a, void* stream) {
   P.ki = a->ki_pack;
   for (int m = 0; m < a->d_rope / 2; ++m)
     P.inv_freq[m] = a->rope_theta != 0.0f ? pow((double)a->rope_theta, -2.0 * m / (double)a->d_rope) : 0.0;
-  dim3 grid((n_out + POOL_ENT - 1) / POOL_ENT, a->B, a->W_IK ? a->d_index / OW : 1);
-  const void* fn;
-  if (OW == 32) fn = pre ? (const void*)pool_kernel<32, 8> : (const void*)pool_kernel<32, 0>;
-  else if (OW == 64) fn = pre ? (const void*)pool_kernel<64, 8> : (const void*)pool_kernel<64, 0>;
-  else fn = pre ? (const void*)pool_kernel<128, 8> : (const void*)pool_kernel<128, 0>;
-  static std::atomic<unsigned> attr_done[6];
-  set_smem_once(fn, 200 * 1024, attr_done[(OW == 32 ? 0 : OW == 64 ? 2 : 4) + (pre ? 1 : 0)]);
+  dim3 grid((n_out + ent - 1) / ent, a->B, a->W_IK ? a->d_index / OW : 1);
+  // kernel variants: [OW 32/64/128][W_IK slice preloaded][one entry, ratio 4 | one entry | POOL_ENT entries]
+  static const void* const table[3][2][3] = {
+      {{(const void*)pool_kernel<32, 0, 1, 4>, (const void*)pool_kernel<32, 0, 1, 0>, (const void*)pool_kernel<32, 0, POOL_ENT, 0>},
+       {(const void*)pool_kernel<32, 8, 1, 4>, (const void*)pool_kernel<32, 8, 1, 0>, (const void*)pool_kernel<32, 8, POOL_ENT, 0>}},
+      {{(const void*)pool_kernel<64, 0, 1, 4>, (const void*)pool_kernel<64, 0, 1, 0>, (const void*)pool_kernel<64, 0, POOL_ENT, 0>},
+       {(const void*)pool_kernel<64, 8, 1, 4>, (const void*)pool_kernel<64, 8, 1, 0>, (const void*)pool_kernel<64, 8, POOL_ENT, 0>}},
+      {{(const void*)pool_kernel<128, 0, 1, 4>, (const void*)pool_kernel<128, 0, 1, 0>, (const void*)pool_kernel<128, 0, POOL_ENT, 0>},
+       {(const void*)pool_kernel<128, 8, 1, 4>, (const void*)pool_kernel<128, 8, 1, 0>, (const void*)pool_kernel<128, 8, POOL_ENT, 0>}}};
+  const int iow = OW == 32 ? 0 : OW == 64 ? 1 : 2, ivar = ent == 1 ? (r4 ? 0 : 1) : 2;
+  const void* fn = table[iow][pre ? 1 : 0][ivar];
+  static std::atomic<unsigned> attr_done[3][2][3];
+  set_smem_once(fn, 200 * 1024, attr_done[iow][pre ? 1 : 0][ivar]);
   void* argv[] = {&P};
-  cudaError_t e = cudaLaunchKernel(fn, grid, dim3(POOL_THREADS), argv, smem, st);
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = pdl_config(grid, dim3(POOL_THREADS), smem, st, attr);
+  cudaError_t e = cudaLaunchKernelExC(&cfg, fn, argv);
   if (e != cudaSuccess) { set_last_cuda_error(e); return CSA_ERR_CUDA; }
   return launch_status();
 }

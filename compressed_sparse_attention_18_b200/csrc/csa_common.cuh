@@ -51,6 +51,41 @@ inline csa_status launch_status() {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// ----------------------------------------------------------------- programmatic dependent launch
+// The step kernels are launched so that they may start while the kernel before them in the stream is
+// still finishing: each does its setup that touches no global memory, then pdl_wait() (the previous
+// grid has completed and its writes are visible) before its first global read.  pdl_trigger() lets the
+// next kernel start launching once every CTA of this one has begun.  Launched any other way, both are
+// no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+inline cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t st, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+template <typename... KArgs, typename... Args>
+inline csa_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args... args) {
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = pdl_config(grid, block, smem, st, attr);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return CSA_ERR_CUDA;
+  }
+  return launch_status();
+}
+
 // Raise a kernel's dynamic shared-memory limit once per device (the attribute is per device); later
 // calls, including those made while a stream is being captured into a CUDA graph, skip the runtime call.
 inline void set_smem_once(const void* func, int bytes, std::atomic<unsigned>& done) {

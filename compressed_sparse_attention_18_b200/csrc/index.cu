@@ -561,7 +561,7 @@ __device__ void hist_find_bin(TopkSmem& sm, const uint32_t* bins, uint32_t R, ui
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, const uint32_t* __restrict__ hist) {
+__global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, uint32_t* __restrict__ hist) {
   // dynamic shared memory: the row [TOPK_CHUNK] (scores, or scores | ids for explicit-id rows), then the
   // boundary-bin candidates: keys [TOPK_HIST_CAND] | ids [TOPK_HIST_CAND]
   extern __shared__ __align__(16) uint32_t s_topk[];
@@ -572,6 +572,8 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
                 TOPK_HIST_PER_THREAD <= 32, "row split");
   static_assert(sizeof(TopkSmem::whist) >= HIST_BINS * 4, "second-level histogram in the per-warp histograms");
   const int row = blockIdx.y;
+  pdl_trigger();
+  pdl_wait();                                  // scores and histogram come from the previous kernel
   int len = min(A.rows_per_seg, A.n_cols);
   if (A.q_pos) {
     const int b = row / A.Nq;
@@ -612,6 +614,9 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
   }
   uint32_t nvalid;
   hist_find_bin(sm, hist + (size_t)row * HIST_BINS, (uint32_t)A.k, &nvalid);   // overlaps the copy
+  // the row's histogram is consumed: leave it zero for the next scoring call (each thread clears the
+  // four bins it read)
+  reinterpret_cast<uint4*>(hist + (size_t)row * HIST_BINS)[blockDim.x - 1 - threadIdx.x] = make_uint4(0, 0, 0, 0);
   const uint32_t K = min((uint32_t)A.k, nvalid);
   const uint32_t Tbin = sm.bcast[0], above = sm.bcast[1], nT = sm.bcast[2];
   const uint32_t need = K - above;
@@ -905,10 +910,13 @@ static csa_status validate_index(const csa_index_args* a, bool need_select) {
   return CSA_OK;
 }
 
-static csa_status run_scores(const csa_index_args* a, float* scores, long long ld, uint32_t* hist, cudaStream_t st) {
+// clear_hist: the histogram is this call's own scratch (fused entry points); a caller's histogram
+// (csa_index_scores) is added into as it stands: zero at first use, and csa_topk clears each row it reads.
+static csa_status run_scores(const csa_index_args* a, float* scores, long long ld, uint32_t* hist, bool clear_hist,
+                             cudaStream_t st) {
   const int n_cols = a->cand ? a->n_cand : a->n_max;
   if (!one_query_per_cta(a)) hist = nullptr;
-  if (hist) {
+  if (hist && clear_hist) {
     cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)a->B * a->Nq * HIST_BINS * 4, st);
     if (e != cudaSuccess) { set_last_cuda_error(e); return CSA_ERR_CUDA; }
   }
@@ -972,8 +980,8 @@ static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const 
     static std::atomic<unsigned> attr_h{0};
     const int smem_h = (TOPK_CHUNK + 2 * TOPK_HIST_CAND) * 4;
     set_smem_once((const void*)topk_hist_kernel, smem_h, attr_h);
-    topk_hist_kernel<<<dim3(1, p.rows), TOPK_THREADS, smem_h, st>>>(ta, hist);
-    csa_status s = launch_status();
+    csa_status s = launch_pdl(topk_hist_kernel, dim3(1, p.rows), dim3(TOPK_THREADS), (size_t)smem_h, st, ta,
+                              const_cast<uint32_t*>(hist));
     if (s != CSA_OK) return s;
   } else if (p.segs == 1) {
     ta.out_idx = a->idx_out;
@@ -1081,7 +1089,7 @@ extern "C" csa_status csa_index_topk_noalloc(const csa_index_args* a, void* stre
   uint8_t* w8 = (uint8_t*)ws;
   float* scores = (float*)(w8 + p.off_scores);
   uint32_t* hist = p.hist ? (uint32_t*)(w8 + p.off_hist) : nullptr;
-  csa_status s = run_scores(a, scores, p.n_cols, hist, st);
+  csa_status s = run_scores(a, scores, p.n_cols, hist, true, st);
   if (s != CSA_OK) return s;
   return run_select(a, p, scores, p.n_cols, hist, w8, st);
 }
@@ -1092,7 +1100,7 @@ extern "C" csa_status csa_index_scores(const csa_index_args* a, float* scores, i
   if ((long long)a->B * a->Nq == 0) return CSA_OK;
   const int n_cols = a->cand ? a->n_cand : a->n_max;
   CSA_REQUIRE(scores != nullptr && ld >= n_cols);
-  return run_scores(a, scores, ld, a->hist, (cudaStream_t)stream);
+  return run_scores(a, scores, ld, a->hist, false, (cudaStream_t)stream);
 }
 
 extern "C" size_t csa_topk_workspace_size(const csa_index_args* a) {
@@ -1130,7 +1138,7 @@ extern "C" csa_status csa_index_topk(const csa_index_args* a, void* ws, size_t w
   uint8_t* w8 = (uint8_t*)ws;
   float* scores = (float*)(w8 + p.off_scores);
   uint32_t* hist = p.hist ? (uint32_t*)(w8 + p.off_hist) : nullptr;
-  csa_status s = run_scores(a, scores, p.n_cols, hist, st);
+  csa_status s = run_scores(a, scores, p.n_cols, hist, true, st);
   if (s != CSA_OK) return s;
   return run_select(a, p, scores, p.n_cols, hist, w8, st);
 }

@@ -87,18 +87,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
   TcSmem& S = *reinterpret_cast<TcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
-  // key tiles of this CTA
-  long long nv = (P.q_pos[b] + 1) / P.ratio;
-  const int ncb = min(P.n_c[b], P.n_max);
-  if (nv > ncb) nv = ncb;
-  if (nv < 0) nv = 0;
-  const int n_vis = (int)nv;
-  const int n_tiles = (n_vis + TC_TILE - 1) / TC_TILE;
-  const int per = (n_tiles + P.ctas_per_row - 1) / P.ctas_per_row;
-  const int t_begin = min(n_tiles, (int)blockIdx.x * per);
-  const int t_end = min(n_tiles, t_begin + per);
-  const int ntile = t_end - t_begin;
-
+  // setup that reads no global memory, then wait for the previous kernel (it may append to the cache)
   if (threadIdx.x == 0) {
     S.err = 0;
     for (int s = 0; s < TC_STAGES; ++s) { mbar_init(&S.full[s], 1); mbar_init(&S.empty[s], 1); }
@@ -113,6 +102,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
   if (warp == 0 && lane == 0) prefetch_tensormap(&kmap);
   for (int i = threadIdx.x; i < TC_HIST_BINS; i += blockDim.x) S.hist[i] = 0;
   if (warp == 1) { tmem_alloc(&S.tmem_base, TC_TMEM_COLS); tmem_relinquish(); }
+  pdl_trigger();
+  pdl_wait();
+  // key tiles of this CTA
+  long long nv = (P.q_pos[b] + 1) / P.ratio;
+  const int ncb = min(P.n_c[b], P.n_max);
+  if (nv > ncb) nv = ncb;
+  if (nv < 0) nv = 0;
+  const int n_vis = (int)nv;
+  const int n_tiles = (n_vis + TC_TILE - 1) / TC_TILE;
+  const int per = (n_tiles + P.ctas_per_row - 1) / P.ctas_per_row;
+  const int t_begin = min(n_tiles, (int)blockIdx.x * per);
+  const int t_end = min(n_tiles, t_begin + per);
+  const int ntile = t_end - t_begin;
+
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = S.tmem_base;
@@ -345,8 +348,7 @@ csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, u
   const int smem = (int)sizeof(TcSmem) + 1024;
   static std::atomic<unsigned> attr_done{0};
   set_smem_once((const void*)index_score_tc_kernel, smem, attr_done);
-  index_score_tc_kernel<<<dim3(per_row, a->B), TC_THREADS, smem, st>>>(map, P);
-  return launch_status();
+  return launch_pdl(index_score_tc_kernel, dim3(per_row, a->B), dim3(TC_THREADS), smem, st, map, P);
 }
 
 cudaError_t compress_take_device_error(uint32_t* out);   // compress.cu

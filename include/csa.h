@@ -168,8 +168,12 @@ typedef struct csa_index_args {
   int32_t* idx_out;
   float* scores_out;
   uint32_t* hist;          /* optional, split calls only: [B*Nq][4096] score histogram that csa_index_scores
-                              fills (single-query rows: Nq == 1 or cand != NULL) and csa_topk uses to find
-                              the k-th score's neighbourhood in one pass; NULL = plain radix selection */
+                              adds into (single-query rows: Nq == 1 or cand != NULL) and csa_topk uses to
+                              find the k-th score's neighbourhood in one pass, leaving every row it read
+                              zero again.  It must be zero before the first csa_index_scores call; a stale
+                              histogram costs time, not correctness (csa_topk checks its counts against
+                              the scores and falls back to the full selection).  NULL = plain radix
+                              selection */
 } csa_index_args;
 
 size_t csa_index_topk_workspace_size(const csa_index_args* args);
