@@ -477,12 +477,12 @@ static csa_status launch_merge(const PT* po, const float* pl, int splits, int H,
 
 // tensor-core decode path (attn_tc.cu)
 bool attn_tc_eligible(const csa_attn_args* a, int hca, int max_splits);
-int attn_tc_splits(const csa_attn_args* a, int hca);
-csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, uint16_t* part_o, float* part_lse,
+void attn_tc_plan(const csa_attn_args* a, int hca, int* splits, int* tpc);
+csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, uint16_t* part_o, float* part_lse,
                           cudaStream_t st);
 
 struct AttnPlan {
-  int splits, cps;
+  int splits, cps, tpc;
   bool tc;
   size_t off_o, off_lse, total;
 };
@@ -493,8 +493,7 @@ static AttnPlan plan_attn(const csa_attn_args* a, int hca) {
   if (attn_tc_eligible(a, hca, MERGE_MAX_SPLITS)) {
     p.tc = true;
     p.cps = 1;
-    p.splits = attn_tc_splits(a, hca);
-    if (p.splits < 1) p.splits = 1;
+    attn_tc_plan(a, hca, &p.splits, &p.tpc);
     size_t o = 0;
     if (p.splits > 1) {
       p.off_o = o;   o = align_up(o + (size_t)rows_tc * p.splits * a->H * a->d * 2, 256);
@@ -563,7 +562,7 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
   if (p.tc) {
     uint16_t* po = p.splits > 1 ? (uint16_t*)((uint8_t*)ws + p.off_o) : nullptr;
     float* pl = p.splits > 1 ? (float*)((uint8_t*)ws + p.off_lse) : nullptr;
-    csa_status s = launch_attn_tc(a, hca, p.splits, po, pl, st);
+    csa_status s = launch_attn_tc(a, hca, p.splits, p.tpc, po, pl, st);
     if (s != CSA_OK || p.splits == 1) return s;
     return launch_merge<uint16_t>(po, pl, p.splits, a->H, a->d, rows, (uint16_t*)a->out, a->lse, st);
   }

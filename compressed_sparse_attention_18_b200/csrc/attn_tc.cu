@@ -40,16 +40,20 @@ struct TaSmem {
   alignas(1024) uint8_t Q[8][64 * 128];        // [dim block][head][128 B]
   alignas(1024) uint8_t P[TA_KEYS * 128];      // [key][64 heads bf16]
   float red_m[4][64], red_l[4][64];            // per lane-quadrant partial max / sum
-  float m[64], inv_l[64], lse[64];
+  alignas(16) float m[64];                     // running max (log2 units)
+  float l[64], fac[64];                        // running sum, this tile's rescale
   int32_t ids[TA_KEYS];                        // entry id of each entry row, -1 if absent
   // per dim block: Q landed, window boxes landed, gathered rows written
   alignas(8) uint64_t bar_q[8], bar_w[8], bar_k[8];
   uint64_t bar_s, bar_p, bar_o[4];
   uint32_t tmem_base;
   uint32_t err;
+  int rescale;                                 // some head's running max moved: O and l are rescaled
 };
+
 struct TaParams {
   int Nq, H, ratio, n_max, k, Wn, window, splits, hca;
+  int tpc;              // key tiles per CTA (a CTA walks tiles split*tpc .. split*tpc + tpc - 1 of its query)
   float g, scale_log2;
   const int64_t* q_pos;
   const uint8_t* codes;
@@ -61,7 +65,7 @@ struct TaParams {
   const int64_t* win_pos0;
   uint16_t* out;        // splits == 1
   float* lse;           // splits == 1 (may be null)
-  uint16_t* part_o;     // [rows][splits][H][512] bf16
+  uint16_t* part_o;     // [rows][splits][H][512] bf16 (splits = CTAs per query)
   float* part_lse;      // [rows][splits][H]
 };
 
@@ -144,6 +148,38 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
   return v[0];
 }
 
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+        "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+        "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Geometry of one 128-key tile of a query's key list [n_sel entries ‖ window rows].
+struct TaTile {
+  int key0, rs, rw, wa, we, zs;
+  long long wrow_base;     // window buffer row of tile row r (r >= rs) is wrow_base + r
+};
+__device__ __forceinline__ TaTile ta_tile(int key0, int n_sel, int n_list, long long wlo, long long p0) {
+  TaTile g;
+  g.key0 = key0;
+  g.rs = min(max(n_sel - key0, 0), TA_KEYS);                        // rows [0, rs): entries
+  g.rw = max(min(n_list - key0, TA_KEYS), 0);                       // rows [rs, rw): window, then empty
+  g.wa = (g.rs + TA_WBOX - 1) / TA_WBOX * TA_WBOX;                   // window rows >= wa come by TMA boxes
+  g.we = g.rw > g.wa ? (g.rw + TA_WBOX - 1) / TA_WBOX * TA_WBOX : g.wa;
+  g.zs = g.rw > g.wa ? g.we : g.rw;                                  // rows >= zs are zero-filled
+  g.wrow_base = (wlo - p0) + (long long)(key0 - n_sel);
+  return g;
+}
+
+// Lazy rescaling: a head keeps its running max until a tile's max exceeds it by more than this (log2
+// units), so probabilities stay <= 2^8 and O is rescaled in tensor memory only when a max jumps.
+constexpr float TA_RESCALE_SLACK = 8.0f;
+
 __global__ void __launch_bounds__(TA_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap wmap,
                    const TaParams P) {
@@ -152,7 +188,6 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bq = blockIdx.x / P.splits, split = blockIdx.x % P.splits;
   const int b = bq / P.Nq;
-  const int key0 = split * TA_KEYS;
   // worker thread t owns tile row t/2 for the gather (its half of the row's FP4 blocks and RoPE slice)
   const int grow = (tid & (TA_WORKERS - 1)) >> 1, ghalf = tid & 1;
   // setup that reads no global memory, then wait for the previous kernel (it writes the selected ids)
@@ -175,10 +210,10 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
     tmem_alloc(&S.tmem_base, TA_TMEM_COLS);
     tmem_relinquish();
   }
+  if (tid < 64) { S.m[tid] = -INFINITY; S.l[tid] = 0.f; }
+  if (tid == 0) S.rescale = 0;
   pdl_trigger();
   pdl_wait();
-  int id_raw = -1;
-  if (!P.hca && tid < TA_WORKERS && key0 + grow < P.k) id_raw = P.idx[(size_t)bq * P.k + key0 + grow];
   const long long tq = P.q_pos[bq];
   const int ncb = min(P.n_c[b], P.n_max);
   int n_sel = P.k;
@@ -194,28 +229,14 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   }
   const int n_list = n_sel + (whi >= wlo ? (int)(whi - wlo + 1) : 0);
   const size_t unit_ho = ((size_t)bq * P.splits + split) * P.H;
-  // tile rows: [0, rs) entries, [rs, rw) window rows, [rw, 128) empty
-  const int rs = min(max(n_sel - key0, 0), TA_KEYS);
-  const int rw = max(min(n_list - key0, TA_KEYS), 0);
-  const int wa = (rs + TA_WBOX - 1) / TA_WBOX * TA_WBOX;            // window rows >= wa come by TMA boxes
-  const int we = rw > wa ? (rw + TA_WBOX - 1) / TA_WBOX * TA_WBOX : wa;
-  const int zs = rw > wa ? we : rw;                                 // rows >= zs are zero-filled
-  // window buffer row of tile row r (r >= rs)
-  const long long wrow_base = (wlo - p0) + (long long)(key0 - n_sel);
-  // entry ids of the tile rows for the softmax masks (the gather threads keep their own copies)
-  if (tid < TA_WORKERS && ghalf == 0) {
-    int id = -1;
-    if (grow < rs) {
-      const int v = P.hca ? key0 + grow : id_raw;
-      if (v >= 0 && v < ncb) id = v;
-    }
-    S.ids[grow] = id;
-  }
+  const int first_key = split * P.tpc * TA_KEYS;
+  // non-empty tiles of this CTA (block-uniform)
+  const int ntile = max(0, min(P.tpc, (n_list - first_key + TA_KEYS - 1) / TA_KEYS));
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = S.tmem_base;
 
-  if (key0 >= n_list) {                          // nothing in this tile: an empty partial
+  if (ntile == 0) {                              // nothing in this CTA's tiles: an empty partial
     if (P.splits > 1) {
       if (tid < P.H) P.part_lse[unit_ho + tid] = -INFINITY;
     } else {
@@ -230,45 +251,59 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   if (warp == 8) {
     // ------------------------------------------------------------------ control: TMA, then MMA issue
     if (lane == 0) {
-      const int nbox = (we - wa) / TA_WBOX;
+      bool ok = true;
 #pragma unroll 1
       for (int j = 0; j < 8; ++j) {
         mbar_arrive_expect_tx(&S.bar_q[j], 64 * 128);
         tma_load_3d(S.Q[j], &qmap, j * 64, 0, bq, &S.bar_q[j]);
-        mbar_arrive_expect_tx(&S.bar_w[j], (uint32_t)(nbox * TA_WBOX * 128));
-        for (int i = 0; i < nbox; ++i)
-          tma_load_3d(&S.K[j][(wa + i * TA_WBOX) * 128], &wmap, j * 64, (int)(wrow_base + wa + i * TA_WBOX), b,
-                      &S.bar_w[j]);
       }
-      bool ok = true;
       const uint32_t ids = idesc_bf16(128, 64, 0, 0);
-#pragma unroll 1
-      for (int j = 0; j < 8 && ok; ++j) {
-        ok = mbar_wait(&S.bar_q[j], 0) && mbar_wait(&S.bar_w[j], 0) && mbar_wait(&S.bar_k[j], 0);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          const uint64_t a = smem_desc(smem_addr(S.K[j]) + s * 32, 16, 1024, 2);
-          const uint64_t bd = smem_desc(smem_addr(S.Q[j]) + s * 32, 16, 1024, 2);
-          mma_bf16_ss(tb + TA_COL_S, a, bd, ids, (j | s) != 0);
-        }
-      }
-      mma_commit(&S.bar_s);
-      ok = ok && mbar_wait(&S.bar_p, 0);
-      if (ok) tc_fence_after();
       const uint32_t ido = idesc_bf16(128, 64, 1, 1);
 #pragma unroll 1
-      for (int mt = 0; mt < 4; ++mt) {
-        if (ok) {
+      for (int t = 0; t < ntile; ++t) {
+        const TaTile g = ta_tile(first_key + t * TA_KEYS, n_sel, n_list, wlo, p0);
+        const int nbox = (g.we - g.wa) / TA_WBOX;
+        // window boxes overwrite the K tile: only once the previous tile's O MMAs have completed (S MMAs
+        // of an entry tile are queued behind them directly)
+        if (t > 0 && nbox > 0 && ok) ok = mbar_wait(&S.bar_o[3], (t - 1) & 1);
+#pragma unroll 1
+        for (int j = 0; j < 8; ++j) {
+          mbar_arrive_expect_tx(&S.bar_w[j], (uint32_t)(nbox * TA_WBOX * 128));
+          if (ok)
+            for (int i = 0; i < nbox; ++i)
+              tma_load_3d(&S.K[j][(g.wa + i * TA_WBOX) * 128], &wmap, j * 64,
+                          (int)(g.wrow_base + g.wa + i * TA_WBOX), b, &S.bar_w[j]);
+        }
+        // S^T = K Q^T, dim block by dim block as the blocks land
+#pragma unroll 1
+        for (int j = 0; j < 8 && ok; ++j) {
+          ok = (t > 0 || mbar_wait(&S.bar_q[j], 0)) && mbar_wait(&S.bar_w[j], t & 1) &&
+               mbar_wait(&S.bar_k[j], t & 1);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            const uint64_t a = smem_desc(smem_addr(S.K[2 * mt]) + s * 2048, 16384, 1024, 2);
-            const uint64_t bd = smem_desc(smem_addr(S.P) + s * 2048, 16384, 1024, 2);
-            mma_bf16_ss(tb + TA_COL_O + 64 * mt, a, bd, ido, s > 0);
+          for (int s2 = 0; s2 < 4; ++s2) {
+            const uint64_t a = smem_desc(smem_addr(S.K[j]) + s2 * 32, 16, 1024, 2);
+            const uint64_t bd = smem_desc(smem_addr(S.Q[j]) + s2 * 32, 16, 1024, 2);
+            mma_bf16_ss(tb + TA_COL_S, a, bd, ids, (j | s2) != 0);
           }
         }
-        mma_commit(&S.bar_o[mt]);
+        mma_commit(&S.bar_s);
+        // O^T (+)= V^T P^T (the K tile read MN-major, P stored [key][head]); O accumulates across tiles
+        ok = ok && mbar_wait(&S.bar_p, t & 1);
+        if (ok) tc_fence_after();
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt) {
+          if (ok) {
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+              const uint64_t a = smem_desc(smem_addr(S.K[2 * mt]) + s2 * 2048, 16384, 1024, 2);
+              const uint64_t bd = smem_desc(smem_addr(S.P) + s2 * 2048, 16384, 1024, 2);
+              mma_bf16_ss(tb + TA_COL_O + 64 * mt, a, bd, ido, t > 0 || s2 > 0);
+            }
+          }
+          mma_commit(&S.bar_o[mt]);
+        }
       }
       if (!ok) atomicOr(&S.err, 1u);
     }
@@ -278,129 +313,204 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
     const uint8_t* codes_b = P.codes + (size_t)b * P.n_max * 224;
     const uint8_t* scales_b = P.scales + (size_t)b * P.n_max * 16;
     const uint16_t* rope_b = P.rope + (size_t)b * P.n_max * 64;
-    int id = -1;
-    if (grow < rs) {
-      const int v = P.hca ? key0 + grow : id_raw;
-      if (v >= 0 && v < ncb) id = v;
-    }
-    // FP4 blocks 2j + ghalf (j = 0..6) of the row and its scale row; loads first
-    uint4 cv[7];
-    uint4 sc16 = make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int j = 0; j < 7; ++j) cv[j] = make_uint4(0, 0, 0, 0);
-    if (id >= 0) {
-      const uint8_t* crow = codes_b + (size_t)id * 224 + ghalf * 16;
-#pragma unroll
-      for (int j = 0; j < 7; ++j) cv[j] = __ldg(reinterpret_cast<const uint4*>(crow + j * 32));
-      sc16 = __ldg(reinterpret_cast<const uint4*>(scales_b + (size_t)id * 16));
-    }
-    // RoPE slice (dim block 7): 4 x 16 B of the row per thread
-    if (grow < rs) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int part = ghalf * 4 + c;
-        uint8_t* dst = &S.K[7][sw128(grow, part)];
-        if (id >= 0) cp16(dst, rope_b + (size_t)id * 64 + part * 8);
-        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-      }
-    }
-    // window rows before the first TMA box, by asynchronous copies
-    {
-      const int r_end = min(wa, rw);
-      const int n = (r_end > rs ? r_end - rs : 0) * 64;
-      for (int i = tid; i < n; i += TA_WORKERS) {
-        const int row = rs + (i >> 6), c = i & 63;
-        const long long wr = wrow_base + row;
-        cp16(&S.K[c >> 3][sw128(row, c & 7)], P.win + ((size_t)b * P.Wn + wr) * 512 + c * 8);
-      }
-    }
-    // empty rows
-    for (int i = tid; i < (TA_KEYS - zs) * 64; i += TA_WORKERS) {
-      const int row = zs + (i >> 6), c = i & 63;
-      *reinterpret_cast<uint4*>(&S.K[c >> 3][sw128(row, c & 7)]) = make_uint4(0, 0, 0, 0);
-    }
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-    // dequantise dim block by dim block: bf16(e2m1 * bf16(e4m3 * g)); each block released to the MMA warp
-    const uint32_t scw[4] = {sc16.x, sc16.y, sc16.z, sc16.w};
-#pragma unroll
-    for (int j = 0; j < 7; ++j) {
-      if (grow < rs) {
-        const int part = 2 * j + ghalf;
-        const uint32_t sb = f_to_bf16_bits(e4m3_to_f32((scw[part >> 2] >> ((part & 3) * 8)) & 0xFFu) * P.g);
-        const uint32_t sc2 = sb | (sb << 16);
-        const uint32_t w4[4] = {cv[j].x, cv[j].y, cv[j].z, cv[j].w};
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          *reinterpret_cast<uint4*>(&S.K[j][sw128(grow, ghalf * 4 + q4)]) = e2m1x8_to_bf16_scaled(w4[q4], sc2);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.bar_k[j]);
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&S.bar_k[7]);
-    asm volatile("bar.sync 1, 256;" ::: "memory");   // workers only: ids visible to the softmax
-
-    // ---- softmax: warp w reads lanes 32*(w%4).. (its keys) and head half w/4
     const int quad = warp & 3, hh = warp >> 2;
     const int key = 32 * quad + lane;
     const uint32_t lane_base = tb + ((uint32_t)(32 * quad) << 16);
-    bool ok = mbar_wait(&S.bar_s, 0);
-    tc_fence_after();
-    float z[32], red[32];
-    {
-      uint32_t sv[32];
-      tmem_ld_x32(lane_base + TA_COL_S + hh * 32, sv);
-      tmem_wait_ld_x32(sv);
-      const bool valid = key < rs ? (S.ids[key] >= 0) : (key < rw);
+    bool ok = true;
+    // this thread's row of a tile: entry id and its FP4 blocks 2j + ghalf, scale row and RoPE quarter,
+    // loaded one tile ahead (registers)
+    // raw id of this thread's row of a tile (loaded one tile before it is used), then its check
+    auto raw_id = [&](const TaTile& g) -> int {
+      const int li = g.key0 + grow;
+      if (grow >= g.rs) return -1;
+      return P.hca ? li : (li < P.k ? P.idx[(size_t)bq * P.k + li] : -1);
+    };
+    auto check_id = [&](int v) -> int { return (v >= 0 && v < ncb) ? v : -1; };
+    uint4 cv[7], sc16, rp[4];
+    auto load_row = [&](int id) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        z[j] = valid ? __uint_as_float(sv[j]) * P.scale_log2 : -INFINITY;
-        red[j] = z[j];
+      for (int j = 0; j < 7; ++j) cv[j] = make_uint4(0, 0, 0, 0);
+      sc16 = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) rp[c] = make_uint4(0, 0, 0, 0);
+      if (id >= 0) {
+        const uint8_t* crow = codes_b + (size_t)id * 224 + ghalf * 16;
+#pragma unroll
+        for (int j = 0; j < 7; ++j) cv[j] = __ldg(reinterpret_cast<const uint4*>(crow + j * 32));
+        sc16 = __ldg(reinterpret_cast<const uint4*>(scales_b + (size_t)id * 16));
+        const uint4* rrow = reinterpret_cast<const uint4*>(rope_b + (size_t)id * 64) + ghalf * 4;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) rp[c] = __ldg(rrow + c);
       }
-    }
-    S.red_m[quad][hh * 32 + lane] = transpose_reduce32<true>(red, lane);
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (tid < 64) S.m[tid] = fmaxf(fmaxf(S.red_m[0][tid], S.red_m[1][tid]), fmaxf(S.red_m[2][tid], S.red_m[3][tid]));
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    {
-      uint32_t pk[16];
-#pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float m0 = S.m[hh * 32 + j], m1 = S.m[hh * 32 + j + 1];
-        const float p0 = m0 == -INFINITY ? 0.f : exp2f(z[j] - m0);
-        const float p1 = m1 == -INFINITY ? 0.f : exp2f(z[j + 1] - m1);
-        red[j] = p0;
-        red[j + 1] = p1;
-        pk[j >> 1] = pack_bf16x2(p0, p1);
+    };
+    TaTile g = ta_tile(first_key, n_sel, n_list, wlo, p0);
+    int id = check_id(raw_id(g));
+    int id_next = ntile > 1 ? raw_id(ta_tile(first_key + TA_KEYS, n_sel, n_list, wlo, p0)) : -1;
+    load_row(id);
+#pragma unroll 1
+    for (int t = 0; t < ntile; ++t) {
+      // a tile of entry rows only can be refilled block by block as the previous tile's O MMAs release
+      // them (O M-tile mt reads dim blocks 2mt, 2mt+1); any other tile waits for all of them first
+      const bool pure = g.rs == TA_KEYS;
+      if (t > 0 && !pure) {
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt) ok = mbar_wait(&S.bar_o[mt], (t - 1) & 1) && ok;
+        tc_fence_after();
       }
+      if (ghalf == 0) S.ids[grow] = id;
+      if (!pure) {
+        // window rows before the first TMA box, by asynchronous copies
+        const int r_end = min(g.wa, g.rw);
+        const int n = (r_end > g.rs ? r_end - g.rs : 0) * 64;
+        for (int i = tid; i < n; i += TA_WORKERS) {
+          const int row = g.rs + (i >> 6), c = i & 63;
+          const long long wr = g.wrow_base + row;
+          cp16(&S.K[c >> 3][sw128(row, c & 7)], P.win + ((size_t)b * P.Wn + wr) * 512 + c * 8);
+        }
+        // empty rows
+        for (int i = tid; i < (TA_KEYS - g.zs) * 64; i += TA_WORKERS) {
+          const int row = g.zs + (i >> 6), c = i & 63;
+          *reinterpret_cast<uint4*>(&S.K[c >> 3][sw128(row, c & 7)]) = make_uint4(0, 0, 0, 0);
+        }
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+      }
+      // dequantise dim block by dim block: bf16(e2m1 * bf16(e4m3 * g)); each block released to the MMA warp
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        *reinterpret_cast<uint4*>(&S.P[sw128(key, hh * 4 + c)]) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&S.bar_p);
-    S.red_l[quad][hh * 32 + lane] = transpose_reduce32<false>(red, lane);
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (tid < 64) {
-      const float l = (S.red_l[0][tid] + S.red_l[1][tid]) + (S.red_l[2][tid] + S.red_l[3][tid]);
-      S.inv_l[tid] = l > 0.f ? 1.f / l : 0.f;
-      S.lse[tid] = l > 0.f ? (S.m[tid] + log2f(l)) * TA_LN2 : -INFINITY;
-    }
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+      for (int j = 0; j < 7; ++j) {
+        if (t > 0 && pure && (j & 1) == 0) {
+          ok = mbar_wait(&S.bar_o[j >> 1], (t - 1) & 1) && ok;
+          tc_fence_after();
+        }
+        if (grow < g.rs) {
+          const int part = 2 * j + ghalf;                  // word (2j + ghalf) / 4 of the scale row: j / 2
+          const uint32_t word = (j >> 1) == 0 ? sc16.x : (j >> 1) == 1 ? sc16.y : (j >> 1) == 2 ? sc16.z : sc16.w;
+          const uint32_t sb = f_to_bf16_bits(e4m3_to_f32((word >> ((part & 3) * 8)) & 0xFFu) * P.g);
+          const uint32_t sc2 = sb | (sb << 16);
+          const uint32_t w4[4] = {cv[j].x, cv[j].y, cv[j].z, cv[j].w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<uint4*>(&S.K[j][sw128(grow, ghalf * 4 + q4)]) = e2m1x8_to_bf16_scaled(w4[q4], sc2);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.bar_k[j]);
+      }
+      if (t > 0 && pure) {
+        ok = mbar_wait(&S.bar_o[3], (t - 1) & 1) && ok;
+        tc_fence_after();
+      }
+      // RoPE slice (dim block 7) of the entry rows
+      if (grow < g.rs) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(&S.K[7][sw128(grow, ghalf * 4 + c)]) = rp[c];
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.bar_k[7]);
+      const TaTile gt = g;
+      // next tile's row (its id arrived during this tile's gather), in flight during this tile's softmax
+      // and MMAs; the id of the tile after it is requested now
+      if (t + 1 < ntile) {
+        g = ta_tile(first_key + (t + 1) * TA_KEYS, n_sel, n_list, wlo, p0);
+        id = check_id(id_next);
+        load_row(id);
+        id_next = t + 2 < ntile ? raw_id(ta_tile(first_key + (t + 2) * TA_KEYS, n_sel, n_list, wlo, p0)) : -1;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");   // workers only: ids visible to the softmax
 
-    // ---- epilogue, M-tile by M-tile as the O MMAs complete: lane = dim, columns = heads
+      // ---- softmax of this tile: warp w reads lanes 32*(w%4).. (its keys) and head half w/4
+      ok = mbar_wait(&S.bar_s, t & 1) && ok;
+      tc_fence_after();
+      // one 32-value array per thread: the scores for the max, reloaded from tensor memory for the
+      // probabilities, which then feed the sum
+      const bool valid = key < gt.rs ? (S.ids[key] >= 0) : (key < gt.rw);
+      float red[32];
+      {
+        uint32_t sv[32];
+        tmem_ld_x32(lane_base + TA_COL_S + hh * 32, sv);
+        tmem_wait_ld_x32(sv);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) red[j] = valid ? __uint_as_float(sv[j]) * P.scale_log2 : -INFINITY;
+      }
+      S.red_m[quad][hh * 32 + lane] = transpose_reduce32<true>(red, lane);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (tid < 64) {
+        const float mt = fmaxf(fmaxf(S.red_m[0][tid], S.red_m[1][tid]), fmaxf(S.red_m[2][tid], S.red_m[3][tid]));
+        const float mo = S.m[tid];
+        float mn = mo, f = 1.f;
+        if (mt > mo + TA_RESCALE_SLACK || (mo == -INFINITY && mt > -INFINITY)) {
+          mn = mt;
+          f = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+        }
+        S.m[tid] = mn;
+        S.fac[tid] = f;
+        S.l[tid] *= f;
+        if (f != 1.f && t > 0) S.rescale = 1;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (t > 0 && S.rescale) {
+        // a running max moved: scale the accumulated O^T columns of this thread's heads
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt) {
+          uint32_t ov[32];
+          tmem_ld_x32(lane_base + TA_COL_O + 64 * mt + hh * 32, ov);
+          tmem_wait_ld_x32(ov);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * S.fac[hh * 32 + j]);
+          tmem_st_x32(lane_base + TA_COL_O + 64 * mt + hh * 32, ov);
+        }
+        tmem_wait_st();
+      }
+      {
+        uint32_t sv[32];
+        tmem_ld_x32(lane_base + TA_COL_S + hh * 32, sv);
+        tmem_wait_ld_x32(sv);
+        uint32_t pk[16];
+        float mh[32];
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 v4 = *reinterpret_cast<const float4*>(&S.m[hh * 32 + j]);
+          mh[j] = v4.x; mh[j + 1] = v4.y; mh[j + 2] = v4.z; mh[j + 3] = v4.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float m0 = mh[j], m1 = mh[j + 1];
+          const float z0 = valid ? __uint_as_float(sv[j]) * P.scale_log2 : -INFINITY;
+          const float z1 = valid ? __uint_as_float(sv[j + 1]) * P.scale_log2 : -INFINITY;
+          const float p0f = m0 == -INFINITY ? 0.f : exp2f(z0 - m0);
+          const float p1f = m1 == -INFINITY ? 0.f : exp2f(z1 - m1);
+          red[j] = p0f;
+          red[j + 1] = p1f;
+          pk[j >> 1] = pack_bf16x2(p0f, p1f);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(&S.P[sw128(key, hh * 4 + c)]) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.bar_p);
+      S.red_l[quad][hh * 32 + lane] = transpose_reduce32<false>(red, lane);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (tid < 64) S.l[tid] += (S.red_l[0][tid] + S.red_l[1][tid]) + (S.red_l[2][tid] + S.red_l[3][tid]);
+      if (tid == 0) S.rescale = 0;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+    }
+
+    // ---- epilogue, M-tile by M-tile as the last O MMAs complete: lane = dim, columns = heads
     float il[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) il[j] = S.inv_l[hh * 32 + j];
+    for (int j = 0; j < 32; ++j) {
+      const float lj = S.l[hh * 32 + j];
+      il[j] = lj > 0.f ? 1.f / lj : 0.f;
+    }
     const int hmax = min(32, P.H - hh * 32);
+    const int tl = ntile - 1;
 #pragma unroll 1
     for (int mt = 0; mt < 4; ++mt) {
-      ok = mbar_wait(&S.bar_o[mt], 0) && ok;
+      ok = mbar_wait(&S.bar_o[mt], tl & 1) && ok;
       tc_fence_after();
       uint32_t ov[32];
       tmem_ld_x32(lane_base + TA_COL_O + 64 * mt + hh * 32, ov);
@@ -420,10 +530,12 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
     }
     if (!ok && lane == 0) atomicOr(&S.err, 1u);
     if (tid < P.H) {
+      const float lh = S.l[tid];
+      const float ls = lh > 0.f ? (S.m[tid] + log2f(lh)) * TA_LN2 : -INFINITY;
       if (P.splits == 1) {
-        if (P.lse) P.lse[(size_t)bq * P.H + tid] = S.lse[tid];
+        if (P.lse) P.lse[(size_t)bq * P.H + tid] = ls;
       } else {
-        P.part_lse[unit_ho + tid] = S.lse[tid];
+        P.part_lse[unit_ho + tid] = ls;
       }
     }
     tc_fence_before();
@@ -436,22 +548,31 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   }
 }
 
-int attn_tc_splits(const csa_attn_args* a, int hca) {
+// Key tiles per query and the CTAs that share them: one tile per CTA while the grid fits one wave of
+// the 148 SMs, else enough tiles per CTA (walked in order, online softmax) to come back to one wave.
+void attn_tc_plan(const csa_attn_args* a, int hca, int* splits, int* tpc) {
   const long long n_win = (a->win_kv && a->Wn > 0) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
   const long long n = (hca ? a->n_max : a->k) + n_win;
-  return (int)((n + TA_KEYS - 1) / TA_KEYS);
+  const long long tiles = n > 0 ? (n + TA_KEYS - 1) / TA_KEYS : 1;
+  const long long rows = (long long)a->B * a->Nq;
+  long long t = (rows * tiles + 147) / 148;
+  if (t < 1) t = 1;
+  if (t > tiles) t = tiles;
+  *tpc = (int)t;
+  *splits = (int)((tiles + t - 1) / t);
 }
 
 bool attn_tc_eligible(const csa_attn_args* a, int hca, int max_splits) {
-  const int splits = attn_tc_splits(a, hca);
+  int splits = 0, tpc = 0;
+  attn_tc_plan(a, hca, &splits, &tpc);
   return a->d == 512 && a->d_rope == 64 && a->H <= 64 && splits >= 1 && splits <= max_splits &&
          ((uintptr_t)a->q & 15) == 0 && (a->n_max == 0 || (((uintptr_t)a->kv_codes & 15) == 0 &&
                                                            ((uintptr_t)a->kv_rope & 15) == 0)) &&
          (!a->win_kv || a->Wn == 0 || ((uintptr_t)a->win_kv & 15) == 0) && tensor_map_encoder() != nullptr;
 }
 
-csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, uint16_t* part_o, float* part_lse,
-                          cudaStream_t st) {
+csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, uint16_t* part_o,
+                          float* part_lse, cudaStream_t st) {
   const long long rows = (long long)a->B * a->Nq;
   CUtensorMap qmap, wmap;
   {
@@ -479,7 +600,7 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, uint16_t*
   }
   TaParams P{};
   P.Nq = a->Nq; P.H = a->H; P.ratio = a->ratio; P.n_max = a->n_max; P.k = hca ? 0 : a->k;
-  P.Wn = Wn; P.window = a->window; P.splits = splits; P.hca = hca; P.g = a->g_kv;
+  P.Wn = Wn; P.window = a->window; P.splits = splits; P.tpc = tpc; P.hca = hca; P.g = a->g_kv;
   const float scale = a->softmax_scale != 0.0f ? a->softmax_scale : 1.0f / sqrtf((float)a->d);
   P.scale_log2 = scale * TA_LOG2E;
   P.q_pos = a->q_pos; P.codes = a->kv_codes; P.scales = a->kv_scales;

@@ -29,7 +29,7 @@ namespace csa {
 
 using namespace sm100;
 
-constexpr int TC_STAGES = 4;
+constexpr int TC_STAGES = 5;
 constexpr int TC_SUB = 128;                      // keys per MMA (M)
 constexpr int TC_TILE = 2 * TC_SUB;              // keys per TMA box / pipeline step
 constexpr int TC_CODE_BYTES = TC_TILE * 64;      // 256 keys x 128 FP4
