@@ -224,11 +224,11 @@ def index_topk(q_I, w, kcache: PackedCache, n_c, q_pos, *, ratio, k, g_q=1.0, ca
 
 
 def index_scores(q_I, w, kcache: PackedCache, n_c, q_pos, scores, *, ratio, g_q=1.0, cand=None, hist=None,
-                 stream=None):
+                 k=None, stream=None):
     """Lightning-indexer scores only, into scores [B*Nq, ld] fp32 (see csa_index_scores); hist
     ([B*Nq, 4096] uint32 as int32, optional, zero before first use) receives the score histogram for
-    topk(), which leaves it zero again."""
-    a = _index_args(q_I, w, kcache, n_c, q_pos, ratio, 1, g_q, cand, 0, 8, None, None, None)
+    topk(), which leaves it zero again; k (optional) is recorded in the call's arguments."""
+    a = _index_args(q_I, w, kcache, n_c, q_pos, ratio, k if k is not None else 1, g_q, cand, 0, 8, None, None, None)
     a.hist = _ptr(hist)
     _check(_lib.csa_index_scores(ctypes.byref(a), _ptr(scores), scores.shape[-1], _stream(stream)),
            "csa_index_scores")

@@ -561,6 +561,102 @@ __device__ void hist_find_bin(TopkSmem& sm, const uint32_t* bins, uint32_t R, ui
   __syncthreads();
 }
 
+// The `need` best of the nT boundary-bin candidates (keys, ids in shared memory) by (key desc, id asc),
+// written at oi/os[above ..]: all of them when they are exactly needed, by rank for a few, else by 8-bit
+// digit levels.  Block-wide (every thread of the block calls it); s_cnt: two words of shared memory.
+__device__ void resolve_boundary(TopkSmem& sm, uint32_t* ckeys, int32_t* cids, uint32_t nT, uint32_t need,
+                                 uint32_t above, int32_t* oi, float* os, uint32_t* s_cnt) {
+  if (need == nT) {
+    for (int j = threadIdx.x; j < (int)nT; j += blockDim.x) {
+      oi[above + j] = cids[j];
+      if (os) os[above + j] = order_key_float(ckeys[j]);
+    }
+  } else if (nT <= (uint32_t)TOPK_RANK_MAX) {
+    if (threadIdx.x < 32) warp_rank_select(ckeys, cids, (int)nT, need, oi, os, above);
+  } else {
+    // boundary bin: 8-bit digits of the remaining key bits (19..12, 11..4, 3..0), one 256-bin histogram
+    // per level scanned by one warp, until at most TOPK_RANK_MAX candidates share the threshold prefix;
+    // those go by rank (key, id, position), all of them by the block radix path if that never happens
+    uint32_t* h2 = &sm.whist[0][0];                                // 256 bins
+    uint32_t* k2 = &sm.whist[1][0];                                // TOPK_RANK_MAX keys, then ids
+    int32_t* i2 = reinterpret_cast<int32_t*>(&sm.whist[1][TOPK_RANK_MAX]);
+    uint32_t pref = 0, pmask = 0, rem = need, base_out = above, n_in = nT;
+    bool ranked = false;
+#pragma unroll 1
+    for (int level = 0; level < 3 && !ranked; ++level) {
+      const int sh = level == 0 ? 12 : level == 1 ? 4 : 0;
+      const uint32_t dm = level == 2 ? 15u : 255u;
+      if (threadIdx.x < 256) h2[threadIdx.x] = 0;
+      if (threadIdx.x == 0) { s_cnt[0] = 0; s_cnt[1] = 0; }
+      __syncthreads();
+      for (int j = threadIdx.x; j < (int)nT; j += blockDim.x) {
+        const uint32_t k = ckeys[j] & 0xFFFFFu;
+        if ((k & pmask) == pref) atomicAdd(&h2[(k >> sh) & dm], 1u);
+      }
+      __syncthreads();
+      if (threadIdx.x < 32) {
+        // lane l owns digits 8(31-l) .. 8(31-l)+7, highest first
+        const int lane = threadIdx.x;
+        uint32_t c[8], tot = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { c[i] = h2[8 * (31 - lane) + 7 - i]; tot += c[i]; }
+        uint32_t incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        uint32_t acc = incl - tot;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (acc < rem && acc + c[i] >= rem) {
+            sm.bcast[0] = 8 * (31 - lane) + 7 - i;
+            sm.bcast[1] = acc;
+            sm.bcast[2] = c[i];
+          }
+          acc += c[i];
+        }
+      }
+      __syncthreads();
+      const uint32_t digit = sm.bcast[0], above2 = sm.bcast[1], n2 = sm.bcast[2];
+      const uint32_t npref = pref | (digit << sh), nmask = pmask | (dm << sh);
+      // write the candidates in a higher digit; keep the threshold digit's few for ranking
+      for (int j = threadIdx.x; j < (int)nT; j += blockDim.x) {
+        const uint32_t k = ckeys[j] & 0xFFFFFu;
+        if ((k & pmask) != pref) continue;
+        const uint32_t dj = (k >> sh) & dm;
+        if (dj > digit) {
+          const uint32_t slot = base_out + atomicAdd(&s_cnt[0], 1u);
+          oi[slot] = cids[j];
+          if (os) os[slot] = order_key_float(ckeys[j]);
+        } else if (dj == digit && n2 <= (uint32_t)TOPK_RANK_MAX) {
+          const uint32_t slot = atomicAdd(&s_cnt[1], 1u);
+          k2[slot] = ckeys[j];
+          i2[slot] = cids[j];
+        }
+      }
+      __syncthreads();
+      base_out += above2;
+      rem -= above2;
+      pref = npref;
+      pmask = nmask;
+      n_in = n2;
+      if (n2 <= (uint32_t)TOPK_RANK_MAX) {
+        if (threadIdx.x < 32) warp_rank_select(k2, i2, (int)n2, rem, oi, os, base_out);
+        ranked = true;
+      }
+    }
+    if (!ranked) {
+      // more than TOPK_RANK_MAX candidates with one full key: exact selection among them
+      for (int j = threadIdx.x; j < (int)nT; j += blockDim.x)
+        if ((ckeys[j] & 0xFFFFFu) != pref) ckeys[j] = 0u;
+      __syncthreads();
+      auto idof = [&](int j) -> uint32_t { return (uint32_t)cids[j]; };
+      select_in_smem(sm, ckeys, (int)nT, rem, n_in, idof, oi, os, base_out);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, uint32_t* __restrict__ hist) {
   // dynamic shared memory: the row [TOPK_CHUNK] (scores, or scores | ids for explicit-id rows), then the
   // boundary-bin candidates: keys [TOPK_HIST_CAND] | ids [TOPK_HIST_CAND]
@@ -692,95 +788,7 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
   // every thread takes the same branch: `done` depends only on block-uniform values
   if (done) {
     __syncthreads();
-    if (need == nT) {
-      for (int j = threadIdx.x; j < (int)nT; j += blockDim.x) {
-        oi[above + j] = cids[j];
-        if (os) os[above + j] = order_key_float(ckeys[j]);
-      }
-    } else if (nT <= (uint32_t)TOPK_RANK_MAX) {
-      if (threadIdx.x < 32) warp_rank_select(ckeys, cids, (int)nT, need, oi, os, above);
-    } else {
-      // boundary bin: 8-bit digits of the remaining key bits (19..12, 11..4, 3..0), one 256-bin histogram
-      // per level scanned by one warp, until at most TOPK_RANK_MAX candidates share the threshold prefix;
-      // those go by rank (key, id, position), all of them by the block radix path if that never happens
-      uint32_t* h2 = &sm.whist[0][0];                                // 256 bins
-      uint32_t* k2 = &sm.whist[1][0];                                // TOPK_RANK_MAX keys, then ids
-      int32_t* i2 = reinterpret_cast<int32_t*>(&sm.whist[1][TOPK_RANK_MAX]);
-      uint32_t pref = 0, pmask = 0, rem = need, base_out = above, n_in = nT;
-      bool ranked = false;
-#pragma unroll 1
-      for (int level = 0; level < 3 && !ranked; ++level) {
-        const int sh = level == 0 ? 12 : level == 1 ? 4 : 0;
-        const uint32_t dm = level == 2 ? 15u : 255u;
-        if (threadIdx.x < 256) h2[threadIdx.x] = 0;
-        if (threadIdx.x == 0) { s_cnt[0] = 0; s_cnt[1] = 0; }
-        __syncthreads();
-        for (int j = threadIdx.x; j < (int)nT; j += blockDim.x) {
-          const uint32_t k = ckeys[j] & 0xFFFFFu;
-          if ((k & pmask) == pref) atomicAdd(&h2[(k >> sh) & dm], 1u);
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {
-          // lane l owns digits 8(31-l) .. 8(31-l)+7, highest first
-          const int lane = threadIdx.x;
-          uint32_t c[8], tot = 0;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) { c[i] = h2[8 * (31 - lane) + 7 - i]; tot += c[i]; }
-          uint32_t incl = tot;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-          }
-          uint32_t acc = incl - tot;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if (acc < rem && acc + c[i] >= rem) {
-              sm.bcast[0] = 8 * (31 - lane) + 7 - i;
-              sm.bcast[1] = acc;
-              sm.bcast[2] = c[i];
-            }
-            acc += c[i];
-          }
-        }
-        __syncthreads();
-        const uint32_t digit = sm.bcast[0], above2 = sm.bcast[1], n2 = sm.bcast[2];
-        const uint32_t npref = pref | (digit << sh), nmask = pmask | (dm << sh);
-        // write the candidates in a higher digit; keep the threshold digit's few for ranking
-        for (int j = threadIdx.x; j < (int)nT; j += blockDim.x) {
-          const uint32_t k = ckeys[j] & 0xFFFFFu;
-          if ((k & pmask) != pref) continue;
-          const uint32_t dj = (k >> sh) & dm;
-          if (dj > digit) {
-            const uint32_t slot = base_out + atomicAdd(&s_cnt[0], 1u);
-            oi[slot] = cids[j];
-            if (os) os[slot] = order_key_float(ckeys[j]);
-          } else if (dj == digit && n2 <= (uint32_t)TOPK_RANK_MAX) {
-            const uint32_t slot = atomicAdd(&s_cnt[1], 1u);
-            k2[slot] = ckeys[j];
-            i2[slot] = cids[j];
-          }
-        }
-        __syncthreads();
-        base_out += above2;
-        rem -= above2;
-        pref = npref;
-        pmask = nmask;
-        n_in = n2;
-        if (n2 <= (uint32_t)TOPK_RANK_MAX) {
-          if (threadIdx.x < 32) warp_rank_select(k2, i2, (int)n2, rem, oi, os, base_out);
-          ranked = true;
-        }
-      }
-      if (!ranked) {
-        // more than TOPK_RANK_MAX candidates with one full key: exact selection among them
-        for (int j = threadIdx.x; j < (int)nT; j += blockDim.x)
-          if ((ckeys[j] & 0xFFFFFu) != pref) ckeys[j] = 0u;
-        __syncthreads();
-        auto idof = [&](int j) -> uint32_t { return (uint32_t)cids[j]; };
-        select_in_smem(sm, ckeys, (int)nT, rem, n_in, idof, oi, os, base_out);
-      }
-    }
+    resolve_boundary(sm, ckeys, cids, nT, need, above, oi, os, s_cnt);
   } else if (K > 0) {
     // inconsistent counts or a boundary bin larger than the candidate buffer: the whole row, in place
     __syncthreads();

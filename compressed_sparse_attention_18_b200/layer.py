@@ -100,7 +100,7 @@ class CSADecodeLayer:
                  W_IK=W_IK, c_out=self.c_new, kI_out=self.kI_new, kv_cache=self.kv, ki_cache=self.ki, row0=self.row0,
                  stream=st)
         mark(1)
-        index_scores(q_I, w, self.ki, self.n_c, self.q_pos, self.scores, ratio=s.r, g_q=s.g_q, hist=self.hist,
+        index_scores(q_I, w, self.ki, self.n_c, self.q_pos, self.scores, ratio=s.r, g_q=s.g_q, hist=self.hist, k=s.k,
                      stream=st)
         mark(2)
         topk(self.scores, self.ki, self.n_c, self.q_pos, B=s.B, Nq=1, ratio=s.r, k=s.k, idx_out=self.idx,

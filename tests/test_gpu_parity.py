@@ -272,6 +272,38 @@ def _attn_case(csa, *, B, Nq, H, d, d_r, n_max, n_c, q_pos, k=0, Wn=128, win_pos
     return out, lse
 
 
+def test_attn_tiles_per_cta_with_rescale(cuda_lib):
+    """Enough rows that each tensor-core CTA walks two 128-key tiles of its query; the second tile's
+    entries have 4x the norm of the first's, so every head's running max jumps past the lazy-rescale
+    slack and the accumulated O and l are rescaled before the second tile is added."""
+    csa = cuda_lib
+    B, H, d, d_r, n_max, k = 80, 64, 512, 64, 512, 256
+    G = gen(21)
+    kv = normal((B, n_max, d), 1.0, G)
+    kv[:, n_max // 2:] *= 4.0
+    q = normal((B, 1, H, d), 1.0, G)
+    cache = csa.PackedCache(B, n_max, d, d_r, DEV, 1.0)
+    csa.pack_fp4(kv.to(DEV), cache)
+    t = 4 * n_max - 1
+    q_pos = torch.full((B, 1), t, dtype=torch.int64)
+    n_c = torch.full((B,), n_max, dtype=torch.int32)
+    idx = torch.empty((B, 1, k), dtype=torch.int32)
+    for b in range(B):
+        lo = torch.randperm(n_max // 2, generator=G)[:k // 2]
+        hi = torch.randperm(n_max // 2, generator=G)[:k // 2] + n_max // 2
+        idx[b, 0] = torch.cat([lo, hi]).to(torch.int32)       # tile 0: small keys, tile 1: large keys
+    out, lse = csa.sparse_attn(q.to(DEV), q_pos.to(DEV), cache, n_c.to(DEV), idx.to(DEV), None, None, ratio=4)
+    torch.cuda.synchronize()
+    scale = d ** -0.5
+    for b in range(0, B, 7):
+        codes, scales, rope = O.pack_fp4(f64(kv[b]), d_r, 1.0)
+        rows = O.entry_kv(codes, scales, rope, d - d_r, 1.0)
+        o_ref, l_ref = O.attention(f64(q[b]), q_pos[b].numpy(), rows, idx[b].numpy(), n_max, np.zeros((0, d)), 0,
+                                   128, scale)
+        assert_close(f64(out[b]), o_ref, OUT_ATOL, OUT_RTOL, f"out b={b}")
+        assert_close(lse[b].cpu().numpy(), l_ref, LSE_ATOL, LSE_RTOL, f"lse b={b}")
+
+
 def test_attn_cfg1_shapes(cuda_lib):
     q_pos = list(range(4080, 4096))
     _attn_case(cuda_lib, B=1, Nq=16, H=8, d=128, d_r=32, n_max=1024, n_c=[1024], q_pos=q_pos, k=64, Wn=143,
