@@ -50,6 +50,9 @@ def parse():
     p.add_argument("--cpu-sample", type=int, default=2, help="sequences the CPU oracle times (cpu_baseline)")
     p.add_argument("--profile", action="store_true",
                    help="profiling case: one layer state, --steps eager steps, no timing (for ncu)")
+    p.add_argument("--rows", action="store_true",
+                   help="time the hot-path rows outside the decode step (HCA pooling and dense attention, "
+                        "cross-layer reuse, hierarchical index), one JSON line each")
     return p.parse_args()
 
 
@@ -431,10 +434,196 @@ def run_e2e(args, layers, inputs, stream, dev, world):
                     "kernels (CUDA graph per layer step)"}
 
 
+def _event_ms(fn, reps, warm=3):
+    """Mean device time of fn() (CUDA events on the current stream, synchronised on both sides)."""
+    for i in range(warm):
+        fn(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(reps):
+        fn(i)
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def _tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        return float(json.load(open(path))["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def run_rows(args):
+    """The rows of the hot path that the decode step does not exercise, each timed with CUDA events on
+    its own synthetic workload (caches rotated so they are read from HBM), against its roofline, with
+    the oracle timed on one sequence beside it."""
+    import compressed_sparse_attention_18_b200 as csa
+    from csa_workloads import CFG4_HCA, CFG4_REUSE, CFG5, decode_inputs, gen, normal
+    from oracle import csa_oracle as O
+    from threadpoolctl import threadpool_limits
+    dev = torch.device("cuda", 0)
+    hbm, hkind = peaks()
+    tfl, tkind = _tensor_peak()
+
+    def f64(x):
+        return x.double().cpu().numpy()
+
+    def emit(d):
+        print(json.dumps(d), flush=True)
+
+    # ---- a1 in HCA mode: 128x pooling of one 1,048,576-token sequence (C, Z read once: 2 GB)
+    s = CFG4_HCA
+    G = gen(3, dev)
+    C = normal((1, s.T, s.d), 1.0, G, dev)
+    Z = normal((1, s.T, s.d), 1.0, G, dev)
+    b_pos = normal((s.r, s.d), 0.1, G, dev, torch.float32)
+    c_out = torch.empty((1, s.T // s.r, s.d), dtype=torch.bfloat16, device=dev)
+    ms = _event_ms(lambda i: csa.compress(C=C, Z=Z, b_pos=b_pos, ratio=s.r, d_rope=s.d_r, rope_theta=10000.0,
+                                          c_out=c_out), 10)
+    nbytes = 2 * s.T * s.d * 2 + (s.T // s.r) * s.d * 2
+    cC, cZ, cb = f64(C[0, :64 * s.r]), f64(Z[0, :64 * s.r]), f64(b_pos)
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        for e in range(64):
+            O.compress_pool(cC[e * s.r:(e + 1) * s.r], cZ[e * s.r:(e + 1) * s.r], cb, s.r, s.d_r, 10000.0, e * s.r)
+        el = time.perf_counter() - t0
+    emit({"row": "a1 compress (HCA pooling, r=128)", "workload": "1 sequence x 1,048,576 tokens -> 8192 entries",
+          "ms": ms, "value": (s.T // s.r) / (ms / 1e3), "unit": "entries/s",
+          "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm, "peak_kind": hkind,
+                       "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / hbm, "algorithmic_bytes": nbytes},
+          "cpu_baseline": {"value": 64 / el, "unit": "entries/s", "cores": 1, "kind": "oracle",
+                           "sample": "64 entries of the same sequence"}})
+    del C, Z, c_out
+    torch.cuda.empty_cache()
+
+    # ---- a6 HCA dense attention: 16 sequences over all 8192 entries + 128-token window; 4 cache copies
+    R = 4
+    states = []
+    for li in range(R):
+        inp = decode_inputs(s, seed=10 + li, device=dev, needles=0)
+        cache = csa.PackedCache(s.B, s.n_c, s.d, s.d_r, dev)
+        csa.pack_fp4(inp["kv_src"], cache)
+        del inp["kv_src"], inp["kI_src"]
+        inp["cache"] = cache
+        inp["out"] = torch.empty((s.B, 1, s.H, s.d), dtype=torch.bfloat16, device=dev)
+        inp["lse"] = torch.empty((s.B, 1, s.H), dtype=torch.float32, device=dev)
+        states.append(inp)
+    torch.cuda.synchronize()
+    st0 = states[0]
+    ws = torch.empty(csa.attn_workspace_size(st0["q"], st0["q_pos"], st0["cache"], st0["n_c"], None, st0["win_kv"],
+                                             st0["win_pos0"], ratio=s.r, window=s.W, hca=True),
+                     dtype=torch.uint8, device=dev)
+
+    def hca(i):
+        st = states[i % R]
+        csa.hca_attn(st["q"], st["q_pos"], st["cache"], st["n_c"], st["win_kv"], st["win_pos0"], ratio=s.r,
+                     out=st["out"], lse=st["lse"], ws=ws)
+    ms = _event_ms(hca, 40)
+    flops = s.B * 4 * s.H * (s.n_c + s.W) * s.d
+    nbytes = s.B * (s.n_c * (s.d_n // 2 + 16 + s.d_r * 2) + s.W * s.d * 2 + 2 * s.H * s.d * 2)
+    rows = O.entry_kv(st0["cache"].codes[0].cpu().numpy(), st0["cache"].scales[0].cpu().numpy(),
+                      f64(st0["cache"].rope[0]), s.d_n, 1.0)
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        O.hca_attention(f64(st0["q"][0]), [s.T - 1], rows, s.n_c, s.r, f64(st0["win_kv"][0]), s.T - s.W, s.W,
+                        s.d ** -0.5)
+        el = time.perf_counter() - t0
+    emit({"row": "a6 HCA dense attention", "workload": "16 sequences x (8192 entries + 128 window), 64 heads x 512",
+          "ms": ms, "value": s.B / (ms / 1e3), "unit": "tokens/s",
+          "roofline": {"bound": "tensor", "achieved": flops / (ms / 1e3) / 1e12, "peak": tfl, "peak_kind": tkind,
+                       "unit": "TFLOP/s", "frac": flops / (ms / 1e3) / 1e12 / tfl, "algorithmic_flops": flops,
+                       "hbm_frac": nbytes / (ms / 1e3) / 1e9 / hbm, "algorithmic_bytes": nbytes},
+          "cpu_baseline": {"value": 1 / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                           "sample": "1 sequence of the same workload"}})
+    del states, ws, st0
+    torch.cuda.empty_cache()
+
+    # ---- a7 cross-layer reuse (layer 1 Full top-2048 over 262,144 entries, layer 2 Reindex -> top-512,
+    # Reuse: attention over layer 2's ids) and hierarchical index (level 1 with a pool of 1024 x 8 blocks,
+    # level 2 Reindex over the pool), 4 sequences each, 2 index-cache copies rotated
+    for name, s in (("a7 reuse (Full -> Reindex -> attention)", CFG4_REUSE), ("a7 hierarchical index", CFG5)):
+        B = 4
+        sts = []
+        for li in range(2):
+            inp = decode_inputs(s, seed=20 + li, device=dev, B=B, needles=0, qnorm_student_t=(s is CFG5))
+            ki = csa.PackedCache(B, s.n_c, s.d_I, 0, dev)
+            csa.pack_fp4(inp["kI_src"], ki)
+            inp["ki"] = ki
+            if s is CFG4_REUSE:
+                kv = csa.PackedCache(B, s.n_c, s.d, s.d_r, dev)
+                csa.pack_fp4(inp["kv_src"], kv)
+                inp["kv"] = kv
+            del inp["kv_src"], inp["kI_src"]
+            G2 = gen(77 + li, dev)
+            inp["qI2"] = normal(inp["q_I"].shape, 1.0, G2, dev)
+            inp["w2"] = normal(inp["w"].shape, 0.35, G2, dev, torch.float32)
+            sts.append(inp)
+        torch.cuda.synchronize()
+        k2 = s.extra.get("k2", s.k)
+
+        def step(i):
+            st = sts[i % 2]
+            if s is CFG5:
+                _, _, pool = csa.index_topk(st["q_I"], st["w"], st["ki"], st["n_c"], st["q_pos"], ratio=s.r, k=s.k,
+                                            pool_blocks=s.pool_blocks)
+                csa.index_topk(st["qI2"], st["w2"], st["ki"], st["n_c"], st["q_pos"], ratio=s.r, k=s.k, cand=pool)
+            else:
+                idx1, _, _ = csa.index_topk(st["q_I"], st["w"], st["ki"], st["n_c"], st["q_pos"], ratio=s.r, k=s.k)
+                idx2, _, _ = csa.index_topk(st["qI2"], st["w2"], st["ki"], st["n_c"], st["q_pos"], ratio=s.r, k=k2,
+                                            cand=idx1)
+                csa.sparse_attn(st["q"], st["q_pos"], st["kv"], st["n_c"], idx2, st["win_kv"], st["win_pos0"],
+                                ratio=s.r)
+        ms = _event_ms(step, 10)
+        per_key = s.d_I // 2 + s.d_I // 32 + 4
+        nbytes = B * (s.n_c * per_key + (s.pool_blocks * 8 if s is CFG5 else s.k) * per_key)
+        if s is CFG4_REUSE:
+            nbytes += B * (k2 * (s.d_n // 2 + 16 + s.d_r * 2) + s.W * s.d * 2 + 2 * s.H * s.d * 2)
+        st = sts[0]
+        codes, scales = st["ki"].codes[0].cpu().numpy(), st["ki"].scales[0].cpu().numpy()
+        t = int(st["q_pos"][0, 0])
+        with threadpool_limits(1):
+            t0 = time.perf_counter()
+            sc, ids = O.index_scores(f64(st["q_I"][0, 0])[None], f64(st["w"][0, 0])[None], 1.0, codes, scales, 1.0,
+                                     [t], s.n_c, s.r)
+            O.topk(sc, ids, s.k)
+            el = time.perf_counter() - t0
+        emit({"row": name, "workload": f"{B} sequences x {s.n_c} entries, top-{s.k}" +
+              (f", pool {s.pool_blocks}x8" if s is CFG5 else f", Reindex -> top-{k2}, attention"),
+              "ms": ms, "value": B / (ms / 1e3), "unit": "tokens/s",
+              "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm, "peak_kind": hkind,
+                           "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / hbm, "algorithmic_bytes": nbytes},
+              "cpu_baseline": {"value": 1 / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                               "sample": "level-1 index + top-k of 1 sequence (a lower bound on the oracle's time)"}})
+        del sts
+        torch.cuda.empty_cache()
+
+
+def run_profile(args):
+    """One layer state, `--steps` eager decode steps: the small case ncu captures run on."""
+    from compressed_sparse_attention_18_b200.layer import CSADecodeLayer, LayerShape
+    from csa_workloads import CFG2, decode_inputs
+    s = CFG2
+    ls = LayerShape(B=s.B, n_max=s.n_c, r=s.r, H=s.H, d=s.d, d_r=s.d_r, H_I=s.H_I, d_I=s.d_I, k=s.k, W=s.W)
+    L = CSADecodeLayer(ls, torch.device("cuda", 0))
+    inp = decode_inputs(s, seed=1, device="cuda")
+    L.load_history(inp["kv_src"], inp["kI_src"], s.n_c)
+    L.win.copy_(inp["win_kv"])
+    del inp["kv_src"], inp["kI_src"]
+    for _ in range(max(args.steps, 1)):
+        L.step(inp["C"], inp["Z"], inp["b_pos"], inp["W_IK"], inp["q"], inp["q_I"], inp["w"])
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": "ok", "steps": max(args.steps, 1), "workload": s.name}), flush=True)
+
+
 def main():
     args = parse()
     if args.profile:
         run_profile(args)
+        return
+    if args.rows:
+        run_rows(args)
         return
     rank, world = dist_init(args.gpus)
     try:
