@@ -276,19 +276,31 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
     for (int i = tid; i < ne * d; i += POOL_THREADS) {
       const int q = i / d, ch = i % d;
       const size_t tok0 = (size_t)b * T + (size_t)(e0 + q) * r;
+      // online softmax over the r slots, 8 slots per round with all their loads issued together
       float m = -INFINITY, l = 0.f, acc = 0.f;
-      for (int j = 0; j < r; ++j) {
-        const float a = bf16_bits_to_f(Z[(tok0 + j) * d + ch]) + b_pos[(size_t)j * d + ch];
-        const float c = bf16_bits_to_f(C[(tok0 + j) * d + ch]);
-        if (a > m) {
-          const float sc = __expf(m - a);
+      for (int j0 = 0; j0 < r; j0 += 8) {
+        float a[8], c[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u;
+          a[u] = j < r ? bf16_bits_to_f(Z[(tok0 + j) * d + ch]) + b_pos[(size_t)j * d + ch] : -INFINITY;
+          c[u] = j < r ? bf16_bits_to_f(C[(tok0 + j) * d + ch]) : 0.f;
+        }
+        float mr = a[0];
+#pragma unroll
+        for (int u = 1; u < 8; ++u) mr = fmaxf(mr, a[u]);
+        if (mr > m) {
+          const float sc = __expf(m - mr);
           l *= sc;
           acc *= sc;
-          m = a;
+          m = mr;
         }
-        const float p = __expf(a - m);
-        l += p;
-        acc = fmaf(p, c, acc);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float p = j0 + u < r ? __expf(a[u] - m) : 0.f;
+          l += p;
+          acc = fmaf(p, c[u], acc);
+        }
       }
       pooled[i] = acc / l;
     }
