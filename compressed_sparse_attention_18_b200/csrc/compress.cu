@@ -210,16 +210,21 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
   const int o_base = z * OW + oc * 8;
   pdl_trigger();
   pdl_wait();                                       // C, Z, the caches may come from the previous kernel
-  // W_IK slice into registers first (its latency overlaps the pooling)
+  // W_IK slice into registers: before short groups (its latency overlaps their pooling), after long
+  // ones (whose pooling needs the registers)
   uint4 wpre[PRE > 0 ? PRE : 1];
-  if (PRE > 0 && P.W_IK) {
+  auto load_w = [&]() {
+    if (PRE > 0 && P.W_IK) {
 #pragma unroll
-    for (int i = 0; i < PRE; ++i) {
-      const int ch = chp + NCHP * i;
-      wpre[i] = ch < d ? __ldg(reinterpret_cast<const uint4*>(P.W_IK + (size_t)ch * d_I + o_base))
-                       : make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < PRE; ++i) {
+        const int ch = chp + NCHP * i;
+        wpre[i] = ch < d ? __ldg(reinterpret_cast<const uint4*>(P.W_IK + (size_t)ch * d_I + o_base))
+                         : make_uint4(0, 0, 0, 0);
+      }
     }
-  }
+  };
+  const bool long_groups = R == 0 && r > 8;
+  if (!long_groups) load_w();
   // RoPE angle of this thread's (entry, pair): pos * inv_freq and its reduction mod 2 pi in double, then
   // sin / cos of the reduced angle (|a| <= pi) in single precision
   const int half = d_r >> 1;
@@ -272,39 +277,79 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
     }
     if (ne * d <= tid && rope_thread) rope_angle();
   } else if (R == 0) {
+    // long groups (r > 8): a thread owns 8 adjacent channels of one entry (16-byte loads of C and Z)
+    // and one phase of the slots (j = ph, ph + split, ...); 4 slots per round with all their loads
+    // issued together, an online softmax per channel, the phases merged by shuffles of adjacent lanes
     if (rope_thread) rope_angle();
-    for (int i = tid; i < ne * d; i += POOL_THREADS) {
-      const int q = i / d, ch = i % d;
+    const int d8 = d >> 3, items = ne * d8;
+    int split = 1;
+    while (split < 16 && 2 * split <= r && 2 * split * items <= POOL_THREADS) split <<= 1;
+    const int per = POOL_THREADS / split, ph = tid & (split - 1);
+    for (int base = 0; base < items; base += per) {   // uniform trip count: every lane reaches the shuffles
+      const int it = base + tid / split;
+      const bool act = it < items;
+      const int q = act ? it / d8 : 0, ch = act ? (it % d8) * 8 : 0;
       const size_t tok0 = (size_t)b * T + (size_t)(e0 + q) * r;
-      // online softmax over the r slots, 8 slots per round with all their loads issued together
-      float m = -INFINITY, l = 0.f, acc = 0.f;
-      for (int j0 = 0; j0 < r; j0 += 8) {
-        float a[8], c[8];
+      float m[8], l[8], acc[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int j = j0 + u;
-          a[u] = j < r ? bf16_bits_to_f(Z[(tok0 + j) * d + ch]) + b_pos[(size_t)j * d + ch] : -INFINITY;
-          c[u] = j < r ? bf16_bits_to_f(C[(tok0 + j) * d + ch]) : 0.f;
-        }
-        float mr = a[0];
+      for (int k = 0; k < 8; ++k) { m[k] = -INFINITY; l[k] = 0.f; acc[k] = 0.f; }
+      for (int j0 = act ? ph : r; j0 < r; j0 += 4 * split) {
+        uint4 zv[4], cv[4];
+        float4 b0[4], b1[4];
 #pragma unroll
-        for (int u = 1; u < 8; ++u) mr = fmaxf(mr, a[u]);
-        if (mr > m) {
-          const float sc = __expf(m - mr);
-          l *= sc;
-          acc *= sc;
-          m = mr;
+        for (int u = 0; u < 4; ++u) {
+          const int j = min(j0 + u * split, r - 1);   // out-of-range slots re-read slot r-1, weight 0 below
+          zv[u] = __ldg(reinterpret_cast<const uint4*>(Z + (tok0 + j) * d + ch));
+          cv[u] = __ldg(reinterpret_cast<const uint4*>(C + (tok0 + j) * d + ch));
+          b0[u] = __ldg(reinterpret_cast<const float4*>(b_pos + (size_t)j * d + ch));
+          b1[u] = __ldg(reinterpret_cast<const float4*>(b_pos + (size_t)j * d + ch + 4));
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float p = j0 + u < r ? __expf(a[u] - m) : 0.f;
-          l += p;
-          acc = fmaf(p, c[u], acc);
+        for (int k = 0; k < 8; ++k) {
+          float a[4], c[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t zw = k < 2 ? zv[u].x : k < 4 ? zv[u].y : k < 6 ? zv[u].z : zv[u].w;
+            const uint32_t cw = k < 2 ? cv[u].x : k < 4 ? cv[u].y : k < 6 ? cv[u].z : cv[u].w;
+            const float4& bb = k < 4 ? b0[u] : b1[u];
+            const float bk = (k & 3) == 0 ? bb.x : (k & 3) == 1 ? bb.y : (k & 3) == 2 ? bb.z : bb.w;
+            const float zf = __uint_as_float((k & 1) ? (zw & 0xFFFF0000u) : (zw << 16));
+            a[u] = j0 + u * split < r ? zf + bk : -INFINITY;
+            c[u] = __uint_as_float((k & 1) ? (cw & 0xFFFF0000u) : (cw << 16));
+          }
+          const float mn = fmaxf(m[k], fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])));
+          const float sc = m[k] == mn ? 1.f : __expf(m[k] - mn);
+          float ls = l[k] * sc, as = acc[k] * sc;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float p = __expf(a[u] - mn);
+            ls += p;
+            as = fmaf(p, c[u], as);
+          }
+          m[k] = mn; l[k] = ls; acc[k] = as;
         }
       }
-      pooled[i] = acc / l;
+      for (int off = 1; off < split; off <<= 1)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float mo = __shfl_xor_sync(0xffffffffu, m[k], off);
+          const float lo = __shfl_xor_sync(0xffffffffu, l[k], off);
+          const float ao = __shfl_xor_sync(0xffffffffu, acc[k], off);
+          const float mn = fmaxf(m[k], mo);
+          const float s1 = m[k] == mn ? 1.f : __expf(m[k] - mn);
+          const float s2 = mo == mn ? 1.f : __expf(mo - mn);
+          l[k] = fmaf(l[k], s1, lo * s2);
+          acc[k] = fmaf(acc[k], s1, ao * s2);
+          m[k] = mn;
+        }
+      if (act && ph == 0) {
+        float* dst = pooled + q * d + ch;
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[0] / l[0], acc[1] / l[1], acc[2] / l[2], acc[3] / l[3]);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4] / l[4], acc[5] / l[5], acc[6] / l[6], acc[7] / l[7]);
+      }
     }
   }
+  if (long_groups) load_w();
   __syncthreads();
   if (rope_thread) {
     const int q = tid / half, mm = tid % half;
@@ -424,6 +469,8 @@ extern "C" csa_status csa_compress(const csa_compress_args* a, void* stream) {
   }
   if (a->ki_pack.codes) CSA_REQUIRE(a->W_IK && a->ki_pack.scales && a->ki_pack.global_scale > 0.0f);
   if (a->W_IK) CSA_SUPPORTED(((uintptr_t)a->W_IK & 15) == 0);
+  // groups longer than 8 slots are read 8 channels (16 bytes) at a time
+  if (a->ratio > 8) CSA_SUPPORTED((((uintptr_t)a->C | (uintptr_t)a->Z | (uintptr_t)a->b_pos) & 15) == 0);
   if (a->W_IK) CSA_SUPPORTED((a->d_index * 2) % 16 == 0);
   CSA_SUPPORTED(POOL_ENT * (a->d_rope / 2) <= POOL_THREADS && a->d_rope / 2 <= POOL_MAX_HALF);
   // k_I output slices: enough CTAs for about one wave when there are few entry groups

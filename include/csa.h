@@ -70,7 +70,8 @@ csa_status csa_device_status(void* stream);
  * Shapes: x[B][T][d_model], W_kv/W_g[d_model][d], C/Z[B][T][d], b_pos[ratio][d] fp32,
  *         W_IK[d][d_index], c_out[B][T/ratio][d], kI_out[B][T/ratio][d_index], pos0[B] int64 (NULL = 0).
  * Limits: d % 8 == 0, d_rope even and <= d, ratio >= 1; projection mode needs d % 128 == 0 and
- *         d_model % 32 == 0 (else CSA_ERR_UNSUPPORTED).  No workspace.
+ *         d_model % 32 == 0; ratio > 8 needs C, Z and b_pos 16-byte aligned (else CSA_ERR_UNSUPPORTED).
+ *         No workspace.
  * ------------------------------------------------------------------------------------------------ */
 /* An FP4 cache to append packed rows to (the layout csa_pack_fp4 writes): row i of sequence b goes to
  * cache row row0[b] + i.  codes == NULL means "no cache". */

@@ -71,7 +71,8 @@ def test_compress_projection_mode_cfg1(cuda_lib):
 
 
 @pytest.mark.parametrize("r,T,d,d_r,pos0", [(4, 4 * 97 + 3, 512, 64, 4 * 1000), (128, 128 * 9 + 17, 512, 64, 0),
-                                            (1, 33, 128, 32, 7)])
+                                            (1, 33, 128, 32, 7), (128, 128 + 5, 512, 64, 128 * 7),
+                                            (16, 16 * 3 + 2, 128, 32, 0), (16, 16 + 3, 128, 32, 16 * 5)])
 def test_compress_pooling_mode(cuda_lib, r, T, d, d_r, pos0):
     csa = cuda_lib
     G = gen(3)
