@@ -26,6 +26,7 @@ ENTRY_POINTS = ("csa_status_string", "csa_version", "csa_last_cuda_error", "csa_
                 "csa_index_topk_noalloc", "csa_device_status")
 
 _u32, _i32, _f32, _vp = ctypes.c_uint32, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p
+CSA_EARLY_START = 1   # see csa.h: part of a call's work may start before the step's earlier kernels end
 
 
 class Fp4Cache(ctypes.Structure):
@@ -51,7 +52,7 @@ class IndexArgs(ctypes.Structure):
                 ("ratio", _i32), ("k", _i32), ("n_max", _i32), ("g_q", _f32), ("g_k", _f32), ("q_I", _vp),
                 ("w", _vp), ("k_codes", _vp), ("k_scales", _vp), ("n_c", _vp), ("q_pos", _vp),
                 ("cand", _vp), ("n_cand", _i32), ("pool_blocks", _i32), ("pool_block_size", _i32),
-                ("pool_out", _vp), ("idx_out", _vp), ("scores_out", _vp), ("hist", _vp)]
+                ("pool_out", _vp), ("idx_out", _vp), ("scores_out", _vp), ("hist", _vp), ("flags", _u32)]
 
 
 class AttnArgs(ctypes.Structure):
@@ -59,7 +60,7 @@ class AttnArgs(ctypes.Structure):
                 ("ratio", _i32), ("n_max", _i32), ("k", _i32), ("Wn", _i32), ("window", _i32),
                 ("g_kv", _f32), ("softmax_scale", _f32), ("q", _vp), ("q_pos", _vp), ("kv_codes", _vp),
                 ("kv_scales", _vp), ("kv_rope", _vp), ("n_c", _vp), ("idx", _vp), ("win_kv", _vp),
-                ("win_pos0", _vp), ("out", _vp), ("lse", _vp)]
+                ("win_pos0", _vp), ("out", _vp), ("lse", _vp), ("flags", _u32)]
 
 
 _lib.csa_status_string.restype = ctypes.c_char_p
@@ -204,7 +205,7 @@ def _index_args(q_I, w, kcache: PackedCache, n_c, q_pos, ratio, k, g_q, cand, po
 
 def index_topk(q_I, w, kcache: PackedCache, n_c, q_pos, *, ratio, k, g_q=1.0, cand=None, pool_blocks=0,
                pool_block_size=8, want_scores=False, idx_out=None, scores_out=None, pool_out=None, ws=None,
-               stream=None):
+               early_start=False, stream=None):
     """Lightning indexer + top-k.  Returns (idx [B,Nq,k] int32, scores [B,Nq,k] or None, pool or None)."""
     B, Nq = q_I.shape[:2]
     dev = q_I.device
@@ -216,6 +217,7 @@ def index_topk(q_I, w, kcache: PackedCache, n_c, q_pos, *, ratio, k, g_q=1.0, ca
         pool_out = torch.empty((B, Nq, pool_blocks * pool_block_size), dtype=torch.int32, device=dev)
     a = _index_args(q_I, w, kcache, n_c, q_pos, ratio, k, g_q, cand, pool_blocks, pool_block_size, pool_out,
                     idx_out, scores_out)
+    a.flags = CSA_EARLY_START if early_start else 0
     nbytes = _lib.csa_index_topk_workspace_size(ctypes.byref(a))
     wbuf = _ws(nbytes, dev, ws)
     _check(_lib.csa_index_topk(ctypes.byref(a), _ptr(wbuf) if wbuf is not None else None, nbytes,
@@ -224,12 +226,14 @@ def index_topk(q_I, w, kcache: PackedCache, n_c, q_pos, *, ratio, k, g_q=1.0, ca
 
 
 def index_scores(q_I, w, kcache: PackedCache, n_c, q_pos, scores, *, ratio, g_q=1.0, cand=None, hist=None,
-                 k=None, stream=None):
+                 k=None, early_start=False, stream=None):
     """Lightning-indexer scores only, into scores [B*Nq, ld] fp32 (see csa_index_scores); hist
     ([B*Nq, 4096] uint32 as int32, optional, zero before first use) receives the score histogram for
-    topk(), which leaves it zero again; k (optional) is recorded in the call's arguments."""
+    topk(), which leaves it zero again; k (optional) is recorded in the call's arguments.
+    early_start: CSA_EARLY_START (only right after the compress call of the same decode step)."""
     a = _index_args(q_I, w, kcache, n_c, q_pos, ratio, k if k is not None else 1, g_q, cand, 0, 8, None, None, None)
     a.hist = _ptr(hist)
+    a.flags = CSA_EARLY_START if early_start else 0
     _check(_lib.csa_index_scores(ctypes.byref(a), _ptr(scores), scores.shape[-1], _stream(stream)),
            "csa_index_scores")
     return scores
@@ -281,13 +285,14 @@ def _attn_args(q, q_pos, cache: PackedCache, n_c, idx, win_kv, win_pos0, ratio, 
 
 
 def _attn(fn, hca, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse, ws,
-          stream):
+          stream, early_start=False):
     B, Nq, H, d = q.shape
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Nq, H), dtype=torch.float32, device=q.device)
     a = _attn_args(q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse)
+    a.flags = CSA_EARLY_START if early_start else 0
     nbytes = _lib.csa_attn_workspace_size(ctypes.byref(a), hca)
     wbuf = _ws(nbytes, q.device, ws)
     _check(fn(ctypes.byref(a), _ptr(wbuf) if wbuf is not None else None, nbytes, _stream(stream)),
@@ -296,10 +301,12 @@ def _attn(fn, hca, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, s
 
 
 def sparse_attn(q, q_pos, cache: PackedCache, n_c, idx, win_kv=None, win_pos0=None, *, ratio=4, window=128,
-                softmax_scale=0.0, out=None, lse=None, ws=None, stream=None):
-    """CSA attention over the selected entries idx [B,Nq,k] plus the window.  Returns (out, lse)."""
+                softmax_scale=0.0, out=None, lse=None, ws=None, early_start=False, stream=None):
+    """CSA attention over the selected entries idx [B,Nq,k] plus the window.  Returns (out, lse).
+    early_start: CSA_EARLY_START (window tiles start before the step's index and top-k kernels end;
+    only inside a decode step that began with compress)."""
     return _attn(_lib.csa_sparse_attn, 0, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window,
-                 softmax_scale, out, lse, ws, stream)
+                 softmax_scale, out, lse, ws, stream, early_start)
 
 
 def hca_attn(q, q_pos, cache: PackedCache, n_c, win_kv=None, win_pos0=None, *, ratio=128, window=128,
@@ -309,6 +316,7 @@ def hca_attn(q, q_pos, cache: PackedCache, n_c, win_kv=None, win_pos0=None, *, r
                  softmax_scale, out, lse, ws, stream)
 
 
-def attn_workspace_size(q, q_pos, cache, n_c, idx, win_kv, win_pos0, *, ratio, window, hca=False):
+def attn_workspace_size(q, q_pos, cache, n_c, idx, win_kv, win_pos0, *, ratio, window, hca=False, early_start=False):
     a = _attn_args(q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, 0.0, None, None)
+    a.flags = CSA_EARLY_START if early_start else 0
     return _lib.csa_attn_workspace_size(ctypes.byref(a), 1 if hca else 0)

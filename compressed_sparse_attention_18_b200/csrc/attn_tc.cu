@@ -54,6 +54,8 @@ struct TaSmem {
 struct TaParams {
   int Nq, H, ratio, n_max, k, Wn, window, splits, hca;
   int tpc;              // key tiles per CTA (a CTA walks tiles split*tpc .. split*tpc + tpc - 1 of its query)
+  int early_rows;       // > 0: CTAs [0, early_rows) each take one query's window tile (split splits - 1)
+                        // without waiting for the previous kernel; the others take the entry tiles
   float g, scale_log2;
   const int64_t* q_pos;
   const uint8_t* codes;
@@ -186,7 +188,12 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   TaSmem& S = *reinterpret_cast<TaSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bq = blockIdx.x / P.splits, split = blockIdx.x % P.splits;
+  // early window: CTA i < early_rows is query i's window tile, the rest split the entry tiles
+  const bool win_cta = (int)blockIdx.x < P.early_rows;
+  const int ent_splits = P.early_rows > 0 ? P.splits - 1 : P.splits;
+  const int jb = (int)blockIdx.x - P.early_rows;
+  const int bq = win_cta ? (int)blockIdx.x : jb / ent_splits;
+  const int split = win_cta ? P.splits - 1 : jb % ent_splits;
   const int b = bq / P.Nq;
   // worker thread t owns tile row t/2 for the gather (its half of the row's FP4 blocks and RoPE slice)
   const int grow = (tid & (TA_WORKERS - 1)) >> 1, ghalf = tid & 1;
@@ -213,7 +220,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   if (tid < 64) { S.m[tid] = -INFINITY; S.l[tid] = 0.f; }
   if (tid == 0) S.rescale = 0;
   pdl_trigger();
-  pdl_wait();
+  if (!win_cta) pdl_wait();                      // window tiles read only q, positions and the window
   const long long tq = P.q_pos[bq];
   const int ncb = min(P.n_c[b], P.n_max);
   int n_sel = P.k;
@@ -229,9 +236,11 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   }
   const int n_list = n_sel + (whi >= wlo ? (int)(whi - wlo + 1) : 0);
   const size_t unit_ho = ((size_t)bq * P.splits + split) * P.H;
-  const int first_key = split * P.tpc * TA_KEYS;
-  // non-empty tiles of this CTA (block-uniform)
-  const int ntile = max(0, min(P.tpc, (n_list - first_key + TA_KEYS - 1) / TA_KEYS));
+  // this CTA's keys: [first_key, key_lim), at most tpc tiles (block-uniform); with the early window the
+  // entry CTAs stop at n_sel and the window CTA starts there (n_sel is then a multiple of the tile)
+  const int first_key = win_cta ? n_sel : split * P.tpc * TA_KEYS;
+  const int key_lim = (P.early_rows > 0 && !win_cta) ? min(n_list, n_sel) : n_list;
+  const int ntile = max(0, min(win_cta ? 1 : P.tpc, (key_lim - first_key + TA_KEYS - 1) / TA_KEYS));
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = S.tmem_base;
@@ -245,6 +254,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       if (P.lse && tid < P.H) P.lse[(size_t)bq * P.H + tid] = -INFINITY;
     }
     if (warp == 8) tmem_dealloc(tb, TA_TMEM_COLS);
+    if (win_cta && tid == 0) pdl_wait();         // the grid completes only after its predecessor
     return;
   }
 
@@ -540,6 +550,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
     }
     tc_fence_before();
   }
+  if (win_cta && tid == 0) pdl_wait();           // the grid completes only after its predecessor
   __syncthreads();
   if (warp == 8) {
     if (S.err && lane == 0) atomicOr(&g_csa_device_error, 1u);
@@ -548,18 +559,29 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   }
 }
 
+// Early window (CSA_EARLY_START): each query's window tile gets a CTA of its own, placed first in the
+// grid, that starts before the step's index and top-k kernels have ended; possible when the window
+// fills one tile right after the k entries (k a multiple of the tile, at most one tile of window).
+bool attn_tc_early(const csa_attn_args* a, int hca) {
+  const long long n_win = (a->win_kv && a->Wn > 0) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
+  return !hca && (a->flags & CSA_EARLY_START) && n_win > 0 && n_win <= TA_KEYS && a->k > 0 && a->k % TA_KEYS == 0;
+}
+
 // Key tiles per query and the CTAs that share them: one tile per CTA while the grid fits one wave of
 // the 148 SMs, else enough tiles per CTA (walked in order, online softmax) to come back to one wave.
+// With the early window the entry tiles alone are planned this way and one window CTA per query is
+// added (it runs while the top-k still holds few SMs).
 void attn_tc_plan(const csa_attn_args* a, int hca, int* splits, int* tpc) {
+  const bool early = attn_tc_early(a, hca);
   const long long n_win = (a->win_kv && a->Wn > 0) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
-  const long long n = (hca ? a->n_max : a->k) + n_win;
+  const long long n = (hca ? a->n_max : a->k) + (early ? 0 : n_win);
   const long long tiles = n > 0 ? (n + TA_KEYS - 1) / TA_KEYS : 1;
   const long long rows = (long long)a->B * a->Nq;
   long long t = (rows * tiles + 147) / 148;
   if (t < 1) t = 1;
   if (t > tiles) t = tiles;
   *tpc = (int)t;
-  *splits = (int)((tiles + t - 1) / t);
+  *splits = (int)((tiles + t - 1) / t) + (early ? 1 : 0);
 }
 
 bool attn_tc_eligible(const csa_attn_args* a, int hca, int max_splits) {
@@ -601,6 +623,7 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
   TaParams P{};
   P.Nq = a->Nq; P.H = a->H; P.ratio = a->ratio; P.n_max = a->n_max; P.k = hca ? 0 : a->k;
   P.Wn = Wn; P.window = a->window; P.splits = splits; P.tpc = tpc; P.hca = hca; P.g = a->g_kv;
+  P.early_rows = attn_tc_early(a, hca) ? (int)rows : 0;
   const float scale = a->softmax_scale != 0.0f ? a->softmax_scale : 1.0f / sqrtf((float)a->d);
   P.scale_log2 = scale * TA_LOG2E;
   P.q_pos = a->q_pos; P.codes = a->kv_codes; P.scales = a->kv_scales;

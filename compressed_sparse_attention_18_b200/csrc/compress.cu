@@ -208,8 +208,11 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int oc = tid % NOC, chp = tid / NOC;
   const int o_base = z * OW + oc * 8;
+  // C, Z, the caches may come from the previous kernel.  Dependents are released only after the wait, so
+  // when the next kernel starts, everything before this one on the stream has completed (the contract
+  // that lets the indexer and the window tiles of attention start early in a decode step)
+  pdl_wait();
   pdl_trigger();
-  pdl_wait();                                       // C, Z, the caches may come from the previous kernel
   // W_IK slice into registers: before short groups (its latency overlaps their pooling), after long
   // ones (whose pooling needs the registers)
   uint4 wpre[PRE > 0 ? PRE : 1];

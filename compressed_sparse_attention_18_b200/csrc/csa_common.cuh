@@ -56,7 +56,9 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // still finishing: each does its setup that touches no global memory, then pdl_wait() (the previous
 // grid has completed and its writes are visible) before its first global read.  pdl_trigger() lets the
 // next kernel start launching once every CTA of this one has begun.  Launched any other way, both are
-// no-ops.
+// no-ops.  Under the early-start option some reads move ahead of the wait (the indexer's key tiles
+// below the newest row, attention's window tiles); every grid still waits once before it completes, so
+// a grid's completion implies its predecessor's.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

@@ -69,6 +69,7 @@ struct TcParams {
   uint32_t* hist;           // [B][4096] or null
   long long ld;
   int n_max, ratio, H_I, ctas_per_row;
+  int early;                // read q_I, w, n_c, q_pos and key rows below n_c[b] - 1 before the wait
   float g_q, gg;
 };
 
@@ -103,10 +104,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
   for (int i = threadIdx.x; i < TC_HIST_BINS; i += blockDim.x) S.hist[i] = 0;
   if (warp == 1) { tmem_alloc(&S.tmem_base, TC_TMEM_COLS); tmem_relinquish(); }
   pdl_trigger();
-  pdl_wait();
+  if (!P.early) pdl_wait();
   // key tiles of this CTA
   long long nv = (P.q_pos[b] + 1) / P.ratio;
   const int ncb = min(P.n_c[b], P.n_max);
+  // early start: the tiles below the one holding row n_c[b] - 1 (the entry the previous kernel may be
+  // appending) are loaded before the wait (rows past a sequence's end that a tile also covers are never
+  // scored)
+  const int wait_tile = P.early ? (ncb - 1 >= 0 ? (ncb - 1) / TC_TILE : -1) : -1;
   if (nv > ncb) nv = ncb;
   if (nv < 0) nv = 0;
   const int n_vis = (int)nv;
@@ -126,8 +131,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
     if (lane == 0) {
       const long long rows_total = (long long)gridDim.y * P.n_max;
       int issued = 0;
+      bool waited = !P.early;
       for (int i = 0; i < ntile && ok; ++i) {
         const int s = i % TC_STAGES, f = i / TC_STAGES;
+        if (!waited && t_begin + i >= wait_tile) { pdl_wait(); waited = true; }
         if (f > 0 && !mbar_wait(&S.empty[s], (f - 1) & 1)) { ok = false; break; }
         const long long row = (long long)b * P.n_max + (long long)(t_begin + i) * TC_TILE;
         long long nrow = rows_total - row;
@@ -278,6 +285,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
     if (!ok && lane == 0) atomicOr(&S.err, 1u);
   }
   __syncthreads();
+  if (P.early && threadIdx.x == 0) pdl_wait();   // this grid completes only after its predecessor
   if (S.err && threadIdx.x == 0) atomicOr(&g_csa_device_error, 1u);
   if (P.hist && S.err == 0) {
     uint32_t* h = P.hist + (size_t)b * TC_HIST_BINS;
@@ -345,6 +353,7 @@ csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, u
   if (per_row > tiles_row) per_row = tiles_row;
   if (per_row < 1) per_row = 1;
   P.ctas_per_row = per_row;
+  P.early = (a->flags & CSA_EARLY_START) ? 1 : 0;
   const int smem = (int)sizeof(TcSmem) + 1024;
   static std::atomic<unsigned> attr_done{0};
   set_smem_once((const void*)index_score_tc_kernel, smem, attr_done);

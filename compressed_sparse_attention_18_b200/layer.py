@@ -38,8 +38,12 @@ class LayerShape:
 
 
 class CSADecodeLayer:
-    def __init__(self, s: LayerShape, device="cuda"):
+    def __init__(self, s: LayerShape, device="cuda", early_start: bool = True):
+        """early_start: the step's indexer streams the key tiles below the new entry while the compressor
+        still runs, and attention runs each query's window tile while the top-k still runs
+        (CSA_EARLY_START; the step's inputs q, q_I, w and the window are never written by its kernels)."""
         self.s = s
+        self.early = early_start
         dev = torch.device(device)
         self.kv = PackedCache(s.B, s.n_max, s.d, s.d_r, dev, s.g_kv)
         self.ki = PackedCache(s.B, s.n_max, s.d_I, 0, dev, s.g_k)
@@ -61,7 +65,7 @@ class CSADecodeLayer:
         self.hist = torch.zeros((s.B, 4096), dtype=torch.int32, device=dev)   # score histogram (uint32 bits)
         ws_i = topk_workspace_size(self.ki, self.n_c, self.q_pos, B=s.B, Nq=1, ratio=s.r, k=s.k)
         ws_a = attn_workspace_size(q, self.q_pos, self.kv, self.n_c, self.idx, self.win, self.win_pos0, ratio=s.r,
-                                   window=s.W)
+                                   window=s.W, early_start=early_start)
         self.ws_index = torch.empty(max(ws_i, 1), dtype=torch.uint8, device=dev)
         self.ws_attn = torch.empty(max(ws_a, 1), dtype=torch.uint8, device=dev)
 
@@ -101,12 +105,12 @@ class CSADecodeLayer:
                  stream=st)
         mark(1)
         index_scores(q_I, w, self.ki, self.n_c, self.q_pos, self.scores, ratio=s.r, g_q=s.g_q, hist=self.hist, k=s.k,
-                     stream=st)
+                     early_start=self.early, stream=st)
         mark(2)
         topk(self.scores, self.ki, self.n_c, self.q_pos, B=s.B, Nq=1, ratio=s.r, k=s.k, idx_out=self.idx,
              hist=self.hist, ws=self.ws_index, stream=st)
         mark(3)
         sparse_attn(q, self.q_pos, self.kv, self.n_c, self.idx, self.win, self.win_pos0, ratio=s.r, window=s.W,
-                    out=self.out, lse=self.lse, ws=self.ws_attn, stream=st)
+                    out=self.out, lse=self.lse, ws=self.ws_attn, early_start=self.early, stream=st)
         mark(4)
         return self.out, self.lse, self.idx

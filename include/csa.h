@@ -54,6 +54,25 @@ int csa_last_cuda_error(void);
  * CSA_OK otherwise, CSA_ERR_CUDA if the synchronisation itself failed. */
 csa_status csa_device_status(void* stream);
 
+/* Overlap inside a decode step.  Every kernel of this library is launched with programmatic
+ * dependent launch: it may become resident while the kernel before it on the stream still runs, and it
+ * waits for that kernel to complete (and its writes to become visible) before it reads anything the
+ * kernel could have written.  csa_compress's last kernel lets its dependents start only after all
+ * work earlier on the stream has completed.
+ * CSA_EARLY_START in `flags` (csa_index_args, csa_attn_args) lets a call do part of its work before
+ * the kernels ahead of it in the step have completed:
+ *   - csa_index_scores / csa_index_topk (Full mode, single query per row): scoring reads q_I, w, n_c,
+ *     q_pos and the key rows [0, n_c[b] - 1) at once and writes scores and hist; only the 256-row
+ *     tile that holds row n_c[b] - 1 waits.  Requires: the kernel just before the call is csa_compress,
+ *     and that call writes none of these inputs except key rows >= n_c[b] - 1.
+ *   - csa_sparse_attn (k % 128 == 0, window <= 128): the window tile of every query runs in a CTA of
+ *     its own that reads q, q_pos, n_c, win_kv, win_pos0 and writes its workspace partial at once; the
+ *     CTAs over the selected entries wait as usual.  Requires: the step's earlier calls since
+ *     csa_compress (csa_index_scores, csa_topk) write none of those inputs, and csa_compress is
+ *     among them.
+ * Paths that cannot use the flag ignore it.  Results are the same with and without it. */
+#define CSA_EARLY_START 1u
+
 /* ------------------------------------------------------------------------------------------------
  * csa_compress — the compressor ([V4 blog] Fig. 3 / Fig. 4; [V4.1 notes] eq.(1) and CSA2 bullet).
  *
@@ -175,6 +194,7 @@ typedef struct csa_index_args {
                               histogram costs time, not correctness (csa_topk checks its counts against
                               the scores and falls back to the full selection).  NULL = plain radix
                               selection */
+  uint32_t flags;          /* CSA_EARLY_START or 0 */
 } csa_index_args;
 
 size_t csa_index_topk_workspace_size(const csa_index_args* args);
@@ -244,6 +264,7 @@ typedef struct csa_attn_args {
   const int64_t* win_pos0;
   void* out;
   float* lse;
+  uint32_t flags;          /* CSA_EARLY_START or 0 */
 } csa_attn_args;
 
 size_t csa_attn_workspace_size(const csa_attn_args* args, int hca);
