@@ -54,8 +54,8 @@ struct TaSmem {
 struct TaParams {
   int Nq, H, ratio, n_max, k, Wn, window, splits, hca;
   int tpc;              // key tiles per CTA (a CTA walks tiles split*tpc .. split*tpc + tpc - 1 of its query)
-  int early_rows;       // > 0: CTAs [0, early_rows) each take one query's window tile (split splits - 1)
-                        // without waiting for the previous kernel; the others take the entry tiles
+  int early_rows;       // > 0 (= rows): CTA i < early_rows is split 0 of query i; it walks the query's
+                        // window tile before waiting for the previous kernel, then its entry tiles
   float g, scale_log2;
   const int64_t* q_pos;
   const uint8_t* codes;
@@ -188,12 +188,13 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   TaSmem& S = *reinterpret_cast<TaSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // early window: CTA i < early_rows is query i's window tile, the rest split the entry tiles
-  const bool win_cta = (int)blockIdx.x < P.early_rows;
-  const int ent_splits = P.early_rows > 0 ? P.splits - 1 : P.splits;
+  // early window: the split-0 CTAs of all queries come first in the grid (they start during the previous
+  // kernel and walk the window tile while it runs), then the other splits
+  const bool early = P.early_rows > 0;
+  const bool first_cta = early && (int)blockIdx.x < P.early_rows;
   const int jb = (int)blockIdx.x - P.early_rows;
-  const int bq = win_cta ? (int)blockIdx.x : jb / ent_splits;
-  const int split = win_cta ? P.splits - 1 : jb % ent_splits;
+  const int bq = !early ? (int)blockIdx.x / P.splits : first_cta ? (int)blockIdx.x : jb / (P.splits - 1);
+  const int split = !early ? (int)blockIdx.x % P.splits : first_cta ? 0 : 1 + jb % (P.splits - 1);
   const int b = bq / P.Nq;
   // worker thread t owns tile row t/2 for the gather (its half of the row's FP4 blocks and RoPE slice)
   const int grow = (tid & (TA_WORKERS - 1)) >> 1, ghalf = tid & 1;
@@ -220,27 +221,59 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   if (tid < 64) { S.m[tid] = -INFINITY; S.l[tid] = 0.f; }
   if (tid == 0) S.rescale = 0;
   pdl_trigger();
-  if (!win_cta) pdl_wait();                      // window tiles read only q, positions and the window
-  const long long tq = P.q_pos[bq];
-  const int ncb = min(P.n_c[b], P.n_max);
+  // before the wait: prefetch the query's selected ids and one line per 2 MB of the sequence's cache
+  // arrays, so the reads right after it find their address translations (and the ids) warm
+  if (!P.hca) {
+    const int lines = (P.k * 4 + 127) / 128;
+    for (int i = tid; i < lines; i += TA_THREADS) prefetch_l2(P.idx + (size_t)bq * P.k + i * 32);
+  }
+  {
+    const size_t n_max = (size_t)P.n_max;
+    const size_t cb = n_max * 224, sb = n_max * 16, rb = n_max * 128, pg = (size_t)1 << 21;
+    const size_t nc = (cb + pg - 1) / pg, ns = (sb + pg - 1) / pg, nr = (rb + pg - 1) / pg;
+    const int j = tid - 64;
+    if (n_max > 0 && j >= 0 && (size_t)j < nc + ns + nr) {
+      const uint8_t* base = (size_t)j < nc ? P.codes + (size_t)b * cb + (size_t)j * pg
+                          : (size_t)j < nc + ns ? P.scales + (size_t)b * sb + ((size_t)j - nc) * pg
+                                                : reinterpret_cast<const uint8_t*>(P.rope) + (size_t)b * rb +
+                                                      ((size_t)j - nc - ns) * pg;
+      prefetch_l2(base);
+    }
+  }
+  // positions and lengths are inputs of the step: under the early start they are read before the wait
+  long long tq = 0, p0 = 0;
+  int ncb = 0;
+  auto load_pos = [&]() {
+    tq = P.q_pos[bq];
+    ncb = min(P.n_c[b], P.n_max);
+    if (P.Wn > 0) p0 = P.win_pos0[b];
+  };
+  if (early) load_pos();
+  if (!first_cta) pdl_wait();                    // (a window tile reads only q, positions and the window)
+  if (!early) load_pos();
   int n_sel = P.k;
   if (P.hca) {                                   // all visible entries: r*i + r - 1 <= t and i < n_c
     long long nv = (tq + 1) / P.ratio;
     n_sel = (int)max(0LL, min(nv, (long long)ncb));
   }
-  long long wlo = 0, whi = -1, p0 = 0;
+  long long wlo = 0, whi = -1;
   if (P.Wn > 0) {
-    p0 = P.win_pos0[b];
     wlo = max(max(0LL, tq - P.window + 1), p0);
     whi = min(tq, p0 + P.Wn - 1);
   }
   const int n_list = n_sel + (whi >= wlo ? (int)(whi - wlo + 1) : 0);
   const size_t unit_ho = ((size_t)bq * P.splits + split) * P.H;
-  // this CTA's keys: [first_key, key_lim), at most tpc tiles (block-uniform); with the early window the
-  // entry CTAs stop at n_sel and the window CTA starts there (n_sel is then a multiple of the tile)
-  const int first_key = win_cta ? n_sel : split * P.tpc * TA_KEYS;
-  const int key_lim = (P.early_rows > 0 && !win_cta) ? min(n_list, n_sel) : n_list;
-  const int ntile = max(0, min(win_cta ? 1 : P.tpc, (key_lim - first_key + TA_KEYS - 1) / TA_KEYS));
+  // this CTA's tiles (block-uniform): up to tpc consecutive tiles of the key list from split*tpc; with the
+  // early window the splits cover the entries only and split 0 takes the window tile first (n_sel is
+  // then a multiple of the tile)
+  const int base_key = split * P.tpc * TA_KEYS;
+  const bool has_win = first_cta && n_list > n_sel;
+  const int n_ent = max(0, min(P.tpc, ((early ? n_sel : n_list) - base_key + TA_KEYS - 1) / TA_KEYS));
+  const int ntile = n_ent + (has_win ? 1 : 0);
+  auto tile_key = [&](int t) -> int {
+    return has_win ? (t == 0 ? n_sel : base_key + (t - 1) * TA_KEYS) : base_key + t * TA_KEYS;
+  };
+  if (first_cta && !has_win) pdl_wait();          // no window rows: the entry tiles need the ids now
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = S.tmem_base;
@@ -254,7 +287,6 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       if (P.lse && tid < P.H) P.lse[(size_t)bq * P.H + tid] = -INFINITY;
     }
     if (warp == 8) tmem_dealloc(tb, TA_TMEM_COLS);
-    if (win_cta && tid == 0) pdl_wait();         // the grid completes only after its predecessor
     return;
   }
 
@@ -271,7 +303,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       const uint32_t ido = idesc_bf16(128, 64, 1, 1);
 #pragma unroll 1
       for (int t = 0; t < ntile; ++t) {
-        const TaTile g = ta_tile(first_key + t * TA_KEYS, n_sel, n_list, wlo, p0);
+        const TaTile g = ta_tile(tile_key(t), n_sel, n_list, wlo, p0);
         const int nbox = (g.we - g.wa) / TA_WBOX;
         // window boxes overwrite the K tile: only once the previous tile's O MMAs have completed (S MMAs
         // of an entry tile are queued behind them directly)
@@ -353,9 +385,9 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
         for (int c = 0; c < 4; ++c) rp[c] = __ldg(rrow + c);
       }
     };
-    TaTile g = ta_tile(first_key, n_sel, n_list, wlo, p0);
-    int id = check_id(raw_id(g));
-    int id_next = ntile > 1 ? raw_id(ta_tile(first_key + TA_KEYS, n_sel, n_list, wlo, p0)) : -1;
+    TaTile g = ta_tile(tile_key(0), n_sel, n_list, wlo, p0);
+    int id = check_id(raw_id(g));                  // a window tile reads no id
+    int id_next = ntile > 1 && !has_win ? raw_id(ta_tile(tile_key(1), n_sel, n_list, wlo, p0)) : -1;
     load_row(id);
 #pragma unroll 1
     for (int t = 0; t < ntile; ++t) {
@@ -421,10 +453,15 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       // next tile's row (its id arrived during this tile's gather), in flight during this tile's softmax
       // and MMAs; the id of the tile after it is requested now
       if (t + 1 < ntile) {
-        g = ta_tile(first_key + (t + 1) * TA_KEYS, n_sel, n_list, wlo, p0);
+        if (has_win && t == 0) {
+          // the window tile is gathered: from here on the ids and entries of the previous kernels
+          pdl_wait();
+          id_next = raw_id(ta_tile(tile_key(1), n_sel, n_list, wlo, p0));
+        }
+        g = ta_tile(tile_key(t + 1), n_sel, n_list, wlo, p0);
         id = check_id(id_next);
         load_row(id);
-        id_next = t + 2 < ntile ? raw_id(ta_tile(first_key + (t + 2) * TA_KEYS, n_sel, n_list, wlo, p0)) : -1;
+        id_next = t + 2 < ntile ? raw_id(ta_tile(tile_key(t + 2), n_sel, n_list, wlo, p0)) : -1;
       }
       asm volatile("bar.sync 1, 256;" ::: "memory");   // workers only: ids visible to the softmax
 
@@ -550,7 +587,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
     }
     tc_fence_before();
   }
-  if (win_cta && tid == 0) pdl_wait();           // the grid completes only after its predecessor
+  if (first_cta && tid == 0) pdl_wait();         // the grid completes only after its predecessor
   __syncthreads();
   if (warp == 8) {
     if (S.err && lane == 0) atomicOr(&g_csa_device_error, 1u);
@@ -559,9 +596,9 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   }
 }
 
-// Early window (CSA_EARLY_START): each query's window tile gets a CTA of its own, placed first in the
-// grid, that starts before the step's index and top-k kernels have ended; possible when the window
-// fills one tile right after the k entries (k a multiple of the tile, at most one tile of window).
+// Early window (CSA_EARLY_START): split 0 of each query, placed first in the grid, attends over the
+// window tile before the step's index and top-k kernels have ended; possible when the window fills one
+// tile right after the k entries (k a multiple of the tile, at most one tile of window).
 bool attn_tc_early(const csa_attn_args* a, int hca) {
   const long long n_win = (a->win_kv && a->Wn > 0) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
   return !hca && (a->flags & CSA_EARLY_START) && n_win > 0 && n_win <= TA_KEYS && a->k > 0 && a->k % TA_KEYS == 0;
@@ -569,8 +606,8 @@ bool attn_tc_early(const csa_attn_args* a, int hca) {
 
 // Key tiles per query and the CTAs that share them: one tile per CTA while the grid fits one wave of
 // the 148 SMs, else enough tiles per CTA (walked in order, online softmax) to come back to one wave.
-// With the early window the entry tiles alone are planned this way and one window CTA per query is
-// added (it runs while the top-k still holds few SMs).
+// With the early window the entry tiles alone are planned this way; split 0 also takes the window tile
+// (first, while the previous kernel still runs).
 void attn_tc_plan(const csa_attn_args* a, int hca, int* splits, int* tpc) {
   const bool early = attn_tc_early(a, hca);
   const long long n_win = (a->win_kv && a->Wn > 0) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
@@ -581,7 +618,7 @@ void attn_tc_plan(const csa_attn_args* a, int hca, int* splits, int* tpc) {
   if (t < 1) t = 1;
   if (t > tiles) t = tiles;
   *tpc = (int)t;
-  *splits = (int)((tiles + t - 1) / t) + (early ? 1 : 0);
+  *splits = (int)((tiles + t - 1) / t);
 }
 
 bool attn_tc_eligible(const csa_attn_args* a, int hca, int max_splits) {

@@ -61,6 +61,9 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // a grid's completion implies its predecessor's.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// L2 prefetch of one line: issued before pdl_wait() it fills the address translation (and L2) for reads
+// right after the wait; L2 is coherent, so a line the previous kernel rewrites later is read fresh.
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 inline cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t st, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};

@@ -391,6 +391,7 @@ struct TopkRowArgs {
   long long out_ld;
 };
 
+
 // Select the K largest of keys[0..len) (0 = not a candidate; nvalid candidates in all) by (key desc,
 // id asc), writing ids / scores to oi[base + slot], os[base + slot] in unspecified order.  Candidates
 // with equal key and equal id (a repeated id) are interchangeable: any of them gives the same output.
@@ -669,6 +670,12 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
   static_assert(sizeof(TopkSmem::whist) >= HIST_BINS * 4, "second-level histogram in the per-warp histograms");
   const int row = blockIdx.y;
   pdl_trigger();
+  if (threadIdx.x < 4 && A.n_cols > 0) {       // warm translations: the row's ends, its histogram, its output
+    const float* r0 = A.in_scores + row * A.in_ld;
+    const void* pf[4] = {r0, r0 + (A.n_cols - 1), hist ? (const void*)(hist + (size_t)row * HIST_BINS) : r0,
+                         A.out_idx ? (const void*)(A.out_idx + row * A.out_ld) : r0};
+    prefetch_l2(pf[threadIdx.x]);
+  }
   pdl_wait();                                  // scores and histogram come from the previous kernel
   int len = min(A.rows_per_seg, A.n_cols);
   if (A.q_pos) {

@@ -29,17 +29,21 @@ namespace csa {
 
 using namespace sm100;
 
-constexpr int TC_STAGES = 5;
+constexpr int TC_STAGES = 3;
+constexpr int TC_CTAS_PER_SM = 3;              // resident CTAs per SM (tensor memory, shared memory)
 constexpr int TC_SUB = 128;                      // keys per MMA (M)
 constexpr int TC_TILE = 2 * TC_SUB;              // keys per TMA box / pipeline step
 constexpr int TC_CODE_BYTES = TC_TILE * 64;      // 256 keys x 128 FP4
 constexpr int TC_SC_BYTES = TC_TILE * 4;         // 256 keys x 4 E4M3 scales
 constexpr int TC_THREADS = 192;
-constexpr int TC_NBUF = 4, TC_LAG = 2;
-constexpr uint32_t TC_TMEM_COLS = 256;
+constexpr int TC_NBUF = 3, TC_LAG = 2;
+constexpr uint32_t TC_TMEM_COLS = 128;
 constexpr uint32_t TC_COL_D = 0;                 // NBUF x (2 sub-tiles x 8 heads)
 constexpr uint32_t TC_COL_SFA = 64;              // NBUF x (2 sub-tiles x 2 atoms x 4 columns)
-constexpr uint32_t TC_COL_SFB = 128;             // 2 atoms x 4 columns
+constexpr uint32_t TC_COL_SFB = 112;             // 2 atoms x 4 columns
+static_assert(TC_COL_D + 16 * TC_NBUF <= TC_COL_SFA && TC_COL_SFA + 16 * TC_NBUF <= TC_COL_SFB &&
+              TC_COL_SFB + 8 <= TC_TMEM_COLS && TC_CTAS_PER_SM * TC_TMEM_COLS <= 512 && TC_LAG < TC_NBUF,
+              "tensor-memory plan");
 constexpr int TC_HIST_BINS = 4096, TC_HIST_SHIFT = 20;
 
 struct TcSmem {
@@ -347,9 +351,9 @@ csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, u
   P.H_I = a->H_I;
   P.g_q = a->g_q;
   P.gg = a->g_q * a->g_k;
-  // at most two resident CTAs per SM (256 tensor-memory columns each): one wave, at most one per tile
+  // TC_CTAS_PER_SM resident CTAs per SM: one wave, at most one per tile
   const int tiles_row = (a->n_max + TC_TILE - 1) / TC_TILE;
-  int per_row = (2 * 148) / a->B;
+  int per_row = (TC_CTAS_PER_SM * 148) / a->B;
   if (per_row > tiles_row) per_row = tiles_row;
   if (per_row < 1) per_row = 1;
   P.ctas_per_row = per_row;

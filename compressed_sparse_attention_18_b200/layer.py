@@ -64,8 +64,9 @@ class CSADecodeLayer:
         self.scores = torch.empty((s.B, s.n_max), dtype=torch.float32, device=dev)
         self.hist = torch.zeros((s.B, 4096), dtype=torch.int32, device=dev)   # score histogram (uint32 bits)
         ws_i = topk_workspace_size(self.ki, self.n_c, self.q_pos, B=s.B, Nq=1, ratio=s.r, k=s.k)
-        ws_a = attn_workspace_size(q, self.q_pos, self.kv, self.n_c, self.idx, self.win, self.win_pos0, ratio=s.r,
-                                   window=s.W, early_start=early_start)
+        # sized for both launch plans (the flag may be switched off later, e.g. for stage-by-stage timing)
+        ws_a = max(attn_workspace_size(q, self.q_pos, self.kv, self.n_c, self.idx, self.win, self.win_pos0,
+                                       ratio=s.r, window=s.W, early_start=e) for e in (True, False))
         self.ws_index = torch.empty(max(ws_i, 1), dtype=torch.uint8, device=dev)
         self.ws_attn = torch.empty(max(ws_a, 1), dtype=torch.uint8, device=dev)
 

@@ -47,15 +47,17 @@ def test_early_start_same_bits_and_fresh_newest_entry(cuda_lib, n_c, B):
     assert torch.equal(La.scores[:, :n_c], Lb.scores[:, :n_c])
     assert torch.equal(torch.sort(ia, dim=-1).values, torch.sort(ib, dim=-1).values)
     assert_close(f64(oa), f64(ob), OUT_ATOL, OUT_RTOL, "out early vs not")
-    # on one selection, both attention plans split the keys the same way at these batch sizes (one
-    # tile per CTA, the window last): bit-identical
+    # on one selection: the early plan (split 0 walks the window tile, then its entry tile) is
+    # deterministic and agrees with the stage-by-stage plan (window in a split of its own) to rounding
     csa = cuda_lib
     o1, l1 = csa.sparse_attn(inp["q"], La.q_pos, La.kv, La.n_c, ia, La.win, La.win_pos0, ratio=s.r, window=s.W,
                              early_start=True)
     o2, l2 = csa.sparse_attn(inp["q"], La.q_pos, La.kv, La.n_c, ia, La.win, La.win_pos0, ratio=s.r, window=s.W,
                              early_start=False)
     torch.cuda.synchronize()
-    assert torch.equal(o1, o2) and torch.equal(l1, l2) and torch.equal(o1, oa) and torch.equal(l1, la)
+    assert torch.equal(o1, oa) and torch.equal(l1, la)
+    assert_close(f64(o1), f64(o2), OUT_ATOL, OUT_RTOL, "out early vs stage-by-stage plan")
+    assert_close(l1.cpu().numpy(), l2.cpu().numpy(), LSE_ATOL, LSE_RTOL, "lse early vs stage-by-stage plan")
     assert torch.equal(La.kv.codes, Lb.kv.codes) and torch.equal(La.ki.codes, Lb.ki.codes)
     assert int(La.hist.abs().sum()) == 0          # the top-k left the histogram clean
     t = int(La.q_pos[0, 0])
