@@ -376,6 +376,12 @@ __device__ uint32_t block_exclusive_scan(TopkSmem& sm, uint32_t v, uint32_t* tot
 // One CTA per row.  Row r: scores at in_scores + r*in_ld, length len (from lens[r] or the visibility
 // rule), ids from in_ids (explicit) or id = id_base + position.  Writes k slots of out_idx /
 // out_scores at row r (stride k_out).
+// Per-row state of the long-row histogram selection: scores emitted above the boundary bin, boundary-bin
+// scores parked, CTAs finished, and whether the row was resolved (else the tournament selects it).
+struct LongRowState {
+  uint32_t up, at, done, ok;
+};
+
 struct TopkRowArgs {
   const float* in_scores;
   const int32_t* in_ids;
@@ -389,6 +395,7 @@ struct TopkRowArgs {
   int32_t* out_idx;
   float* out_scores;
   long long out_ld;
+  const LongRowState* skip;   // rows whose state says resolved are left alone (null: none)
 };
 
 
@@ -476,6 +483,7 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(TopkRowArgs A) {
   __shared__ TopkSmem sm;
   const int seg = blockIdx.x;                  // segment (chunk) of the row
   const int row = blockIdx.y;
+  if (A.skip && A.skip[row].ok) return;        // selected by the long-row histogram pass
   const int col0 = A.col_base + seg * A.rows_per_seg;
   int len = min(A.rows_per_seg, A.n_cols - col0);
   if (A.q_pos) {
@@ -818,6 +826,106 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
   }
 }
 
+// Long rows (several TOPK_CHUNK segments) with the row histogram of the scorer: CTA (seg, row) reads its
+// segment once, emits every score above the boundary bin at a slot from the row's counter and parks the
+// boundary-bin scores in the row's buffer (warp-aggregated atomics); the row's last CTA checks the counts
+// against the histogram, resolves the boundary bin and marks the row resolved.  Counts that disagree (a
+// stale histogram) or a boundary bin larger than the buffer leave the row to the tournament kernels that
+// follow, which skip resolved rows.  The last CTA clears the histogram row.
+__global__ void __launch_bounds__(TOPK_THREADS) topk_long_kernel(TopkRowArgs A, uint32_t* __restrict__ hist,
+                                                                 LongRowState* __restrict__ state,
+                                                                 uint32_t* __restrict__ cand) {
+  extern __shared__ __align__(16) uint32_t s_lc[];   // boundary-bin keys [TOPK_HIST_CAND] | ids [TOPK_HIST_CAND]
+  __shared__ __align__(16) TopkSmem sm;
+  __shared__ uint32_t s_cnt[2];
+  __shared__ uint32_t s_last;
+  const int seg = blockIdx.x, row = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  pdl_trigger();
+  pdl_wait();                                  // scores and histogram come from the previous kernel
+  int len = A.n_cols;
+  if (A.q_pos) {
+    const int b = row / A.Nq;
+    long long nv = (A.q_pos[row] + 1) / A.ratio;
+    if (nv > A.n_c[b]) nv = A.n_c[b];
+    len = (int)max(0LL, min((long long)len, nv));
+  }
+  uint32_t* hrow = hist + (size_t)row * HIST_BINS;
+  uint32_t nvalid;
+  hist_find_bin(sm, hrow, (uint32_t)A.k, &nvalid);
+  const uint32_t K = min((uint32_t)A.k, nvalid);
+  const uint32_t T = sm.bcast[0], above = sm.bcast[1], nT = sm.bcast[2];
+  LongRowState& rs = state[row];
+  uint32_t* ck = cand + (size_t)row * 2 * TOPK_HIST_CAND;
+  int32_t* ci = reinterpret_cast<int32_t*>(ck + TOPK_HIST_CAND);
+  int32_t* oi = A.out_idx + row * A.out_ld;
+  float* os = A.out_scores ? A.out_scores + row * A.out_ld : nullptr;
+  const float* src = A.in_scores + row * A.in_ld;
+  const int c0 = seg * TOPK_CHUNK, c1 = min(len, c0 + TOPK_CHUNK);
+  if (K > 0) {
+    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll 4
+    for (int base = c0; base < c1; base += blockDim.x) {   // block-uniform trip count
+      const int j = base + threadIdx.x;
+      const float v = j < c1 ? src[j] : -INFINITY;
+      const uint32_t bin = float_order_key(v) >> HIST_SHIFT;
+      const bool valid = v > -INFINITY;
+      const bool up = valid && bin > T, at = valid && bin == T;
+      const uint32_t mu = __ballot_sync(0xffffffffu, up), ma = __ballot_sync(0xffffffffu, at);
+      if (mu) {
+        uint32_t b0 = 0;
+        if (lane == 0) b0 = atomicAdd(&rs.up, (uint32_t)__popc(mu));
+        b0 = __shfl_sync(0xffffffffu, b0, 0);
+        const uint32_t slot = b0 + (uint32_t)__popc(mu & lt);
+        if (up && slot < above) {
+          oi[slot] = j;
+          if (os) os[slot] = v + 0.0f;
+        }
+      }
+      if (ma) {
+        uint32_t b0 = 0;
+        if (lane == 0) b0 = atomicAdd(&rs.at, (uint32_t)__popc(ma));
+        b0 = __shfl_sync(0xffffffffu, b0, 0);
+        const uint32_t c = b0 + (uint32_t)__popc(ma & lt);
+        if (at && c < (uint32_t)TOPK_HIST_CAND) {
+          ck[c] = float_order_key(v);
+          ci[c] = j;
+        }
+      }
+    }
+  }
+  // the last CTA of the row resolves it
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(&rs.done, 1u) == gridDim.x - 1 ? 1u : 0u;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const uint32_t n_up = *reinterpret_cast<volatile uint32_t*>(&rs.up);
+  const uint32_t n_at = *reinterpret_cast<volatile uint32_t*>(&rs.at);
+  const bool good = K == 0 || (n_up == above && n_at == nT && nT <= (uint32_t)TOPK_HIST_CAND);
+  if (good && K > 0) {
+    uint32_t* ckeys = s_lc;
+    int32_t* cids = reinterpret_cast<int32_t*>(s_lc + TOPK_HIST_CAND);
+    for (int c = threadIdx.x; c < (int)nT; c += blockDim.x) {
+      ckeys[c] = *reinterpret_cast<volatile uint32_t*>(ck + c);
+      cids[c] = *reinterpret_cast<volatile int32_t*>(ci + c);
+    }
+    __syncthreads();
+    resolve_boundary(sm, ckeys, cids, nT, K - above, above, oi, os, s_cnt);
+  }
+  if (good)
+    for (int s2 = (int)K + threadIdx.x; s2 < A.k; s2 += blockDim.x) {
+      oi[s2] = -1;
+      if (os) os[s2] = -INFINITY;
+    }
+  // every CTA of the row has read the histogram (it counted itself done afterwards): clear it
+  reinterpret_cast<uint4*>(hrow)[threadIdx.x] = make_uint4(0, 0, 0, 0);
+  if (threadIdx.x == 0) rs.ok = good ? 1u : 0u;
+}
+
 // ------------------------------------------------------------------------- hierarchical pool
 __global__ void block_max_kernel(const float* __restrict__ scores, long long ld, int n_cols,
                                  const int64_t* __restrict__ q_pos, const int32_t* __restrict__ n_c, int ratio,
@@ -861,8 +969,8 @@ csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, u
 // ------------------------------------------------------------------------------ orchestration
 struct IndexPlan {
   int rows, n_cols, segs, seg_len;
-  bool hist;   // single-query rows that fit one top-k pass: histogram-guided selection
-  size_t off_scores, off_tidx, off_tsc, off_bs, off_bidx, off_hist, sel_total, total;
+  bool hist;   // single-query rows: histogram-guided selection (long rows: segment CTAs + tournament fallback)
+  size_t off_scores, off_tidx, off_tsc, off_bs, off_bidx, off_lstate, off_lcand, off_hist, sel_total, total;
 };
 
 static bool one_query_per_cta(const csa_index_args* a) { return a->cand != nullptr || a->Nq == 1; }
@@ -882,6 +990,10 @@ static IndexPlan plan_index(const csa_index_args* a) {
     p.off_tidx = o; o = align_up(o + (size_t)p.rows * p.segs * a->k * 4, 256);
     p.off_tsc = o;  o = align_up(o + (size_t)p.rows * p.segs * a->k * 4, 256);
   }
+  if (p.segs > 1 && one_query_per_cta(a)) {
+    p.off_lstate = o; o = align_up(o + (size_t)p.rows * sizeof(LongRowState), 256);
+    p.off_lcand = o;  o = align_up(o + (size_t)p.rows * 2 * TOPK_HIST_CAND * 4, 256);
+  }
   if (a->pool_blocks > 0) {
     const int G = a->pool_block_size;
     const int nblk = (p.n_cols + G - 1) / G;
@@ -891,7 +1003,7 @@ static IndexPlan plan_index(const csa_index_args* a) {
   p.sel_total = o;
   p.off_scores = o;
   o = align_up(o + (size_t)p.rows * p.n_cols * 4, 256);
-  p.hist = one_query_per_cta(a) && p.segs == 1;
+  p.hist = one_query_per_cta(a);
   p.off_hist = o;
   if (p.hist) o = align_up(o + (size_t)p.rows * HIST_BINS * 4, 256);
   p.total = o;
@@ -1005,6 +1117,28 @@ static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const 
     csa_status s = launch_topk(ta, p.rows, 1, a->cand != nullptr, st);
     if (s != CSA_OK) return s;
   } else {
+    const LongRowState* skip = nullptr;
+    if (hist != nullptr && p.hist) {
+      // histogram pass over the segments; rows it cannot resolve go through the tournament below
+      LongRowState* lst = (LongRowState*)(w8 + p.off_lstate);
+      const cudaError_t e = cudaMemsetAsync(lst, 0, (size_t)p.rows * sizeof(LongRowState), st);
+      if (e != cudaSuccess) {
+        set_last_cuda_error(e);
+        return CSA_ERR_CUDA;
+      }
+      TopkRowArgs tl = ta;
+      tl.out_idx = a->idx_out;
+      tl.out_scores = a->scores_out;
+      tl.out_ld = a->k;
+      static std::atomic<unsigned> attr_l{0};
+      const int smem_l = 2 * TOPK_HIST_CAND * 4;
+      set_smem_once((const void*)topk_long_kernel, smem_l, attr_l);
+      csa_status s = launch_pdl(topk_long_kernel, dim3(p.segs, p.rows), dim3(TOPK_THREADS), (size_t)smem_l, st, tl,
+                                const_cast<uint32_t*>(hist), lst, (uint32_t*)(w8 + p.off_lcand));
+      if (s != CSA_OK) return s;
+      skip = lst;
+    }
+    ta.skip = skip;
     int32_t* tidx = (int32_t*)(w8 + p.off_tidx);
     float* tsc = (float*)(w8 + p.off_tsc);
     ta.out_idx = tidx;
@@ -1022,6 +1156,7 @@ static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const 
     tb.out_idx = a->idx_out;
     tb.out_scores = a->scores_out;
     tb.out_ld = a->k;
+    tb.skip = skip;
     CSA_SUPPORTED(tb.n_cols <= TOPK_CHUNK_IDS);
     s = launch_topk(tb, p.rows, 1, true, st);
     if (s != CSA_OK) return s;

@@ -188,6 +188,49 @@ def test_index_tournament_long_row(cuda_lib):
                 k=256, seed=3)
 
 
+def test_index_long_rows_histogram_pass(cuda_lib):
+    # rows of 3 and 4 top-k chunks: the histogram pass selects them (segment CTAs, the last one resolves
+    # the boundary bin); the second row's visible length ends inside its third chunk
+    n = 4 * 32768 - 100
+    _index_case(cuda_lib, B=2, n_max=n, n_c=[n, 70000], d_I=128, H_I=8, Nq=1, q_pos=[4 * n - 1, 4 * 69000 + 1],
+                k=2048, seed=10)
+
+
+def test_index_long_row_boundary_overflow_falls_back(cuda_lib):
+    # 70000 equal scores: the boundary bin holds more candidates than the row buffer, the tournament
+    # selects the row instead; the smallest ids must win
+    idx, swaps = _index_case(cuda_lib, B=1, n_max=70000, n_c=[70000], d_I=128, H_I=8, Nq=1, q_pos=[280000], k=10,
+                             seed=11, identical_keys=True)
+    assert swaps == 0 and sorted(idx[0, 0].tolist()) == list(range(10))
+
+
+def test_topk_long_row_stale_histogram(cuda_lib):
+    # split calls: the histogram is scored into twice before the top-k reads it (counts no longer match
+    # the scores), so the long rows fall back to the tournament; the selection is still exact
+    csa = cuda_lib
+    G = gen(12)
+    B, n, k = 2, 50000, 300
+    kI = normal((B, n, 128), 1.0, G)
+    qI = normal((B, 1, 8, 128), 1.0, G)
+    w = normal((B, 1, 8), 8 ** -0.5, G, dtype=torch.float32)
+    kc = csa.PackedCache(B, n, 128, 0, DEV, 1.0)
+    csa.pack_fp4(kI.to(DEV), kc)
+    n_c = torch.tensor([n, n - 5000], dtype=torch.int32, device=DEV)
+    q_pos = torch.tensor([[4 * n - 1], [4 * (n - 5000) - 1]], dtype=torch.int64, device=DEV)
+    scores = torch.empty((B, n), dtype=torch.float32, device=DEV)
+    hist = torch.zeros((B, 4096), dtype=torch.int32, device=DEV)
+    for _ in range(2):
+        csa.index_scores(qI.to(DEV), w.to(DEV), kc, n_c, q_pos, scores, ratio=4, hist=hist, k=k)
+    idx, sc, _ = csa.topk(scores, kc, n_c, q_pos, B=B, Nq=1, ratio=4, k=k, hist=hist, want_scores=True)
+    torch.cuda.synchronize()
+    assert int(hist.abs().sum()) == 0                     # the top-k left the histogram rows it read zero
+    for b in range(B):
+        codes, scales, _ = O.pack_fp4(f64(kI[b]), 0, 1.0)
+        s_ref, ids = O.index_scores(f64(qI[b]), f64(w[b]), 1.0, codes, scales, 1.0, q_pos[b].cpu().numpy(),
+                                    int(n_c[b]), 4)
+        check_topk_row(idx[b, 0].cpu().numpy(), s_ref[0], ids[0], k, f"stale histogram b={b}")
+
+
 def test_index_reindex_candidates(cuda_lib):
     G = gen(5)
     B, Nq, n_max, n_cand = 2, 2, 3000, 2048
