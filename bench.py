@@ -15,6 +15,7 @@ Prints one JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -53,6 +54,9 @@ def parse():
     p.add_argument("--rows", action="store_true",
                    help="time the hot-path rows outside the decode step (HCA pooling and dense attention, "
                         "cross-layer reuse, hierarchical index), one JSON line each")
+    p.add_argument("--flops", action="store_true",
+                   help="analytic precision-weighted decode FLOPs per token from 4K to 1M context next to the "
+                        "measured decode step at each context, one JSON line each")
     return p.parse_args()
 
 
@@ -92,6 +96,34 @@ def attention_bytes(s, B):
     query heads (bf16) in, the output heads (bf16) and lse out."""
     entry = s.d_n // 2 + 16 + s.d_r * 2
     return B * (s.k * (entry + 4) + s.W * s.d * 2 + s.H * s.d * 2 * 2 + s.H * 4)
+
+
+# Precision weights of the decode-FLOP curve ("DeepSeek-V4.1-Flash - Pushing the Limits of KV Cache
+# Compression", Fig. 2: BF16 operations count 1, FP8 0.5, FP4 0.25).
+FLOP_WEIGHT = {"bf16": 1.0, "fp8": 0.5, "fp4": 0.25, "fp32": 1.0}
+
+
+def decode_flops(T, s, mode="full", pool=16384):
+    """Precision-weighted FLOPs of one decode token of one attention layer at context T (tokens), by part.
+
+    Counted as this path computes them: the indexer's q_I.k_I products in FP4 (2 H_I d_I per scored
+    entry) and its ReLU-weighted head sum in fp32 (2 H_I per entry); the attention's two tensor-core
+    products in bf16 (2 H d each per key, keys = min(k, entries) + window; HCA: every entry + window);
+    the compressor's k_I projection of the new entry in bf16 (2 d d_I, once per r tokens).  The C, Z
+    projections come from upstream layers and the top-k compares, so neither counts.  Modes: "full"
+    scores every visible entry, "reindex" only a candidate pool of `pool` entries (the hierarchical
+    indexer's later layers), "reuse" runs no indexer, "hca" is the dense 128x layer."""
+    w = FLOP_WEIGHT
+    r = 128 if mode == "hca" else s.r
+    n = T // r
+    parts = {}
+    if mode != "hca":
+        parts["compressor_k_I"] = w["bf16"] * 2 * s.d * s.d_I / r
+    scored = {"full": n, "reindex": min(n, pool), "reuse": 0, "hca": 0}[mode]
+    parts["indexer"] = w["fp4"] * 2 * s.H_I * s.d_I * scored + w["fp32"] * 2 * s.H_I * scored
+    keys = (n if mode == "hca" else min(s.k, n)) + min(s.W, T)
+    parts["attention"] = w["bf16"] * 4 * s.H * s.d * keys
+    return {"total": sum(parts.values()), "parts": parts, "entries": n, "keys": keys}
 
 
 def sources_hash(paths):
@@ -608,6 +640,61 @@ def run_rows(args):
         torch.cuda.empty_cache()
 
 
+def run_flops(args):
+    """Analytic weighted FLOPs per token (every layer mode) next to the measured decode step (a Full-mode
+    CSA layer: compress, index, top-k, attention) at contexts 4K .. 1M, B = 8 sequences, L2 flushed
+    before every timed step."""
+    import compressed_sparse_attention_18_b200 as csa  # noqa: F401  (loads the library)
+    from compressed_sparse_attention_18_b200.layer import CSADecodeLayer, LayerShape
+    from csa_workloads import CFG2, decode_inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B = 8
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)       # larger than the 126 MB L2
+    stream = torch.cuda.Stream(dev)
+    for T in (4096, 16384, 65536, 131072, 262144, 1048576):
+        s = dataclasses.replace(CFG2, name=f"decode_{T // 1024}k", B=B, T=T)
+        ls = LayerShape(B=B, n_max=s.n_c, r=s.r, H=s.H, d=s.d, d_r=s.d_r, H_I=s.H_I, d_I=s.d_I, k=s.k, W=s.W)
+        L = CSADecodeLayer(ls, dev)
+        inp = decode_inputs(s, seed=5, device=dev, B=B, needles=0)
+        L.load_history(inp["kv_src"], inp["kI_src"], s.n_c)
+        L.win.copy_(inp["win_kv"])
+        del inp["kv_src"], inp["kI_src"]
+        torch.cuda.synchronize()
+
+        def step():
+            L.step(inp["C"], inp["Z"], inp["b_pos"], inp["W_IK"], inp["q"], inp["q_I"], inp["w"], stream=stream)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                step()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+            step()
+        times = []
+        for i in range(max(args.warmup, 3) + 30):
+            with torch.cuda.stream(stream):
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            if i >= max(args.warmup, 3):
+                times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        curve = {m: decode_flops(T, s, m) for m in ("full", "reindex", "reuse", "hca")}
+        print(json.dumps({"row": "decode FLOP curve", "context_tokens": T, "entries": s.n_c, "B": B,
+                          "weighted_mflop_per_token": {m: c["total"] / 1e6 for m, c in curve.items()},
+                          "full_parts_mflop": {k: v / 1e6 for k, v in curve["full"]["parts"].items()},
+                          "measured_full_layer": {"ms_per_step": ms, "us_per_token": ms * 1e3 / B,
+                                                  "tokens_per_s": B / (ms / 1e3), "l2": "flushed before each step"}}),
+              flush=True)
+        del g, L, inp
+        torch.cuda.empty_cache()
+
+
 def run_profile(args):
     """One layer state, `--steps` eager decode steps: the small case ncu captures run on."""
     from compressed_sparse_attention_18_b200.layer import CSADecodeLayer, LayerShape
@@ -632,6 +719,9 @@ def main():
         return
     if args.rows:
         run_rows(args)
+        return
+    if args.flops:
+        run_flops(args)
         return
     rank, world = dist_init(args.gpus)
     try:

@@ -15,7 +15,7 @@ def _load():
 
 def test_bench_modes_exist():
     b = _load()
-    for name in ("run_ours", "run_reference", "run_e2e", "run_profile", "run_rows", "cpu_baseline"):
+    for name in ("run_ours", "run_reference", "run_e2e", "run_profile", "run_rows", "run_flops", "cpu_baseline"):
         assert callable(getattr(b, name)), name
 
 
@@ -34,3 +34,27 @@ def test_algorithmic_bytes():
     # per sequence: 512 entries x (224 codes + 16 scales + 128 rope + 4 id) + 128 KB window + q + out + lse
     assert b.attention_bytes(CFG2, 1) == 512 * 372 + 128 * 1024 + 2 * 64 * 1024 + 64 * 4
     assert b.score_kernel_bytes(CFG2, 1) == 32768 * 72 + 8 * 128 * 2 + 8 * 4
+
+
+def test_decode_flop_curve():
+    """Closed forms of the weighted decode-FLOP model at the cfg2 layer shape (H=64, d=512, 8x128
+    indexer, top-512, window 128, r=4)."""
+    b = _load()
+    from csa_workloads import CFG2
+    s = CFG2
+    full = b.decode_flops(131072, s, "full")
+    n = 131072 // 4
+    assert full["entries"] == n and full["keys"] == 512 + 128
+    assert full["parts"]["indexer"] == 0.25 * 2 * 8 * 128 * n + 2 * 8 * n
+    assert full["parts"]["attention"] == 4 * 64 * 512 * 640
+    assert full["parts"]["compressor_k_I"] == 2 * 512 * 128 / 4
+    # below k entries every entry is attended; the window is capped by the context
+    small = b.decode_flops(1024, s, "full")
+    assert small["keys"] == 256 + 128
+    # Reuse runs no indexer: constant in the context once k entries exist; Reindex is constant once the
+    # context outgrows its pool; Full grows linearly with the entries; HCA attends over T/128 entries
+    assert b.decode_flops(4096, s, "reuse")["total"] == b.decode_flops(1 << 20, s, "reuse")["total"]
+    assert b.decode_flops(1 << 18, s, "reindex")["total"] == b.decode_flops(1 << 20, s, "reindex")["total"]
+    f4, f1m = b.decode_flops(4096, s, "full")["total"], b.decode_flops(1 << 20, s, "full")["total"]
+    assert abs((f1m - f4) - (0.25 * 2048 + 16) * ((1 << 18) - 1024)) < 1e-3 * f1m
+    assert b.decode_flops(1 << 20, s, "hca")["parts"]["attention"] == 4 * 64 * 512 * (8192 + 128)
