@@ -60,7 +60,7 @@ class AttnArgs(ctypes.Structure):
                 ("ratio", _i32), ("n_max", _i32), ("k", _i32), ("Wn", _i32), ("window", _i32),
                 ("g_kv", _f32), ("softmax_scale", _f32), ("q", _vp), ("q_pos", _vp), ("kv_codes", _vp),
                 ("kv_scales", _vp), ("kv_rope", _vp), ("n_c", _vp), ("idx", _vp), ("win_kv", _vp),
-                ("win_pos0", _vp), ("out", _vp), ("lse", _vp), ("flags", _u32)]
+                ("win_pos0", _vp), ("out", _vp), ("lse", _vp), ("flags", _u32), ("out_rope_theta", _f32)]
 
 
 _lib.csa_status_string.restype = ctypes.c_char_p
@@ -285,7 +285,7 @@ def _attn_args(q, q_pos, cache: PackedCache, n_c, idx, win_kv, win_pos0, ratio, 
 
 
 def _attn(fn, hca, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse, ws,
-          stream, early_start=False):
+          stream, early_start=False, out_rope_theta=0.0):
     B, Nq, H, d = q.shape
     if out is None:
         out = torch.empty_like(q)
@@ -293,6 +293,7 @@ def _attn(fn, hca, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, s
         lse = torch.empty((B, Nq, H), dtype=torch.float32, device=q.device)
     a = _attn_args(q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse)
     a.flags = CSA_EARLY_START if early_start else 0
+    a.out_rope_theta = out_rope_theta
     nbytes = _lib.csa_attn_workspace_size(ctypes.byref(a), hca)
     wbuf = _ws(nbytes, q.device, ws)
     _check(fn(ctypes.byref(a), _ptr(wbuf) if wbuf is not None else None, nbytes, _stream(stream)),
@@ -301,19 +302,20 @@ def _attn(fn, hca, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, s
 
 
 def sparse_attn(q, q_pos, cache: PackedCache, n_c, idx, win_kv=None, win_pos0=None, *, ratio=4, window=128,
-                softmax_scale=0.0, out=None, lse=None, ws=None, early_start=False, stream=None):
+                softmax_scale=0.0, out=None, lse=None, ws=None, early_start=False, out_rope_theta=0.0, stream=None):
     """CSA attention over the selected entries idx [B,Nq,k] plus the window.  Returns (out, lse).
     early_start: CSA_EARLY_START (window tiles start before the step's index and top-k kernels end;
-    only inside a decode step that began with compress)."""
+    only inside a decode step that began with compress).  out_rope_theta: inverse-RoPE epilogue on the
+    output's RoPE channels at the query position (0 = off)."""
     return _attn(_lib.csa_sparse_attn, 0, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window,
-                 softmax_scale, out, lse, ws, stream, early_start)
+                 softmax_scale, out, lse, ws, stream, early_start, out_rope_theta)
 
 
 def hca_attn(q, q_pos, cache: PackedCache, n_c, win_kv=None, win_pos0=None, *, ratio=128, window=128,
-             softmax_scale=0.0, out=None, lse=None, ws=None, stream=None):
+             softmax_scale=0.0, out=None, lse=None, ws=None, out_rope_theta=0.0, stream=None):
     """HCA attention over every visible entry plus the window.  Returns (out, lse)."""
     return _attn(_lib.hca_dense_attn, 1, q, q_pos, cache, n_c, None, win_kv, win_pos0, ratio, window,
-                 softmax_scale, out, lse, ws, stream)
+                 softmax_scale, out, lse, ws, stream, out_rope_theta=out_rope_theta)
 
 
 def attn_workspace_size(q, q_pos, cache, n_c, idx, win_kv, win_pos0, *, ratio, window, hca=False, early_start=False):

@@ -381,11 +381,41 @@ __device__ __forceinline__ void load_dims<float, 4>(const float* p, float* v) {
   v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
 }
 
+// Inverse-RoPE epilogue on one (query, head) row held one lane-slice of DPL dims per lane (lane l: dims
+// DPL l .. DPL l + DPL - 1): the RoPE channels (the last DR) sit on lanes L0 .. 31, the first half of each
+// pair (m) HL lanes before its second half (m + DR/2); every lane of the warp must call it.
+// (x1, x2) -> (x1 cos a + x2 sin a, -x1 sin a + x2 cos a), a = t theta^(-2m/DR): the angle in double,
+// reduced by 2 pi (split in two parts) before the single-precision sin / cos.
+template <int D>
+__device__ __forceinline__ void inverse_rope_lanes(float* y, int lane, long long t, float theta) {
+  constexpr int DPL = D / 32, DR = D == 512 ? 64 : 32, L0 = (D - DR) / DPL, HL = DR / 2 / DPL;
+  float pz[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) pz[i] = __shfl_xor_sync(0xffffffffu, y[i], HL);
+  if (lane < L0) return;
+  const int jl = lane - L0;
+  const bool first = jl < HL;
+  const int m0 = (jl % HL) * DPL;
+  const double l2t = log2((double)theta);
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    const double ang = (double)t * exp2(-2.0 * (double)(m0 + i) / DR * l2t);
+    const double kk = rint(ang * 0.15915494309189535);             // 1 / (2 pi)
+    double red = fma(-kk, 6.283185307179586, ang);                  // 2 pi, high part
+    red = fma(-kk, 2.4492935982947064e-16, red);                    // 2 pi, low part
+    float sn, cs;
+    sincosf((float)red, &sn, &cs);
+    const float x1 = first ? y[i] : pz[i], x2 = first ? pz[i] : y[i];
+    y[i] = first ? fmaf(x1, cs, x2 * sn) : fmaf(-x1, sn, x2 * cs);
+  }
+}
+
 template <typename PT, int D>
 __global__ void __launch_bounds__(MERGE_WARPS * 32) attn_merge_kernel(const PT* __restrict__ part_o,
                                                                      const float* __restrict__ part_lse, int splits,
                                                                      int H, long long units, uint16_t* __restrict__ out,
-                                                                     float* __restrict__ lse) {
+                                                                     float* __restrict__ lse,
+                                                                     const int64_t* __restrict__ q_pos, float rope_theta) {
   constexpr int DPL = D / 32;
   constexpr int MERGE_CHUNK = D == 512 ? 6 : 8;   // splits whose partials are in flight at once
   const int lane = threadIdx.x & 31;
@@ -450,10 +480,13 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) attn_merge_kernel(const PT* 
     }
   }
   const float inv = sum > 0.f ? 1.f / sum : 0.f;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) acc[i] *= inv;
+  if (rope_theta != 0.f) inverse_rope_lanes<D>(acc, lane, q_pos[bq], rope_theta);
   uint16_t* o = out + (bq * H + h) * (long long)D + lane * DPL;
   uint32_t pk[DPL / 2];
 #pragma unroll
-  for (int i = 0; i < DPL / 2; ++i) pk[i] = pack_bf16x2(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+  for (int i = 0; i < DPL / 2; ++i) pk[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
   if (DPL == 16) {
     reinterpret_cast<uint4*>(o)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
@@ -465,14 +498,48 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) attn_merge_kernel(const PT* 
 
 template <typename PT>
 static csa_status launch_merge(const PT* po, const float* pl, int splits, int H, int D, long long rows, uint16_t* out,
-                               float* lse, cudaStream_t st) {
+                               float* lse, const int64_t* q_pos, float rope_theta, cudaStream_t st) {
   const long long units = rows * H;
   const unsigned grid = (unsigned)((units + MERGE_WARPS - 1) / MERGE_WARPS);
   if (D == 512)
     return launch_pdl(attn_merge_kernel<PT, 512>, dim3(grid), dim3(MERGE_WARPS * 32), 0, st, po, pl, splits, H, units,
-                      out, lse);
+                      out, lse, q_pos, rope_theta);
   return launch_pdl(attn_merge_kernel<PT, 128>, dim3(grid), dim3(MERGE_WARPS * 32), 0, st, po, pl, splits, H, units,
-                    out, lse);
+                    out, lse, q_pos, rope_theta);
+}
+
+// Inverse-RoPE epilogue in place on a finished bf16 output (launches without split partials): one warp
+// per (query, head), the same lane layout and rotation as the merge.
+template <int D>
+__global__ void __launch_bounds__(MERGE_WARPS * 32) out_rope_kernel(uint16_t* __restrict__ out, int H, long long units,
+                                                                    const int64_t* __restrict__ q_pos, float rope_theta) {
+  constexpr int DPL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const long long unit = (long long)blockIdx.x * MERGE_WARPS + (threadIdx.x >> 5);
+  pdl_trigger();
+  pdl_wait();
+  if (unit >= units) return;
+  uint16_t* o = out + unit * (long long)D + lane * DPL;
+  float y[DPL];
+  load_dims<uint16_t, DPL>(o, y);
+  inverse_rope_lanes<D>(y, lane, q_pos[unit / H], rope_theta);
+  uint32_t pk[DPL / 2];
+#pragma unroll
+  for (int i = 0; i < DPL / 2; ++i) pk[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
+  if (DPL == 16) {
+    reinterpret_cast<uint4*>(o)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    reinterpret_cast<uint4*>(o)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  } else {
+    *reinterpret_cast<uint2*>(o) = make_uint2(pk[0], pk[1]);
+  }
+}
+
+static csa_status launch_out_rope(uint16_t* out, int H, int D, long long rows, const int64_t* q_pos, float theta,
+                                  cudaStream_t st) {
+  const long long units = rows * H;
+  const unsigned grid = (unsigned)((units + MERGE_WARPS - 1) / MERGE_WARPS);
+  if (D == 512) return launch_pdl(out_rope_kernel<512>, dim3(grid), dim3(MERGE_WARPS * 32), 0, st, out, H, units, q_pos, theta);
+  return launch_pdl(out_rope_kernel<128>, dim3(grid), dim3(MERGE_WARPS * 32), 0, st, out, H, units, q_pos, theta);
 }
 
 // tensor-core decode path (attn_tc.cu)
@@ -563,8 +630,13 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
     uint16_t* po = p.splits > 1 ? (uint16_t*)((uint8_t*)ws + p.off_o) : nullptr;
     float* pl = p.splits > 1 ? (float*)((uint8_t*)ws + p.off_lse) : nullptr;
     csa_status s = launch_attn_tc(a, hca, p.splits, p.tpc, po, pl, st);
-    if (s != CSA_OK || p.splits == 1) return s;
-    return launch_merge<uint16_t>(po, pl, p.splits, a->H, a->d, rows, (uint16_t*)a->out, a->lse, st);
+    if (s != CSA_OK) return s;
+    if (p.splits == 1)
+      return a->out_rope_theta != 0.0f
+                 ? launch_out_rope((uint16_t*)a->out, a->H, a->d, rows, a->q_pos, a->out_rope_theta, st)
+                 : CSA_OK;
+    return launch_merge<uint16_t>(po, pl, p.splits, a->H, a->d, rows, (uint16_t*)a->out, a->lse, a->q_pos,
+                                  a->out_rope_theta, st);
   }
   AttnParams P{};
   P.B = a->B; P.Nq = a->Nq; P.H = a->H; P.d_r = a->d_rope; P.ratio = a->ratio; P.n_max = a->n_max;
@@ -584,8 +656,13 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
     s = launch_attn<512, 2>(P, units, st);
   else
     s = launch_attn<128, 8>(P, units, st);
-  if (s != CSA_OK || p.splits == 1) return s;
-  return launch_merge<float>(P.part_o, P.part_lse, p.splits, a->H, a->d, rows, (uint16_t*)a->out, a->lse, st);
+  if (s != CSA_OK) return s;
+  if (p.splits == 1)
+    return a->out_rope_theta != 0.0f
+               ? launch_out_rope((uint16_t*)a->out, a->H, a->d, rows, a->q_pos, a->out_rope_theta, st)
+               : CSA_OK;
+  return launch_merge<float>(P.part_o, P.part_lse, p.splits, a->H, a->d, rows, (uint16_t*)a->out, a->lse, a->q_pos,
+                             a->out_rope_theta, st);
 }
 
 }  // namespace csa

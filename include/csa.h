@@ -265,6 +265,12 @@ typedef struct csa_attn_args {
   void* out;
   float* lse;
   uint32_t flags;          /* CSA_EARLY_START or 0 */
+  /* Inverse-RoPE epilogue ([V4.1 notes] §実装上の工夫, inference kernels: the fused
+     "RoPE-attention-RoPE-cast" kernel): nonzero rotates the last d_rope channels of out by the
+     inverse of the query's RoPE, angle -t * out_rope_theta^(-2m/d_rope) for the half-split pair
+     (m, m + d_rope/2), before the bf16 cast; the values' RoPE channels, rotated at their own positions,
+     then come out relative to the query.  lse is unchanged.  0 = off. */
+  float out_rope_theta;
 } csa_attn_args;
 
 size_t csa_attn_workspace_size(const csa_attn_args* args, int hca);

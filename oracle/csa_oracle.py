@@ -15,7 +15,9 @@ Sources (page titles; section / figure / equation):
   [V4.1 notes] "DeepSeek-V4.1-Flash - Pushing the Limits of KV Cache Compression" — §提案手法/アーキテクチャ:
               CED bullet eq.(1) (C, Z projections), CSA2 bullet + Fig. 4 (Full/Reindex/Reuse),
               Hierarchical Sparse Indexer bullet + Fig. 5, FP4 主 KV キャッシュ bullet.
-Readings of what the pages leave open are those written in SPEC.md (S1-S8).
+Where the pages leave a step open, the reading taken is stated at the function that takes it; the
+section tags S1-S8 below name the parts of the layer (compressor, pack, indexer, top-k, attention,
+window, hierarchical pool, reuse).
 
 Pinned by tests/test_oracle_*.py against closed forms, invariants, library routines (torch's FP8
 cast, torch SDPA) and brute force on tiny inputs.  Parity of the end-to-end layer against the pages
@@ -368,12 +370,16 @@ def window_rows(t: int, win_kv, win_pos0: int, W: int):
 
 
 def attention(q, q_pos, kv_rows, idx, n_c: int, win_kv, win_pos0: int, W: int, scale: float,
-              round_out: bool = True):
+              round_out: bool = True, out_rope_theta: float = 0.0, d_rope: int = 0):
     """One sequence.  q [Nq, H, d] (bf16 values, already rotated); kv_rows [n, d] dequantized entries;
     idx [Nq, k] selected entry ids (entries < 0 or >= n_c skipped); window buffer win_kv [Wn, d] at
     positions win_pos0 ...  One joint softmax over selected ∪ window with logits scale·(q·K);
     K = V (one shared KV head).  Returns (out [Nq, H, d] (bf16-rounded unless round_out=False),
-    lse [Nq, H] natural log, -inf for an empty set)."""
+    lse [Nq, H] natural log, -inf for an empty set).
+    out_rope_theta != 0: the "RoPE-attention-RoPE-cast" epilogue ([V4.1 notes] §実装上の工夫, inference
+    kernels): before the bf16 cast the last d_rope channels of out are rotated back by the query's
+    own RoPE (position -t), so the values' rotations come out relative to the query (a reading: the
+    pages name the kernel, not its formula)."""
     q = np.asarray(q, np.float64)
     Nq, H, d = q.shape
     out = np.zeros((Nq, H, d))
@@ -390,13 +396,15 @@ def attention(q, q_pos, kv_rows, idx, n_c: int, win_kv, win_pos0: int, W: int, s
         ssum = e.sum(axis=1, keepdims=True)
         lse[qi] = (mx + np.log(ssum))[:, 0]
         out[qi] = (e / ssum) @ K
+        if out_rope_theta != 0.0 and d_rope:
+            out[qi] = rope_rotate(out[qi], np.full(H, -float(q_pos[qi])), d_rope, out_rope_theta)
     if round_out:
         out = bf16_round(out)
     return out, lse
 
 
 def hca_attention(q, q_pos, kv_rows, n_c: int, r: int, win_kv, win_pos0: int, W: int, scale: float,
-                  round_out: bool = True):
+                  round_out: bool = True, out_rope_theta: float = 0.0, d_rope: int = 0):
     """HCA: attention over every visible compressed entry (i < n_c, r i + r - 1 <= t) plus the window."""
     q_pos = np.asarray(q_pos, np.int64)
     Nq = q.shape[0]
@@ -405,7 +413,7 @@ def hca_attention(q, q_pos, kv_rows, n_c: int, r: int, win_kv, win_pos0: int, W:
     idx = np.full((Nq, max(kmax, 1)), -1, dtype=np.int64)
     for qi in range(Nq):
         idx[qi, : n_vis[qi]] = np.arange(n_vis[qi])
-    return attention(q, q_pos, kv_rows, idx, n_c, win_kv, win_pos0, W, scale, round_out)
+    return attention(q, q_pos, kv_rows, idx, n_c, win_kv, win_pos0, W, scale, round_out, out_rope_theta, d_rope)
 
 
 def lse_merge(out1, lse1, out2, lse2):

@@ -1,4 +1,5 @@
-"""Comparison helpers for the GPU-vs-oracle parity tests (tolerances of SPEC S8)."""
+"""Comparison helpers for the GPU-vs-oracle parity tests: the bf16-output, lse and score tolerances and
+the accepted top-k boundary swaps."""
 from __future__ import annotations
 
 import logging

@@ -272,7 +272,7 @@ def test_index_k_larger_than_visible(cuda_lib):
 # -------------------------------------------------------------------------------------- attention
 
 def _attn_case(csa, *, B, Nq, H, d, d_r, n_max, n_c, q_pos, k=0, Wn=128, win_pos0=None, hca=False, ratio=4,
-               seed=0, g=1.0, q_scale=1.0):
+               seed=0, g=1.0, q_scale=1.0, rope_theta=0.0):
     G = gen(seed)
     kv = normal((B, n_max, d), 1.0, G)
     q = normal((B, Nq, H, d), q_scale, G)
@@ -294,11 +294,11 @@ def _attn_case(csa, *, B, Nq, H, d, d_r, n_max, n_c, q_pos, k=0, Wn=128, win_pos
     if hca:
         out, lse = csa.hca_attn(q.to(DEV), q_pos_t.to(DEV), cache, n_c_t.to(DEV),
                                 win.to(DEV) if win is not None else None, wp0.to(DEV) if win is not None else None,
-                                ratio=ratio)
+                                ratio=ratio, out_rope_theta=rope_theta)
     else:
         out, lse = csa.sparse_attn(q.to(DEV), q_pos_t.to(DEV), cache, n_c_t.to(DEV), idx.to(DEV),
                                    win.to(DEV) if win is not None else None, wp0.to(DEV) if win is not None else None,
-                                   ratio=ratio)
+                                   ratio=ratio, out_rope_theta=rope_theta)
     torch.cuda.synchronize()
     scale = d ** -0.5
     for b in range(B):
@@ -307,13 +307,28 @@ def _attn_case(csa, *, B, Nq, H, d, d_r, n_max, n_c, q_pos, k=0, Wn=128, win_pos
         wb = f64(win[b]) if win is not None else np.zeros((0, d))
         if hca:
             o_ref, l_ref = O.hca_attention(f64(q[b]), q_pos_t[b].numpy(), rows, n_c[b], ratio, wb, win_pos0[b], 128,
-                                           scale)
+                                           scale, out_rope_theta=rope_theta, d_rope=d_r)
         else:
             o_ref, l_ref = O.attention(f64(q[b]), q_pos_t[b].numpy(), rows, idx[b].numpy(), n_c[b], wb, win_pos0[b],
-                                       128, scale)
+                                       128, scale, out_rope_theta=rope_theta, d_rope=d_r)
         assert_close(f64(out[b]), o_ref, OUT_ATOL, OUT_RTOL, f"out b={b}")
         assert_close(lse[b].cpu().numpy(), l_ref, LSE_ATOL, LSE_RTOL, f"lse b={b}")
     return out, lse
+
+
+@pytest.mark.parametrize("k,Wn", [(512, 128), (64, 0)])   # split partials + merge; one tile, no merge
+def test_attn_inverse_rope_epilogue(cuda_lib, k, Wn):
+    n = 4096
+    _attn_case(cuda_lib, B=2, Nq=1, H=64, d=512, d_r=64, n_max=n, n_c=[n, n - 7], q_pos=[4 * n - 1, 4 * n - 30],
+               k=k, Wn=Wn, seed=31, rope_theta=10000.0)
+
+
+def test_attn_inverse_rope_epilogue_d128_and_hca(cuda_lib):
+    q_pos = list(range(4080, 4096))
+    _attn_case(cuda_lib, B=1, Nq=16, H=8, d=128, d_r=32, n_max=1024, n_c=[1024], q_pos=q_pos, k=64, seed=32,
+               rope_theta=10000.0)
+    _attn_case(cuda_lib, B=2, Nq=1, H=64, d=512, d_r=64, n_max=300, n_c=[300, 150],
+               q_pos=[128 * 300 - 1, 128 * 150 + 5], hca=True, ratio=128, seed=33, rope_theta=10000.0)
 
 
 def test_attn_tiles_per_cta_with_rescale(cuda_lib):

@@ -1,4 +1,4 @@
-"""Pins for the oracle's number formats and FP4 pack (SPEC S2), no GPU.
+"""Pins for the oracle's number formats and FP4 pack, no GPU.
 
 Each check ties the oracle to something other than itself: the OCP format tables (golden fixtures),
 torch's FP8 E4M3 cast (a library routine), brute-force nearest-value search, exact round trips and

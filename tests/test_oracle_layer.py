@@ -1,4 +1,4 @@
-"""Pins for the oracle's compressor, indexer, top-k, attention and reuse paths (SPEC S1, S3-S7), no GPU.
+"""Pins for the oracle's compressor, indexer, top-k, attention and reuse paths, no GPU.
 
 Each check ties the oracle to something it does not compute itself: closed forms (uniform / one-hot /
 known gates, RoPE at position 0 and on unit vectors), library routines (torch matmul, torch SDPA),
@@ -246,6 +246,28 @@ def test_attention_one_key_and_constant_values():
     out, _ = O.attention(q, [100], const, np.array([[0, 1, 2, 3]]), 4, np.tile(kv[1], (5, 1)), 96, 128,
                          0.3, round_out=False)
     assert np.allclose(out[0], np.tile(kv[1], (3, 1)), rtol=1e-14, atol=1e-14)   # rows sum to 1
+
+
+def test_attention_inverse_rope_epilogue_closed_form():
+    """One key (softmax weight 1): out is the key, whose RoPE pairs were stored rotated at its position
+    p.  The epilogue rotates them back by the query position t, so pair m comes out as its raw value
+    rotated by (p - t) * theta^(-2m/d_rope); the unit raw pair (1, 0) gives (cos, sin) of that angle."""
+    d, d_r, theta = 12, 4, 10000.0
+    f = [1.0, theta ** -0.5]                                   # theta^(-2m/d_r), m = 0, 1
+    for p, t in ((900, 900), (901, 900), (37, 4095)):
+        key = np.zeros(d)
+        key[:8] = np.arange(1, 9)
+        for m in range(2):                                     # raw pair (1, 0) stored rotated at p
+            key[8 + m], key[10 + m] = math.cos(p * f[m]), math.sin(p * f[m])
+        q = np.ones((1, 1, d))
+        out, _ = O.attention(q, [t], key[None], np.array([[0]]), 1, np.zeros((0, d)), 0, 128, 0.1,
+                             round_out=False, out_rope_theta=theta, d_rope=d_r)
+        assert np.array_equal(out[0, 0, :8], key[:8])          # channels outside the RoPE slice untouched
+        for m in range(2):
+            a = (p - t) * f[m]
+            assert abs(out[0, 0, 8 + m] - math.cos(a)) < 1e-9 and abs(out[0, 0, 10 + m] - math.sin(a)) < 1e-9
+        off, _ = O.attention(q, [t], key[None], np.array([[0]]), 1, np.zeros((0, d)), 0, 128, 0.1, round_out=False)
+        assert np.array_equal(off[0, 0], key)                  # theta = 0: no epilogue
 
 
 def test_attention_lse_merge_of_disjoint_sets():
