@@ -60,13 +60,30 @@ def parse():
     return p.parse_args()
 
 
-def dist_init(n):
+def dist_init(n, backend=None):
+    """One process per GPU (torchrun env); NCCL on GPUs, gloo when the host has none (CPU tests)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if world > 1:
         import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return rank, world
+
+
+def max_over_ranks(x, world, device):
+    """The slowest rank's time: every multi-GPU number is the max over ranks."""
+    if world > 1:
+        t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+    return float(x)
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units all ranks processed per second over the max-over-ranks time (weak scaling: fixed work per rank)."""
+    return units_per_rank * world / (ms / 1e3)
 
 
 def config_dict(s):
@@ -349,12 +366,8 @@ def run_ours(args, rank, world):
     stream.synchronize()
     stage = [[marks[li][j].elapsed_time(marks[li][j + 1]) for j in range(4)] for li in range(LAYERS)]
     score_ms = statistics.mean(st[1] for st in stage)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
-    tokens = s.B * args.steps * world
-    value = tokens / (ms / 1e3)
+    ms = max_over_ranks(ms, world, dev)
+    value = whole_job_rate(s.B * args.steps, world, ms)
 
     # ---- end to end through the public API: pinned host inputs in, result out, every step
     e2e = run_e2e(args, layers, inputs, stream, dev, world)
@@ -463,12 +476,9 @@ def run_e2e(args, layers, inputs, stream, dev, world):
     t1.record(d2h)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, world, dev)
     B = layers[0].s.B
-    return {"value": B * steps * world / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": nbytes_in,
+    return {"value": whole_job_rate(B * steps, world, ms), "unit": UNIT, "h2d_bytes_per_step": nbytes_in,
             "d2h_bytes_per_step": nbytes_out, "steps": steps,
             "note": "pinned host buffers; copies on two copy streams overlapped with the neighbouring steps' "
                     "kernels (CUDA graph per layer step)"}
