@@ -177,6 +177,54 @@ def dequant_fp4(codes, scales, d_n: int, g: float = 1.0):
 
 
 # --------------------------------------------------------------------------------------------
+# S6  FP8 window — [V4.1 notes] FP4 主 KV キャッシュ bullet (the sliding-window KV stays in FP8, being
+#     more sensitive to quantisation); [V4 blog] storage paragraph (FP8 KV with the RoPE channels in
+#     BF16).  The pages fix the element format, not its scaling: reading taken here, one fp32 scale per
+#     64 channels of a row (the attention's 64-channel blocks), s = fp32(amax / 448), elements
+#     E4M3 RNE with saturation, an all-zero block has scale 0 and codes 0; RoPE channels stay bf16.
+# --------------------------------------------------------------------------------------------
+
+FP8_WIN_BLOCK = 64
+
+
+def pack_fp8_window(rows, d_rope: int):
+    """Window rows [n, d] (bf16 values as float64) -> (codes u8 [n, d_n] E4M3 bit patterns, scales fp32
+    [n, d_n / 64], rope float64 [n, d_rope])."""
+    rows = np.asarray(rows, np.float64)
+    n, d = rows.shape
+    d_n = d - d_rope
+    assert d_n % FP8_WIN_BLOCK == 0
+    blocks = rows[:, :d_n].reshape(n, d_n // FP8_WIN_BLOCK, FP8_WIN_BLOCK)
+    amax = np.abs(blocks).max(axis=-1)
+    scale = (fp32(amax) / np.float32(E4M3_MAX)).astype(np.float32)          # fp32 division
+    safe = np.where(scale > 0, scale, np.float32(1.0))
+    q = (fp32(blocks) / safe[..., None]).astype(np.float32)                  # fp32 division
+    v = e4m3_rne_satfinite(q.astype(np.float64))
+    v = np.where(scale[..., None] > 0, v, 0.0)
+    codes = e4m3_encode(np.abs(v)) | np.where(v < 0, 0x80, 0).astype(np.uint8)
+    return codes.reshape(n, d_n).astype(np.uint8), scale, rows[:, d_n:].copy()
+
+
+def dequant_fp8_window(codes, scales, rope):
+    """Window rows [n, d] float64: e4m3(code) * scale of its 64-channel block, then the bf16 RoPE part."""
+    codes = np.asarray(codes)
+    n, d_n = codes.shape
+    vals = e4m3_decode(codes).reshape(n, d_n // FP8_WIN_BLOCK, FP8_WIN_BLOCK)
+    vals = vals * np.asarray(scales, np.float64)[..., None]
+    return np.concatenate([vals.reshape(n, d_n), np.asarray(rope, np.float64)], axis=-1)
+
+
+def paged_rows(pool, block_table, page: int, n: int):
+    """Logical entries 0 .. n-1 of one sequence in a paged cache: entry i lives in slot i % page of the
+    physical page block_table[i // page] of ``pool[n_pages, page, ...]`` (a reading for the paged cache:
+    the pages name paged KV for serving but give no layout)."""
+    pool = np.asarray(pool)
+    table = np.asarray(block_table, np.int64)
+    i = np.arange(n)
+    return pool[table[i // page], i % page]
+
+
+# --------------------------------------------------------------------------------------------
 # S1  Compressor — [V4 blog] §ハイブリッド注意, Fig. 3 (4x softmax-gated pooling with a learned
 #     positional bias) and Fig. 4 (128x for HCA); [V4.1 notes] CED bullet eq.(1) (C, Z are separate
 #     projections of the hidden state) and CSA2 bullet (no overlapping entries; indexer K projected

@@ -161,3 +161,59 @@ def test_pack_tiny_block_scale_underflow_zeroes_block():
     assert np.all(codes == 0) and sc[0, 0] == 0
     codes, sc, _ = O.pack_fp4(src, 0, 2.0 ** -8)           # a global scale brings it back in range
     assert sc[0, 0] != 0 and np.all(O.dequant_fp4(codes, sc, 32, 2.0 ** -8) > 0)
+
+
+# ------------------------------------------------------------------------------------ FP8 window
+
+def test_fp8_window_exact_round_trip_at_power_of_two_scales():
+    """Blocks built from E4M3 grid values times 2^k with 448 * 2^k present: the block scale is exactly
+    2^k and every code comes back (positive and negative codes, subnormals included)."""
+    grid = O.e4m3_decode(np.arange(0, 0x7F))                  # every finite non-negative E4M3 value
+    rng = np.random.default_rng(5)
+    for k in (-8, 0, 3):
+        vals = rng.choice(grid, size=(4, 128)) * rng.choice([-1.0, 1.0], size=(4, 128))
+        vals[:, 0] = 448.0
+        vals[:, 64] = -448.0
+        rows = np.concatenate([vals * 2.0 ** k, rng.standard_normal((4, 32))], axis=1)
+        codes, scales, rope = O.pack_fp8_window(rows, 32)
+        assert np.all(scales == np.float32(2.0 ** k))
+        assert np.array_equal(O.dequant_fp8_window(codes, scales, rope), rows)
+
+
+def test_fp8_window_error_bound_zero_blocks_and_rope():
+    """|x - x_hat| <= half an E4M3 step at |x| / s (2^-4 relative for normals, 2^-10 s for subnormals);
+    an all-zero block packs to scale 0 and zero codes; the RoPE channels pass through."""
+    rng = np.random.default_rng(6)
+    rows = O.bf16_round(rng.standard_normal((16, 192)) * np.exp(rng.uniform(-6, 6, size=(16, 1))))
+    rows[3, :64] = 0.0
+    codes, scales, rope = O.pack_fp8_window(rows, 64)
+    assert scales[3, 0] == 0 and not codes[3, :64].any()
+    back = O.dequant_fp8_window(codes, scales, rope)
+    assert np.array_equal(back[:, 128:], rows[:, 128:])
+    s = np.repeat(scales.astype(np.float64), 64, axis=1)
+    x = rows[:, :128]
+    err = np.abs(back[:, :128] - x)
+    a = np.abs(x) / np.where(s > 0, s, 1.0)
+    bound = np.where(a >= 2.0 ** -6, np.ldexp(1.0, np.floor(np.log2(np.maximum(a, 2.0 ** -6))).astype(int) - 4),
+                     2.0 ** -10) * s
+    assert np.all(err <= bound * (1 + 1e-6) + 1e-300)
+    assert np.all(np.abs(back[:, :128]).max(axis=1) <= 448.0 * s.max(axis=1) * (1 + 1e-7))
+
+
+def test_paged_rows_brute_force_and_identity_table():
+    """Entry i of a paged cache is slot i % page of page table[i // page]: checked element by element
+    against a loop over the pages, and an identity table over a contiguous pool gives the rows back."""
+    rng = np.random.default_rng(7)
+    page, n_pages = 16, 12
+    pool = rng.standard_normal((n_pages, page, 5))
+    table = rng.permutation(n_pages)[:7]
+    n = 7 * page - 3
+    got = O.paged_rows(pool, table, page, n)
+    want = []
+    for p_i, phys in enumerate(table):
+        for slot in range(page):
+            if p_i * page + slot < n:
+                want.append(pool[phys, slot])
+    assert np.array_equal(got, np.array(want))
+    flat = rng.standard_normal((4 * page, 5))
+    assert np.array_equal(O.paged_rows(flat.reshape(4, page, 5), np.arange(4), page, 4 * page - 1), flat[:-1])
