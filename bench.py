@@ -54,6 +54,9 @@ def parse():
     p.add_argument("--rows", action="store_true",
                    help="time the hot-path rows outside the decode step (HCA pooling and dense attention, "
                         "cross-layer reuse, hierarchical index), one JSON line each")
+    p.add_argument("--spec", action="store_true",
+                   help="multi-query decode with speculative positions: 5 draft positions per sequence, "
+                        "B=32 at 128K context (index + top-k + attention), one JSON line")
     p.add_argument("--flops", action="store_true",
                    help="analytic precision-weighted decode FLOPs per token from 4K to 1M context next to the "
                         "measured decode step at each context, one JSON line each")
@@ -705,6 +708,58 @@ def run_flops(args):
         torch.cuda.empty_cache()
 
 
+def run_spec(args):
+    """Speculative multi-position decode: every sequence scores, selects and attends for 5 consecutive
+    draft positions at once (one multi-query index pass reads each key once for all 5), B = 32 at 128K
+    context, 4 cache states rotated, CUDA events around the timed steps."""
+    import compressed_sparse_attention_18_b200 as csa
+    from csa_workloads import CFG2, decode_inputs, gen, normal
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    s = CFG2
+    B, Nq, R = s.B, 5, 4
+    n = s.n_c
+    t0 = 4 * n - 5
+    Wn = s.W + Nq - 1
+    states = []
+    for li in range(R):
+        inp = decode_inputs(s, seed=60 + li, device=dev, needles=0)
+        G = gen(70 + li, dev)
+        st = {"q_I": normal((B, Nq, s.H_I, s.d_I), 1.0, G, dev), "w": normal((B, Nq, s.H_I), s.H_I ** -0.5, G, dev,
+                                                                          torch.float32),
+              "q": normal((B, Nq, s.H, s.d), 1.0, G, dev), "win": normal((B, Wn, s.d), 1.0, G, dev)}
+        st["ki"] = csa.PackedCache(B, n, s.d_I, 0, dev)
+        csa.pack_fp4(inp["kI_src"], st["ki"])
+        st["kv"] = csa.PackedCache(B, n, s.d, s.d_r, dev)
+        csa.pack_fp4(inp["kv_src"], st["kv"])
+        del inp
+        states.append(st)
+    q_pos = (t0 + torch.arange(Nq, device=dev)).view(1, Nq).repeat(B, 1).contiguous()
+    win_pos0 = torch.full((B,), t0 - s.W + 1, dtype=torch.int64, device=dev)
+    n_c = torch.full((B,), n, dtype=torch.int32, device=dev)
+    st0 = states[0]
+    idx = torch.empty((B, Nq, s.k), dtype=torch.int32, device=dev)
+    out = torch.empty((B, Nq, s.H, s.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Nq, s.H), dtype=torch.float32, device=dev)
+    ws_i = torch.empty(max(csa.index_topk_workspace_size(st0["q_I"], st0["w"], st0["ki"], n_c, q_pos, ratio=s.r,
+                                                         k=s.k), 1), dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(max(csa.attn_workspace_size(st0["q"], q_pos, st0["kv"], n_c, idx, st0["win"], win_pos0,
+                                                   ratio=s.r, window=s.W), 1), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    def step(i):
+        st = states[i % R]
+        csa.index_topk(st["q_I"], st["w"], st["ki"], n_c, q_pos, ratio=s.r, k=s.k, idx_out=idx, ws=ws_i)
+        csa.sparse_attn(st["q"], q_pos, st["kv"], n_c, idx, st["win"], win_pos0, ratio=s.r, window=s.W, out=out,
+                        lse=lse, ws=ws_a)
+    ms = _event_ms(step, 40)
+    print(json.dumps({"row": "speculative decode (5 draft positions per sequence)", "B": B, "positions": Nq,
+                      "context_tokens": s.T, "entries": n, "top_k": s.k, "window": s.W, "ms_per_step": ms,
+                      "value": B * Nq / (ms / 1e3), "unit": "tokens/s",
+                      "note": "index + top-k + attention per step (compress of the drafts' groups not included); "
+                              "4 cache states rotated (inputs larger than L2)"}), flush=True)
+
+
 def run_profile(args):
     """One layer state, `--steps` eager decode steps: the small case ncu captures run on."""
     from compressed_sparse_attention_18_b200.layer import CSADecodeLayer, LayerShape
@@ -732,6 +787,9 @@ def main():
         return
     if args.flops:
         run_flops(args)
+        return
+    if args.spec:
+        run_spec(args)
         return
     rank, world = dist_init(args.gpus)
     try:

@@ -15,7 +15,7 @@ def _load():
 
 def test_bench_modes_exist():
     b = _load()
-    for name in ("run_ours", "run_reference", "run_e2e", "run_profile", "run_rows", "run_flops", "cpu_baseline"):
+    for name in ("run_ours", "run_reference", "run_e2e", "run_profile", "run_rows", "run_flops", "run_spec", "cpu_baseline"):
         assert callable(getattr(b, name)), name
 
 

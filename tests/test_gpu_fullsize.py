@@ -166,3 +166,41 @@ def test_reuse_cfg4_full_size(cuda_lib):
     sc2, ids2 = O.index_scores(f64(qI2[b, 0])[None], f64(w2[b, 0])[None], 1.0, codes, scales, 1.0, [t], s.n_c, s.r,
                                keys=idx1[b].cpu().numpy())
     check_topk_row(idx2[b, 0].cpu().numpy(), sc2[0], ids2[0], s.extra["k2"], "layer 2 reindex")
+
+
+def test_speculative_decode_five_positions_full_context(cuda_lib):
+    """Multi-query decode with speculative positions: 5 consecutive draft positions t .. t+4 per
+    sequence over a 128K-token context (32768 entries), each with its own visible set, top-512 and
+    128-token window (the window buffer holds 132 tokens); every value of sequence 0 against the oracle."""
+    csa = cuda_lib
+    s = CFG2
+    B, Nq, n = 2, 5, s.n_c
+    inp = decode_inputs(s, seed=41, device=DEV, B=B, needles=0)
+    G = gen(42, DEV)
+    q_I = normal((B, Nq, s.H_I, s.d_I), 1.0, G, DEV)
+    w = normal((B, Nq, s.H_I), s.H_I ** -0.5, G, DEV, torch.float32)
+    q = normal((B, Nq, s.H, s.d), 1.0, G, DEV)
+    t0 = 4 * n - 5                                          # first draft position: n - 1 entries visible
+    q_pos = (t0 + torch.arange(Nq, device=DEV)).view(1, Nq).repeat(B, 1).contiguous()
+    Wn = s.W + Nq - 1
+    win = normal((B, Wn, s.d), 1.0, G, DEV)
+    win_pos0 = torch.full((B,), t0 - s.W + 1, dtype=torch.int64, device=DEV)
+    ki = csa.PackedCache(B, n, s.d_I, 0, DEV)
+    csa.pack_fp4(inp["kI_src"], ki)
+    kv = csa.PackedCache(B, n, s.d, s.d_r, DEV)
+    csa.pack_fp4(inp["kv_src"], kv)
+    n_c = torch.full((B,), n, dtype=torch.int32, device=DEV)
+    idx, _, _ = csa.index_topk(q_I, w, ki, n_c, q_pos, ratio=s.r, k=s.k)
+    out, lse = csa.sparse_attn(q, q_pos, kv, n_c, idx, win, win_pos0, ratio=s.r, window=s.W)
+    torch.cuda.synchronize()
+    b = 0
+    codes, scales = np_u8(ki.codes[b]), np_u8(ki.scales[b])
+    tp = q_pos[b].cpu().numpy()
+    sc, ids = O.index_scores(f64(q_I[b]), f64(w[b]), 1.0, codes, scales, 1.0, tp, n, s.r)
+    for qq in range(Nq):
+        check_topk_row(idx[b, qq].cpu().numpy(), sc[qq], ids[qq], s.k, f"draft position {qq}")
+    rows = O.entry_kv(np_u8(kv.codes[b]), np_u8(kv.scales[b]), f64(kv.rope[b]), s.d_n, 1.0)
+    o_ref, l_ref = O.attention(f64(q[b]), tp, rows, idx[b].cpu().numpy(), n, f64(win[b]), t0 - s.W + 1, s.W,
+                               s.d ** -0.5)
+    assert_close(f64(out[b]), o_ref, OUT_ATOL, OUT_RTOL, "out")
+    assert_close(lse[b].cpu().numpy(), l_ref, LSE_ATOL, LSE_RTOL, "lse")
