@@ -596,6 +596,7 @@ static csa_status validate_attn(const csa_attn_args* a, int hca) {
   CSA_SUPPORTED((a->d == 512 && a->d_rope == 64) || (a->d == 128 && a->d_rope == 32));
   CSA_SUPPORTED(a->H <= (a->d == 512 ? 64 : 16));
   CSA_REQUIRE(a->g_kv > 0.0f);
+  CSA_REQUIRE(a->out_rope_theta >= 0.0f);        // (false for NaN too)
   if (!hca) CSA_REQUIRE(a->k >= 1);
   if ((long long)a->B * a->Nq == 0) return CSA_OK;
   CSA_REQUIRE(a->q && a->q_pos && a->n_c && a->out);

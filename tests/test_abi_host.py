@@ -98,6 +98,12 @@ def test_invalid_arguments_are_rejected_on_the_host(csa):
     assert lib.hca_dense_attn(ctypes.byref(aa), None, 0, None) == 2
     aa = csa.AttnArgs(ctypes.sizeof(csa.AttnArgs), 1, 1, 64, 512, 64, 4, 16, 8, 0, 128, 1.0, 0.0)
     assert lib.csa_sparse_attn(ctypes.byref(aa), None, 0, None) == 1   # null q / idx
+    for bad in (-1.0, float("nan")):                                   # inverse-RoPE base must be >= 0
+        aa = csa.AttnArgs(ctypes.sizeof(csa.AttnArgs), 0, 1, 64, 512, 64, 4, 16, 8, 0, 128, 1.0, 0.0)
+        aa.out_rope_theta = bad
+        assert lib.csa_sparse_attn(ctypes.byref(aa), None, 0, None) == 1
+        aa.out_rope_theta = 10000.0
+        assert lib.csa_sparse_attn(ctypes.byref(aa), None, 0, None) == 0   # B = 0: nothing to do
     # compress: bad ratio, projection mode with unsupported width
     ca = csa.CompressArgs(ctypes.sizeof(csa.CompressArgs), 1, 8, 64, 64, 0, 0, 0, 0.0)
     assert lib.csa_compress(ctypes.byref(ca), None) == 1
