@@ -1,7 +1,9 @@
 // Attention on the 5th-generation tensor cores (tcgen05, bf16 in, fp32 accumulators in tensor memory), for
-// rows with a 512-wide shared KV head (64-wide RoPE slice): one CTA takes one query (all heads) and one tile
-// of 128 keys of its key list [selected (or, dense, all visible) entries ‖ window rows]; the partials of a
-// query's tiles are merged by attn_merge_kernel.
+// rows with a 512-wide shared KV head (64-wide RoPE slice): one CTA takes one query (all heads) and `tpc`
+// consecutive tiles of 128 keys of its key list [selected (or, dense, all visible) entries ‖ window rows],
+// walked with an online softmax; the partials of a query's CTAs are merged by attn_merge_kernel.  Under
+// the early start (CSA_EARLY_START) the split-0 CTAs come first in the grid and attend over the window
+// tile before waiting for the kernel that writes the selected ids.
 // Sources: "DeepSeek-V4: エージェントが実際に使える100万トークンのコンテキスト", §ハイブリッド注意, Fig. 3 (attention
 // over the top-k compressed entries plus a sliding-window branch under one softmax; the 128x layer attends
 // densely over all visible entries).
@@ -14,8 +16,8 @@
 //                                                 read through an MN-major descriptor (V = K)
 // Tile assembly: Q and window rows arrive by TMA (3-D maps, 128-byte swizzle, rows outside the buffers read
 // as zero); FP4 entries are gathered by id and dequantised by all 8 warps into the same swizzled layout.
-// Partial (O / l in bf16, lse = ln l + m in fp32) per (query, tile) go to the workspace; with one tile the
-// CTA writes the bf16 output and lse itself.
+// Partials (O / l in bf16, lse = ln l + m in fp32) per (query, CTA) go to the workspace; with one CTA per
+// query it writes the bf16 output and lse itself.
 #include <cstring>
 
 #include "csa_common.cuh"
