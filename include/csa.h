@@ -190,10 +190,13 @@ typedef struct csa_index_args {
   uint32_t* hist;          /* optional, split calls only: [B*Nq][4096] score histogram that csa_index_scores
                               adds into (single-query rows: Nq == 1 or cand != NULL) and csa_topk uses to
                               find the k-th score's neighbourhood in one pass, leaving every row it read
-                              zero again.  It must be zero before the first csa_index_scores call; a stale
-                              histogram costs time, not correctness (csa_topk checks its counts against
-                              the scores and falls back to the full selection).  NULL = plain radix
-                              selection */
+                              zero again.  It must be zero before the first csa_index_scores call and
+                              then hold the counts that call added.  Other counts cost time, not
+                              correctness, while the histogram still counts at least k scores of a row
+                              (csa_topk checks the counts at and above the k-th score's bin against the
+                              scores and falls back to the full selection); a row whose histogram counts
+                              fewer than k scores (e.g. one no scoring call filled) is taken to hold only
+                              that many.  NULL = plain radix selection */
   uint32_t flags;          /* CSA_EARLY_START or 0 */
 } csa_index_args;
 
