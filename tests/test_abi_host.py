@@ -65,6 +65,50 @@ def test_ctypes_mirrors_match_the_c_structs(csa, tmp_path):
     assert got == want
 
 
+def test_a_c_program_links_and_calls_the_abi(csa, tmp_path):
+    """The ABI from plain C: a program compiled against include/csa.h and linked with the library gets
+    the documented statuses for host-side argument errors and the workspace queries (no GPU needed)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "csa.h"
+int main(void) {
+  csa_pack_args p; memset(&p, 0, sizeof p);
+  p.struct_size = sizeof p; p.B = 1; p.n = 1; p.d = 40; p.n_max = 1; p.global_scale = 1.0f;
+  int s1 = csa_pack_fp4(&p, NULL);                       /* (d - d_rope) % 32 != 0 */
+  p.struct_size = sizeof p + 4;
+  int s2 = csa_pack_fp4(&p, NULL);                       /* struct_size mismatch */
+  csa_attn_args a; memset(&a, 0, sizeof a);
+  a.struct_size = sizeof a; a.B = 1; a.Nq = 1; a.H = 65; a.d = 512; a.d_rope = 64; a.ratio = 4;
+  a.n_max = 16; a.k = 8; a.window = 128; a.g_kv = 1.0f;
+  int s3 = csa_sparse_attn(&a, NULL, 0, NULL);           /* 65 heads: unsupported */
+  csa_index_args i; memset(&i, 0, sizeof i);
+  i.struct_size = sizeof i; i.B = 2; i.Nq = 1; i.H_I = 8; i.d_I = 128; i.ratio = 4; i.k = 16; i.n_max = 4096;
+  i.g_q = 1.0f; i.g_k = 1.0f;
+  size_t ws0 = csa_index_topk_workspace_size(&i);        /* no tensors: invalid, 0 */
+  static char dummy[256];                                /* never dereferenced by a size query */
+  i.q_I = dummy; i.w = (const float*)dummy; i.k_codes = (const uint8_t*)dummy; i.k_scales = (const uint8_t*)dummy;
+  i.n_c = (const int32_t*)dummy; i.q_pos = (const int64_t*)dummy; i.idx_out = (int32_t*)dummy;
+  size_t ws = ws0 == 0 ? csa_index_topk_workspace_size(&i) : 0;
+  printf("%d %d %d %zu %s %d\n", s1, s2, s3, ws, csa_status_string(s3), csa_version());
+  return 0;
+}
+""")
+    exe = tmp_path / "use"
+    libdir = os.path.dirname(csa.LIB_PATH)
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir,
+                    "-l:" + os.path.basename(csa.LIB_PATH), "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert out[:3] == ["2", "1", "2"] and out[4] == "CSA_ERR_UNSUPPORTED"
+    assert int(out[3]) >= 2 * 4096 * 4 and int(out[5]) == csa.version()
+
+
 def test_invalid_arguments_are_rejected_on_the_host(csa):
     lib = csa._lib
     # pack: d_n not a multiple of 32 -> unsupported; null pointers -> invalid
