@@ -37,7 +37,7 @@ extern "C" {
 typedef enum csa_status {
   CSA_OK = 0,
   CSA_ERR_INVALID = 1,      /* a NULL pointer, a bad size or a struct_size mismatch                    */
-  CSA_ERR_UNSUPPORTED = 2,  /* a valid shape this build has no kernel for (e.g. d_I not 64/128)         */
+  CSA_ERR_UNSUPPORTED = 2,  /* a valid shape the library has no kernel for (e.g. d_I not 64/128)       */
   CSA_ERR_WORKSPACE = 3,    /* ws_bytes smaller than *_workspace_size() for the same arguments          */
   CSA_ERR_CUDA = 4,         /* a kernel launch or CUDA runtime call failed (see csa_last_cuda_error)   */
   CSA_ERR_DEVICE = 5        /* reserved: device-side check failed                                       */
