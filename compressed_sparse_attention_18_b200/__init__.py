@@ -23,7 +23,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 ENTRY_POINTS = ("csa_status_string", "csa_version", "csa_last_cuda_error", "csa_compress", "csa_pack_fp4",
                 "csa_index_topk_workspace_size", "csa_index_topk", "csa_index_scores", "csa_topk_workspace_size",
                 "csa_topk", "csa_attn_workspace_size", "csa_sparse_attn", "hca_dense_attn",
-                "csa_index_topk_noalloc", "csa_device_status")
+                "csa_index_topk_noalloc", "csa_device_status", "csa_check_error_path")
 
 _u32, _i32, _f32, _vp = ctypes.c_uint32, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p
 CSA_EARLY_START = 1   # see csa.h: part of a call's work may start before the step's earlier kernels end
@@ -69,6 +69,8 @@ _lib.csa_version.restype = ctypes.c_int
 _lib.csa_last_cuda_error.restype = ctypes.c_int
 _lib.csa_device_status.restype = ctypes.c_int
 _lib.csa_device_status.argtypes = [_vp]
+_lib.csa_check_error_path.restype = ctypes.c_int
+_lib.csa_check_error_path.argtypes = [_u32, _vp]
 for _name, _st in (("csa_compress", CompressArgs), ("csa_pack_fp4", PackArgs)):
     getattr(_lib, _name).restype = ctypes.c_int
     getattr(_lib, _name).argtypes = [ctypes.POINTER(_st), _vp]
@@ -102,6 +104,12 @@ def version() -> int:
 def device_status(stream=None):
     """Synchronise and raise if a kernel recorded a device-side error (a bounded wait gave up)."""
     _check(_lib.csa_device_status(_stream(stream)), "device status")
+
+
+def check_error_path(polls: int = 1000, stream=None):
+    """Launch the library's error-path self-check: a bounded wait on a barrier nothing arrives on gives
+    up after `polls` polls and records the device error that device_status() then reports."""
+    _check(_lib.csa_check_error_path(int(polls), _stream(stream)), "check_error_path")
 
 
 def _check(status: int, what: str):

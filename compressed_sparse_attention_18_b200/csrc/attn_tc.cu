@@ -674,6 +674,5 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
   return launch_pdl(attn_tc_kernel, dim3((unsigned)(rows * splits)), dim3(TA_THREADS), (size_t)smem, st, qmap, wmap, P);
 }
 
-cudaError_t attn_take_device_error(uint32_t* out) { return take_device_error_here(out); }
 
 }  // namespace csa

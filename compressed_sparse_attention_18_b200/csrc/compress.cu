@@ -434,8 +434,6 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
   }
 }
 
-cudaError_t compress_take_device_error(uint32_t* out) { return take_device_error_here(out); }
-
 }  // namespace csa
 
 using namespace csa;

@@ -13,11 +13,16 @@
 
 namespace csa {
 
-// Device-side error word of this translation unit (bounded waits that gave up); every unit that
-// uses it exposes it to csa_device_status() through take_device_error_here().
+// Device-side error word (a bounded wait gave up).  Without relocatable device code every
+// translation unit that includes this header holds its own copy; each copy's reader is registered at
+// library load (below), and csa_device_status() reads and clears every registered copy.
 static __device__ uint32_t g_csa_device_error = 0;
 
-// Read and clear this unit's device error word (host side).
+typedef cudaError_t (*DeviceErrorReader)(uint32_t* out);
+// Library-wide list of the units' readers (abi.cu).
+void register_device_error_reader(DeviceErrorReader f);
+
+// Read and clear this unit's device error word (host side), OR-ing it into *out.
 static inline cudaError_t take_device_error_here(uint32_t* out) {
   uint32_t v = 0, zero = 0;
   cudaError_t e = cudaMemcpyFromSymbol(&v, g_csa_device_error, sizeof(v));
@@ -25,6 +30,10 @@ static inline cudaError_t take_device_error_here(uint32_t* out) {
   *out |= v;
   return e;
 }
+
+namespace {
+const bool g_device_error_reader_registered = (register_device_error_reader(&take_device_error_here), true);
+}  // namespace
 
 // ----------------------------------------------------------------------------- host-side status
 

@@ -1218,9 +1218,26 @@ static csa_status noalloc_scratch(void** out) {
   return CSA_OK;
 }
 
+// ------------------------------------------------------------------ device error path check
+// One thread waits on an mbarrier that nothing arrives on, with the given poll limit, exactly as the
+// pipelines' bounded waits do; when the wait gives up it records device error 1, as they do.
+__global__ void error_path_check_kernel(uint32_t polls) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  sm100::mbar_init(&bar, 1);
+  sm100::fence_mbar_init();
+  if (!sm100::mbar_wait(&bar, 0, polls)) atomicOr(&g_csa_device_error, 1u);
+}
+
 }  // namespace csa
 
 using namespace csa;
+
+extern "C" csa_status csa_check_error_path(uint32_t polls, void* stream) {
+  CSA_REQUIRE(polls >= 1 && polls <= (1u << 20));
+  error_path_check_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(polls);
+  return launch_status();
+}
 
 extern "C" csa_status csa_index_topk_noalloc(const csa_index_args* a, void* stream) {
   csa_status v = validate_index(a, true);

@@ -364,20 +364,4 @@ csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, u
   return launch_pdl(index_score_tc_kernel, dim3(per_row, a->B), dim3(TC_THREADS), smem, st, map, P);
 }
 
-cudaError_t compress_take_device_error(uint32_t* out);   // compress.cu
-cudaError_t attn_take_device_error(uint32_t* out);       // attn_tc.cu
-
 }  // namespace csa
-
-extern "C" csa_status csa_device_status(void* stream) {
-  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
-  uint32_t v = 0;
-  if (e == cudaSuccess) e = csa::take_device_error_here(&v);
-  if (e == cudaSuccess) e = csa::compress_take_device_error(&v);
-  if (e == cudaSuccess) e = csa::attn_take_device_error(&v);
-  if (e != cudaSuccess) {
-    csa::set_last_cuda_error(e);
-    return CSA_ERR_CUDA;
-  }
-  return v ? CSA_ERR_DEVICE : CSA_OK;
-}

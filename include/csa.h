@@ -17,7 +17,11 @@
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy default
  *     stream).  Argument errors are detected on the host before any launch and returned as
  *     CSA_ERR_INVALID / CSA_ERR_UNSUPPORTED / CSA_ERR_WORKSPACE; nothing is launched then.
- *     A launch failure returns CSA_ERR_CUDA.  No exception crosses the ABI; no global mutable state.
+ *     A launch failure returns CSA_ERR_CUDA.  No exception crosses the ABI.
+ *   - Global mutable state: two device-side items only.  (1) The device error word that bounded waits
+ *     set when they give up (one per device, read and cleared by csa_device_status).  (2) The static
+ *     scratch array of csa_index_topk_noalloc (CSA_NOALLOC_SCRATCH_BYTES per device).  Host-side
+ *     caches (tensor-map encoder, kernel attributes set once per device) hold no per-call data.
  *   - Arguments are passed as structs whose first field `struct_size` must equal sizeof(struct).
  *   - FP4 formats (E2M1 codes, one E4M3 scale per 32 elements, per-tensor fp32 global scale g):
  *       codes[n][d_n/2] u8 (element 2j in the low nibble of byte j), scales[n][S_pad] u8
@@ -40,7 +44,7 @@ typedef enum csa_status {
   CSA_ERR_UNSUPPORTED = 2,  /* a valid shape the library has no kernel for (e.g. d_I not 64/128)       */
   CSA_ERR_WORKSPACE = 3,    /* ws_bytes smaller than *_workspace_size() for the same arguments          */
   CSA_ERR_CUDA = 4,         /* a kernel launch or CUDA runtime call failed (see csa_last_cuda_error)   */
-  CSA_ERR_DEVICE = 5        /* reserved: device-side check failed                                       */
+  CSA_ERR_DEVICE = 5        /* a device-side bounded wait gave up (csa_device_status)                  */
 } csa_status;
 
 /* Human-readable name of a status code (static string). */
@@ -49,10 +53,17 @@ const char* csa_status_string(int status);
 int csa_version(void);
 /* The cudaError_t of the last CSA_ERR_CUDA returned on the calling host thread (0 if none). */
 int csa_last_cuda_error(void);
-/* Synchronises `stream`, then reports and clears the device-side error word of the current device:
+/* Synchronises `stream`, then reports and clears the device-side error word of the current device
+ * (every kernel of the library writes it):
  * CSA_ERR_DEVICE if a kernel gave up a bounded wait (a pipeline stalled; its outputs are incomplete),
  * CSA_OK otherwise, CSA_ERR_CUDA if the synchronisation itself failed. */
 csa_status csa_device_status(void* stream);
+/* Exercises the error path above without a fault: launches one thread that waits, `polls` times with
+ * a short sleep between polls (1 <= polls <= 2^20, i.e. well under a second), on a barrier nothing
+ * arrives on, then records device error 1 exactly as a stalled pipeline does.  The next
+ * csa_device_status returns CSA_ERR_DEVICE (and clears the word).  No output; nothing else changes.
+ * A library self-check, not part of the layer: the pages have no counterpart. */
+csa_status csa_check_error_path(uint32_t polls, void* stream);
 
 /* Overlap inside a decode step.  Every kernel of this library is launched with programmatic
  * dependent launch: it may become resident while the kernel before it on the stream still runs, and it

@@ -299,13 +299,6 @@ def compress(x=None, W_kv=None, W_g=None, C=None, Z=None, *, b_pos, r, d_rope=0,
 #     one score per compressed block per query)
 # --------------------------------------------------------------------------------------------
 
-def visible_mask(q_pos, n_c: int, r: int, n_keys: int):
-    """Key i visible to the query at position t iff i < n_c and r i + r - 1 <= t.  -> bool [Nq, n_keys]"""
-    i = np.arange(n_keys)
-    t = np.asarray(q_pos, np.int64)[:, None]
-    return (i[None, :] < n_c) & (r * i[None, :] + r - 1 <= t)
-
-
 def index_scores(qI, w, g_q, k_codes, k_scales, g_k, q_pos, n_c: int, r: int, keys=None):
     """Scores s(t, i) for one sequence.
 

@@ -29,9 +29,13 @@ def assert_close(got, ref, atol, rtol, what=""):
     ref = np.asarray(ref, np.float64)
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
     both_inf = np.isinf(got) & np.isinf(ref) & (np.sign(got) == np.sign(ref))
+    both_nan = np.isnan(got) & np.isnan(ref)
     err = np.abs(got - ref)
-    err[both_inf] = 0.0
-    bad = err > atol + rtol * np.abs(np.where(both_inf, 0.0, ref))
+    err[both_inf | both_nan] = 0.0
+    bad = err > atol + rtol * np.abs(np.where(both_inf | both_nan, 0.0, ref))
+    # a NaN (or an infinity) on one side only is always a mismatch: NaN compares False above
+    bad |= np.isnan(got) != np.isnan(ref)
+    bad |= (np.isinf(got) | np.isinf(ref)) & ~both_inf
     if np.any(bad):
         i = np.argwhere(bad)[0]
         raise AssertionError(f"{what}: {bad.sum()} / {bad.size} elements out of tolerance; first at {tuple(i)}: "
@@ -51,7 +55,10 @@ def check_topk_row(gpu_idx, ref_scores, ref_ids, k, what=""):
     ref_set = set(ids[order[:k_eff]].tolist())
     got = gpu_idx[gpu_idx >= 0]
     assert len(got) == k_eff, f"{what}: {len(got)} selected, expected {k_eff}"
-    assert np.all(gpu_idx[k_eff:] == -1) or True
+    # slot order is unspecified: every slot is a selected id or the padding -1, and exactly k - k_eff
+    # slots (of the k written) are padding
+    assert np.all((gpu_idx >= 0) | (gpu_idx == -1)), f"{what}: slots other than ids and -1"
+    assert int(np.sum(gpu_idx == -1)) == len(gpu_idx) - k_eff, f"{what}: padding count"
     got_set = set(got.tolist())
     assert len(got_set) == len(got), f"{what}: duplicate ids"
     if got_set == ref_set:

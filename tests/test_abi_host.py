@@ -148,6 +148,9 @@ def test_invalid_arguments_are_rejected_on_the_host(csa):
         assert lib.csa_sparse_attn(ctypes.byref(aa), None, 0, None) == 1
         aa.out_rope_theta = 10000.0
         assert lib.csa_sparse_attn(ctypes.byref(aa), None, 0, None) == 0   # B = 0: nothing to do
+    # error-path self-check: the poll count is checked before any launch
+    assert lib.csa_check_error_path(0, None) == 1
+    assert lib.csa_check_error_path((1 << 20) + 1, None) == 1
     # compress: bad ratio, projection mode with unsupported width
     ca = csa.CompressArgs(ctypes.sizeof(csa.CompressArgs), 1, 8, 64, 64, 0, 0, 0, 0.0)
     assert lib.csa_compress(ctypes.byref(ca), None) == 1

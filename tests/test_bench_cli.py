@@ -3,6 +3,8 @@ import importlib.util
 import os
 import sys
 
+import pytest
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -58,3 +60,41 @@ def test_decode_flop_curve():
     f4, f1m = b.decode_flops(4096, s, "full")["total"], b.decode_flops(1 << 20, s, "full")["total"]
     assert abs((f1m - f4) - (0.25 * 2048 + 16) * ((1 << 18) - 1024)) < 1e-3 * f1m
     assert b.decode_flops(1 << 20, s, "hca")["parts"]["attention"] == 4 * 64 * 512 * (8192 + 128)
+
+
+@pytest.mark.parametrize("steps,warmup", [(20, 5), (16, 8), (3, 3), (20000, 64)])
+def test_no_graph_capture_inside_the_timed_region(steps, warmup):
+    """bench.py's timed loop only replays graphs: every capture happens in prepare(), before t0.  With
+    the driver's --steps 20 --warmup 5 the loop needs the 8-step and the 4-step graphs, which a warm-up
+    of 5 steps alone would not have built."""
+    import contextlib
+
+    bench = _load()
+    log = []
+
+    class FakeGraph:
+        def replay(self):
+            log.append("replay")
+
+    def capture(g):
+        log.append("capture")
+        return contextlib.nullcontext()
+
+    sg = bench.StepGraphs(lambda n, marks: log.append(("launch", n, marks)), lambda flag: None, None, bench.LAYERS,
+                          graph_cls=FakeGraph, capture=capture)
+    # the same calls, in the same order, as run_ours before its timing events
+    sg.prepare(max(warmup, 3), steps)
+    sg.prepare(bench.LAYERS, with_marks=True)
+    sg.freeze()
+    sg.run(max(warmup, 3))
+    log.clear()                                   # t0.record(stream)
+    sg.run(steps)                                 # the timed region
+    assert "capture" not in log and not any(isinstance(e, tuple) for e in log)
+    assert log.count("replay") == steps // bench.LAYERS + (1 if steps % bench.LAYERS else 0)
+    log.clear()                                   # the stage replay after t1
+    sg.run(bench.LAYERS, with_marks=True)
+    assert log == ["replay"]
+    prepared = {n for n, m in sg.graphs if not m}
+    missing = next(n for n in range(1, bench.LAYERS) if n not in prepared)
+    with pytest.raises(RuntimeError):             # an unprepared count is refused once frozen
+        sg.run(missing)

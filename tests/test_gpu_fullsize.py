@@ -7,7 +7,8 @@ import torch
 
 from csa_workloads import CFG2, CFG4_HCA, CFG4_REUSE, CFG5, decode_inputs, gen, normal
 from oracle import csa_oracle as O
-from tests.cmp_utils import (LSE_ATOL, LSE_RTOL, OUT_ATOL, OUT_RTOL, assert_close, check_topk_row, f64, np_u8)
+from tests.cmp_utils import (LSE_ATOL, LSE_RTOL, OUT_ATOL, OUT_RTOL, SCORE_RTOL, assert_close, check_topk_row, f64,
+                             np_u8)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -67,6 +68,11 @@ def test_decode_cfg2_full_size(cuda_lib):
         assert np.array_equal(np_u8(layer.kv.scales[b, : s.n_c - 1]), hs)
         # index + top-k on the same cache bytes
         sc, ids, _, _ = _seq_oracle_index(layer, inp, b, s)
+        # the whole score row the top-k read, element by element (visible keys = all n_c entries)
+        n_c = int(layer.n_c[b])
+        rowmax = float(np.max(np.abs(sc[0][:n_c])))
+        assert np.all(np.isfinite(sc[0][:n_c]))
+        assert_close(gpu_scores[b, :n_c], sc[0][:n_c], SCORE_RTOL * rowmax, SCORE_RTOL, f"cfg2 score row b={b}")
         check_topk_row(idx[b, 0].cpu().numpy(), sc[0], ids[0], s.k, f"cfg2 b={b}")
         # attention on the GPU's selection (same upstream bytes)
         rows = O.entry_kv(np_u8(layer.kv.codes[b]), np_u8(layer.kv.scales[b]), f64(layer.kv.rope[b]), s.d_n, 1.0)

@@ -24,17 +24,27 @@ def _args(csa, q_I, w, kc, n_c, q_pos, k, idx, sc):
                          None, 0, 0, 8, None, idx.data_ptr(), sc.data_ptr())
 
 
-def test_noalloc_matches_workspace_entry_point(cuda_lib):
+# (B, cache rows, n_c per sequence, last visible group per sequence): rows of one 32768-score segment
+# (the single-CTA top-k), and a 70000-score row that the multi-segment top-k splits over several CTAs
+# (its per-row state, candidate and tournament buffers all live in the shared static array)
+CASES = [(4, 20000, [20000, 19993, 5000, 300], [19999, 19999, 4000, 299]),
+         (1, 70000, [70000], [69999])]
+
+
+@pytest.mark.parametrize("B,n,ncs,groups", CASES, ids=["one_segment", "multi_segment_70000"])
+def test_noalloc_matches_workspace_entry_point(cuda_lib, B, n, ncs, groups):
     csa = cuda_lib
     lib = csa._lib
     torch.cuda.set_device(0)
     g = torch.Generator(device=DEV).manual_seed(21)
-    B, n, d_I, H_I, k = 4, 20000, 128, 8, 256
+    d_I, H_I, k = 128, 8, 256
     kI = torch.randn((B, n, d_I), generator=g, device=DEV).to(torch.bfloat16)
     kc = csa.PackedCache(B, n, d_I, 0, DEV)
     csa.pack_fp4(kI, kc)
-    n_c = torch.tensor([n, n - 7, 5000, 300], dtype=torch.int32, device=DEV)
-    q_pos = torch.tensor([[4 * n - 1], [4 * n - 1], [4 * 4000 + 2], [4 * 300 - 1]], dtype=torch.int64, device=DEV)
+    n_c = torch.tensor(ncs, dtype=torch.int32, device=DEV)
+    q_pos = torch.tensor([[4 * gi + 3] for gi in groups], dtype=torch.int64, device=DEV)
+    if B == 4:
+        q_pos[2, 0] = 4 * 4000 + 2                     # a query whose last group is still incomplete
     stream = torch.cuda.current_stream().cuda_stream
     for call in range(2):
         q_I = torch.randn((B, 1, H_I, d_I), generator=g, device=DEV).to(torch.bfloat16)
@@ -59,7 +69,8 @@ def test_noalloc_matches_workspace_entry_point(cuda_lib):
             rs = dict(zip(r.tolist(), sc_ref[b, 0].cpu().numpy().tolist()))
             os_ = dict(zip(o.tolist(), sc[b, 0].cpu().numpy().tolist()))
             assert all(rs[i] == os_[i] or (np.isneginf(rs[i]) and np.isneginf(os_[i])) for i in rs)
-        assert (idx[3, 0] >= 0).sum() == min(k, 300)
+        if B == 4:
+            assert (idx[3, 0] >= 0).sum() == min(k, 300)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_lib):
