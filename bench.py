@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--spec", action="store_true",
                    help="multi-query decode with speculative positions: 5 draft positions per sequence, "
                         "B=32 at 128K context (index + top-k + attention), one JSON line")
+    p.add_argument("--prefill", action="store_true",
+                   help="chunked causal prefill of one 32768-token sequence (4096-token chunks), one JSON line")
     p.add_argument("--flops", action="store_true",
                    help="analytic precision-weighted decode FLOPs per token from 4K to 1M context next to the "
                         "measured decode step at each context, one JSON line each")
@@ -553,11 +555,15 @@ def _event_ms(fn, reps, warm=3):
     return a.elapsed_time(b) / reps
 
 
-def _tensor_peak():
+def _tensor_peak(sustained=False):
+    """bf16 dense peak: the burst figure for a kernel timed alone, the sustained one inside a long step."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
-        return float(json.load(open(path))["bf16_tflops"]), "measured"
-    return 1590.0, "fallback"
+        d = json.load(open(path))
+        if sustained and "bf16_tflops_sustained" in d:
+            return float(d["bf16_tflops_sustained"]), "measured"
+        return float(d["bf16_tflops"]), "measured"
+    return (1400.0 if sustained else 1590.0), "fallback"
 
 
 def run_rows(args):
@@ -812,6 +818,164 @@ def run_spec(args):
                               "4 cache states rotated (inputs larger than L2)"}), flush=True)
 
 
+def prefill_work(s):
+    """Algorithmic work of the whole chunked prefill of one sequence (s.T tokens): the compressor's two
+    projections (bf16 FLOPs), the causal indexer's FP4 products (query t scores (t+1) // r entries), and
+    attention over min(k, visible) entries plus min(W, t+1) window rows per query and head (two bf16
+    products of d per key)."""
+    t = torch.arange(s.T, dtype=torch.float64)
+    n_vis = torch.div(t + 1, s.r, rounding_mode="floor")
+    proj = 2.0 * 2 * s.T * s.d_m * s.d
+    index = float(n_vis.sum()) * s.H_I * s.d_I * 2
+    keys = torch.clamp(n_vis, max=s.k) + torch.clamp(t + 1, max=s.W)
+    attn = float(keys.sum()) * s.H * s.d * 4
+    return {"projection": proj, "index": index, "attention": attn}
+
+
+def run_prefill(args):
+    """Chunked causal prefill of one 32768-token sequence in 4096-token chunks (d_m = 4096, 64 heads x
+    512, indexer 8 x 128 FP4, top-512, window 128).  Per chunk: the compressor (projection GEMM on the
+    tensor cores, gated pooling, FP4 append of the chunk's 1024 entries and their indexer keys), the
+    multi-query indexer over every entry so far with the causal mask, top-512 per query, attention over
+    the selected entries plus the window.  One step = the 8 chunks, replayed from one CUDA graph; inputs
+    (x 256 MB, q 2 GB) are larger than L2.  One JSON line."""
+    import compressed_sparse_attention_18_b200 as csa
+    from csa_workloads import CFG3, gen, normal
+    from oracle import csa_oracle as O
+    from threadpoolctl import threadpool_limits
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    s = CFG3
+    Lc = s.extra["chunk"]
+    nch, n = s.T // Lc, s.n_c
+    epc = Lc // s.r
+    G = gen(40, dev)
+    x = normal((nch, Lc, s.d_m), 1.0, G, dev)
+    W_kv = normal((s.d_m, s.d), s.d_m ** -0.5, G, dev)
+    W_g = normal((s.d_m, s.d), s.d_m ** -0.5, G, dev)
+    b_pos = normal((s.r, s.d), 0.1, G, dev, torch.float32)
+    W_IK = normal((s.d, s.d_I), s.d ** -0.5, G, dev)
+    q = normal((nch, Lc, s.H, s.d), 1.0, G, dev)
+    q_I = normal((nch, Lc, s.H_I, s.d_I), 1.0, G, dev)
+    w = normal((nch, Lc, s.H_I), s.H_I ** -0.5, G, dev, torch.float32)
+    C = torch.zeros((1, s.T, s.d), dtype=torch.bfloat16, device=dev)     # every token's C: the window KV
+    Z = torch.empty((1, Lc, s.d), dtype=torch.bfloat16, device=dev)
+    c_out = torch.empty((1, epc, s.d), dtype=torch.bfloat16, device=dev)
+    kI_out = torch.empty((1, epc, s.d_I), dtype=torch.bfloat16, device=dev)
+    kv = csa.PackedCache(1, n, s.d, s.d_r, dev)
+    ki = csa.PackedCache(1, n, s.d_I, 0, dev)
+    row0 = [torch.tensor([epc * c], dtype=torch.int32, device=dev) for c in range(nch)]
+    pos0 = [torch.tensor([Lc * c], dtype=torch.int64, device=dev) for c in range(nch)]
+    n_c = [torch.tensor([epc * (c + 1)], dtype=torch.int32, device=dev) for c in range(nch)]
+    q_pos = [(Lc * c + torch.arange(Lc, dtype=torch.int64, device=dev)).view(1, Lc) for c in range(nch)]
+    win_pos0 = torch.zeros((1,), dtype=torch.int64, device=dev)
+    idx = torch.empty((1, Lc, s.k), dtype=torch.int32, device=dev)
+    out = torch.empty((1, Lc, s.H, s.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((1, Lc, s.H), dtype=torch.float32, device=dev)
+    ws_i = torch.empty(max(csa.index_topk_workspace_size(q_I[:1], w[:1], ki, n_c[-1], q_pos[-1], ratio=s.r, k=s.k), 1),
+                       dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(max(max(csa.attn_workspace_size(q[c:c + 1], q_pos[c], kv, n_c[c], idx, C, win_pos0, ratio=s.r,
+                                                       window=s.W) for c in range(nch)), 1),
+                       dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize()
+
+    def chunk(c, marks=None):
+        def mark(i):
+            if marks is not None:
+                marks[i].record(stream)
+        mark(0)
+        csa.compress(x=x[c:c + 1], W_kv=W_kv, W_g=W_g, b_pos=b_pos, ratio=s.r, d_rope=s.d_r, rope_theta=10000.0,
+                     pos0=pos0[c], W_IK=W_IK, C=C[:, Lc * c:Lc * (c + 1)], Z=Z, c_out=c_out, kI_out=kI_out,
+                     kv_cache=kv, ki_cache=ki, row0=row0[c], stream=stream)
+        mark(1)
+        csa.index_topk(q_I[c:c + 1], w[c:c + 1], ki, n_c[c], q_pos[c], ratio=s.r, k=s.k, idx_out=idx, ws=ws_i,
+                       stream=stream)
+        mark(2)
+        csa.sparse_attn(q[c:c + 1], q_pos[c], kv, n_c[c], idx, C, win_pos0, ratio=s.r, window=s.W, out=out, lse=lse,
+                        ws=ws_a, stream=stream)
+        mark(3)
+
+    def prefill(marks=None):
+        for c in range(nch):
+            chunk(c, marks[c] if marks is not None else None)
+
+    with torch.cuda.stream(stream):
+        prefill()                                       # eager warm-up (kernel attributes set)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        prefill()
+    steps, warm = max(args.steps if args.steps < 1000 else 10, 1), max(args.warmup if args.warmup < 1000 else 3, 3)
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            g.replay()
+    stream.synchronize()
+    clk = ClockSampler(0)
+    clk.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            g.replay()
+    e1.record(stream)
+    stream.synchronize()
+    clocks = clk.stop()
+    ms = e0.elapsed_time(e1) / steps
+    # per-stage times: eager chunks with an event at every stage boundary (serialised stages)
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nch)]
+    with torch.cuda.stream(stream):
+        prefill(marks)
+    stream.synchronize()
+    stage = {name: sum(marks[c][i].elapsed_time(marks[c][i + 1]) for c in range(nch))
+             for i, name in enumerate(("compress", "index_topk", "attention"))}
+    work = prefill_work(s)
+    tfl, tkind = _tensor_peak()
+    tfl_s = _tensor_peak(sustained=True)[0]
+
+    def tf(flops, ms_):
+        return flops / (ms_ / 1e3) / 1e12
+
+    # oracle on a bounded sample: the projection of 4 tokens, and index + top-k + attention of 2 queries
+    # of the last chunk (over all 8192 entries), 1 thread
+    f64 = lambda t_: t_.double().cpu().numpy()  # noqa: E731
+    codes, scales = kv.codes[0].cpu().numpy(), kv.scales[0].cpu().numpy()
+    kcodes, kscales = ki.codes[0].cpu().numpy(), ki.scales[0].cpu().numpy()
+    rows = O.entry_kv(codes, scales, f64(kv.rope[0]), s.d_n, 1.0)
+    win = f64(C[0, s.T - Lc - s.W:])
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        O.project(f64(x[-1, :4]), f64(W_kv))
+        O.project(f64(x[-1, :4]), f64(W_g))
+        for qq in (Lc - 2, Lc - 1):
+            t = s.T - Lc + qq
+            sc, ids = O.index_scores(f64(q_I[-1, qq])[None], f64(w[-1, qq])[None], 1.0, kcodes, kscales, 1.0, [t], n,
+                                     s.r)
+            sel, _ = O.topk(sc, ids, s.k)
+            O.attention(f64(q[-1, qq])[None], [t], rows, sel, n, win, s.T - Lc - s.W, s.W, s.d ** -0.5)
+        el = time.perf_counter() - t0
+    line = {"row": "cfg3 chunked causal prefill", "workload": s.name,
+            "config": {"B": 1, "tokens": s.T, "chunk": Lc, "d_model": s.d_m, "heads": s.H, "head_dim": s.d,
+                       "indexer": f"{s.H_I}x{s.d_I} fp4", "top_k": s.k, "window": s.W,
+                       "l2": "inputs larger than L2 (x 256 MB, q 2 GB)", "cuda_graph": True},
+            "steps": steps, "warmup": warm, "ms_per_step": ms, "value": s.T / (ms / 1e3), "unit": "tokens/s",
+            "clocks": clocks,
+            "stages_ms": stage, "stages_plan": "eager chunks with an event at every stage boundary",
+            "tflops": {"projection": tf(work["projection"], stage["compress"]),
+                       "index_fp4": tf(work["index"], stage["index_topk"]),
+                       "attention": tf(work["attention"], stage["attention"])},
+            "algorithmic_flops": work,
+            "roofline": {"bound": "tensor", "kernel": "attention stage (attn_tc_kernel)",
+                         "achieved": tf(work["attention"], stage["attention"]), "peak": tfl_s,
+                         "peak_kind": tkind + " sustained", "unit": "TFLOP/s",
+                         "frac": tf(work["attention"], stage["attention"]) / tfl_s},
+            "cpu_baseline": {"value": 2 / el, "unit": "query tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": "projection of 4 tokens + index/top-k/attention of 2 queries of the last "
+                                       "chunk, numpy fp64, 1 thread"}}
+    print(json.dumps(line), flush=True)
+
+
 def run_profile(args):
     """One layer state, `--steps` eager decode steps: the small case ncu captures run on."""
     from compressed_sparse_attention_18_b200.layer import CSADecodeLayer, LayerShape
@@ -842,6 +1006,9 @@ def main():
         return
     if args.spec:
         run_spec(args)
+        return
+    if args.prefill:
+        run_prefill(args)
         return
     rank, world = dist_init(args.gpus)
     try:

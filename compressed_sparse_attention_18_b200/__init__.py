@@ -23,15 +23,21 @@ _lib = ctypes.CDLL(LIB_PATH)
 ENTRY_POINTS = ("csa_status_string", "csa_version", "csa_last_cuda_error", "csa_compress", "csa_pack_fp4",
                 "csa_index_topk_workspace_size", "csa_index_topk", "csa_index_scores", "csa_topk_workspace_size",
                 "csa_topk", "csa_attn_workspace_size", "csa_sparse_attn", "hca_dense_attn",
-                "csa_index_topk_noalloc", "csa_device_status", "csa_check_error_path")
+                "csa_index_topk_noalloc", "csa_device_status", "csa_check_error_path",
+                "csa_pack_fp8_window")
+# (PagedCache: a paged pool + block table, accepted wherever a PackedCache is)
 
 _u32, _i32, _f32, _vp = ctypes.c_uint32, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p
 CSA_EARLY_START = 1   # see csa.h: part of a call's work may start before the step's earlier kernels end
 
 
+class PageMap(ctypes.Structure):
+    _fields_ = [("table", _vp), ("page_size", _i32), ("width", _i32), ("n_pages", _i32)]
+
+
 class Fp4Cache(ctypes.Structure):
     _fields_ = [("codes", _vp), ("scales", _vp), ("rope", _vp), ("row0", _vp), ("n_max", _i32),
-                ("global_scale", _f32)]
+                ("global_scale", _f32), ("pages", PageMap)]
 
 
 class CompressArgs(ctypes.Structure):
@@ -44,7 +50,7 @@ class CompressArgs(ctypes.Structure):
 class PackArgs(ctypes.Structure):
     _fields_ = [("struct_size", _u32), ("B", _i32), ("n", _i32), ("d", _i32), ("d_rope", _i32),
                 ("n_max", _i32), ("global_scale", _f32), ("src", _vp), ("row0", _vp), ("codes", _vp),
-                ("scales", _vp), ("rope", _vp)]
+                ("scales", _vp), ("rope", _vp), ("pages", PageMap)]
 
 
 class IndexArgs(ctypes.Structure):
@@ -52,7 +58,7 @@ class IndexArgs(ctypes.Structure):
                 ("ratio", _i32), ("k", _i32), ("n_max", _i32), ("g_q", _f32), ("g_k", _f32), ("q_I", _vp),
                 ("w", _vp), ("k_codes", _vp), ("k_scales", _vp), ("n_c", _vp), ("q_pos", _vp),
                 ("cand", _vp), ("n_cand", _i32), ("pool_blocks", _i32), ("pool_block_size", _i32),
-                ("pool_out", _vp), ("idx_out", _vp), ("scores_out", _vp), ("hist", _vp), ("flags", _u32)]
+                ("pool_out", _vp), ("idx_out", _vp), ("scores_out", _vp), ("hist", _vp), ("flags", _u32), ("k_pages", PageMap)]
 
 
 class AttnArgs(ctypes.Structure):
@@ -60,7 +66,13 @@ class AttnArgs(ctypes.Structure):
                 ("ratio", _i32), ("n_max", _i32), ("k", _i32), ("Wn", _i32), ("window", _i32),
                 ("g_kv", _f32), ("softmax_scale", _f32), ("q", _vp), ("q_pos", _vp), ("kv_codes", _vp),
                 ("kv_scales", _vp), ("kv_rope", _vp), ("n_c", _vp), ("idx", _vp), ("win_kv", _vp),
-                ("win_pos0", _vp), ("out", _vp), ("lse", _vp), ("flags", _u32), ("out_rope_theta", _f32)]
+                ("win_pos0", _vp), ("out", _vp), ("lse", _vp), ("flags", _u32), ("out_rope_theta", _f32),
+                ("win_format", _u32), ("win_codes", _vp), ("win_scales", _vp), ("win_rope", _vp), ("kv_pages", PageMap)]
+
+
+class Fp8WindowArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("B", _i32), ("n", _i32), ("d", _i32), ("d_rope", _i32), ("Wn", _i32),
+                ("src", _vp), ("row0", _vp), ("codes", _vp), ("scales", _vp), ("rope", _vp)]
 
 
 _lib.csa_status_string.restype = ctypes.c_char_p
@@ -71,7 +83,7 @@ _lib.csa_device_status.restype = ctypes.c_int
 _lib.csa_device_status.argtypes = [_vp]
 _lib.csa_check_error_path.restype = ctypes.c_int
 _lib.csa_check_error_path.argtypes = [_u32, _vp]
-for _name, _st in (("csa_compress", CompressArgs), ("csa_pack_fp4", PackArgs)):
+for _name, _st in (("csa_compress", CompressArgs), ("csa_pack_fp4", PackArgs), ("csa_pack_fp8_window", Fp8WindowArgs)):
     getattr(_lib, _name).restype = ctypes.c_int
     getattr(_lib, _name).argtypes = [ctypes.POINTER(_st), _vp]
 _lib.csa_index_topk_workspace_size.restype = ctypes.c_size_t
@@ -145,11 +157,36 @@ def _ws(nbytes: int, device, ws=None):
 
 # ------------------------------------------------------------------------------------------- API
 
+def _page_map(cache):
+    """The cache's csa_page_map (a NULL table for the contiguous layout)."""
+    t = getattr(cache, "table", None)
+    if t is None:
+        return PageMap()
+    return PageMap(_ptr(t), cache.page_size, t.shape[-1], cache.n_pages)
+
+
+class PagedCache:
+    """A paged FP4 cache: pools of n_pages pages x page_size entries (codes u8, scales u8, rope bf16) and a
+    block table [B, width] int32; entry i of sequence b lives in slot i % page_size of page
+    table[b, i // page_size] (csa_page_map).  Used wherever a PackedCache is."""
+
+    def __init__(self, B, n_max, d, d_rope, device, page_size, n_pages, table, global_scale=1.0):
+        d_n = d - d_rope
+        s_pad = (d_n // 32 + 3) // 4 * 4
+        rows = n_pages * page_size
+        self.B, self.n_max, self.d, self.d_rope, self.g = B, n_max, d, d_rope, float(global_scale)
+        self.page_size, self.n_pages = page_size, n_pages
+        self.table = table.to(device=device, dtype=torch.int32).contiguous()
+        self.codes = torch.zeros((rows, d_n // 2), dtype=torch.uint8, device=device)
+        self.scales = torch.zeros((rows, s_pad), dtype=torch.uint8, device=device)
+        self.rope = torch.zeros((rows, d_rope if d_rope else 0), dtype=torch.bfloat16, device=device)
+
+
 def _fp4_target(cache, row0):
     if cache is None:
         return Fp4Cache()
     return Fp4Cache(_ptr(cache.codes), _ptr(cache.scales), _ptr(cache.rope) if cache.d_rope else None, _ptr(row0),
-                    cache.n_max, cache.g)
+                    cache.n_max, cache.g, _page_map(cache))
 
 
 def compress(*, b_pos, ratio, d_rope=0, rope_theta=0.0, pos0=None, x=None, W_kv=None, W_g=None, C=None, Z=None,
@@ -197,7 +234,8 @@ def pack_fp4(src, cache: PackedCache, row0=None, stream=None):
     """Pack src [B, n, d] bf16 into cache rows row0[b] + j (row0 int32 [B] or None = 0)."""
     B, n, d = src.shape
     a = PackArgs(ctypes.sizeof(PackArgs), B, n, d, cache.d_rope, cache.n_max, cache.g, _ptr(src), _ptr(row0),
-                 _ptr(cache.codes), _ptr(cache.scales), _ptr(cache.rope) if cache.d_rope else None)
+                 _ptr(cache.codes), _ptr(cache.scales), _ptr(cache.rope) if cache.d_rope else None,
+                 _page_map(cache))
     _check(_lib.csa_pack_fp4(ctypes.byref(a), _stream(stream)), "csa_pack_fp4")
     return cache
 
@@ -205,10 +243,12 @@ def pack_fp4(src, cache: PackedCache, row0=None, stream=None):
 def _index_args(q_I, w, kcache: PackedCache, n_c, q_pos, ratio, k, g_q, cand, pool_blocks, pool_block_size,
                 pool_out, idx_out, scores_out):
     B, Nq, H_I, d_I = q_I.shape
-    return IndexArgs(ctypes.sizeof(IndexArgs), B, Nq, H_I, d_I, ratio, k, kcache.n_max, g_q, kcache.g, _ptr(q_I),
-                     _ptr(w), _ptr(kcache.codes), _ptr(kcache.scales), _ptr(n_c), _ptr(q_pos), _ptr(cand),
-                     cand.shape[-1] if cand is not None else 0, pool_blocks, pool_block_size, _ptr(pool_out),
-                     _ptr(idx_out), _ptr(scores_out))
+    a = IndexArgs(ctypes.sizeof(IndexArgs), B, Nq, H_I, d_I, ratio, k, kcache.n_max, g_q, kcache.g, _ptr(q_I),
+                  _ptr(w), _ptr(kcache.codes), _ptr(kcache.scales), _ptr(n_c), _ptr(q_pos), _ptr(cand),
+                  cand.shape[-1] if cand is not None else 0, pool_blocks, pool_block_size, _ptr(pool_out),
+                  _ptr(idx_out), _ptr(scores_out))
+    a.k_pages = _page_map(kcache)
+    return a
 
 
 def index_topk(q_I, w, kcache: PackedCache, n_c, q_pos, *, ratio, k, g_q=1.0, cand=None, pool_blocks=0,
@@ -283,13 +323,46 @@ def index_topk_workspace_size(q_I, w, kcache, n_c, q_pos, *, ratio, k, g_q=1.0, 
     return _lib.csa_index_topk_workspace_size(ctypes.byref(a))
 
 
+class Fp8Window:
+    """FP8 sliding-window rows [B, Wn, d] as csa_pack_fp8_window writes them: E4M3 codes [B, Wn, d_n],
+    fp32 scales per 64 channels [B, Wn, round_up(d_n / 64, 4)], RoPE channels bf16 [B, Wn, d_rope]."""
+
+    def __init__(self, B, Wn, d, d_rope, device):
+        d_n = d - d_rope
+        self.B, self.Wn, self.d, self.d_rope = B, Wn, d, d_rope
+        self.codes = torch.zeros((B, Wn, d_n), dtype=torch.uint8, device=device)
+        self.scales = torch.zeros((B, Wn, (d_n // 64 + 3) // 4 * 4), dtype=torch.float32, device=device)
+        self.rope = torch.zeros((B, Wn, d_rope), dtype=torch.bfloat16, device=device)
+
+    @property
+    def shape(self):
+        return (self.B, self.Wn, self.d)
+
+
+def pack_fp8_window(src, win: Fp8Window, row0=None, stream=None):
+    """FP8-pack bf16 window rows src [B, n, d] into win rows row0[b] + j (csa_pack_fp8_window)."""
+    B, n, d = src.shape
+    a = Fp8WindowArgs(ctypes.sizeof(Fp8WindowArgs), B, n, d, win.d_rope, win.Wn, _ptr(src), _ptr(row0),
+                      _ptr(win.codes), _ptr(win.scales), _ptr(win.rope) if win.d_rope else None)
+    _check(_lib.csa_pack_fp8_window(ctypes.byref(a), _stream(stream)), "csa_pack_fp8_window")
+# (PagedCache: a paged pool + block table, accepted wherever a PackedCache is)
+    return win
+
+
 def _attn_args(q, q_pos, cache: PackedCache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse):
+    """win_kv: bf16 rows [B, Wn, d] or an Fp8Window."""
     B, Nq, H, d = q.shape
     k = idx.shape[-1] if idx is not None else 0
     Wn = win_kv.shape[1] if win_kv is not None else 0
-    return AttnArgs(ctypes.sizeof(AttnArgs), B, Nq, H, d, cache.d_rope, ratio, cache.n_max, k, Wn, window, cache.g,
-                    softmax_scale, _ptr(q), _ptr(q_pos), _ptr(cache.codes), _ptr(cache.scales), _ptr(cache.rope),
-                    _ptr(n_c), _ptr(idx), _ptr(win_kv), _ptr(win_pos0), _ptr(out), _ptr(lse))
+    fp8 = isinstance(win_kv, Fp8Window)
+    a = AttnArgs(ctypes.sizeof(AttnArgs), B, Nq, H, d, cache.d_rope, ratio, cache.n_max, k, Wn, window, cache.g,
+                 softmax_scale, _ptr(q), _ptr(q_pos), _ptr(cache.codes), _ptr(cache.scales), _ptr(cache.rope),
+                 _ptr(n_c), _ptr(idx), None if fp8 else _ptr(win_kv), _ptr(win_pos0), _ptr(out), _ptr(lse))
+    if fp8:
+        a.win_format = 1
+        a.win_codes, a.win_scales, a.win_rope = _ptr(win_kv.codes), _ptr(win_kv.scales), _ptr(win_kv.rope)
+    a.kv_pages = _page_map(cache)
+    return a
 
 
 def _attn(fn, hca, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse, ws,

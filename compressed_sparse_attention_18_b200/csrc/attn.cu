@@ -67,6 +67,7 @@ struct AttnParams {
   float* lse;
   float* part_o;    // [B*Nq][splits][H][D]
   float* part_lse;  // [B*Nq][splits][H]
+  csa_page_map pm;         // cache rows (table == NULL: contiguous [B][n_max])
 };
 
 template <int D, int DS>
@@ -135,9 +136,6 @@ __global__ void __launch_bounds__(AT_WARPS * 32, 1) attn_kernel(AttnParams P) {
 
   const uint32_t sQa = (uint32_t)__cvta_generic_to_shared(sQ);
   const uint32_t sKa = (uint32_t)__cvta_generic_to_shared(sK);
-  const uint8_t* codes_b = P.codes + (size_t)b * P.n_max * (d_n / 2);
-  const uint8_t* scales_b = P.scales + (size_t)b * P.n_max * S_pad;
-  const uint16_t* rope_b = P.rope + (size_t)b * P.n_max * P.d_r;
   const int32_t* idx_row = P.idx ? P.idx + (size_t)bq * P.k : nullptr;
 
   for (int c = c_begin; c < c_end; ++c) {
@@ -151,18 +149,21 @@ __global__ void __launch_bounds__(AT_WARPS * 32, 1) attn_kernel(AttnParams P) {
       long long src = 0;
       if (li < n_sel) {
         const int id = P.hca ? li : idx_row[li];
-        if (id >= 0 && id < ncb) { kind = 1; src = id; }
+        if (id >= 0 && id < ncb) {
+          src = page_row(P.pm, b, P.n_max, id);      // row in the (contiguous or paged) cache arrays
+          kind = src >= 0 ? 1 : 0;
+        }
       } else if (li < n_list) {
         kind = 2;
         src = (wlo + (li - n_sel)) - P.win_pos0[b];
       }
       if (kind == 1) {
         const uint32_t dst = sRawa + row * RAW;
-        if (lane < d_n / 32) cpa16(dst + lane * 16, codes_b + src * (d_n / 2) + lane * 16);
+        if (lane < d_n / 32) cpa16(dst + lane * 16, P.codes + src * (d_n / 2) + lane * 16);
         else if (lane >= 16 && lane < 16 + P.d_r / 8)
-          cpa16(dst + RAW_ROPE + (lane - 16) * 16, rope_b + src * P.d_r + (lane - 16) * 8);
+          cpa16(dst + RAW_ROPE + (lane - 16) * 16, P.rope + src * P.d_r + (lane - 16) * 8);
         else if (lane == 31)
-          for (int q4 = 0; q4 < S_pad; q4 += 4) cpa4(dst + RAW_SC + q4, scales_b + src * S_pad + q4);
+          for (int q4 = 0; q4 < S_pad; q4 += 4) cpa4(dst + RAW_SC + q4, P.scales + src * S_pad + q4);
       } else if (kind == 2) {
         const uint16_t* wrow = P.win + ((size_t)b * P.Wn + src) * D;
         for (int cc = lane; cc < CH; cc += 32) cpa16(sKa + swz<D>(row, cc), wrow + cc * 8);
@@ -543,10 +544,11 @@ static csa_status launch_out_rope(uint16_t* out, int H, int D, long long rows, c
 }
 
 // tensor-core decode path (attn_tc.cu)
-bool attn_tc_eligible(const csa_attn_args* a, int hca, int max_splits);
 void attn_tc_plan(const csa_attn_args* a, int hca, int* splits, int* tpc);
 csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, uint16_t* part_o, float* part_lse,
                           cudaStream_t st);
+
+bool attn_tc_eligible(const csa_attn_args* a, int hca, int max_splits);
 
 struct AttnPlan {
   int splits, cps, tpc;
@@ -570,7 +572,7 @@ static AttnPlan plan_attn(const csa_attn_args* a, int hca) {
     return p;
   }
   const long long n_sel = hca ? a->n_max : a->k;
-  const long long n_win = (a->win_kv && a->Wn > 0) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
+  const long long n_win = attn_has_window(a) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
   const long long chunks = (n_sel + n_win + AT_KC - 1) / AT_KC;
   const long long rows = (long long)a->B * a->Nq;
   long long splits = rows >= 148 ? 1 : 148 / rows;
@@ -597,12 +599,22 @@ static csa_status validate_attn(const csa_attn_args* a, int hca) {
   CSA_SUPPORTED(a->H <= (a->d == 512 ? 64 : 16));
   CSA_REQUIRE(a->g_kv > 0.0f);
   CSA_REQUIRE(a->out_rope_theta >= 0.0f);        // (false for NaN too)
+  CSA_REQUIRE(a->win_format == CSA_WIN_BF16 || a->win_format == CSA_WIN_FP8);
   if (!hca) CSA_REQUIRE(a->k >= 1);
+  {
+    const csa_status pv = check_page_map(a->kv_pages, a->n_max);
+    if (pv != CSA_OK) return pv;
+  }
   if ((long long)a->B * a->Nq == 0) return CSA_OK;
   CSA_REQUIRE(a->q && a->q_pos && a->n_c && a->out);
   CSA_REQUIRE(a->n_max == 0 || (a->kv_codes && a->kv_scales && a->kv_rope));
   if (!hca) CSA_REQUIRE(a->idx != nullptr);
-  if (a->Wn > 0) CSA_REQUIRE(a->win_kv && a->win_pos0);
+  if (a->Wn > 0 && a->win_format == CSA_WIN_BF16) CSA_REQUIRE(a->win_kv && a->win_pos0);
+  if (a->Wn > 0 && a->win_format == CSA_WIN_FP8) {
+    CSA_REQUIRE(a->win_codes && a->win_scales && a->win_rope && a->win_pos0);
+    // FP8 window rows are read by the tensor-core path only (d = 512, 16-byte aligned rows)
+    CSA_SUPPORTED(attn_tc_eligible(a, hca, MERGE_MAX_SPLITS));
+  }
   return CSA_OK;
 }
 
@@ -647,7 +659,7 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
   const float scale = a->softmax_scale != 0.0f ? a->softmax_scale : 1.0f / sqrtf((float)a->d);
   P.scale_log2 = scale * LOG2E;
   P.q = (const uint16_t*)a->q; P.q_pos = a->q_pos; P.codes = a->kv_codes; P.scales = a->kv_scales;
-  P.rope = (const uint16_t*)a->kv_rope; P.n_c = a->n_c; P.idx = hca ? nullptr : a->idx;
+  P.rope = (const uint16_t*)a->kv_rope; P.n_c = a->n_c; P.idx = hca ? nullptr : a->idx; P.pm = a->kv_pages;
   P.win = (const uint16_t*)a->win_kv; P.win_pos0 = a->win_pos0; P.out = (uint16_t*)a->out; P.lse = a->lse;
   P.part_o = p.splits > 1 ? (float*)((uint8_t*)ws + p.off_o) : nullptr;
   P.part_lse = p.splits > 1 ? (float*)((uint8_t*)ws + p.off_lse) : nullptr;

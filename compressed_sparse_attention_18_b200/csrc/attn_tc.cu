@@ -71,42 +71,17 @@ struct TaParams {
   float* lse;           // splits == 1 (may be null)
   uint16_t* part_o;     // [rows][splits][H][512] bf16 (splits = CTAs per query)
   float* part_lse;      // [rows][splits][H]
+  int win_fp8;          // window rows are FP8 (codes / scales / rope below) instead of bf16 rows in `win`
+  const uint8_t* wcodes;   // [B][Wn][448] E4M3
+  const float* wscales;    // [B][Wn][8] fp32 (7 used)
+  const uint16_t* wrope;   // [B][Wn][64] bf16
+  csa_page_map pm;         // cache rows (table == NULL: contiguous [B][n_max])
 };
 
 __device__ __forceinline__ uint32_t sw128(int row, int chunk) { return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4)); }
 
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, bool acc) {
-  asm volatile("{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
-               ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"((uint32_t)acc) : "memory");
-}
-// kind::f16 instruction descriptor: bf16 A and B, fp32 accumulate; a_mn / b_mn select MN-major operands.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
 __device__ __forceinline__ void cp16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src));
-}
-
-__device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr) : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld_x32(uint32_t* r) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
-                 "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]),
-                 "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
-                 "+r"(r[30]), "+r"(r[31])
-               :: "memory");
 }
 
 __device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
@@ -132,6 +107,16 @@ __device__ __forceinline__ uint4 e2m1x8_to_bf16_scaled(uint32_t w, uint32_t sc2)
   o.z = hmul2_bf16(__byte_perm(lb, hb, 0x5140) | (__byte_perm(x, w, 0x6622) & 0x80008000u), sc2);
   o.w = hmul2_bf16(__byte_perm(lb, hb, 0x7362) | (__byte_perm(x, w, 0x7733) & 0x80008000u), sc2);
   return o;
+}
+
+// Two E4M3 codes (low byte first) times an fp32 scale -> packed bf16x2: exact E4M3 -> f16 conversion,
+// the product rounded to fp32, then to bf16.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2_scaled(uint32_t two, float sc) {
+  uint32_t h2;
+  const uint16_t in = (uint16_t)two;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+  return pack_bf16x2(f.x * sc, f.y * sc);
 }
 
 // 32 values per lane reduced across the warp's 32 lanes, transposed: on return lane l holds the reduction of
@@ -168,12 +153,13 @@ struct TaTile {
   int key0, rs, rw, wa, we, zs;
   long long wrow_base;     // window buffer row of tile row r (r >= rs) is wrow_base + r
 };
-__device__ __forceinline__ TaTile ta_tile(int key0, int n_sel, int n_list, long long wlo, long long p0) {
+// FP8 window rows are gathered and dequantised by the workers (no TMA boxes: wa = we = rw).
+__device__ __forceinline__ TaTile ta_tile(int key0, int n_sel, int n_list, long long wlo, long long p0, bool fp8) {
   TaTile g;
   g.key0 = key0;
   g.rs = min(max(n_sel - key0, 0), TA_KEYS);                        // rows [0, rs): entries
   g.rw = max(min(n_list - key0, TA_KEYS), 0);                       // rows [rs, rw): window, then empty
-  g.wa = (g.rs + TA_WBOX - 1) / TA_WBOX * TA_WBOX;                   // window rows >= wa come by TMA boxes
+  g.wa = fp8 ? g.rw : (g.rs + TA_WBOX - 1) / TA_WBOX * TA_WBOX;      // window rows >= wa come by TMA boxes
   g.we = g.rw > g.wa ? (g.rw + TA_WBOX - 1) / TA_WBOX * TA_WBOX : g.wa;
   g.zs = g.rw > g.wa ? g.we : g.rw;                                  // rows >= zs are zero-filled
   g.wrow_base = (wlo - p0) + (long long)(key0 - n_sel);
@@ -229,7 +215,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
     const int lines = (P.k * 4 + 127) / 128;
     for (int i = tid; i < lines; i += TA_THREADS) prefetch_l2(P.idx + (size_t)bq * P.k + i * 32);
   }
-  {
+  if (P.pm.table == nullptr) {
     const size_t n_max = (size_t)P.n_max;
     const size_t cb = n_max * 224, sb = n_max * 16, rb = n_max * 128, pg = (size_t)1 << 21;
     const size_t nc = (cb + pg - 1) / pg, ns = (sb + pg - 1) / pg, nr = (rb + pg - 1) / pg;
@@ -305,7 +291,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       const uint32_t ido = idesc_bf16(128, 64, 1, 1);
 #pragma unroll 1
       for (int t = 0; t < ntile; ++t) {
-        const TaTile g = ta_tile(tile_key(t), n_sel, n_list, wlo, p0);
+        const TaTile g = ta_tile(tile_key(t), n_sel, n_list, wlo, p0, P.win_fp8 != 0);
         const int nbox = (g.we - g.wa) / TA_WBOX;
         // window boxes overwrite the K tile: only once the previous tile's O MMAs have completed (S MMAs
         // of an entry tile are queued behind them directly)
@@ -354,9 +340,6 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------------------------- workers
-    const uint8_t* codes_b = P.codes + (size_t)b * P.n_max * 224;
-    const uint8_t* scales_b = P.scales + (size_t)b * P.n_max * 16;
-    const uint16_t* rope_b = P.rope + (size_t)b * P.n_max * 64;
     const int quad = warp & 3, hh = warp >> 2;
     const int key = 32 * quad + lane;
     const uint32_t lane_base = tb + ((uint32_t)(32 * quad) << 16);
@@ -377,20 +360,44 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       sc16 = make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int c = 0; c < 4; ++c) rp[c] = make_uint4(0, 0, 0, 0);
-      if (id >= 0) {
-        const uint8_t* crow = codes_b + (size_t)id * 224 + ghalf * 16;
+      const long long r = id >= 0 ? page_row(P.pm, b, P.n_max, id) : -1;   // row in the cache arrays
+      if (r >= 0) {
+        const uint8_t* crow = P.codes + (size_t)r * 224 + ghalf * 16;
 #pragma unroll
         for (int j = 0; j < 7; ++j) cv[j] = __ldg(reinterpret_cast<const uint4*>(crow + j * 32));
-        sc16 = __ldg(reinterpret_cast<const uint4*>(scales_b + (size_t)id * 16));
-        const uint4* rrow = reinterpret_cast<const uint4*>(rope_b + (size_t)id * 64) + ghalf * 4;
+        sc16 = __ldg(reinterpret_cast<const uint4*>(P.scales + (size_t)r * 16));
+        const uint4* rrow = reinterpret_cast<const uint4*>(P.rope + (size_t)r * 64) + ghalf * 4;
 #pragma unroll
         for (int c = 0; c < 4; ++c) rp[c] = __ldg(rrow + c);
       }
     };
-    TaTile g = ta_tile(tile_key(0), n_sel, n_list, wlo, p0);
+    // FP8 window row of a tile (rows [rs, rw)) in the same registers an entry row uses: codes of this
+    // thread's 32 channels of 64-channel blocks 0-2 in cv[0..5], the 7 block scales in cv[6] (0-3) and
+    // sc16 (4-6), the RoPE quarter in rp; blocks 3-6 are read into cv[0..6], sc16 during the gather.
+    auto is_win8 = [&](const TaTile& gg) { return P.win_fp8 && grow >= gg.rs && grow < gg.rw; };
+    auto win8_ptr = [&](const TaTile& gg) -> const uint8_t* {
+      return P.wcodes + ((size_t)b * P.Wn + (size_t)(gg.wrow_base + grow)) * 448 + ghalf * 32;
+    };
+    auto load_win8 = [&](const TaTile& gg) {
+      const size_t wr = (size_t)b * P.Wn + (size_t)(gg.wrow_base + grow);
+      const uint4* crow = reinterpret_cast<const uint4*>(win8_ptr(gg));
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        cv[2 * j] = __ldg(crow + 4 * j);
+        cv[2 * j + 1] = __ldg(crow + 4 * j + 1);
+      }
+      const uint4* srow = reinterpret_cast<const uint4*>(P.wscales + wr * 8);
+      cv[6] = __ldg(srow);
+      sc16 = __ldg(srow + 1);
+      const uint4* rrow = reinterpret_cast<const uint4*>(P.wrope + wr * 64) + ghalf * 4;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) rp[c] = __ldg(rrow + c);
+    };
+    TaTile g = ta_tile(tile_key(0), n_sel, n_list, wlo, p0, P.win_fp8 != 0);
     int id = check_id(raw_id(g));                  // a window tile reads no id
-    int id_next = ntile > 1 && !has_win ? raw_id(ta_tile(tile_key(1), n_sel, n_list, wlo, p0)) : -1;
+    int id_next = ntile > 1 && !has_win ? raw_id(ta_tile(tile_key(1), n_sel, n_list, wlo, p0, P.win_fp8 != 0)) : -1;
     load_row(id);
+    if (is_win8(g)) load_win8(g);
 #pragma unroll 1
     for (int t = 0; t < ntile; ++t) {
       // a tile of entry rows only can be refilled block by block as the previous tile's O MMAs release
@@ -405,7 +412,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       if (!pure) {
         // window rows before the first TMA box, by asynchronous copies
         const int r_end = min(g.wa, g.rw);
-        const int n = (r_end > g.rs ? r_end - g.rs : 0) * 64;
+        const int n = P.win_fp8 ? 0 : (r_end > g.rs ? r_end - g.rs : 0) * 64;
         for (int i = tid; i < n; i += TA_WORKERS) {
           const int row = g.rs + (i >> 6), c = i & 63;
           const long long wr = g.wrow_base + row;
@@ -418,9 +425,25 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
         }
         asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
       }
+      const bool win8_row = is_win8(g);
+      float ws3 = 0.f, ws4 = 0.f, ws5 = 0.f, ws6 = 0.f;
       // dequantise dim block by dim block: bf16(e2m1 * bf16(e4m3 * g)); each block released to the MMA warp
 #pragma unroll
       for (int j = 0; j < 7; ++j) {
+        if (win8_row && j == 3) {
+          // blocks 0-2 are done: keep scales 3-6, read the codes of blocks 3-6 into the same registers
+          ws3 = __uint_as_float(cv[6].w);
+          ws4 = __uint_as_float(sc16.x);
+          ws5 = __uint_as_float(sc16.y);
+          ws6 = __uint_as_float(sc16.z);
+          const uint4* crow = reinterpret_cast<const uint4*>(win8_ptr(g));
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            cv[2 * i] = __ldg(crow + 4 * (3 + i));
+            if (i < 3) cv[2 * i + 1] = __ldg(crow + 4 * (3 + i) + 1);
+          }
+          sc16 = __ldg(crow + 4 * 6 + 1);
+        }
         if (t > 0 && pure && (j & 1) == 0) {
           ok = mbar_wait(&S.bar_o[j >> 1], (t - 1) & 1) && ok;
           tc_fence_after();
@@ -434,6 +457,19 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4)
             *reinterpret_cast<uint4*>(&S.K[j][sw128(grow, ghalf * 4 + q4)]) = e2m1x8_to_bf16_scaled(w4[q4], sc2);
+        } else if (win8_row) {
+          // FP8 window row: bf16(e4m3 * scale of the 64-channel block)
+          const float sc = j == 0 ? __uint_as_float(cv[6].x) : j == 1 ? __uint_as_float(cv[6].y)
+                         : j == 2 ? __uint_as_float(cv[6].z) : j == 3 ? ws3 : j == 4 ? ws4 : j == 5 ? ws5 : ws6;
+          const uint4 c0 = j < 3 ? cv[2 * j] : cv[2 * (j - 3)];
+          const uint4 c1 = j < 3 ? cv[2 * j + 1] : j < 6 ? cv[2 * (j - 3) + 1] : sc16;
+          const uint32_t w8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<uint4*>(&S.K[j][sw128(grow, ghalf * 4 + q4)]) =
+                make_uint4(e4m3x2_to_bf16x2_scaled(w8[2 * q4] & 0xFFFFu, sc), e4m3x2_to_bf16x2_scaled(w8[2 * q4] >> 16, sc),
+                           e4m3x2_to_bf16x2_scaled(w8[2 * q4 + 1] & 0xFFFFu, sc),
+                           e4m3x2_to_bf16x2_scaled(w8[2 * q4 + 1] >> 16, sc));
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -443,8 +479,8 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
         ok = mbar_wait(&S.bar_o[3], (t - 1) & 1) && ok;
         tc_fence_after();
       }
-      // RoPE slice (dim block 7) of the entry rows
-      if (grow < g.rs) {
+      // RoPE slice (dim block 7) of the entry rows (and of FP8 window rows)
+      if (grow < g.rs || win8_row) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(&S.K[7][sw128(grow, ghalf * 4 + c)]) = rp[c];
       }
@@ -458,12 +494,13 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
         if (has_win && t == 0) {
           // the window tile is gathered: from here on the ids and entries of the previous kernels
           pdl_wait();
-          id_next = raw_id(ta_tile(tile_key(1), n_sel, n_list, wlo, p0));
+          id_next = raw_id(ta_tile(tile_key(1), n_sel, n_list, wlo, p0, P.win_fp8 != 0));
         }
-        g = ta_tile(tile_key(t + 1), n_sel, n_list, wlo, p0);
+        g = ta_tile(tile_key(t + 1), n_sel, n_list, wlo, p0, P.win_fp8 != 0);
         id = check_id(id_next);
         load_row(id);
-        id_next = t + 2 < ntile ? raw_id(ta_tile(tile_key(t + 2), n_sel, n_list, wlo, p0)) : -1;
+        if (is_win8(g)) load_win8(g);
+        id_next = t + 2 < ntile ? raw_id(ta_tile(tile_key(t + 2), n_sel, n_list, wlo, p0, P.win_fp8 != 0)) : -1;
       }
       asm volatile("bar.sync 1, 256;" ::: "memory");   // workers only: ids visible to the softmax
 
@@ -602,7 +639,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
 // window tile before the step's index and top-k kernels have ended; possible when the window fills one
 // tile right after the k entries (k a multiple of the tile, at most one tile of window).
 bool attn_tc_early(const csa_attn_args* a, int hca) {
-  const long long n_win = (a->win_kv && a->Wn > 0) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
+  const long long n_win = attn_has_window(a) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
   return !hca && (a->flags & CSA_EARLY_START) && n_win > 0 && n_win <= TA_KEYS && a->k > 0 && a->k % TA_KEYS == 0;
 }
 
@@ -612,7 +649,7 @@ bool attn_tc_early(const csa_attn_args* a, int hca) {
 // (first, while the previous kernel still runs).
 void attn_tc_plan(const csa_attn_args* a, int hca, int* splits, int* tpc) {
   const bool early = attn_tc_early(a, hca);
-  const long long n_win = (a->win_kv && a->Wn > 0) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
+  const long long n_win = attn_has_window(a) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
   const long long n = (hca ? a->n_max : a->k) + (early ? 0 : n_win);
   const long long tiles = n > 0 ? (n + TA_KEYS - 1) / TA_KEYS : 1;
   const long long rows = (long long)a->B * a->Nq;
@@ -629,7 +666,11 @@ bool attn_tc_eligible(const csa_attn_args* a, int hca, int max_splits) {
   return a->d == 512 && a->d_rope == 64 && a->H <= 64 && splits >= 1 && splits <= max_splits &&
          ((uintptr_t)a->q & 15) == 0 && (a->n_max == 0 || (((uintptr_t)a->kv_codes & 15) == 0 &&
                                                            ((uintptr_t)a->kv_rope & 15) == 0)) &&
-         (!a->win_kv || a->Wn == 0 || ((uintptr_t)a->win_kv & 15) == 0) && tensor_map_encoder() != nullptr;
+         (a->win_format == CSA_WIN_FP8
+              ? (!attn_has_window(a) || ((((uintptr_t)a->win_codes | (uintptr_t)a->win_scales | (uintptr_t)a->win_rope) &
+                                          15) == 0))
+              : (!a->win_kv || a->Wn == 0 || ((uintptr_t)a->win_kv & 15) == 0)) &&
+         tensor_map_encoder() != nullptr;
 }
 
 csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, uint16_t* part_o,
@@ -646,8 +687,9 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return CSA_ERR_CUDA;
   }
-  const int Wn = (a->win_kv && a->Wn > 0) ? a->Wn : 0;
-  if (Wn > 0) {
+  const bool fp8 = a->win_format == CSA_WIN_FP8;
+  const int Wn = attn_has_window(a) ? a->Wn : 0;
+  if (Wn > 0 && !fp8) {
     const cuuint64_t gdim[3] = {512, (cuuint64_t)Wn, (cuuint64_t)a->B};
     const cuuint64_t gstride[2] = {1024, (cuuint64_t)Wn * 1024};
     const cuuint32_t box[3] = {64, TA_WBOX, 1};
@@ -668,6 +710,14 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
   P.q_pos = a->q_pos; P.codes = a->kv_codes; P.scales = a->kv_scales;
   P.rope = (const uint16_t*)a->kv_rope; P.n_c = a->n_c; P.idx = hca ? nullptr : a->idx; P.win = (const uint16_t*)a->win_kv;
   P.win_pos0 = a->win_pos0; P.out = (uint16_t*)a->out; P.lse = a->lse; P.part_o = part_o; P.part_lse = part_lse;
+  P.win_fp8 = fp8 ? 1 : 0;
+  P.pm = a->kv_pages;
+  if (fp8) {
+    P.win = nullptr;
+    P.wcodes = a->win_codes;
+    P.wscales = a->win_scales;
+    P.wrope = (const uint16_t*)a->win_rope;
+  }
   const int smem = (int)sizeof(TaSmem) + 1024;
   static std::atomic<unsigned> attr_done{0};
   set_smem_once((const void*)attn_tc_kernel, smem, attr_done);

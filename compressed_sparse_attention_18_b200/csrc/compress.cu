@@ -11,132 +11,9 @@
 
 namespace csa {
 
-// ------------------------------------------------------------------------------------------ GEMM
-// C[M][N] = A[M][K] · W[K][N], bf16 in, fp32 accumulate, bf16 out.  128x128x32 tiles, 8 warps
-// (2 x 4, 64x32 each), 3-stage cp.async pipeline, ldmatrix from XOR-swizzled shared memory.
-// blockIdx.z selects (W0, C0) or (W1, C1) so both projections run in one launch.
-
-constexpr int GBM = 128, GBN = 128, GBK = 32, GSTAGES = 3;
-constexpr int G_A_BYTES = GBM * GBK * 2;   // 8 KB
-constexpr int G_B_BYTES = GBK * GBN * 2;   // 8 KB
-constexpr int G_SMEM = GSTAGES * (G_A_BYTES + G_B_BYTES);
-
-__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g, bool pred) {
-  const int sz = pred ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(g), "r"(sz));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, const uint32_t* b) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-__global__ void __launch_bounds__(256) gemm_bf16_kernel(const uint16_t* __restrict__ A,
-                                                        const uint16_t* __restrict__ W0,
-                                                        const uint16_t* __restrict__ W1, uint16_t* C0,
-                                                        uint16_t* C1, int M, int N, int K) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const uint16_t* W = blockIdx.z ? W1 : W0;
-  uint16_t* C = blockIdx.z ? C1 : C0;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int wm = warp >> 2, wn = warp & 3;
-  const int m0 = blockIdx.y * GBM, n0 = blockIdx.x * GBN;
-  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
-  auto sA = [&](int st) { return sbase + st * (G_A_BYTES + G_B_BYTES); };
-  auto sB = [&](int st) { return sbase + st * (G_A_BYTES + G_B_BYTES) + G_A_BYTES; };
-
-  auto load_stage = [&](int st, int k0) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int c = tid + i * 256;          // A: 128 rows x 4 chunks
-      const int row = c >> 2, col = c & 3;
-      const int gm = m0 + row;
-      const bool ok = gm < M;
-      const uint16_t* g = A + (size_t)(ok ? gm : 0) * K + k0 + col * 8;
-      cp_async16(sA(st) + row * 64 + ((col ^ ((row >> 1) & 3)) << 4), g, ok);
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int c = tid + i * 256;          // B: 32 rows (k) x 16 chunks (n)
-      const int row = c >> 4, col = c & 15;
-      const uint16_t* g = W + (size_t)(k0 + row) * N + n0 + col * 8;
-      cp_async16(sB(st) + row * 256 + ((col ^ (row & 7)) << 4), g, true);
-    }
-  };
-
-  float acc[4][4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.0f;
-
-  const int KT = K / GBK;
-#pragma unroll
-  for (int s = 0; s < GSTAGES - 1; ++s) {
-    if (s < KT) load_stage(s, s * GBK);
-    cp_async_commit();
-  }
-  for (int kt = 0; kt < KT; ++kt) {
-    cp_async_wait<GSTAGES - 2>();
-    __syncthreads();
-    const int nxt = kt + GSTAGES - 1;
-    if (nxt < KT) load_stage(nxt % GSTAGES, nxt * GBK);
-    cp_async_commit();
-    const int st = kt % GSTAGES;
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-      uint32_t af[4][4], bfr[4][2];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int row = wm * 64 + i * 16 + (lane & 15);
-        const int chunk = kk * 2 + (lane >> 4);
-        ldsm_x4(sA(st) + row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4), af[i][0], af[i][1], af[i][2], af[i][3]);
-      }
-#pragma unroll
-      for (int j = 0; j < 4; j += 2) {
-        const int krow = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int nchunk = (wn * 32 + j * 8) / 8 + (lane >> 4);
-        ldsm_x4_t(sB(st) + krow * 256 + ((nchunk ^ (krow & 7)) << 4), bfr[j][0], bfr[j][1], bfr[j + 1][0],
-                  bfr[j + 1][1]);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) mma_bf16(acc[i][j], af[i], bfr[j]);
-    }
-  }
-  cp_async_wait<0>();
-  // epilogue: bf16 round, 32-bit stores
-  const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int col = n0 + wn * 32 + j * 8 + 2 * t;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int row = m0 + wm * 64 + i * 16 + g + h * 8;
-        if (row < M)
-          *reinterpret_cast<uint32_t*>(C + (size_t)row * N + col) = pack_bf16x2(acc[i][j][2 * h], acc[i][j][2 * h + 1]);
-      }
-    }
-}
+// The projections C = x·W_kv, Z = x·W_g run on the tensor cores (project_tc.cu).
+csa_status run_projection_tc(const void* x, const void* W0, const void* W1, void* C, void* Z, long long M, int N,
+                             int K, cudaStream_t st);
 
 // --------------------------------------------------------------------------------------- pooling
 // One CTA per (sequence, group of POOL_ENT entries, slice of OW indexer-key outputs).  Threads walk the
@@ -171,7 +48,8 @@ __device__ __forceinline__ void pack_row_to_cache(const float* row, int d, int d
                                                   int entry) {
   const int d_n = d - d_r;
   const int S = d_n / 32, S_pad = (S + 3) & ~3;
-  const long long dst = (long long)b * cc.n_max + (cc.row0 ? cc.row0[b] : 0) + entry;
+  const long long dst = page_row(cc.pages, b, cc.n_max, (long long)(cc.row0 ? cc.row0[b] : 0) + entry);
+  if (dst < 0) return;                          // a page outside the pool: nothing is written
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int blk = warp; blk < S; blk += nw)
     pack_block_warp(row[blk * 32 + lane], cc.global_scale, cc.codes + dst * (d_n / 2) + blk * 16,
@@ -426,7 +304,8 @@ __global__ void __launch_bounds__(POOL_THREADS) pool_kernel(PoolParams P) {
     const int S = d_I / 32, S_pad = (S + 3) & ~3;
     for (int t = warp; t < ne * (OW / 32); t += POOL_WARPS) {
       const int q = t / (OW / 32), blk = z * (OW / 32) + t % (OW / 32);
-      const long long dst = (long long)b * cc.n_max + (cc.row0 ? cc.row0[b] : 0) + e0 + q;
+      const long long dst = page_row(cc.pages, b, cc.n_max, (long long)(cc.row0 ? cc.row0[b] : 0) + e0 + q);
+      if (dst < 0) continue;
       pack_block_warp(krow[q * OW + (t % (OW / 32)) * 32 + lane], cc.global_scale, cc.codes + dst * (d_I / 2) + blk * 16,
                       cc.scales + dst * S_pad + blk);
       if (z == 0 && lane < S_pad - S) cc.scales[dst * S_pad + S + lane] = 0;
@@ -448,16 +327,12 @@ extern "C" csa_status csa_compress(const csa_compress_args* a, void* stream) {
   cudaStream_t st = (cudaStream_t)stream;
   if (a->x) {
     CSA_REQUIRE(a->W_kv && a->W_g && a->d_model > 0);
-    CSA_SUPPORTED(a->d % GBN == 0 && a->d_model % GBK == 0);
+    CSA_SUPPORTED(a->d % 128 == 0 && a->d_model % 8 == 0);
+    CSA_SUPPORTED((((uintptr_t)a->x | (uintptr_t)a->W_kv | (uintptr_t)a->W_g | (uintptr_t)a->C | (uintptr_t)a->Z) &
+                   15) == 0);
     const long long M = (long long)a->B * a->T;
     if (M > 0) {
-      static std::atomic<unsigned> attr_done{0};
-      set_smem_once((const void*)gemm_bf16_kernel, G_SMEM, attr_done);
-      dim3 grid(a->d / GBN, (unsigned)((M + GBM - 1) / GBM), 2);
-      gemm_bf16_kernel<<<grid, 256, G_SMEM, st>>>((const uint16_t*)a->x, (const uint16_t*)a->W_kv,
-                                                   (const uint16_t*)a->W_g, (uint16_t*)a->C, (uint16_t*)a->Z,
-                                                   (int)M, a->d, a->d_model);
-      csa_status s = launch_status();
+      csa_status s = run_projection_tc(a->x, a->W_kv, a->W_g, a->C, a->Z, M, a->d, a->d_model, st);
       if (s != CSA_OK) return s;
     }
   }
@@ -469,6 +344,11 @@ extern "C" csa_status csa_compress(const csa_compress_args* a, void* stream) {
     CSA_SUPPORTED((a->d - a->d_rope) % 32 == 0);
   }
   if (a->ki_pack.codes) CSA_REQUIRE(a->W_IK && a->ki_pack.scales && a->ki_pack.global_scale > 0.0f);
+  for (const csa_fp4_cache* cc : {&a->kv_pack, &a->ki_pack})
+    if (cc->codes) {
+      const csa_status pv = check_page_map(cc->pages, cc->n_max);
+      if (pv != CSA_OK) return pv;
+    }
   if (a->W_IK) CSA_SUPPORTED(((uintptr_t)a->W_IK & 15) == 0);
   // groups longer than 8 slots are read 8 channels (16 bytes) at a time
   if (a->ratio > 8) CSA_SUPPORTED((((uintptr_t)a->C | (uintptr_t)a->Z | (uintptr_t)a->b_pos) & 15) == 0);

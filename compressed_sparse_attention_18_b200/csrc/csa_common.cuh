@@ -60,6 +60,33 @@ inline csa_status launch_status() {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Row of logical entry i of sequence b in a cache laid out by `m` (see csa_page_map); -1 if its page id
+// is outside the pool (a caller error: the entry is then skipped, never addressed).
+__host__ __device__ __forceinline__ long long page_row(const csa_page_map& m, int b, long long n_max, long long i) {
+  if (m.table == nullptr) return (long long)b * n_max + i;
+  const int pg = m.table[(long long)b * m.width + i / m.page_size];
+  if (pg < 0 || pg >= m.n_pages) return -1;
+  return (long long)pg * m.page_size + i % m.page_size;
+}
+
+// Host check of a page map: NULL table, or page_size % 128 == 0 and enough pages per sequence.
+inline csa_status check_page_map(const csa_page_map& m, long long n_max) {
+  if (m.table == nullptr) return CSA_OK;
+  if (m.page_size <= 0 || m.page_size % 128 != 0 || m.width <= 0 || m.n_pages <= 0) return CSA_ERR_UNSUPPORTED;
+  if ((long long)m.width * m.page_size < n_max) return CSA_ERR_INVALID;
+  return CSA_OK;
+}
+
+// Rows a contiguous or paged cache array spans (the extent of its tensor map).
+inline long long cache_rows(const csa_page_map& m, int B, long long n_max) {
+  return m.table ? (long long)m.n_pages * m.page_size : (long long)B * n_max;
+}
+
+// A call of the attention has window rows: bf16 rows in win_kv, or FP8 rows in win_codes.
+inline bool attn_has_window(const csa_attn_args* a) {
+  return a->Wn > 0 && (a->win_format == CSA_WIN_FP8 ? a->win_codes != nullptr : a->win_kv != nullptr);
+}
+
 // ----------------------------------------------------------------- programmatic dependent launch
 // The step kernels are launched so that they may start while the kernel before them in the stream is
 // still finishing: each does its setup that touches no global memory, then pdl_wait() (the previous

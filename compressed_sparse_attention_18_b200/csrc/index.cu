@@ -77,7 +77,7 @@ struct KeyRow {
 
 template <int DI>
 __device__ __forceinline__ void load_key(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                                         int key, bool valid, int t, KeyRow<DI>& raw, uint32_t& sc) {
+                                         long long key, bool valid, int t, KeyRow<DI>& raw, uint32_t& sc) {
   constexpr int S_PAD = ((DI / 32) + 3) & ~3;
   if (!valid) {
 #pragma unroll
@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
     const uint8_t* __restrict__ k_codes, const uint8_t* __restrict__ k_scales, int n_max,
     const int32_t* __restrict__ n_c, const int64_t* __restrict__ q_pos, int ratio,
     const int32_t* __restrict__ cand, int n_cand, float* __restrict__ scores, long long ld, int tpw,
-    uint32_t* __restrict__ hist) {
+    uint32_t* __restrict__ hist, const csa_page_map pm) {
   constexpr int STEPS = DI / 16;
   constexpr int BREGS = DI / 8;           // f16x2 registers of one head slice per thread
   constexpr int S_PAD = ((DI / 32) + 3) & ~3;
@@ -153,20 +153,21 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
 
   const int chunk_end = min(n_cols, chunk0 + keys_per_cta);
   const int col_end = cand ? chunk_end : min(chunk_end, max_vis);
-  const uint8_t* codes_b = k_codes + (size_t)b * n_max * (DI / 2);
-  const uint8_t* scales_b = k_scales + (size_t)b * n_max * S_PAD;
   const int32_t* cand_row = cand ? cand + ((size_t)b * Nq + q0) * n_cand : nullptr;
   const long long t0 = s_t[0];
 
-  auto key_of = [&](int col, int& key, bool& ok) {
+  // key = the row of the key's codes / scales in the (contiguous or paged) cache arrays
+  auto key_of = [&](int col, long long& key, bool& ok) {
+    int id;
     if (cand_row) {
-      const int id = col < col_end ? cand_row[col] : -1;
-      key = id;
+      id = col < col_end ? cand_row[col] : -1;
       ok = id >= 0 && id < ncb && (long long)ratio * id + ratio - 1 <= t0;
     } else {
-      key = col;
+      id = col;
       ok = col < col_end && col < ncb;
     }
+    key = ok ? page_row(pm, b, n_max, id) : -1;
+    ok = ok && key >= 0;
   };
 
   const int first_col = chunk0 + warp * tpw * 16;
@@ -179,7 +180,7 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
       bq0[4 * i] = v.x; bq0[4 * i + 1] = v.y; bq0[4 * i + 2] = v.z; bq0[4 * i + 3] = v.w;
     }
   }
-  int key[2][2];
+  long long key[2][2];
   bool kval[2][2];
   KeyRow<DI> raw[2][2];
   uint32_t sc[2][2];
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     key_of(first_col + g + 8 * h, key[0][h], kval[0][h]);
-    load_key<DI>(codes_b, scales_b, key[0][h], kval[0][h], t, raw[0][h], sc[0][h]);
+    load_key<DI>(k_codes, k_scales, key[0][h], kval[0][h], t, raw[0][h], sc[0][h]);
   }
 #pragma unroll 2
   for (int tile = 0; tile < tpw; ++tile) {
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         key_of(col0 + 16 + g + 8 * h, key[cur ^ 1][h], kval[cur ^ 1][h]);
-        load_key<DI>(codes_b, scales_b, key[cur ^ 1][h], kval[cur ^ 1][h], t, raw[cur ^ 1][h], sc[cur ^ 1][h]);
+        load_key<DI>(k_codes, k_scales, key[cur ^ 1][h], kval[cur ^ 1][h], t, raw[cur ^ 1][h], sc[cur ^ 1][h]);
       }
     }
     uint32_t a[2][KeyRow<DI>::REGS];
@@ -962,9 +963,11 @@ __global__ void pool_expand_kernel(const int32_t* __restrict__ blk, int P, int G
   pool[(long long)row * P * G + s] = out;
 }
 
-// tensor-core scoring of single-query Full rows (index_tc.cu)
+// tensor-core scoring of single-query Full rows (index_tc.cu) and of multi-query Full rows (index_mq_tc.cu)
 bool index_tc_eligible(const csa_index_args* a);
 csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, uint32_t* hist, cudaStream_t st);
+bool index_mq_tc_eligible(const csa_index_args* a);
+csa_status run_scores_mq_tc(const csa_index_args* a, float* scores, long long ld, cudaStream_t st);
 
 // ------------------------------------------------------------------------------ orchestration
 struct IndexPlan {
@@ -1030,6 +1033,10 @@ static csa_status validate_index(const csa_index_args* a, bool need_select) {
     const int nblk = (a->n_max + a->pool_block_size - 1) / a->pool_block_size;
     CSA_SUPPORTED(nblk <= TOPK_CHUNK && a->pool_blocks <= 4096);
   }
+  {
+    const csa_status pv = check_page_map(a->k_pages, a->n_max);
+    if (pv != CSA_OK) return pv;
+  }
   if ((long long)a->B * a->Nq == 0) return CSA_OK;
   CSA_REQUIRE(a->n_c && a->q_pos);
   if (need_select) CSA_REQUIRE(a->idx_out != nullptr);
@@ -1048,6 +1055,7 @@ static csa_status run_scores(const csa_index_args* a, float* scores, long long l
     if (e != cudaSuccess) { set_last_cuda_error(e); return CSA_ERR_CUDA; }
   }
   if (index_tc_eligible(a)) return run_scores_tc(a, scores, ld, hist, st);
+  if (index_mq_tc_eligible(a)) return run_scores_mq_tc(a, scores, ld, st);
   const int qt = a->cand ? 1 : (a->Nq < IDX_QT ? a->Nq : IDX_QT);
   const long long qtiles = (long long)a->B * (a->cand ? a->Nq : (a->Nq + qt - 1) / qt);
   // key range per CTA: enough CTAs for about one wave, at least one 16-key tile per warp
@@ -1065,12 +1073,12 @@ static csa_status run_scores(const csa_index_args* a, float* scores, long long l
     set_smem_once((const void*)index_score_kernel<128>, IDX_QT * IDX_HEADS * 128 * 2 + HIST_BINS * 4, attr128);
     index_score_kernel<128><<<grid, IDX_WARPS * 32, smem, st>>>(
         (const uint16_t*)a->q_I, a->w, a->H_I, a->g_q, gg, a->Nq, qt, a->k_codes, a->k_scales, a->n_max, a->n_c,
-        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld, (int)tpw, hist);
+        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld, (int)tpw, hist, a->k_pages);
   } else {
     set_smem_once((const void*)index_score_kernel<64>, IDX_QT * IDX_HEADS * 64 * 2 + HIST_BINS * 4, attr64);
     index_score_kernel<64><<<grid, IDX_WARPS * 32, smem, st>>>(
         (const uint16_t*)a->q_I, a->w, a->H_I, a->g_q, gg, a->Nq, qt, a->k_codes, a->k_scales, a->n_max, a->n_c,
-        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld, (int)tpw, hist);
+        a->q_pos, a->ratio, a->cand, a->n_cand, scores, ld, (int)tpw, hist, a->k_pages);
   }
   return launch_status();
 }

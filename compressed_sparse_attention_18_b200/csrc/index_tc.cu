@@ -75,6 +75,7 @@ struct TcParams {
   int n_max, ratio, H_I, ctas_per_row;
   int early;                // read q_I, w, n_c, q_pos and key rows below n_c[b] - 1 before the wait
   float g_q, gg;
+  csa_page_map pm;          // key rows (table == NULL: contiguous [B][n_max])
 };
 
 // FP4-quantise 32 elements held one per lane (pack rule, global scale g); returns this lane's code.
@@ -140,13 +141,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
         const int s = i % TC_STAGES, f = i / TC_STAGES;
         if (!waited && t_begin + i >= wait_tile) { pdl_wait(); waited = true; }
         if (f > 0 && !mbar_wait(&S.empty[s], (f - 1) & 1)) { ok = false; break; }
-        const long long row = (long long)b * P.n_max + (long long)(t_begin + i) * TC_TILE;
-        long long nrow = rows_total - row;
-        if (nrow > TC_TILE) nrow = TC_TILE;
-        const uint32_t sc_bytes = (uint32_t)nrow * 4;          // multiple of 16: n_max % 4 == 0
-        mbar_arrive_expect_tx(&S.full[s], TC_CODE_BYTES + sc_bytes);
-        tma_load_2d(S.codes[s], &kmap, 0, (int)row, &S.full[s]);
-        bulk_load(S.sc[s], P.k_scales + row * 4, sc_bytes, &S.full[s]);
+        // two 128-row sub-tiles, each inside one page of a paged pool; rows past a sequence's end that a
+        // tile also covers are never scored (a sub-tile of an absent page is left as it was)
+        long long row[2];
+        uint32_t sc_bytes[2], tx = 0;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const long long li = (long long)(t_begin + i) * TC_TILE + u * TC_SUB;
+          if (P.pm.table == nullptr) {
+            row[u] = (long long)b * P.n_max + li;
+            long long nrow = rows_total - row[u];
+            if (nrow > TC_SUB) nrow = TC_SUB;
+            if (nrow < 0) nrow = 0;
+            sc_bytes[u] = (uint32_t)nrow * 4;                   // multiple of 16: n_max % 4 == 0
+          } else {
+            row[u] = li < P.n_max ? page_row(P.pm, b, P.n_max, li) : -1;
+            sc_bytes[u] = row[u] >= 0 ? TC_SUB * 4 : 0;
+          }
+          if (sc_bytes[u] > 0) tx += TC_SUB * 64 + sc_bytes[u];
+        }
+        mbar_arrive_expect_tx(&S.full[s], tx);
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+          if (sc_bytes[u] > 0) {
+            tma_load_2d(S.codes[s] + u * (TC_SUB * 64), &kmap, 0, (int)row[u], &S.full[s]);
+            bulk_load(S.sc[s] + u * (TC_SUB * 4), P.k_scales + row[u] * 4, sc_bytes[u], &S.full[s]);
+          }
         ++issued;
       }
       if (!ok) atomicOr(&S.err, 1u);
@@ -323,15 +343,16 @@ EncodeTiledFn tensor_map_encoder() {
 
 bool index_tc_eligible(const csa_index_args* a) {
   return a->cand == nullptr && a->Nq == 1 && a->d_I == 128 && a->H_I <= 8 && a->n_max % 4 == 0 && a->n_max > 0 &&
+         cache_rows(a->k_pages, a->B, a->n_max) < 0x7fffffffLL &&
          (reinterpret_cast<uintptr_t>(a->k_codes) & 15) == 0 && (reinterpret_cast<uintptr_t>(a->k_scales) & 15) == 0 &&
          tensor_map_encoder() != nullptr;
 }
 
 csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, uint32_t* hist, cudaStream_t st) {
   CUtensorMap map;
-  const cuuint64_t gdim[2] = {64, (cuuint64_t)a->B * (cuuint64_t)a->n_max};
+  const cuuint64_t gdim[2] = {64, (cuuint64_t)cache_rows(a->k_pages, a->B, a->n_max)};
   const cuuint64_t gstride[1] = {64};
-  const cuuint32_t box[2] = {64, TC_TILE};
+  const cuuint32_t box[2] = {64, TC_SUB};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = tensor_map_encoder()(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void*)a->k_codes, gdim, gstride, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -351,6 +372,7 @@ csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, u
   P.H_I = a->H_I;
   P.g_q = a->g_q;
   P.gg = a->g_q * a->g_k;
+  P.pm = a->k_pages;
   // TC_CTAS_PER_SM resident CTAs per SM: one wave, at most one per tile
   const int tiles_row = (a->n_max + TC_TILE - 1) / TC_TILE;
   int per_row = (TC_CTAS_PER_SM * 148) / a->B;

@@ -84,6 +84,21 @@ csa_status csa_check_error_path(uint32_t polls, void* stream);
  * Paths that cannot use the flag ignore it.  Results are the same with and without it. */
 #define CSA_EARLY_START 1u
 
+/* Paged caches ([V4.1 notes] §実装上の工夫: serving keeps the compressed KV in pages; the pages give no
+ * layout, so this library fixes one).  A csa_page_map sends logical entry i of sequence b to row
+ *   table[b * width + i / page_size] * page_size + i % page_size
+ * of the arrays it accompanies, which are then pools [n_pages * page_size][...] instead of [B][n_max][...].
+ * table == NULL means the contiguous layout (row = b * n_max + i).  page_size % 128 == 0, so every
+ * 128-entry tile of the tensor-core kernels lies in one page; width * page_size >= n_max.  A page id
+ * outside [0, n_pages) is a caller error: the kernels then neither read nor write outside the pool (such
+ * a page is skipped), but results that depend on its entries are unspecified. */
+typedef struct csa_page_map {
+  const int32_t* table;    /* [B][width] device int32, or NULL */
+  int32_t page_size;
+  int32_t width;
+  int32_t n_pages;
+} csa_page_map;
+
 /* ------------------------------------------------------------------------------------------------
  * csa_compress — the compressor ([V4 blog] Fig. 3 / Fig. 4; [V4.1 notes] eq.(1) and CSA2 bullet).
  *
@@ -112,6 +127,7 @@ typedef struct csa_fp4_cache {
   const int32_t* row0;     /* [B] (NULL = 0) */
   int32_t n_max;
   float global_scale;
+  csa_page_map pages;      /* paged pool (table == NULL: contiguous [B][n_max]) */
 } csa_fp4_cache;
 
 typedef struct csa_compress_args {
@@ -156,9 +172,36 @@ typedef struct csa_pack_args {
   uint8_t* codes;
   uint8_t* scales;
   void* rope;
+  csa_page_map pages;      /* paged pool (table == NULL: contiguous [B][n_max]) */
 } csa_pack_args;
 
 csa_status csa_pack_fp4(const csa_pack_args* args, void* stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * csa_pack_fp8_window — FP8 pack of sliding-window KV rows ([V4.1 notes] FP4 主 KV キャッシュ bullet: the
+ * window's uncompressed KV stays FP8; [V4 blog] storage paragraph: the RoPE channels stay BF16).
+ *
+ * The pages fix FP8 (E4M3) but not its scaling; this library uses one fp32 scale per 64 channels:
+ * for rows src[b][j] (j < n), written to window row row0[b] + j of sequence b, per 64-block of the first
+ * d - d_rope channels: scale = fp32(amax / 448) (correctly rounded fp32 division); scale == 0 zeroes the
+ * block; else code_e = E4M3_rne_satfinite(fp32(x_e / scale)), -0 -> +0.  The last d_rope channels are
+ * copied.  Dequantised element = e4m3(code) * scale.
+ * Shapes: src[B][n][d] bf16; codes[B][Wn][d-d_rope] u8; scales[B][Wn][SW] fp32 with
+ *         SW = round_up((d-d_rope)/64, 4) (pad entries 0); rope[B][Wn][d_rope] bf16; row0[B] int32 (NULL = 0).
+ * Limits: (d - d_rope) % 64 == 0, d_rope % 8 == 0, row0[b] + n <= Wn (not checked on the device).
+ *         No workspace.
+ * ------------------------------------------------------------------------------------------------ */
+typedef struct csa_fp8_window_args {
+  uint32_t struct_size;
+  int32_t B, n, d, d_rope, Wn;
+  const void* src;
+  const int32_t* row0;
+  uint8_t* codes;
+  float* scales;
+  void* rope;
+} csa_fp8_window_args;
+
+csa_status csa_pack_fp8_window(const csa_fp8_window_args* args, void* stream);
 
 /* ------------------------------------------------------------------------------------------------
  * csa_index_topk — lightning indexer scores + per-query top-k ([V4 blog] §ハイブリッド注意, Fig. 3;
@@ -209,6 +252,7 @@ typedef struct csa_index_args {
                               fewer than k scores (e.g. one no scoring call filled) is taken to hold only
                               that many.  NULL = plain radix selection */
   uint32_t flags;          /* CSA_EARLY_START or 0 */
+  csa_page_map k_pages;    /* k_codes / k_scales as a paged pool (table == NULL: contiguous) */
 } csa_index_args;
 
 size_t csa_index_topk_workspace_size(const csa_index_args* args);
@@ -285,7 +329,20 @@ typedef struct csa_attn_args {
      (m, m + d_rope/2), before the bf16 cast; the values' RoPE channels, rotated at their own positions,
      then come out relative to the query.  lse is unchanged.  0 = off. */
   float out_rope_theta;
+  /* Window format ([V4.1 notes] FP4 主 KV キャッシュ bullet: the window KV stays FP8).  CSA_WIN_BF16: the
+     window rows are win_kv (above).  CSA_WIN_FP8: they are the FP8 rows csa_pack_fp8_window writes,
+     win_codes[B][Wn][d-d_rope], win_scales[B][Wn][SW] fp32, win_rope[B][Wn][d_rope] bf16 (win_kv is then
+     ignored), dequantised as bf16(e4m3 * scale) before the tensor cores.  FP8 needs d = 512 (the
+     tensor-core path) and 16-byte aligned buffers (else CSA_ERR_UNSUPPORTED). */
+  uint32_t win_format;
+  const uint8_t* win_codes;
+  const float* win_scales;
+  const void* win_rope;
+  csa_page_map kv_pages;   /* kv_codes / kv_scales / kv_rope as a paged pool (table == NULL: contiguous) */
 } csa_attn_args;
+
+#define CSA_WIN_BF16 0u
+#define CSA_WIN_FP8 1u
 
 size_t csa_attn_workspace_size(const csa_attn_args* args, int hca);
 csa_status csa_sparse_attn(const csa_attn_args* args, void* ws, size_t ws_bytes, void* stream);

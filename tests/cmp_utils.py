@@ -30,7 +30,8 @@ def assert_close(got, ref, atol, rtol, what=""):
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
     both_inf = np.isinf(got) & np.isinf(ref) & (np.sign(got) == np.sign(ref))
     both_nan = np.isnan(got) & np.isnan(ref)
-    err = np.abs(got - ref)
+    with np.errstate(invalid="ignore"):
+        err = np.abs(got - ref)
     err[both_inf | both_nan] = 0.0
     bad = err > atol + rtol * np.abs(np.where(both_inf | both_nan, 0.0, ref))
     # a NaN (or an infinity) on one side only is always a mismatch: NaN compares False above

@@ -55,13 +55,14 @@ def test_ctypes_mirrors_match_the_c_structs(csa, tmp_path):
     if cc is None:
         pytest.skip("no C compiler")
     src = tmp_path / "sz.c"
-    src.write_text('#include <stdio.h>\n#include "csa.h"\nint main(void){printf("%zu %zu %zu %zu %zu\\n",'
+    src.write_text('#include <stdio.h>\n#include "csa.h"\nint main(void){printf("%zu %zu %zu %zu %zu %zu\\n",'
                    'sizeof(csa_compress_args),sizeof(csa_fp4_cache),sizeof(csa_pack_args),'
-                   'sizeof(csa_index_args),sizeof(csa_attn_args));return 0;}\n')
+                   'sizeof(csa_index_args),sizeof(csa_attn_args),sizeof(csa_fp8_window_args));return 0;}\n')
     exe = tmp_path / "sz"
     subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
     got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
-    want = [ctypes.sizeof(t) for t in (csa.CompressArgs, csa.Fp4Cache, csa.PackArgs, csa.IndexArgs, csa.AttnArgs)]
+    want = [ctypes.sizeof(t) for t in (csa.CompressArgs, csa.Fp4Cache, csa.PackArgs, csa.IndexArgs, csa.AttnArgs,
+                                       csa.Fp8WindowArgs)]
     assert got == want
 
 
@@ -148,6 +149,19 @@ def test_invalid_arguments_are_rejected_on_the_host(csa):
         assert lib.csa_sparse_attn(ctypes.byref(aa), None, 0, None) == 1
         aa.out_rope_theta = 10000.0
         assert lib.csa_sparse_attn(ctypes.byref(aa), None, 0, None) == 0   # B = 0: nothing to do
+    # paged caches: page sizes off the 128-entry tile, or a table too narrow for n_max, are refused
+    a = csa.PackArgs(ctypes.sizeof(csa.PackArgs), 1, 4, 64, 0, 300, 1.0, 256, None, 256, 256, None)
+    a.pages = csa.PageMap(256, 100, 3, 8)
+    assert lib.csa_pack_fp4(ctypes.byref(a), None) == 2
+    a.pages = csa.PageMap(256, 128, 2, 8)
+    assert lib.csa_pack_fp4(ctypes.byref(a), None) == 1
+    ia = csa.IndexArgs(ctypes.sizeof(csa.IndexArgs), 2, 1, 8, 128, 4, 16, 4096, 1.0, 1.0)
+    ia.k_pages = csa.PageMap(256, 64, 64, 128)
+    assert lib.csa_index_topk(ctypes.byref(ia), None, 0, None) == 2
+    # FP8 window: an unknown format is invalid; FP8 on the d = 128 path is unsupported
+    aa = csa.AttnArgs(ctypes.sizeof(csa.AttnArgs), 0, 1, 64, 512, 64, 4, 16, 8, 0, 128, 1.0, 0.0)
+    aa.win_format = 7
+    assert lib.csa_sparse_attn(ctypes.byref(aa), None, 0, None) == 1
     # error-path self-check: the poll count is checked before any launch
     assert lib.csa_check_error_path(0, None) == 1
     assert lib.csa_check_error_path((1 << 20) + 1, None) == 1

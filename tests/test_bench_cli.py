@@ -98,3 +98,17 @@ def test_no_graph_capture_inside_the_timed_region(steps, warmup):
     missing = next(n for n in range(1, bench.LAYERS) if n not in prepared)
     with pytest.raises(RuntimeError):             # an unprepared count is refused once frozen
         sg.run(missing)
+
+
+def test_prefill_work_closed_forms():
+    """The prefill FLOP counts: projection 4 T d_m d; the causal indexer scores sum_t floor((t+1)/r)
+    entries = 2 (T/r)(T/r - 1) + ... (closed form for T a multiple of r); attention keys by a plain loop."""
+    b = _load()
+    from csa_workloads import CFG3 as s
+    w = b.prefill_work(s)
+    assert w["projection"] == 4 * s.T * s.d_m * s.d
+    m = s.T // s.r
+    scored = s.r * m * (m - 1) // 2 + m                      # sum_{u=1}^{T} floor(u / r)
+    assert w["index"] == scored * s.H_I * s.d_I * 2
+    keys = sum(min(s.k, (t + 1) // s.r) + min(s.W, t + 1) for t in range(s.T))
+    assert w["attention"] == keys * s.H * s.d * 4

@@ -272,7 +272,9 @@ def test_index_k_larger_than_visible(cuda_lib):
 # -------------------------------------------------------------------------------------- attention
 
 def _attn_case(csa, *, B, Nq, H, d, d_r, n_max, n_c, q_pos, k=0, Wn=128, win_pos0=None, hca=False, ratio=4,
-               seed=0, g=1.0, q_scale=1.0, rope_theta=0.0):
+               seed=0, g=1.0, q_scale=1.0, rope_theta=0.0, win_fp8=False, early_start=False):
+    """win_fp8: the window rows are FP8-packed on the GPU (csa_pack_fp8_window) and the oracle attends over
+    its own FP8 pack of the same bf16 rows, dequantised (the pack itself is checked bit-exact elsewhere)."""
     G = gen(seed)
     kv = normal((B, n_max, d), 1.0, G)
     q = normal((B, Nq, H, d), q_scale, G)
@@ -291,20 +293,26 @@ def _attn_case(csa, *, B, Nq, H, d, d_r, n_max, n_c, q_pos, k=0, Wn=128, win_pos
             for qq in range(Nq):
                 perm = torch.randperm(n_max + 40, generator=G)[:k].to(torch.int32) - 20   # some < 0, some >= n_c
                 idx[b, qq] = perm
+    win_arg = win.to(DEV) if win is not None else None
+    if win is not None and win_fp8:
+        win_arg = csa.Fp8Window(B, Wn, d, d_r, DEV)
+        csa.pack_fp8_window(win.to(DEV), win_arg)
     if hca:
-        out, lse = csa.hca_attn(q.to(DEV), q_pos_t.to(DEV), cache, n_c_t.to(DEV),
-                                win.to(DEV) if win is not None else None, wp0.to(DEV) if win is not None else None,
-                                ratio=ratio, out_rope_theta=rope_theta)
+        out, lse = csa.hca_attn(q.to(DEV), q_pos_t.to(DEV), cache, n_c_t.to(DEV), win_arg,
+                                wp0.to(DEV) if win is not None else None, ratio=ratio, out_rope_theta=rope_theta)
     else:
-        out, lse = csa.sparse_attn(q.to(DEV), q_pos_t.to(DEV), cache, n_c_t.to(DEV), idx.to(DEV),
-                                   win.to(DEV) if win is not None else None, wp0.to(DEV) if win is not None else None,
-                                   ratio=ratio, out_rope_theta=rope_theta)
+        out, lse = csa.sparse_attn(q.to(DEV), q_pos_t.to(DEV), cache, n_c_t.to(DEV), idx.to(DEV), win_arg,
+                                   wp0.to(DEV) if win is not None else None, ratio=ratio, out_rope_theta=rope_theta,
+                                   early_start=early_start)
     torch.cuda.synchronize()
     scale = d ** -0.5
     for b in range(B):
         codes, scales, rope = O.pack_fp4(f64(kv[b]), d_r, g)
         rows = O.entry_kv(codes, scales, rope, d - d_r, g)
         wb = f64(win[b]) if win is not None else np.zeros((0, d))
+        if win is not None and win_fp8:
+            wc, ws, wr = O.pack_fp8_window(wb, d_r)
+            wb = O.dequant_fp8_window(wc, ws, wr)
         if hca:
             o_ref, l_ref = O.hca_attention(f64(q[b]), q_pos_t[b].numpy(), rows, n_c[b], ratio, wb, win_pos0[b], 128,
                                            scale, out_rope_theta=rope_theta, d_rope=d_r)
@@ -404,3 +412,55 @@ def test_attn_hca_empty_set(cuda_lib):
     out, lse = _attn_case(cuda_lib, B=1, Nq=1, H=64, d=512, d_r=64, n_max=16, n_c=[0], q_pos=[100], hca=True,
                           ratio=128, Wn=0, seed=8)
     assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+
+
+# ------------------------------------------------------------------------------------ FP8 window
+
+@pytest.mark.parametrize("d,d_r", [(512, 64), (128, 0), (192, 64)])
+def test_pack_fp8_window_bit_exact(cuda_lib, d, d_r):
+    csa = cuda_lib
+    B, n, Wn = 3, 45, 70
+    G = gen(41)
+    x = torch.randn((B, n, d), generator=G)
+    x[0, 0] = 0.0                                        # all-zero row: scale 0, codes 0
+    x[0, 1] *= 1e-30                                     # tiny scales (fp32 subnormal range)
+    x[0, 2, :64] = torch.tensor(O.e4m3_decode(np.arange(64)) * 3.0)   # scaled E4M3 grid values
+    x[1, 3] *= 3e4                                       # large rows
+    x[2, 4, 1::2] = -1e-6                                # elements rounding to -0 -> +0
+    x[2, 5, :64] = 0.0
+    x[2, 5, 7] = -2.0                                    # one nonzero: its code is exactly -448
+    src = x.to(torch.bfloat16)
+    win = csa.Fp8Window(B, Wn, d, d_r, DEV)
+    row0 = torch.tensor([0, 11, Wn - n], dtype=torch.int32, device=DEV)
+    csa.pack_fp8_window(src.to(DEV), win, row0)
+    torch.cuda.synchronize()
+    nb = (d - d_r) // 64
+    for b in range(B):
+        codes, scales, rope = O.pack_fp8_window(f64(src[b]), d_r)
+        r0 = int(row0[b])
+        assert np.array_equal(np_u8(win.codes[b, r0:r0 + n]), codes), f"codes b={b}"
+        got_s = win.scales[b, r0:r0 + n].cpu().numpy()
+        assert np.array_equal(got_s[:, :nb].view(np.uint32), scales.astype(np.float32).view(np.uint32)), f"scales b={b}"
+        assert np.all(got_s[:, nb:] == 0.0)
+        if d_r:
+            assert np.array_equal(bf16_bits(win.rope[b, r0:r0 + n]), bf16_bits(src[b, :, d - d_r:]))
+    assert int(win.codes[0, n:].abs().sum()) == 0        # rows outside [row0, row0 + n) untouched
+
+
+@pytest.mark.parametrize("early", [False, True])
+def test_attn_fp8_window_decode(cuda_lib, early):
+    n_c = [2048, 700, 2048, 1000]
+    q_pos = [4 * 2048 - 1, 4 * 700 - 1, 4 * 1500 + 3, 4 * 1000 - 1]
+    _attn_case(cuda_lib, B=4, Nq=1, H=64, d=512, d_r=64, n_max=2048, n_c=n_c, q_pos=q_pos, k=512, seed=42,
+               win_fp8=True, early_start=early)
+
+
+def test_attn_fp8_window_partial_multi_query_and_hca(cuda_lib):
+    # a window buffer holding part of the window, a query near the start, several queries per sequence
+    _attn_case(cuda_lib, B=2, Nq=1, H=64, d=512, d_r=64, n_max=64, n_c=[64, 2], q_pos=[255, 9], k=64, Wn=50,
+               win_pos0=[206, 0], seed=43, win_fp8=True)
+    q_pos = list(range(3000, 3000 + 37))
+    _attn_case(cuda_lib, B=1, Nq=37, H=64, d=512, d_r=64, n_max=800, n_c=[800], q_pos=q_pos, k=200, Wn=300,
+               seed=44, win_fp8=True)
+    _attn_case(cuda_lib, B=2, Nq=1, H=64, d=512, d_r=64, n_max=300, n_c=[300, 300],
+               q_pos=[128 * 300 - 1, 128 * 150 + 5], hca=True, ratio=128, seed=45, win_fp8=True)
