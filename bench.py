@@ -4,8 +4,8 @@ compressed entries per sequence, top-512, window 128, 64 heads x 512) on B200.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One step = the whole hot path for one decode token of every sequence: compress the completed group
-(pooling), FP4-pack the new entry and its indexer key, lightning-indexer scores over all entries,
-top-k, attention over the selected entries plus the window.  Eight independent layer states (3.7 GB)
+(pooling), FP4-pack the new entry and its indexer key, lightning-indexer scores over all entries and
+the top-k (one fused launch), attention over the selected entries plus the window.  Eight independent layer states (3.7 GB)
 are rotated so every step reads its caches from HBM, not from the 126 MB L2.  Steps are replayed from
 CUDA graphs; timing uses CUDA events on the launching stream, max over ranks.  Under torchrun every
 rank runs its own batch of 32 sequences (weak scaling, no collective on the data path).
@@ -106,10 +106,10 @@ def peaks():
     return 6650.0, "fallback"
 
 
-def score_kernel_bytes(s, B):
-    """Algorithmic bytes of one index-score launch: every visible key (64 B codes + 4 B scales), the
-    score written per key, the queries (bf16) and head weights."""
-    return B * (s.n_c * (s.d_I // 2 + s.d_I // 32 + 4) + s.H_I * s.d_I * 2 + s.H_I * 4)
+def index_topk_bytes(s, B):
+    """Algorithmic bytes of one fused index + top-k launch: every visible key (64 B codes + 4 B scales),
+    the queries (bf16) and head weights in, the k selected ids out (the scores stay on chip)."""
+    return B * (s.n_c * (s.d_I // 2 + s.d_I // 32) + s.H_I * s.d_I * 2 + s.H_I * 4 + s.k * 4)
 
 
 def attention_bytes(s, B):
@@ -418,7 +418,7 @@ def run_ours(args, rank, world):
     steps.run(LAYERS, with_marks=True)
     stream.synchronize()
     stage = [[marks[li][j].elapsed_time(marks[li][j + 1]) for j in range(4)] for li in range(LAYERS)]
-    score_ms = statistics.mean(st[1] for st in stage)
+    score_ms = statistics.mean(st[1] + st[2] for st in stage)          # fused index + top-k (stage 2 empty)
     ms = max_over_ranks(ms, world, dev)
     value = whole_job_rate(s.B * args.steps, world, ms)
 
@@ -431,7 +431,7 @@ def run_ours(args, rank, world):
     attn_ms = statistics.mean(st[3] for st in stage)
     abytes = attention_bytes(s, s.B)
     a_achieved = abytes / (attn_ms / 1e3) / 1e9
-    bpl = score_kernel_bytes(s, s.B)
+    bpl = index_topk_bytes(s, s.B)
     achieved = bpl / (score_ms / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -439,18 +439,19 @@ def run_ours(args, rank, world):
         "dtype": "fp4-e2m1/bf16", "data": "synthetic", "config": config_dict(s),
         "gpu_launches": CSADecodeLayer.KERNELS_PER_STEP * args.steps,
         "clocks": clocks,
-        "stages_ms": {"compress_pack": statistics.mean(st[0] for st in stage), "index_score": score_ms,
-                      "topk": statistics.mean(st[2] for st in stage), "attention": attn_ms},
+        "stages_ms": {"compress_pack": statistics.mean(st[0] for st in stage), "index_topk": score_ms,
+                      "attention": attn_ms},
         "stages_plan": "serialised stage-by-stage replay (an event at every stage boundary, no early start); "
                        "value/ms_per_step time the overlapped schedule",
-        # the dominant stage: tcgen05 attention over one 128-key tile per CTA plus the split merge
-        "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel + attn_merge_kernel (attention stage)",
+        # the dominant stage: tcgen05 attention over one 128-key tile per CTA, merged in the query's cluster
+        "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel (attention stage, in-cluster merge)",
                      "timed_on": "serialised stage-by-stage replay",
                      "achieved": a_achieved, "peak": hbm, "peak_kind": kind, "unit": "GB/s",
                      "frac": a_achieved / hbm, "traffic": profiled_traffic(ATTN_PROFILE, ATTN_SRC),
                      "algorithmic_bytes_per_launch": abytes},
-        # the streaming stage: every FP4 indexer key of every sequence (stage = histogram clear + kernel)
-        "roofline_index": {"bound": "hbm", "kernel": "index_score_tc_kernel", "timed_on": "serialised stage-by-stage replay",
+        # the streaming stage: every FP4 indexer key of every sequence, scored and selected in one launch
+        "roofline_index": {"bound": "hbm", "kernel": "index_score_tc_kernel<fused> (index + top-k)",
+                           "timed_on": "serialised stage-by-stage replay",
                            "achieved": achieved, "peak": hbm,
                            "peak_kind": kind, "unit": "GB/s", "frac": achieved / hbm,
                            "traffic": profiled_traffic(SCORE_PROFILE, INDEX_SRC), "algorithmic_bytes_per_launch": bpl},
@@ -976,6 +977,44 @@ def run_prefill(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_prefill(args):
+    """Profiling case of the chunked prefill: the compressor fills the caches chunk by chunk (8 launches
+    of the projection and pooling), then the last chunk's indexer, top-k and attention run once, eagerly
+    (about 20 launches in all, 2.5 GB on the device)."""
+    import compressed_sparse_attention_18_b200 as csa
+    from csa_workloads import CFG3, gen, normal
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    s = CFG3
+    Lc = s.extra["chunk"]
+    nch, n, epc = s.T // Lc, s.n_c, Lc // s.r
+    G = gen(40, dev)
+    x = normal((Lc, s.d_m), 1.0, G, dev).view(1, Lc, s.d_m)
+    W_kv = normal((s.d_m, s.d), s.d_m ** -0.5, G, dev)
+    W_g = normal((s.d_m, s.d), s.d_m ** -0.5, G, dev)
+    b_pos = normal((s.r, s.d), 0.1, G, dev, torch.float32)
+    W_IK = normal((s.d, s.d_I), s.d ** -0.5, G, dev)
+    C = torch.zeros((1, s.T, s.d), dtype=torch.bfloat16, device=dev)
+    Z = torch.empty((1, Lc, s.d), dtype=torch.bfloat16, device=dev)
+    kv = csa.PackedCache(1, n, s.d, s.d_r, dev)
+    ki = csa.PackedCache(1, n, s.d_I, 0, dev)
+    for c in range(nch):
+        csa.compress(x=x, W_kv=W_kv, W_g=W_g, b_pos=b_pos, ratio=s.r, d_rope=s.d_r, rope_theta=10000.0,
+                     pos0=torch.tensor([Lc * c], dtype=torch.int64, device=dev), W_IK=W_IK,
+                     C=C[:, Lc * c:Lc * (c + 1)], Z=Z, kv_cache=kv, ki_cache=ki,
+                     row0=torch.tensor([epc * c], dtype=torch.int32, device=dev))
+    q = normal((1, Lc, s.H, s.d), 1.0, G, dev)
+    q_I = normal((1, Lc, s.H_I, s.d_I), 1.0, G, dev)
+    w = normal((1, Lc, s.H_I), s.H_I ** -0.5, G, dev, torch.float32)
+    n_c = torch.tensor([n], dtype=torch.int32, device=dev)
+    q_pos = (s.T - Lc + torch.arange(Lc, dtype=torch.int64, device=dev)).view(1, Lc)
+    idx, _, _ = csa.index_topk(q_I, w, ki, n_c, q_pos, ratio=s.r, k=s.k)
+    csa.sparse_attn(q, q_pos, kv, n_c, idx, C, torch.zeros((1,), dtype=torch.int64, device=dev), ratio=s.r,
+                    window=s.W)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": "ok", "workload": s.name, "chunk": nch - 1}), flush=True)
+
+
 def run_profile(args):
     """One layer state, `--steps` eager decode steps: the small case ncu captures run on."""
     from compressed_sparse_attention_18_b200.layer import CSADecodeLayer, LayerShape
@@ -996,7 +1035,7 @@ def run_profile(args):
 def main():
     args = parse()
     if args.profile:
-        run_profile(args)
+        run_profile_prefill(args) if args.prefill else run_profile(args)
         return
     if args.rows:
         run_rows(args)

@@ -29,6 +29,7 @@ ENTRY_POINTS = ("csa_status_string", "csa_version", "csa_last_cuda_error", "csa_
 
 _u32, _i32, _f32, _vp = ctypes.c_uint32, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p
 CSA_EARLY_START = 1   # see csa.h: part of a call's work may start before the step's earlier kernels end
+CSA_NO_CLUSTER = 2    # see csa.h: merge a query's split partials through the workspace, not in a cluster
 
 
 class PageMap(ctypes.Structure):
@@ -366,14 +367,14 @@ def _attn_args(q, q_pos, cache: PackedCache, n_c, idx, win_kv, win_pos0, ratio, 
 
 
 def _attn(fn, hca, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse, ws,
-          stream, early_start=False, out_rope_theta=0.0):
+          stream, early_start=False, out_rope_theta=0.0, cluster=True):
     B, Nq, H, d = q.shape
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Nq, H), dtype=torch.float32, device=q.device)
     a = _attn_args(q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse)
-    a.flags = CSA_EARLY_START if early_start else 0
+    a.flags = (CSA_EARLY_START if early_start else 0) | (0 if cluster else CSA_NO_CLUSTER)
     a.out_rope_theta = out_rope_theta
     nbytes = _lib.csa_attn_workspace_size(ctypes.byref(a), hca)
     wbuf = _ws(nbytes, q.device, ws)
@@ -383,13 +384,15 @@ def _attn(fn, hca, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, s
 
 
 def sparse_attn(q, q_pos, cache: PackedCache, n_c, idx, win_kv=None, win_pos0=None, *, ratio=4, window=128,
-                softmax_scale=0.0, out=None, lse=None, ws=None, early_start=False, out_rope_theta=0.0, stream=None):
+                softmax_scale=0.0, out=None, lse=None, ws=None, early_start=False, out_rope_theta=0.0, cluster=True,
+                stream=None):
     """CSA attention over the selected entries idx [B,Nq,k] plus the window.  Returns (out, lse).
     early_start: CSA_EARLY_START (window tiles start before the step's index and top-k kernels end;
     only inside a decode step that began with compress).  out_rope_theta: inverse-RoPE epilogue on the
-    output's RoPE channels at the query position (0 = off)."""
+    output's RoPE channels at the query position (0 = off).  cluster=False: CSA_NO_CLUSTER (split
+    partials merged through the workspace instead of inside a thread-block cluster)."""
     return _attn(_lib.csa_sparse_attn, 0, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window,
-                 softmax_scale, out, lse, ws, stream, early_start, out_rope_theta)
+                 softmax_scale, out, lse, ws, stream, early_start, out_rope_theta, cluster)
 
 
 def hca_attn(q, q_pos, cache: PackedCache, n_c, win_kv=None, win_pos0=None, *, ratio=128, window=128,
@@ -399,7 +402,8 @@ def hca_attn(q, q_pos, cache: PackedCache, n_c, win_kv=None, win_pos0=None, *, r
                  softmax_scale, out, lse, ws, stream, out_rope_theta=out_rope_theta)
 
 
-def attn_workspace_size(q, q_pos, cache, n_c, idx, win_kv, win_pos0, *, ratio, window, hca=False, early_start=False):
+def attn_workspace_size(q, q_pos, cache, n_c, idx, win_kv, win_pos0, *, ratio, window, hca=False, early_start=False,
+                        cluster=True):
     a = _attn_args(q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, 0.0, None, None)
-    a.flags = CSA_EARLY_START if early_start else 0
+    a.flags = (CSA_EARLY_START if early_start else 0) | (0 if cluster else CSA_NO_CLUSTER)
     return _lib.csa_attn_workspace_size(ctypes.byref(a), 1 if hca else 0)

@@ -545,6 +545,7 @@ static csa_status launch_out_rope(uint16_t* out, int H, int D, long long rows, c
 
 // tensor-core decode path (attn_tc.cu)
 void attn_tc_plan(const csa_attn_args* a, int hca, int* splits, int* tpc);
+bool attn_tc_cluster(int splits);
 csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, uint16_t* part_o, float* part_lse,
                           cudaStream_t st);
 
@@ -564,7 +565,8 @@ static AttnPlan plan_attn(const csa_attn_args* a, int hca) {
     p.cps = 1;
     attn_tc_plan(a, hca, &p.splits, &p.tpc);
     size_t o = 0;
-    if (p.splits > 1) {
+    const bool cluster = attn_tc_cluster(p.splits) && !(a->flags & CSA_NO_CLUSTER);
+    if (p.splits > 1 && !cluster) {                       // (a cluster merges its query's partials on chip)
       p.off_o = o;   o = align_up(o + (size_t)rows_tc * p.splits * a->H * a->d * 2, 256);
       p.off_lse = o; o = align_up(o + (size_t)rows_tc * p.splits * a->H * 4, 256);
     }
@@ -640,11 +642,12 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
   CSA_REQUIRE(p.total == 0 || ws != nullptr);
   cudaStream_t st = (cudaStream_t)stream;
   if (p.tc) {
-    uint16_t* po = p.splits > 1 ? (uint16_t*)((uint8_t*)ws + p.off_o) : nullptr;
-    float* pl = p.splits > 1 ? (float*)((uint8_t*)ws + p.off_lse) : nullptr;
+    const bool merged = p.splits == 1 || (attn_tc_cluster(p.splits) && !(a->flags & CSA_NO_CLUSTER));
+    uint16_t* po = !merged ? (uint16_t*)((uint8_t*)ws + p.off_o) : nullptr;
+    float* pl = !merged ? (float*)((uint8_t*)ws + p.off_lse) : nullptr;
     csa_status s = launch_attn_tc(a, hca, p.splits, p.tpc, po, pl, st);
     if (s != CSA_OK) return s;
-    if (p.splits == 1)
+    if (merged)
       return a->out_rope_theta != 0.0f
                  ? launch_out_rope((uint16_t*)a->out, a->H, a->d, rows, a->q_pos, a->out_rope_theta, st)
                  : CSA_OK;

@@ -36,6 +36,7 @@ constexpr uint32_t TA_COL_S = 0;           // S^T: 64 columns
 constexpr uint32_t TA_COL_O = 64;          // O^T: 4 x 64 columns
 constexpr float TA_LOG2E = 1.4426950408889634f;
 constexpr float TA_LN2 = 0.6931471805599453f;
+constexpr int TA_MAX_CLUSTER = 8;          // portable cluster size: queries split over <= 8 CTAs merge in-cluster
 
 struct TaSmem {
   alignas(1024) uint8_t K[8][TA_KEYS * 128];   // [dim block of 64][key][128 B], 128-byte swizzle
@@ -51,11 +52,15 @@ struct TaSmem {
   uint32_t tmem_base;
   uint32_t err;
   int rescale;                                 // some head's running max moved: O and l are rescaled
+  float cf[TA_MAX_CLUSTER][64];                // cluster merge: weight of each CTA's partial per head
+  float cL[64];                                // cluster merge: 1 / total softmax sum per head
 };
 
 struct TaParams {
   int Nq, H, ratio, n_max, k, Wn, window, splits, hca;
   int tpc;              // key tiles per CTA (a CTA walks tiles split*tpc .. split*tpc + tpc - 1 of its query)
+  int cluster;          // the `splits` CTAs of a query form one thread-block cluster and merge their
+                        // partials through distributed shared memory (no workspace partials, no merge kernel)
   int early_rows;       // > 0 (= rows): CTA i < early_rows is split 0 of query i; it walks the query's
                         // window tile before waiting for the previous kernel, then its entry tiles
   float g, scale_log2;
@@ -178,11 +183,13 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // early window: the split-0 CTAs of all queries come first in the grid (they start during the previous
   // kernel and walk the window tile while it runs), then the other splits
+  // (with a cluster per query the CTAs of a query are consecutive: rank = split)
   const bool early = P.early_rows > 0;
-  const bool first_cta = early && (int)blockIdx.x < P.early_rows;
+  const bool by_query = !early || P.cluster;
+  const bool first_cta = early && (P.cluster ? (int)blockIdx.x % P.splits == 0 : (int)blockIdx.x < P.early_rows);
   const int jb = (int)blockIdx.x - P.early_rows;
-  const int bq = !early ? (int)blockIdx.x / P.splits : first_cta ? (int)blockIdx.x : jb / (P.splits - 1);
-  const int split = !early ? (int)blockIdx.x % P.splits : first_cta ? 0 : 1 + jb % (P.splits - 1);
+  const int bq = by_query ? (int)blockIdx.x / P.splits : first_cta ? (int)blockIdx.x : jb / (P.splits - 1);
+  const int split = by_query ? (int)blockIdx.x % P.splits : first_cta ? 0 : 1 + jb % (P.splits - 1);
   const int b = bq / P.Nq;
   // worker thread t owns tile row t/2 for the gather (its half of the row's FP4 blocks and RoPE slice)
   const int grow = (tid & (TA_WORKERS - 1)) >> 1, ghalf = tid & 1;
@@ -266,7 +273,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   tc_fence_after();
   const uint32_t tb = S.tmem_base;
 
-  if (ntile == 0) {                              // nothing in this CTA's tiles: an empty partial
+  if (ntile == 0 && !P.cluster) {               // nothing in this CTA's tiles: an empty partial
     if (P.splits > 1) {
       if (tid < P.H) P.part_lse[unit_ho + tid] = -INFINITY;
     } else {
@@ -278,7 +285,9 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
     return;
   }
 
-  if (warp == 8) {
+  if (ntile == 0) {
+    // an empty member of a cluster: m = -inf, l = 0 (its staged O is never read)
+  } else if (warp == 8) {
     // ------------------------------------------------------------------ control: TMA, then MMA issue
     if (lane == 0) {
       bool ok = true;
@@ -594,15 +603,26 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
     }
     const int hmax = min(32, P.H - hh * 32);
     const int tl = ntile - 1;
+    if (P.cluster) {
+      // stage the unnormalised O (fp32, [head][512 dims]) over the K tile once every O MMA has read it
+      ok = mbar_wait(&S.bar_o[3], tl & 1) && ok;
+      tc_fence_after();
+    }
+    float* stage = reinterpret_cast<float*>(&S.K[0][0]);
 #pragma unroll 1
     for (int mt = 0; mt < 4; ++mt) {
-      ok = mbar_wait(&S.bar_o[mt], tl & 1) && ok;
-      tc_fence_after();
+      if (!P.cluster) {
+        ok = mbar_wait(&S.bar_o[mt], tl & 1) && ok;
+        tc_fence_after();
+      }
       uint32_t ov[32];
       tmem_ld_x32(lane_base + TA_COL_O + 64 * mt + hh * 32, ov);
       tmem_wait_ld_x32(ov);
       const int dim = 128 * mt + 32 * quad + lane;
-      if (P.splits == 1) {
+      if (P.cluster) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stage[(hh * 32 + j) * 512 + dim] = __uint_as_float(ov[j]);
+      } else if (P.splits == 1) {
         uint16_t* o = P.out + ((size_t)bq * P.H + hh * 32) * 512 + dim;
 #pragma unroll
         for (int j = 0; j < 32; ++j)
@@ -615,7 +635,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       }
     }
     if (!ok && lane == 0) atomicOr(&S.err, 1u);
-    if (tid < P.H) {
+    if (tid < P.H && !P.cluster) {
       const float lh = S.l[tid];
       const float ls = lh > 0.f ? (S.m[tid] + log2f(lh)) * TA_LN2 : -INFINITY;
       if (P.splits == 1) {
@@ -627,6 +647,76 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
     tc_fence_before();
   }
   if (first_cta && tid == 0) pdl_wait();         // the grid completes only after its predecessor
+  if (P.cluster) {
+    // ---- merge of the query's partials inside its cluster: every CTA's m, l (per head) and staged O
+    // are visible after the barrier; CTA `split` writes dims [d0, d1) of the output
+    cluster_sync_all();
+    const int ns = P.splits;
+    if (tid < 64) {
+      float mr[TA_MAX_CLUSTER], lr[TA_MAX_CLUSTER], M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < TA_MAX_CLUSTER; ++r) {
+        mr[r] = -INFINITY;
+        lr[r] = 0.f;
+        if (r < ns) {
+          mr[r] = ld_peer_f32(peer_addr(&S.m[tid], r));
+          lr[r] = ld_peer_f32(peer_addr(&S.l[tid], r));
+          if (lr[r] > 0.f) M = fmaxf(M, mr[r]);
+        }
+      }
+      float L = 0.f;
+#pragma unroll
+      for (int r = 0; r < TA_MAX_CLUSTER; ++r) {
+        const float f = (r < ns && lr[r] > 0.f) ? exp2f(mr[r] - M) : 0.f;
+        S.cf[r][tid] = f;
+        L += f * lr[r];
+      }
+      S.cL[tid] = L > 0.f ? 1.f / L : 0.f;
+      if (split == 0 && P.lse && tid < P.H) P.lse[(size_t)bq * P.H + tid] = L > 0.f ? (M + log2f(L)) * TA_LN2 : -INFINITY;
+    }
+    __syncthreads();
+    const int per = ((512 + ns - 1) / ns + 3) & ~3;
+    const int d0 = min(512, split * per), d1 = min(512, d0 + per);
+    const int groups = (d1 - d0) >> 2;
+    uint32_t base[TA_MAX_CLUSTER];
+#pragma unroll
+    for (int r = 0; r < TA_MAX_CLUSTER; ++r) base[r] = r < ns ? peer_addr(&S.K[0][0], r) : 0u;
+    // two outputs per thread per round, all their peer loads issued before the first is used
+    const int items = P.H * groups;
+    for (int it0 = tid; it0 < items; it0 += 2 * TA_THREADS) {
+      float4 v[2][TA_MAX_CLUSTER];
+      int hs[2], ds[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int it = it0 + u * TA_THREADS;
+        hs[u] = it < items ? it / groups : 0;
+        ds[u] = d0 + 4 * (it < items ? it % groups : 0);
+#pragma unroll
+        for (int r = 0; r < TA_MAX_CLUSTER; ++r)
+          v[u][r] = (it < items && r < ns && S.cf[r][hs[u]] != 0.f)
+                        ? ld_peer_v4(base[r] + (uint32_t)((hs[u] * 512 + ds[u]) * 4))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (it0 + u * TA_THREADS >= items) continue;
+        const int h = hs[u];
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < TA_MAX_CLUSTER; ++r) {
+          const float f = r < ns ? S.cf[r][h] : 0.f;
+          acc.x = fmaf(f, v[u][r].x, acc.x); acc.y = fmaf(f, v[u][r].y, acc.y);
+          acc.z = fmaf(f, v[u][r].z, acc.z); acc.w = fmaf(f, v[u][r].w, acc.w);
+        }
+        const float il = S.cL[h];
+        uint2 o2;
+        o2.x = pack_bf16x2(acc.x * il, acc.y * il);
+        o2.y = pack_bf16x2(acc.z * il, acc.w * il);
+        *reinterpret_cast<uint2*>(P.out + ((size_t)bq * P.H + h) * 512 + ds[u]) = o2;
+      }
+    }
+    cluster_sync_all();                          // the peers have read this CTA's shared memory
+  }
   __syncthreads();
   if (warp == 8) {
     if (S.err && lane == 0) atomicOr(&g_csa_device_error, 1u);
@@ -659,6 +749,9 @@ void attn_tc_plan(const csa_attn_args* a, int hca, int* splits, int* tpc) {
   *tpc = (int)t;
   *splits = (int)((tiles + t - 1) / t);
 }
+
+// Queries split over 2..8 CTAs merge inside a thread-block cluster (no workspace, no merge kernel).
+bool attn_tc_cluster(int splits) { return splits >= 2 && splits <= TA_MAX_CLUSTER; }
 
 bool attn_tc_eligible(const csa_attn_args* a, int hca, int max_splits) {
   int splits = 0, tpc = 0;
@@ -705,6 +798,7 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
   P.Nq = a->Nq; P.H = a->H; P.ratio = a->ratio; P.n_max = a->n_max; P.k = hca ? 0 : a->k;
   P.Wn = Wn; P.window = a->window; P.splits = splits; P.tpc = tpc; P.hca = hca; P.g = a->g_kv;
   P.early_rows = attn_tc_early(a, hca) ? (int)rows : 0;
+  P.cluster = (attn_tc_cluster(splits) && !(a->flags & CSA_NO_CLUSTER)) ? 1 : 0;
   const float scale = a->softmax_scale != 0.0f ? a->softmax_scale : 1.0f / sqrtf((float)a->d);
   P.scale_log2 = scale * TA_LOG2E;
   P.q_pos = a->q_pos; P.codes = a->kv_codes; P.scales = a->kv_scales;
@@ -721,7 +815,21 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
   const int smem = (int)sizeof(TaSmem) + 1024;
   static std::atomic<unsigned> attr_done{0};
   set_smem_once((const void*)attn_tc_kernel, smem, attr_done);
-  return launch_pdl(attn_tc_kernel, dim3((unsigned)(rows * splits)), dim3(TA_THREADS), (size_t)smem, st, qmap, wmap, P);
+  if (!P.cluster)
+    return launch_pdl(attn_tc_kernel, dim3((unsigned)(rows * splits)), dim3(TA_THREADS), (size_t)smem, st, qmap, wmap, P);
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = pdl_config(dim3((unsigned)(rows * splits)), dim3(TA_THREADS), (size_t)smem, st, attr);
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)splits;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, qmap, wmap, P);
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return CSA_ERR_CUDA;
+  }
+  return launch_status();
 }
 
 

@@ -269,19 +269,21 @@ __global__ void __launch_bounds__(IDX_WARPS * 32) index_score_kernel(
 // candidate lists).  MSB-first radix passes with 8-bit digits find the threshold, then every element
 // above it is emitted and the ties are taken in (id, position) order.
 
-struct TopkSmem {
+template <int NW>                           // warps of the block
+struct TopkSmemT {
   uint32_t hist[256];
-  uint32_t whist[TOPK_THREADS / 32][256];   // per-warp histograms: contention only inside a warp
-  uint32_t scan[TOPK_THREADS / 32];
+  uint32_t whist[NW][256];                  // per-warp histograms: contention only inside a warp
+  uint32_t scan[NW];
   uint32_t bcast[4];
   uint32_t counter;
   uint32_t tie_taken;
 };
+using TopkSmem = TopkSmemT<TOPK_THREADS / 32>;
 
 // Find the R-th largest value of key(j) over positions j < n with filt(j).  Returns the threshold
 // key; *n_above = number of filtered elements with key > threshold.
-template <class KeyF, class FiltF>
-__device__ uint32_t radix_threshold(TopkSmem& sm, int n, uint32_t R, KeyF key, FiltF filt, uint32_t* n_above) {
+template <class SM, class KeyF, class FiltF>
+__device__ uint32_t radix_threshold(SM& sm, int n, uint32_t R, KeyF key, FiltF filt, uint32_t* n_above) {
   uint32_t prefix = 0, mask = 0, rem = R;
   for (int shift = 24; shift >= 0; shift -= 8) {
     const int nw = blockDim.x >> 5, wid = threadIdx.x >> 5;
@@ -347,7 +349,8 @@ __device__ uint32_t radix_threshold(TopkSmem& sm, int n, uint32_t R, KeyF key, F
 }
 
 // Exclusive block scan of one value per thread; returns the prefix, *total = sum.
-__device__ uint32_t block_exclusive_scan(TopkSmem& sm, uint32_t v, uint32_t* total) {
+template <class SM>
+__device__ uint32_t block_exclusive_scan(SM& sm, uint32_t v, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
 #pragma unroll
@@ -403,8 +406,8 @@ struct TopkRowArgs {
 // Select the K largest of keys[0..len) (0 = not a candidate; nvalid candidates in all) by (key desc,
 // id asc), writing ids / scores to oi[base + slot], os[base + slot] in unspecified order.  Candidates
 // with equal key and equal id (a repeated id) are interchangeable: any of them gives the same output.
-template <class IdF>
-__device__ void select_in_smem(TopkSmem& sm, const uint32_t* keys, int len, uint32_t K, uint32_t nvalid, IdF idof,
+template <class SM, class IdF>
+__device__ void select_in_smem(SM& sm, const uint32_t* keys, int len, uint32_t K, uint32_t nvalid, IdF idof,
                                int32_t* oi, float* os, uint32_t base) {
   auto valid = [&](int j) { return keys[j] != 0u; };
   uint32_t T1 = 0, above1 = 0, T2 = 0xFFFFFFFFu, need_pos = 0;
@@ -451,7 +454,8 @@ __device__ void select_in_smem(TopkSmem& sm, const uint32_t* keys, int len, uint
 
 // Load one row segment into shared memory as order-preserving keys (0 = not a candidate) and, with
 // explicit ids, the ids; returns the number of candidates.  8 independent loads in flight per thread.
-__device__ uint32_t load_row_keys(TopkSmem& sm, const float* __restrict__ src, const int32_t* __restrict__ isrc,
+template <class SM>
+__device__ uint32_t load_row_keys(SM& sm, const float* __restrict__ src, const int32_t* __restrict__ isrc,
                                   int len, uint32_t* keys, int32_t* ids) {
   uint32_t nvalid_loc = 0;
   constexpr int U = 8;
@@ -479,9 +483,13 @@ __device__ uint32_t load_row_keys(TopkSmem& sm, const float* __restrict__ src, c
   return nvalid;
 }
 
-__global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(TopkRowArgs A) {
+// THREADS x one row segment of at most CAP scores (CAP ids after them for explicit-id rows): the full
+// 1024-thread kernel for segments up to 32768 scores, a 256-thread one with row-sized shared memory
+// (several CTAs per SM) for rows of at most 8192 (multi-query prefill rows, candidate lists).
+template <int THREADS, int CAP>
+__global__ void __launch_bounds__(THREADS) topk_kernel(TopkRowArgs A) {
   extern __shared__ __align__(16) uint32_t s_keys[];
-  __shared__ TopkSmem sm;
+  __shared__ TopkSmemT<THREADS / 32> sm;
   const int seg = blockIdx.x;                  // segment (chunk) of the row
   const int row = blockIdx.y;
   if (A.skip && A.skip[row].ok) return;        // selected by the long-row histogram pass
@@ -495,7 +503,7 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(TopkRowArgs A) {
   }
   if (len < 0) len = 0;
   uint32_t* keys = s_keys;
-  int32_t* ids = reinterpret_cast<int32_t*>(s_keys + (A.in_ids ? TOPK_CHUNK_IDS : 0));
+  int32_t* ids = reinterpret_cast<int32_t*>(s_keys + (A.in_ids ? CAP : 0));
   const float* src = A.in_scores + row * A.in_ld + col0;
   const int32_t* isrc = A.in_ids ? A.in_ids + row * A.in_ld + col0 : nullptr;
   const uint32_t nvalid = load_row_keys(sm, src, isrc, len, keys, ids);
@@ -968,6 +976,9 @@ bool index_tc_eligible(const csa_index_args* a);
 csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, uint32_t* hist, cudaStream_t st);
 bool index_mq_tc_eligible(const csa_index_args* a);
 csa_status run_scores_mq_tc(const csa_index_args* a, float* scores, long long ld, cudaStream_t st);
+// fused decode indexer + top-k in one cluster per row (index_tc.cu)
+bool index_topk_fused_eligible(const csa_index_args* a);
+csa_status run_index_topk_fused(const csa_index_args* a, cudaStream_t st);
 
 // ------------------------------------------------------------------------------ orchestration
 struct IndexPlan {
@@ -1083,13 +1094,24 @@ static csa_status run_scores(const csa_index_args* a, float* scores, long long l
   return launch_status();
 }
 
+constexpr int TOPK_SHORT = 8192;        // rows up to this length go to the 256-thread kernel
+constexpr int TOPK_SHORT_THREADS = 256;
+
 static csa_status launch_topk(TopkRowArgs ta, int rows, int segs, bool ids, cudaStream_t st) {
   static_assert(TOPK_CHUNK_IDS * 8 == TOPK_CHUNK * 4, "one shared-memory size for both row kinds");
+  dim3 grid(segs, rows);
+  if (segs == 1 && ta.rows_per_seg <= TOPK_SHORT) {
+    // shared memory sized to the row: keys of rows_per_seg columns (explicit ids follow at TOPK_SHORT)
+    const size_t smem = ids ? (size_t)TOPK_SHORT * 8 : align_up((size_t)ta.rows_per_seg, 4) * 4;
+    static std::atomic<unsigned> attr_s{0};
+    set_smem_once((const void*)topk_kernel<TOPK_SHORT_THREADS, TOPK_SHORT>, TOPK_SHORT * 8, attr_s);
+    topk_kernel<TOPK_SHORT_THREADS, TOPK_SHORT><<<grid, TOPK_SHORT_THREADS, smem, st>>>(ta);
+    return launch_status();
+  }
   const size_t smem = (size_t)TOPK_CHUNK * 4;
   static std::atomic<unsigned> attr_done{0};
-  set_smem_once((const void*)topk_kernel, (int)smem, attr_done);
-  dim3 grid(segs, rows);
-  topk_kernel<<<grid, TOPK_THREADS, smem, st>>>(ta);
+  set_smem_once((const void*)topk_kernel<TOPK_THREADS, TOPK_CHUNK_IDS>, (int)smem, attr_done);
+  topk_kernel<TOPK_THREADS, TOPK_CHUNK_IDS><<<grid, TOPK_THREADS, smem, st>>>(ta);
   return launch_status();
 }
 
@@ -1307,6 +1329,7 @@ extern "C" csa_status csa_index_topk(const csa_index_args* a, void* ws, size_t w
   if (v != CSA_OK) return v;
   const IndexPlan p = plan_index(a);
   if (p.rows == 0) return CSA_OK;
+  if (index_topk_fused_eligible(a)) return run_index_topk_fused(a, (cudaStream_t)stream);   // no workspace used
   CSA_REQUIRE(ws != nullptr);
   if (ws_bytes < p.total) return CSA_ERR_WORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;

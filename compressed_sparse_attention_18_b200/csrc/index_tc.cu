@@ -46,15 +46,28 @@ static_assert(TC_COL_D + 16 * TC_NBUF <= TC_COL_SFA && TC_COL_SFA + 16 * TC_NBUF
               "tensor-memory plan");
 constexpr int TC_HIST_BINS = 4096, TC_HIST_SHIFT = 20;
 
-struct TcSmem {
-  alignas(1024) uint8_t codes[TC_STAGES][TC_CODE_BYTES];
+// FUSED: the decode row is scored by a cluster of FT_CLUSTER CTAs that keep their scores in shared memory
+// and select the row's top-k themselves (no score row in global memory, no separate top-k kernel).
+constexpr int FT_CLUSTER = 8;
+constexpr int FT_SCAP = 4096;                    // scores one CTA holds (16 tiles): rows up to 32768 keys
+constexpr int FT_CAND = 4096;                    // boundary-bin candidates gathered in CTA 0 (its code stages)
+
+template <bool FUSED>
+struct TcSmemT {
+  static constexpr int STAGES = FUSED ? 4 : TC_STAGES;   // fused: 2 CTAs per SM, 8 per row, 4 tiles in flight each
+  alignas(1024) uint8_t codes[STAGES][TC_CODE_BYTES];
   alignas(1024) uint8_t qtile[8 * 64];
-  alignas(16) uint8_t sc[TC_STAGES][TC_SC_BYTES];
+  alignas(16) uint8_t sc[STAGES][TC_SC_BYTES];
   uint32_t hist[TC_HIST_BINS];
+  float scores[FUSED ? FT_SCAP : 1];             // fused: scores of this CTA's keys [key_lo, key_lo + nk)
+  uint32_t gsl[FUSED ? TC_HIST_BINS / FT_CLUSTER : 1];   // fused: this CTA's slice of the row histogram
+  uint32_t h256[FUSED ? 256 : 1];
+  uint32_t stot, a_cnt, e_cnt, ctr0, ctr1, ctr2;
+  uint32_t bc[8];
   float wq[8];
   uint8_t qsc[8][4];
-  alignas(8) uint64_t full[TC_STAGES];
-  alignas(8) uint64_t empty[TC_STAGES];
+  alignas(8) uint64_t full[STAGES];
+  alignas(8) uint64_t empty[STAGES];
   alignas(8) uint64_t sfa_full[TC_NBUF];
   alignas(8) uint64_t acc_full[TC_NBUF];
   alignas(8) uint64_t acc_empty[TC_NBUF];
@@ -76,6 +89,9 @@ struct TcParams {
   int early;                // read q_I, w, n_c, q_pos and key rows below n_c[b] - 1 before the wait
   float g_q, gg;
   csa_page_map pm;          // key rows (table == NULL: contiguous [B][n_max])
+  int32_t* idx_out;         // fused: [B][k]
+  float* scores_out;        // fused: [B][k] or null
+  int k;
 };
 
 // FP4-quantise 32 elements held one per lane (pack rule, global scale g); returns this lane's code.
@@ -87,10 +103,16 @@ __device__ __forceinline__ uint32_t quant_lane(float x, float g, uint32_t* s_cod
   return s != 0.0f ? f32_to_e2m1(__fdiv_rn(x, __fmul_rn(s, g))) : 0u;
 }
 
+template <class SM>
+__device__ void fused_select(SM& S, const TcParams& P, int b, int n_vis, int key_lo, int nk, int span);
+
+template <bool FUSED>
 __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                        const TcParams P) {
+  using SM = TcSmemT<FUSED>;
+  constexpr int TC_STAGES = SM::STAGES;
   extern __shared__ uint8_t smem_raw[];
-  TcSmem& S = *reinterpret_cast<TcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SM& S = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   // setup that reads no global memory, then wait for the previous kernel (it may append to the cache)
@@ -104,6 +126,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
     }
     mbar_init(&S.q_ready, 4);
     fence_mbar_init();
+    S.stot = 0; S.a_cnt = 0; S.e_cnt = 0; S.ctr0 = 0; S.ctr1 = 0; S.ctr2 = 0;
   }
   if (warp == 0 && lane == 0) prefetch_tensormap(&kmap);
   for (int i = threadIdx.x; i < TC_HIST_BINS; i += blockDim.x) S.hist[i] = 0;
@@ -255,7 +278,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
     float wq[8];
 #pragma unroll
     for (int h = 0; h < 8; ++h) wq[h] = S.wq[h];
-    float* srow = P.scores + (size_t)b * P.ld;
+    float* srow = FUSED ? nullptr : P.scores + (size_t)b * P.ld;
+    const int key_lo = t_begin * TC_TILE;
     uint32_t d[16];
     auto finish = [&](int i) {
       // d holds tile i's accumulators (issued by the caller): release them, then score
@@ -271,8 +295,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
 #pragma unroll
           for (int h = 0; h < 8; ++h) sc = fmaf(wq[h], fmaxf(__uint_as_float(d[8 * u + h]), 0.f), sc);
           sc += 0.0f;
-          srow[key] = sc;
-          if (P.hist) atomicAdd(&S.hist[float_order_key(sc) >> TC_HIST_SHIFT], 1u);
+          if constexpr (FUSED) {
+            S.scores[key - key_lo] = sc;
+            atomicAdd(&S.hist[float_order_key(sc) >> TC_HIST_SHIFT], 1u);
+          } else {
+            srow[key] = sc;
+            if (P.hist) atomicAdd(&S.hist[float_order_key(sc) >> TC_HIST_SHIFT], 1u);
+          }
         }
       }
     };
@@ -311,7 +340,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
   __syncthreads();
   if (P.early && threadIdx.x == 0) pdl_wait();   // this grid completes only after its predecessor
   if (S.err && threadIdx.x == 0) atomicOr(&g_csa_device_error, 1u);
-  if (P.hist && S.err == 0) {
+  if constexpr (FUSED) {
+    const int key_lo = t_begin * TC_TILE;
+    fused_select(S, P, b, n_vis, key_lo, max(0, min(n_vis, t_end * TC_TILE) - key_lo), per * TC_TILE);
+  } else if (P.hist && S.err == 0) {
     uint32_t* h = P.hist + (size_t)b * TC_HIST_BINS;
     for (int i = threadIdx.x; i < TC_HIST_BINS; i += blockDim.x) {
       const uint32_t c = S.hist[i];
@@ -322,6 +354,238 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
     tc_fence_after();
     tmem_dealloc(tbase, TC_TMEM_COLS);
   }
+}
+
+// ------------------------------------------------------------------------- fused top-k selection
+// The CTAs of the row's cluster hold its scores; k_eff = min(k, n_vis) of them are selected by (score desc,
+// key id asc) without leaving the chip:
+//   1. the row histogram (top 12 bits of the order-preserving key, each CTA's own counts) is summed in
+//      slices over the cluster, and every CTA finds the bin T holding the k_eff-th score;
+//   2. each CTA writes its keys above T at slots from a prefix over the cluster's counts;
+//   3. the keys in bin T: all of them when exactly needed, else they are gathered in CTA 0 (or, past
+//      FT_CAND of them, read from the peers in place) and CTA 0 resolves them exactly by 8-bit digits of
+//      the composite (order key, ~id) below the bin's bits.
+// Every CTA executes every cluster barrier, whatever its own state.
+struct FtCand {
+  uint32_t key;
+  int32_t id;
+};
+
+// Resolve `need` of the candidates get(j) (j < n; false = not a candidate) in CTA 0: composite v = key << 32 |
+// ~id, all sharing the top 12 key bits; written at oi / os[base + ...] (S.ctr2 counts the slots used).
+template <class SM, class Get>
+__device__ void fused_resolve(SM& S, int n, uint32_t need, uint32_t base, Get get, int32_t* oi, float* os) {
+  const uint32_t limit = base + need;                   // slots of this resolution: [base, base + need)
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint64_t prefix = 0, mask = 0;
+  bool done = false;
+  // digits of the 52 bits below the bin: [51:44] [43:36] [35:28] [27:20] [19:12] [11:4], then [3:0]
+#pragma unroll 1
+  for (int lv = 0; lv < 7 && !done; ++lv) {
+    const int sh = lv < 6 ? 44 - 8 * lv : 0;
+    const uint32_t dm = lv < 6 ? 255u : 15u;
+    for (int i = tid; i < 256; i += blockDim.x) S.h256[i] = 0;
+    __syncthreads();
+    for (int j = tid; j < n; j += blockDim.x) {
+      FtCand c;
+      if (!get(j, c)) continue;
+      const uint64_t v = ((uint64_t)c.key << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)c.id);
+      if ((v & mask) == prefix) atomicAdd(&S.h256[(uint32_t)(v >> sh) & dm], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l owns digits 8 (31 - l) .. + 7, highest first
+      uint32_t c[8], tot = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { c[i] = S.h256[8 * (31 - lane) + 7 - i]; tot += c[i]; }
+      uint32_t incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      uint32_t acc = incl - tot;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (acc < need && acc + c[i] >= need) { S.bc[4] = 8 * (31 - lane) + 7 - i; S.bc[5] = acc; S.bc[6] = c[i]; }
+        acc += c[i];
+      }
+    }
+    __syncthreads();
+    const uint32_t digit = S.bc[4], above = S.bc[5], cnt = S.bc[6];
+    const uint64_t nprefix = prefix | ((uint64_t)digit << sh), nmask = mask | ((uint64_t)dm << sh);
+    done = need == above + cnt;                          // every candidate of the threshold digit is taken
+    for (int j = tid; j < n; j += blockDim.x) {
+      FtCand c;
+      if (!get(j, c)) continue;
+      const uint64_t v = ((uint64_t)c.key << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)c.id);
+      if ((v & mask) != prefix) continue;
+      const uint32_t dj = (uint32_t)(v >> sh) & dm;
+      if (dj > digit || (done && dj == digit)) {
+        const uint32_t slot = base + atomicAdd(&S.ctr2, 1u);
+        if (slot < limit) {                             // (always, unless a bounded wait gave up upstream)
+          oi[slot] = c.id;
+          if (os) os[slot] = order_key_float(c.key);
+        }
+      }
+    }
+    need -= above;
+    prefix = nprefix;
+    mask = nmask;
+    __syncthreads();
+  }
+}
+
+// span = keys per CTA of the row (CTA r holds keys [r span, r span + span) of those visible)
+template <class SM>
+__device__ void fused_select(SM& S, const TcParams& P, int b, int n_vis, int key_lo, int nk, int span) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t rank = blockIdx.x, nr = gridDim.x;              // the cluster spans blockIdx.x
+  const uint32_t K = (uint32_t)min(P.k, n_vis);
+  int32_t* oi = P.idx_out + (size_t)b * P.k;
+  float* os = P.scores_out ? P.scores_out + (size_t)b * P.k : nullptr;
+  if (rank == 0)
+    for (int j = (int)K + tid; j < P.k; j += blockDim.x) {
+      oi[j] = -1;
+      if (os) os[j] = -INFINITY;
+    }
+  constexpr int SL = TC_HIST_BINS / FT_CLUSTER;
+  // (1) every CTA's histogram is complete
+  cluster_sync_all();
+  {
+    uint32_t part = 0;
+    for (int i = tid; i < SL; i += blockDim.x) {
+      uint32_t v = 0;
+      for (uint32_t r = 0; r < nr; ++r) v += ld_peer_u32(peer_addr(&S.hist[rank * SL + i], r));
+      S.gsl[i] = v;
+      part += v;
+    }
+    part = __reduce_add_sync(0xffffffffu, part);
+    if (lane == 0 && part) atomicAdd(&S.stot, part);
+  }
+  // (2) the slices of the row histogram are complete
+  cluster_sync_all();
+  if (warp == 0 && K > 0) {
+    // slice holding the K-th score (slices of higher bins on higher ranks), then its bin
+    const uint32_t tot = lane < (int)nr ? ld_peer_u32(peer_addr(&S.stot, lane)) : 0u;
+    uint32_t suf = tot;                                          // sum over ranks >= lane
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, suf, o);
+      if (lane + o < 32) suf += y;
+    }
+    const uint32_t above_s = suf - tot;
+    const uint32_t hit = __ballot_sync(0xffffffffu, lane < (int)nr && above_s < K && K <= suf);
+    const int sl = hit ? __ffs(hit) - 1 : 0;
+    const uint32_t above_sl = __shfl_sync(0xffffffffu, above_s, sl);
+    uint32_t bins[SL / 32], lt = 0;
+#pragma unroll
+    for (int i = 0; i < SL / 32; ++i) {
+      bins[i] = ld_peer_u32(peer_addr(&S.gsl[(SL / 32) * lane + i], sl));
+      lt += bins[i];
+    }
+    uint32_t lsuf = lt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, lsuf, o);
+      if (lane + o < 32) lsuf += y;
+    }
+    uint32_t acc = above_sl + lsuf - lt;
+#pragma unroll
+    for (int i = SL / 32 - 1; i >= 0; --i) {
+      if (acc < K && acc + bins[i] >= K) {
+        S.bc[0] = (uint32_t)(sl * SL + (SL / 32) * lane + i);
+        S.bc[1] = acc;
+        S.bc[2] = bins[i];
+      }
+      acc += bins[i];
+    }
+  }
+  __syncthreads();
+  const uint32_t T = S.bc[0], above = K > 0 ? S.bc[1] : 0u;
+  // (3) this CTA's keys above T and in T
+  if (K > 0) {
+    uint32_t a = 0, e = 0;
+    for (int i = tid; i < nk; i += blockDim.x) {
+      const uint32_t bin = float_order_key(S.scores[i]) >> TC_HIST_SHIFT;
+      a += bin > T;
+      e += bin == T;
+    }
+    a = __reduce_add_sync(0xffffffffu, a);
+    e = __reduce_add_sync(0xffffffffu, e);
+    if (lane == 0) {
+      if (a) atomicAdd(&S.a_cnt, a);
+      if (e) atomicAdd(&S.e_cnt, e);
+    }
+  }
+  cluster_sync_all();
+  // (4) slots: prefix of the counts over lower ranks
+  if (warp == 0) {
+    const uint32_t a = lane < (int)nr ? ld_peer_u32(peer_addr(&S.a_cnt, lane)) : 0u;
+    const uint32_t e = lane < (int)nr ? ld_peer_u32(peer_addr(&S.e_cnt, lane)) : 0u;
+    uint32_t pa = a, pe = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t ya = __shfl_up_sync(0xffffffffu, pa, o), ye = __shfl_up_sync(0xffffffffu, pe, o);
+      if (lane >= o) { pa += ya; pe += ye; }
+    }
+    const uint32_t E = __shfl_sync(0xffffffffu, pe, 31);
+    if (lane == (int)rank) { S.bc[4] = pa - a; S.bc[5] = pe - e; }
+    if (lane == 0) S.bc[6] = E;
+  }
+  __syncthreads();
+  const uint32_t pa = S.bc[4], pe = S.bc[5], E = S.bc[6];
+  const uint32_t need = K - above;
+  const bool take_all = need == E;
+  const bool gather = K > 0 && !take_all && E <= FT_CAND;
+  FtCand* cand = reinterpret_cast<FtCand*>(&S.codes[0][0]);           // CTA 0's buffer (code stages are idle)
+  static_assert(sizeof(S.codes) >= FT_CAND * sizeof(FtCand), "candidate buffer");
+  if (K > 0) {
+    for (int i = tid; i < nk; i += blockDim.x) {
+      const float v = S.scores[i];
+      const uint32_t key = float_order_key(v), bin = key >> TC_HIST_SHIFT;
+      // (slot checks hold by construction; they keep a row whose streaming gave up inside its k slots)
+      if (bin > T) {
+        const uint32_t slot = pa + atomicAdd(&S.ctr0, 1u);
+        if (slot < above) {
+          oi[slot] = key_lo + i;
+          if (os) os[slot] = v;
+        }
+      } else if (bin == T) {
+        const uint32_t j = pe + atomicAdd(&S.ctr1, 1u);
+        if (take_all) {
+          if (above + j < K) {
+            oi[above + j] = key_lo + i;
+            if (os) os[above + j] = v;
+          }
+        } else if (gather && j < E) {
+          st_peer_u32(peer_addr(&cand[j].key, 0), key);
+          st_peer_u32(peer_addr(&cand[j].id, 0), (uint32_t)(key_lo + i));
+        }
+      }
+    }
+  }
+  // (5) the boundary candidates are in CTA 0 (or in place)
+  cluster_sync_all();
+  if (rank == 0 && K > 0 && !take_all) {
+    if (gather) {
+      fused_resolve(S, (int)E, need, above, [&](int j, FtCand& c) { c = cand[j]; return true; }, oi, os);
+    } else {
+      // more candidates than the buffer: read them where they are (rank r holds keys r span + i), filtered
+      // by bin T
+      fused_resolve(S, (int)(nr * span), need, above, [&](int j, FtCand& c) {
+        const uint32_t r = (uint32_t)j / (uint32_t)span, i = (uint32_t)j % (uint32_t)span;
+        const uint32_t lo = r * (uint32_t)span;
+        if (lo + i >= (uint32_t)n_vis) return false;
+        const float v = __uint_as_float(ld_peer_u32(peer_addr(&S.scores[i], r)));
+        c.key = float_order_key(v);
+        c.id = (int32_t)(lo + i);
+        return (c.key >> TC_HIST_SHIFT) == T;
+      }, oi, os);
+    }
+  }
+  // (6) the peers are done with this CTA's shared memory
+  cluster_sync_all();
 }
 
 // --------------------------------------------------------------------------------------- host
@@ -348,42 +612,83 @@ bool index_tc_eligible(const csa_index_args* a) {
          tensor_map_encoder() != nullptr;
 }
 
-csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, uint32_t* hist, cudaStream_t st) {
-  CUtensorMap map;
+static bool encode_key_map(const csa_index_args* a, CUtensorMap* map) {
   const cuuint64_t gdim[2] = {64, (cuuint64_t)cache_rows(a->k_pages, a->B, a->n_max)};
   const cuuint64_t gstride[1] = {64};
   const cuuint32_t box[2] = {64, TC_SUB};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = tensor_map_encoder()(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void*)a->k_codes, gdim, gstride, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return CSA_ERR_CUDA;
+  return tensor_map_encoder()(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void*)a->k_codes, gdim, gstride, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static TcParams tc_params(const csa_index_args* a) {
   TcParams P{};
   P.q_I = (const uint16_t*)a->q_I;
   P.w = a->w;
   P.k_scales = a->k_scales;
   P.n_c = a->n_c;
   P.q_pos = a->q_pos;
-  P.scores = scores;
-  P.hist = hist;
-  P.ld = ld;
   P.n_max = a->n_max;
   P.ratio = a->ratio;
   P.H_I = a->H_I;
   P.g_q = a->g_q;
   P.gg = a->g_q * a->g_k;
   P.pm = a->k_pages;
+  P.early = (a->flags & CSA_EARLY_START) ? 1 : 0;
+  return P;
+}
+
+csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, uint32_t* hist, cudaStream_t st) {
+  CUtensorMap map;
+  if (!encode_key_map(a, &map)) return CSA_ERR_CUDA;
+  TcParams P = tc_params(a);
+  P.scores = scores;
+  P.hist = hist;
+  P.ld = ld;
   // TC_CTAS_PER_SM resident CTAs per SM: one wave, at most one per tile
   const int tiles_row = (a->n_max + TC_TILE - 1) / TC_TILE;
   int per_row = (TC_CTAS_PER_SM * 148) / a->B;
   if (per_row > tiles_row) per_row = tiles_row;
   if (per_row < 1) per_row = 1;
   P.ctas_per_row = per_row;
-  P.early = (a->flags & CSA_EARLY_START) ? 1 : 0;
-  const int smem = (int)sizeof(TcSmem) + 1024;
+  const int smem = (int)sizeof(TcSmemT<false>) + 1024;
   static std::atomic<unsigned> attr_done{0};
-  set_smem_once((const void*)index_score_tc_kernel, smem, attr_done);
-  return launch_pdl(index_score_tc_kernel, dim3(per_row, a->B), dim3(TC_THREADS), smem, st, map, P);
+  set_smem_once((const void*)index_score_tc_kernel<false>, smem, attr_done);
+  return launch_pdl(index_score_tc_kernel<false>, dim3(per_row, a->B), dim3(TC_THREADS), smem, st, map, P);
+}
+
+// Fused decode indexer + top-k: single-query Full rows of at most FT_CLUSTER x FT_SCAP keys, no pool.
+bool index_topk_fused_eligible(const csa_index_args* a) {
+  return index_tc_eligible(a) && a->pool_blocks == 0 && a->idx_out != nullptr &&
+         a->n_max <= FT_CLUSTER * FT_SCAP && a->k >= 1 && a->k <= 4096;
+}
+
+csa_status run_index_topk_fused(const csa_index_args* a, cudaStream_t st) {
+  CUtensorMap map;
+  if (!encode_key_map(a, &map)) return CSA_ERR_CUDA;
+  TcParams P = tc_params(a);
+  P.idx_out = a->idx_out;
+  P.scores_out = a->scores_out;
+  P.k = a->k;
+  P.ctas_per_row = FT_CLUSTER;
+  static_assert(FT_CLUSTER * FT_SCAP >= FT_CLUSTER * TC_TILE && FT_SCAP % TC_TILE == 0, "tile split");
+  const int smem = (int)sizeof(TcSmemT<true>) + 1024;
+  static std::atomic<unsigned> attr_done{0};
+  set_smem_once((const void*)index_score_tc_kernel<true>, smem, attr_done);
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = pdl_config(dim3(FT_CLUSTER, a->B), dim3(TC_THREADS), (size_t)smem, st, attr);
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = FT_CLUSTER;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, index_score_tc_kernel<true>, map, P);
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return CSA_ERR_CUDA;
+  }
+  return launch_status();
 }
 
 }  // namespace csa

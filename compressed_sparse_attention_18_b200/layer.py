@@ -6,8 +6,9 @@ layer's hot path (sources: "DeepSeek-V4: エージェントが実際に使える
 Fig. 3): the token that completes a group of r folds the group into one compressed entry
 (csa_compress, pooling mode: C and Z are the token projections the model already computed) and the
 same launch appends the entry and its indexer key to the FP4 caches; the lightning indexer scores every
-entry (csa_index_scores), the top-k entries are selected (csa_topk) and attention runs over them plus
-the window (csa_sparse_attn).
+entry and the top-k entries are selected (csa_index_topk: on B200 one thread-block cluster per sequence
+keeps the scores on chip and selects them itself), and attention runs over them plus the window
+(csa_sparse_attn: the CTAs of a query merge their partial softmax inside their cluster).
 """
 from __future__ import annotations
 
@@ -15,8 +16,8 @@ from dataclasses import dataclass
 
 import torch
 
-from . import PackedCache, attn_workspace_size, compress, index_scores, pack_fp4, sparse_attn, topk, \
-    topk_workspace_size
+from . import PackedCache, attn_workspace_size, compress, index_scores, index_topk, index_topk_workspace_size, \
+    pack_fp4, sparse_attn, topk, topk_workspace_size
 
 
 @dataclass
@@ -38,12 +39,18 @@ class LayerShape:
 
 
 class CSADecodeLayer:
-    def __init__(self, s: LayerShape, device="cuda", early_start: bool = True):
+    def __init__(self, s: LayerShape, device="cuda", early_start: bool = True, fused_index: bool = True,
+                 cluster_merge: bool = True):
         """early_start: the step's indexer streams the key tiles below the new entry while the compressor
         still runs, and attention runs each query's window tile while the top-k still runs
-        (CSA_EARLY_START; the step's inputs q, q_I, w and the window are never written by its kernels)."""
+        (CSA_EARLY_START; the step's inputs q, q_I, w and the window are never written by its kernels).
+        fused_index: one csa_index_topk call (on B200 the scores stay on chip and each row is selected by
+        its cluster); False: csa_index_scores into `scores` + csa_topk (the score row is materialised).
+        cluster_merge: a query's attention splits merge inside their cluster (False: CSA_NO_CLUSTER)."""
         self.s = s
         self.early = early_start
+        self.fused = fused_index
+        self.cluster = cluster_merge
         dev = torch.device(device)
         self.kv = PackedCache(s.B, s.n_max, s.d, s.d_r, dev, s.g_kv)
         self.ki = PackedCache(s.B, s.n_max, s.d_I, 0, dev, s.g_k)
@@ -63,10 +70,12 @@ class CSADecodeLayer:
         q = torch.empty((s.B, 1, s.H, s.d), dtype=torch.bfloat16, device=dev)
         self.scores = torch.empty((s.B, s.n_max), dtype=torch.float32, device=dev)
         self.hist = torch.zeros((s.B, 4096), dtype=torch.int32, device=dev)   # score histogram (uint32 bits)
-        ws_i = topk_workspace_size(self.ki, self.n_c, self.q_pos, B=s.B, Nq=1, ratio=s.r, k=s.k)
+        ws_i = max(topk_workspace_size(self.ki, self.n_c, self.q_pos, B=s.B, Nq=1, ratio=s.r, k=s.k),
+                   index_topk_workspace_size(qI, w, self.ki, self.n_c, self.q_pos, ratio=s.r, k=s.k))
         # sized for both launch plans (the flag may be switched off later, e.g. for stage-by-stage timing)
         ws_a = max(attn_workspace_size(q, self.q_pos, self.kv, self.n_c, self.idx, self.win, self.win_pos0,
-                                       ratio=s.r, window=s.W, early_start=e) for e in (True, False))
+                                       ratio=s.r, window=s.W, early_start=e, cluster=cluster_merge)
+                   for e in (True, False))
         self.ws_index = torch.empty(max(ws_i, 1), dtype=torch.uint8, device=dev)
         self.ws_attn = torch.empty(max(ws_a, 1), dtype=torch.uint8, device=dev)
 
@@ -86,13 +95,20 @@ class CSADecodeLayer:
         self.q_pos.fill_(t)
         self.win_pos0.fill_(t - s.W + 1)
 
-    KERNELS_PER_STEP = 5   # pool + FP4 append, index score, top-k, attention, split-K merge
+    # kernels of one step on B200 (fused path): pool + FP4 append, index + top-k (one cluster per row),
+    # attention (one cluster per query merges its splits); split path: pool, index score, top-k, attention
+    KERNELS_PER_STEP = 3
+
+    @property
+    def kernels_per_step(self):
+        return (3 if self.fused else 4) + (0 if self.cluster else 1)
 
     def step(self, C, Z, b_pos, W_IK, q, q_I, w, stream=None, marks=None):
         """One decode step.  C, Z [B, r, d] bf16 (projections of the group's r tokens), q [B,1,H,d],
         q_I [B,1,H_I,d_I], w [B,1,H_I].  The window buffer must already hold tokens t-W+1 .. t.
         marks: optional 5 CUDA events recorded between the stages (compress+pack | index scores |
-        top-k | attention).  Returns (out [B,1,H,d] bf16, lse [B,1,H] fp32, idx [B,1,k] int32)."""
+        top-k | attention; with the fused index the second stage is the whole index + top-k and the third
+        is empty).  Returns (out [B,1,H,d] bf16, lse [B,1,H] fp32, idx [B,1,k] int32)."""
         s = self.s
         st = stream if stream is not None else torch.cuda.current_stream()
 
@@ -105,13 +121,19 @@ class CSADecodeLayer:
                  W_IK=W_IK, c_out=self.c_new, kI_out=self.kI_new, kv_cache=self.kv, ki_cache=self.ki, row0=self.row0,
                  stream=st)
         mark(1)
-        index_scores(q_I, w, self.ki, self.n_c, self.q_pos, self.scores, ratio=s.r, g_q=s.g_q, hist=self.hist, k=s.k,
-                     early_start=self.early, stream=st)
-        mark(2)
-        topk(self.scores, self.ki, self.n_c, self.q_pos, B=s.B, Nq=1, ratio=s.r, k=s.k, idx_out=self.idx,
-             hist=self.hist, ws=self.ws_index, stream=st)
+        if self.fused:
+            index_topk(q_I, w, self.ki, self.n_c, self.q_pos, ratio=s.r, k=s.k, g_q=s.g_q, idx_out=self.idx,
+                       ws=self.ws_index, early_start=self.early, stream=st)
+            mark(2)
+        else:
+            index_scores(q_I, w, self.ki, self.n_c, self.q_pos, self.scores, ratio=s.r, g_q=s.g_q, hist=self.hist,
+                         k=s.k, early_start=self.early, stream=st)
+            mark(2)
+            topk(self.scores, self.ki, self.n_c, self.q_pos, B=s.B, Nq=1, ratio=s.r, k=s.k, idx_out=self.idx,
+                 hist=self.hist, ws=self.ws_index, stream=st)
         mark(3)
         sparse_attn(q, self.q_pos, self.kv, self.n_c, self.idx, self.win, self.win_pos0, ratio=s.r, window=s.W,
-                    out=self.out, lse=self.lse, ws=self.ws_attn, early_start=self.early, stream=st)
+                    out=self.out, lse=self.lse, ws=self.ws_attn, early_start=self.early, cluster=self.cluster,
+                    stream=st)
         mark(4)
         return self.out, self.lse, self.idx

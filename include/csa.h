@@ -83,6 +83,11 @@ csa_status csa_check_error_path(uint32_t polls, void* stream);
  *     among them.
  * Paths that cannot use the flag ignore it.  Results are the same with and without it. */
 #define CSA_EARLY_START 1u
+/* CSA_NO_CLUSTER in csa_attn_args.flags: a query whose keys are split over 2..8 CTAs normally merges
+ * the partial softmax results inside the CTAs' thread-block cluster (distributed shared memory; no
+ * workspace).  With this flag the partials go through the workspace and a merge kernel instead (e.g.
+ * where cluster launches are unavailable).  Results agree to rounding. */
+#define CSA_NO_CLUSTER 2u
 
 /* Paged caches ([V4.1 notes] §実装上の工夫: serving keeps the compressed KV in pages; the pages give no
  * layout, so this library fixes one).  A csa_page_map sends logical entry i of sequence b to row

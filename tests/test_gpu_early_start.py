@@ -15,11 +15,11 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _layer(n_c, B, inp, early):
+def _layer(n_c, B, inp, early, fused=False):
     from compressed_sparse_attention_18_b200.layer import CSADecodeLayer, LayerShape
     s = CFG2
     ls = LayerShape(B=B, n_max=(n_c + 7) // 8 * 8, r=s.r, H=s.H, d=s.d, d_r=s.d_r, H_I=s.H_I, d_I=s.d_I, k=s.k, W=s.W)
-    L = CSADecodeLayer(ls, DEV, early_start=early)
+    L = CSADecodeLayer(ls, DEV, early_start=early, fused_index=fused)
     L.load_history(inp["kv_src"], inp["kI_src"], n_c)
     L.win.copy_(inp["win_kv"])
     return L
@@ -34,14 +34,21 @@ def _run(L, inp, steps=3):
 
 # n_c: newest entry inside a partial 256-row tile, first row of a tile, last row of a tile, in the third
 # tile (the cache capacity is n_c rounded up to 8 rows, as the tensor-core scorer needs a multiple of 4)
+# fused: the early layer selects with the fused indexer + top-k (scores kept on chip); its score row is
+# then recomputed by a separate scoring call on the same cache bytes, which must give the same bits
+@pytest.mark.parametrize("fused", [False, True], ids=["split", "fused"])
 @pytest.mark.parametrize("n_c,B", [(4096 + 36, 16), (4096 + 1, 16), (4096, 16), (700, 24)])
-def test_early_start_same_bits_and_fresh_newest_entry(cuda_lib, n_c, B):
+def test_early_start_same_bits_and_fresh_newest_entry(cuda_lib, n_c, B, fused):
     s = CFG2
+    csa = cuda_lib
     inp = decode_inputs(s, seed=11, device=DEV, n_c=n_c, B=B)
-    La = _layer(n_c, B, inp, early=True)
+    La = _layer(n_c, B, inp, early=True, fused=fused)
     Lb = _layer(n_c, B, inp, early=False)
     oa, la, ia = _run(La, inp)
     ob, lb, ib = _run(Lb, inp)
+    if fused:
+        csa.index_scores(inp["q_I"], inp["w"], La.ki, La.n_c, La.q_pos, La.scores, ratio=s.r)
+        torch.cuda.synchronize()
     # scores are bit-identical; selections compare as sets (their order is unspecified, and it decides
     # the order in which attention sums the entries, so the two layers' outputs agree to rounding)
     assert torch.equal(La.scores[:, :n_c], Lb.scores[:, :n_c])
@@ -49,7 +56,6 @@ def test_early_start_same_bits_and_fresh_newest_entry(cuda_lib, n_c, B):
     assert_close(f64(oa), f64(ob), OUT_ATOL, OUT_RTOL, "out early vs not")
     # on one selection: the early plan (split 0 walks the window tile, then its entry tile) is
     # deterministic and agrees with the stage-by-stage plan (window in a split of its own) to rounding
-    csa = cuda_lib
     o1, l1 = csa.sparse_attn(inp["q"], La.q_pos, La.kv, La.n_c, ia, La.win, La.win_pos0, ratio=s.r, window=s.W,
                              early_start=True)
     o2, l2 = csa.sparse_attn(inp["q"], La.q_pos, La.kv, La.n_c, ia, La.win, La.win_pos0, ratio=s.r, window=s.W,
@@ -59,7 +65,7 @@ def test_early_start_same_bits_and_fresh_newest_entry(cuda_lib, n_c, B):
     assert_close(f64(o1), f64(o2), OUT_ATOL, OUT_RTOL, "out early vs stage-by-stage plan")
     assert_close(l1.cpu().numpy(), l2.cpu().numpy(), LSE_ATOL, LSE_RTOL, "lse early vs stage-by-stage plan")
     assert torch.equal(La.kv.codes, Lb.kv.codes) and torch.equal(La.ki.codes, Lb.ki.codes)
-    assert int(La.hist.abs().sum()) == 0          # the top-k left the histogram clean
+    assert int(La.hist.abs().sum()) == 0 and int(Lb.hist.abs().sum()) == 0   # the top-k left the histogram clean
     t = int(La.q_pos[0, 0])
     for b in (0, B - 1):
         codes, scales = np_u8(La.ki.codes[b, :n_c]), np_u8(La.ki.scales[b, :n_c])

@@ -123,7 +123,9 @@ def test_paged_reindex_candidates(cuda_lib):
     csa.pack_fp4(kI.to(DEV), cache)
     qI = normal((B, 1, 8, 128), 1.0, G)
     w = normal((B, 1, 8), 0.35, G, dtype=torch.float32)
-    cand = torch.randint(-5, n_max + 5, (B, 1, n_cand), generator=G, dtype=torch.int32)
+    # distinct ids (a repeated id may legitimately be selected twice), some -1 and some past n_c
+    cand = torch.stack([(torch.randperm(n_max + 10, generator=G)[:n_cand] - 5).view(1, n_cand)
+                        for _ in range(B)]).to(torch.int32)
     n_c = [2048, 1500]
     q_pos = np.array([[4 * 2048 - 1], [4 * 1500 - 1]], np.int64)
     idx, _, _ = csa.index_topk(qI.to(DEV), w.to(DEV), cache, torch.tensor(n_c, dtype=torch.int32, device=DEV),
@@ -184,7 +186,7 @@ def test_paged_attention(cuda_lib, case):
 def test_paged_map_rejected_when_malformed(cuda_lib):
     """Page sizes off the 128-entry tile and tables too narrow for n_max are refused on the host."""
     csa = cuda_lib
-    G = gen(57)
+    G = gen(57, DEV)
     src = normal((1, 10, 128), 1.0, G, DEV)
     bad = csa.PagedCache(1, 200, 128, 0, DEV, 100, 4, torch.zeros((1, 2), dtype=torch.int32))
     with pytest.raises(csa.CSAError, match="UNSUPPORTED"):
