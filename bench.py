@@ -4,8 +4,8 @@ compressed entries per sequence, top-512, window 128, 64 heads x 512) on B200.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One step = the whole hot path for one decode token of every sequence: compress the completed group
-(pooling), FP4-pack the new entry and its indexer key, lightning-indexer scores over all entries and
-the top-k (one fused launch), attention over the selected entries plus the window.  Eight independent layer states (3.7 GB)
+(pooling), FP4-pack the new entry and its indexer key, lightning-indexer scores over all entries,
+top-k, attention over the selected entries plus the window.  Eight independent layer states (3.7 GB)
 are rotated so every step reads its caches from HBM, not from the 126 MB L2.  Steps are replayed from
 CUDA graphs; timing uses CUDA events on the launching stream, max over ranks.  Under torchrun every
 rank runs its own batch of 32 sequences (weak scaling, no collective on the data path).
@@ -106,9 +106,15 @@ def peaks():
     return 6650.0, "fallback"
 
 
+def score_kernel_bytes(s, B):
+    """Algorithmic bytes of one index-score launch: every visible key (64 B codes + 4 B scales), the
+    score written per key, the queries (bf16) and head weights."""
+    return B * (s.n_c * (s.d_I // 2 + s.d_I // 32 + 4) + s.H_I * s.d_I * 2 + s.H_I * 4)
+
+
 def index_topk_bytes(s, B):
-    """Algorithmic bytes of one fused index + top-k launch: every visible key (64 B codes + 4 B scales),
-    the queries (bf16) and head weights in, the k selected ids out (the scores stay on chip)."""
+    """Algorithmic bytes of one on-chip index + top-k launch (CSA_ONCHIP_TOPK): every visible key (64 B
+    codes + 4 B scales), the queries (bf16) and head weights in, the k selected ids out."""
     return B * (s.n_c * (s.d_I // 2 + s.d_I // 32) + s.H_I * s.d_I * 2 + s.H_I * 4 + s.k * 4)
 
 
@@ -418,7 +424,7 @@ def run_ours(args, rank, world):
     steps.run(LAYERS, with_marks=True)
     stream.synchronize()
     stage = [[marks[li][j].elapsed_time(marks[li][j + 1]) for j in range(4)] for li in range(LAYERS)]
-    score_ms = statistics.mean(st[1] + st[2] for st in stage)          # fused index + top-k (stage 2 empty)
+    score_ms = statistics.mean(st[1] for st in stage)
     ms = max_over_ranks(ms, world, dev)
     value = whole_job_rate(s.B * args.steps, world, ms)
 
@@ -431,26 +437,26 @@ def run_ours(args, rank, world):
     attn_ms = statistics.mean(st[3] for st in stage)
     abytes = attention_bytes(s, s.B)
     a_achieved = abytes / (attn_ms / 1e3) / 1e9
-    bpl = index_topk_bytes(s, s.B)
+    bpl = score_kernel_bytes(s, s.B)
     achieved = bpl / (score_ms / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp4-e2m1/bf16", "data": "synthetic", "config": config_dict(s),
-        "gpu_launches": CSADecodeLayer.KERNELS_PER_STEP * args.steps,
+        "gpu_launches": layers[0].kernels_per_step * args.steps,
         "clocks": clocks,
-        "stages_ms": {"compress_pack": statistics.mean(st[0] for st in stage), "index_topk": score_ms,
-                      "attention": attn_ms},
+        "stages_ms": {"compress_pack": statistics.mean(st[0] for st in stage), "index_score": score_ms,
+                      "topk": statistics.mean(st[2] for st in stage), "attention": attn_ms},
         "stages_plan": "serialised stage-by-stage replay (an event at every stage boundary, no early start); "
                        "value/ms_per_step time the overlapped schedule",
-        # the dominant stage: tcgen05 attention over one 128-key tile per CTA, merged in the query's cluster
-        "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel (attention stage, in-cluster merge)",
+        # the dominant stage: tcgen05 attention over one 128-key tile per CTA plus the split merge
+        "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel + attn_merge_kernel (attention stage)",
                      "timed_on": "serialised stage-by-stage replay",
                      "achieved": a_achieved, "peak": hbm, "peak_kind": kind, "unit": "GB/s",
                      "frac": a_achieved / hbm, "traffic": profiled_traffic(ATTN_PROFILE, ATTN_SRC),
                      "algorithmic_bytes_per_launch": abytes},
-        # the streaming stage: every FP4 indexer key of every sequence, scored and selected in one launch
-        "roofline_index": {"bound": "hbm", "kernel": "index_score_tc_kernel<fused> (index + top-k)",
+        # the streaming stage: every FP4 indexer key of every sequence
+        "roofline_index": {"bound": "hbm", "kernel": "index_score_tc_kernel",
                            "timed_on": "serialised stage-by-stage replay",
                            "achieved": achieved, "peak": hbm,
                            "peak_kind": kind, "unit": "GB/s", "frac": achieved / hbm,

@@ -29,7 +29,8 @@ ENTRY_POINTS = ("csa_status_string", "csa_version", "csa_last_cuda_error", "csa_
 
 _u32, _i32, _f32, _vp = ctypes.c_uint32, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p
 CSA_EARLY_START = 1   # see csa.h: part of a call's work may start before the step's earlier kernels end
-CSA_NO_CLUSTER = 2    # see csa.h: merge a query's split partials through the workspace, not in a cluster
+CSA_CLUSTER_MERGE = 2  # see csa.h: a query's split partials merge inside their thread-block cluster
+CSA_ONCHIP_TOPK = 4   # see csa.h: decode rows scored and selected inside one cluster (scores stay on chip)
 
 
 class PageMap(ctypes.Structure):
@@ -254,8 +255,9 @@ def _index_args(q_I, w, kcache: PackedCache, n_c, q_pos, ratio, k, g_q, cand, po
 
 def index_topk(q_I, w, kcache: PackedCache, n_c, q_pos, *, ratio, k, g_q=1.0, cand=None, pool_blocks=0,
                pool_block_size=8, want_scores=False, idx_out=None, scores_out=None, pool_out=None, ws=None,
-               early_start=False, stream=None):
-    """Lightning indexer + top-k.  Returns (idx [B,Nq,k] int32, scores [B,Nq,k] or None, pool or None)."""
+               early_start=False, onchip=False, stream=None):
+    """Lightning indexer + top-k.  Returns (idx [B,Nq,k] int32, scores [B,Nq,k] or None, pool or None).
+    onchip: CSA_ONCHIP_TOPK (decode rows scored and selected inside one cluster, scores never in HBM)."""
     B, Nq = q_I.shape[:2]
     dev = q_I.device
     if idx_out is None:
@@ -266,7 +268,7 @@ def index_topk(q_I, w, kcache: PackedCache, n_c, q_pos, *, ratio, k, g_q=1.0, ca
         pool_out = torch.empty((B, Nq, pool_blocks * pool_block_size), dtype=torch.int32, device=dev)
     a = _index_args(q_I, w, kcache, n_c, q_pos, ratio, k, g_q, cand, pool_blocks, pool_block_size, pool_out,
                     idx_out, scores_out)
-    a.flags = CSA_EARLY_START if early_start else 0
+    a.flags = (CSA_EARLY_START if early_start else 0) | (CSA_ONCHIP_TOPK if onchip else 0)
     nbytes = _lib.csa_index_topk_workspace_size(ctypes.byref(a))
     wbuf = _ws(nbytes, dev, ws)
     _check(_lib.csa_index_topk(ctypes.byref(a), _ptr(wbuf) if wbuf is not None else None, nbytes,
@@ -367,14 +369,14 @@ def _attn_args(q, q_pos, cache: PackedCache, n_c, idx, win_kv, win_pos0, ratio, 
 
 
 def _attn(fn, hca, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse, ws,
-          stream, early_start=False, out_rope_theta=0.0, cluster=True):
+          stream, early_start=False, out_rope_theta=0.0, cluster=False):
     B, Nq, H, d = q.shape
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Nq, H), dtype=torch.float32, device=q.device)
     a = _attn_args(q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, softmax_scale, out, lse)
-    a.flags = (CSA_EARLY_START if early_start else 0) | (0 if cluster else CSA_NO_CLUSTER)
+    a.flags = (CSA_EARLY_START if early_start else 0) | (CSA_CLUSTER_MERGE if cluster else 0)
     a.out_rope_theta = out_rope_theta
     nbytes = _lib.csa_attn_workspace_size(ctypes.byref(a), hca)
     wbuf = _ws(nbytes, q.device, ws)
@@ -384,13 +386,13 @@ def _attn(fn, hca, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, s
 
 
 def sparse_attn(q, q_pos, cache: PackedCache, n_c, idx, win_kv=None, win_pos0=None, *, ratio=4, window=128,
-                softmax_scale=0.0, out=None, lse=None, ws=None, early_start=False, out_rope_theta=0.0, cluster=True,
+                softmax_scale=0.0, out=None, lse=None, ws=None, early_start=False, out_rope_theta=0.0, cluster=False,
                 stream=None):
     """CSA attention over the selected entries idx [B,Nq,k] plus the window.  Returns (out, lse).
     early_start: CSA_EARLY_START (window tiles start before the step's index and top-k kernels end;
     only inside a decode step that began with compress).  out_rope_theta: inverse-RoPE epilogue on the
-    output's RoPE channels at the query position (0 = off).  cluster=False: CSA_NO_CLUSTER (split
-    partials merged through the workspace instead of inside a thread-block cluster)."""
+    output's RoPE channels at the query position (0 = off).  cluster=True: CSA_CLUSTER_MERGE (split
+    partials merged inside a thread-block cluster instead of through the workspace)."""
     return _attn(_lib.csa_sparse_attn, 0, q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window,
                  softmax_scale, out, lse, ws, stream, early_start, out_rope_theta, cluster)
 
@@ -403,7 +405,7 @@ def hca_attn(q, q_pos, cache: PackedCache, n_c, win_kv=None, win_pos0=None, *, r
 
 
 def attn_workspace_size(q, q_pos, cache, n_c, idx, win_kv, win_pos0, *, ratio, window, hca=False, early_start=False,
-                        cluster=True):
+                        cluster=False):
     a = _attn_args(q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, 0.0, None, None)
-    a.flags = (CSA_EARLY_START if early_start else 0) | (0 if cluster else CSA_NO_CLUSTER)
+    a.flags = (CSA_EARLY_START if early_start else 0) | (CSA_CLUSTER_MERGE if cluster else 0)
     return _lib.csa_attn_workspace_size(ctypes.byref(a), 1 if hca else 0)

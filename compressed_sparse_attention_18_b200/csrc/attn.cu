@@ -565,7 +565,7 @@ static AttnPlan plan_attn(const csa_attn_args* a, int hca) {
     p.cps = 1;
     attn_tc_plan(a, hca, &p.splits, &p.tpc);
     size_t o = 0;
-    const bool cluster = attn_tc_cluster(p.splits) && !(a->flags & CSA_NO_CLUSTER);
+    const bool cluster = attn_tc_cluster(p.splits) && (a->flags & CSA_CLUSTER_MERGE);
     if (p.splits > 1 && !cluster) {                       // (a cluster merges its query's partials on chip)
       p.off_o = o;   o = align_up(o + (size_t)rows_tc * p.splits * a->H * a->d * 2, 256);
       p.off_lse = o; o = align_up(o + (size_t)rows_tc * p.splits * a->H * 4, 256);
@@ -642,7 +642,7 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
   CSA_REQUIRE(p.total == 0 || ws != nullptr);
   cudaStream_t st = (cudaStream_t)stream;
   if (p.tc) {
-    const bool merged = p.splits == 1 || (attn_tc_cluster(p.splits) && !(a->flags & CSA_NO_CLUSTER));
+    const bool merged = p.splits == 1 || (attn_tc_cluster(p.splits) && (a->flags & CSA_CLUSTER_MERGE));
     uint16_t* po = !merged ? (uint16_t*)((uint8_t*)ws + p.off_o) : nullptr;
     float* pl = !merged ? (float*)((uint8_t*)ws + p.off_lse) : nullptr;
     csa_status s = launch_attn_tc(a, hca, p.splits, p.tpc, po, pl, st);

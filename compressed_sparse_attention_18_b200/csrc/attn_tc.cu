@@ -175,6 +175,9 @@ __device__ __forceinline__ TaTile ta_tile(int key0, int n_sel, int n_list, long 
 // units), so probabilities stay <= 2^8 and O is rescaled in tensor memory only when a max jumps.
 constexpr float TA_RESCALE_SLACK = 8.0f;
 
+// W8: the window rows are FP8 (a separate instantiation keeps the bf16 path's code compact: each launch
+// runs with a cold instruction cache)
+template <bool W8>
 __global__ void __launch_bounds__(TA_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap wmap,
                    const TaParams P) {
@@ -300,7 +303,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       const uint32_t ido = idesc_bf16(128, 64, 1, 1);
 #pragma unroll 1
       for (int t = 0; t < ntile; ++t) {
-        const TaTile g = ta_tile(tile_key(t), n_sel, n_list, wlo, p0, P.win_fp8 != 0);
+        const TaTile g = ta_tile(tile_key(t), n_sel, n_list, wlo, p0, W8);
         const int nbox = (g.we - g.wa) / TA_WBOX;
         // window boxes overwrite the K tile: only once the previous tile's O MMAs have completed (S MMAs
         // of an entry tile are queued behind them directly)
@@ -383,7 +386,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
     // FP8 window row of a tile (rows [rs, rw)) in the same registers an entry row uses: codes of this
     // thread's 32 channels of 64-channel blocks 0-2 in cv[0..5], the 7 block scales in cv[6] (0-3) and
     // sc16 (4-6), the RoPE quarter in rp; blocks 3-6 are read into cv[0..6], sc16 during the gather.
-    auto is_win8 = [&](const TaTile& gg) { return P.win_fp8 && grow >= gg.rs && grow < gg.rw; };
+    auto is_win8 = [&](const TaTile& gg) { return W8 && grow >= gg.rs && grow < gg.rw; };
     auto win8_ptr = [&](const TaTile& gg) -> const uint8_t* {
       return P.wcodes + ((size_t)b * P.Wn + (size_t)(gg.wrow_base + grow)) * 448 + ghalf * 32;
     };
@@ -402,9 +405,9 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) rp[c] = __ldg(rrow + c);
     };
-    TaTile g = ta_tile(tile_key(0), n_sel, n_list, wlo, p0, P.win_fp8 != 0);
+    TaTile g = ta_tile(tile_key(0), n_sel, n_list, wlo, p0, W8);
     int id = check_id(raw_id(g));                  // a window tile reads no id
-    int id_next = ntile > 1 && !has_win ? raw_id(ta_tile(tile_key(1), n_sel, n_list, wlo, p0, P.win_fp8 != 0)) : -1;
+    int id_next = ntile > 1 && !has_win ? raw_id(ta_tile(tile_key(1), n_sel, n_list, wlo, p0, W8)) : -1;
     load_row(id);
     if (is_win8(g)) load_win8(g);
 #pragma unroll 1
@@ -421,7 +424,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       if (!pure) {
         // window rows before the first TMA box, by asynchronous copies
         const int r_end = min(g.wa, g.rw);
-        const int n = P.win_fp8 ? 0 : (r_end > g.rs ? r_end - g.rs : 0) * 64;
+        const int n = W8 ? 0 : (r_end > g.rs ? r_end - g.rs : 0) * 64;
         for (int i = tid; i < n; i += TA_WORKERS) {
           const int row = g.rs + (i >> 6), c = i & 63;
           const long long wr = g.wrow_base + row;
@@ -503,13 +506,13 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
         if (has_win && t == 0) {
           // the window tile is gathered: from here on the ids and entries of the previous kernels
           pdl_wait();
-          id_next = raw_id(ta_tile(tile_key(1), n_sel, n_list, wlo, p0, P.win_fp8 != 0));
+          id_next = raw_id(ta_tile(tile_key(1), n_sel, n_list, wlo, p0, W8));
         }
-        g = ta_tile(tile_key(t + 1), n_sel, n_list, wlo, p0, P.win_fp8 != 0);
+        g = ta_tile(tile_key(t + 1), n_sel, n_list, wlo, p0, W8);
         id = check_id(id_next);
         load_row(id);
         if (is_win8(g)) load_win8(g);
-        id_next = t + 2 < ntile ? raw_id(ta_tile(tile_key(t + 2), n_sel, n_list, wlo, p0, P.win_fp8 != 0)) : -1;
+        id_next = t + 2 < ntile ? raw_id(ta_tile(tile_key(t + 2), n_sel, n_list, wlo, p0, W8)) : -1;
       }
       asm volatile("bar.sync 1, 256;" ::: "memory");   // workers only: ids visible to the softmax
 
@@ -750,7 +753,8 @@ void attn_tc_plan(const csa_attn_args* a, int hca, int* splits, int* tpc) {
   *splits = (int)((tiles + t - 1) / t);
 }
 
-// Queries split over 2..8 CTAs merge inside a thread-block cluster (no workspace, no merge kernel).
+// Queries split over 2..8 CTAs can merge inside a thread-block cluster (CSA_CLUSTER_MERGE: no workspace,
+// no merge kernel).
 bool attn_tc_cluster(int splits) { return splits >= 2 && splits <= TA_MAX_CLUSTER; }
 
 bool attn_tc_eligible(const csa_attn_args* a, int hca, int max_splits) {
@@ -798,7 +802,7 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
   P.Nq = a->Nq; P.H = a->H; P.ratio = a->ratio; P.n_max = a->n_max; P.k = hca ? 0 : a->k;
   P.Wn = Wn; P.window = a->window; P.splits = splits; P.tpc = tpc; P.hca = hca; P.g = a->g_kv;
   P.early_rows = attn_tc_early(a, hca) ? (int)rows : 0;
-  P.cluster = (attn_tc_cluster(splits) && !(a->flags & CSA_NO_CLUSTER)) ? 1 : 0;
+  P.cluster = (attn_tc_cluster(splits) && (a->flags & CSA_CLUSTER_MERGE)) ? 1 : 0;
   const float scale = a->softmax_scale != 0.0f ? a->softmax_scale : 1.0f / sqrtf((float)a->d);
   P.scale_log2 = scale * TA_LOG2E;
   P.q_pos = a->q_pos; P.codes = a->kv_codes; P.scales = a->kv_scales;
@@ -814,9 +818,11 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
   }
   const int smem = (int)sizeof(TaSmem) + 1024;
   static std::atomic<unsigned> attr_done{0};
-  set_smem_once((const void*)attn_tc_kernel, smem, attr_done);
+  static std::atomic<unsigned> attr_done8{0};
+  auto* kfn = fp8 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  set_smem_once((const void*)kfn, smem, fp8 ? attr_done8 : attr_done);
   if (!P.cluster)
-    return launch_pdl(attn_tc_kernel, dim3((unsigned)(rows * splits)), dim3(TA_THREADS), (size_t)smem, st, qmap, wmap, P);
+    return launch_pdl(kfn, dim3((unsigned)(rows * splits)), dim3(TA_THREADS), (size_t)smem, st, qmap, wmap, P);
   cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = pdl_config(dim3((unsigned)(rows * splits)), dim3(TA_THREADS), (size_t)smem, st, attr);
   attr[1].id = cudaLaunchAttributeClusterDimension;
@@ -824,7 +830,7 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
   cfg.numAttrs = 2;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, qmap, wmap, P);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, qmap, wmap, P);
   if (e != cudaSuccess) {
     set_last_cuda_error(e);
     return CSA_ERR_CUDA;

@@ -13,11 +13,12 @@
 //
 // Warp roles (320 threads):
 //   warp 0      TMA producer: 128 x 64 B FP4 key tile (64-byte swizzle) + the tile's 512 B of key scales;
-//   warp 1      allocates tensor memory (512 columns) and issues the MMAs (one thread);
+//   warp 1      allocates tensor memory (512 columns) and issues the copies and MMAs (one thread);
+//   warp 1      also lays each tile's key scales out for a tcgen05.cp into tensor memory;
 //   warps 2..9  set-up: all ten warps FP4-quantise the 128 (query, head) rows (one thread per 32-element
-//               block); then warps 2..5 write the query scale factors, and per tile the key scale
-//               factors, into their tensor-memory lane quadrant; warps 2..9 read the accumulators
-//               (quadrant = warp % 4, queries 8 ((warp - 2) / 4) .. + 7), score and store.
+//               block); then warps 2..5 write the query scale factors into their tensor-memory lane
+//               quadrant; warps 2..9 read the accumulators (quadrant = warp % 4, queries
+//               8 ((warp - 2) / 4) .. + 7), score and store.
 // Tensor memory: NBUF accumulator buffers of 128 columns, NBUF x 8 key-scale columns, 8 query-scale
 // columns.  Every wait is bounded; a wait that gives up records device error 1 and the kernel leaves.
 #include "csa_common.cuh"
@@ -45,6 +46,7 @@ struct MqSmem {
   alignas(1024) uint8_t qtile[MQ_N * 64];
   alignas(16) uint8_t sc[MQ_STAGES][MQ_KEYS * 4];
   alignas(16) uint32_t qsc[MQ_N];          // 4 E4M3 block scales of each (query, head) row
+  alignas(16) uint32_t sfx[2][2][32][4];   // key scale factors in copy order, 2 slots: [atom][lane][col]
   alignas(16) float wq[MQ_N];
   int nvis[MQ_QB];
   alignas(8) uint64_t full[MQ_STAGES];
@@ -189,16 +191,42 @@ __global__ void __launch_bounds__(MQ_THREADS, 1) index_mq_tc_kernel(const __grid
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_mxf4_ue4m3(MQ_KEYS, MQ_N);
-      const uint32_t qa = smem_addr(S.qtile);
-      if (ntile > 0 && !mbar_wait(&S.q_ready, 0)) ok = false;
-      for (int i = 0; i < ntile && ok; ++i) {
-        const int s = i % MQ_STAGES, a = i % MQ_NBUF, use = i / MQ_NBUF;
-        if (!mbar_wait(&S.full[s], (i / MQ_STAGES) & 1)) { ok = false; break; }
-        if (!mbar_wait(&S.sfa_full[a], use & 1)) { ok = false; break; }
-        if (use > 0 && !mbar_wait(&S.acc_empty[a], (use - 1) & 1)) { ok = false; break; }
+    // The warp lays tile i's key scales out in copy order (atom k, lane L: the scales of keys L, L+32,
+    // L+64, L+96 as UE4M3 x4, blocks 0,0,1,1 for k = 0 and 2,2,3,3 for k = 1); lane 0 copies them into
+    // tensor memory and issues the MMAs (copies and MMAs run in issue order).
+    const uint32_t idesc = idesc_mxf4_ue4m3(MQ_KEYS, MQ_N);
+    const uint32_t qa = smem_addr(S.qtile);
+    if (ntile > 0 && !mbar_wait(&S.q_ready, 0)) ok = false;
+    ok = __all_sync(0xffffffffu, ok);
+    for (int i = 0; i < ntile && ok; ++i) {
+      const int s = i % MQ_STAGES, a = i % MQ_NBUF, use = i / MQ_NBUF;
+      ok = __all_sync(0xffffffffu, mbar_wait(&S.full[s], (i / MQ_STAGES) & 1));
+      // slot i & 1 was last copied for tile i - 2: that copy completed with tile i - 2's MMAs
+      if (ok && i >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&S.acc_full[(i - 2) % MQ_NBUF], ((i - 2) / MQ_NBUF) & 1));
+      if (!ok) break;
+      const int x = i & 1;
+      {
+        const uint32_t* sc = reinterpret_cast<const uint32_t*>(S.sc[s]);
+        uint32_t v[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) v[c] = sc[lane + 32 * c];
+        *reinterpret_cast<uint4*>(S.sfx[x][0][lane]) =
+            make_uint4(__byte_perm(v[0], 0, 0x1100), __byte_perm(v[1], 0, 0x1100), __byte_perm(v[2], 0, 0x1100),
+                       __byte_perm(v[3], 0, 0x1100));
+        *reinterpret_cast<uint4*>(S.sfx[x][1][lane]) =
+            make_uint4(__byte_perm(v[0], 0, 0x3322), __byte_perm(v[1], 0, 0x3322), __byte_perm(v[2], 0, 0x3322),
+                       __byte_perm(v[3], 0, 0x3322));
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0 && use > 0 && !mbar_wait(&S.acc_empty[a], (use - 1) & 1)) ok = false;
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      if (lane == 0) {
         tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          tmem_cp_32x128b_x4(tbase + MQ_COL_SFA + 8 * a + 4 * k, smem_desc(smem_addr(S.sfx[x][k]), 16, 128, LAYOUT_NONE));
         const uint32_t ca = smem_addr(S.codes[s]);
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
@@ -210,12 +238,13 @@ __global__ void __launch_bounds__(MQ_THREADS, 1) index_mq_tc_kernel(const __grid
         mma_commit(&S.acc_full[a]);
         mma_commit(&S.empty[s]);
       }
-      mma_commit(&S.done);
-      if (!ok) atomicOr(&S.err, 1u);
+      __syncwarp();
     }
+    if (lane == 0) mma_commit(&S.done);
+    if (!ok && lane == 0) atomicOr(&S.err, 1u);
     __syncwarp();
   } else {
-    // ------------------------------------------------ scale factors + epilogue
+    // ------------------------------------------------ query scale factors + epilogue
     const int q = warp & 3;                        // tensor-memory lane quadrant
     const int grp = (warp - 2) >> 2;               // queries 8 grp .. 8 grp + 7
     const bool sf_writer = grp == 0;
@@ -239,49 +268,27 @@ __global__ void __launch_bounds__(MQ_THREADS, 1) index_mq_tc_kernel(const __grid
 #pragma unroll
     for (int j = 0; j < 8; ++j) nvis[j] = S.nvis[8 * grp + j];
     uint32_t d[64];
-    for (int i = 0; i < ntile + MQ_LAG && ok; ++i) {
-      const int e = i - MQ_LAG;                    // tile whose accumulators are read now
-      if (e >= 0) {
-        if (!mbar_wait(&S.acc_full[e % MQ_NBUF], (e / MQ_NBUF) & 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t col = MQ_COL_D + 128 * (e % MQ_NBUF) + 64 * grp;
-        tmem_ld_x32(lane_base + col, d);
-        tmem_ld_x32(lane_base + col + 32, d + 32);
-      }
-      if (i < ntile && sf_writer) {
-        const int s = i % MQ_STAGES, a = i % MQ_NBUF;
-        if (!mbar_wait(&S.full[s], (i / MQ_STAGES) & 1)) { ok = false; break; }
-        // key scale factors of tile i: key lane + 32 c at lane `lane`, column c / 4 + c
-        const uint32_t* sc = reinterpret_cast<const uint32_t*>(S.sc[s]);
-        uint32_t v[4];
+    for (int e = 0; e < ntile && ok; ++e) {
+      if (!mbar_wait(&S.acc_full[e % MQ_NBUF], (e / MQ_NBUF) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t col = MQ_COL_D + 128 * (e % MQ_NBUF) + 64 * grp;
+      tmem_ld_x32(lane_base + col, d);
+      tmem_ld_x32(lane_base + col + 32, d + 32);
+      tmem_wait_ld_x32(d);
+      tmem_wait_ld_x32(d + 32);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.acc_empty[e % MQ_NBUF]);
+      const int key = (t_begin + e) * MQ_KEYS + 32 * q + lane;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) v[c] = sc[lane + 32 * c];
-        tmem_st_x4(lane_base + MQ_COL_SFA + 8 * a, __byte_perm(v[0], 0, 0x1100), __byte_perm(v[1], 0, 0x1100),
-                   __byte_perm(v[2], 0, 0x1100), __byte_perm(v[3], 0, 0x1100));
-        tmem_st_x4(lane_base + MQ_COL_SFA + 8 * a + 4, __byte_perm(v[0], 0, 0x3322), __byte_perm(v[1], 0, 0x3322),
-                   __byte_perm(v[2], 0, 0x3322), __byte_perm(v[3], 0, 0x3322));
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.sfa_full[a]);
-      }
-      if (e >= 0) {
-        tmem_wait_ld_x32(d);
-        tmem_wait_ld_x32(d + 32);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.acc_empty[e % MQ_NBUF]);
-        const int key = (t_begin + e) * MQ_KEYS + 32 * q + lane;
+      for (int j = 0; j < 8; ++j) {
+        const float4 w0 = wq4[2 * j], w1 = wq4[2 * j + 1];
+        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        float sc = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float4 w0 = wq4[2 * j], w1 = wq4[2 * j + 1];
-          const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-          float sc = 0.0f;
-#pragma unroll
-          for (int h = 0; h < 8; ++h) sc = fmaf(wv[h], fmaxf(__uint_as_float(d[8 * j + h]), 0.0f), sc);
-          sc += 0.0f;
-          if (key < nvis[j]) P.scores[((size_t)b * P.Nq + q0 + 8 * grp + j) * P.ld + key] = sc;
-        }
+        for (int h = 0; h < 8; ++h) sc = fmaf(wv[h], fmaxf(__uint_as_float(d[8 * j + h]), 0.0f), sc);
+        sc += 0.0f;
+        if (key < nvis[j]) P.scores[((size_t)b * P.Nq + q0 + 8 * grp + j) * P.ld + key] = sc;
       }
     }
     if (!ok && lane == 0) atomicOr(&S.err, 1u);

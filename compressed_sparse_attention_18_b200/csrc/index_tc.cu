@@ -58,6 +58,7 @@ struct TcSmemT {
   alignas(1024) uint8_t codes[STAGES][TC_CODE_BYTES];
   alignas(1024) uint8_t qtile[8 * 64];
   alignas(16) uint8_t sc[STAGES][TC_SC_BYTES];
+  alignas(16) uint32_t sfx[2][2][2][32][4];  // key scale factors in copy order, 2 slots: [sub-tile][atom][lane][col]
   uint32_t hist[TC_HIST_BINS];
   float scores[FUSED ? FT_SCAP : 1];             // fused: scores of this CTA's keys [key_lo, key_lo + nk)
   uint32_t gsl[FUSED ? TC_HIST_BINS / FT_CLUSTER : 1];   // fused: this CTA's slice of the row histogram
@@ -199,16 +200,50 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_mxf4_ue4m3(TC_SUB, 8);
-      const uint32_t qa = smem_addr(S.qtile);
-      if (ntile > 0 && !mbar_wait(&S.q_ready, 0)) ok = false;
-      for (int i = 0; i < ntile && ok; ++i) {
-        const int s = i % TC_STAGES, a = i % TC_NBUF, use = i / TC_NBUF;
-        if (!mbar_wait(&S.full[s], (i / TC_STAGES) & 1)) { ok = false; break; }
-        if (!mbar_wait(&S.sfa_full[a], use & 1)) { ok = false; break; }
-        if (use > 0 && !mbar_wait(&S.acc_empty[a], (use - 1) & 1)) { ok = false; break; }
+    // The whole warp lays tile i's key scales out in copy order (sub-tile u, atom k, lane L: the scales
+    // of keys L, L+32, L+64, L+96 as UE4M3 x4, blocks 0,0,1,1 for k = 0 and 2,2,3,3 for k = 1); lane 0
+    // copies them into tensor memory and issues the MMAs (copies and MMAs run in issue order).
+    const uint32_t idesc = idesc_mxf4_ue4m3(TC_SUB, 8);
+    const uint32_t qa = smem_addr(S.qtile);
+    if (ntile > 0 && !mbar_wait(&S.q_ready, 0)) ok = false;
+    ok = __all_sync(0xffffffffu, ok);
+    for (int i = 0; i < ntile && ok; ++i) {
+      const int s = i % TC_STAGES, a = i % TC_NBUF, use = i / TC_NBUF;
+      ok = __all_sync(0xffffffffu, mbar_wait(&S.full[s], (i / TC_STAGES) & 1));
+      // slot i & 1 was last copied for tile i - 2: that copy completed with tile i - 2's MMAs
+      if (ok && i >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&S.acc_full[(i - 2) % TC_NBUF], ((i - 2) / TC_NBUF) & 1));
+      if (!ok) break;
+      const int x = i & 1;
+      {
+        const uint32_t* sc = reinterpret_cast<const uint32_t*>(S.sc[s]);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          uint32_t v[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) v[c] = sc[TC_SUB * u + 32 * c + lane];
+          *reinterpret_cast<uint4*>(S.sfx[x][u][0][lane]) =
+              make_uint4(__byte_perm(v[0], 0, 0x1100), __byte_perm(v[1], 0, 0x1100), __byte_perm(v[2], 0, 0x1100),
+                         __byte_perm(v[3], 0, 0x1100));
+          *reinterpret_cast<uint4*>(S.sfx[x][u][1][lane]) =
+              make_uint4(__byte_perm(v[0], 0, 0x3322), __byte_perm(v[1], 0, 0x3322), __byte_perm(v[2], 0, 0x3322),
+                         __byte_perm(v[3], 0, 0x3322));
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) {
+        if (use > 0 && !mbar_wait(&S.acc_empty[a], (use - 1) & 1)) ok = false;
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      if (lane == 0) {
         tc_fence_after();
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+            tmem_cp_32x128b_x4(tbase + TC_COL_SFA + 16 * a + 8 * u + 4 * k,
+                               smem_desc(smem_addr(S.sfx[x][u][k]), 16, 128, LAYOUT_NONE));
         const uint32_t ca = smem_addr(S.codes[s]);
 #pragma unroll
         for (int u = 0; u < 2; ++u)
@@ -222,11 +257,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
         mma_commit(&S.acc_full[a]);
         mma_commit(&S.empty[s]);
       }
-      if (!ok) atomicOr(&S.err, 1u);
+      __syncwarp();
     }
+    if (!ok && lane == 0) atomicOr(&S.err, 1u);
     __syncwarp();
   } else {
-    // ------------------------------------------------------ scale factors + epilogue
+    // ------------------------------------------------------ query tile + epilogue
     const int q = warp & 3;                                      // tensor-memory lane quadrant
     const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
     {
@@ -305,35 +341,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
         }
       }
     };
-    for (int i = 0; i < ntile + TC_LAG && ok; ++i) {
-      const int e = i - TC_LAG;                                  // tile whose accumulators are read now
-      if (e >= 0) {
-        if (!mbar_wait(&S.acc_full[e % TC_NBUF], (e / TC_NBUF) & 1)) { ok = false; break; }
-        tc_fence_after();
-        tmem_ld_x16(lane_base + TC_COL_D + 16 * (e % TC_NBUF), d);
-      }
-      if (i < ntile) {
-        const int s = i % TC_STAGES, a = i % TC_NBUF;
-        if (!mbar_wait(&S.full[s], (i / TC_STAGES) & 1)) { ok = false; break; }
-        // key scale factors of tile i: sub-tile u, lane L of every quadrant holds rows L%32 + 32j
-        const uint32_t* sc = reinterpret_cast<const uint32_t*>(S.sc[s]);
-        uint32_t v[8], wsf[16];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = sc[lane + 32 * j];
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            wsf[8 * u + j] = __byte_perm(v[4 * u + j], 0, 0x1100);       // atom k = 0: blocks 0,0,1,1
-            wsf[8 * u + 4 + j] = __byte_perm(v[4 * u + j], 0, 0x3322);   // atom k = 1: blocks 2,2,3,3
-          }
-        tmem_st_x16(lane_base + TC_COL_SFA + 16 * a, wsf);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.sfa_full[a]);
-      }
-      if (e >= 0) finish(e);
+    for (int e = 0; e < ntile && ok; ++e) {
+      if (!mbar_wait(&S.acc_full[e % TC_NBUF], (e / TC_NBUF) & 1)) { ok = false; break; }
+      tc_fence_after();
+      tmem_ld_x16(lane_base + TC_COL_D + 16 * (e % TC_NBUF), d);
+      finish(e);
     }
     if (!ok && lane == 0) atomicOr(&S.err, 1u);
   }
@@ -658,9 +670,10 @@ csa_status run_scores_tc(const csa_index_args* a, float* scores, long long ld, u
   return launch_pdl(index_score_tc_kernel<false>, dim3(per_row, a->B), dim3(TC_THREADS), smem, st, map, P);
 }
 
-// Fused decode indexer + top-k: single-query Full rows of at most FT_CLUSTER x FT_SCAP keys, no pool.
+// Fused decode indexer + top-k (CSA_ONCHIP_TOPK): single-query Full rows of at most FT_CLUSTER x FT_SCAP
+// keys, no pool.
 bool index_topk_fused_eligible(const csa_index_args* a) {
-  return index_tc_eligible(a) && a->pool_blocks == 0 && a->idx_out != nullptr &&
+  return (a->flags & CSA_ONCHIP_TOPK) && index_tc_eligible(a) && a->pool_blocks == 0 && a->idx_out != nullptr &&
          a->n_max <= FT_CLUSTER * FT_SCAP && a->k >= 1 && a->k <= 4096;
 }
 

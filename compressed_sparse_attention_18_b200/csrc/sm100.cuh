@@ -159,6 +159,15 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64
       ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
+// Copy a 32-row x 128-bit matrix from shared memory (descriptor, no swizzle: 8-row core matrices 128 B
+// apart) into tensor memory at taddr, replicated into the lanes of all four warp quadrants (the layout of
+// block-scale factors of an M = 128 operand).  Asynchronous; ordered before the MMAs this thread issues
+// after it, and covered by its next commit.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+constexpr uint32_t LAYOUT_NONE = 0;
+
 // Arrive on `bar` once every MMA this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -206,23 +215,25 @@ __device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
 }
 __device__ __forceinline__ float ld_peer_f32(uint32_t addr) {
   float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
   return v;
 }
 __device__ __forceinline__ float4 ld_peer_v4(uint32_t addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr) : "memory");
+               : "r"(addr));
   return v;
 }
 __device__ __forceinline__ uint32_t ld_peer_u32(uint32_t addr) {
   uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
 __device__ __forceinline__ void st_peer_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+// (The peer loads are volatile without a memory clobber: they stay after the cluster barrier that
+// precedes them, and independent loads can be in flight together.)
 // Every thread of every CTA of the cluster: writes before it are visible to the cluster's reads after it.
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");

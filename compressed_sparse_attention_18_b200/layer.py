@@ -6,9 +6,9 @@ layer's hot path (sources: "DeepSeek-V4: エージェントが実際に使える
 Fig. 3): the token that completes a group of r folds the group into one compressed entry
 (csa_compress, pooling mode: C and Z are the token projections the model already computed) and the
 same launch appends the entry and its indexer key to the FP4 caches; the lightning indexer scores every
-entry and the top-k entries are selected (csa_index_topk: on B200 one thread-block cluster per sequence
-keeps the scores on chip and selects them itself), and attention runs over them plus the window
-(csa_sparse_attn: the CTAs of a query merge their partial softmax inside their cluster).
+entry (csa_index_scores, with the row histogram) and the top-k entries are selected (csa_topk), or both in
+one cluster per sequence with the scores kept on chip (csa_index_topk with CSA_ONCHIP_TOPK), and attention
+runs over them plus the window (csa_sparse_attn; optionally merging its splits inside their cluster).
 """
 from __future__ import annotations
 
@@ -39,14 +39,16 @@ class LayerShape:
 
 
 class CSADecodeLayer:
-    def __init__(self, s: LayerShape, device="cuda", early_start: bool = True, fused_index: bool = True,
-                 cluster_merge: bool = True):
+    def __init__(self, s: LayerShape, device="cuda", early_start: bool = True, fused_index: bool = False,
+                 cluster_merge: bool = False):
         """early_start: the step's indexer streams the key tiles below the new entry while the compressor
         still runs, and attention runs each query's window tile while the top-k still runs
         (CSA_EARLY_START; the step's inputs q, q_I, w and the window are never written by its kernels).
-        fused_index: one csa_index_topk call (on B200 the scores stay on chip and each row is selected by
-        its cluster); False: csa_index_scores into `scores` + csa_topk (the score row is materialised).
-        cluster_merge: a query's attention splits merge inside their cluster (False: CSA_NO_CLUSTER)."""
+        fused_index: one csa_index_topk call with CSA_ONCHIP_TOPK (the scores stay on chip and each row is
+        selected by its cluster); default: csa_index_scores into `scores` with its histogram + csa_topk
+        (measured faster for the 128K decode step).
+        cluster_merge: a query's attention splits merge inside their cluster (CSA_CLUSTER_MERGE); default:
+        through the workspace and a merge kernel (measured faster for the 128K decode step)."""
         self.s = s
         self.early = early_start
         self.fused = fused_index
@@ -95,9 +97,9 @@ class CSADecodeLayer:
         self.q_pos.fill_(t)
         self.win_pos0.fill_(t - s.W + 1)
 
-    # kernels of one step on B200 (fused path): pool + FP4 append, index + top-k (one cluster per row),
-    # attention (one cluster per query merges its splits); split path: pool, index score, top-k, attention
-    KERNELS_PER_STEP = 3
+    # kernels of one step with the default options: pool + FP4 append, index scores, top-k, attention,
+    # split merge (the on-chip top-k removes the top-k launch, the cluster merge the merge launch)
+    KERNELS_PER_STEP = 5
 
     @property
     def kernels_per_step(self):
@@ -123,7 +125,7 @@ class CSADecodeLayer:
         mark(1)
         if self.fused:
             index_topk(q_I, w, self.ki, self.n_c, self.q_pos, ratio=s.r, k=s.k, g_q=s.g_q, idx_out=self.idx,
-                       ws=self.ws_index, early_start=self.early, stream=st)
+                       ws=self.ws_index, early_start=self.early, onchip=True, stream=st)
             mark(2)
         else:
             index_scores(q_I, w, self.ki, self.n_c, self.q_pos, self.scores, ratio=s.r, g_q=s.g_q, hist=self.hist,

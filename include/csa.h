@@ -83,11 +83,18 @@ csa_status csa_check_error_path(uint32_t polls, void* stream);
  *     among them.
  * Paths that cannot use the flag ignore it.  Results are the same with and without it. */
 #define CSA_EARLY_START 1u
-/* CSA_NO_CLUSTER in csa_attn_args.flags: a query whose keys are split over 2..8 CTAs normally merges
- * the partial softmax results inside the CTAs' thread-block cluster (distributed shared memory; no
- * workspace).  With this flag the partials go through the workspace and a merge kernel instead (e.g.
- * where cluster launches are unavailable).  Results agree to rounding. */
-#define CSA_NO_CLUSTER 2u
+/* CSA_CLUSTER_MERGE in csa_attn_args.flags: a query whose keys are split over 2..8 CTAs merges the
+ * partial softmax results inside the CTAs' thread-block cluster (distributed shared memory; no workspace
+ * partials, no merge kernel).  Without it the partials go through the workspace and a merge kernel,
+ * which measured faster for the 128K decode step on B200 (the cluster's CTAs must be co-scheduled in one
+ * GPC, and the merge adds code to a cold-instruction-cache kernel).  Results agree to rounding. */
+#define CSA_CLUSTER_MERGE 2u
+/* CSA_ONCHIP_TOPK in csa_index_args.flags (csa_index_topk, single-query Full rows of at most 32768 keys,
+ * d_I = 128, no pool): score and select each row inside one thread-block cluster of 8 CTAs, the scores
+ * never leaving shared memory.  Without it the scores go to the workspace with their histogram and a
+ * top-k kernel selects them, which measured faster for the 128K decode step on B200 (more CTAs stream
+ * the keys).  The selected sets are identical. */
+#define CSA_ONCHIP_TOPK 4u
 
 /* Paged caches ([V4.1 notes] §実装上の工夫: serving keeps the compressed KV in pages; the pages give no
  * layout, so this library fixes one).  A csa_page_map sends logical entry i of sequence b to row
@@ -256,7 +263,7 @@ typedef struct csa_index_args {
                               scores and falls back to the full selection); a row whose histogram counts
                               fewer than k scores (e.g. one no scoring call filled) is taken to hold only
                               that many.  NULL = plain radix selection */
-  uint32_t flags;          /* CSA_EARLY_START or 0 */
+  uint32_t flags;          /* CSA_EARLY_START | CSA_ONCHIP_TOPK, or 0 */
   csa_page_map k_pages;    /* k_codes / k_scales as a paged pool (table == NULL: contiguous) */
 } csa_index_args;
 
@@ -327,7 +334,7 @@ typedef struct csa_attn_args {
   const int64_t* win_pos0;
   void* out;
   float* lse;
-  uint32_t flags;          /* CSA_EARLY_START or 0 */
+  uint32_t flags;          /* CSA_EARLY_START | CSA_CLUSTER_MERGE, or 0 */
   /* Inverse-RoPE epilogue ([V4.1 notes] §実装上の工夫, inference kernels: the fused
      "RoPE-attention-RoPE-cast" kernel): nonzero rotates the last d_rope channels of out by the
      inverse of the query's RoPE, angle -t * out_rope_theta^(-2m/d_rope) for the half-split pair

@@ -35,7 +35,8 @@ def test_algorithmic_bytes():
     from csa_workloads import CFG2
     # per sequence: 512 entries x (224 codes + 16 scales + 128 rope + 4 id) + 128 KB window + q + out + lse
     assert b.attention_bytes(CFG2, 1) == 512 * 372 + 128 * 1024 + 2 * 64 * 1024 + 64 * 4
-    # fused index + top-k: 68 B per key read (64 codes + 4 scales), q_I and w in, 512 ids out
+    assert b.score_kernel_bytes(CFG2, 1) == 32768 * 72 + 8 * 128 * 2 + 8 * 4
+    # on-chip index + top-k: 68 B per key read (64 codes + 4 scales), q_I and w in, 512 ids out
     assert b.index_topk_bytes(CFG2, 1) == 32768 * 68 + 8 * 128 * 2 + 8 * 4 + 512 * 4
 
 

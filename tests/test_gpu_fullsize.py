@@ -34,10 +34,11 @@ def test_decode_cfg2_full_size(cuda_lib):
     layer.win.copy_(inp["win_kv"])
     out, lse, idx = layer.step(inp["C"], inp["Z"], inp["b_pos"], inp["W_IK"], inp["q"], inp["q_I"], inp["w"])
     torch.cuda.synchronize()
-    assert layer.fused                             # the step selected with the fused indexer + top-k
-    # the score rows the step selected from (kept on chip there), recomputed by the scoring call alone
-    cuda_lib.index_scores(inp["q_I"], inp["w"], layer.ki, layer.n_c, layer.q_pos, layer.scores, ratio=s.r)
+    # the on-chip top-k (scores kept in each row's cluster) selects the same sets from the same cache
+    idx_on, _, _ = cuda_lib.index_topk(inp["q_I"], inp["w"], layer.ki, layer.n_c, layer.q_pos, ratio=s.r, k=s.k,
+                                       onchip=True)
     torch.cuda.synchronize()
+    assert torch.equal(torch.sort(idx_on, dim=-1).values, torch.sort(idx, dim=-1).values)
     # property at full size, every sequence: a planted needle whose oracle score clears the kernel's
     # k-th score (with the boundary tolerance) is selected.  (A sequence whose head weights are all
     # <= 0 gives every key a score <= 0, so needles are not high-scoring there by construction.)

@@ -83,8 +83,9 @@ def test_paged_compress_append(cuda_lib):
         assert np.array_equal(gc[r0:], kc) and np.array_equal(gs[r0:], ks), f"k_I b={b}"
 
 
-@pytest.mark.parametrize("Nq,d_I,H_I", [(1, 128, 8), (5, 128, 8), (3, 64, 4)])
-def test_paged_index_topk(cuda_lib, Nq, d_I, H_I):
+@pytest.mark.parametrize("Nq,d_I,H_I,onchip", [(1, 128, 8, False), (1, 128, 8, True), (5, 128, 8, False),
+                                               (3, 64, 4, False)])
+def test_paged_index_topk(cuda_lib, Nq, d_I, H_I, onchip):
     """Decode (one query), speculative 5 positions, and the d_I = 64 path, over a paged index cache."""
     csa = cuda_lib
     B, n_max, page, k = 3, 3000, 256, 200
@@ -101,7 +102,7 @@ def test_paged_index_topk(cuda_lib, Nq, d_I, H_I):
     qp = torch.as_tensor(q_pos, device=DEV)
     scores = torch.full((B * Nq, n_max), float("nan"), dtype=torch.float32, device=DEV)
     csa.index_scores(qI.to(DEV), w.to(DEV), cache, n_c_t, qp, scores, ratio=4)
-    idx, _, _ = csa.index_topk(qI.to(DEV), w.to(DEV), cache, n_c_t, qp, ratio=4, k=k)
+    idx, _, _ = csa.index_topk(qI.to(DEV), w.to(DEV), cache, n_c_t, qp, ratio=4, k=k, onchip=onchip)
     torch.cuda.synchronize()
     got = scores.view(B, Nq, n_max).cpu().numpy()
     for b in range(B):

@@ -107,7 +107,7 @@ def test_compress_pooling_mode(cuda_lib, r, T, d, d_r, pos0):
 # ---------------------------------------------------------------------------------------- indexer
 
 def _index_case(csa, *, B, n_max, n_c, d_I, H_I, Nq, q_pos, k, g_q=1.0, g_k=1.0, key_std=1.0, seed=0,
-                cand=None, pool_blocks=0, identical_keys=False):
+                cand=None, pool_blocks=0, identical_keys=False, onchip=False):
     G = gen(seed)
     kI = normal((B, n_max, d_I), key_std, G)
     if identical_keys:
@@ -120,7 +120,7 @@ def _index_case(csa, *, B, n_max, n_c, d_I, H_I, Nq, q_pos, k, g_q=1.0, g_k=1.0,
     q_pos_t = torch.tensor(q_pos, dtype=torch.int64).view(B, Nq)
     idx, sc, pool = csa.index_topk(qI.to(DEV), w.to(DEV), kc, n_c_t.to(DEV), q_pos_t.to(DEV), ratio=4, k=k, g_q=g_q,
                                    cand=cand.to(DEV) if cand is not None else None, pool_blocks=pool_blocks,
-                                   want_scores=True)
+                                   want_scores=True, onchip=onchip)
     torch.cuda.synchronize()
     swaps = 0
     for b in range(B):
@@ -171,10 +171,22 @@ def test_index_cfg1_small_layer(cuda_lib):
                 g_q=1.0, g_k=2.0 ** -4, key_std=0.03)
 
 
-def test_index_decode_ragged(cuda_lib):
+ONCHIP = pytest.mark.parametrize("onchip", [False, True], ids=["split", "onchip"])
+
+
+@ONCHIP
+def test_index_decode_ragged(cuda_lib, onchip):
     n_c = [4096, 1000, 37, 2048]
     q_pos = [4 * 4096 - 1, 4 * 1000 - 1, 4 * 37 - 1, 4 * 500 + 2]   # last: only 500 visible
-    _index_case(cuda_lib, B=4, n_max=4096, n_c=n_c, d_I=128, H_I=8, Nq=1, q_pos=q_pos, k=512, seed=1)
+    _index_case(cuda_lib, B=4, n_max=4096, n_c=n_c, d_I=128, H_I=8, Nq=1, q_pos=q_pos, k=512, seed=1, onchip=onchip)
+
+
+def test_index_onchip_full_row_and_k_above_visible(cuda_lib):
+    """The on-chip top-k at its largest row (32768 keys: 16 tiles per CTA of the cluster) and with
+    k larger than the visible entries (slots past k_eff are -1)."""
+    n = 32768
+    _index_case(cuda_lib, B=2, n_max=n, n_c=[n, 300], d_I=128, H_I=8, Nq=1, q_pos=[4 * n - 1, 4 * 300 - 1],
+                k=512, seed=13, onchip=True)
 
 
 def test_index_prefill_causal_multi_query(cuda_lib):
@@ -247,18 +259,20 @@ def test_index_hierarchical_pool(cuda_lib):
                 q_pos=[4 * 8192 - 1, 4 * 4000 + 1], k=128, seed=6, pool_blocks=64)
 
 
-def test_index_exact_ties_take_smallest_ids(cuda_lib):
+@ONCHIP
+def test_index_exact_ties_take_smallest_ids(cuda_lib, onchip):
     idx, swaps = _index_case(cuda_lib, B=1, n_max=64, n_c=[64], d_I=128, H_I=8, Nq=1, q_pos=[255], k=10, seed=7,
-                             identical_keys=True)
+                             identical_keys=True, onchip=onchip)
     assert swaps == 0
     assert sorted(idx[0, 0].tolist()) == list(range(10))
 
 
-def test_index_exact_ties_overflow_the_boundary_buffer(cuda_lib):
+@ONCHIP
+def test_index_exact_ties_overflow_the_boundary_buffer(cuda_lib, onchip):
     # 20000 equal scores: the histogram's boundary bin holds more candidates than the selection buffer,
     # so the row takes the full selection path; the smallest ids must still win
     idx, swaps = _index_case(cuda_lib, B=1, n_max=20000, n_c=[20000], d_I=128, H_I=8, Nq=1, q_pos=[80000], k=10,
-                             seed=9, identical_keys=True)
+                             seed=9, identical_keys=True, onchip=onchip)
     assert swaps == 0 and sorted(idx[0, 0].tolist()) == list(range(10))
 
 
@@ -272,7 +286,7 @@ def test_index_k_larger_than_visible(cuda_lib):
 # -------------------------------------------------------------------------------------- attention
 
 def _attn_case(csa, *, B, Nq, H, d, d_r, n_max, n_c, q_pos, k=0, Wn=128, win_pos0=None, hca=False, ratio=4,
-               seed=0, g=1.0, q_scale=1.0, rope_theta=0.0, win_fp8=False, early_start=False, cluster=True):
+               seed=0, g=1.0, q_scale=1.0, rope_theta=0.0, win_fp8=False, early_start=False, cluster=False):
     """win_fp8: the window rows are FP8-packed on the GPU (csa_pack_fp8_window) and the oracle attends over
     its own FP8 pack of the same bf16 rows, dequantised (the pack itself is checked bit-exact elsewhere)."""
     G = gen(seed)
@@ -477,7 +491,7 @@ def test_attn_fp8_window_partial_multi_query_and_hca(cuda_lib):
 def test_attn_cluster_merge_sizes(cuda_lib, k, cluster):
     """Two decode queries whose key lists span 2, 4, 6, 8 and 9 tiles of 128 keys (k entries + the
     128-row window): 2..8 CTAs per query merge inside their thread-block cluster, 9 go through the
-    workspace partials and the merge kernel; with CSA_NO_CLUSTER every split count takes the merge kernel."""
+    workspace partials and the merge kernel; without CSA_CLUSTER_MERGE every split count takes the merge kernel."""
     n = 4096
     _attn_case(cuda_lib, B=2, Nq=1, H=64, d=512, d_r=64, n_max=n, n_c=[n, n - 100], q_pos=[4 * n - 1, 4 * n - 401],
                k=k, seed=60 + k // 128, cluster=cluster)
