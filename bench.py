@@ -49,6 +49,9 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=400)
     p.add_argument("--cpu-sample", type=int, default=2, help="sequences the CPU oracle times (cpu_baseline)")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the other workloads (cfg1, cfg3 prefill, cfg4, cfg5) that a 1-GPU run times after the "
+                        "headline")
     p.add_argument("--profile", action="store_true",
                    help="profiling case: one layer state, --steps eager steps, no timing (for ncu)")
     p.add_argument("--rows", action="store_true",
@@ -466,6 +469,8 @@ def run_ours(args, rank, world):
     }
     if world == 1 or rank == 0:
         line["cpu_baseline"] = cpu_baseline(args.cpu_sample) if (world == 1 and args.cpu_sample > 0) else None
+    if world == 1 and not args.no_configs:
+        line["other_configs"] = other_configs()
     print(json.dumps(line), flush=True)
 
 
@@ -573,14 +578,15 @@ def _tensor_peak(sustained=False):
     return (1400.0 if sustained else 1590.0), "fallback"
 
 
-def run_rows(args):
+def rows_measure(with_cpu=True):
     """The rows of the hot path that the decode step does not exercise, each timed with CUDA events on
     its own synthetic workload (caches rotated so they are read from HBM), against its roofline, with
-    the oracle timed on one sequence beside it."""
+    the oracle timed on one sequence beside it (with_cpu).  Returns one dict per row."""
     import compressed_sparse_attention_18_b200 as csa
     from csa_workloads import CFG4_HCA, CFG4_REUSE, CFG5, decode_inputs, gen, normal
-    from oracle import csa_oracle as O
     from threadpoolctl import threadpool_limits
+    if with_cpu:
+        from oracle import csa_oracle as O
     dev = torch.device("cuda", 0)
     hbm, hkind = peaks()
     tfl, tkind = _tensor_peak()
@@ -588,8 +594,21 @@ def run_rows(args):
     def f64(x):
         return x.double().cpu().numpy()
 
+    res = []
+
     def emit(d):
-        print(json.dumps(d), flush=True)
+        if not with_cpu:
+            d.pop("cpu_baseline", None)
+        res.append(d)
+
+    def cpu_time(fn):
+        """seconds of one single-threaded oracle call (None when the oracle is not timed)"""
+        if not with_cpu:
+            return None
+        with threadpool_limits(1):
+            t0 = time.perf_counter()
+            fn()
+            return time.perf_counter() - t0
 
     # ---- a1 in HCA mode: 128x pooling of one 1,048,576-token sequence (C, Z read once: 2 GB)
     s = CFG4_HCA
@@ -602,16 +621,16 @@ def run_rows(args):
                                           c_out=c_out), 10)
     nbytes = 2 * s.T * s.d * 2 + (s.T // s.r) * s.d * 2
     cC, cZ, cb = f64(C[0, :64 * s.r]), f64(Z[0, :64 * s.r]), f64(b_pos)
-    with threadpool_limits(1):
-        t0 = time.perf_counter()
+
+    def pool64():
         for e in range(64):
             O.compress_pool(cC[e * s.r:(e + 1) * s.r], cZ[e * s.r:(e + 1) * s.r], cb, s.r, s.d_r, 10000.0, e * s.r)
-        el = time.perf_counter() - t0
+    el = cpu_time(pool64)
     emit({"row": "a1 compress (HCA pooling, r=128)", "workload": "1 sequence x 1,048,576 tokens -> 8192 entries",
           "ms": ms, "value": (s.T // s.r) / (ms / 1e3), "unit": "entries/s",
           "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm, "peak_kind": hkind,
                        "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / hbm, "algorithmic_bytes": nbytes},
-          "cpu_baseline": {"value": 64 / el, "unit": "entries/s", "cores": 1, "kind": "oracle",
+          "cpu_baseline": {"value": 64 / el if el else None, "unit": "entries/s", "cores": 1, "kind": "oracle",
                            "sample": "64 entries of the same sequence"}})
     del C, Z, c_out
     torch.cuda.empty_cache()
@@ -641,19 +660,18 @@ def run_rows(args):
     ms = _event_ms(hca, 40)
     flops = s.B * 4 * s.H * (s.n_c + s.W) * s.d
     nbytes = s.B * (s.n_c * (s.d_n // 2 + 16 + s.d_r * 2) + s.W * s.d * 2 + 2 * s.H * s.d * 2)
-    rows = O.entry_kv(st0["cache"].codes[0].cpu().numpy(), st0["cache"].scales[0].cpu().numpy(),
-                      f64(st0["cache"].rope[0]), s.d_n, 1.0)
-    with threadpool_limits(1):
-        t0 = time.perf_counter()
-        O.hca_attention(f64(st0["q"][0]), [s.T - 1], rows, s.n_c, s.r, f64(st0["win_kv"][0]), s.T - s.W, s.W,
-                        s.d ** -0.5)
-        el = time.perf_counter() - t0
+    el = None
+    if with_cpu:
+        rows = O.entry_kv(st0["cache"].codes[0].cpu().numpy(), st0["cache"].scales[0].cpu().numpy(),
+                          f64(st0["cache"].rope[0]), s.d_n, 1.0)
+        el = cpu_time(lambda: O.hca_attention(f64(st0["q"][0]), [s.T - 1], rows, s.n_c, s.r, f64(st0["win_kv"][0]),
+                                              s.T - s.W, s.W, s.d ** -0.5))
     emit({"row": "a6 HCA dense attention", "workload": "16 sequences x (8192 entries + 128 window), 64 heads x 512",
           "ms": ms, "value": s.B / (ms / 1e3), "unit": "tokens/s",
           "roofline": {"bound": "tensor", "achieved": flops / (ms / 1e3) / 1e12, "peak": tfl, "peak_kind": tkind,
                        "unit": "TFLOP/s", "frac": flops / (ms / 1e3) / 1e12 / tfl, "algorithmic_flops": flops,
                        "hbm_frac": nbytes / (ms / 1e3) / 1e9 / hbm, "algorithmic_bytes": nbytes},
-          "cpu_baseline": {"value": 1 / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+          "cpu_baseline": {"value": 1 / el if el else None, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                            "sample": "1 sequence of the same workload"}})
     del states, ws, st0
     torch.cuda.empty_cache()
@@ -698,24 +716,32 @@ def run_rows(args):
         nbytes = B * (s.n_c * per_key + (s.pool_blocks * 8 if s is CFG5 else s.k) * per_key)
         if s is CFG4_REUSE:
             nbytes += B * (k2 * (s.d_n // 2 + 16 + s.d_r * 2) + s.W * s.d * 2 + 2 * s.H * s.d * 2)
-        st = sts[0]
-        codes, scales = st["ki"].codes[0].cpu().numpy(), st["ki"].scales[0].cpu().numpy()
-        t = int(st["q_pos"][0, 0])
-        with threadpool_limits(1):
-            t0 = time.perf_counter()
-            sc, ids = O.index_scores(f64(st["q_I"][0, 0])[None], f64(st["w"][0, 0])[None], 1.0, codes, scales, 1.0,
-                                     [t], s.n_c, s.r)
-            O.topk(sc, ids, s.k)
-            el = time.perf_counter() - t0
+        el = None
+        if with_cpu:
+            st = sts[0]
+            codes, scales = st["ki"].codes[0].cpu().numpy(), st["ki"].scales[0].cpu().numpy()
+            t = int(st["q_pos"][0, 0])
+
+            def level1():
+                sc, ids = O.index_scores(f64(st["q_I"][0, 0])[None], f64(st["w"][0, 0])[None], 1.0, codes, scales,
+                                         1.0, [t], s.n_c, s.r)
+                O.topk(sc, ids, s.k)
+            el = cpu_time(level1)
         emit({"row": name, "workload": f"{B} sequences x {s.n_c} entries, top-{s.k}" +
               (f", pool {s.pool_blocks}x8" if s is CFG5 else f", Reindex -> top-{k2}, attention"),
               "ms": ms, "value": B / (ms / 1e3), "unit": "tokens/s",
               "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm, "peak_kind": hkind,
                            "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / hbm, "algorithmic_bytes": nbytes},
-              "cpu_baseline": {"value": 1 / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+              "cpu_baseline": {"value": 1 / el if el else None, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                                "sample": "level-1 index + top-k of 1 sequence (a lower bound on the oracle's time)"}})
         del sts
         torch.cuda.empty_cache()
+    return res
+
+
+def run_rows(args):
+    for d in rows_measure(with_cpu=True):
+        print(json.dumps(d), flush=True)
 
 
 def run_flops(args):
@@ -825,6 +851,88 @@ def run_spec(args):
                               "4 cache states rotated (inputs larger than L2)"}), flush=True)
 
 
+def cfg1_measure(reps=100):
+    """The small layer (4096-token sequence, 8 heads x 128, indexer 4 x 64, top-64, 16 decode positions).
+    One pass = the compressor in projection mode over the whole sequence (C = x W_kv and Z = x W_g on the
+    tensor cores, gated pooling with RoPE, k_I, FP4 appends of the 1024 entries and their indexer keys),
+    then index + top-64 and attention over the selected entries plus the 128-token window for the 16
+    positions.  The pass is replayed from one CUDA graph; L2 is flushed (a 256 MB write) before every
+    timed pass and each pass is bracketed by its own events.  Returns the row's dict."""
+    import compressed_sparse_attention_18_b200 as csa
+    from csa_workloads import CFG1, small_layer_inputs
+    s = CFG1
+    dev = torch.device("cuda", 0)
+    inp = small_layer_inputs(s, seed=0, device=dev)
+    n = s.n_c
+    bf, i32, i64 = torch.bfloat16, torch.int32, torch.int64
+    kv = csa.PackedCache(1, n, s.d, s.d_r, dev, s.g)
+    ki = csa.PackedCache(1, n, s.d_I, 0, dev, s.g)
+    C = torch.empty((1, s.T, s.d), dtype=bf, device=dev)
+    Z = torch.empty((1, s.T, s.d), dtype=bf, device=dev)
+    c_out = torch.empty((1, n, s.d), dtype=bf, device=dev)
+    kI_out = torch.empty((1, n, s.d_I), dtype=bf, device=dev)
+    row0 = torch.zeros((1,), dtype=i32, device=dev)
+    pos0 = torch.zeros((1,), dtype=i64, device=dev)
+    win_pos0 = torch.zeros((1,), dtype=i64, device=dev)
+    n_c = torch.full((1,), n, dtype=i32, device=dev)
+    idx = torch.empty((1, s.Nq, s.k), dtype=i32, device=dev)
+    out = torch.empty((1, s.Nq, s.H, s.d), dtype=bf, device=dev)
+    lse = torch.empty((1, s.Nq, s.H), dtype=torch.float32, device=dev)
+    q_pos = inp["q_pos"]
+    ws_i = torch.empty(max(csa.index_topk_workspace_size(inp["q_I"], inp["w"], ki, n_c, q_pos, ratio=s.r, k=s.k), 1),
+                       dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(max(csa.attn_workspace_size(inp["q"], q_pos, kv, n_c, idx, C, win_pos0, ratio=s.r,
+                                                   window=s.W), 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
+
+    def one_pass():
+        csa.compress(x=inp["x"], W_kv=inp["W_kv"], W_g=inp["W_g"], b_pos=inp["b_pos"], ratio=s.r, d_rope=s.d_r,
+                     rope_theta=10000.0, pos0=pos0, W_IK=inp["W_IK"], C=C, Z=Z, c_out=c_out, kI_out=kI_out,
+                     kv_cache=kv, ki_cache=ki, row0=row0, stream=stream)
+        csa.index_topk(inp["q_I"], inp["w"], ki, n_c, q_pos, ratio=s.r, k=s.k, idx_out=idx, ws=ws_i, stream=stream)
+        csa.sparse_attn(inp["q"], q_pos, kv, n_c, idx, C, win_pos0, ratio=s.r, window=s.W, out=out, lse=lse,
+                        ws=ws_a, stream=stream)
+
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        one_pass()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        one_pass()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        for a, b in ev:
+            flush.fill_(1)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+    stream.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / reps
+    hbm, kind = peaks()
+    # dominant algorithmic bytes: x and both weights read, C and Z written once and read once by the pooling,
+    # the two FP4 caches written; the 16 positions' index and attention reads are a few hundred KB more
+    nbytes = (s.T * s.d_m * 2 + 2 * s.d_m * s.d * 2 + 2 * 2 * s.T * s.d * 2
+              + n * (s.d_n // 2 + s.d_n // 32 + 2 * s.d_r) + n * (s.d_I // 2 + s.d_I // 32))
+    return {"row": "cfg1 small layer (compress 4096 tokens + 16 decode positions)", "workload": s.name,
+            "ms": ms, "value": s.Nq / (ms / 1e3), "unit": "query tokens/s",
+            "tokens_compressed_per_s": s.T / (ms / 1e3), "l2": "flushed before every timed pass",
+            "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm, "peak_kind": kind,
+                         "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / hbm, "algorithmic_bytes": nbytes}}
+
+
+def other_configs():
+    """Every other workload of the hot path timed on the device in the default run (the oracle is timed
+    only for the headline workload here; `--prefill` and `--rows` time it beside each row)."""
+    res = [cfg1_measure(), prefill_measure(3, 3, with_cpu=False)]
+    torch.cuda.empty_cache()
+    res += rows_measure(with_cpu=False)
+    return res
+
+
 def prefill_work(s):
     """Algorithmic work of the whole chunked prefill of one sequence (s.T tokens): the compressor's two
     projections (bf16 FLOPs), the causal indexer's FP4 products (query t scores (t+1) // r entries), and
@@ -840,15 +948,21 @@ def prefill_work(s):
 
 
 def run_prefill(args):
+    steps = max(args.steps if args.steps < 1000 else 10, 1)
+    warm = max(args.warmup if args.warmup < 1000 else 3, 3)
+    print(json.dumps(prefill_measure(steps, warm, with_cpu=True)), flush=True)
+
+
+def prefill_measure(steps, warm, with_cpu=True):
     """Chunked causal prefill of one 32768-token sequence in 4096-token chunks (d_m = 4096, 64 heads x
     512, indexer 8 x 128 FP4, top-512, window 128).  Per chunk: the compressor (projection GEMM on the
     tensor cores, gated pooling, FP4 append of the chunk's 1024 entries and their indexer keys), the
     multi-query indexer over every entry so far with the causal mask, top-512 per query, attention over
     the selected entries plus the window.  One step = the 8 chunks, replayed from one CUDA graph; inputs
-    (x 256 MB, q 2 GB) are larger than L2.  One JSON line."""
+    (x 256 MB, q 2 GB) are larger than L2.  Returns the JSON line's dict (the oracle timed beside it when
+    with_cpu)."""
     import compressed_sparse_attention_18_b200 as csa
     from csa_workloads import CFG3, gen, normal
-    from oracle import csa_oracle as O
     from threadpoolctl import threadpool_limits
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -913,7 +1027,6 @@ def run_prefill(args):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
         prefill()
-    steps, warm = max(args.steps if args.steps < 1000 else 10, 1), max(args.warmup if args.warmup < 1000 else 3, 3)
     with torch.cuda.stream(stream):
         for _ in range(warm):
             g.replay()
@@ -944,24 +1057,27 @@ def run_prefill(args):
     def tf(flops, ms_):
         return flops / (ms_ / 1e3) / 1e12
 
-    # oracle on a bounded sample: the projection of 4 tokens, and index + top-k + attention of 2 queries
-    # of the last chunk (over all 8192 entries), 1 thread
-    f64 = lambda t_: t_.double().cpu().numpy()  # noqa: E731
-    codes, scales = kv.codes[0].cpu().numpy(), kv.scales[0].cpu().numpy()
-    kcodes, kscales = ki.codes[0].cpu().numpy(), ki.scales[0].cpu().numpy()
-    rows = O.entry_kv(codes, scales, f64(kv.rope[0]), s.d_n, 1.0)
-    win = f64(C[0, s.T - Lc - s.W:])
-    with threadpool_limits(1):
-        t0 = time.perf_counter()
-        O.project(f64(x[-1, :4]), f64(W_kv))
-        O.project(f64(x[-1, :4]), f64(W_g))
-        for qq in (Lc - 2, Lc - 1):
-            t = s.T - Lc + qq
-            sc, ids = O.index_scores(f64(q_I[-1, qq])[None], f64(w[-1, qq])[None], 1.0, kcodes, kscales, 1.0, [t], n,
-                                     s.r)
-            sel, _ = O.topk(sc, ids, s.k)
-            O.attention(f64(q[-1, qq])[None], [t], rows, sel, n, win, s.T - Lc - s.W, s.W, s.d ** -0.5)
-        el = time.perf_counter() - t0
+    el = None
+    if with_cpu:
+        # oracle on a bounded sample: the projection of 4 tokens, and index + top-k + attention of 2 queries
+        # of the last chunk (over all 8192 entries), 1 thread
+        from oracle import csa_oracle as O
+        f64 = lambda t_: t_.double().cpu().numpy()  # noqa: E731
+        codes, scales = kv.codes[0].cpu().numpy(), kv.scales[0].cpu().numpy()
+        kcodes, kscales = ki.codes[0].cpu().numpy(), ki.scales[0].cpu().numpy()
+        rows = O.entry_kv(codes, scales, f64(kv.rope[0]), s.d_n, 1.0)
+        win = f64(C[0, s.T - Lc - s.W:])
+        with threadpool_limits(1):
+            t0 = time.perf_counter()
+            O.project(f64(x[-1, :4]), f64(W_kv))
+            O.project(f64(x[-1, :4]), f64(W_g))
+            for qq in (Lc - 2, Lc - 1):
+                t = s.T - Lc + qq
+                sc, ids = O.index_scores(f64(q_I[-1, qq])[None], f64(w[-1, qq])[None], 1.0, kcodes, kscales, 1.0,
+                                         [t], n, s.r)
+                sel, _ = O.topk(sc, ids, s.k)
+                O.attention(f64(q[-1, qq])[None], [t], rows, sel, n, win, s.T - Lc - s.W, s.W, s.d ** -0.5)
+            el = time.perf_counter() - t0
     line = {"row": "cfg3 chunked causal prefill", "workload": s.name,
             "config": {"B": 1, "tokens": s.T, "chunk": Lc, "d_model": s.d_m, "heads": s.H, "head_dim": s.d,
                        "indexer": f"{s.H_I}x{s.d_I} fp4", "top_k": s.k, "window": s.W,
@@ -979,8 +1095,10 @@ def run_prefill(args):
                          "frac": tf(work["attention"], stage["attention"]) / tfl_s},
             "cpu_baseline": {"value": 2 / el, "unit": "query tokens/s", "cores": 1, "kind": "oracle",
                              "sample": "projection of 4 tokens + index/top-k/attention of 2 queries of the last "
-                                       "chunk, numpy fp64, 1 thread"}}
-    print(json.dumps(line), flush=True)
+                                       "chunk, numpy fp64, 1 thread"} if el else None}
+    if not with_cpu:
+        line.pop("cpu_baseline")
+    return line
 
 
 def run_profile_prefill(args):
