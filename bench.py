@@ -400,11 +400,13 @@ def run_ours(args, rank, world):
     steps.prepare(max(args.warmup, 3), args.steps)
     steps.prepare(LAYERS, with_marks=True)
     steps.freeze()
-    steps.run(max(args.warmup, 3))
-    stream.synchronize()
     clk = ClockSampler(local)
     clk.start()
     time.sleep(0.3)
+    # the warm-up steps run right before the timed region (after the sampler's start-up, which leaves the
+    # GPU idle), then a synchronize and the barrier
+    steps.run(max(args.warmup, 3))
+    stream.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -1027,13 +1029,13 @@ def prefill_measure(steps, warm, with_cpu=True):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
         prefill()
+    clk = ClockSampler(0)
+    clk.start()
+    time.sleep(0.3)
     with torch.cuda.stream(stream):
         for _ in range(warm):
             g.replay()
     stream.synchronize()
-    clk = ClockSampler(0)
-    clk.start()
-    time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     with torch.cuda.stream(stream):

@@ -58,6 +58,7 @@ struct TaSmem {
 
 struct TaParams {
   int Nq, H, ratio, n_max, k, Wn, window, splits, hca;
+  int rows;             // B * Nq
   int tpc;              // key tiles per CTA (a CTA walks tiles split*tpc .. split*tpc + tpc - 1 of its query)
   int cluster;          // the `splits` CTAs of a query form one thread-block cluster and merge their
                         // partials through distributed shared memory (no workspace partials, no merge kernel)
@@ -728,6 +729,484 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------------------------------------------
+// Persistent variant, for many queries of several tiles each with one CTA per query (the chunked
+// prefill's 4096 queries per chunk, multi-position decode): one CTA per SM takes the queries blockIdx.x,
+// blockIdx.x + gridDim.x, ... one after another, each over all of its key tiles.  The tiles of its queries
+// form one stream through the same barriers: the next query's Q is loaded by TMA as soon as the S MMAs of
+// the current query's last tile have read Q, the next query's first tile is gathered as the current
+// query's last O MMAs release the K tile, and the current query's epilogue runs while that tile's S MMAs
+// do.  BF16 window rows only.
+
+// A query's positions and lengths, read one query ahead (plain loads, used a tile or more later).
+struct TaUnitRaw {
+  int bq, nc;
+  long long tq, wp0;
+};
+struct TaUnit {
+  int bq, b, n_sel, n_list, ntile, ncb;
+  int wofs;             // window buffer row of the first window key (wlo - win_pos0)
+};
+
+__device__ __forceinline__ TaUnitRaw ta_unit_load(const TaParams& P, int bq) {
+  TaUnitRaw r;
+  const int b = bq / P.Nq;
+  r.bq = bq;
+  r.tq = P.q_pos[bq];
+  r.nc = P.n_c[b];
+  r.wp0 = P.Wn > 0 ? P.win_pos0[b] : 0;
+  return r;
+}
+
+// The query's key list [n_sel entries ‖ window rows] (the per-query kernel's rule).
+__device__ __forceinline__ TaUnit ta_unit(const TaParams& P, const TaUnitRaw& r) {
+  TaUnit u;
+  u.bq = r.bq;
+  u.b = r.bq / P.Nq;
+  u.ncb = min(r.nc, P.n_max);
+  u.n_sel = P.k;
+  if (P.hca) u.n_sel = (int)max(0LL, min((r.tq + 1) / P.ratio, (long long)u.ncb));
+  long long wlo = 0, whi = -1;
+  if (P.Wn > 0) {
+    wlo = max(max(0LL, r.tq - P.window + 1), r.wp0);
+    whi = min(r.tq, r.wp0 + P.Wn - 1);
+  }
+  u.wofs = whi >= wlo ? (int)(wlo - r.wp0) : 0;   // in [0, Wn) when the window is not empty
+  u.n_list = u.n_sel + (whi >= wlo ? (int)(whi - wlo + 1) : 0);
+  u.ntile = (u.n_list + TA_KEYS - 1) / TA_KEYS;
+  return u;
+}
+
+// Tile t of a query's key list.
+__device__ __forceinline__ TaTile ta_tile_u(const TaUnit& u, int t) {
+  return ta_tile(t * TA_KEYS, u.n_sel, u.n_list, u.wofs, 0, false);
+}
+
+// The first query with keys among units kk, kk+1, ... of this CTA (from `raw` if those are unit kk's
+// positions), writing the outputs of the ones without keys (zero rows, lse = -inf) with threads
+// tid < nthreads; bq = -1 if there is none.
+__device__ __forceinline__ TaUnit ta_next_unit(const TaParams& P, int kk, int nu, TaUnitRaw raw, int tid,
+                                               int nthreads) {
+  TaUnit uu{};
+  uu.bq = -1;
+#pragma unroll 1
+  for (; kk < nu; ++kk) {
+    const int bq = (int)blockIdx.x + kk * (int)gridDim.x;
+    if (raw.bq != bq) raw = ta_unit_load(P, bq);
+    uu = ta_unit(P, raw);
+    if (uu.ntile > 0) return uu;
+    for (int i = tid; i < P.H * 256; i += nthreads) reinterpret_cast<uint32_t*>(P.out + (size_t)bq * P.H * 512)[i] = 0u;
+    if (P.lse && tid < P.H) P.lse[(size_t)bq * P.H + tid] = -INFINITY;
+    uu.bq = -1;
+  }
+  return uu;
+}
+
+// Epilogue of a query, by the 8 worker warps once its last O MMAs have completed (phase `par` of bar_o):
+// O^T / l from tensor memory to bf16 rows [head][512], and lse; resets the running max and sum for
+// the next query.  Returns false if a wait gave up.
+__device__ __forceinline__ bool ta_epilogue(TaSmem& S, const TaParams& P, int bq, uint32_t par, uint32_t lane_base,
+                                            int hh, int quad, int lane, int tid) {
+  bool ok = true;
+  if (tid < 64) {
+    const float lh = S.l[tid];
+    S.fac[tid] = lh > 0.f ? 1.f / lh : 0.f;
+    if (tid < P.H && P.lse) P.lse[(size_t)bq * P.H + tid] = lh > 0.f ? (S.m[tid] + log2f(lh)) * TA_LN2 : -INFINITY;
+    S.m[tid] = -INFINITY;
+    S.l[tid] = 0.f;
+  }
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+  const int hmax = min(32, P.H - hh * 32);
+#pragma unroll 1
+  for (int mt = 0; mt < 4; ++mt) {
+    ok = ok && mbar_wait(&S.bar_o[mt], par);
+    tc_fence_after();
+    uint32_t ov[32];
+    tmem_ld_x32(lane_base + TA_COL_O + 64 * mt + hh * 32, ov);
+    tmem_wait_ld_x32(ov);
+    const int dim = 128 * mt + 32 * quad + lane;
+    uint16_t* o = P.out + ((size_t)bq * P.H + hh * 32) * 512 + dim;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      const float4 il = *reinterpret_cast<const float4*>(&S.fac[hh * 32 + j]);
+      if (j < hmax) o[(size_t)j * 512] = (uint16_t)f_to_bf16_bits(__uint_as_float(ov[j]) * il.x);
+      if (j + 1 < hmax) o[(size_t)(j + 1) * 512] = (uint16_t)f_to_bf16_bits(__uint_as_float(ov[j + 1]) * il.y);
+      if (j + 2 < hmax) o[(size_t)(j + 2) * 512] = (uint16_t)f_to_bf16_bits(__uint_as_float(ov[j + 2]) * il.z);
+      if (j + 3 < hmax) o[(size_t)(j + 3) * 512] = (uint16_t)f_to_bf16_bits(__uint_as_float(ov[j + 3]) * il.w);
+    }
+  }
+  tc_fence_before();
+  asm volatile("bar.sync 1, 256;" ::: "memory");   // every worker has read fac (the softmax rewrites it)
+  return ok;
+}
+
+__global__ void __launch_bounds__(TA_THREADS, 1)
+    attn_tc_persist_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap wmap,
+                           const TaParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  TaSmem& S = *reinterpret_cast<TaSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grow = (tid & (TA_WORKERS - 1)) >> 1, ghalf = tid & 1;
+  // this CTA's queries: unit u is query blockIdx.x + u * gridDim.x
+  const int nu = (int)blockIdx.x < P.rows ? (P.rows - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  auto unit_q = [&](int u) { return (int)blockIdx.x + u * (int)gridDim.x; };
+  if (warp == 8) {
+    if (lane == 0) {
+      S.err = 0;
+      for (int j = 0; j < 8; ++j) {
+        mbar_init(&S.bar_q[j], 1);
+        mbar_init(&S.bar_w[j], 1);
+        mbar_init(&S.bar_k[j], TA_WORKERS / 32);
+      }
+      mbar_init(&S.bar_s, 1);
+      mbar_init(&S.bar_p, TA_WORKERS / 32);
+      for (int j = 0; j < 4; ++j) mbar_init(&S.bar_o[j], 1);
+      fence_mbar_init();
+      prefetch_tensormap(&qmap);
+      prefetch_tensormap(&wmap);
+    }
+    __syncwarp();
+    tmem_alloc(&S.tmem_base, TA_TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (tid < 64) { S.m[tid] = -INFINITY; S.l[tid] = 0.f; }
+  if (tid == 0) S.rescale = 0;
+  pdl_trigger();
+  pdl_wait();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = S.tmem_base;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------------ control: TMA, then MMA issue
+    if (lane == 0) {
+      bool ok = true;
+      const uint32_t ids = idesc_bf16(128, 64, 0, 0);
+      const uint32_t ido = idesc_bf16(128, 64, 1, 1);
+      auto load_q = [&](int bq) {
+#pragma unroll 1
+        for (int j = 0; j < 8; ++j) {
+          mbar_arrive_expect_tx(&S.bar_q[j], 64 * 128);
+          tma_load_3d(S.Q[j], &qmap, j * 64, 0, bq, &S.bar_q[j]);
+        }
+      };
+      // first query with keys (a query without keys has no tiles: the workers write its output)
+      int k = 0;
+      TaUnit u{};
+      for (; k < nu; ++k) {
+        u = ta_unit(P, ta_unit_load(P, unit_q(k)));
+        if (u.ntile > 0) break;
+      }
+      if (k < nu) load_q(u.bq);
+      uint32_t f = 0, qk = 0;                  // tiles and queries with keys so far
+#pragma unroll 1
+      while (k < nu && ok) {
+        const TaUnitRaw nraw = k + 1 < nu ? ta_unit_load(P, unit_q(k + 1)) : TaUnitRaw{};
+#pragma unroll 1
+        for (int t = 0; t < u.ntile && ok; ++t, ++f) {
+          const TaTile g = ta_tile_u(u, t);
+          const int nbox = (g.we - g.wa) / TA_WBOX;
+          // window boxes overwrite the K tile: only once the previous tile's O MMAs have completed
+          if (f > 0 && nbox > 0) ok = mbar_wait(&S.bar_o[3], (f - 1) & 1);
+#pragma unroll 1
+          for (int j = 0; j < 8; ++j) {
+            mbar_arrive_expect_tx(&S.bar_w[j], (uint32_t)(nbox * TA_WBOX * 128));
+            if (ok)
+              for (int i = 0; i < nbox; ++i)
+                tma_load_3d(&S.K[j][(g.wa + i * TA_WBOX) * 128], &wmap, j * 64,
+                            (int)(g.wrow_base + g.wa + i * TA_WBOX), u.b, &S.bar_w[j]);
+          }
+#pragma unroll 1
+          for (int j = 0; j < 8 && ok; ++j) {
+            ok = (t > 0 || mbar_wait(&S.bar_q[j], qk & 1)) && mbar_wait(&S.bar_w[j], f & 1) &&
+                 mbar_wait(&S.bar_k[j], f & 1);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int s2 = 0; s2 < 4; ++s2) {
+              const uint64_t a = smem_desc(smem_addr(S.K[j]) + s2 * 32, 16, 1024, 2);
+              const uint64_t bd = smem_desc(smem_addr(S.Q[j]) + s2 * 32, 16, 1024, 2);
+              mma_bf16_ss(tb + TA_COL_S, a, bd, ids, (j | s2) != 0);
+            }
+          }
+          mma_commit(&S.bar_s);
+          if (t + 1 == u.ntile && k + 1 < nu && ok) {
+            // the next query with keys; its Q replaces this one's once this tile's S MMAs have read it
+            int kn = k + 1;
+            TaUnit un = ta_unit(P, nraw);
+            while (un.ntile == 0 && ++kn < nu) un = ta_unit(P, ta_unit_load(P, unit_q(kn)));
+            if (kn < nu) {
+              ok = mbar_wait(&S.bar_s, f & 1);
+              if (ok) load_q(un.bq);
+            }
+          }
+          // O^T (+)= V^T P^T; the first tile of a query starts its accumulator afresh (the previous
+          // query's epilogue has read it: the workers arrive on bar_p only after that)
+          ok = ok && mbar_wait(&S.bar_p, f & 1);
+          if (ok) tc_fence_after();
+#pragma unroll 1
+          for (int mt = 0; mt < 4; ++mt) {
+            if (ok) {
+#pragma unroll
+              for (int s2 = 0; s2 < 8; ++s2) {
+                const uint64_t a = smem_desc(smem_addr(S.K[2 * mt]) + s2 * 2048, 16384, 1024, 2);
+                const uint64_t bd = smem_desc(smem_addr(S.P) + s2 * 2048, 16384, 1024, 2);
+                mma_bf16_ss(tb + TA_COL_O + 64 * mt, a, bd, ido, t > 0 || s2 > 0);
+              }
+            }
+            mma_commit(&S.bar_o[mt]);
+          }
+        }
+        ++qk;
+        // advance to the next query with keys (the same scan as above)
+        int kn = k + 1;
+        TaUnit un{};
+        if (kn < nu) {
+          un = ta_unit(P, nraw);
+          while (un.ntile == 0 && ++kn < nu) un = ta_unit(P, ta_unit_load(P, unit_q(kn)));
+        }
+        k = kn;
+        u = un;
+      }
+      if (!ok) atomicOr(&S.err, 1u);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------------------------- workers
+    const int quad = warp & 3, hh = warp >> 2;
+    const int key = 32 * quad + lane;
+    const uint32_t lane_base = tb + ((uint32_t)(32 * quad) << 16);
+    bool ok = true;
+    uint4 cv[7], sc16, rp[4];
+    auto load_row = [&](int b, int id) {
+#pragma unroll
+      for (int j = 0; j < 7; ++j) cv[j] = make_uint4(0, 0, 0, 0);
+      sc16 = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) rp[c] = make_uint4(0, 0, 0, 0);
+      const long long r = id >= 0 ? page_row(P.pm, b, P.n_max, id) : -1;
+      if (r >= 0) {
+        const uint8_t* crow = P.codes + (size_t)r * 224 + ghalf * 16;
+#pragma unroll
+        for (int j = 0; j < 7; ++j) cv[j] = __ldg(reinterpret_cast<const uint4*>(crow + j * 32));
+        sc16 = __ldg(reinterpret_cast<const uint4*>(P.scales + (size_t)r * 16));
+        const uint4* rrow = reinterpret_cast<const uint4*>(P.rope + (size_t)r * 64) + ghalf * 4;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) rp[c] = __ldg(rrow + c);
+      }
+    };
+    auto raw_id = [&](const TaUnit& uu, const TaTile& gg) -> int {
+      if (grow >= gg.rs) return -1;
+      const int li = gg.key0 + grow;
+      return P.hca ? li : (li < P.k ? P.idx[(size_t)uu.bq * P.k + li] : -1);
+    };
+    auto check_id = [&](const TaUnit& uu, int v) -> int { return (v >= 0 && v < uu.ncb) ? v : -1; };
+    // the first query with keys at or after unit kk (from its raw positions, if they are those of unit
+    // kk), writing the outputs of the ones without keys; bq = -1 if there is none
+    auto next_unit = [&](int kk, TaUnitRaw raw) -> TaUnit {
+      return ta_next_unit(P, kk, nu, raw, tid, TA_WORKERS);
+    };
+    auto unit_index = [&](const TaUnit& uu) { return uu.bq < 0 ? nu : (uu.bq - (int)blockIdx.x) / (int)gridDim.x; };
+    auto epilogue = [&](int bq, uint32_t par) { ok = ta_epilogue(S, P, bq, par, lane_base, hh, quad, lane, tid) && ok; };
+
+    TaUnit u = nu > 0 ? next_unit(0, ta_unit_load(P, unit_q(0))) : TaUnit{};
+    if (nu == 0) u.bq = -1;
+    int k = unit_index(u);
+    int bq_done = -1;                           // query awaiting its epilogue
+    TaUnitRaw nraw{};
+    nraw.bq = -1;
+    if (k + 1 < nu) nraw = ta_unit_load(P, unit_q(k + 1));
+    int id = -1;
+    if (k < nu) {
+      id = check_id(u, raw_id(u, ta_tile_u(u, 0)));
+      load_row(u.b, id);
+    }
+    uint32_t f = 0;
+    int t = 0;
+#pragma unroll 1
+    while (k < nu) {
+      // the tile after this one (this query's next, or the next query's first): its id is read now and
+      // its row after this tile's gather
+      int kn = k, tn = t + 1;
+      TaUnit un = u;
+      if (tn == u.ntile) {
+        un = next_unit(k + 1, nraw);
+        kn = unit_index(un);
+        tn = 0;
+      }
+      const bool more = kn < nu;
+      const int raw_next = more ? raw_id(un, ta_tile_u(un, tn)) : -1;
+      const TaTile g = ta_tile_u(u, t);
+
+      // ---- gather: the K tile is refilled block by block as the previous tile's O MMAs release it
+      const bool pure = g.rs == TA_KEYS;
+      if (f > 0 && !pure) {
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt) ok = ok && mbar_wait(&S.bar_o[mt], (f - 1) & 1);
+        tc_fence_after();
+      }
+      if (ghalf == 0) S.ids[grow] = id;
+      if (!pure) {
+        const int r_end = min(g.wa, g.rw);
+        const int n = (r_end > g.rs ? r_end - g.rs : 0) * 64;
+        for (int i = tid; i < n; i += TA_WORKERS) {
+          const int row = g.rs + (i >> 6), c = i & 63;
+          const long long wr = g.wrow_base + row;
+          cp16(&S.K[c >> 3][sw128(row, c & 7)], P.win + ((size_t)u.b * P.Wn + wr) * 512 + c * 8);
+        }
+        for (int i = tid; i < (TA_KEYS - g.zs) * 64; i += TA_WORKERS) {
+          const int row = g.zs + (i >> 6), c = i & 63;
+          *reinterpret_cast<uint4*>(&S.K[c >> 3][sw128(row, c & 7)]) = make_uint4(0, 0, 0, 0);
+        }
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+      }
+#pragma unroll
+      for (int j = 0; j < 7; ++j) {
+        if (f > 0 && pure && (j & 1) == 0) {
+          ok = ok && mbar_wait(&S.bar_o[j >> 1], (f - 1) & 1);
+          tc_fence_after();
+        }
+        if (grow < g.rs) {
+          const int part = 2 * j + ghalf;
+          const uint32_t word = (j >> 1) == 0 ? sc16.x : (j >> 1) == 1 ? sc16.y : (j >> 1) == 2 ? sc16.z : sc16.w;
+          const uint32_t sb = f_to_bf16_bits(e4m3_to_f32((word >> ((part & 3) * 8)) & 0xFFu) * P.g);
+          const uint32_t sc2 = sb | (sb << 16);
+          const uint32_t w4[4] = {cv[j].x, cv[j].y, cv[j].z, cv[j].w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<uint4*>(&S.K[j][sw128(grow, ghalf * 4 + q4)]) = e2m1x8_to_bf16_scaled(w4[q4], sc2);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.bar_k[j]);
+      }
+      if (f > 0 && pure) {
+        ok = ok && mbar_wait(&S.bar_o[3], (f - 1) & 1);
+        tc_fence_after();
+      }
+      if (grow < g.rs) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(&S.K[7][sw128(grow, ghalf * 4 + c)]) = rp[c];
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.bar_k[7]);
+      // the next tile's row, in flight during this tile's softmax and MMAs
+      if (more) {
+        id = check_id(un, raw_next);
+        load_row(un.b, id);
+      }
+      // what the softmax needs of this tile; then the cursor moves on (one query's geometry stays live)
+      const int rs_t = g.rs, rw_t = g.rw, t_cur = t;
+      const int bq_ends = t + 1 == u.ntile ? u.bq : -1;
+      k = kn;
+      t = tn;
+      u = un;
+      asm volatile("bar.sync 1, 256;" ::: "memory");   // workers only: ids visible to the softmax
+
+      // ---- the previous query's epilogue: its last O MMAs completed before this tile's gather
+      if (bq_done >= 0) {
+        epilogue(bq_done, (f - 1) & 1);
+        bq_done = -1;
+      }
+
+      // ---- softmax of this tile (as in the per-query kernel)
+      ok = ok && mbar_wait(&S.bar_s, f & 1);
+      tc_fence_after();
+      const bool valid = key < rs_t ? (S.ids[key] >= 0) : (key < rw_t);
+      float red[32];
+      {
+        uint32_t sv[32];
+        tmem_ld_x32(lane_base + TA_COL_S + hh * 32, sv);
+        tmem_wait_ld_x32(sv);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) red[j] = valid ? __uint_as_float(sv[j]) * P.scale_log2 : -INFINITY;
+      }
+      S.red_m[quad][hh * 32 + lane] = transpose_reduce32<true>(red, lane);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (tid < 64) {
+        const float mt = fmaxf(fmaxf(S.red_m[0][tid], S.red_m[1][tid]), fmaxf(S.red_m[2][tid], S.red_m[3][tid]));
+        const float mo = S.m[tid];
+        float mn = mo, fc = 1.f;
+        if (mt > mo + TA_RESCALE_SLACK || (mo == -INFINITY && mt > -INFINITY)) {
+          mn = mt;
+          fc = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+        }
+        S.m[tid] = mn;
+        S.fac[tid] = fc;
+        S.l[tid] *= fc;
+        if (fc != 1.f && t_cur > 0) S.rescale = 1;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (t_cur > 0 && S.rescale) {
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt) {
+          uint32_t ov[32];
+          tmem_ld_x32(lane_base + TA_COL_O + 64 * mt + hh * 32, ov);
+          tmem_wait_ld_x32(ov);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * S.fac[hh * 32 + j]);
+          tmem_st_x32(lane_base + TA_COL_O + 64 * mt + hh * 32, ov);
+        }
+        tmem_wait_st();
+      }
+      {
+        uint32_t sv[32];
+        tmem_ld_x32(lane_base + TA_COL_S + hh * 32, sv);
+        tmem_wait_ld_x32(sv);
+        uint32_t pk[16];
+        float mh[32];
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 v4 = *reinterpret_cast<const float4*>(&S.m[hh * 32 + j]);
+          mh[j] = v4.x; mh[j + 1] = v4.y; mh[j + 2] = v4.z; mh[j + 3] = v4.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float m0 = mh[j], m1 = mh[j + 1];
+          const float z0 = valid ? __uint_as_float(sv[j]) * P.scale_log2 : -INFINITY;
+          const float z1 = valid ? __uint_as_float(sv[j + 1]) * P.scale_log2 : -INFINITY;
+          const float p0f = m0 == -INFINITY ? 0.f : exp2f(z0 - m0);
+          const float p1f = m1 == -INFINITY ? 0.f : exp2f(z1 - m1);
+          red[j] = p0f;
+          red[j + 1] = p1f;
+          pk[j >> 1] = pack_bf16x2(p0f, p1f);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(&S.P[sw128(key, hh * 4 + c)]) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.bar_p);
+      S.red_l[quad][hh * 32 + lane] = transpose_reduce32<false>(red, lane);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (tid < 64) S.l[tid] += (S.red_l[0][tid] + S.red_l[1][tid]) + (S.red_l[2][tid] + S.red_l[3][tid]);
+      if (tid == 0) S.rescale = 0;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+
+      if (bq_ends >= 0) {
+        bq_done = bq_ends;
+        // positions of the query after the next one, read now and used when the next one ends
+        nraw.bq = -1;
+        if (k + 1 < nu) nraw = ta_unit_load(P, unit_q(k + 1));
+      }
+      ++f;
+    }
+    if (bq_done >= 0) epilogue(bq_done, (f - 1) & 1);
+    if (!ok && lane == 0) atomicOr(&S.err, 1u);
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 8) {
+    if (S.err && lane == 0) atomicOr(&g_csa_device_error, 1u);
+    tc_fence_after();
+    tmem_dealloc(tb, TA_TMEM_COLS);
+  }
+}
+
 // Early window (CSA_EARLY_START): split 0 of each query, placed first in the grid, attends over the
 // window tile before the step's index and top-k kernels have ended; possible when the window fills one
 // tile right after the k entries (k a multiple of the tile, at most one tile of window).
@@ -751,6 +1230,13 @@ void attn_tc_plan(const csa_attn_args* a, int hca, int* splits, int* tpc) {
   if (t > tiles) t = tiles;
   *tpc = (int)t;
   *splits = (int)((tiles + t - 1) / t);
+}
+
+// One CTA per query and more queries than one wave of CTAs, BF16 window: the persistent kernel.
+bool attn_tc_persistent(const csa_attn_args* a, int hca, int splits) {
+  const long long rows = (long long)a->B * a->Nq;
+  return splits == 1 && rows > 148 && rows <= 0x7fffffffLL && a->win_format == CSA_WIN_BF16 &&
+         !attn_tc_early(a, hca);
 }
 
 // Queries split over 2..8 CTAs can merge inside a thread-block cluster (CSA_CLUSTER_MERGE: no workspace,
@@ -799,7 +1285,7 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
     memset(&wmap, 0, sizeof(wmap));            // never read: no window rows
   }
   TaParams P{};
-  P.Nq = a->Nq; P.H = a->H; P.ratio = a->ratio; P.n_max = a->n_max; P.k = hca ? 0 : a->k;
+  P.Nq = a->Nq; P.H = a->H; P.ratio = a->ratio; P.n_max = a->n_max; P.k = hca ? 0 : a->k; P.rows = (int)rows;
   P.Wn = Wn; P.window = a->window; P.splits = splits; P.tpc = tpc; P.hca = hca; P.g = a->g_kv;
   P.early_rows = attn_tc_early(a, hca) ? (int)rows : 0;
   P.cluster = (attn_tc_cluster(splits) && (a->flags & CSA_CLUSTER_MERGE)) ? 1 : 0;
@@ -817,6 +1303,18 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
     P.wrope = (const uint16_t*)a->win_rope;
   }
   const int smem = (int)sizeof(TaSmem) + 1024;
+  if (attn_tc_persistent(a, hca, splits)) {
+    // more queries than SMs, one CTA each: one persistent CTA per SM walks its queries back to back
+    int sms = 148;
+    {
+      int dev = 0;
+      if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    static std::atomic<unsigned> attr_done_p{0};
+    set_smem_once((const void*)attn_tc_persist_kernel, smem, attr_done_p);
+    const unsigned grid = (unsigned)(rows < sms ? rows : sms);
+    return launch_pdl(attn_tc_persist_kernel, dim3(grid), dim3(TA_THREADS), (size_t)smem, st, qmap, wmap, P);
+  }
   static std::atomic<unsigned> attr_done{0};
   static std::atomic<unsigned> attr_done8{0};
   auto* kfn = fp8 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
