@@ -502,6 +502,9 @@ static csa_status launch_merge(const PT* po, const float* pl, int splits, int H,
                                float* lse, const int64_t* q_pos, float rope_theta, cudaStream_t st) {
   const long long units = rows * H;
   const unsigned grid = (unsigned)((units + MERGE_WARPS - 1) / MERGE_WARPS);
+  static std::atomic<unsigned> attr512{0}, attr128{0};
+  set_smem_once((const void*)attn_merge_kernel<PT, 512>, 0, attr512);
+  set_smem_once((const void*)attn_merge_kernel<PT, 128>, 0, attr128);
   if (D == 512)
     return launch_pdl(attn_merge_kernel<PT, 512>, dim3(grid), dim3(MERGE_WARPS * 32), 0, st, po, pl, splits, H, units,
                       out, lse, q_pos, rope_theta);
@@ -539,6 +542,9 @@ static csa_status launch_out_rope(uint16_t* out, int H, int D, long long rows, c
                                   cudaStream_t st) {
   const long long units = rows * H;
   const unsigned grid = (unsigned)((units + MERGE_WARPS - 1) / MERGE_WARPS);
+  static std::atomic<unsigned> attr512{0}, attr128{0};
+  set_smem_once((const void*)out_rope_kernel<512>, 0, attr512);
+  set_smem_once((const void*)out_rope_kernel<128>, 0, attr128);
   if (D == 512) return launch_pdl(out_rope_kernel<512>, dim3(grid), dim3(MERGE_WARPS * 32), 0, st, out, H, units, q_pos, theta);
   return launch_pdl(out_rope_kernel<128>, dim3(grid), dim3(MERGE_WARPS * 32), 0, st, out, H, units, q_pos, theta);
 }

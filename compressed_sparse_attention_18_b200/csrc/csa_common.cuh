@@ -129,12 +129,17 @@ inline csa_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 
 // Raise a kernel's dynamic shared-memory limit once per device (the attribute is per device); later
 // calls, including those made while a stream is being captured into a CUDA graph, skip the runtime call.
+// Every kernel also asks for the largest shared-memory carveout: an SM runs CTAs of one carveout at a
+// time, so a kernel that needs little shared memory would otherwise hold SMs in a small-carveout setting
+// and keep the CTAs of the next kernel (launched early, programmatic dependent launch) off them until
+// its own CTAs have left.
 inline void set_smem_once(const void* func, int bytes, std::atomic<unsigned>& done) {
   int dev = 0;
   cudaGetDevice(&dev);
   const unsigned bit = 1u << (dev & 31);
   if (done.load(std::memory_order_acquire) & bit) return;
-  cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (bytes > 0) cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   done.fetch_or(bit, std::memory_order_acq_rel);
 }
 
