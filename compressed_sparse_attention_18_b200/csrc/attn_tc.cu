@@ -503,18 +503,17 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       const TaTile gt = g;
       // next tile's row (its id arrived during this tile's gather), in flight during this tile's softmax
       // and MMAs; the id of the tile after it is requested now
-      if (t + 1 < ntile) {
-        if (has_win && t == 0) {
-          // the window tile is gathered: from here on the ids and entries of the previous kernels
-          pdl_wait();
-          id_next = raw_id(ta_tile(tile_key(1), n_sel, n_list, wlo, p0, W8));
-        }
+      auto advance = [&]() {
         g = ta_tile(tile_key(t + 1), n_sel, n_list, wlo, p0, W8);
         id = check_id(id_next);
         load_row(id);
         if (is_win8(g)) load_win8(g);
         id_next = t + 2 < ntile ? raw_id(ta_tile(tile_key(t + 2), n_sel, n_list, wlo, p0, W8)) : -1;
-      }
+      };
+      // the window tile (split 0 under the early start) runs its softmax too before the wait; its
+      // entry tile's ids and rows are read after it
+      const bool win_first = has_win && t == 0;
+      if (t + 1 < ntile && !win_first) advance();
       asm volatile("bar.sync 1, 256;" ::: "memory");   // workers only: ids visible to the softmax
 
       // ---- softmax of this tile: warp w reads lanes 32*(w%4).. (its keys) and head half w/4
@@ -596,6 +595,12 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       if (tid < 64) S.l[tid] += (S.red_l[0][tid] + S.red_l[1][tid]) + (S.red_l[2][tid] + S.red_l[3][tid]);
       if (tid == 0) S.rescale = 0;
       asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (win_first && t + 1 < ntile) {
+        // from here on the ids and entries of the previous kernels
+        pdl_wait();
+        id_next = raw_id(ta_tile(tile_key(1), n_sel, n_list, wlo, p0, W8));
+        advance();
+      }
     }
 
     // ---- epilogue, M-tile by M-tile as the last O MMAs complete: lane = dim, columns = heads

@@ -159,6 +159,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       const long long rows_total = (long long)gridDim.y * P.n_max;
+      // every key is read once per call: its lines go first when L2 needs room, so the stream does not
+      // push out what the step reuses (the kernels' code, scores, ids, partials)
+      const uint64_t stream_policy = l2_policy_evict_first();
       int issued = 0;
       bool waited = !P.early;
       for (int i = 0; i < ntile && ok; ++i) {
@@ -188,8 +191,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) index_score_tc_kernel(const __g
 #pragma unroll
         for (int u = 0; u < 2; ++u)
           if (sc_bytes[u] > 0) {
-            tma_load_2d(S.codes[s] + u * (TC_SUB * 64), &kmap, 0, (int)row[u], &S.full[s]);
-            bulk_load(S.sc[s] + u * (TC_SUB * 4), P.k_scales + row[u] * 4, sc_bytes[u], &S.full[s]);
+            tma_load_2d_hint(S.codes[s] + u * (TC_SUB * 64), &kmap, 0, (int)row[u], &S.full[s], stream_policy);
+            bulk_load_hint(S.sc[s] + u * (TC_SUB * 4), P.k_scales + row[u] * 4, sc_bytes[u], &S.full[s],
+                           stream_policy);
           }
         ++issued;
       }
