@@ -24,7 +24,7 @@ ENTRY_POINTS = ("csa_status_string", "csa_version", "csa_last_cuda_error", "csa_
                 "csa_index_topk_workspace_size", "csa_index_topk", "csa_index_scores", "csa_topk_workspace_size",
                 "csa_topk", "csa_attn_workspace_size", "csa_sparse_attn", "hca_dense_attn",
                 "csa_index_topk_noalloc", "csa_device_status", "csa_check_error_path",
-                "csa_pack_fp8_window")
+                "csa_pack_fp8_window", "csa_attn_kernel_count")
 # (PagedCache: a paged pool + block table, accepted wherever a PackedCache is)
 
 _u32, _i32, _f32, _vp = ctypes.c_uint32, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p
@@ -102,6 +102,8 @@ _lib.csa_topk.restype = ctypes.c_int
 _lib.csa_topk.argtypes = [ctypes.POINTER(IndexArgs), _vp, ctypes.c_int64, _vp, ctypes.c_size_t, _vp]
 _lib.csa_attn_workspace_size.restype = ctypes.c_size_t
 _lib.csa_attn_workspace_size.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_int]
+_lib.csa_attn_kernel_count.restype = ctypes.c_int
+_lib.csa_attn_kernel_count.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_int]
 for _name in ("csa_sparse_attn", "hca_dense_attn"):
     getattr(_lib, _name).restype = ctypes.c_int
     getattr(_lib, _name).argtypes = [ctypes.POINTER(AttnArgs), _vp, ctypes.c_size_t, _vp]
@@ -149,12 +151,12 @@ def _stream(stream):
     return s.cuda_stream
 
 
-def _ws(nbytes: int, device, ws=None):
+def _ws(nbytes: int, device, ws=None, zero=False):
     if nbytes == 0:
         return None
     if ws is not None and ws.numel() * ws.element_size() >= nbytes:
         return ws
-    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return (torch.zeros if zero else torch.empty)(nbytes, dtype=torch.uint8, device=device)
 
 
 # ------------------------------------------------------------------------------------------- API
@@ -406,6 +408,16 @@ def hca_attn(q, q_pos, cache: PackedCache, n_c, win_kv=None, win_pos0=None, *, r
 
 def attn_workspace_size(q, q_pos, cache, n_c, idx, win_kv, win_pos0, *, ratio, window, hca=False, early_start=False,
                         cluster=False):
+    """Bytes of workspace one call with these arguments needs (csa_attn_workspace_size)."""
     a = _attn_args(q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, 0.0, None, None)
     a.flags = (CSA_EARLY_START if early_start else 0) | (CSA_CLUSTER_MERGE if cluster else 0)
     return _lib.csa_attn_workspace_size(ctypes.byref(a), 1 if hca else 0)
+
+
+def attn_kernel_count(q, q_pos, cache, n_c, idx, win_kv, win_pos0, *, ratio, window, hca=False, early_start=False,
+                      cluster=False, out_rope_theta=0.0):
+    """Kernels one attention call with these arguments launches (csa_attn_kernel_count)."""
+    a = _attn_args(q, q_pos, cache, n_c, idx, win_kv, win_pos0, ratio, window, 0.0, None, None)
+    a.flags = (CSA_EARLY_START if early_start else 0) | (CSA_CLUSTER_MERGE if cluster else 0)
+    a.out_rope_theta = out_rope_theta
+    return _lib.csa_attn_kernel_count(ctypes.byref(a), 1 if hca else 0)

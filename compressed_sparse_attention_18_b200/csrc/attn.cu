@@ -600,7 +600,9 @@ static AttnPlan plan_attn(const csa_attn_args* a, int hca) {
   return p;
 }
 
-static csa_status validate_attn(const csa_attn_args* a, int hca) {
+// ptrs = false (workspace-size and kernel-count queries): shapes, flags and the page map only; the buffers
+// may not exist yet
+static csa_status validate_attn(const csa_attn_args* a, int hca, bool ptrs = true) {
   CSA_REQUIRE(a != nullptr && a->struct_size == sizeof(csa_attn_args));
   CSA_REQUIRE(a->B >= 0 && a->Nq >= 0 && a->H >= 1 && a->ratio >= 1 && a->n_max >= 0 && a->Wn >= 0 && a->window >= 1);
   CSA_SUPPORTED((a->d == 512 && a->d_rope == 64) || (a->d == 128 && a->d_rope == 32));
@@ -613,7 +615,7 @@ static csa_status validate_attn(const csa_attn_args* a, int hca) {
     const csa_status pv = check_page_map(a->kv_pages, a->n_max);
     if (pv != CSA_OK) return pv;
   }
-  if ((long long)a->B * a->Nq == 0) return CSA_OK;
+  if ((long long)a->B * a->Nq == 0 || !ptrs) return CSA_OK;
   CSA_REQUIRE(a->q && a->q_pos && a->n_c && a->out);
   CSA_REQUIRE(a->n_max == 0 || (a->kv_codes && a->kv_scales && a->kv_rope));
   if (!hca) CSA_REQUIRE(a->idx != nullptr);
@@ -648,11 +650,12 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
   CSA_REQUIRE(p.total == 0 || ws != nullptr);
   cudaStream_t st = (cudaStream_t)stream;
   if (p.tc) {
-    const bool merged = p.splits == 1 || (attn_tc_cluster(p.splits) && (a->flags & CSA_CLUSTER_MERGE));
-    uint16_t* po = !merged ? (uint16_t*)((uint8_t*)ws + p.off_o) : nullptr;
-    float* pl = !merged ? (float*)((uint8_t*)ws + p.off_lse) : nullptr;
+    const bool on_chip = p.splits == 1 || (attn_tc_cluster(p.splits) && (a->flags & CSA_CLUSTER_MERGE));
+    uint16_t* po = !on_chip ? (uint16_t*)((uint8_t*)ws + p.off_o) : nullptr;
+    float* pl = !on_chip ? (float*)((uint8_t*)ws + p.off_lse) : nullptr;
     csa_status s = launch_attn_tc(a, hca, p.splits, p.tpc, po, pl, st);
     if (s != CSA_OK) return s;
+    const bool merged = on_chip;
     if (merged)
       return a->out_rope_theta != 0.0f
                  ? launch_out_rope((uint16_t*)a->out, a->H, a->d, rows, a->q_pos, a->out_rope_theta, st)
@@ -692,8 +695,20 @@ static csa_status run_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, vo
 using namespace csa;
 
 extern "C" size_t csa_attn_workspace_size(const csa_attn_args* a, int hca) {
-  if (validate_attn(a, hca) != CSA_OK) return 0;
+  if (validate_attn(a, hca, false) != CSA_OK) return 0;
   return plan_attn(a, hca).total;
+}
+
+extern "C" int csa_attn_kernel_count(const csa_attn_args* a, int hca) {
+  if (validate_attn(a, hca, false) != CSA_OK) return -1;
+  if ((long long)a->B * a->Nq == 0) return 0;
+  const AttnPlan p = plan_attn(a, hca);
+  const bool rope = a->out_rope_theta != 0.0f;
+  if (p.tc) {
+    const bool on_chip = p.splits == 1 || (attn_tc_cluster(p.splits) && (a->flags & CSA_CLUSTER_MERGE));
+    return on_chip ? (rope ? 2 : 1) : 2;
+  }
+  return p.splits > 1 ? 2 : (rope ? 2 : 1);
 }
 
 extern "C" csa_status csa_sparse_attn(const csa_attn_args* a, void* ws, size_t ws_bytes, void* stream) {

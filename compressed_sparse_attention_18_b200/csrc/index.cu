@@ -1024,7 +1024,8 @@ static IndexPlan plan_index(const csa_index_args* a) {
   return p;
 }
 
-static csa_status validate_index(const csa_index_args* a, bool need_select) {
+// ptrs = false (workspace-size queries): shapes, flags and the page map only; the buffers may not exist yet
+static csa_status validate_index(const csa_index_args* a, bool need_select, bool ptrs = true) {
   CSA_REQUIRE(a != nullptr && a->struct_size == sizeof(csa_index_args));
   CSA_REQUIRE(a->B >= 0 && a->Nq >= 0 && a->H_I >= 1 && a->ratio >= 1 && a->k >= 1 && a->n_max >= 0);
   CSA_SUPPORTED(a->d_I == 64 || a->d_I == 128);
@@ -1040,7 +1041,7 @@ static csa_status validate_index(const csa_index_args* a, bool need_select) {
     if (segs > 1) CSA_SUPPORTED((long long)segs * a->k <= TOPK_CHUNK_IDS);
   }
   if (a->pool_blocks > 0) {
-    CSA_REQUIRE(a->pool_block_size >= 1 && a->pool_out != nullptr);
+    CSA_REQUIRE(a->pool_block_size >= 1 && (a->pool_out != nullptr || !ptrs));
     const int nblk = (a->n_max + a->pool_block_size - 1) / a->pool_block_size;
     CSA_SUPPORTED(nblk <= TOPK_CHUNK && a->pool_blocks <= 4096);
   }
@@ -1048,7 +1049,7 @@ static csa_status validate_index(const csa_index_args* a, bool need_select) {
     const csa_status pv = check_page_map(a->k_pages, a->n_max);
     if (pv != CSA_OK) return pv;
   }
-  if ((long long)a->B * a->Nq == 0) return CSA_OK;
+  if ((long long)a->B * a->Nq == 0 || !ptrs) return CSA_OK;
   CSA_REQUIRE(a->n_c && a->q_pos);
   if (need_select) CSA_REQUIRE(a->idx_out != nullptr);
   else CSA_REQUIRE(a->q_I && a->w && a->k_codes && a->k_scales);
@@ -1301,7 +1302,7 @@ extern "C" csa_status csa_index_scores(const csa_index_args* a, float* scores, i
 }
 
 extern "C" size_t csa_topk_workspace_size(const csa_index_args* a) {
-  if (validate_index(a, true) != CSA_OK) return 0;
+  if (validate_index(a, true, false) != CSA_OK) return 0;
   return plan_index(a).sel_total;
 }
 
@@ -1318,7 +1319,7 @@ extern "C" csa_status csa_topk(const csa_index_args* a, const float* scores, int
 }
 
 extern "C" size_t csa_index_topk_workspace_size(const csa_index_args* a) {
-  if (validate_index(a, true) != CSA_OK || validate_index(a, false) != CSA_OK) return 0;
+  if (validate_index(a, true, false) != CSA_OK) return 0;
   return plan_index(a).total;
 }
 

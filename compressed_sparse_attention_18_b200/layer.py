@@ -16,8 +16,8 @@ from dataclasses import dataclass
 
 import torch
 
-from . import PackedCache, attn_workspace_size, compress, index_scores, index_topk, index_topk_workspace_size, \
-    pack_fp4, sparse_attn, topk, topk_workspace_size
+from . import PackedCache, attn_kernel_count, attn_workspace_size, compress, index_scores, index_topk, \
+    index_topk_workspace_size, pack_fp4, sparse_attn, topk, topk_workspace_size
 
 
 @dataclass
@@ -80,6 +80,9 @@ class CSADecodeLayer:
                    for e in (True, False))
         self.ws_index = torch.empty(max(ws_i, 1), dtype=torch.uint8, device=dev)
         self.ws_attn = torch.empty(max(ws_a, 1), dtype=torch.uint8, device=dev)
+        self._attn_kernels = {e: attn_kernel_count(q, self.q_pos, self.kv, self.n_c, self.idx, self.win,
+                                                   self.win_pos0, ratio=s.r, window=s.W, early_start=e,
+                                                   cluster=cluster_merge) for e in (True, False)}
 
     def load_history(self, kv_src, kI_src, n_c: int):
         """Pack a prefix of n_c - 1 compressed entries (and index keys) into the caches: rows [B, n, d]."""
@@ -97,13 +100,11 @@ class CSADecodeLayer:
         self.q_pos.fill_(t)
         self.win_pos0.fill_(t - s.W + 1)
 
-    # kernels of one step with the default options: pool + FP4 append, index scores, top-k, attention,
-    # split merge (the on-chip top-k removes the top-k launch, the cluster merge the merge launch)
-    KERNELS_PER_STEP = 5
-
     @property
     def kernels_per_step(self):
-        return (3 if self.fused else 4) + (0 if self.cluster else 1)
+        """pool + FP4 append, index scores and top-k (one launch with the on-chip top-k), and the attention
+        call's kernels (csa_attn_kernel_count: the attention, and the split merge when a query is split)."""
+        return (2 if self.fused else 3) + self._attn_kernels[self.early]
 
     def step(self, C, Z, b_pos, W_IK, q, q_I, w, stream=None, marks=None):
         """One decode step.  C, Z [B, r, d] bf16 (projections of the group's r tokens), q [B,1,H,d],

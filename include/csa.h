@@ -12,7 +12,9 @@
  * Conventions for every entry point:
  *   - Every pointer is caller-owned DEVICE memory (unless stated otherwise); the library allocates
  *     nothing.  Scratch comes from a caller workspace whose size the matching *_workspace_size() call
- *     returns for the same arguments (0 means none is needed; ws may then be NULL).
+ *     returns for the same arguments (0 means none is needed; ws may then be NULL).  The size (and
+ *     kernel-count) queries read the shapes, flags, page maps and the alignment of the input buffers
+ *     given; output buffers may still be NULL then.
  *   - bf16 = IEEE bfloat16 stored as uint16; tensors are dense row-major with the shapes given.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy default
  *     stream).  Argument errors are detected on the host before any launch and returned as
@@ -318,6 +320,8 @@ csa_status csa_index_topk_noalloc(const csa_index_args* args, void* stream);
  *         lse[B][Nq][H] fp32 (may be NULL).
  * Limits: d in {128, 512} with d_rope == 64 (d = 512) or 32 (d = 128); H <= 64.
  * Workspace: csa_attn_workspace_size() (split-K partials); `hca` selects the HCA key set.
+ * csa_attn_kernel_count: how many kernels one call with these arguments launches (-1 if the arguments
+ *   are invalid, 0 for an empty batch); no GPU work.
  * ------------------------------------------------------------------------------------------------ */
 typedef struct csa_attn_args {
   uint32_t struct_size;
@@ -357,6 +361,7 @@ typedef struct csa_attn_args {
 #define CSA_WIN_FP8 1u
 
 size_t csa_attn_workspace_size(const csa_attn_args* args, int hca);
+int csa_attn_kernel_count(const csa_attn_args* args, int hca);
 csa_status csa_sparse_attn(const csa_attn_args* args, void* ws, size_t ws_bytes, void* stream);
 csa_status hca_dense_attn(const csa_attn_args* args, void* ws, size_t ws_bytes, void* stream);
 

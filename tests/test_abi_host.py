@@ -92,12 +92,10 @@ int main(void) {
   csa_index_args i; memset(&i, 0, sizeof i);
   i.struct_size = sizeof i; i.B = 2; i.Nq = 1; i.H_I = 8; i.d_I = 128; i.ratio = 4; i.k = 16; i.n_max = 4096;
   i.g_q = 1.0f; i.g_k = 1.0f;
-  size_t ws0 = csa_index_topk_workspace_size(&i);        /* no tensors: invalid, 0 */
-  static char dummy[256];                                /* never dereferenced by a size query */
-  i.q_I = dummy; i.w = (const float*)dummy; i.k_codes = (const uint8_t*)dummy; i.k_scales = (const uint8_t*)dummy;
-  i.n_c = (const int32_t*)dummy; i.q_pos = (const int64_t*)dummy; i.idx_out = (int32_t*)dummy;
-  size_t ws = ws0 == 0 ? csa_index_topk_workspace_size(&i) : 0;
-  printf("%d %d %d %zu %s %d\n", s1, s2, s3, ws, csa_status_string(s3), csa_version());
+  size_t ws = csa_index_topk_workspace_size(&i);         /* shapes only: no buffer needed */
+  i.k = 0;
+  size_t ws_bad = csa_index_topk_workspace_size(&i);     /* k = 0: invalid, 0 */
+  printf("%d %d %d %zu %s %d %zu\n", s1, s2, s3, ws, csa_status_string(s3), csa_version(), ws_bad);
   return 0;
 }
 """)
@@ -107,7 +105,7 @@ int main(void) {
                     "-l:" + os.path.basename(csa.LIB_PATH), "-Wl,-rpath," + libdir], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     assert out[:3] == ["2", "1", "2"] and out[4] == "CSA_ERR_UNSUPPORTED"
-    assert int(out[3]) >= 2 * 4096 * 4 and int(out[5]) == csa.version()
+    assert int(out[3]) >= 2 * 4096 * 4 and int(out[5]) == csa.version() and out[6] == "0"
 
 
 def test_invalid_arguments_are_rejected_on_the_host(csa):
@@ -178,6 +176,35 @@ def test_workspace_sizes_scale_with_the_problem(csa):
             setattr(a, f, 256)
         return lib.csa_attn_workspace_size(ctypes.byref(a), 0)
     # (without a GPU driver the tensor-core path is not eligible: these are the d = 512 mma.sync plan's sizes;
-    # on a B200 a decode query split over 2..8 CTAs merges inside its cluster and needs no workspace)
+    # on a B200 a decode query split over 2..4 CTAs keeps per-query counters and bf16 partials there)
     assert attn_ws(32, 512) > 0                                     # decode: split-K partials
     assert attn_ws(1024, 512) == 0                                  # enough queries: no split
+    # a size query needs no output buffer (the workspace is sized before the outputs exist)
+    a = csa.AttnArgs(ctypes.sizeof(csa.AttnArgs), 32, 1, 64, 512, 64, 4, 32768, 512, 128, 128, 1.0, 0.0)
+    for f in ("q", "q_pos", "kv_codes", "kv_scales", "kv_rope", "n_c", "idx", "win_kv", "win_pos0"):
+        setattr(a, f, 256)
+    assert lib.csa_attn_workspace_size(ctypes.byref(a), 0) == attn_ws(32, 512)
+    assert lib.csa_attn_kernel_count(ctypes.byref(a), 0) == 2
+    ia = csa.IndexArgs(ctypes.sizeof(csa.IndexArgs), 32, 1, 8, 128, 4, 512, 32768, 1.0, 1.0)
+    for f in ("q_I", "w", "k_codes", "k_scales", "n_c", "q_pos"):
+        setattr(ia, f, 256)
+    assert lib.csa_index_topk_workspace_size(ctypes.byref(ia)) > 0          # idx_out still NULL
+
+
+def test_attn_kernel_count_host_checks(csa):
+    """csa_attn_kernel_count: -1 for arguments the call would reject, 0 for an empty batch, else the
+    launches of the plan (the mma.sync plan here: attention + merge when a query is split)."""
+    lib = csa._lib
+
+    def args(B, k, Wn=128):
+        a = csa.AttnArgs(ctypes.sizeof(csa.AttnArgs), B, 1, 64, 512, 64, 4, 32768, k, Wn, 128, 1.0, 0.0)
+        for f in ("q", "q_pos", "kv_codes", "kv_scales", "kv_rope", "n_c", "idx", "win_kv", "win_pos0", "out"):
+            setattr(a, f, 256)
+        return a
+    assert lib.csa_attn_kernel_count(ctypes.byref(args(32, 0)), 0) == -1          # k = 0 for the CSA key set
+    bad = args(32, 512)
+    bad.struct_size = 4
+    assert lib.csa_attn_kernel_count(ctypes.byref(bad), 0) == -1
+    assert lib.csa_attn_kernel_count(ctypes.byref(args(0, 512)), 0) == 0
+    assert lib.csa_attn_kernel_count(ctypes.byref(args(32, 512)), 0) == 2          # split queries: + merge
+    assert lib.csa_attn_kernel_count(ctypes.byref(args(1024, 512)), 0) == 1        # one CTA per query

@@ -494,6 +494,49 @@ def test_attn_persistent_hca_variable_tiles(cuda_lib, Wn):
         assert bool(torch.all(out.cpu()[empty] == 0)) and bool(torch.all(torch.isneginf(lse.cpu()[empty])))
 
 
+@pytest.mark.parametrize("early_start", [False, True], ids=["plain", "early"])
+def test_attn_workspace_reused_across_calls_and_plans(cuda_lib, early_start):
+    """One caller workspace, sized by the size query before any output exists, serves repeated calls and
+    calls of the other launch plan (early start or not) for the same queries: identical results every
+    time, and against the oracle; the kernel-count query matches the plan (attention + split merge)."""
+    csa = cuda_lib
+    B, n = 6, 2048
+    q_pos = [4 * n - 1 - 37 * b for b in range(B)]
+    G = gen(71)
+    kv = normal((B, n, 512), 1.0, G)
+    q = normal((B, 1, 64, 512), 1.0, G).to(DEV)
+    win = normal((B, 128, 512), 1.0, G).to(DEV)
+    wp0 = torch.tensor([t - 127 for t in q_pos], dtype=torch.int64, device=DEV)
+    qp = torch.tensor(q_pos, dtype=torch.int64, device=DEV).view(B, 1)
+    n_c = torch.full((B,), n, dtype=torch.int32, device=DEV)
+    # k = 384: 3 entry tiles (+ the window tile): 3 or 4 CTAs per query in both plans
+    idx = torch.stack([torch.randperm(n, generator=G)[:384] for _ in range(B)]).view(B, 1, 384).to(torch.int32).to(DEV)
+    cache = csa.PackedCache(B, n, 512, 64, DEV, 1.0)
+    csa.pack_fp4(kv.to(DEV), cache)
+    nbytes = max(csa.attn_workspace_size(q, qp, cache, n_c, idx, win, wp0, ratio=4, window=128, early_start=e)
+                 for e in (False, True))
+    assert nbytes > 0
+    ws = torch.full((nbytes,), 0xA5, dtype=torch.uint8, device=DEV)
+    assert csa.attn_kernel_count(q, qp, cache, n_c, idx, win, wp0, ratio=4, window=128,
+                                 early_start=early_start) == 2
+    outs = []
+    for rep in range(3):
+        # another plan (the other early-start setting) in between, on the same workspace
+        csa.sparse_attn(q, qp, cache, n_c, idx, win, wp0, ratio=4, ws=ws, early_start=not early_start)
+        out, lse = csa.sparse_attn(q, qp, cache, n_c, idx, win, wp0, ratio=4, ws=ws, early_start=early_start)
+        torch.cuda.synchronize()
+        outs.append((out.clone(), lse.clone()))
+    assert all(torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1]) for o, l in outs[1:])
+    scale = 512 ** -0.5
+    for b in range(B):
+        codes, scales, rope = O.pack_fp4(f64(kv[b]), 64, 1.0)
+        rows = O.entry_kv(codes, scales, rope, 448, 1.0)
+        o_ref, l_ref = O.attention(f64(q[b]), [q_pos[b]], rows, idx[b].cpu().numpy(), n, f64(win[b]), q_pos[b] - 127,
+                                   128, scale)
+        assert_close(f64(outs[0][0][b]), o_ref, OUT_ATOL, OUT_RTOL, f"out b={b}")
+        assert_close(outs[0][1][b].cpu().numpy(), l_ref, LSE_ATOL, LSE_RTOL, f"lse b={b}")
+
+
 def test_attn_hca(cuda_lib):
     _attn_case(cuda_lib, B=2, Nq=1, H=64, d=512, d_r=64, n_max=300, n_c=[300, 300],
                q_pos=[128 * 300 - 1, 128 * 150 + 5], hca=True, ratio=128, seed=7)
@@ -561,8 +604,9 @@ def test_attn_fp8_window_partial_multi_query_and_hca(cuda_lib):
 @pytest.mark.parametrize("k", [128, 384, 640, 896, 1024])
 def test_attn_cluster_merge_sizes(cuda_lib, k, cluster):
     """Two decode queries whose key lists span 2, 4, 6, 8 and 9 tiles of 128 keys (k entries + the
-    128-row window): 2..8 CTAs per query merge inside their thread-block cluster, 9 go through the
-    workspace partials and the merge kernel; without CSA_CLUSTER_MERGE every split count takes the merge kernel."""
+    128-row window): with CSA_CLUSTER_MERGE 2..8 CTAs per query merge inside their thread-block cluster and
+    9 go through the workspace partials and the merge kernel; without it 2..4 CTAs per query are merged
+    by the query's last CTA and more by the merge kernel."""
     n = 4096
     _attn_case(cuda_lib, B=2, Nq=1, H=64, d=512, d_r=64, n_max=n, n_c=[n, n - 100], q_pos=[4 * n - 1, 4 * n - 401],
                k=k, seed=60 + k // 128, cluster=cluster)
