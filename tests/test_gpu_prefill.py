@@ -177,3 +177,40 @@ def test_index_multiquery_ragged_everywhere(cuda_lib, H_I):
         for q in range(Nq):
             assert np.all(np.isnan(got[b, q, n_vis[q]:])), f"b={b} q={q}: columns past the visible range written"
             check_topk_row(idx[b, q].cpu().numpy(), s_ref[q], ids[q], k, f"b={b} q={q}")
+
+
+# ------------------------------------------------------------------- top-k of prefill-length rows
+
+@pytest.mark.parametrize("n_equal", [8192, 1500, 40])
+def test_topk_prefill_rows_with_ties(cuda_lib, n_equal):
+    """Top-512 of rows of 8192 scores (the chunked prefill's rows, one CTA of 256 threads per row):
+    n_equal scores share the value at the selection boundary, so the tie break (id ascending) decides:
+    the whole row, 1500 or 40 of them.  Sets exactly as the oracle's (score desc, id asc); rows that see
+    fewer than k entries pad with -1."""
+    csa = cuda_lib
+    rows, n, k = 6, 8192, 512
+    rng = np.random.default_rng(80 + n_equal)
+    sc = rng.standard_normal((rows, n)).astype(np.float32)
+    for r in range(rows):
+        perm = rng.permutation(n)
+        top = perm[: k - 100]                       # clearly above the tie value
+        tie = perm[k - 100: k - 100 + n_equal] if n_equal < n else perm
+        sc[r, top] = 10.0 + rng.random(len(top)).astype(np.float32)
+        sc[r, tie] = 3.0
+        if n_equal == n:
+            sc[r, :] = 3.0
+    q_pos = np.full((1, rows), 4 * n - 1, np.int64)
+    q_pos[0, -1] = 4 * 300 - 1                     # sees 300 entries only: k_eff = 300
+    kc = csa.PackedCache(1, n, 128, 0, DEV)
+    scores = torch.as_tensor(sc, device=DEV)
+    n_c = torch.tensor([n], dtype=torch.int32, device=DEV)
+    idx, _, _ = csa.topk(scores, kc, n_c, torch.as_tensor(q_pos, device=DEV), B=1, Nq=rows, ratio=4, k=k)
+    torch.cuda.synchronize()
+    got = idx[0].cpu().numpy()
+    for r in range(rows):
+        nv = min(n, (int(q_pos[0, r]) + 1) // 4)
+        s = sc[r].astype(np.float64).copy()
+        s[nv:] = -np.inf
+        ref, _ = O.topk(s[None], np.arange(n)[None], k)
+        assert set(got[r][got[r] >= 0].tolist()) == set(ref[0][ref[0] >= 0].tolist()), f"row {r}"
+        assert np.all(got[r][min(k, nv):] == -1) and np.all(got[r][: min(k, nv)] >= 0), f"row {r} padding"
