@@ -90,6 +90,14 @@ __device__ __forceinline__ void cp16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src));
 }
 
+// 2^x by the hardware approximation (one special-function instruction, relative error about 2^-22;
+// results below 2^-126 flush to zero): P is rounded to bf16 right after, and l sums these same values.
+__device__ __forceinline__ float ta_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
@@ -575,8 +583,8 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
           const float m0 = mh[j], m1 = mh[j + 1];
           const float z0 = valid ? __uint_as_float(sv[j]) * P.scale_log2 : -INFINITY;
           const float z1 = valid ? __uint_as_float(sv[j + 1]) * P.scale_log2 : -INFINITY;
-          const float p0f = m0 == -INFINITY ? 0.f : exp2f(z0 - m0);
-          const float p1f = m1 == -INFINITY ? 0.f : exp2f(z1 - m1);
+          const float p0f = m0 == -INFINITY ? 0.f : ta_exp2(z0 - m0);
+          const float p1f = m1 == -INFINITY ? 0.f : ta_exp2(z1 - m1);
           red[j] = p0f;
           red[j + 1] = p1f;
           pk[j >> 1] = pack_bf16x2(p0f, p1f);
@@ -1171,8 +1179,8 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
           const float m0 = mh[j], m1 = mh[j + 1];
           const float z0 = valid ? __uint_as_float(sv[j]) * P.scale_log2 : -INFINITY;
           const float z1 = valid ? __uint_as_float(sv[j + 1]) * P.scale_log2 : -INFINITY;
-          const float p0f = m0 == -INFINITY ? 0.f : exp2f(z0 - m0);
-          const float p1f = m1 == -INFINITY ? 0.f : exp2f(z1 - m1);
+          const float p0f = m0 == -INFINITY ? 0.f : ta_exp2(z0 - m0);
+          const float p1f = m1 == -INFINITY ? 0.f : ta_exp2(z1 - m1);
           red[j] = p0f;
           red[j + 1] = p1f;
           pk[j >> 1] = pack_bf16x2(p0f, p1f);
