@@ -896,6 +896,9 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       bool ok = true;
       const uint32_t ids = idesc_bf16(128, 64, 0, 0);
       const uint32_t ido = idesc_bf16(128, 64, 1, 1);
+      // descriptor bases (an offset below 256 KB adds to the 14-bit address field without a carry)
+      const uint64_t kdesc = smem_desc(smem_addr(S.K[0]), 16, 1024, 2), qdesc = smem_desc(smem_addr(S.Q[0]), 16, 1024, 2);
+      const uint64_t vdesc = smem_desc(smem_addr(S.K[0]), 16384, 1024, 2), pdesc = smem_desc(smem_addr(S.P), 16384, 1024, 2);
       auto load_q = [&](int bq) {
 #pragma unroll 1
         for (int j = 0; j < 8; ++j) {
@@ -929,17 +932,21 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
                 tma_load_3d(&S.K[j][(g.wa + i * TA_WBOX) * 128], &wmap, j * 64,
                             (int)(g.wrow_base + g.wa + i * TA_WBOX), u.b, &S.bar_w[j]);
           }
-#pragma unroll 1
-          for (int j = 0; j < 8 && ok; ++j) {
-            ok = (t > 0 || mbar_wait(&S.bar_q[j], qk & 1)) && mbar_wait(&S.bar_w[j], f & 1) &&
-                 mbar_wait(&S.bar_k[j], f & 1);
-            if (!ok) break;
-            tc_fence_after();
+          // S^T = K Q^T, dim block by dim block as the blocks land.  At N = 64 the tensor pipe keeps up with
+          // one MMA per ~75 cycles only when they are issued back to back: the loops are unrolled, the
+          // descriptors advance by adds, and a landed block costs a non-blocking test, not a wait.
 #pragma unroll
-            for (int s2 = 0; s2 < 4; ++s2) {
-              const uint64_t a = smem_desc(smem_addr(S.K[j]) + s2 * 32, 16, 1024, 2);
-              const uint64_t bd = smem_desc(smem_addr(S.Q[j]) + s2 * 32, 16, 1024, 2);
-              mma_bf16_ss(tb + TA_COL_S, a, bd, ids, (j | s2) != 0);
+          for (int j = 0; j < 8; ++j) {
+            if (ok && !((t > 0 || mbar_test(&S.bar_q[j], qk & 1)) && mbar_test(&S.bar_w[j], f & 1) &&
+                        mbar_test(&S.bar_k[j], f & 1)))
+              ok = (t > 0 || mbar_wait(&S.bar_q[j], qk & 1)) && mbar_wait(&S.bar_w[j], f & 1) &&
+                   mbar_wait(&S.bar_k[j], f & 1);
+            if (ok) {
+              tc_fence_after();
+#pragma unroll
+              for (int s2 = 0; s2 < 4; ++s2)
+                mma_bf16_ss(tb + TA_COL_S, kdesc + (uint64_t)((j * TA_KEYS * 128 + s2 * 32) >> 4),
+                            qdesc + (uint64_t)((j * 64 * 128 + s2 * 32) >> 4), ids, (j | s2) != 0);
             }
           }
           mma_commit(&S.bar_s);
@@ -957,15 +964,13 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
           // query's epilogue has read it: the workers arrive on bar_p only after that)
           ok = ok && mbar_wait(&S.bar_p, f & 1);
           if (ok) tc_fence_after();
-#pragma unroll 1
+#pragma unroll
           for (int mt = 0; mt < 4; ++mt) {
             if (ok) {
 #pragma unroll
-              for (int s2 = 0; s2 < 8; ++s2) {
-                const uint64_t a = smem_desc(smem_addr(S.K[2 * mt]) + s2 * 2048, 16384, 1024, 2);
-                const uint64_t bd = smem_desc(smem_addr(S.P) + s2 * 2048, 16384, 1024, 2);
-                mma_bf16_ss(tb + TA_COL_O + 64 * mt, a, bd, ido, t > 0 || s2 > 0);
-              }
+              for (int s2 = 0; s2 < 8; ++s2)
+                mma_bf16_ss(tb + TA_COL_O + 64 * mt, vdesc + (uint64_t)((2 * mt * TA_KEYS * 128 + s2 * 2048) >> 4),
+                            pdesc + (uint64_t)((s2 * 2048) >> 4), ido, t > 0 || s2 > 0);
             }
             mma_commit(&S.bar_o[mt]);
           }
