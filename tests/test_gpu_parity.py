@@ -537,6 +537,19 @@ def test_attn_workspace_reused_across_calls_and_plans(cuda_lib, early_start):
         assert_close(outs[0][1][b].cpu().numpy(), l_ref, LSE_ATOL, LSE_RTOL, f"lse b={b}")
 
 
+@pytest.mark.parametrize("hca", [False, True], ids=["sparse", "hca"])
+def test_attn_ctas_walking_many_tiles(cuda_lib, hca):
+    """Few queries with long key lists: each CTA walks 3-4 tiles of 128 keys (the back-to-back MMA issue
+    variant), splits merged by the merge kernel, ragged last tiles and a partial window."""
+    B, Nq, n = 5, 4, 2048
+    rng = np.random.default_rng(90 + hca)
+    q_pos = rng.integers(4 * 1500, 4 * n, size=(B, Nq))
+    q_pos[0, 0] = 4 * n - 1
+    kw = dict(hca=True, ratio=4) if hca else dict(k=1800)
+    _attn_case(cuda_lib, B=B, Nq=Nq, H=64, d=512, d_r=64, n_max=n, n_c=[n, n - 37, 1700, n, 1999],
+               q_pos=q_pos.ravel().tolist(), Wn=160, seed=91 + hca, **kw)
+
+
 def test_attn_hca(cuda_lib):
     _attn_case(cuda_lib, B=2, Nq=1, H=64, d=512, d_r=64, n_max=300, n_c=[300, 300],
                q_pos=[128 * 300 - 1, 128 * 150 + 5], hca=True, ratio=128, seed=7)
