@@ -555,9 +555,9 @@ constexpr int TOPK_HIST_CAND = 4096;     // boundary-bin candidates held in shar
 // Bin T (of HIST_BINS, thread t owning bins 4(T-1-t)..+3 counted from the top) holding the R-th largest
 // element given per-bin counts; returns {T, count above T, count in T} in sm.bcast[0..2] (zeros if R == 0
 // or R > total).  *total receives the number of counted elements.
-__device__ void hist_find_bin(TopkSmem& sm, const uint32_t* bins, uint32_t R, uint32_t* total) {
+// (hv: the four bins 4*owner .. 4*owner+3 this thread loaded, owner = blockDim.x - 1 - threadIdx.x)
+__device__ void hist_find_bin_v(TopkSmem& sm, const uint4 hv, uint32_t R, uint32_t* total) {
   const int owner = (int)blockDim.x - 1 - (int)threadIdx.x;
-  const uint4 hv = reinterpret_cast<const uint4*>(bins)[owner];
   const uint32_t mine = hv.x + hv.y + hv.z + hv.w;
   const uint32_t above_me = block_exclusive_scan(sm, mine, total);
   if (threadIdx.x == 0) { sm.bcast[0] = 0; sm.bcast[1] = 0; sm.bcast[2] = 0; }
@@ -577,6 +577,11 @@ __device__ void hist_find_bin(TopkSmem& sm, const uint32_t* bins, uint32_t R, ui
     }
   }
   __syncthreads();
+}
+
+__device__ void hist_find_bin(TopkSmem& sm, const uint32_t* bins, uint32_t R, uint32_t* total) {
+  const int owner = (int)blockDim.x - 1 - (int)threadIdx.x;
+  hist_find_bin_v(sm, reinterpret_cast<const uint4*>(bins)[owner], R, total);
 }
 
 // The `need` best of the nT boundary-bin candidates (keys, ids in shared memory) by (key desc, id asc),
@@ -711,7 +716,10 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
   uint32_t* ckeys = s_topk + TOPK_CHUNK;
   int32_t* cids = reinterpret_cast<int32_t*>(s_topk + TOPK_CHUNK + TOPK_HIST_CAND);
 
-  // the row into shared memory: one bulk copy when aligned, else plain loads
+  // the row's histogram first (16 KB, each thread its four bins), so those loads do not queue behind the
+  // row's copy; then the row into shared memory: one bulk copy when aligned, else plain loads
+  const uint4 hv = reinterpret_cast<const uint4*>(hist + (size_t)row * HIST_BINS)[blockDim.x - 1 - threadIdx.x];
+  __syncthreads();
   const uint32_t bytes = (uint32_t)len * 4u;
   const bool bulk = len > 0 && (len & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0 &&
                     (!isrc || (reinterpret_cast<uintptr_t>(isrc) & 15) == 0);
@@ -733,7 +741,7 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
     }
   }
   uint32_t nvalid;
-  hist_find_bin(sm, hist + (size_t)row * HIST_BINS, (uint32_t)A.k, &nvalid);   // overlaps the copy
+  hist_find_bin_v(sm, hv, (uint32_t)A.k, &nvalid);                             // overlaps the copy
   // the row's histogram is consumed: leave it zero for the next scoring call (each thread clears the
   // four bins it read)
   reinterpret_cast<uint4*>(hist + (size_t)row * HIST_BINS)[blockDim.x - 1 - threadIdx.x] = make_uint4(0, 0, 0, 0);
