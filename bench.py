@@ -543,6 +543,19 @@ def run_e2e(args, layers, inputs, stream, dev, world):
         for i in range(2 * s_layers):
             one(i)
     torch.cuda.synchronize()
+    # the packed inputs are the step's inputs: layer 0 run from them selects the same entries as when run
+    # from the original input tensors (the top-k writes its k ids in no fixed slot order, so they are
+    # compared as sorted lists) and gives the same output up to the summation order that slot order sets
+    got = staged[0]["out"].clone()
+    got_idx = layers[0].idx.sort(dim=-1).values
+    L0, i0 = layers[0], inputs[0]
+    with torch.cuda.stream(stream):
+        L0.step(i0["C"], i0["Z"], i0["b_pos"], i0["W_IK"], i0["q"], i0["q_I"], i0["w"], stream=stream)
+    torch.cuda.synchronize()
+    ref = L0.out.cpu().float()
+    if not torch.equal(got_idx, L0.idx.sort(dim=-1).values) or \
+            (got.float() - ref).abs().max().item() > 2.0 ** -6 * max(ref.abs().max().item(), 1.0):
+        raise RuntimeError("end-to-end path: the packed inputs do not reproduce the step's result")
     if world > 1:
         torch.distributed.barrier()
     t0 = torch.cuda.Event(enable_timing=True)
