@@ -353,61 +353,83 @@ constexpr int MERGE_MAX_SPLITS = 128;
 // together, so a merge of up to that many splits costs about one memory round trip.  Partials are fp32 (CUDA-core path) or bf16 (tensor-core path).
 constexpr int MERGE_WARPS = 4;
 
+// One split's partial for this lane's dims, held as loaded (bf16 pairs stay packed: 8 registers for 16
+// dims) and widened to fp32 only where it is summed, so a chunk of splits in flight costs few registers.
 template <typename PT, int DPL>
-__device__ __forceinline__ void load_dims(const PT* p, float* v);
+struct PartDims;
 template <>
-__device__ __forceinline__ void load_dims<uint16_t, 16>(const uint16_t* p, float* v) {
-  const uint4 a = *reinterpret_cast<const uint4*>(p), b = *reinterpret_cast<const uint4*>(p + 8);
-  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) { v[2 * i] = __uint_as_float(w[i] << 16); v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u); }
-}
-template <>
-__device__ __forceinline__ void load_dims<uint16_t, 4>(const uint16_t* p, float* v) {
-  const uint2 a = *reinterpret_cast<const uint2*>(p);
-  v[0] = __uint_as_float(a.x << 16); v[1] = __uint_as_float(a.x & 0xFFFF0000u);
-  v[2] = __uint_as_float(a.y << 16); v[3] = __uint_as_float(a.y & 0xFFFF0000u);
-}
-template <>
-__device__ __forceinline__ void load_dims<float, 16>(const float* p, float* v) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float4 f = reinterpret_cast<const float4*>(p)[i];
-    v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+struct PartDims<uint16_t, 16> {
+  uint4 a, b;
+  __device__ __forceinline__ void load(const uint16_t* p) {
+    a = *reinterpret_cast<const uint4*>(p);
+    b = *reinterpret_cast<const uint4*>(p + 8);
   }
-}
+  __device__ __forceinline__ float get(int i) const {
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    return (i & 1) ? __uint_as_float(w[i >> 1] & 0xFFFF0000u) : __uint_as_float(w[i >> 1] << 16);
+  }
+};
 template <>
-__device__ __forceinline__ void load_dims<float, 4>(const float* p, float* v) {
-  const float4 f = *reinterpret_cast<const float4*>(p);
-  v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-}
+struct PartDims<uint16_t, 4> {
+  uint2 a;
+  __device__ __forceinline__ void load(const uint16_t* p) { a = *reinterpret_cast<const uint2*>(p); }
+  __device__ __forceinline__ float get(int i) const {
+    const uint32_t w = i < 2 ? a.x : a.y;
+    return (i & 1) ? __uint_as_float(w & 0xFFFF0000u) : __uint_as_float(w << 16);
+  }
+};
+template <>
+struct PartDims<float, 16> {
+  float4 f[4];
+  __device__ __forceinline__ void load(const float* p) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = reinterpret_cast<const float4*>(p)[i];
+  }
+  __device__ __forceinline__ float get(int i) const {
+    const float4 v = f[i >> 2];
+    return (i & 3) == 0 ? v.x : (i & 3) == 1 ? v.y : (i & 3) == 2 ? v.z : v.w;
+  }
+};
+template <>
+struct PartDims<float, 4> {
+  float4 f;
+  __device__ __forceinline__ void load(const float* p) { f = *reinterpret_cast<const float4*>(p); }
+  __device__ __forceinline__ float get(int i) const { return i == 0 ? f.x : i == 1 ? f.y : i == 2 ? f.z : f.w; }
+};
 
 // Inverse-RoPE epilogue on one (query, head) row held one lane-slice of DPL dims per lane (lane l: dims
 // DPL l .. DPL l + DPL - 1): the RoPE channels (the last DR) sit on lanes L0 .. 31, the first half of each
 // pair (m) HL lanes before its second half (m + DR/2); every lane of the warp must call it.
 // (x1, x2) -> (x1 cos a + x2 sin a, -x1 sin a + x2 cos a), a = t theta^(-2m/DR): the angle in double,
-// reduced by 2 pi (split in two parts) before the single-precision sin / cos.
+// reduced by 2 pi (split in two parts) before the single-precision sin / cos.  Lane l computes the
+// rotation of pair m = l mod DR/2 once, and the RoPE lanes fetch theirs by shuffles, so the warp spends
+// one angle per lane rather than DPL per RoPE lane.
 template <int D>
 __device__ __forceinline__ void inverse_rope_lanes(float* y, int lane, long long t, float theta) {
   constexpr int DPL = D / 32, DR = D == 512 ? 64 : 32, L0 = (D - DR) / DPL, HL = DR / 2 / DPL;
   float pz[DPL];
 #pragma unroll
   for (int i = 0; i < DPL; ++i) pz[i] = __shfl_xor_sync(0xffffffffu, y[i], HL);
-  if (lane < L0) return;
-  const int jl = lane - L0;
-  const bool first = jl < HL;
-  const int m0 = (jl % HL) * DPL;
-  const double l2t = log2((double)theta);
-#pragma unroll
-  for (int i = 0; i < DPL; ++i) {
-    const double ang = (double)t * exp2(-2.0 * (double)(m0 + i) / DR * l2t);
+  float sn_l, cs_l;
+  {
+    const int m = lane % (DR / 2);
+    const double ang = (double)t * exp2(-2.0 * (double)m / DR * log2((double)theta));
     const double kk = rint(ang * 0.15915494309189535);             // 1 / (2 pi)
     double red = fma(-kk, 6.283185307179586, ang);                  // 2 pi, high part
     red = fma(-kk, 2.4492935982947064e-16, red);                    // 2 pi, low part
-    float sn, cs;
-    sincosf((float)red, &sn, &cs);
-    const float x1 = first ? y[i] : pz[i], x2 = first ? pz[i] : y[i];
-    y[i] = first ? fmaf(x1, cs, x2 * sn) : fmaf(-x1, sn, x2 * cs);
+    sincosf((float)red, &sn_l, &cs_l);
+  }
+  const int jl = lane - L0;
+  const bool first = jl < HL;
+  const int m0 = ((jl >= 0 ? jl : 0) % HL) * DPL;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    const float sn = __shfl_sync(0xffffffffu, sn_l, m0 + i);
+    const float cs = __shfl_sync(0xffffffffu, cs_l, m0 + i);
+    if (jl >= 0) {
+      const float x1 = first ? y[i] : pz[i], x2 = first ? pz[i] : y[i];
+      y[i] = first ? fmaf(x1, cs, x2 * sn) : fmaf(-x1, sn, x2 * cs);
+    }
   }
 }
 
@@ -421,7 +443,9 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) attn_merge_kernel(const PT* 
   constexpr int MERGE_CHUNK = D == 512 ? 6 : 8;   // splits whose partials are in flight at once
   const int lane = threadIdx.x & 31;
   const long long unit = (long long)blockIdx.x * MERGE_WARPS + (threadIdx.x >> 5);
-  pdl_trigger();
+  // the kernel after the merge is launched only once every merge CTA has stored its rows (the trigger is
+  // at the end): launched earlier, its CTAs crowd onto the few SMs the merge leaves free (in a decode step
+  // the next compressor then holds three CTAs on an SM and keeps the indexer it runs beside off it)
   pdl_wait();
   if (unit >= units) return;
   const long long bq = unit / H;
@@ -435,11 +459,12 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) attn_merge_kernel(const PT* 
   if (splits <= MERGE_CHUNK) {
     // one round: every lane loads all split lse values (broadcast) and its dims of every partial; empty
     // splits (lse = -inf, partial never written) are dropped by a select, never multiplied
-    float v[MERGE_CHUNK][DPL], ls[MERGE_CHUNK];
+    PartDims<PT, DPL> v[MERGE_CHUNK];
+    float ls[MERGE_CHUNK];
 #pragma unroll
     for (int c = 0; c < MERGE_CHUNK; ++c) {
       ls[c] = c < splits ? lrow[(long long)c * H] : -INFINITY;
-      if (c < splits) load_dims<PT, DPL>(base + (long long)c * H * D, v[c]);
+      if (c < splits) v[c].load(base + (long long)c * H * D);
     }
 #pragma unroll
     for (int c = 0; c < MERGE_CHUNK; ++c) mx = fmaxf(mx, ls[c]);
@@ -449,7 +474,7 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) attn_merge_kernel(const PT* 
       sum += w;
       if (w != 0.f)
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w, v[c][i], acc[i]);
+        for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w, v[c].get(i), acc[i]);
     }
   } else {
     // max and weights of the split lse values (lanes hold splits s = lane, lane + 32, ...)
@@ -461,7 +486,7 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) attn_merge_kernel(const PT* 
     }
     sum = warp_sum(sum);
     for (int s0 = 0; s0 < splits; s0 += MERGE_CHUNK) {
-      float v[MERGE_CHUNK][DPL];
+      PartDims<PT, DPL> v[MERGE_CHUNK];
       float wgt[MERGE_CHUNK];
 #pragma unroll
       for (int c = 0; c < MERGE_CHUNK; ++c) {
@@ -471,13 +496,13 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) attn_merge_kernel(const PT* 
           const float l = lrow[(long long)s * H];
           wgt[c] = (mx == -INFINITY || l == -INFINITY) ? 0.f : exp2f((l - mx) * LOG2E);
         }
-        if (wgt[c] != 0.f) load_dims<PT, DPL>(base + (long long)s * H * D, v[c]);
+        if (wgt[c] != 0.f) v[c].load(base + (long long)s * H * D);
       }
 #pragma unroll
       for (int c = 0; c < MERGE_CHUNK; ++c)
         if (wgt[c] != 0.f)
 #pragma unroll
-          for (int i = 0; i < DPL; ++i) acc[i] = fmaf(wgt[c], v[c][i], acc[i]);
+          for (int i = 0; i < DPL; ++i) acc[i] = fmaf(wgt[c], v[c].get(i), acc[i]);
     }
   }
   const float inv = sum > 0.f ? 1.f / sum : 0.f;
@@ -495,6 +520,7 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) attn_merge_kernel(const PT* 
     *reinterpret_cast<uint2*>(o) = make_uint2(pk[0], pk[1]);
   }
   if (lse && lane == 0) lse[bq * H + h] = sum > 0.f ? mx + logf(sum) : -INFINITY;
+  pdl_trigger();
 }
 
 template <typename PT>
@@ -524,8 +550,11 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) out_rope_kernel(uint16_t* __
   pdl_wait();
   if (unit >= units) return;
   uint16_t* o = out + unit * (long long)D + lane * DPL;
+  PartDims<uint16_t, DPL> raw;
+  raw.load(o);
   float y[DPL];
-  load_dims<uint16_t, DPL>(o, y);
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) y[i] = raw.get(i);
   inverse_rope_lanes<D>(y, lane, q_pos[unit / H], rope_theta);
   uint32_t pk[DPL / 2];
 #pragma unroll
