@@ -521,21 +521,24 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(TopkRowArgs A) {
 }
 
 
-// Exact selection of the `need` best of n <= 64 candidates (key desc, id asc, position asc) by one warp:
-// each candidate's rank is the number of candidates that beat it.  Writes the winners at oi/os[base + rank].
-__device__ void warp_rank_select(const uint32_t* keys, const int32_t* ids, int n, uint32_t need, int32_t* oi,
-                                 float* os, uint32_t base) {
-  const int lane = threadIdx.x & 31;
-  for (int i = lane; i < n; i += 32) {
+// Exact selection of the `need` best of n <= 64 candidates (key desc, id asc, position asc) by the whole
+// block: warp w ranks candidates w, w + #warps, ... (its lanes split the comparisons; a candidate's rank is
+// the number of candidates that beat it) and writes the winners at oi/os[base + rank].  Every thread of
+// the block calls it.
+__device__ void block_rank_select(const uint32_t* keys, const int32_t* ids, int n, uint32_t need, int32_t* oi,
+                                  float* os, uint32_t base) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int i = warp; i < n; i += nw) {
     const uint32_t ki = keys[i];
     const int32_t ii = ids[i];
-    uint32_t rank = 0;
-    for (int j = 0; j < n; ++j) {
+    uint32_t beat = 0;
+    for (int j = lane; j < n; j += 32) {
       const uint32_t kj = keys[j];
       const int32_t ij = ids[j];
-      rank += (kj > ki) || (kj == ki && (ij < ii || (ij == ii && j < i)));
+      beat += (kj > ki) || (kj == ki && (ij < ii || (ij == ii && j < i)));
     }
-    if (rank < need) {
+    const uint32_t rank = __reduce_add_sync(0xffffffffu, beat);
+    if (lane == 0 && rank < need) {
       oi[base + rank] = ii;
       if (os) os[base + rank] = order_key_float(ki);
     }
@@ -558,12 +561,31 @@ constexpr int TOPK_HIST_CAND = 4096;     // boundary-bin candidates held in shar
 // (hv: the four bins 4*owner .. 4*owner+3 this thread loaded, owner = blockDim.x - 1 - threadIdx.x)
 __device__ void hist_find_bin_v(TopkSmem& sm, const uint4 hv, uint32_t R, uint32_t* total) {
   const int owner = (int)blockDim.x - 1 - (int)threadIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const uint32_t mine = hv.x + hv.y + hv.z + hv.w;
-  const uint32_t above_me = block_exclusive_scan(sm, mine, total);
-  if (threadIdx.x == 0) { sm.bcast[0] = 0; sm.bcast[1] = 0; sm.bcast[2] = 0; }
+  // counts above this thread's bins: an inclusive scan inside the warp (threads in order of descending
+  // bins), then every warp scans the warp totals itself (two barriers in all)
+  uint32_t x = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sm.scan[warp] = x;
   __syncthreads();
-  const uint32_t K = min(R, *total);
-  if (K > 0 && above_me < K && K <= above_me + mine) {
+  const uint32_t wt = lane < nw ? sm.scan[lane] : 0u;
+  uint32_t wi = wt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+    if (lane >= o) wi += y;
+  }
+  const uint32_t wbase = __shfl_sync(0xffffffffu, wi - wt, warp);
+  const uint32_t tot = __shfl_sync(0xffffffffu, wi, nw - 1);
+  *total = tot;
+  const uint32_t above_me = wbase + x - mine;
+  const uint32_t K = min(R, tot);
+  if (K > 0 && above_me < K && K <= above_me + mine) {       // exactly one thread holds the K-th count
     const uint32_t c[4] = {hv.w, hv.z, hv.y, hv.x};
     uint32_t acc = above_me;
     for (int i = 0; i < 4; ++i) {
@@ -576,6 +598,7 @@ __device__ void hist_find_bin_v(TopkSmem& sm, const uint4 hv, uint32_t R, uint32
       acc += c[i];
     }
   }
+  if (K == 0 && threadIdx.x == 0) { sm.bcast[0] = 0; sm.bcast[1] = 0; sm.bcast[2] = 0; }
   __syncthreads();
 }
 
@@ -595,7 +618,7 @@ __device__ void resolve_boundary(TopkSmem& sm, uint32_t* ckeys, int32_t* cids, u
       if (os) os[above + j] = order_key_float(ckeys[j]);
     }
   } else if (nT <= (uint32_t)TOPK_RANK_MAX) {
-    if (threadIdx.x < 32) warp_rank_select(ckeys, cids, (int)nT, need, oi, os, above);
+    block_rank_select(ckeys, cids, (int)nT, need, oi, os, above);
   } else {
     // boundary bin: 8-bit digits of the remaining key bits (19..12, 11..4, 3..0), one 256-bin histogram
     // per level scanned by one warp, until at most TOPK_RANK_MAX candidates share the threshold prefix;
@@ -665,7 +688,7 @@ __device__ void resolve_boundary(TopkSmem& sm, uint32_t* ckeys, int32_t* cids, u
       pmask = nmask;
       n_in = n2;
       if (n2 <= (uint32_t)TOPK_RANK_MAX) {
-        if (threadIdx.x < 32) warp_rank_select(k2, i2, (int)n2, rem, oi, os, base_out);
+        block_rank_select(k2, i2, (int)n2, rem, oi, os, base_out);
         ranked = true;
       }
     }
@@ -760,7 +783,10 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
     const bool fast = !isrc && Tbin > 0;                          // no ids; -inf lies below the bin
     uint32_t m_up = 0, m_at = 0;
     if (fast) {
-#pragma unroll 2
+      // one compare per score (at or above the bin: about k of the row), then the few set bits are split
+      // into above the bin / in it
+      uint32_t m_ge = 0;
+#pragma unroll
       for (int i = 0; i < TOPK_HIST_PER_THREAD / 4; ++i) {
         const int j0 = 4 * (threadIdx.x + TOPK_THREADS * i);
         float4 f4 = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
@@ -771,13 +797,14 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
           if (j0 + 1 < len) f4.y = s_row[j0 + 1];
           if (j0 + 2 < len) f4.z = s_row[j0 + 2];
         }
-        const uint32_t u = (uint32_t)(f4.x > hi) | ((uint32_t)(f4.y > hi) << 1) | ((uint32_t)(f4.z > hi) << 2) |
-                           ((uint32_t)(f4.w > hi) << 3);
-        const uint32_t g = (uint32_t)(f4.x >= lo) | ((uint32_t)(f4.y >= lo) << 1) | ((uint32_t)(f4.z >= lo) << 2) |
-                           ((uint32_t)(f4.w >= lo) << 3);
-        m_up |= u << (4 * i);
-        m_at |= (g & ~u) << (4 * i);
+        m_ge |= ((uint32_t)(f4.x >= lo) | ((uint32_t)(f4.y >= lo) << 1) | ((uint32_t)(f4.z >= lo) << 2) |
+                 ((uint32_t)(f4.w >= lo) << 3)) << (4 * i);
       }
+      for (uint32_t mk = m_ge; mk; mk &= mk - 1u) {
+        const int e = __ffs(mk) - 1;
+        if (s_row[4 * (threadIdx.x + TOPK_THREADS * (e >> 2)) + (e & 3)] > hi) m_up |= 1u << e;
+      }
+      m_at = m_ge & ~m_up;
     } else {
 #pragma unroll 1
       for (int i = 0; i < TOPK_HIST_PER_THREAD / 4; ++i) {
