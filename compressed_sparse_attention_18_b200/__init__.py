@@ -293,8 +293,10 @@ def index_scores(q_I, w, kcache: PackedCache, n_c, q_pos, scores, *, ratio, g_q=
 
 
 def topk(scores, kcache: PackedCache, n_c, q_pos, *, B, Nq, ratio, k, cand=None, pool_blocks=0, pool_block_size=8,
-         want_scores=False, idx_out=None, scores_out=None, pool_out=None, hist=None, ws=None, stream=None):
-    """Top-k (+ hierarchical pool) over a score matrix written by index_scores (see csa_topk)."""
+         want_scores=False, idx_out=None, scores_out=None, pool_out=None, hist=None, ws=None, early_start=False,
+         stream=None):
+    """Top-k (+ hierarchical pool) over a score matrix written by index_scores (see csa_topk).
+    early_start: CSA_EARLY_START (only right after the index_scores call of the same decode step)."""
     dev = scores.device
     if idx_out is None:
         idx_out = torch.empty((B, Nq, k), dtype=torch.int32, device=dev)
@@ -306,6 +308,7 @@ def topk(scores, kcache: PackedCache, n_c, q_pos, *, B, Nq, ratio, k, cand=None,
     a = IndexArgs(ctypes.sizeof(IndexArgs), B, Nq, 1, d_I, ratio, k, kcache.n_max, 1.0, kcache.g, None, None,
                   None, None, _ptr(n_c), _ptr(q_pos), _ptr(cand), cand.shape[-1] if cand is not None else 0,
                   pool_blocks, pool_block_size, _ptr(pool_out), _ptr(idx_out), _ptr(scores_out), _ptr(hist))
+    a.flags = CSA_EARLY_START if early_start else 0
     nbytes = _lib.csa_topk_workspace_size(ctypes.byref(a))
     wbuf = _ws(nbytes, dev, ws)
     _check(_lib.csa_topk(ctypes.byref(a), _ptr(scores), scores.shape[-1], _ptr(wbuf) if wbuf is not None else None,

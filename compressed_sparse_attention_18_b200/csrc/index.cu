@@ -400,6 +400,7 @@ struct TopkRowArgs {
   float* out_scores;
   long long out_ld;
   const LongRowState* skip;   // rows whose state says resolved are left alone (null: none)
+  int early;                  // histogram rows: q_pos and n_c are read before the wait (CSA_EARLY_START)
 };
 
 
@@ -666,19 +667,41 @@ __device__ void resolve_boundary(TopkSmem& sm, uint32_t* ckeys, int32_t* cids, u
       __syncthreads();
       const uint32_t digit = sm.bcast[0], above2 = sm.bcast[1], n2 = sm.bcast[2];
       const uint32_t npref = pref | (digit << sh), nmask = pmask | (dm << sh);
-      // write the candidates in a higher digit; keep the threshold digit's few for ranking
-      for (int j = threadIdx.x; j < (int)nT; j += blockDim.x) {
-        const uint32_t k = ckeys[j] & 0xFFFFFu;
-        if ((k & pmask) != pref) continue;
-        const uint32_t dj = (k >> sh) & dm;
-        if (dj > digit) {
-          const uint32_t slot = base_out + atomicAdd(&s_cnt[0], 1u);
-          oi[slot] = cids[j];
-          if (os) os[slot] = order_key_float(ckeys[j]);
-        } else if (dj == digit && n2 <= (uint32_t)TOPK_RANK_MAX) {
-          const uint32_t slot = atomicAdd(&s_cnt[1], 1u);
-          k2[slot] = ckeys[j];
-          i2[slot] = cids[j];
+      // write the candidates in a higher digit; keep the threshold digit's few for ranking (slots from one
+      // shared counter per warp and kind: lanes take theirs from the ballot below them)
+      const int lane = threadIdx.x & 31;
+      for (int j0 = 0; j0 + (int)(threadIdx.x & ~31u) < (int)nT; j0 += blockDim.x) {
+        const int j = j0 + (int)threadIdx.x;
+        bool up = false, at = false;
+        uint32_t kj = 0;
+        int32_t ij = 0;
+        if (j < (int)nT) {
+          kj = ckeys[j];
+          ij = cids[j];
+          const uint32_t k = kj & 0xFFFFFu;
+          if ((k & pmask) == pref) {
+            const uint32_t dj = (k >> sh) & dm;
+            up = dj > digit;
+            at = dj == digit && n2 <= (uint32_t)TOPK_RANK_MAX;
+          }
+        }
+        const uint32_t bu = __ballot_sync(0xffffffffu, up), ba = __ballot_sync(0xffffffffu, at);
+        uint32_t su = 0, sa = 0;
+        if (lane == 0) {
+          if (bu) su = atomicAdd(&s_cnt[0], (uint32_t)__popc(bu));
+          if (ba) sa = atomicAdd(&s_cnt[1], (uint32_t)__popc(ba));
+        }
+        su = __shfl_sync(0xffffffffu, su, 0);
+        sa = __shfl_sync(0xffffffffu, sa, 0);
+        const uint32_t below = (1u << lane) - 1u;
+        if (up) {
+          const uint32_t slot = base_out + su + (uint32_t)__popc(bu & below);
+          oi[slot] = ij;
+          if (os) os[slot] = order_key_float(kj);
+        } else if (at) {
+          const uint32_t slot = sa + (uint32_t)__popc(ba & below);
+          k2[slot] = kj;
+          i2[slot] = ij;
         }
       }
       __syncthreads();
@@ -721,15 +744,25 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
                          A.out_idx ? (const void*)(A.out_idx + row * A.out_ld) : r0};
     prefetch_l2(pf[threadIdx.x]);
   }
-  pdl_wait();                                  // scores and histogram come from the previous kernel
-  int len = min(A.rows_per_seg, A.n_cols);
-  if (A.q_pos) {
-    const int b = row / A.Nq;
-    long long nv = (A.q_pos[row] + 1) / A.ratio;
-    if (nv > A.n_c[b]) nv = A.n_c[b];
-    len = (int)max(0LL, min((long long)len, nv));
+  // the row's visible length: under the early start the positions (inputs of the step that no kernel of
+  // it writes) are read before the wait, so the row's copy can be issued the moment the scores are final
+  auto row_len = [&]() -> int {
+    int n = min(A.rows_per_seg, A.n_cols);
+    if (A.q_pos) {
+      const int b = row / A.Nq;
+      long long nv = (A.q_pos[row] + 1) / A.ratio;
+      if (nv > A.n_c[b]) nv = A.n_c[b];
+      n = (int)max(0LL, min((long long)n, nv));
+    }
+    return max(n, 0);
+  };
+  int len = A.early ? row_len() : 0;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&row_bar, 1);
+    sm100::fence_mbar_init();
   }
-  if (len < 0) len = 0;
+  pdl_wait();                                  // scores and histogram come from the previous kernel
+  if (!A.early) len = row_len();
   int32_t* oi = A.out_idx + row * A.out_ld;
   float* os = A.out_scores ? A.out_scores + row * A.out_ld : nullptr;
   const float* src = A.in_scores + row * A.in_ld;
@@ -747,8 +780,6 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_hist_kernel(TopkRowArgs A, 
   const bool bulk = len > 0 && (len & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0 &&
                     (!isrc || (reinterpret_cast<uintptr_t>(isrc) & 15) == 0);
   if (bulk && threadIdx.x == 0) {
-    sm100::mbar_init(&row_bar, 1);
-    sm100::fence_mbar_init();
     sm100::mbar_arrive_expect_tx(&row_bar, bytes * (isrc ? 2u : 1u));
     for (uint32_t off = 0; off < bytes; off += 32768u) {
       const uint32_t n = min(32768u, bytes - off);
@@ -1165,6 +1196,7 @@ static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const 
   ta.Nq = a->Nq;
   ta.rows_per_seg = p.seg_len;
   ta.k = a->k;
+  ta.early = (a->flags & CSA_EARLY_START) ? 1 : 0;
   if (a->cand) CSA_SUPPORTED(ld == a->n_cand);   // explicit ids are read with the score row stride
   if (p.segs == 1 && hist != nullptr && p.hist) {
     ta.out_idx = a->idx_out;

@@ -133,7 +133,7 @@ class CSADecodeLayer:
                          k=s.k, early_start=self.early, stream=st)
             mark(2)
             topk(self.scores, self.ki, self.n_c, self.q_pos, B=s.B, Nq=1, ratio=s.r, k=s.k, idx_out=self.idx,
-                 hist=self.hist, ws=self.ws_index, stream=st)
+                 hist=self.hist, ws=self.ws_index, early_start=self.early, stream=st)
         mark(3)
         sparse_attn(q, self.q_pos, self.kv, self.n_c, self.idx, self.win, self.win_pos0, ratio=s.r, window=s.W,
                     out=self.out, lse=self.lse, ws=self.ws_attn, early_start=self.early, cluster=self.cluster,

@@ -78,6 +78,10 @@ csa_status csa_check_error_path(uint32_t polls, void* stream);
  *     q_pos and the key rows [0, n_c[b] - 1) at once and writes scores and hist; only the 256-row
  *     tile that holds row n_c[b] - 1 waits.  Requires: the kernel just before the call is csa_compress,
  *     and that call writes none of these inputs except key rows >= n_c[b] - 1.
+ *   - csa_topk / the selection of csa_index_topk (single-CTA histogram rows): reads n_c and q_pos before
+ *     the scores are final, so the row's copy starts the moment they are.  Requires: the call follows
+ *     csa_index_scores (csa_index_topk: its own scoring) of the same step, which follows csa_compress,
+ *     and none of these calls writes n_c or q_pos.
  *   - csa_sparse_attn (k % 128 == 0, window <= 128): the window tile of every query runs in a CTA of
  *     its own that reads q, q_pos, n_c, win_kv, win_pos0 and writes its workspace partial at once; the
  *     CTAs over the selected entries wait as usual.  Requires: the step's earlier calls since
