@@ -383,6 +383,16 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       for (int c = 0; c < 4; ++c) rp[c] = make_uint4(0, 0, 0, 0);
       const long long r = id >= 0 ? page_row(P.pm, b, P.n_max, id) : -1;   // row in the cache arrays
       if (r >= 0) {
+        // the row's lines are requested from L2 first: a prefetch holds no L1 miss slot, and the 128 random
+        // rows of a tile otherwise reach DRAM only as fast as the SM's outstanding misses drain
+        if (ghalf == 0) {
+          prefetch_l2(P.codes + (size_t)r * 224);
+          prefetch_l2(P.codes + (size_t)r * 224 + 223);
+          prefetch_l2(P.scales + (size_t)r * 16);
+        } else {
+          prefetch_l2(P.codes + (size_t)r * 224 + 112);
+          prefetch_l2(P.rope + (size_t)r * 64);
+        }
         const uint8_t* crow = P.codes + (size_t)r * 224 + ghalf * 16;
 #pragma unroll
         for (int j = 0; j < 7; ++j) cv[j] = __ldg(reinterpret_cast<const uint4*>(crow + j * 32));
