@@ -115,3 +115,36 @@ def test_early_start_window_ragged_and_absent(cuda_lib):
             o_ref, l_ref = O.attention(f64(inp["q"][b]), [tb], rows, idx[b].cpu().numpy(), n_c,
                                        np.zeros((0, s.d)), 0, s.W, s.d ** -0.5)
             assert_close(f64(o0[b]), o_ref, OUT_ATOL, OUT_RTOL, f"out no window b={b} early={early}")
+
+
+def test_topk_early_start_same_selection(cuda_lib):
+    """csa_topk with CSA_EARLY_START reads each row's positions before its wait: on rows of different
+    lengths and visibilities it selects exactly what the plain call selects (and leaves the histogram
+    rows it read zero), the selection being the oracle's."""
+    csa = cuda_lib
+    from csa_workloads import gen, normal
+    G = gen(31)
+    B, n, k = 5, 9000, 512
+    n_c = [9000, 513, 1, 4000, 8999]
+    q_pos = [4 * 9000 - 1, 4 * 513 - 1, 3, 4 * 3000 + 1, 4 * 8999 - 1]
+    kI = normal((B, n, 128), 1.0, G)
+    qI = normal((B, 1, 8, 128), 1.0, G).to(DEV)
+    w = normal((B, 1, 8), 8 ** -0.5, G, dtype=torch.float32).to(DEV)
+    kc = csa.PackedCache(B, n, 128, 0, DEV, 1.0)
+    csa.pack_fp4(kI.to(DEV), kc)
+    n_c_t = torch.tensor(n_c, dtype=torch.int32, device=DEV)
+    q_pos_t = torch.tensor(q_pos, dtype=torch.int64, device=DEV).view(B, 1)
+    scores = torch.empty((B, n), dtype=torch.float32, device=DEV)
+    h1 = torch.zeros((B, 4096), dtype=torch.int32, device=DEV)
+    csa.index_scores(qI, w, kc, n_c_t, q_pos_t, scores, ratio=4, hist=h1, k=k)
+    h2 = h1.clone()
+    i1, _, _ = csa.topk(scores, kc, n_c_t, q_pos_t, B=B, Nq=1, ratio=4, k=k, hist=h1)
+    i2, _, _ = csa.topk(scores, kc, n_c_t, q_pos_t, B=B, Nq=1, ratio=4, k=k, hist=h2, early_start=True)
+    torch.cuda.synchronize()
+    assert int(h1.abs().sum()) == 0 and int(h2.abs().sum()) == 0
+    assert torch.equal(i1.sort(dim=-1).values, i2.sort(dim=-1).values)
+    for b in range(B):
+        codes, scales, _ = O.pack_fp4(f64(kI[b]), 0, 1.0)
+        s_ref, ids = O.index_scores(f64(qI[b].cpu()), f64(w[b].cpu()), 1.0, codes, scales, 1.0,
+                                    q_pos_t[b].cpu().numpy(), n_c[b], 4)
+        check_topk_row(i2[b, 0].cpu().numpy(), s_ref[0], ids[0], k, f"early top-k b={b}")
