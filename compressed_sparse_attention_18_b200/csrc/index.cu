@@ -915,7 +915,6 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_long_kernel(TopkRowArgs A, 
   __shared__ uint32_t s_cnt[2];
   __shared__ uint32_t s_last;
   const int seg = blockIdx.x, row = blockIdx.y;
-  const int lane = threadIdx.x & 31;
   pdl_trigger();
   pdl_wait();                                  // scores and histogram come from the previous kernel
   int len = A.n_cols;
@@ -938,34 +937,55 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_long_kernel(TopkRowArgs A, 
   const float* src = A.in_scores + row * A.in_ld;
   const int c0 = seg * TOPK_CHUNK, c1 = min(len, c0 + TOPK_CHUNK);
   if (K > 0) {
-    const uint32_t lt = (1u << lane) - 1u;
-#pragma unroll 4
-    for (int base = c0; base < c1; base += blockDim.x) {   // block-uniform trip count
-      const int j = base + threadIdx.x;
-      const float v = j < c1 ? src[j] : -INFINITY;
-      const uint32_t bin = float_order_key(v) >> HIST_SHIFT;
-      const bool valid = v > -INFINITY;
-      const bool up = valid && bin > T, at = valid && bin == T;
-      const uint32_t mu = __ballot_sync(0xffffffffu, up), ma = __ballot_sync(0xffffffffu, at);
-      if (mu) {
-        uint32_t b0 = 0;
-        if (lane == 0) b0 = atomicAdd(&rs.up, (uint32_t)__popc(mu));
-        b0 = __shfl_sync(0xffffffffu, b0, 0);
-        const uint32_t slot = b0 + (uint32_t)__popc(mu & lt);
-        if (up && slot < above) {
-          oi[slot] = j;
-          if (os) os[slot] = v + 0.0f;
-        }
+    // this CTA's 32 scores per thread as bit masks (above the boundary bin / in it), one block scan, then one
+    // reservation per CTA in the row's counters (not one dependent atomic per warp and hit)
+    const bool vec = (reinterpret_cast<uintptr_t>(src) & 15) == 0;   // block-uniform
+    uint32_t m_up = 0, m_at = 0;
+#pragma unroll
+    for (int i = 0; i < TOPK_HIST_PER_THREAD / 4; ++i) {
+      const int j0 = c0 + 4 * (threadIdx.x + TOPK_THREADS * i);
+      float f[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (vec && j0 + 3 < c1) {
+        const float4 f4 = *reinterpret_cast<const float4*>(src + j0);
+        f[0] = f4.x; f[1] = f4.y; f[2] = f4.z; f[3] = f4.w;
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (j0 + c < c1) f[c] = src[j0 + c];
       }
-      if (ma) {
-        uint32_t b0 = 0;
-        if (lane == 0) b0 = atomicAdd(&rs.at, (uint32_t)__popc(ma));
-        b0 = __shfl_sync(0xffffffffu, b0, 0);
-        const uint32_t c = b0 + (uint32_t)__popc(ma & lt);
-        if (at && c < (uint32_t)TOPK_HIST_CAND) {
-          ck[c] = float_order_key(v);
-          ci[c] = j;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t bin = float_order_key(f[c]) >> HIST_SHIFT;
+        const bool valid = f[c] > -INFINITY;
+        if (valid && bin > T) m_up |= 1u << (4 * i + c);
+        if (valid && bin == T) m_at |= 1u << (4 * i + c);
+      }
+    }
+    uint32_t tot;
+    const uint32_t pre = block_exclusive_scan(sm, (uint32_t)__popc(m_up) | ((uint32_t)__popc(m_at) << 16), &tot);
+    if (threadIdx.x == 0) {
+      s_cnt[0] = (tot & 0xFFFFu) ? atomicAdd(&rs.up, tot & 0xFFFFu) : 0u;
+      s_cnt[1] = (tot >> 16) ? atomicAdd(&rs.at, tot >> 16) : 0u;
+    }
+    __syncthreads();
+    uint32_t su = s_cnt[0] + (pre & 0xFFFFu), sa = s_cnt[1] + (pre >> 16);
+#pragma unroll 1
+    for (uint32_t mk = m_up | m_at; mk; mk &= mk - 1u) {
+      const int e = __ffs(mk) - 1;
+      const int j = c0 + 4 * (threadIdx.x + TOPK_THREADS * (e >> 2)) + (e & 3);
+      const float v = src[j];
+      if ((m_up >> e) & 1u) {
+        if (su < above) {
+          oi[su] = j;
+          if (os) os[su] = v + 0.0f;
         }
+        ++su;
+      } else {
+        if (sa < (uint32_t)TOPK_HIST_CAND) {
+          ck[sa] = float_order_key(v);
+          ci[sa] = j;
+        }
+        ++sa;
       }
     }
   }
@@ -1002,21 +1022,39 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_long_kernel(TopkRowArgs A, 
 }
 
 // ------------------------------------------------------------------------- hierarchical pool
-__global__ void block_max_kernel(const float* __restrict__ scores, long long ld, int n_cols,
-                                 const int64_t* __restrict__ q_pos, const int32_t* __restrict__ n_c, int ratio,
-                                 int Nq, int G, int nblk, float* __restrict__ bs) {
+// Block scores of the hierarchical pool (max over the visible keys of each block of G) and their row
+// histogram (top 12 bits of the order-preserving key; blocks without a visible key are -inf and not
+// counted), so the pool's top blocks are selected like a decode row.  CTA: BM_THREADS threads x
+// BM_PER_THREAD blocks of one row; its histogram is added to the row's (zero on entry).
+constexpr int BM_THREADS = 1024, BM_PER_THREAD = 4;
+__global__ void __launch_bounds__(BM_THREADS) block_max_kernel(const float* __restrict__ scores, long long ld,
+                                                               int n_cols, const int64_t* __restrict__ q_pos,
+                                                               const int32_t* __restrict__ n_c, int ratio, int Nq,
+                                                               int G, int nblk, float* __restrict__ bs,
+                                                               uint32_t* __restrict__ bhist) {
+  __shared__ uint32_t h[HIST_BINS];
   const int row = blockIdx.y;
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= nblk) return;
+  for (int i = threadIdx.x; i < HIST_BINS; i += blockDim.x) h[i] = 0;
   long long nv = (q_pos[row] + 1) / ratio;
   if (nv > n_c[row / Nq]) nv = n_c[row / Nq];
   if (nv > n_cols) nv = n_cols;
-  float m = -INFINITY;
-  for (int e = 0; e < G; ++e) {
-    const long long i = (long long)j * G + e;
-    if (i < nv) m = fmaxf(m, scores[row * ld + i]);
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < BM_PER_THREAD; ++u) {
+    const int j = (blockIdx.x * BM_PER_THREAD + u) * BM_THREADS + threadIdx.x;
+    if (j >= nblk) break;
+    float m = -INFINITY;
+    for (int e = 0; e < G; ++e) {
+      const long long i = (long long)j * G + e;
+      if (i < nv) m = fmaxf(m, scores[row * ld + i]);
+    }
+    bs[(long long)row * nblk + j] = m;
+    if (m > -INFINITY) atomicAdd(&h[float_order_key(m) >> HIST_SHIFT], 1u);
   }
-  bs[(long long)row * nblk + j] = m;
+  __syncthreads();
+  uint32_t* hr = bhist + (size_t)row * HIST_BINS;
+  for (int i = threadIdx.x; i < HIST_BINS; i += blockDim.x)
+    if (h[i]) atomicAdd(&hr[i], h[i]);
 }
 
 __global__ void pool_expand_kernel(const int32_t* __restrict__ blk, int P, int G, const float* __restrict__ scores,
@@ -1050,7 +1088,7 @@ csa_status run_index_topk_fused(const csa_index_args* a, cudaStream_t st);
 struct IndexPlan {
   int rows, n_cols, segs, seg_len;
   bool hist;   // single-query rows: histogram-guided selection (long rows: segment CTAs + tournament fallback)
-  size_t off_scores, off_tidx, off_tsc, off_bs, off_bidx, off_lstate, off_lcand, off_hist, sel_total, total;
+  size_t off_scores, off_tidx, off_tsc, off_bs, off_bidx, off_bhist, off_lstate, off_lcand, off_hist, sel_total, total;
 };
 
 static bool one_query_per_cta(const csa_index_args* a) { return a->cand != nullptr || a->Nq == 1; }
@@ -1079,6 +1117,7 @@ static IndexPlan plan_index(const csa_index_args* a) {
     const int nblk = (p.n_cols + G - 1) / G;
     p.off_bs = o;   o = align_up(o + (size_t)p.rows * nblk * 4, 256);
     p.off_bidx = o; o = align_up(o + (size_t)p.rows * a->pool_blocks * 4, 256);
+    p.off_bhist = o; o = align_up(o + (size_t)p.rows * HIST_BINS * 4, 256);
   }
   p.sel_total = o;
   p.off_scores = o;
@@ -1264,10 +1303,18 @@ static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const 
     const int nblk = (p.n_cols + G - 1) / G;
     float* bs = (float*)(w8 + p.off_bs);
     int32_t* bidx = (int32_t*)(w8 + p.off_bidx);
-    block_max_kernel<<<dim3((nblk + 255) / 256, p.rows), 256, 0, st>>>(scores, ld, p.n_cols, a->q_pos, a->n_c,
-                                                                        a->ratio, a->Nq, G, nblk, bs);
+    uint32_t* bhist = (uint32_t*)(w8 + p.off_bhist);
+    cudaError_t e = cudaMemsetAsync(bhist, 0, (size_t)p.rows * HIST_BINS * 4, st);
+    if (e != cudaSuccess) {
+      set_last_cuda_error(e);
+      return CSA_ERR_CUDA;
+    }
+    const int per_cta = BM_THREADS * BM_PER_THREAD;
+    block_max_kernel<<<dim3((nblk + per_cta - 1) / per_cta, p.rows), BM_THREADS, 0, st>>>(
+        scores, ld, p.n_cols, a->q_pos, a->n_c, a->ratio, a->Nq, G, nblk, bs, bhist);
     csa_status s = launch_status();
     if (s != CSA_OK) return s;
+    // the top blocks by (block score desc, block id asc): the histogram-guided row selection
     TopkRowArgs tc{};
     tc.in_scores = bs;
     tc.in_ld = nblk;
@@ -1276,7 +1323,10 @@ static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const 
     tc.k = a->pool_blocks;
     tc.out_idx = bidx;
     tc.out_ld = a->pool_blocks;
-    s = launch_topk(tc, p.rows, 1, false, st);
+    static std::atomic<unsigned> attr_p{0};
+    const int smem_h = (TOPK_CHUNK + 2 * TOPK_HIST_CAND) * 4;
+    set_smem_once((const void*)topk_hist_kernel, smem_h, attr_p);
+    s = launch_pdl(topk_hist_kernel, dim3(1, p.rows), dim3(TOPK_THREADS), (size_t)smem_h, st, tc, bhist);
     if (s != CSA_OK) return s;
     const int PG = a->pool_blocks * G;
     pool_expand_kernel<<<dim3((PG + 255) / 256, p.rows), 256, 0, st>>>(bidx, a->pool_blocks, G, scores, ld,
