@@ -546,12 +546,13 @@ __device__ void block_rank_select(const uint32_t* keys, const int32_t* ids, int 
   }
 }
 
-// Histogram-guided selection for one row (decode / Reindex rows): the score kernel has counted the
-// row's scores in 4096 bins of the top 12 bits of their order-preserving keys.  The bin holding the
-// K-th largest score is found from the histogram; one pass over the row (bit masks in registers) emits
-// every score in a higher bin, at slots from one block scan, and collects the boundary bin's scores.
-// One warp resolves those on the remaining key bits.  If the boundary bin overflows the candidate
-// buffer the row is selected by the full path instead.
+// Histogram-guided selection for one row (decode / Reindex rows, and the hierarchical pool's block scores):
+// the kernel before it has counted the row's scores in 4096 bins of the top 12 bits of their
+// order-preserving keys.  The bin holding the K-th largest score is found from the histogram; one pass over
+// the row (bit masks in registers) emits every score in a higher bin, at slots from one block scan, and
+// collects the boundary bin's scores.  The block resolves those on the remaining key bits (digit levels,
+// then a rank over all warps).  If the boundary bin overflows the candidate buffer the row is selected by
+// the full path instead.
 constexpr int TOPK_HIST_PER_THREAD = TOPK_CHUNK / TOPK_THREADS;   // 32 scores per thread, 8 x float4
 constexpr int TOPK_RANK_MAX = 64;
 constexpr int TOPK_HIST_CAND = 4096;     // boundary-bin candidates held in shared memory
