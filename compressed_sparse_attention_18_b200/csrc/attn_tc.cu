@@ -761,31 +761,36 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
 // query's last O MMAs release the K tile, and the current query's epilogue runs while that tile's S MMAs
 // do.  BF16 window rows only.
 
-// A query's positions and lengths, read one query ahead (plain loads, used a tile or more later).
+// A unit is split `split` of query bq (uid = bq * splits + split): tiles [split * tpc, split * tpc + tpc) of
+// the query's key list.  Its positions and lengths are read one unit ahead (plain loads, used a tile or
+// more later).
 struct TaUnitRaw {
-  int bq, nc;
+  int uid, nc;
   long long tq, wp0;
 };
 struct TaUnit {
-  int bq, b, n_sel, n_list, ntile, ncb;
+  int uid, bq, split, b, n_sel, n_list, ncb;
+  int t0, ntile;        // the unit's first tile of the query's list and its number of tiles
   int wofs;             // window buffer row of the first window key (wlo - win_pos0)
 };
 
-__device__ __forceinline__ TaUnitRaw ta_unit_load(const TaParams& P, int bq) {
+__device__ __forceinline__ TaUnitRaw ta_unit_load(const TaParams& P, int uid) {
   TaUnitRaw r;
-  const int b = bq / P.Nq;
-  r.bq = bq;
+  const int bq = uid / P.splits, b = bq / P.Nq;
+  r.uid = uid;
   r.tq = P.q_pos[bq];
   r.nc = P.n_c[b];
   r.wp0 = P.Wn > 0 ? P.win_pos0[b] : 0;
   return r;
 }
 
-// The query's key list [n_sel entries ‖ window rows] (the per-query kernel's rule).
+// The query's key list [n_sel entries ‖ window rows] (the per-query kernel's rule) and the unit's part.
 __device__ __forceinline__ TaUnit ta_unit(const TaParams& P, const TaUnitRaw& r) {
   TaUnit u;
-  u.bq = r.bq;
-  u.b = r.bq / P.Nq;
+  u.uid = r.uid;
+  u.bq = r.uid / P.splits;
+  u.split = r.uid % P.splits;
+  u.b = u.bq / P.Nq;
   u.ncb = min(r.nc, P.n_max);
   u.n_sel = P.k;
   if (P.hca) u.n_sel = (int)max(0LL, min((r.tq + 1) / P.ratio, (long long)u.ncb));
@@ -796,45 +801,55 @@ __device__ __forceinline__ TaUnit ta_unit(const TaParams& P, const TaUnitRaw& r)
   }
   u.wofs = whi >= wlo ? (int)(wlo - r.wp0) : 0;   // in [0, Wn) when the window is not empty
   u.n_list = u.n_sel + (whi >= wlo ? (int)(whi - wlo + 1) : 0);
-  u.ntile = (u.n_list + TA_KEYS - 1) / TA_KEYS;
+  u.t0 = u.split * P.tpc;
+  u.ntile = max(0, min(P.tpc, (u.n_list + TA_KEYS - 1) / TA_KEYS - u.t0));
   return u;
 }
 
-// Tile t of a query's key list.
+// Tile t of a unit (tile t0 + t of its query's key list).
 __device__ __forceinline__ TaTile ta_tile_u(const TaUnit& u, int t) {
-  return ta_tile(t * TA_KEYS, u.n_sel, u.n_list, u.wofs, 0, false);
+  return ta_tile((u.t0 + t) * TA_KEYS, u.n_sel, u.n_list, u.wofs, 0, false);
 }
 
-// The first query with keys among units kk, kk+1, ... of this CTA (from `raw` if those are unit kk's
-// positions), writing the outputs of the ones without keys (zero rows, lse = -inf) with threads
-// tid < nthreads; bq = -1 if there is none.
+// The first unit with keys among units kk, kk+1, ... of this CTA (from `raw` if those are unit kk's
+// positions), writing the outputs of the ones without keys with threads tid < nthreads: zero rows and
+// lse = -inf, or an empty partial (lse = -inf) when queries are split; bq = -1 if there is none.
 __device__ __forceinline__ TaUnit ta_next_unit(const TaParams& P, int kk, int nu, TaUnitRaw raw, int tid,
                                                int nthreads) {
   TaUnit uu{};
   uu.bq = -1;
 #pragma unroll 1
   for (; kk < nu; ++kk) {
-    const int bq = (int)blockIdx.x + kk * (int)gridDim.x;
-    if (raw.bq != bq) raw = ta_unit_load(P, bq);
+    const int uid = (int)blockIdx.x + kk * (int)gridDim.x;
+    if (raw.uid != uid) raw = ta_unit_load(P, uid);
     uu = ta_unit(P, raw);
     if (uu.ntile > 0) return uu;
-    for (int i = tid; i < P.H * 256; i += nthreads) reinterpret_cast<uint32_t*>(P.out + (size_t)bq * P.H * 512)[i] = 0u;
-    if (P.lse && tid < P.H) P.lse[(size_t)bq * P.H + tid] = -INFINITY;
+    if (P.splits > 1) {
+      if (tid < P.H) P.part_lse[(size_t)uid * P.H + tid] = -INFINITY;
+    } else {
+      for (int i = tid; i < P.H * 256; i += nthreads)
+        reinterpret_cast<uint32_t*>(P.out + (size_t)uu.bq * P.H * 512)[i] = 0u;
+      if (P.lse && tid < P.H) P.lse[(size_t)uu.bq * P.H + tid] = -INFINITY;
+    }
     uu.bq = -1;
   }
   return uu;
 }
 
-// Epilogue of a query, by the 8 worker warps once its last O MMAs have completed (phase `par` of bar_o):
-// O^T / l from tensor memory to bf16 rows [head][512], and lse; resets the running max and sum for
-// the next query.  Returns false if a wait gave up.
-__device__ __forceinline__ bool ta_epilogue(TaSmem& S, const TaParams& P, int bq, uint32_t par, uint32_t lane_base,
+// Epilogue of a unit, by the 8 worker warps once its last O MMAs have completed (phase `par` of bar_o):
+// O^T / l from tensor memory to bf16 rows [head][512], and lse, into the output (one unit per query) or
+// the unit's partial (split queries, merged by the split-merge kernel); resets the running max and sum
+// for the next unit.  Returns false if a wait gave up.
+__device__ __forceinline__ bool ta_epilogue(TaSmem& S, const TaParams& P, int uid, uint32_t par, uint32_t lane_base,
                                             int hh, int quad, int lane, int tid) {
   bool ok = true;
+  const bool part = P.splits > 1;
+  uint16_t* orow = part ? P.part_o + (size_t)uid * P.H * 512 : P.out + (size_t)uid * P.H * 512;
+  float* lrow = part ? P.part_lse + (size_t)uid * P.H : (P.lse ? P.lse + (size_t)uid * P.H : nullptr);
   if (tid < 64) {
     const float lh = S.l[tid];
     S.fac[tid] = lh > 0.f ? 1.f / lh : 0.f;
-    if (tid < P.H && P.lse) P.lse[(size_t)bq * P.H + tid] = lh > 0.f ? (S.m[tid] + log2f(lh)) * TA_LN2 : -INFINITY;
+    if (tid < P.H && lrow) lrow[tid] = lh > 0.f ? (S.m[tid] + log2f(lh)) * TA_LN2 : -INFINITY;
     S.m[tid] = -INFINITY;
     S.l[tid] = 0.f;
   }
@@ -848,7 +863,7 @@ __device__ __forceinline__ bool ta_epilogue(TaSmem& S, const TaParams& P, int bq
     tmem_ld_x32(lane_base + TA_COL_O + 64 * mt + hh * 32, ov);
     tmem_wait_ld_x32(ov);
     const int dim = 128 * mt + 32 * quad + lane;
-    uint16_t* o = P.out + ((size_t)bq * P.H + hh * 32) * 512 + dim;
+    uint16_t* o = orow + (size_t)hh * 32 * 512 + dim;
 #pragma unroll
     for (int j = 0; j < 32; j += 4) {
       const float4 il = *reinterpret_cast<const float4*>(&S.fac[hh * 32 + j]);
@@ -870,9 +885,10 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
   TaSmem& S = *reinterpret_cast<TaSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int grow = (tid & (TA_WORKERS - 1)) >> 1, ghalf = tid & 1;
-  // this CTA's queries: unit u is query blockIdx.x + u * gridDim.x
-  const int nu = (int)blockIdx.x < P.rows ? (P.rows - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-  auto unit_q = [&](int u) { return (int)blockIdx.x + u * (int)gridDim.x; };
+  // this CTA's units: its k-th is unit blockIdx.x + k * gridDim.x of the rows * splits
+  const int n_units = P.rows * P.splits;
+  const int nu = (int)blockIdx.x < n_units ? (n_units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  auto unit_q = [&](int k) { return (int)blockIdx.x + k * (int)gridDim.x; };
   if (warp == 8) {
     if (lane == 0) {
       S.err = 0;
@@ -1034,15 +1050,15 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
     auto next_unit = [&](int kk, TaUnitRaw raw) -> TaUnit {
       return ta_next_unit(P, kk, nu, raw, tid, TA_WORKERS);
     };
-    auto unit_index = [&](const TaUnit& uu) { return uu.bq < 0 ? nu : (uu.bq - (int)blockIdx.x) / (int)gridDim.x; };
-    auto epilogue = [&](int bq, uint32_t par) { ok = ta_epilogue(S, P, bq, par, lane_base, hh, quad, lane, tid) && ok; };
+    auto unit_index = [&](const TaUnit& uu) { return uu.bq < 0 ? nu : (uu.uid - (int)blockIdx.x) / (int)gridDim.x; };
+    auto epilogue = [&](int uid, uint32_t par) { ok = ta_epilogue(S, P, uid, par, lane_base, hh, quad, lane, tid) && ok; };
 
     TaUnit u = nu > 0 ? next_unit(0, ta_unit_load(P, unit_q(0))) : TaUnit{};
     if (nu == 0) u.bq = -1;
     int k = unit_index(u);
-    int bq_done = -1;                           // query awaiting its epilogue
+    int bq_done = -1;                           // unit (uid) awaiting its epilogue
     TaUnitRaw nraw{};
-    nraw.bq = -1;
+    nraw.uid = -1;
     if (k + 1 < nu) nraw = ta_unit_load(P, unit_q(k + 1));
     int id = -1;
     if (k < nu) {
@@ -1126,7 +1142,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       }
       // what the softmax needs of this tile; then the cursor moves on (one query's geometry stays live)
       const int rs_t = g.rs, rw_t = g.rw, t_cur = t;
-      const int bq_ends = t + 1 == u.ntile ? u.bq : -1;
+      const int bq_ends = t + 1 == u.ntile ? u.uid : -1;
       k = kn;
       t = tn;
       u = un;
@@ -1218,7 +1234,7 @@ __global__ void __launch_bounds__(TA_THREADS, 1)
       if (bq_ends >= 0) {
         bq_done = bq_ends;
         // positions of the query after the next one, read now and used when the next one ends
-        nraw.bq = -1;
+        nraw.uid = -1;
         if (k + 1 < nu) nraw = ta_unit_load(P, unit_q(k + 1));
       }
       ++f;
@@ -1243,28 +1259,77 @@ bool attn_tc_early(const csa_attn_args* a, int hca) {
   return !hca && (a->flags & CSA_EARLY_START) && n_win > 0 && n_win <= TA_KEYS && a->k > 0 && a->k % TA_KEYS == 0;
 }
 
-// Key tiles per query and the CTAs that share them: one tile per CTA while the grid fits one wave of
-// the 148 SMs, else enough tiles per CTA (walked in order, online softmax) to come back to one wave.
-// With the early window the entry tiles alone are planned this way; split 0 also takes the window tile
-// (first, while the previous kernel still runs).
+// The persistent kernel (one CTA per SM walking units back to back) takes the plans with BF16 window rows,
+// no early window and at least two tiles per SM on average; HCA (entries streamed from HBM in order) only
+// with more queries than SMs, as the per-query kernel measured faster for few long HCA queries.
+static bool attn_tc_persist_ok(const csa_attn_args* a, int hca, long long rows, long long tiles) {
+  return (hca ? rows > 148 : rows * tiles >= 2 * 148) && rows <= 0x7fffffffLL && a->win_format == CSA_WIN_BF16 && !attn_tc_early(a, hca);
+}
+
+// Tiles per unit for the persistent kernel: units (query, split) are dealt to the CTAs in turn, so the
+// plan that finishes first is found by adding up each CTA's units.  Costs in tile-times (≈ 6.9 µs): a unit
+// its tiles plus an epilogue of TA_EPI_TILES; splitting adds the merge launch (TA_MERGE_TILES) and each
+// unit's partial (H rows of 512 bf16) written and read back at the HBM rate (≈ 6 TB/s).  Queries enough
+// to keep every CTA busy with whole queries stay unsplit.
+constexpr double TA_EPI_TILES = 0.4, TA_MERGE_TILES = 0.5, TA_TILE_US = 6.9, TA_HBM_BYTES_PER_US = 6.0e6;
+static int attn_tc_persist_tpc(long long rows, long long tiles, int H) {
+  const double part_tiles = (double)H * 512 * 2 * 2 / (TA_HBM_BYTES_PER_US * TA_TILE_US);
+  if (rows >= 4 * 148) return (int)tiles;
+  double best = 1e300;
+  long long best_tpc = tiles;
+  const long long max_splits = tiles < 32 ? tiles : 32;
+  for (long long sp = 1; sp <= max_splits; ++sp) {
+    const long long tpc = (tiles + sp - 1) / sp, splits = (tiles + tpc - 1) / tpc;
+    if (splits != sp || rows * splits > 0x7fffffffLL) continue;   // the same plan as a smaller split count
+    const long long units = rows * splits, grid = units < 148 ? units : 148;
+    double worst = 0.0;
+    for (long long c = 0; c < grid; ++c) {
+      double load = 0.0;
+      for (long long uid = c; uid < units; uid += grid) {
+        const long long sidx = uid % splits, nt = tiles - sidx * tpc < tpc ? tiles - sidx * tpc : tpc;
+        load += (double)nt + TA_EPI_TILES;
+      }
+      if (load > worst) worst = load;
+    }
+    if (splits > 1) worst += TA_MERGE_TILES + (double)units * part_tiles;
+    if (worst < best - 1e-9) {
+      best = worst;
+      best_tpc = tpc;
+    }
+  }
+  return (int)best_tpc;
+}
+
+// Key tiles per query and the CTAs that share them.  Per-query kernel: one tile per CTA while the grid fits
+// one wave of the 148 SMs, else enough tiles per CTA (walked in order, online softmax) to come back to one
+// wave; with the early window the entry tiles alone are planned this way and split 0 also takes the window
+// tile (first, while the previous kernel still runs).  Persistent kernel: see attn_tc_persist_tpc.
 void attn_tc_plan(const csa_attn_args* a, int hca, int* splits, int* tpc) {
   const bool early = attn_tc_early(a, hca);
   const long long n_win = attn_has_window(a) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
   const long long n = (hca ? a->n_max : a->k) + (early ? 0 : n_win);
   const long long tiles = n > 0 ? (n + TA_KEYS - 1) / TA_KEYS : 1;
   const long long rows = (long long)a->B * a->Nq;
-  long long t = (rows * tiles + 147) / 148;
-  if (t < 1) t = 1;
-  if (t > tiles) t = tiles;
+  long long t;
+  if (attn_tc_persist_ok(a, hca, rows, tiles)) {
+    t = attn_tc_persist_tpc(rows, tiles, a->H);
+  } else {
+    t = (rows * tiles + 147) / 148;
+    if (t < 1) t = 1;
+    if (t > tiles) t = tiles;
+  }
   *tpc = (int)t;
   *splits = (int)((tiles + t - 1) / t);
 }
 
-// One CTA per query and more queries than one wave of CTAs, BF16 window: the persistent kernel.
+// The persistent kernel's plans (the same decision attn_tc_plan made).
 bool attn_tc_persistent(const csa_attn_args* a, int hca, int splits) {
-  const long long rows = (long long)a->B * a->Nq;
-  return splits == 1 && rows > 148 && rows <= 0x7fffffffLL && a->win_format == CSA_WIN_BF16 &&
-         !attn_tc_early(a, hca);
+  (void)splits;
+  const bool early = attn_tc_early(a, hca);
+  const long long n_win = attn_has_window(a) ? (a->Wn < a->window ? a->Wn : a->window) : 0;
+  const long long n = (hca ? a->n_max : a->k) + (early ? 0 : n_win);
+  const long long tiles = n > 0 ? (n + TA_KEYS - 1) / TA_KEYS : 1;
+  return attn_tc_persist_ok(a, hca, (long long)a->B * a->Nq, tiles);
 }
 
 // Queries split over 2..8 CTAs can merge inside a thread-block cluster (CSA_CLUSTER_MERGE: no workspace,
@@ -1332,7 +1397,7 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
   }
   const int smem = (int)sizeof(TaSmem) + 1024;
   if (attn_tc_persistent(a, hca, splits)) {
-    // more queries than SMs, one CTA each: one persistent CTA per SM walks its queries back to back
+    // one persistent CTA per SM walks its units (query, split) back to back
     int sms = 148;
     {
       int dev = 0;
@@ -1340,7 +1405,8 @@ csa_status launch_attn_tc(const csa_attn_args* a, int hca, int splits, int tpc, 
     }
     static std::atomic<unsigned> attr_done_p{0};
     set_smem_once((const void*)attn_tc_persist_kernel, smem, attr_done_p);
-    const unsigned grid = (unsigned)(rows < sms ? rows : sms);
+    const long long units = rows * splits;
+    const unsigned grid = (unsigned)(units < sms ? units : sms);
     return launch_pdl(attn_tc_persist_kernel, dim3(grid), dim3(TA_THREADS), (size_t)smem, st, qmap, wmap, P);
   }
   static std::atomic<unsigned> attr_done{0};
