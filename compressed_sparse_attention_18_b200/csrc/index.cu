@@ -25,6 +25,7 @@ constexpr int IDX_QT = 32;             // max queries per CTA (query fragments s
 constexpr int TOPK_THREADS = 1024;
 constexpr int TOPK_CHUNK = 32768;      // max row length held in shared memory (implicit ids)
 constexpr int TOPK_CHUNK_IDS = 16384;  // max row length with explicit ids
+constexpr int TOPK_SHORT = 8192;        // rows up to this length go to the 256-thread kernel
 constexpr int HIST_BINS = 4096;        // score histogram: top 12 bits of the order-preserving key
 constexpr int HIST_SHIFT = 20;
 
@@ -1058,6 +1059,35 @@ __global__ void __launch_bounds__(BM_THREADS) block_max_kernel(const float* __re
     if (h[i]) atomicAdd(&hr[i], h[i]);
 }
 
+// Row histograms for score rows no scorer counted (multi-query rows): the visible scores of a row (j <
+// n_vis(t)) in HIST_BINS bins of the top 12 bits of their order-preserving keys, added to the row's
+// histogram (zero on entry).  CTA: RH_THREADS threads x RH_PER_THREAD scores of one row.
+constexpr int RH_THREADS = 1024, RH_PER_THREAD = 4;
+__global__ void __launch_bounds__(RH_THREADS) row_hist_kernel(const float* __restrict__ scores, long long ld,
+                                                              int n_cols, const int64_t* __restrict__ q_pos,
+                                                              const int32_t* __restrict__ n_c, int ratio, int Nq,
+                                                              uint32_t* __restrict__ hist) {
+  __shared__ uint32_t h[HIST_BINS];
+  const int row = blockIdx.y;
+  for (int i = threadIdx.x; i < HIST_BINS; i += blockDim.x) h[i] = 0;
+  long long nv = (q_pos[row] + 1) / ratio;
+  if (nv > n_c[row / Nq]) nv = n_c[row / Nq];
+  if (nv > n_cols) nv = n_cols;
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < RH_PER_THREAD; ++u) {
+    const long long j = ((long long)blockIdx.x * RH_PER_THREAD + u) * RH_THREADS + threadIdx.x;
+    if (j < nv) {
+      const float v = scores[row * ld + j];
+      if (v > -INFINITY) atomicAdd(&h[float_order_key(v) >> HIST_SHIFT], 1u);
+    }
+  }
+  __syncthreads();
+  uint32_t* hr = hist + (size_t)row * HIST_BINS;
+  for (int i = threadIdx.x; i < HIST_BINS; i += blockDim.x)
+    if (h[i]) atomicAdd(&hr[i], h[i]);
+}
+
 __global__ void pool_expand_kernel(const int32_t* __restrict__ blk, int P, int G, const float* __restrict__ scores,
                                    long long ld, int n_cols, const int64_t* __restrict__ q_pos,
                                    const int32_t* __restrict__ n_c, int ratio, int Nq, int32_t* __restrict__ pool) {
@@ -1089,7 +1119,9 @@ csa_status run_index_topk_fused(const csa_index_args* a, cudaStream_t st);
 struct IndexPlan {
   int rows, n_cols, segs, seg_len;
   bool hist;   // single-query rows: histogram-guided selection (long rows: segment CTAs + tournament fallback)
-  size_t off_scores, off_tidx, off_tsc, off_bs, off_bidx, off_bhist, off_lstate, off_lcand, off_hist, sel_total, total;
+  bool mq_hist;  // multi-query rows longer than TOPK_SHORT: a row-histogram pass, then the same selection
+  size_t off_scores, off_tidx, off_tsc, off_bs, off_bidx, off_bhist, off_mqhist, off_lstate, off_lcand, off_hist,
+      sel_total, total;
 };
 
 static bool one_query_per_cta(const csa_index_args* a) { return a->cand != nullptr || a->Nq == 1; }
@@ -1119,6 +1151,10 @@ static IndexPlan plan_index(const csa_index_args* a) {
     p.off_bs = o;   o = align_up(o + (size_t)p.rows * nblk * 4, 256);
     p.off_bidx = o; o = align_up(o + (size_t)p.rows * a->pool_blocks * 4, 256);
     p.off_bhist = o; o = align_up(o + (size_t)p.rows * HIST_BINS * 4, 256);
+  }
+  p.mq_hist = !one_query_per_cta(a) && p.segs == 1 && p.seg_len > TOPK_SHORT;
+  if (p.mq_hist) {
+    p.off_mqhist = o; o = align_up(o + (size_t)p.rows * HIST_BINS * 4, 256);
   }
   p.sel_total = o;
   p.off_scores = o;
@@ -1201,7 +1237,6 @@ static csa_status run_scores(const csa_index_args* a, float* scores, long long l
   return launch_status();
 }
 
-constexpr int TOPK_SHORT = 8192;        // rows up to this length go to the 256-thread kernel
 constexpr int TOPK_SHORT_THREADS = 256;
 
 static csa_status launch_topk(TopkRowArgs ta, int rows, int segs, bool ids, cudaStream_t st) {
@@ -1247,6 +1282,28 @@ static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const 
     set_smem_once((const void*)topk_hist_kernel, smem_h, attr_h);
     csa_status s = launch_pdl(topk_hist_kernel, dim3(1, p.rows), dim3(TOPK_THREADS), (size_t)smem_h, st, ta,
                               const_cast<uint32_t*>(hist));
+    if (s != CSA_OK) return s;
+  } else if (p.segs == 1 && p.mq_hist) {
+    // multi-query rows: their histograms first (visible scores only), then the histogram-guided selection
+    ta.out_idx = a->idx_out;
+    ta.out_scores = a->scores_out;
+    ta.out_ld = a->k;
+    ta.early = 0;
+    uint32_t* mh = (uint32_t*)(w8 + p.off_mqhist);
+    const cudaError_t e = cudaMemsetAsync(mh, 0, (size_t)p.rows * HIST_BINS * 4, st);
+    if (e != cudaSuccess) {
+      set_last_cuda_error(e);
+      return CSA_ERR_CUDA;
+    }
+    const int per_cta = RH_THREADS * RH_PER_THREAD;
+    row_hist_kernel<<<dim3((p.n_cols + per_cta - 1) / per_cta, p.rows), RH_THREADS, 0, st>>>(
+        scores, ld, p.n_cols, a->q_pos, a->n_c, a->ratio, a->Nq, mh);
+    csa_status s = launch_status();
+    if (s != CSA_OK) return s;
+    static std::atomic<unsigned> attr_m{0};
+    const int smem_h = (TOPK_CHUNK + 2 * TOPK_HIST_CAND) * 4;
+    set_smem_once((const void*)topk_hist_kernel, smem_h, attr_m);
+    s = launch_pdl(topk_hist_kernel, dim3(1, p.rows), dim3(TOPK_THREADS), (size_t)smem_h, st, ta, mh);
     if (s != CSA_OK) return s;
   } else if (p.segs == 1) {
     ta.out_idx = a->idx_out;

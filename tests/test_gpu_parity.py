@@ -194,6 +194,14 @@ def test_index_prefill_causal_multi_query(cuda_lib):
     _index_case(cuda_lib, B=1, n_max=512, n_c=[300], d_I=128, H_I=8, Nq=48, q_pos=q_pos, k=64, seed=2)
 
 
+def test_index_multiquery_rows_histogram_pass(cuda_lib):
+    """Multi-query rows longer than 8192 keys (speculative positions): the selection counts each row's
+    visible scores in a histogram pass, then selects like a decode row.  Positions of one sequence see
+    different prefixes (9000 to 20000 keys, some ending inside a 4096-score slice)."""
+    q_pos = [4 * 20000 - 1, 4 * 12000 + 1, 4 * 9000 + 3, 4 * 15000 - 1, 4 * 10000, 4 * 14000 + 2]
+    _index_case(cuda_lib, B=2, n_max=20000, n_c=[20000, 15000], d_I=128, H_I=8, Nq=3, q_pos=q_pos, k=512, seed=61)
+
+
 def test_index_tournament_long_row(cuda_lib):
     n = 40000                                             # > one 32768-column top-k chunk
     _index_case(cuda_lib, B=2, n_max=n, n_c=[n, n - 123], d_I=128, H_I=8, Nq=1, q_pos=[4 * n - 1, 4 * n - 1],
