@@ -286,7 +286,8 @@ csa_status csa_index_scores(const csa_index_args* args, float* scores, int64_t l
 /* csa_topk — the selection half of csa_index_topk ([V4 blog] Fig. 3: top-k per query; [V4.1 notes]
  * Fig. 5: hierarchical pool) over a score matrix laid out as csa_index_scores writes it, with the
  * same args (q_I, w, k_codes, k_scales may be NULL).  In Reindex mode ld must equal n_cand.
- * Workspace: csa_topk_workspace_size() (tournament buffers for rows longer than 32768, pool scores). */
+ * Workspace: csa_topk_workspace_size() (tournament buffers for rows longer than 32768, pool block scores
+ * and their histograms, row histograms for multi-query rows longer than 8192 keys). */
 size_t csa_topk_workspace_size(const csa_index_args* args);
 csa_status csa_topk(const csa_index_args* args, const float* scores, int64_t ld, void* ws, size_t ws_bytes,
                     void* stream);
