@@ -335,10 +335,13 @@ csa_status run_scores_mq_tc(const csa_index_args* a, float* scores, long long ld
   P.g_q = a->g_q;
   P.gg = a->g_q * a->g_k;
   P.pm = a->k_pages;
-  // key splits per query block: about two waves of CTAs in all, each CTA at least 8 key tiles
+  // key splits per query block: at most two waves of CTAs in all (one CTA per SM: the tensor memory),
+  // rounded down so that few query blocks do not spill into a third, short wave; 2 while the query blocks
+  // alone fill one to two waves; each CTA at least 8 key tiles
   const long long qblocks = (long long)a->B * ((a->Nq + MQ_QB - 1) / MQ_QB);
   const int tiles_row = (a->n_max + MQ_KEYS - 1) / MQ_KEYS;
-  long long splits = (2 * 148 + qblocks - 1) / qblocks;
+  long long splits = (2 * 148) / qblocks;
+  if (splits < 2 && qblocks < 2 * 148) splits = 2;
   if (splits > (tiles_row + 7) / 8) splits = (tiles_row + 7) / 8;
   if (splits < 1) splits = 1;
   P.splits = (int)splits;
