@@ -502,6 +502,24 @@ def test_attn_persistent_hca_variable_tiles(cuda_lib, Wn):
         assert bool(torch.all(out.cpu()[empty] == 0)) and bool(torch.all(torch.isneginf(lse.cpu()[empty])))
 
 
+@pytest.mark.parametrize("Wn", [0, 128])
+def test_attn_persistent_hca_split_units(cuda_lib, Wn):
+    """HCA over 160 queries of up to 8-9 tiles (1024 entries, plus the window): more queries than SMs but
+    few tiles each, so the persistent kernel deals (query, split) units of 2-3 tiles to the SMs and the
+    merge combines them.  Visible counts from 0 to 1024 entries: units past a query's keys write empty
+    partials, and a query without any keys comes out zero with lse = -inf."""
+    rng = np.random.default_rng(55)
+    B, Nq = 2, 80
+    q_pos = rng.integers(0, 128 * 1100, size=(B, Nq))
+    q_pos[0, ::7] = rng.integers(0, 127, size=len(q_pos[0, ::7]))
+    out, lse = _attn_case(cuda_lib, B=B, Nq=Nq, H=64, d=512, d_r=64, n_max=1024, n_c=[1024, 700],
+                          q_pos=q_pos.ravel().tolist(), hca=True, ratio=128, Wn=Wn,
+                          win_pos0=[int(q_pos[b].max()) - Wn + 1 for b in range(B)] if Wn else None, seed=56)
+    if Wn == 0:
+        empty = torch.as_tensor(q_pos < 127)
+        assert bool(torch.all(out.cpu()[empty] == 0)) and bool(torch.all(torch.isneginf(lse.cpu()[empty])))
+
+
 @pytest.mark.parametrize("early_start", [False, True], ids=["plain", "early"])
 def test_attn_workspace_reused_across_calls_and_plans(cuda_lib, early_start):
     """One caller workspace, sized by the size query before any output exists, serves repeated calls and
