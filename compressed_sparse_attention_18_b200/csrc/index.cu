@@ -494,6 +494,8 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(TopkRowArgs A) {
   __shared__ TopkSmemT<THREADS / 32> sm;
   const int seg = blockIdx.x;                  // segment (chunk) of the row
   const int row = blockIdx.y;
+  pdl_trigger();
+  pdl_wait();                                  // scores (and the long-row pass's flags) come from the previous kernel
   if (A.skip && A.skip[row].ok) return;        // selected by the long-row histogram pass
   const int col0 = A.col_base + seg * A.rows_per_seg;
   int len = min(A.rows_per_seg, A.n_cols - col0);
@@ -1247,14 +1249,12 @@ static csa_status launch_topk(TopkRowArgs ta, int rows, int segs, bool ids, cuda
     const size_t smem = ids ? (size_t)TOPK_SHORT * 8 : align_up((size_t)ta.rows_per_seg, 4) * 4;
     static std::atomic<unsigned> attr_s{0};
     set_smem_once((const void*)topk_kernel<TOPK_SHORT_THREADS, TOPK_SHORT>, TOPK_SHORT * 8, attr_s);
-    topk_kernel<TOPK_SHORT_THREADS, TOPK_SHORT><<<grid, TOPK_SHORT_THREADS, smem, st>>>(ta);
-    return launch_status();
+    return launch_pdl(topk_kernel<TOPK_SHORT_THREADS, TOPK_SHORT>, grid, dim3(TOPK_SHORT_THREADS), smem, st, ta);
   }
   const size_t smem = (size_t)TOPK_CHUNK * 4;
   static std::atomic<unsigned> attr_done{0};
   set_smem_once((const void*)topk_kernel<TOPK_THREADS, TOPK_CHUNK_IDS>, (int)smem, attr_done);
-  topk_kernel<TOPK_THREADS, TOPK_CHUNK_IDS><<<grid, TOPK_THREADS, smem, st>>>(ta);
-  return launch_status();
+  return launch_pdl(topk_kernel<TOPK_THREADS, TOPK_CHUNK_IDS>, grid, dim3(TOPK_THREADS), smem, st, ta);
 }
 
 static csa_status run_select(const csa_index_args* a, const IndexPlan& p, const float* scores, long long ld,
